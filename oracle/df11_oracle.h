@@ -1,0 +1,109 @@
+/*
+ * df11_oracle.h -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, single-threaded C restatement of the DFloat11 (DF11) codec:
+ * split a BF16 word into exponent and sign|mantissa bytes, Huffman-code the
+ * exponent with a canonical, length-limited code, write the bitstream, derive
+ * the per-thread gap / per-chunk output-position metadata, and decode the
+ * stream one bit at a time.  It exists to check the product library and its
+ * GPU kernel; nothing in the product path may call it.  It shares no code,
+ * header, table or constant with the library under huffman_decode_b200/.
+ *
+ * Sources (the web pages this method is described on):
+ *   [DF11-page] "DFloat11: lossless BFloat16 compression" (ai-infrastructure.net),
+ *               sections "What it is", "Architecture" and
+ *               "How it works: the core algorithm" (executed numpy sketch and
+ *               its printed output).
+ *
+ * Every function below names the passage it follows.  All functions return 0
+ * on success and a negative value on a detected error.
+ */
+#ifndef DF11_ORACLE_H
+#define DF11_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* [DF11-page] "What it is" / split_bf16: the exponent is bits 14..7 of the
+ * BF16 word; the raw byte keeps the sign in bit 7 and the 7 mantissa bits. */
+void orc_split(const uint16_t *w, uint64_t n, uint8_t *exp_out, uint8_t *sm_out);
+
+/* [DF11-page] join_bf16: the inverse of orc_split. */
+void orc_join(const uint8_t *exp_in, const uint8_t *sm_in, uint64_t n, uint16_t *w_out);
+
+/* Adds the 256-bin exponent histogram of exp[0..n) into counts (not cleared). */
+void orc_histogram_add(const uint8_t *exp, uint64_t n, uint64_t counts[256]);
+
+/* Shannon entropy in bits of the distribution given by counts (fp64). */
+double orc_entropy(const uint64_t counts[256]);
+
+/* [DF11-page] huffman_lengths: plain Huffman with the page's tie rule --
+ * a min-queue keyed by (count, insertion index); live symbols enter in
+ * ascending symbol order, each merged node takes the next index; every merge
+ * deepens every symbol under both children by one.  One live symbol gets
+ * length 1.  len[s] = 0 for absent symbols.  Returns the number of live
+ * symbols, or -1 if there are none. */
+int orc_huffman_lengths(const uint64_t counts[256], uint8_t len[256]);
+
+/* Optimal code lengths under a maximum length `cap` by package-merge
+ * (Larmore & Hirschberg, "A fast algorithm for optimal length-limited Huffman
+ * codes", J. ACM 37(3), 1990), written out with explicit per-item symbol
+ * multiplicities.  Needs 2 <= live symbols <= 2^cap.  Returns the number of
+ * live symbols or -1. */
+int orc_package_merge_lengths(const uint64_t counts[256], int cap, uint8_t len[256]);
+
+/* The code lengths DF11 uses under a length cap ([DF11-page] "Architecture",
+ * hierarchical lookup tables: real exponent trees reach 24-32 bits and the
+ * format must bound them): the page's Huffman lengths when their maximum is
+ * within the cap, else package-merge.  Both are optimal. */
+int orc_code_lengths(const uint64_t counts[256], int cap, uint8_t len[256]);
+
+/* [DF11-page] canonical_codes: symbols in ascending (length, symbol) order;
+ * the first gets code 0; each next code is the previous plus one, shifted
+ * left by the growth in length.  code[s] is right-aligned in len[s] bits. */
+int orc_canonical_codes(const uint8_t len[256], uint32_t code[256]);
+
+/* Sum over symbols of count * length. */
+uint64_t orc_total_bits(const uint64_t counts[256], const uint8_t len[256]);
+
+/* [DF11-page] encode: codes concatenated in element order, most significant
+ * bit first.  Stream bit i is bit (7 - i%8) of byte i/8.  The caller zeroes
+ * `stream` (stream_bytes long).  Returns the bit count through *total_bits. */
+int orc_encode(const uint8_t *exp, uint64_t n, const uint8_t len[256],
+               const uint32_t code[256], uint8_t *stream, uint64_t stream_bytes,
+               uint64_t *total_bits);
+
+/* Bit-by-bit canonical decode (no lookup tables) of n symbols starting at
+ * stream bit `start_bit`.  Reading past stream_bytes or meeting a bit pattern
+ * that is no code returns -1.  *end_bit receives the bit after the last code. */
+int orc_decode(const uint8_t *stream, uint64_t stream_bytes, uint64_t start_bit,
+               uint64_t n, const uint8_t len[256], uint8_t *exp_out, uint64_t *end_bit);
+
+/* First code in the 16-bit MSB-first window v: the symbol and its length, or
+ * -1 when no code is a prefix of v (only possible with a single live symbol). */
+int orc_first_code(uint32_t v16, const uint8_t len[256], int *sym, int *clen);
+
+/* orc_first_code for every 16-bit window: sym_out/len_out[v] (len 0 = none). */
+int orc_first_code_table(const uint8_t len[256], int16_t *sym_out, uint8_t *len_out);
+
+/* [DF11-page] "Architecture", two-phase kernel: each thread owns a fixed
+ * slice of bytes_per_thread bytes of the stream; Gaps holds the bit offset of
+ * the first code that starts inside the slice; one output position is kept
+ * per group of threads_per_chunk threads.  Code k starts at
+ * s_k = sum_{j<k} len(exp_j); s_n = total_bits is counted as a start so a
+ * slice whose codes all began earlier still points at the end.
+ *   gap[g]   = min{ s_k >= B*g } - B*g for slices with B*g < total_bits, else 0
+ *   pos[c]   = #{ k < n : s_k < c*T*B },  c = 0..n_chunks  (B = 8*bytes_per_thread)
+ * gap is unpacked (one byte per thread, n_threads = n_chunks*T entries). */
+int orc_metadata(const uint8_t *exp, uint64_t n, const uint8_t len[256],
+                 uint32_t threads_per_chunk, uint32_t bytes_per_thread,
+                 uint64_t n_chunks, uint8_t *gap, uint32_t *pos);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DF11_ORACLE_H */

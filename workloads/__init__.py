@@ -1,0 +1,141 @@
+"""Seeded synthetic BF16 weight blocks, shared by the tests, the benchmark,
+the smoke check and the oracle's pins.
+
+This module only draws random numbers and rounds them to BF16; it holds none
+of the codec's arithmetic.  The shapes follow the models the DFloat11 pages
+measure (Llama-3.1-8B transformer blocks, a FLUX.1-style DiT block); trained
+checkpoints are not available, so normal / Student-t draws stand in for them.
+Every generator is deterministic in its seed.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# --------------------------------------------------------------- rounding
+
+
+def to_bf16(x: np.ndarray) -> np.ndarray:
+    """float32 -> BF16 bit patterns, round to nearest even (finite inputs).
+
+    The rounding the page "DFloat11: lossless BFloat16 compression" uses to
+    make its synthetic tensor (section "How it works: the core algorithm").
+    """
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    return ((u + np.uint32(0x7FFF) + r) >> np.uint32(16)).astype(np.uint16)
+
+
+def _normal_bf16(rng: np.random.Generator, shape, sigma: float) -> np.ndarray:
+    n = int(np.prod(shape))
+    x = rng.standard_normal(n, dtype=np.float32)
+    x *= np.float32(sigma)
+    return to_bf16(x).reshape(shape)
+
+
+# ------------------------------------------------------------------ blocks
+
+LLAMA8B_BLOCK_SHAPES = [
+    ("q_proj", (4096, 4096)),
+    ("k_proj", (1024, 4096)),
+    ("v_proj", (1024, 4096)),
+    ("o_proj", (4096, 4096)),
+    ("gate_proj", (14336, 4096)),
+    ("up_proj", (14336, 4096)),
+    ("down_proj", (4096, 14336)),
+]
+
+FLUX_BLOCK_SHAPES = (
+    [("qkv", (9216, 3072)), ("proj", (3072, 3072)), ("mlp_in", (12288, 3072)),
+     ("mlp_out", (3072, 12288)), ("adaln", (18432, 3072))]
+    + [(f"small_{i:02d}", (3072, 256)) for i in range(64)]
+)
+
+
+def single_matrix(seed: int = 0, shape=(1024, 1024), sigma: float = 0.02):
+    """One matrix of N(0, sigma) weights: the page's worked-example recipe
+    (numpy default_rng(seed).normal(0, sigma) in float64, cast to float32)."""
+    rng = np.random.default_rng(seed)
+    x = rng.normal(0.0, sigma, int(np.prod(shape))).astype(np.float32)
+    return [("w", to_bf16(x).reshape(shape))]
+
+
+def llama_block(seed: int = 1000, scale_div: int = 1):
+    """A Llama-3.1-8B-shaped transformer block: 7 matrices, per-matrix sigma
+    drawn uniformly from [0.01, 0.04] (all 7 drawn first), then float32
+    normals.  scale_div > 1 shrinks every row count (small test variant)."""
+    rng = np.random.default_rng(seed)
+    sig = rng.uniform(0.01, 0.04, len(LLAMA8B_BLOCK_SHAPES))
+    out = []
+    for (name, (r, c)), s in zip(LLAMA8B_BLOCK_SHAPES, sig):
+        out.append((name, _normal_bf16(rng, (max(1, r // scale_div), c), float(s))))
+    return out
+
+
+def llama_model_seeds(n_blocks: int = 32, first_seed: int = 1000):
+    """Seeds of the blocks of the 8B-scale stream (block i uses first_seed+i)."""
+    return [first_seed + i for i in range(n_blocks)]
+
+
+def flux_block(seed: int = 5000, scale_div: int = 1):
+    """FLUX.1-style DiT block, hidden 3072, N(0, 0.02): 5 large matrices and
+    64 small 3072x256 ones, in that order."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for name, (r, c) in FLUX_BLOCK_SHAPES:
+        out.append((name, _normal_bf16(rng, (max(1, r // scale_div), c), 0.02)))
+    return out
+
+
+SPECIAL_BF16 = [0x0000, 0x8000, 0x7F80, 0xFF80, 0x7FC0, 0xFFC1, 0x7F81]
+
+
+def heavy_tail(seed: int = 4001, shape=(4096, 4096)):
+    """Student-t (nu=3) * 0.02; 0.1% of entries get a uniformly random exponent
+    field (sign and mantissa kept); then 64 copies each of +-0, +-Inf and three
+    NaN patterns, and 1024 random subnormals, at random positions."""
+    rng = np.random.default_rng(seed)
+    n = int(np.prod(shape))
+    x = (rng.standard_t(3, n) * 0.02).astype(np.float32)
+    w = to_bf16(x)
+    k = max(1, n // 1000)
+    idx = rng.choice(n, size=k, replace=False)
+    new_exp = rng.integers(0, 256, k).astype(np.uint16)
+    w[idx] = (w[idx] & np.uint16(0x807F)) | (new_exp << np.uint16(7))
+    specials = np.repeat(np.array(SPECIAL_BF16, np.uint16), 64)
+    sub_sign = rng.integers(0, 2, 1024).astype(np.uint16) << np.uint16(15)
+    sub_mant = rng.integers(1, 128, 1024).astype(np.uint16)
+    specials = np.concatenate([specials, sub_sign | sub_mant])
+    pos = rng.choice(n, size=specials.size, replace=False)
+    w[pos] = specials
+    return [("heavy_tail", w.reshape(shape))]
+
+
+def single_exponent(seed: int = 4002, shape=(4096, 4096), exponent: int = 0x79):
+    """N(0, 0.02) with every exponent field forced to one value."""
+    rng = np.random.default_rng(seed)
+    n = int(np.prod(shape))
+    w = to_bf16(rng.standard_normal(n, dtype=np.float32) * np.float32(0.02))
+    w = (w & np.uint16(0x807F)) | np.uint16(exponent << 7)
+    return [("single_exponent", w.reshape(shape))]
+
+
+def uniform_bits(seed: int = 4003, shape=(4096, 4096)):
+    """Uniformly random 16-bit patterns (every exponent, NaNs and Infs included)."""
+    rng = np.random.default_rng(seed)
+    w = rng.integers(0, 65536, int(np.prod(shape)), dtype=np.uint16)
+    return [("uniform_bits", w.reshape(shape))]
+
+
+# The five workloads by name; each returns a list of (name, uint16 array).
+WORKLOADS = {
+    "single_1024x1024": lambda: single_matrix(0),
+    "llama8b_block": lambda: llama_block(1000),
+    "adversarial_heavy_tail": lambda: heavy_tail(4001),
+    "adversarial_single_exponent": lambda: single_exponent(4002),
+    "adversarial_uniform_bits": lambda: uniform_bits(4003),
+    "flux_dit_block": lambda: flux_block(5000),
+}
+
+
+def numel(mats) -> int:
+    return int(sum(m.size for _, m in mats))
