@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""DF11 block-decode benchmark on B200.
+
+One step = one df11_decompress_async launch decoding a whole Llama-3.1-8B
+shaped transformer block (7 matrices, 218,103,808 BF16 weights, one codebook)
+from HBM-resident compressed arrays into a BF16 buffer.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Metric: (compressed bytes read + 2 bytes x weights written) / kernel time, in
+GB/s (1e9), with Gweights/s and the fraction of the measured HBM copy peak.
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own block
+(seed 1000 + rank); blocks are independent, so there is no collective on the
+data path and scaling is weak; the time is the max over ranks.
+
+--impl reference times the CPU oracle (serial bit-by-bit decode) on bounded
+samples of the same block, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "DF11 decode GB/s (compressed in + BF16 out), Gweights/s, % of B200 HBM peak"
+UNIT = "GB/s"
+WORKLOAD = "llama8b_block"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "huffman_decode_b200", "csrc", "df11_decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--threads-per-chunk", type=int, default=256)
+    ap.add_argument("--e2e-steps", type=int, default=20,
+                    help="steps of the end-to-end measurement (capped at --steps)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_hash() -> str:
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(n_weights: int):
+    """DRAM bytes per launch from the committed ncu summary, scaled to this
+    launch's weights, or None when the kernel changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_sha256_16") != kernel_hash():
+        return None
+    return float(d["dram_bytes_per_weight"]) * n_weights
+
+
+def make_block(seed: int):
+    return [m for _, m in workloads.llama_block(seed)]
+
+
+# ----------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML during the timed
+    region (background thread, ~5 ms period)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reason_bits = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+                self.reason_bits |= int(self._reasons(self.handle))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def start(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        reasons = [n for b, n in self.REASONS.items() if self.reason_bits & b and b != 0x1]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------- CPU oracle legs
+
+def oracle_sample_plan(ob, n_slices: int):
+    """Split the oracle artifact into n_slices runs of whole chunks; each run
+    decodes serially from its first code start."""
+    T = 256
+    bounds = np.linspace(0, ob.n_chunks, n_slices + 1).astype(np.int64)
+    plan = []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        if b <= a:
+            continue
+        g = int(a) * T
+        start_bit = 64 * g + int(ob.gap[g])
+        plan.append((start_bit, int(ob.pos[a]), int(ob.pos[b] - ob.pos[a])))
+    return plan
+
+
+def time_oracle_decode(oracle, ob, plan_item):
+    start_bit, first, count = plan_item
+    t0 = time.perf_counter()
+    e, _ = oracle.decode(ob.stream, count, ob.lengths, start_bit=start_bit)
+    w = oracle.join(e, ob.signmant[first: first + count])
+    dt = time.perf_counter() - t0
+    return dt, w
+
+
+def cpu_baseline(oracle, hb, cb, bytes_per_weight, seconds):
+    """The oracle's serial decode of the whole block (repeated until about
+    `seconds` of CPU time, at most 4 passes), one core."""
+    total_w = 0
+    total_t = 0.0
+    passes = 0
+    while passes < 4 and (passes == 0 or total_t < seconds):
+        t0 = time.perf_counter()
+        e, _ = oracle.decode(hb.exp_stream, hb.n_elements, cb.lengths())
+        oracle.join(e, hb.signmant[: hb.n_elements])
+        total_t += time.perf_counter() - t0
+        total_w += hb.n_elements
+        passes += 1
+    return {"value": round(total_w * bytes_per_weight / total_t / 1e9, 4), "unit": UNIT,
+            "cores": 1, "kind": "oracle",
+            "gweights_per_s": round(total_w / total_t / 1e9, 5),
+            "sample": f"{passes} full serial decode pass(es) of the llama8b_block "
+                      f"({hb.n_elements} weights each) by the oracle, one thread, "
+                      f"{total_t:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    mats = make_block(1000)
+    n = int(sum(m.size for m in mats))
+    ob = oracle.compress_block(mats)
+    comp_bytes = ob.stream.nbytes + ob.gap.size // 2 + ob.pos.nbytes + (n + 15) // 16 * 16
+    bytes_per_weight = (comp_bytes + 2 * n) / n
+    plan = oracle_sample_plan(ob, 64)
+    for i in range(args.warmup):
+        time_oracle_decode(oracle, ob, plan[i % len(plan)])
+    total_t = 0.0
+    total_w = 0
+    for i in range(args.steps):
+        dt, _ = time_oracle_decode(oracle, ob, plan[i % len(plan)])
+        total_t += dt
+        total_w += plan[i % len(plan)][2]
+    value = total_w * bytes_per_weight / total_t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_t / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "n_weights": n, "seed": 1000,
+                   "sample_per_step": "1/64 of the block's chunks, decoded serially"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"each step decodes 1/64 of the llama8b_block "
+                                   f"(~{n // 64} weights) serially, one thread"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------- GPU arm
+
+def run_b200(args):
+    import torch
+    import torch.distributed as dist
+
+    import huffman_decode_b200 as df11
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    seed = 1000 + rank
+    mats = make_block(seed)
+    t0 = time.perf_counter()
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats, args.threads_per_chunk)
+    compress_s = time.perf_counter() - t0
+    if df11.validate(hb) != 0:
+        raise RuntimeError("compressed block failed validation")
+    n = hb.n_elements
+    comp_bytes = hb.compressed_bytes()
+    bytes_per_step = comp_bytes + 2 * n
+
+    db = hb.to_device(dev)
+    out = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    want = torch.from_numpy(np.concatenate([m.reshape(-1) for m in mats]).view(np.int16)).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    cblk = db.c_struct()
+
+    def step():
+        df11.decompress_async(db, out, err, stream=stream, c_block=cblk)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    bit_exact = bool(torch.equal(out.view(torch.int16), want)) and int(err.item()) == 0
+    if not bit_exact:
+        raise RuntimeError("decode is not bit-exact; refusing to report a number")
+    del want
+
+    sampler = ClockSampler(local)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    end.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = start.elapsed_time(end)
+
+    # ---- end to end: pinned host arrays -> device, decode, BF16 -> host
+    e2e = None
+    if not args.no_e2e:
+        k = max(1, min(args.e2e_steps, args.steps))
+        host = {name: torch.from_numpy(a.view(np.uint8)).pin_memory() for name, a in hb.arrays().items()}
+        host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
+        h2d = sum(t.numel() for t in host.values())
+        d2h = host_out.numel() * 2 + 4
+        host_err = torch.empty(1, dtype=torch.int32, pin_memory=True)
+
+        def e2e_step():
+            for name, t in host.items():
+                db.tensors[name].copy_(t, non_blocking=True)
+            step()
+            host_out.copy_(out, non_blocking=True)
+            host_err.copy_(err, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        s2 = torch.cuda.Event(enable_timing=True)
+        e2 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        s2.record(stream)
+        for _ in range(k):
+            e2e_step()
+        e2.record(stream)
+        e2.synchronize()
+        e2e_ms = s2.elapsed_time(e2)
+        e2e = {"ms": e2e_ms, "k": k, "h2d": h2d, "d2h": d2h}
+
+    # ---- max over ranks, bytes summed over ranks
+    if world > 1:
+        t = torch.tensor([ms, e2e["ms"] / e2e["k"] if e2e else 0.0], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        b = torch.tensor([bytes_per_step, n], dtype=torch.float64, device=dev)
+        dist.all_reduce(b, op=dist.ReduceOp.SUM)
+        ms_max = float(t[0])
+        e2e_ms_per_step = float(t[1])
+        job_bytes, job_weights = float(b[0]), float(b[1])
+    else:
+        ms_max = ms
+        e2e_ms_per_step = e2e["ms"] / e2e["k"] if e2e else 0.0
+        job_bytes, job_weights = float(bytes_per_step), float(n)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        cpu = cpu_baseline(oracle, hb, cb, bytes_per_step / n, args.cpu_baseline_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    ms_per_step = ms_max / args.steps
+    value = job_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    launch_s = ms / args.steps * 1e-3              # this rank's own kernel time per launch
+    achieved = bytes_per_step / launch_s / 1e9
+    traffic = profiled_traffic(n)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "n_weights": n, "n_matrices": len(mats),
+                   "seed": seed, "threads_per_chunk": args.threads_per_chunk,
+                   "bits_per_weight": round(8 + cb.total_bits / n, 4),
+                   "compressed_bytes": comp_bytes, "bytes_per_step": bytes_per_step,
+                   "l2": "inputs larger than L2 (%.2f GB touched per step vs 126 MB L2), no flush"
+                         % (bytes_per_step / 1e9),
+                   "parallelism": f"replicas x{world}, one block per GPU, no collective"},
+        "gweights_per_s": round(job_weights * args.steps / (ms_max * 1e-3) / 1e9, 2),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "bit_exact": bit_exact,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "algorithmic_bytes_per_launch": bytes_per_step},
+        "clocks": clocks,
+        "gpu_launches": args.steps,
+        "host_compress_s": round(compress_s, 3),
+    }
+    if e2e:
+        line["e2e"] = {"value": round(job_bytes / (e2e_ms_per_step * 1e-3) / 1e9, 2), "unit": UNIT,
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e_ms_per_step, 4), "steps": e2e["k"]}
+    if cpu:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_b200(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

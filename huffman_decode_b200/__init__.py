@@ -1,0 +1,12 @@
+"""DFloat11 exponent-stream codec for NVIDIA B200 (sm_100a).
+
+Lossless BF16 weight compression: the exponent byte of every weight is
+canonical-Huffman coded (length cap 16), the sign|mantissa byte is kept raw,
+and one GPU launch per block rebuilds the bit-exact BF16 matrices.  The work
+happens in libdf11.so (C ABI in include/df11.h); this package only binds it.
+"""
+from .df11 import (  # noqa: F401
+    DEVERR_BAD_CODE, DEVERR_BAD_POS, DEVERR_COUNT, DF11Error, DeviceBlock,
+    EXPORTED_SYMBOLS, HostBlock, build_codebook, compress, compress_sizes,
+    decompress_async, library_path, load_library, validate,
+)

@@ -1,0 +1,308 @@
+"""Python binding of the DF11 C ABI (include/df11.h): argument marshalling only.
+
+Every step of the codec runs in libdf11.so -- the host compressor in C++,
+the decode in the sm_100a kernel.  torch is used for device memory and
+streams; numpy for host buffers.  Names follow the C calls:
+
+    cb  = build_codebook(mats, max_code_len=16)
+    hb  = compress(cb, mats, threads_per_chunk=256)
+    validate(hb)
+    db  = hb.to_device("cuda")
+    decompress_async(db, out, error=None, stream=None)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import build as _build
+
+# ------------------------------------------------------------ constants
+
+DF11_OK = 0
+STATUS_NAMES = {
+    0: "DF11_OK", 1: "DF11_ERR_INVALID_ARGUMENT", 2: "DF11_ERR_BUFFER_TOO_SMALL",
+    3: "DF11_ERR_OVERFLOW", 4: "DF11_ERR_CORRUPT", 5: "DF11_ERR_CUDA", 6: "DF11_ERR_TIMEOUT",
+}
+DEVERR_COUNT = 0x1
+DEVERR_BAD_CODE = 0x2
+DEVERR_BAD_POS = 0x4
+MAX_CODE_LEN = 16
+STREAM_PAD = 16
+BYTES_PER_THREAD = 8
+
+EXPORTED_SYMBOLS = (
+    "df11_build_codebook", "df11_compress_sizes", "df11_compress", "df11_validate",
+    "df11_decompress_async", "df11_status_string",
+)
+
+
+class DF11Error(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call} returned {STATUS_NAMES.get(status, status)}")
+
+
+# ------------------------------------------------------- C structures
+
+class Codebook(ctypes.Structure):
+    _fields_ = [
+        ("histogram", ctypes.c_uint64 * 256),
+        ("code", ctypes.c_uint32 * 256),
+        ("code_len", ctypes.c_uint8 * 256),
+        ("max_code_len", ctypes.c_uint32),
+        ("n_symbols", ctypes.c_uint32),
+        ("n_tables", ctypes.c_uint32),
+        ("longest_code", ctypes.c_uint32),
+        ("n_elements", ctypes.c_uint64),
+        ("total_bits", ctypes.c_uint64),
+        ("lut", ctypes.c_uint16 * (256 * 256)),
+    ]
+
+    def lengths(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self.code_len).copy()
+
+    def codes(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self.code).copy()
+
+    def counts(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self.histogram).copy()
+
+    def tables(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self.lut)[: self.n_tables * 256].copy()
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("threads_per_chunk", ctypes.c_uint32), ("bytes_per_thread", ctypes.c_uint32)]
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [
+        ("n_chunks", ctypes.c_uint64), ("n_threads", ctypes.c_uint64),
+        ("exp_stream_bytes", ctypes.c_uint64), ("gaps_bytes", ctypes.c_uint64),
+        ("chunk_pos_count", ctypes.c_uint64), ("signmant_bytes", ctypes.c_uint64),
+        ("lut_entries", ctypes.c_uint64),
+    ]
+
+
+class Header(ctypes.Structure):
+    _fields_ = [
+        ("max_code_len", ctypes.c_uint32), ("threads_per_chunk", ctypes.c_uint32),
+        ("bytes_per_thread", ctypes.c_uint32), ("n_tables", ctypes.c_uint32),
+        ("total_bits", ctypes.c_uint64), ("n_elements", ctypes.c_uint64),
+        ("n_chunks", ctypes.c_uint64),
+    ]
+
+
+class _Block(ctypes.Structure):
+    _fields_ = [
+        ("hdr", Header),
+        ("exp_stream", ctypes.c_void_p), ("exp_stream_bytes", ctypes.c_uint64),
+        ("gaps", ctypes.c_void_p), ("gaps_bytes", ctypes.c_uint64),
+        ("chunk_pos", ctypes.c_void_p), ("chunk_pos_count", ctypes.c_uint64),
+        ("signmant", ctypes.c_void_p), ("signmant_bytes", ctypes.c_uint64),
+        ("lut", ctypes.c_void_p), ("lut_entries", ctypes.c_uint64),
+    ]
+
+
+# ------------------------------------------------------------ loading
+
+_lib = None
+
+
+def load_library(path: str | None = None):
+    """Loads libdf11.so (building it first if a source is newer).  Raises if
+    the library cannot be built or loaded: there is no fallback path."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    if path is None:
+        path = _build.build()
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    U32 = ctypes.c_uint32
+    U64 = ctypes.c_uint64
+    S = ctypes.c_int
+    for name, res, args in (
+        ("df11_build_codebook", S, [P, P, U32, U32, P]),
+        ("df11_compress_sizes", S, [P, P, P]),
+        ("df11_compress", S, [P, P, P, P, U32, P]),
+        ("df11_validate", S, [P]),
+        ("df11_decompress_async", S, [P, P, U64, P, P]),
+        ("df11_status_string", ctypes.c_char_p, [S]),
+    ):
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == _build.LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def _check(status: int, call: str):
+    if status != DF11_OK:
+        raise DF11Error(status, call)
+
+
+def _mats_args(mats):
+    arrs = [np.ascontiguousarray(m, dtype=np.uint16).reshape(-1) for m in mats]
+    ptrs = (ctypes.c_void_p * len(arrs))(*[a.ctypes.data for a in arrs])
+    numel = (ctypes.c_uint64 * len(arrs))(*[a.size for a in arrs])
+    return arrs, ptrs, numel
+
+
+# ------------------------------------------------------------ host calls
+
+def build_codebook(mats, max_code_len: int = MAX_CODE_LEN) -> Codebook:
+    """df11_build_codebook over a list of BF16 bit-pattern arrays (uint16)."""
+    arrs, ptrs, numel = _mats_args(mats)
+    cb = Codebook()
+    _check(load_library().df11_build_codebook(ptrs, numel, len(arrs), max_code_len,
+                                               ctypes.byref(cb)), "df11_build_codebook")
+    return cb
+
+
+def compress_sizes(cb: Codebook, threads_per_chunk: int = 256,
+                   bytes_per_thread: int = BYTES_PER_THREAD) -> Sizes:
+    z = Sizes()
+    ly = Layout(threads_per_chunk, bytes_per_thread)
+    _check(load_library().df11_compress_sizes(ctypes.byref(cb), ctypes.byref(ly),
+                                              ctypes.byref(z)), "df11_compress_sizes")
+    return z
+
+
+@dataclass
+class HostBlock:
+    """A compressed block in host memory (numpy arrays owned by Python)."""
+    header: Header
+    exp_stream: np.ndarray
+    gaps: np.ndarray
+    chunk_pos: np.ndarray
+    signmant: np.ndarray
+    lut: np.ndarray
+    matrix_numel: list = field(default_factory=list)
+
+    def c_struct(self) -> _Block:
+        b = _Block()
+        b.hdr = self.header
+        for name in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut"):
+            a = getattr(self, name)
+            setattr(b, name, a.ctypes.data)
+        b.exp_stream_bytes = self.exp_stream.nbytes
+        b.gaps_bytes = self.gaps.nbytes
+        b.chunk_pos_count = self.chunk_pos.size
+        b.signmant_bytes = self.signmant.nbytes
+        b.lut_entries = self.lut.size
+        return b
+
+    @property
+    def n_elements(self) -> int:
+        return int(self.header.n_elements)
+
+    def compressed_bytes(self) -> int:
+        """Bytes a decode reads: stream, gaps, positions, sign|mantissa, tables."""
+        return int(self.exp_stream.nbytes + self.gaps.nbytes + self.chunk_pos.nbytes
+                   + self.signmant.nbytes + self.lut.nbytes)
+
+    def arrays(self):
+        return {n: getattr(self, n) for n in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")}
+
+    def to_device(self, device="cuda", pin: bool = False) -> "DeviceBlock":
+        import torch
+        t = {}
+        for name, a in self.arrays().items():
+            src = torch.from_numpy(a.view(np.uint8))
+            if pin:
+                src = src.pin_memory()
+            t[name] = src.to(device, non_blocking=pin)
+        return DeviceBlock(header=self.header, tensors=t,
+                           sizes={n: a.nbytes for n, a in self.arrays().items()},
+                           matrix_numel=list(self.matrix_numel))
+
+
+def compress(cb: Codebook, mats, threads_per_chunk: int = 256,
+             bytes_per_thread: int = BYTES_PER_THREAD) -> HostBlock:
+    """df11_compress into freshly allocated numpy buffers of the exact sizes."""
+    arrs, ptrs, numel = _mats_args(mats)
+    z = compress_sizes(cb, threads_per_chunk, bytes_per_thread)
+    hb = HostBlock(
+        header=Header(),
+        exp_stream=np.empty(z.exp_stream_bytes, np.uint8),
+        gaps=np.empty(z.gaps_bytes, np.uint8),
+        chunk_pos=np.empty(z.chunk_pos_count, np.uint32),
+        signmant=np.empty(z.signmant_bytes, np.uint8),
+        lut=np.empty(z.lut_entries, np.uint16),
+        matrix_numel=[a.size for a in arrs],
+    )
+    blk = hb.c_struct()
+    ly = Layout(threads_per_chunk, bytes_per_thread)
+    _check(load_library().df11_compress(ctypes.byref(cb), ctypes.byref(ly), ptrs, numel,
+                                        len(arrs), ctypes.byref(blk)), "df11_compress")
+    hb.header = blk.hdr
+    return hb
+
+
+def validate(hb: HostBlock) -> int:
+    """df11_validate; returns the status code (0 = structurally sound)."""
+    blk = hb.c_struct()
+    return int(load_library().df11_validate(ctypes.byref(blk)))
+
+
+# ------------------------------------------------------------ device call
+
+@dataclass
+class DeviceBlock:
+    """The block's arrays as uint8 torch tensors on one GPU."""
+    header: Header
+    tensors: dict
+    sizes: dict
+    matrix_numel: list = field(default_factory=list)
+
+    def c_struct(self) -> _Block:
+        b = _Block()
+        b.hdr = self.header
+        for name, t in self.tensors.items():
+            setattr(b, name, t.data_ptr())
+        b.exp_stream_bytes = self.sizes["exp_stream"]
+        b.gaps_bytes = self.sizes["gaps"]
+        b.chunk_pos_count = self.sizes["chunk_pos"] // 4
+        b.signmant_bytes = self.sizes["signmant"]
+        b.lut_entries = self.sizes["lut"] // 2
+        return b
+
+    @property
+    def n_elements(self) -> int:
+        return int(self.header.n_elements)
+
+    def compressed_bytes(self) -> int:
+        return int(sum(self.sizes.values()))
+
+
+def decompress_async(db: DeviceBlock, out, error=None, stream=None, c_block=None,
+                     capacity: int | None = None) -> None:
+    """df11_decompress_async: one kernel launch decoding the whole block into
+    `out` (a CUDA tensor of >= n_elements 16-bit elements, e.g. bfloat16 or
+    int16) on `stream` (torch.cuda.Stream, raw handle, or the current stream).
+    `error` is an optional int32 CUDA tensor the kernel ORs error bits into;
+    `capacity` (default out.numel()) is the element count the kernel may write."""
+    import torch
+    if stream is None:
+        handle = torch.cuda.current_stream(out.device).cuda_stream
+    elif isinstance(stream, int):
+        handle = stream
+    else:
+        handle = stream.cuda_stream
+    if out.element_size() != 2 or not out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CUDA tensor of 16-bit elements")
+    blk = c_block if c_block is not None else db.c_struct()
+    err_ptr = error.data_ptr() if error is not None else None
+    cap = out.numel() if capacity is None else min(int(capacity), out.numel())
+    _check(load_library().df11_decompress_async(ctypes.byref(blk), out.data_ptr(), cap,
+                                                err_ptr, handle), "df11_decompress_async")

@@ -1,0 +1,208 @@
+/*
+ * df11.h -- C ABI of the DFloat11 (DF11) exponent-stream codec for B200.
+ *
+ * DF11 stores a BF16 weight as a canonical Huffman code of its 8-bit exponent
+ * plus one raw byte (sign << 7 | 7-bit mantissa); decoding on the GPU rebuilds
+ * the bit-exact BF16 matrices of one transformer block in one launch.
+ * Method: "DFloat11: lossless BFloat16 compression" (ai-infrastructure.net),
+ * sections "What it is" (field split), "Architecture" (hierarchical lookup
+ * tables, the two-phase kernel with Gaps and BlockOutputPos, block-level
+ * batching) and "How it works: the core algorithm" (Huffman lengths,
+ * canonical codes, MSB-first encoding).
+ *
+ * Conventions for every call:
+ *   - Plain C, no exceptions cross the ABI; each call returns df11_status.
+ *   - The caller owns every buffer.  The library allocates no device memory,
+ *     keeps no pointer after a call returns and never synchronises a stream.
+ *   - Host buffers are host pointers; fields documented as "device" are CUDA
+ *     device pointers on the current device.
+ *
+ * Artifact format (one block = every matrix that shares one codebook):
+ *   exponent code  canonical Huffman code, length 1..max_code_len (<= 16),
+ *                  codes assigned in ascending (length, symbol) order.
+ *   exp_stream     codes of all elements, in element order, MSB-first: stream
+ *                  bit i is bit 7 - i%8 of byte i/8.  Zero padded to
+ *                  n_threads * bytes_per_thread + DF11_STREAM_PAD bytes.
+ *   thread slice   thread g owns stream bits [64g, 64g+64) (bytes_per_thread
+ *                  is 8) and decodes every code that STARTS in that slice and
+ *                  before total_bits; a code may run up to 15 bits past it.
+ *   gaps           4-bit offset, per thread, of the first code start in its
+ *                  slice (the end of the stream counts as a start; slices at
+ *                  or past the end hold 0).  Two per byte, thread 2j in the
+ *                  low nibble of byte j.
+ *   chunk_pos      uint32[n_chunks+1]: chunk c (threads_per_chunk threads)
+ *                  writes elements [chunk_pos[c], chunk_pos[c+1]); the last
+ *                  entry is n_elements.  (The pages keep one such 32-bit
+ *                  position per thread block: "BlockOutputPos".)
+ *   signmant       uint8[n_elements] (padded to a multiple of 16): byte k is
+ *                  (sign << 7) | mantissa of element k.
+ *   lut            n_tables * 256 uint16 entries; table 0 is indexed by the
+ *                  next 8 stream bits.  Entry bits:
+ *                    bit 15 = 1       pointer: bits 0..7 name the sub-table
+ *                                     (1..n_tables-1) indexed by the 8 bits
+ *                                     after the first 8;
+ *                    bit 15 = 0       leaf: bits 0..7 the exponent, bits 8..12
+ *                                     the total code length (1..16);
+ *                    bit 14 = 1       no code has this prefix (only in a
+ *                                     single-symbol codebook); bits 8..12 hold
+ *                                     1; a decoder that reads it reports a
+ *                                     corrupt stream.
+ */
+#ifndef DF11_H
+#define DF11_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DF11_OK = 0,
+    DF11_ERR_INVALID_ARGUMENT = 1, /* bad pointer, size, layout or parameter    */
+    DF11_ERR_BUFFER_TOO_SMALL = 2, /* a caller buffer is shorter than required  */
+    DF11_ERR_OVERFLOW = 3,         /* element count >= 2^32                     */
+    DF11_ERR_CORRUPT = 4,          /* artifact fails a structural check         */
+    DF11_ERR_CUDA = 5,             /* a CUDA runtime call failed                */
+    DF11_ERR_TIMEOUT = 6           /* reserved for bounded device waits         */
+} df11_status;
+
+/* Bits the decoder ORs into the caller's device error word. */
+#define DF11_DEVERR_COUNT 0x1u    /* a chunk decoded a different number of codes
+                                     than chunk_pos says (corrupt stream/gaps) */
+#define DF11_DEVERR_BAD_CODE 0x2u /* a window hit a "no code" or bad pointer
+                                     entry (corrupt stream or table)           */
+#define DF11_DEVERR_BAD_POS 0x4u  /* chunk_pos not monotone or beyond
+                                     out_capacity; that chunk writes nothing   */
+
+#define DF11_MAX_CODE_LEN 16u     /* longest code the format allows           */
+#define DF11_MIN_CODE_LEN_CAP 8u  /* smallest cap accepted by build_codebook  */
+#define DF11_STREAM_PAD 16u       /* zero bytes after the last thread slice   */
+#define DF11_BYTES_PER_THREAD 8u  /* the only slice width this build decodes  */
+
+/* Codebook of one block.  Caller-allocated plain data (about 134 KB). */
+typedef struct {
+    uint64_t histogram[256];   /* exponent counts over the block's matrices   */
+    uint32_t code[256];        /* canonical code, right-aligned in code_len   */
+    uint8_t code_len[256];     /* 0 = exponent absent                          */
+    uint32_t max_code_len;     /* the cap the lengths were built under         */
+    uint32_t n_symbols;        /* exponents that occur                         */
+    uint32_t n_tables;         /* lookup tables used in lut (1..256)           */
+    uint32_t longest_code;     /* max code_len                                 */
+    uint64_t n_elements;       /* total elements histogrammed                  */
+    uint64_t total_bits;       /* sum histogram[s] * code_len[s]              */
+    uint16_t lut[256 * 256];   /* first n_tables * 256 entries used            */
+} df11_codebook;
+
+/* Compress-time layout: threads per chunk (decode CTA width) and bytes of
+ * stream per thread.  This build decodes threads_per_chunk in {128, 256, 512}
+ * and bytes_per_thread == 8. */
+typedef struct {
+    uint32_t threads_per_chunk;
+    uint32_t bytes_per_thread;
+} df11_layout;
+
+/* Exact sizes of the arrays df11_compress fills. */
+typedef struct {
+    uint64_t n_chunks;
+    uint64_t n_threads;         /* n_chunks * threads_per_chunk                */
+    uint64_t exp_stream_bytes;  /* n_threads * bytes_per_thread + STREAM_PAD   */
+    uint64_t gaps_bytes;        /* n_threads / 2                               */
+    uint64_t chunk_pos_count;   /* n_chunks + 1 (uint32 entries)               */
+    uint64_t signmant_bytes;    /* n_elements rounded up to a multiple of 16   */
+    uint64_t lut_entries;       /* n_tables * 256 (uint16 entries)             */
+} df11_sizes;
+
+/* Header fields shared by the host and device views of a block. */
+typedef struct {
+    uint32_t max_code_len;
+    uint32_t threads_per_chunk;
+    uint32_t bytes_per_thread;
+    uint32_t n_tables;
+    uint64_t total_bits;
+    uint64_t n_elements;
+    uint64_t n_chunks;
+} df11_header;
+
+/* A compressed block in host memory; every array is caller-owned and sized by
+ * df11_compress_sizes.  `*_bytes` / `*_count` fields give the buffer lengths. */
+typedef struct {
+    df11_header hdr;
+    uint8_t *exp_stream;  uint64_t exp_stream_bytes;
+    uint8_t *gaps;        uint64_t gaps_bytes;
+    uint32_t *chunk_pos;  uint64_t chunk_pos_count;
+    uint8_t *signmant;    uint64_t signmant_bytes;
+    uint16_t *lut;        uint64_t lut_entries;
+} df11_host_block;
+
+/* The same block after the caller copied each array to the GPU (device
+ * pointers).  exp_stream, chunk_pos and lut must be 16-byte aligned, signmant
+ * 8-byte aligned (any cudaMalloc / torch allocation is). */
+typedef struct {
+    df11_header hdr;
+    const uint8_t *exp_stream;  uint64_t exp_stream_bytes;
+    const uint8_t *gaps;        uint64_t gaps_bytes;
+    const uint32_t *chunk_pos;  uint64_t chunk_pos_count;
+    const uint8_t *signmant;    uint64_t signmant_bytes;
+    const uint16_t *lut;        uint64_t lut_entries;
+} df11_device_block;
+
+/* Host.  Histograms the exponents of n_mats BF16 matrices (bit patterns,
+ * host memory, mats[i] holds numel[i] elements), builds optimal code lengths
+ * under max_code_len (in [8, 16]; exactly optimal, not a heuristic), the
+ * canonical codes and the two-level 256-entry lookup tables.
+ * ("What it is"; "Architecture", hierarchical lookup tables; "How it works",
+ * huffman_lengths / canonical_codes.)
+ * Errors: INVALID_ARGUMENT for null pointers, n_mats == 0, zero elements or a
+ * cap outside [8, 16]; OVERFLOW when the element count reaches 2^32. */
+df11_status df11_build_codebook(const uint16_t *const *mats, const uint64_t *numel,
+                                uint32_t n_mats, uint32_t max_code_len,
+                                df11_codebook *out);
+
+/* Host.  Sizes of every array df11_compress fills for this codebook and
+ * layout, from the histogram alone (no pass over the data).
+ * Errors: INVALID_ARGUMENT for an unsupported layout or an empty codebook. */
+df11_status df11_compress_sizes(const df11_codebook *cb, const df11_layout *layout,
+                                df11_sizes *out);
+
+/* Host.  Encodes one block ("Architecture": Gaps, BlockOutputPos; "How it
+ * works": encode).  `out` carries caller buffers of at least the sizes
+ * df11_compress_sizes reports; the call fills them and out->hdr.  The
+ * matrices must be the ones the codebook was built from (same histogram).
+ * Errors: INVALID_ARGUMENT (bad pointers/layout, histogram mismatch),
+ * BUFFER_TOO_SMALL, OVERFLOW. */
+df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
+                          const uint16_t *const *mats, const uint64_t *numel,
+                          uint32_t n_mats, df11_host_block *out);
+
+/* Host.  Structural checks of a block without decoding it: header against
+ * array sizes, chunk_pos monotone from 0 to n_elements, every gap below the
+ * code-length cap, every table entry well formed.  Returns CORRUPT on the
+ * first failure, INVALID_ARGUMENT for null pointers. */
+df11_status df11_validate(const df11_host_block *blk);
+
+/* GPU.  Enqueues ONE kernel launch on `stream` (a cudaStream_t; NULL = the
+ * legacy default stream) that decodes every element of the block into
+ * out_bf16[0 .. n_elements) (device, 16-byte aligned, BF16 bit patterns);
+ * matrix i of the block starts at the sum of the previous matrices' sizes.
+ * ("Architecture": one batched decode per transformer block.)
+ * Host-side checks only: INVALID_ARGUMENT for null or misaligned pointers,
+ * an unsupported layout, array sizes that disagree with the header, or
+ * out_capacity < n_elements; CUDA when the launch fails.  Problems found on
+ * the device (a corrupt artifact) OR DF11_DEVERR_* bits into *d_error
+ * (device uint32, may be NULL; the caller zeroes it); the kernel never writes
+ * outside [0, out_capacity) and never traps.  Safe to call concurrently on
+ * different streams. */
+df11_status df11_decompress_async(const df11_device_block *blk, uint16_t *out_bf16,
+                                  uint64_t out_capacity, uint32_t *d_error,
+                                  void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *df11_status_string(df11_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DF11_H */

@@ -1,0 +1,246 @@
+"""GPU decode (sm_100a kernel, called through the C ABI) against the oracle.
+
+Every output element must equal the oracle's serial bit-by-bit decode of the
+same artifact, which must equal the input BF16 bits: zero tolerance, this is
+integer work.  Workloads: the five configurations at full size plus small and
+degenerate cases.  Page: "DFloat11: lossless BFloat16 compression".
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+import huffman_decode_b200 as df11
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+
+
+def _flat(mats):
+    return np.concatenate([np.ascontiguousarray(m, dtype=np.uint16).reshape(-1) for m in mats])
+
+
+def gpu_decode(hb, capacity=None, guard=0, stream=None):
+    """Decode on cuda:0 into a buffer with `guard` extra elements set to a
+    sentinel; returns (output incl. guard as uint16, error word)."""
+    db = hb.to_device("cuda")
+    n = hb.n_elements
+    out = torch.full((n + guard,), 0x5A5A, dtype=torch.int16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    df11.decompress_async(db, out, err, stream=stream, capacity=capacity)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().view(np.uint16), int(err.item())
+
+
+def check_block(mats, threads_per_chunk=256, oracle_decode=True):
+    w = _flat(mats)
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats, threads_per_chunk)
+    got, err = gpu_decode(hb, guard=8)
+    assert err == 0
+    assert np.all(got[w.size:] == 0x5A5A), "wrote past the block"
+    got = got[: w.size]
+    if oracle_decode:
+        ref = oracle.decode_block(hb.exp_stream, hb.n_elements, cb.lengths(), hb.signmant)
+        assert np.array_equal(ref, w)
+        bad = np.nonzero(got != ref)[0]
+    else:
+        bad = np.nonzero(got != w)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, first at {bad[:8]}"
+    return cb, hb
+
+
+# ------------------------------------------------------------- small cases
+
+SMALL = {
+    "single_1024x1024": lambda: workloads.single_matrix(0),
+    "llama_block_div64": lambda: workloads.llama_block(1000, scale_div=64),
+    "flux_block_div64": lambda: workloads.flux_block(5000, scale_div=64),
+    "heavy_tail_1024": lambda: workloads.heavy_tail(4001, (1024, 1024)),
+    "single_exponent_1024": lambda: workloads.single_exponent(4002, (1024, 1024)),
+    "uniform_bits_1024": lambda: workloads.uniform_bits(4003, (1024, 1024)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+@pytest.mark.parametrize("tpc", [128, 256, 512])
+def test_small_workloads(name, tpc):
+    check_block([m for _, m in SMALL[name]()], threads_per_chunk=tpc)
+
+
+def test_all_bf16_patterns():
+    allw = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    check_block([allw])
+    rng = np.random.default_rng(11)
+    check_block([allw, rng.permutation(allw), allw[::-1].copy()])
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 7, 8, 9, 15, 16, 17, 31, 33, 255, 257])
+def test_tiny_sizes(n):
+    rng = np.random.default_rng(n)
+    w = workloads.to_bf16((rng.standard_normal(n) * 0.02).astype(np.float32))
+    check_block([w])
+
+
+@pytest.mark.parametrize("delta", [-1, 0, 1])
+@pytest.mark.parametrize("tpc", [128, 256])
+def test_chunk_boundary(delta, tpc):
+    n = tpc * 64 + delta                 # 1-bit codes: total bits == elements
+    rng = np.random.default_rng(77)
+    e = np.where(rng.random(n) < 0.5, 0x7A, 0x7B).astype(np.uint16)
+    w = (e << np.uint16(7)) | rng.integers(0, 256, n).astype(np.uint16) & np.uint16(0x807F)
+    cb, hb = check_block([w], threads_per_chunk=tpc)
+    assert hb.header.n_chunks == (1 if delta <= 0 else 2)
+
+
+def test_many_matrices_keep_caller_order():
+    rng = np.random.default_rng(5)
+    mats = [workloads.to_bf16((rng.standard_normal(int(k)) * s).astype(np.float32))
+            for k, s in zip(rng.integers(1, 5000, 40), rng.uniform(0.001, 0.1, 40))]
+    check_block(mats)
+
+
+def test_two_streams_concurrently():
+    a = [m for _, m in workloads.llama_block(1003, scale_div=32)]
+    b = [m for _, m in workloads.heavy_tail(4005, (1024, 2048))]
+    ha = df11.compress(df11.build_codebook(a), a)
+    hbk = df11.compress(df11.build_codebook(b), b)
+    da, dbk = ha.to_device("cuda"), hbk.to_device("cuda")
+    oa = torch.empty(ha.n_elements, dtype=torch.int16, device="cuda")
+    ob = torch.empty(hbk.n_elements, dtype=torch.int16, device="cuda")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        df11.decompress_async(da, oa, stream=s1)
+        df11.decompress_async(dbk, ob, stream=s2)
+    torch.cuda.synchronize()
+    assert np.array_equal(oa.cpu().numpy().view(np.uint16), _flat(a))
+    assert np.array_equal(ob.cpu().numpy().view(np.uint16), _flat(b))
+
+
+# ------------------------------------------------- corrupt input, no trap
+
+def _small_block(seed=21):
+    mats = [m for _, m in workloads.llama_block(seed, scale_div=512)]
+    cb = df11.build_codebook(mats)
+    return mats, cb, df11.compress(cb, mats)
+
+
+def test_wrong_chunk_position_sets_count_bit():
+    mats, cb, hb = _small_block()
+    assert hb.header.n_chunks >= 3
+    hb.chunk_pos[1] += 1
+    got, err = gpu_decode(hb, guard=64)
+    assert err & df11.DEVERR_COUNT
+    assert np.all(got[hb.n_elements:] == 0x5A5A)
+    w = _flat(mats)
+    assert np.array_equal(got[: hb.chunk_pos[1] - 1], w[: hb.chunk_pos[1] - 1])
+
+
+def test_non_monotone_and_out_of_range_positions_write_nothing_outside():
+    mats, cb, hb = _small_block()
+    hb.chunk_pos[2] = hb.chunk_pos[1] - 1
+    got, err = gpu_decode(hb, guard=64)
+    assert err & df11.DEVERR_BAD_POS
+    assert np.all(got[hb.n_elements:] == 0x5A5A)
+    mats, cb, hb = _small_block()
+    n = hb.n_elements
+    hb.chunk_pos[-1] = n + 40          # past the caller's capacity
+    got, err = gpu_decode(hb, capacity=n, guard=64)
+    assert err & df11.DEVERR_BAD_POS
+    assert np.all(got[n:] == 0x5A5A)
+
+
+def test_no_code_window_sets_bad_code_bit():
+    mats = [m for _, m in workloads.single_exponent(4002, (64, 64))]
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats)
+    assert cb.n_symbols == 1 and not hb.exp_stream.any()
+    hb.exp_stream[100] = 0x80          # a '1' bit: no code starts with it
+    got, err = gpu_decode(hb, guard=16)
+    assert err & df11.DEVERR_BAD_CODE
+    assert np.all(got[hb.n_elements:] == 0x5A5A)
+
+
+def _thread_counts(stream, lengths, gap, total_bits, chunk, tpc):
+    """Codes each thread of `chunk` decodes, by the oracle's bit-by-bit decode
+    under the kernel's contract (codes starting in the slice, from its gap)."""
+    n = 0
+    for t in range(tpc):
+        g = chunk * tpc + t
+        p = 64 * g + int(gap[g])
+        end = min(64 * (g + 1), total_bits)
+        while p < end:
+            _, p = oracle.decode(stream, 1, lengths, start_bit=p)
+            n += 1
+    return n
+
+
+def test_flipped_bit_detected_when_chunk_count_changes():
+    """A flipped stream bit desyncs only the thread(s) that read it; the
+    kernel reports it whenever that changes the chunk's code count."""
+    mats = [m for _, m in workloads.single_matrix(0, shape=(64, 512))]
+    cb = df11.build_codebook(mats)
+    L = cb.lengths()
+    rng = np.random.default_rng(99)
+    flagged = 0
+    for trial in range(12):
+        hb = df11.compress(cb, mats)
+        gaps = np.empty(hb.gaps.size * 2, np.uint8)
+        gaps[0::2], gaps[1::2] = hb.gaps & 15, hb.gaps >> 4
+        bit = int(rng.integers(0, hb.header.total_bits))
+        hb.exp_stream[bit // 8] ^= np.uint8(0x80 >> (bit % 8))
+        chunk = bit // (256 * 64)
+        changed = False
+        for c in {max(chunk - 1, 0), chunk}:
+            want = int(hb.chunk_pos[c + 1] - hb.chunk_pos[c])
+            changed |= _thread_counts(hb.exp_stream, L, gaps, hb.header.total_bits, c, 256) != want
+        _, err = gpu_decode(hb)
+        assert bool(err & df11.DEVERR_COUNT) == changed
+        flagged += changed
+    assert flagged > 0
+
+
+# --------------------------------------------------------- full workloads
+
+@pytest.mark.parametrize("name", ["single_1024x1024", "llama8b_block", "adversarial_heavy_tail",
+                                  "adversarial_single_exponent", "adversarial_uniform_bits",
+                                  "flux_dit_block"])
+def test_full_size_workload(name):
+    """The configurations at full size, in the launch configuration the
+    benchmark times (256 threads per chunk), every element compared."""
+    mats = [m for _, m in workloads.WORKLOADS[name]()]
+    check_block(mats, threads_per_chunk=256)
+
+
+def test_model_stream_blocks_into_one_reused_buffer():
+    """The 8B-scale stream decodes block after block into one BF16 buffer on
+    one stream; blocks at both ends of the 32-block stream, full size."""
+    seeds = workloads.llama_model_seeds(32)
+    picks = [seeds[0], seeds[1], seeds[-1]]
+    out = None
+    for sd in picks:
+        mats = [m for _, m in workloads.llama_block(sd)]
+        cb = df11.build_codebook(mats)
+        hb = df11.compress(cb, mats)
+        db = hb.to_device("cuda")
+        if out is None:
+            out = torch.empty(hb.n_elements, dtype=torch.int16, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        df11.decompress_async(db, out, err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        got = out.cpu().numpy().view(np.uint16)
+        if sd == picks[-1]:
+            ref = oracle.decode_block(hb.exp_stream, hb.n_elements, cb.lengths(), hb.signmant)
+            assert np.array_equal(got, ref)
+        assert np.array_equal(got, _flat(mats))
+        del db

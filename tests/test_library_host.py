@@ -1,0 +1,280 @@
+"""Host half of the C-ABI library against the oracle (no GPU needed).
+
+The library's codebook must reach the optimal cost the oracle computes; the
+oracle re-encodes the block from the library's code lengths and must get the
+library's stream, gaps, chunk positions and sign|mantissa bytes byte for byte;
+every 16-bit window walked through the library's two-level tables must give
+the oracle's first code.  Page: "DFloat11: lossless BFloat16 compression".
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+import huffman_decode_b200 as df11
+from huffman_decode_b200 import df11 as binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "df11.h")).read()
+    return sorted(set(re.findall(r"^(?:df11_status|const char \*)\s*(df11_\w+)\s*\(", src, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert set(names) == set(df11.EXPORTED_SYMBOLS)
+    df11.load_library()                       # builds it if needed
+    lib = ctypes.CDLL(df11.library_path())    # a fresh handle, no prototypes set
+    for n in names:
+        assert hasattr(lib, n), n
+    lib.df11_status_string.restype = ctypes.c_char_p
+    assert lib.df11_status_string(0) == b"ok"
+
+
+def _flat(mats):
+    return np.concatenate([np.ascontiguousarray(m, dtype=np.uint16).reshape(-1) for m in mats])
+
+
+def check_format_parity(mats, threads_per_chunk=256, cap=16):
+    """Library artifact == the oracle's artifact built from the library's
+    code lengths; the library's lengths reach the oracle's optimal cost."""
+    cb = df11.build_codebook(mats, cap)
+    hb = df11.compress(cb, mats, threads_per_chunk)
+    assert df11.validate(hb) == 0
+    w = _flat(mats)
+    e, s = oracle.split(w)
+    counts = oracle.histogram(e)
+    assert np.array_equal(cb.counts(), counts)
+    L = cb.lengths()
+    best = oracle.code_lengths(counts, cap)
+    assert oracle.total_bits(counts, L) == oracle.total_bits(counts, best)
+    assert int(L.max()) <= cap
+    ob = oracle.compress_block(mats, cap=cap, threads_per_chunk=threads_per_chunk, lengths=L)
+    assert np.array_equal(cb.codes(), ob.codes)
+    h = hb.header
+    assert (h.total_bits, h.n_elements, h.n_chunks) == (ob.total_bits, w.size, ob.n_chunks)
+    assert np.array_equal(hb.exp_stream, ob.stream)
+    gaps = np.empty(hb.gaps.size * 2, np.uint8)
+    gaps[0::2], gaps[1::2] = hb.gaps & 15, hb.gaps >> 4
+    assert np.array_equal(gaps, ob.gap)
+    assert np.array_equal(hb.chunk_pos, ob.pos)
+    assert np.array_equal(hb.signmant[: w.size], ob.signmant)
+    assert not hb.signmant[w.size:].any()
+    check_tables(hb.lut, int(h.n_tables), L)
+    return cb, hb, ob
+
+
+def check_tables(lut, n_tables, lengths):
+    """Walk every 16-bit window through the two-level tables as the format
+    defines them and compare with the oracle's bit-by-bit first code."""
+    sym, ln = oracle.first_code_table(lengths)
+    t = lut.reshape(-1, 256)[:n_tables].astype(np.int64)
+    v = np.arange(65536)
+    e = t[0][v >> 8]
+    ptr = (e & 0x8000) != 0
+    assert np.all((e[ptr] & 0xFF) >= 1) and np.all((e[ptr] & 0xFF) < n_tables)
+    e[ptr] = t[e[ptr] & 0xFF, v[ptr] & 0xFF]
+    assert not np.any(e & 0x8000)                     # no third level
+    nocode = (e & 0x4000) != 0
+    assert np.array_equal(nocode, ln == 0)
+    ok = ~nocode
+    assert np.array_equal(e[ok] & 0xFF, sym[ok])
+    assert np.array_equal((e[ok] >> 8) & 0x1F, ln[ok])
+
+
+SMALL_WORKLOADS = {
+    "single_1024x1024": lambda: workloads.single_matrix(0),
+    "llama_block_div64": lambda: workloads.llama_block(1000, scale_div=64),
+    "flux_block_div64": lambda: workloads.flux_block(5000, scale_div=64),
+    "heavy_tail_512": lambda: workloads.heavy_tail(4001, (512, 512)),
+    "single_exponent_512": lambda: workloads.single_exponent(4002, (512, 512)),
+    "uniform_bits_512": lambda: workloads.uniform_bits(4003, (512, 512)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL_WORKLOADS))
+def test_format_parity_small_workloads(name):
+    mats = [m for _, m in SMALL_WORKLOADS[name]()]
+    check_format_parity(mats)
+
+
+@pytest.mark.parametrize("tpc", [128, 256, 512])
+def test_format_parity_layouts(tpc):
+    mats = [m for _, m in workloads.llama_block(1001, scale_div=128)]
+    check_format_parity(mats, threads_per_chunk=tpc)
+
+
+@pytest.mark.parametrize("cap", [8, 9, 12, 15, 16])
+def test_codebook_optimal_under_cap(cap):
+    """Fibonacci-like counts push the natural Huffman depth to 23; the
+    library's lengths must meet the oracle's package-merge optimum."""
+    fib = [1, 1]
+    while len(fib) < 24:
+        fib.append(fib[-1] + fib[-2])
+    rng = np.random.default_rng(cap)
+    e = np.repeat(np.arange(100, 124, dtype=np.uint16), fib)
+    rng.shuffle(e)
+    w = (e << np.uint16(7)) | rng.integers(0, 256, e.size).astype(np.uint16) & np.uint16(0x807F)
+    check_format_parity([w], cap=cap)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_codebook_random_alphabets(seed):
+    rng = np.random.default_rng(50 + seed)
+    n_sym = int(rng.integers(2, 257))
+    syms = rng.choice(256, n_sym, replace=False).astype(np.uint16)
+    p = rng.dirichlet(np.full(n_sym, float(rng.uniform(0.05, 2.0))))
+    e = rng.choice(syms, 20000, p=p)
+    w = (e << np.uint16(7)) | (rng.integers(0, 65536, e.size).astype(np.uint16) & np.uint16(0x807F))
+    check_format_parity([w], cap=int(rng.integers(8, 17)) if n_sym <= 256 else 16)
+
+
+def test_all_bf16_patterns_and_tiny_sizes():
+    allw = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    check_format_parity([allw])
+    for n in (1, 2, 7, 8, 9, 15, 16, 17):
+        check_format_parity([allw[12345: 12345 + n]])
+    # several matrices, including a one-element one, in caller order
+    check_format_parity([allw[:5], allw[40000:40001], allw[100:1100]])
+
+
+@pytest.mark.parametrize("delta", [-1, 0, 1])
+def test_chunk_boundary(delta):
+    """Stream lengths one bit under, at and over a whole chunk (256 x 64 bits)."""
+    chunk_bits = 256 * 64
+    # two symbols of 1 bit each: total bits == element count
+    n = chunk_bits + delta
+    rng = np.random.default_rng(7)
+    e = np.where(rng.random(n) < 0.5, 0x7A, 0x7B).astype(np.uint16)
+    w = (e << np.uint16(7)) | rng.integers(0, 128, n).astype(np.uint16)
+    cb, hb, ob = check_format_parity([w])
+    assert hb.header.total_bits == n
+    assert hb.header.n_chunks == (1 if delta <= 0 else 2)
+
+
+def test_decode_of_library_artifact_by_oracle():
+    mats = [m for _, m in workloads.heavy_tail(4001, (256, 512))]
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats)
+    out = oracle.decode_block(hb.exp_stream, hb.n_elements, cb.lengths(), hb.signmant)
+    assert np.array_equal(out, _flat(mats))
+
+
+# ----------------------------------------------------------- error paths
+
+def test_build_codebook_errors():
+    w = np.arange(100, dtype=np.uint16)
+    for cap in (0, 7, 17, 32):
+        with pytest.raises(df11.DF11Error) as ei:
+            df11.build_codebook([w], cap)
+        assert ei.value.status == 1
+    with pytest.raises(df11.DF11Error) as ei:
+        df11.build_codebook([np.zeros(0, np.uint16)])
+    assert ei.value.status == 1
+    lib = df11.load_library()
+    cb = binding.Codebook()
+    assert lib.df11_build_codebook(None, None, 0, 16, ctypes.byref(cb)) == 1
+
+
+def test_compress_errors():
+    rng = np.random.default_rng(3)
+    w = rng.integers(0, 65536, 5000).astype(np.uint16)
+    cb = df11.build_codebook([w])
+    with pytest.raises(df11.DF11Error) as ei:               # different data
+        df11.compress(cb, [w[::-1].copy() ^ np.uint16(0x0080)])
+    assert ei.value.status == 1
+    for tpc in (0, 64, 300, 1024):
+        with pytest.raises(df11.DF11Error):
+            df11.compress(cb, [w], threads_per_chunk=tpc)
+    with pytest.raises(df11.DF11Error):
+        df11.compress(cb, [w], bytes_per_thread=4)
+    # a buffer one entry short
+    hb = df11.compress(cb, [w])
+    blk = hb.c_struct()
+    blk.chunk_pos_count -= 1
+    lib = df11.load_library()
+    arrs, ptrs, numel = binding._mats_args([w])
+    ly = binding.Layout(256, 8)
+    assert lib.df11_compress(ctypes.byref(cb), ctypes.byref(ly), ptrs, numel, 1,
+                             ctypes.byref(blk)) == 2
+
+
+def _fresh_block():
+    mats = [m for _, m in workloads.llama_block(1002, scale_div=256)]
+    cb = df11.build_codebook(mats)
+    return df11.compress(cb, mats)
+
+
+def test_validate_flags_corruption():
+    hb = _fresh_block()
+    assert df11.validate(hb) == 0
+    bad = _fresh_block(); bad.chunk_pos[1], bad.chunk_pos[2] = bad.chunk_pos[2], bad.chunk_pos[1]
+    assert df11.validate(bad) == 4
+    bad = _fresh_block(); bad.chunk_pos[-1] -= 1
+    assert df11.validate(bad) == 4
+    bad = _fresh_block()                       # a gap past the end of the stream
+    g = bad.gaps.size * 2 - 1
+    assert 64 * g >= bad.header.total_bits
+    bad.gaps[g // 2] |= 0x50
+    assert df11.validate(bad) == 4
+    bad = _fresh_block(); bad.gaps[0] |= 0x01  # thread 0 always starts at bit 0
+    assert df11.validate(bad) == 4
+    bad = _fresh_block(); bad.lut[5] = 0x8000 | 200
+    assert df11.validate(bad) == 4
+    bad = _fresh_block(); bad.lut[0] = 0
+    assert df11.validate(bad) == 4
+    bad = _fresh_block(); bad.header.n_chunks += 1
+    assert df11.validate(bad) == 4
+    bad = _fresh_block(); bad.header.total_bits = bad.header.n_elements - 1
+    assert df11.validate(bad) == 4
+
+
+def test_decompress_rejects_bad_arguments_before_any_cuda_call():
+    """Host-side checks only; every case fails before the library touches the
+    CUDA runtime, so this runs without a GPU."""
+    hb = _fresh_block()
+    lib = df11.load_library()
+    fake = 1 << 20                                   # 16-byte aligned, never dereferenced
+
+    def dev_block(**over):
+        b = binding._Block()
+        b.hdr = hb.header
+        for name in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut"):
+            setattr(b, name, fake)
+        b.exp_stream_bytes = hb.exp_stream.nbytes
+        b.gaps_bytes = hb.gaps.nbytes
+        b.chunk_pos_count = hb.chunk_pos.size
+        b.signmant_bytes = hb.signmant.nbytes
+        b.lut_entries = hb.lut.size
+        for k, v in over.items():
+            setattr(b, k, v)
+        return b
+
+    n = hb.n_elements
+    call = lambda b, out=fake, cap=n, err=None: lib.df11_decompress_async(
+        ctypes.byref(b), out, cap, err, None)
+    assert lib.df11_decompress_async(None, fake, n, None, None) == 1
+    assert call(dev_block(), out=None) == 1
+    assert call(dev_block(), cap=n - 1) == 1                       # too little room
+    assert call(dev_block(exp_stream=None)) == 1
+    assert call(dev_block(gaps_bytes=hb.gaps.nbytes - 1)) == 1
+    assert call(dev_block(chunk_pos_count=hb.chunk_pos.size - 1)) == 1
+    assert call(dev_block(lut_entries=hb.lut.size - 1)) == 1
+    assert call(dev_block(exp_stream=fake + 4)) == 1               # misaligned
+    assert call(dev_block(), out=fake + 2) == 1
+    assert call(dev_block(), err=fake + 1) == 1
+    h = binding.Header.from_buffer_copy(hb.header)
+    h.threads_per_chunk = 64
+    assert call(dev_block(hdr=h)) == 1
+    h = binding.Header.from_buffer_copy(hb.header)
+    h.n_chunks += 1
+    assert call(dev_block(hdr=h)) == 1
+    h = binding.Header.from_buffer_copy(hb.header)
+    h.n_tables = 0
+    assert call(dev_block(hdr=h)) == 1

@@ -20,9 +20,20 @@ def to_bf16(x: np.ndarray) -> np.ndarray:
     The rounding the page "DFloat11: lossless BFloat16 compression" uses to
     make its synthetic tensor (section "How it works: the core algorithm").
     """
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    r = (u >> np.uint32(16)) & np.uint32(1)
-    return ((u + np.uint32(0x7FFF) + r) >> np.uint32(16)).astype(np.uint16)
+    u = np.ascontiguousarray(x, dtype=np.float32).reshape(-1).view(np.uint32)
+    out = np.empty(u.size, np.uint16)
+    step = 1 << 20
+    r = np.empty(min(step, u.size), np.uint32)
+    for lo in range(0, u.size, step):
+        a = u[lo: lo + step]
+        t = r[: a.size]
+        np.right_shift(a, 16, out=t)
+        np.bitwise_and(t, 1, out=t)
+        np.add(t, 0x7FFF, out=t)
+        np.add(t, a, out=t)
+        np.right_shift(t, 16, out=t)
+        out[lo: lo + a.size] = t
+    return out.reshape(np.shape(x))
 
 
 def _normal_bf16(rng: np.random.Generator, shape, sigma: float) -> np.ndarray:
