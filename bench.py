@@ -50,7 +50,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--threads-per-chunk", type=int, default=256)
+    ap.add_argument("--bytes-per-thread", type=int, default=8, choices=[8, 16],
+                    help="stream bytes each decoding thread owns (format layout)")
+    ap.add_argument("--scale-div", type=int, default=1,
+                    help="divide every row count of the block (smaller case for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=20,
                     help="steps of the end-to-end measurement (capped at --steps)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -87,8 +90,8 @@ def profiled_traffic(n_weights: int):
     return float(d["dram_bytes_per_weight"]) * n_weights
 
 
-def make_block(seed: int):
-    return [m for _, m in workloads.llama_block(seed)]
+def make_block(seed: int, scale_div: int = 1):
+    return [m for _, m in workloads.llama_block(seed, scale_div=scale_div)]
 
 
 # ----------------------------------------------------------- clocks
@@ -144,17 +147,16 @@ class ClockSampler:
 
 # ------------------------------------------------------- CPU oracle legs
 
-def oracle_sample_plan(ob, n_slices: int):
+def oracle_sample_plan(ob, n_slices: int, threads_per_chunk: int = 32, slice_bits: int = 64):
     """Split the oracle artifact into n_slices runs of whole chunks; each run
     decodes serially from its first code start."""
-    T = 256
     bounds = np.linspace(0, ob.n_chunks, n_slices + 1).astype(np.int64)
     plan = []
     for a, b in zip(bounds[:-1], bounds[1:]):
         if b <= a:
             continue
-        g = int(a) * T
-        start_bit = 64 * g + int(ob.gap[g])
+        g = int(a) * threads_per_chunk
+        start_bit = slice_bits * g + int(ob.gap[g])
         plan.append((start_bit, int(ob.pos[a]), int(ob.pos[b] - ob.pos[a])))
     return plan
 
@@ -245,10 +247,10 @@ def run_b200(args):
                                 device_id=dev)
 
     seed = 1000 + rank
-    mats = make_block(seed)
+    mats = make_block(seed, args.scale_div)
     t0 = time.perf_counter()
     cb = df11.build_codebook(mats)
-    hb = df11.compress(cb, mats, args.threads_per_chunk)
+    hb = df11.compress(cb, mats, 32, args.bytes_per_thread)
     compress_s = time.perf_counter() - t0
     if df11.validate(hb) != 0:
         raise RuntimeError("compressed block failed validation")
@@ -360,8 +362,9 @@ def run_b200(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "u8", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n_weights": n, "n_matrices": len(mats),
-                   "seed": seed, "threads_per_chunk": args.threads_per_chunk,
+        "config": {"workload": WORKLOAD if args.scale_div == 1 else f"{WORKLOAD}/rows{args.scale_div}",
+                   "n_weights": n, "n_matrices": len(mats),
+                   "seed": seed, "threads_per_chunk": 32, "bytes_per_thread": args.bytes_per_thread,
                    "bits_per_weight": round(8 + cb.total_bits / n, 4),
                    "compressed_bytes": comp_bytes, "bytes_per_step": bytes_per_step,
                    "l2": "inputs larger than L2 (%.2f GB touched per step vs 126 MB L2), no flush"

@@ -1,25 +1,31 @@
 // df11_decode.cu -- GPU decode of one DF11 block into BF16 (sm_100a).
 //
 // Method: "DFloat11: lossless BFloat16 compression" (ai-infrastructure.net),
-// section "Architecture": each thread owns a fixed 8-byte slice of the
-// exponent stream and starts at its Gaps offset; a block-wide prefix sum of
-// per-thread counts places the outputs; exponents are joined with the raw
-// sign|mantissa bytes and written with coalesced stores; one launch covers
-// every matrix of a block.
+// section "Architecture": each thread owns a fixed slice of the exponent
+// stream and starts at its Gaps offset; a prefix sum of per-thread code
+// counts places the outputs; exponents are joined with the raw sign|mantissa
+// bytes and written with coalesced stores; one launch covers every matrix of
+// a block (block-level batching).
 //
 // B200 design (differs from the page's two-phase kernel):
-//   * single decode pass: each thread decodes its slice once, packing four
-//     exponents per 32-bit word into a shared-memory slot column (conflict
-//     free: at any loop step all active lanes write the same slot row);
-//   * warp-shuffle + block scan of the counts; the words are then compacted
-//     into a contiguous exponent buffer placed at the chunk's 8-element
-//     alignment, so the merge reads 8 exponents and 8 sign|mantissa bytes
-//     per thread and writes one 16-byte BF16 vector per thread;
-//   * 16-bit table entries carrying (symbol, total length) or a sub-table
-//     pointer, sanitised once per CTA when copied to shared memory, so the
-//     hot loop needs no bounds checks;
-//   * persistent CTAs, grid = resident CTAs per SM x SM count.
-// No tensor cores: this is integer decode, bounded by HBM and issue rate.
+//   * one warp = one chunk: output positions are stored per 32 threads, so
+//     every warp decodes, scans (shuffles), compacts and stores on its own,
+//     with no block-wide barrier after the prologue;
+//   * single decode pass with a multi-code table: a 10-bit window indexes a
+//     1024-entry table (built in shared memory from the format's two-level
+//     16-bit tables) that yields up to three whole codes per lookup; longer
+//     codes fall back to the two-level tables;
+//   * decoded exponents are packed four per word into a per-warp slot column
+//     (row k holds word k of every lane: conflict-free stores), then moved
+//     into a contiguous, 8-element-aligned exponent buffer with funnel-shifted
+//     word stores (shared-memory OR only on words two lanes share);
+//   * the sign|mantissa bytes of the chunk and the next chunk's stream words
+//     are loaded into registers before decoding, so their latency hides
+//     behind the decode;
+//   * the merge joins 8 exponents with 8 sign|mantissa bytes per lane and
+//     writes one 16-byte BF16 vector per lane;
+//   * persistent CTAs: grid = resident CTAs per SM x SM count.
+// No tensor cores: this is integer decode, bounded by HBM traffic and issue.
 #include "df11.h"
 
 #include <cuda_runtime.h>
@@ -29,10 +35,12 @@
 
 namespace {
 
-constexpr int kSlotRows = 16;          // 64 codes max per 64-bit slice, 4 per word
-constexpr int kSliceBits = 64;
 constexpr uint32_t kLutPointer = 0x8000u;
 constexpr uint32_t kLutNoCode = 0x4000u | (1u << 8);
+constexpr int kWindowBits = 10;                    // multi-code table index width
+constexpr int kMultiEntries = 1 << kWindowBits;
+constexpr int kMaxCodesPerEntry = 3;
+constexpr int kPrefetchGroups = 4;                 // 8-byte sign|mantissa groups per lane
 
 struct DecodeParams {
     const uint8_t *stream;
@@ -48,16 +56,29 @@ struct DecodeParams {
     uint32_t n_tables;
 };
 
-template <int T>
+// Shared-memory layout per CTA: multi-code table, per-warp slot columns and
+// exponent buffers, then the two-level tables.
+template <int W>
+struct Geometry {
+    static constexpr int kSliceBits = 8 * W;              // 64 or 128
+    static constexpr int kMaxCodes = kSliceBits;          // 1-bit codes at most
+    static constexpr int kSlotRows = kMaxCodes / 4;
+    static constexpr int kSlotBytes = kSlotRows * 32 * 4; // per warp
+    static constexpr int kEbufBytes = 32 * kMaxCodes + 16; // per warp, multiple of 16
+    static constexpr int kWords = W / 4 + 1;              // stream words per lane incl. halo
+};
+
+template <int W, int WARPS>
 constexpr size_t smem_bytes_for(uint32_t n_tables)
 {
-    return (size_t)kSlotRows * T * 4 + (size_t)kSliceBits * T + 16 + (size_t)n_tables * 512;
+    using G = Geometry<W>;
+    return (size_t)kMultiEntries * 4 + (size_t)WARPS * (G::kSlotBytes + G::kEbufBytes) +
+           (size_t)n_tables * 512;
 }
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
-// Two BF16 words from two exponent bytes (low 16 bits of e, s) and two
-// sign|mantissa bytes: v = [s0 e0 s1 e1] as bytes; per 16-bit half,
+// Two BF16 words from v = [s0 e0 s1 e1] (bytes, low first): per 16-bit half,
 // exponent -> bits 14..7, sign -> bit 15, mantissa -> bits 6..0.
 __device__ __forceinline__ uint32_t join2(uint32_t v)
 {
@@ -69,160 +90,295 @@ __device__ __forceinline__ uint16_t join1(uint32_t e, uint32_t s)
     return (uint16_t)(((s & 0x80u) << 8) | (e << 7) | (s & 0x7Fu));
 }
 
-template <int T>
-__global__ void __launch_bounds__(T) df11_decode_kernel(DecodeParams p)
+// Loads lane's stream words (big-endian, MSB-first bit order) and gap.
+template <int W>
+__device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, uint32_t (&w)[Geometry<W>::kWords],
+                                           uint32_t &gap)
 {
+    const uint8_t *src = p.stream + (uint64_t)W * g;
+    if constexpr (W == 8) {
+        const uint2 a = *reinterpret_cast<const uint2 *>(src);
+        w[0] = bswap32(a.x);
+        w[1] = bswap32(a.y);
+        w[2] = bswap32(*reinterpret_cast<const uint32_t *>(src + 8));
+    } else {
+        const uint4 a = *reinterpret_cast<const uint4 *>(src);
+        w[0] = bswap32(a.x);
+        w[1] = bswap32(a.y);
+        w[2] = bswap32(a.z);
+        w[3] = bswap32(a.w);
+        w[4] = bswap32(*reinterpret_cast<const uint32_t *>(src + 16));
+    }
+    gap = (p.gaps[g >> 1] >> ((g & 1) * 4)) & 0xFu;
+}
+
+template <int W, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
+{
+    using G = Geometry<W>;
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t *slots = reinterpret_cast<uint32_t *>(smem);               // [kSlotRows][T]
-    uint8_t *ebuf = smem + (size_t)kSlotRows * T * 4;                   // 64*T + 16
-    uint16_t *lut = reinterpret_cast<uint16_t *>(ebuf + kSliceBits * T + 16);
-    __shared__ uint32_t warp_excl[T / 32];
-    __shared__ uint32_t chunk_info[3];
+    uint32_t *multi = reinterpret_cast<uint32_t *>(smem);
+    uint8_t *warp_area = smem + kMultiEntries * 4;
+    uint16_t *lut = reinterpret_cast<uint16_t *>(warp_area + WARPS * (G::kSlotBytes + G::kEbufBytes));
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const uint32_t n_tables = p.n_tables;
 
-    // Tables -> shared memory.  Anything malformed becomes a "no code" entry
-    // (length 1), so the decode loop below always advances and never indexes
-    // outside the tables.
-    for (uint32_t i = tid; i < n_tables * 256u; i += T) {
+    // ---- prologue: two-level tables, sanitised ------------------------------
+    // Anything malformed becomes "no code" (length 1), so decoding always
+    // advances and never indexes outside the tables.
+    for (uint32_t i = tid; i < n_tables * 256u; i += WARPS * 32) {
         uint32_t e = p.lut[i];
         if (e & kLutPointer) {
-            uint32_t to = e & 0xFFu;
+            const uint32_t to = e & 0xFFu;
             if (i >= 256u || to == 0 || to >= n_tables || (e & 0x7F00u))
                 e = kLutNoCode;
         } else {
-            uint32_t l = (e >> 8) & 0x1Fu;
+            const uint32_t l = (e >> 8) & 0x1Fu;
             if ((e & 0x4000u) || l == 0 || l > 16)
                 e = kLutNoCode;
         }
         lut[i] = (uint16_t)e;
     }
     __syncthreads();
+    // ---- prologue: multi-code table -----------------------------------------
+    // Entry for a 10-bit window: the whole codes it starts with (at most 3),
+    // as symbols in bytes 0..2, their count in bits 24..25 and their total
+    // length in bits 28..31.  0 when the first code is longer than the window
+    // (or is no code): the decoder then takes the two-level path.
+    for (int idx = tid; idx < kMultiEntries; idx += WARPS * 32) {
+        const uint32_t win = (uint32_t)idx << (32 - kWindowBits);
+        uint32_t t = 0, n = 0, syms = 0;
+        while (n < kMaxCodesPerEntry) {
+            const uint32_t v = win << t;
+            uint32_t e = lut[v >> 24];
+            if (e & kLutPointer)
+                e = lut[((e & 0xFFu) << 8) | ((v >> 16) & 0xFFu)];
+            if (e & 0x4000u)
+                break;
+            const uint32_t l = (e >> 8) & 0x1Fu;
+            if (t + l > (uint32_t)kWindowBits)
+                break;
+            syms |= (e & 0xFFu) << (8 * n);
+            ++n;
+            t += l;
+        }
+        multi[idx] = n ? (syms | (n << 24) | (t << 28)) : 0u;
+    }
+    __syncthreads();
+
+    uint32_t *slots = reinterpret_cast<uint32_t *>(warp_area + warp * (G::kSlotBytes + G::kEbufBytes));
+    uint8_t *ebuf = warp_area + warp * (G::kSlotBytes + G::kEbufBytes) + G::kSlotBytes;
+    uint32_t *ebuf32 = reinterpret_cast<uint32_t *>(ebuf);
+
+    const uint64_t stride = (uint64_t)gridDim.x * WARPS;
+    uint64_t chunk = (uint64_t)blockIdx.x * WARPS + warp;
+    if (chunk >= p.n_chunks)
+        return;
 
     uint32_t err = 0;
-    for (uint64_t chunk = blockIdx.x; chunk < p.n_chunks; chunk += gridDim.x) {
-        // ---- decode this thread's slice -------------------------------
-        const uint64_t g = chunk * T + tid;
-        const uint64_t bit0 = g * kSliceBits;
-        const uint2 v01 = *reinterpret_cast<const uint2 *>(p.stream + 8 * g);
-        const uint32_t v2 = *reinterpret_cast<const uint32_t *>(p.stream + 8 * g + 8);
-        const uint32_t gap = (p.gaps[g >> 1] >> ((g & 1) * 4)) & 0xFu;
-        const int end = bit0 >= p.total_bits ? 0
-                        : (int)min((uint64_t)kSliceBits, p.total_bits - bit0);
-        uint32_t hi = bswap32(v01.x), lo = bswap32(v01.y);
-        const uint32_t w2 = bswap32(v2);
-        int bitpos = (int)gap;
-        uint32_t count = 0, acc = 0, seen = 0;
+    uint32_t w[G::kWords];
+    uint32_t gap;
+    load_slice<W>(p, chunk * 32 + lane, w, gap);
+    uint32_t pos0 = p.chunk_pos[chunk], pos1 = p.chunk_pos[chunk + 1];
+
+    for (;;) {
+        // ---- positions of this chunk (warp-uniform) ------------------------
+        const bool pos_ok = pos0 <= pos1 && (uint64_t)pos1 <= p.out_limit &&
+                            pos1 - pos0 <= (uint32_t)(32 * G::kMaxCodes);
+        const uint32_t head = pos0 & 7u;
+        const uint64_t base = (uint64_t)pos0 - head;           // 8-element aligned
+        const uint32_t groups = pos_ok ? (head + (pos1 - pos0) + 7) >> 3 : 0u;
+
+        // ---- loads for later: sign|mantissa of this chunk, next slice -------
+        uint2 pre[kPrefetchGroups];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int lim = min(end, 32 * (half + 1));
-            while (bitpos < lim) {
-                const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
+        for (int j = 0; j < kPrefetchGroups; ++j) {
+            const uint32_t i = lane + 32 * j;
+            if (i < groups)
+                pre[j] = __ldg(reinterpret_cast<const uint2 *>(p.signmant + base + 8ull * i));
+            else
+                pre[j] = make_uint2(0u, 0u);
+        }
+        const uint64_t next = chunk + stride;
+        const bool has_next = next < p.n_chunks;
+        uint32_t nw[G::kWords];
+        uint32_t ngap = 0, npos0 = 0, npos1 = 0;
+        if (has_next) {
+            load_slice<W>(p, next * 32 + lane, nw, ngap);
+            npos0 = p.chunk_pos[next];
+            npos1 = p.chunk_pos[next + 1];
+        }
+
+        if (!pos_ok) {
+            err |= DF11_DEVERR_BAD_POS;
+        } else {
+            // ---- decode this lane's slice ----------------------------------
+            // Codes starting in [gap, end) belong to this lane.  While at
+            // least kWindowBits bits remain before `end`, every code a table
+            // entry returns starts inside the slice; the last few bits go
+            // through the checked tail loop.
+            const uint64_t bit0 = (chunk * 32 + lane) * (uint64_t)G::kSliceBits;
+            const int end = bit0 >= p.total_bits
+                                ? 0
+                                : (int)min((uint64_t)G::kSliceBits, p.total_bits - bit0);
+            int bitpos = (int)gap;
+            uint32_t count = 0, nb = 0, row = 0, accl = 0, acch = 0, seen = 0;
+            // appends the codes of entry r (symbols in bytes 0..2, count in
+            // bits 24..25) to the lane's packed slot column
+            auto append = [&](uint32_t r) {
+                const uint32_t n = (r >> 24) & 3u;
+                const uint64_t s = (uint64_t)(r & 0xFFFFFFu) << (8 * nb);
+                accl |= (uint32_t)s;
+                acch |= (uint32_t)(s >> 32);
+                nb += n;
+                count += n;
+                if (nb >= 4) {
+                    slots[row * 32 + lane] = accl;
+                    ++row;
+                    accl = acch;
+                    acch = 0;
+                    nb -= 4;
+                }
+            };
+            // one code through the two-level tables, as an entry with count 1
+            auto single = [&](uint32_t win, uint32_t &adv) -> uint32_t {
                 uint32_t e = lut[win >> 24];
                 if (e & kLutPointer)
                     e = lut[((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)];
                 seen |= e;
-                acc = (acc >> 8) | (e << 24);
-                bitpos += (int)((e >> 8) & 0x1Fu);
-                ++count;
-                if ((count & 3u) == 0)
-                    slots[((count >> 2) - 1) * T + tid] = acc;
-            }
-            hi = lo;
-            lo = w2;
-        }
-        if (count & 3u)
-            slots[(count >> 2) * T + tid] = acc >> (8 * (4 - (count & 3u)));
-        if (seen & 0x4000u)
-            err |= DF11_DEVERR_BAD_CODE;
-
-        // ---- block scan of the counts ----------------------------------
-        uint32_t incl = count;
+                adv = (e >> 8) & 0x1Fu;
+                return (e & 0xFFu) | (1u << 24);
+            };
 #pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d)
-                incl += y;
-        }
-        if (lane == 31)
-            warp_excl[warp] = incl;
-        if (tid == 0) {
-            chunk_info[0] = p.chunk_pos[chunk];
-            chunk_info[1] = p.chunk_pos[chunk + 1];
-        }
-        __syncthreads();
-        if (warp == 0) {
-            const uint32_t ws = lane < T / 32 ? warp_excl[lane] : 0u;
-            uint32_t wi = ws;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, wi, d);
-                if (lane >= d)
-                    wi += y;
-            }
-            if (lane < T / 32)
-                warp_excl[lane] = wi - ws;
-            if (lane == 31)
-                chunk_info[2] = wi;
-        }
-        __syncthreads();
-
-        const uint32_t pos0 = chunk_info[0];
-        const uint32_t pos1 = chunk_info[1];
-        const uint32_t total = chunk_info[2];
-        // uniform across the CTA: every thread takes the same branch
-        if (pos1 < pos0 || (uint64_t)pos1 > p.out_limit || pos1 - pos0 > (uint32_t)(kSliceBits * T)) {
-            err |= DF11_DEVERR_BAD_POS;
-            __syncthreads();  // chunk_info is rewritten by the next chunk
-            continue;
-        }
-        if (total != pos1 - pos0)
-            err |= DF11_DEVERR_COUNT;
-        const uint32_t n_write = min(total, pos1 - pos0);
-
-        // ---- compaction into the chunk's exponent buffer ----------------
-        const uint32_t head = pos0 & 7u;
-        const uint32_t off = warp_excl[warp] + incl - count;
-        uint8_t *dst = ebuf + head + off;
-        for (uint32_t q = 0; q * 4 < count; ++q) {
-            const uint32_t w = slots[q * T + tid];
-#pragma unroll
-            for (uint32_t b = 0; b < 4; ++b) {
-                const uint32_t k = q * 4 + b;
-                if (k < count && off + k < n_write)
-                    dst[k] = (uint8_t)(w >> (8 * b));
-            }
-        }
-        __syncthreads();
-
-        // ---- merge with sign|mantissa and store -------------------------
-        const uint64_t base = (uint64_t)pos0 - head;       // 8-element aligned
-        const uint32_t span = head + n_write;
-        const uint32_t groups = (span + 7) / 8;
-        for (uint32_t i = tid; i < groups; i += T) {
-            const uint32_t l0 = 8 * i;
-            const uint64_t g0 = base + l0;
-            if (l0 >= head && l0 + 8 <= span) {
-                const uint2 e8 = *reinterpret_cast<const uint2 *>(ebuf + l0);
-                const uint2 s8 = __ldg(reinterpret_cast<const uint2 *>(p.signmant + g0));
-                uint4 o;
-                o.x = join2(__byte_perm(s8.x, e8.x, 0x5140));
-                o.y = join2(__byte_perm(s8.x, e8.x, 0x7362));
-                o.z = join2(__byte_perm(s8.y, e8.y, 0x5140));
-                o.w = join2(__byte_perm(s8.y, e8.y, 0x7362));
-                *reinterpret_cast<uint4 *>(p.out + g0) = o;
-            } else {
-                for (uint32_t j = 0; j < 8; ++j) {
-                    const uint32_t l = l0 + j;
-                    if (l >= head && l < span)
-                        p.out[base + l] = join1(ebuf[l], p.signmant[base + l]);
+            for (int h = 0; h < G::kWords - 1; ++h) {
+                const uint32_t hi = w[h], lo = w[h + 1];
+                const int lim = min(end - kWindowBits, 32 * (h + 1));
+                while (bitpos < lim) {
+                    const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
+                    uint32_t r = multi[win >> (32 - kWindowBits)];
+                    uint32_t adv = r >> 28;
+                    if (r < (1u << 28))
+                        r = single(win, adv);
+                    bitpos += (int)adv;
+                    append(r);
                 }
             }
+            while (bitpos < end) {
+                const int h = bitpos >> 5;
+                uint32_t hi = w[0], lo = w[1];
+#pragma unroll
+                for (int k = 1; k < G::kWords - 1; ++k) {
+                    if (h == k) {
+                        hi = w[k];
+                        lo = w[k + 1];
+                    }
+                }
+                const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
+                uint32_t r = multi[win >> (32 - kWindowBits)];
+                uint32_t adv = r >> 28;
+                if (r < (1u << 28) || bitpos + (int)adv > end)
+                    r = single(win, adv);
+                bitpos += (int)adv;
+                append(r);
+            }
+            if (nb)
+                slots[row * 32 + lane] = accl;
+            if (seen & 0x4000u)
+                err |= DF11_DEVERR_BAD_CODE;
+
+            // ---- warp scan of the counts ------------------------------------
+            uint32_t incl = count;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+                if (lane >= d)
+                    incl += y;
+            }
+            const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+            const uint32_t off = incl - count;
+            if (total != pos1 - pos0)
+                err |= DF11_DEVERR_COUNT;
+            const uint32_t n_write = min(total, pos1 - pos0);
+
+            // ---- compaction into the exponent buffer ------------------------
+            for (int i = lane; i < G::kEbufBytes / 16; i += 32)
+                reinterpret_cast<uint4 *>(ebuf)[i] = make_uint4(0u, 0u, 0u, 0u);
+            __syncwarp();
+            const uint32_t nbytes = off < n_write ? min(count, n_write - off) : 0u;
+            if (nbytes) {
+                const uint32_t a = head + off;                 // byte address in ebuf
+                const uint32_t sh = (a & 3u) * 8;
+                const uint32_t first = a >> 2;
+                const uint32_t last = (a + nbytes - 1) >> 2;
+                const bool end_partial = ((a + nbytes) & 3u) != 0;
+                const uint32_t nwords = (nbytes + 3) >> 2;
+                const uint32_t tail_mask = (nbytes & 3u) ? (1u << (8 * (nbytes & 3u))) - 1 : ~0u;
+                uint32_t prev = 0;
+                for (uint32_t j = 0; j <= last - first; ++j) {
+                    uint32_t cur = 0;
+                    if (j < nwords) {
+                        cur = slots[j * 32 + lane];
+                        if (j == nwords - 1)
+                            cur &= tail_mask;
+                    }
+                    const uint32_t v = __funnelshift_l(prev, cur, sh);
+                    prev = cur;
+                    const bool shared = (j == 0 && sh != 0) || (first + j == last && end_partial);
+                    if (shared)
+                        atomicOr(ebuf32 + first + j, v);
+                    else
+                        ebuf32[first + j] = v;
+                }
+            }
+            __syncwarp();
+
+            // ---- merge with sign|mantissa and store -------------------------
+            const uint32_t span = head + n_write;
+            const uint32_t mgroups = (span + 7) >> 3;
+            auto merge_group = [&](uint32_t i, uint2 s8) {
+                const uint32_t l0 = 8 * i;
+                const uint64_t g0 = base + l0;
+                if (l0 >= head && l0 + 8 <= span) {
+                    const uint2 e8 = *reinterpret_cast<const uint2 *>(ebuf + l0);
+                    uint4 o;
+                    o.x = join2(__byte_perm(s8.x, e8.x, 0x5140));
+                    o.y = join2(__byte_perm(s8.x, e8.x, 0x7362));
+                    o.z = join2(__byte_perm(s8.y, e8.y, 0x5140));
+                    o.w = join2(__byte_perm(s8.y, e8.y, 0x7362));
+                    *reinterpret_cast<uint4 *>(p.out + g0) = o;
+                } else {
+                    for (uint32_t k = 0; k < 8; ++k) {
+                        const uint32_t l = l0 + k;
+                        if (l >= head && l < span) {
+                            const uint32_t sb = ((k < 4 ? s8.x : s8.y) >> (8 * (k & 3))) & 0xFFu;
+                            p.out[base + l] = join1(ebuf[l], sb);
+                        }
+                    }
+                }
+            };
+#pragma unroll
+            for (int j = 0; j < kPrefetchGroups; ++j) {
+                const uint32_t i = lane + 32 * j;
+                if (i < mgroups)
+                    merge_group(i, pre[j]);
+            }
+            for (uint32_t i = lane + 32 * kPrefetchGroups; i < mgroups; i += 32)
+                merge_group(i, __ldg(reinterpret_cast<const uint2 *>(p.signmant + base + 8ull * i)));
+            __syncwarp();
         }
-        __syncthreads();
+
+        if (!has_next)
+            break;
+        chunk = next;
+#pragma unroll
+        for (int k = 0; k < G::kWords; ++k)
+            w[k] = nw[k];
+        gap = ngap;
+        pos0 = npos0;
+        pos1 = npos1;
     }
     if (err && p.err)
         atomicOr(p.err, err);
@@ -231,22 +387,23 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(DecodeParams p)
 // ------------------------------------------------------------ launch
 
 constexpr int kMaxDevices = 64;
-// resident CTAs per SM, by device, threads-per-chunk variant and table count
-std::atomic<int> g_occupancy[kMaxDevices][3][257];
+constexpr int kWarpsPerCta = 8;
+// resident CTAs per SM, by device, slice width and table count
+std::atomic<int> g_occupancy[kMaxDevices][2][257];
 std::atomic<int> g_sm_count[kMaxDevices];
-std::atomic<int> g_attr_done[kMaxDevices][3];
+std::atomic<int> g_attr_done[kMaxDevices][2];
 
-template <int T>
-df11_status launch(const DecodeParams &prm, int dev, int variant, cudaStream_t stream)
+template <int W>
+df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream)
 {
-    const size_t smem = smem_bytes_for<T>(prm.n_tables);
-    if (!g_attr_done[dev][variant].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(df11_decode_kernel<T>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem_bytes_for<T>(256));
-        if (e != cudaSuccess)
+    constexpr int v = W == 8 ? 0 : 1;
+    auto kernel = df11_decode_kernel<W, kWarpsPerCta>;
+    const size_t smem = smem_bytes_for<W, kWarpsPerCta>(prm.n_tables);
+    if (!g_attr_done[dev][v].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_bytes_for<W, kWarpsPerCta>(256)) != cudaSuccess)
             return DF11_ERR_CUDA;
-        g_attr_done[dev][variant].store(1, std::memory_order_release);
+        g_attr_done[dev][v].store(1, std::memory_order_release);
     }
     int sms = g_sm_count[dev].load(std::memory_order_relaxed);
     if (sms == 0) {
@@ -254,18 +411,20 @@ df11_status launch(const DecodeParams &prm, int dev, int variant, cudaStream_t s
             return DF11_ERR_CUDA;
         g_sm_count[dev].store(sms, std::memory_order_relaxed);
     }
-    int occ = g_occupancy[dev][variant][prm.n_tables].load(std::memory_order_relaxed);
+    int occ = g_occupancy[dev][v][prm.n_tables].load(std::memory_order_relaxed);
     if (occ == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, df11_decode_kernel<T>, T, smem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kWarpsPerCta * 32, smem) !=
             cudaSuccess)
             return DF11_ERR_CUDA;
         if (occ < 1)
             return DF11_ERR_CUDA;
-        g_occupancy[dev][variant][prm.n_tables].store(occ, std::memory_order_relaxed);
+        g_occupancy[dev][v][prm.n_tables].store(occ, std::memory_order_relaxed);
     }
+    const uint64_t warps_needed = prm.n_chunks;
+    const uint64_t ctas_needed = (warps_needed + kWarpsPerCta - 1) / kWarpsPerCta;
     const uint64_t resident = (uint64_t)occ * (uint64_t)sms;
-    const unsigned grid = (unsigned)(prm.n_chunks < resident ? prm.n_chunks : resident);
-    df11_decode_kernel<T><<<grid, T, smem, stream>>>(prm);
+    const unsigned grid = (unsigned)(ctas_needed < resident ? ctas_needed : resident);
+    kernel<<<grid, kWarpsPerCta * 32, smem, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
@@ -280,24 +439,26 @@ extern "C" df11_status df11_decompress_async(const df11_device_block *blk, uint1
     if (!blk || !out_bf16)
         return DF11_ERR_INVALID_ARGUMENT;
     const df11_header &h = blk->hdr;
-    const uint32_t T = h.threads_per_chunk;
-    if ((T != 128 && T != 256 && T != 512) || h.bytes_per_thread != DF11_BYTES_PER_THREAD)
+    const uint32_t W = h.bytes_per_thread;
+    if (h.threads_per_chunk != DF11_THREADS_PER_CHUNK || (W != 8 && W != 16))
         return DF11_ERR_INVALID_ARGUMENT;
     if (h.n_elements == 0 || h.n_elements >= (1ull << 32) || h.n_tables < 1 || h.n_tables > 256 ||
         h.total_bits == 0 || out_capacity < h.n_elements)
         return DF11_ERR_INVALID_ARGUMENT;
-    const uint64_t chunk_bits = (uint64_t)T * kSliceBits;
+    const uint64_t chunk_bits = (uint64_t)DF11_THREADS_PER_CHUNK * 8 * W;
     if (h.n_chunks != (h.total_bits + chunk_bits - 1) / chunk_bits)
         return DF11_ERR_INVALID_ARGUMENT;
-    const uint64_t n_threads = h.n_chunks * T;
+    const uint64_t n_threads = h.n_chunks * DF11_THREADS_PER_CHUNK;
     if (!blk->exp_stream || !blk->gaps || !blk->chunk_pos || !blk->signmant || !blk->lut)
         return DF11_ERR_INVALID_ARGUMENT;
-    if (blk->exp_stream_bytes < n_threads * 8 + DF11_STREAM_PAD || blk->gaps_bytes < n_threads / 2 ||
-        blk->chunk_pos_count < h.n_chunks + 1 || blk->signmant_bytes < h.n_elements ||
+    if (blk->exp_stream_bytes < n_threads * W + DF11_STREAM_PAD || blk->gaps_bytes < n_threads / 2 ||
+        blk->chunk_pos_count < h.n_chunks + 1 ||
+        blk->signmant_bytes < (h.n_elements + 15) / 16 * 16 ||
         blk->lut_entries < (uint64_t)h.n_tables * 256)
         return DF11_ERR_INVALID_ARGUMENT;
     if (!aligned(blk->exp_stream, 16) || !aligned(blk->chunk_pos, 16) || !aligned(blk->lut, 16) ||
-        !aligned(blk->signmant, 8) || !aligned(out_bf16, 16) || !aligned(d_error, 4))
+        !aligned(blk->signmant, 16) || !aligned(blk->gaps, 16) || !aligned(out_bf16, 16) ||
+        !aligned(d_error, 4))
         return DF11_ERR_INVALID_ARGUMENT;
 
     int dev = 0;
@@ -317,9 +478,5 @@ extern "C" df11_status df11_decompress_async(const df11_device_block *blk, uint1
     prm.out_limit = h.n_elements < out_capacity ? h.n_elements : out_capacity;
     prm.n_tables = h.n_tables;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    switch (T) {
-    case 128: return launch<128>(prm, dev, 0, s);
-    case 256: return launch<256>(prm, dev, 1, s);
-    default: return launch<512>(prm, dev, 2, s);
-    }
+    return W == 8 ? launch<8>(prm, dev, s) : launch<16>(prm, dev, s);
 }

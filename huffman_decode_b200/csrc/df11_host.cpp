@@ -18,7 +18,6 @@
 
 namespace {
 
-constexpr uint32_t kSliceBits = 64;  // 8 bytes of stream per decoding thread
 
 // ------------------------------------------------------------ threading
 
@@ -263,8 +262,8 @@ bool layout_ok(const df11_layout *ly)
 {
     if (!ly)
         return false;
-    uint32_t t = ly->threads_per_chunk;
-    return (t == 128 || t == 256 || t == 512) && ly->bytes_per_thread == DF11_BYTES_PER_THREAD;
+    return ly->threads_per_chunk == DF11_THREADS_PER_CHUNK &&
+           (ly->bytes_per_thread == 8 || ly->bytes_per_thread == 16);
 }
 
 df11_sizes sizes_for(uint64_t total_bits, uint64_t n_elements, uint32_t n_tables,
@@ -372,6 +371,7 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
     const uint8_t *len = cb->code_len;
     const uint32_t *code = cb->code;
     const uint32_t T = layout->threads_per_chunk;
+    const uint64_t kSliceBits = 8ull * layout->bytes_per_thread;
     const uint64_t N = v.total;
     const uint64_t total_bits = cb->total_bits;
 
@@ -504,6 +504,7 @@ df11_status df11_validate(const df11_host_block *b)
         b->signmant_bytes < h.n_elements || b->lut_entries < z.lut_entries)
         return DF11_ERR_CORRUPT;
     // output positions: 0 .. n_elements, monotone, at most one code per bit
+    const uint64_t kSliceBits = 8ull * h.bytes_per_thread;
     const uint64_t chunk_bits = (uint64_t)h.threads_per_chunk * kSliceBits;
     if (b->chunk_pos[0] != 0 || b->chunk_pos[h.n_chunks] != h.n_elements)
         return DF11_ERR_CORRUPT;

@@ -5,7 +5,7 @@ the decode in the sm_100a kernel.  torch is used for device memory and
 streams; numpy for host buffers.  Names follow the C calls:
 
     cb  = build_codebook(mats, max_code_len=16)
-    hb  = compress(cb, mats, threads_per_chunk=256)
+    hb  = compress(cb, mats, bytes_per_thread=8)
     validate(hb)
     db  = hb.to_device("cuda")
     decompress_async(db, out, error=None, stream=None)
@@ -32,7 +32,9 @@ DEVERR_BAD_CODE = 0x2
 DEVERR_BAD_POS = 0x4
 MAX_CODE_LEN = 16
 STREAM_PAD = 16
+THREADS_PER_CHUNK = 32
 BYTES_PER_THREAD = 8
+LAYOUTS = ((32, 8), (32, 16))   # (threads_per_chunk, bytes_per_thread) this build decodes
 
 EXPORTED_SYMBOLS = (
     "df11_build_codebook", "df11_compress_sizes", "df11_compress", "df11_validate",
@@ -169,7 +171,7 @@ def build_codebook(mats, max_code_len: int = MAX_CODE_LEN) -> Codebook:
     return cb
 
 
-def compress_sizes(cb: Codebook, threads_per_chunk: int = 256,
+def compress_sizes(cb: Codebook, threads_per_chunk: int = THREADS_PER_CHUNK,
                    bytes_per_thread: int = BYTES_PER_THREAD) -> Sizes:
     z = Sizes()
     ly = Layout(threads_per_chunk, bytes_per_thread)
@@ -227,7 +229,7 @@ class HostBlock:
                            matrix_numel=list(self.matrix_numel))
 
 
-def compress(cb: Codebook, mats, threads_per_chunk: int = 256,
+def compress(cb: Codebook, mats, threads_per_chunk: int = THREADS_PER_CHUNK,
              bytes_per_thread: int = BYTES_PER_THREAD) -> HostBlock:
     """df11_compress into freshly allocated numpy buffers of the exact sizes."""
     arrs, ptrs, numel = _mats_args(mats)

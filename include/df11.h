@@ -23,17 +23,20 @@
  *   exp_stream     codes of all elements, in element order, MSB-first: stream
  *                  bit i is bit 7 - i%8 of byte i/8.  Zero padded to
  *                  n_threads * bytes_per_thread + DF11_STREAM_PAD bytes.
- *   thread slice   thread g owns stream bits [64g, 64g+64) (bytes_per_thread
- *                  is 8) and decodes every code that STARTS in that slice and
- *                  before total_bits; a code may run up to 15 bits past it.
+ *   thread slice   with B = 8 * bytes_per_thread, thread g owns stream bits
+ *                  [B*g, B*g + B) and decodes every code that STARTS in that
+ *                  slice and before total_bits; a code may run up to 15 bits
+ *                  past it.
  *   gaps           4-bit offset, per thread, of the first code start in its
  *                  slice (the end of the stream counts as a start; slices at
  *                  or past the end hold 0).  Two per byte, thread 2j in the
  *                  low nibble of byte j.
- *   chunk_pos      uint32[n_chunks+1]: chunk c (threads_per_chunk threads)
- *                  writes elements [chunk_pos[c], chunk_pos[c+1]); the last
- *                  entry is n_elements.  (The pages keep one such 32-bit
- *                  position per thread block: "BlockOutputPos".)
+ *   chunk_pos      uint32[n_chunks+1]: chunk c (threads_per_chunk = 32
+ *                  threads, one warp) writes elements [chunk_pos[c],
+ *                  chunk_pos[c+1]); the last entry is n_elements.  (The pages
+ *                  keep one such 32-bit position per thread block,
+ *                  "BlockOutputPos"; here it is one per warp, so warps never
+ *                  wait for each other.)
  *   signmant       uint8[n_elements] (padded to a multiple of 16): byte k is
  *                  (sign << 7) | mantissa of element k.
  *   lut            n_tables * 256 uint16 entries; table 0 is indexed by the
@@ -79,7 +82,7 @@ typedef enum {
 #define DF11_MAX_CODE_LEN 16u     /* longest code the format allows           */
 #define DF11_MIN_CODE_LEN_CAP 8u  /* smallest cap accepted by build_codebook  */
 #define DF11_STREAM_PAD 16u       /* zero bytes after the last thread slice   */
-#define DF11_BYTES_PER_THREAD 8u  /* the only slice width this build decodes  */
+#define DF11_THREADS_PER_CHUNK 32u /* one warp per chunk                       */
 
 /* Codebook of one block.  Caller-allocated plain data (about 134 KB). */
 typedef struct {
@@ -95,9 +98,9 @@ typedef struct {
     uint16_t lut[256 * 256];   /* first n_tables * 256 entries used            */
 } df11_codebook;
 
-/* Compress-time layout: threads per chunk (decode CTA width) and bytes of
- * stream per thread.  This build decodes threads_per_chunk in {128, 256, 512}
- * and bytes_per_thread == 8. */
+/* Compress-time layout: threads per chunk and bytes of stream per thread.
+ * This build uses threads_per_chunk == 32 (one warp) and bytes_per_thread in
+ * {8, 16} (64- or 128-bit slices; the pages use 8). */
 typedef struct {
     uint32_t threads_per_chunk;
     uint32_t bytes_per_thread;

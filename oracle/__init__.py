@@ -230,7 +230,7 @@ class OracleBlock:
     signmant: np.ndarray     # uint8[n_elements]
 
 
-def compress_block(mats, cap: int = 16, threads_per_chunk: int = 256,
+def compress_block(mats, cap: int = 16, threads_per_chunk: int = 32,
                    bytes_per_thread: int = 8, pad_bytes: int = 16,
                    lengths: np.ndarray | None = None) -> OracleBlock:
     """Split, histogram over all matrices, code lengths under `cap` (or the

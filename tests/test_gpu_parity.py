@@ -40,10 +40,10 @@ def gpu_decode(hb, capacity=None, guard=0, stream=None):
     return out.cpu().numpy().view(np.uint16), int(err.item())
 
 
-def check_block(mats, threads_per_chunk=256, oracle_decode=True):
+def check_block(mats, bytes_per_thread=8, oracle_decode=True):
     w = _flat(mats)
     cb = df11.build_codebook(mats)
-    hb = df11.compress(cb, mats, threads_per_chunk)
+    hb = df11.compress(cb, mats, 32, bytes_per_thread)
     got, err = gpu_decode(hb, guard=8)
     assert err == 0
     assert np.all(got[w.size:] == 0x5A5A), "wrote past the block"
@@ -70,35 +70,52 @@ SMALL = {
 }
 
 
+BPT = [8, 16]
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
-@pytest.mark.parametrize("tpc", [128, 256, 512])
-def test_small_workloads(name, tpc):
-    check_block([m for _, m in SMALL[name]()], threads_per_chunk=tpc)
+@pytest.mark.parametrize("bpt", BPT)
+def test_small_workloads(name, bpt):
+    check_block([m for _, m in SMALL[name]()], bytes_per_thread=bpt)
 
 
-def test_all_bf16_patterns():
+@pytest.mark.parametrize("bpt", BPT)
+def test_all_bf16_patterns(bpt):
     allw = np.arange(65536, dtype=np.uint32).astype(np.uint16)
-    check_block([allw])
+    check_block([allw], bytes_per_thread=bpt)
     rng = np.random.default_rng(11)
-    check_block([allw, rng.permutation(allw), allw[::-1].copy()])
+    check_block([allw, rng.permutation(allw), allw[::-1].copy()], bytes_per_thread=bpt)
 
 
-@pytest.mark.parametrize("n", [1, 2, 3, 7, 8, 9, 15, 16, 17, 31, 33, 255, 257])
-def test_tiny_sizes(n):
+@pytest.mark.parametrize("n", [1, 2, 3, 7, 8, 9, 15, 16, 17, 31, 33, 255, 257, 4097])
+@pytest.mark.parametrize("bpt", BPT)
+def test_tiny_sizes(n, bpt):
     rng = np.random.default_rng(n)
     w = workloads.to_bf16((rng.standard_normal(n) * 0.02).astype(np.float32))
-    check_block([w])
+    check_block([w], bytes_per_thread=bpt)
 
 
 @pytest.mark.parametrize("delta", [-1, 0, 1])
-@pytest.mark.parametrize("tpc", [128, 256])
-def test_chunk_boundary(delta, tpc):
-    n = tpc * 64 + delta                 # 1-bit codes: total bits == elements
+@pytest.mark.parametrize("bpt", BPT)
+def test_chunk_boundary(delta, bpt):
+    n = 32 * 8 * bpt + delta            # 1-bit codes: total bits == elements
     rng = np.random.default_rng(77)
     e = np.where(rng.random(n) < 0.5, 0x7A, 0x7B).astype(np.uint16)
     w = (e << np.uint16(7)) | rng.integers(0, 256, n).astype(np.uint16) & np.uint16(0x807F)
-    cb, hb = check_block([w], threads_per_chunk=tpc)
+    cb, hb = check_block([w], bytes_per_thread=bpt)
     assert hb.header.n_chunks == (1 if delta <= 0 else 2)
+
+
+@pytest.mark.parametrize("bpt", BPT)
+def test_codes_crossing_slice_ends(bpt):
+    """Short codes packed so that many slices end inside a multi-code table
+    window: codes past a slice end belong to the next lane."""
+    rng = np.random.default_rng(123)
+    syms = np.array([0x70, 0x71, 0x72, 0x73, 0x74, 0x75, 0x76, 0x77], np.uint16)
+    p = np.array([0.4, 0.2, 0.15, 0.1, 0.07, 0.05, 0.02, 0.01])
+    e = rng.choice(syms, 300000, p=p)
+    w = (e << np.uint16(7)) | rng.integers(0, 256, e.size).astype(np.uint16) & np.uint16(0x807F)
+    check_block([w], bytes_per_thread=bpt)
 
 
 def test_many_matrices_keep_caller_order():
@@ -106,6 +123,7 @@ def test_many_matrices_keep_caller_order():
     mats = [workloads.to_bf16((rng.standard_normal(int(k)) * s).astype(np.float32))
             for k, s in zip(rng.integers(1, 5000, 40), rng.uniform(0.001, 0.1, 40))]
     check_block(mats)
+    check_block(mats, bytes_per_thread=16)
 
 
 def test_two_streams_concurrently():
@@ -198,11 +216,11 @@ def test_flipped_bit_detected_when_chunk_count_changes():
         gaps[0::2], gaps[1::2] = hb.gaps & 15, hb.gaps >> 4
         bit = int(rng.integers(0, hb.header.total_bits))
         hb.exp_stream[bit // 8] ^= np.uint8(0x80 >> (bit % 8))
-        chunk = bit // (256 * 64)
+        chunk = bit // (32 * 64)
         changed = False
         for c in {max(chunk - 1, 0), chunk}:
             want = int(hb.chunk_pos[c + 1] - hb.chunk_pos[c])
-            changed |= _thread_counts(hb.exp_stream, L, gaps, hb.header.total_bits, c, 256) != want
+            changed |= _thread_counts(hb.exp_stream, L, gaps, hb.header.total_bits, c, 32) != want
         _, err = gpu_decode(hb)
         assert bool(err & df11.DEVERR_COUNT) == changed
         flagged += changed
@@ -214,11 +232,12 @@ def test_flipped_bit_detected_when_chunk_count_changes():
 @pytest.mark.parametrize("name", ["single_1024x1024", "llama8b_block", "adversarial_heavy_tail",
                                   "adversarial_single_exponent", "adversarial_uniform_bits",
                                   "flux_dit_block"])
-def test_full_size_workload(name):
-    """The configurations at full size, in the launch configuration the
-    benchmark times (256 threads per chunk), every element compared."""
+@pytest.mark.parametrize("bpt", BPT)
+def test_full_size_workload(name, bpt):
+    """The configurations at full size, in both layouts (the benchmark times
+    the default one), every element compared with the oracle."""
     mats = [m for _, m in workloads.WORKLOADS[name]()]
-    check_block(mats, threads_per_chunk=256)
+    check_block(mats, bytes_per_thread=bpt)
 
 
 def test_model_stream_blocks_into_one_reused_buffer():

@@ -41,11 +41,12 @@ def _flat(mats):
     return np.concatenate([np.ascontiguousarray(m, dtype=np.uint16).reshape(-1) for m in mats])
 
 
-def check_format_parity(mats, threads_per_chunk=256, cap=16):
+def check_format_parity(mats, bytes_per_thread=8, cap=16):
     """Library artifact == the oracle's artifact built from the library's
     code lengths; the library's lengths reach the oracle's optimal cost."""
+    threads_per_chunk = 32
     cb = df11.build_codebook(mats, cap)
-    hb = df11.compress(cb, mats, threads_per_chunk)
+    hb = df11.compress(cb, mats, threads_per_chunk, bytes_per_thread)
     assert df11.validate(hb) == 0
     w = _flat(mats)
     e, s = oracle.split(w)
@@ -55,7 +56,8 @@ def check_format_parity(mats, threads_per_chunk=256, cap=16):
     best = oracle.code_lengths(counts, cap)
     assert oracle.total_bits(counts, L) == oracle.total_bits(counts, best)
     assert int(L.max()) <= cap
-    ob = oracle.compress_block(mats, cap=cap, threads_per_chunk=threads_per_chunk, lengths=L)
+    ob = oracle.compress_block(mats, cap=cap, threads_per_chunk=threads_per_chunk,
+                               bytes_per_thread=bytes_per_thread, lengths=L)
     assert np.array_equal(cb.codes(), ob.codes)
     h = hb.header
     assert (h.total_bits, h.n_elements, h.n_chunks) == (ob.total_bits, w.size, ob.n_chunks)
@@ -99,15 +101,10 @@ SMALL_WORKLOADS = {
 
 
 @pytest.mark.parametrize("name", sorted(SMALL_WORKLOADS))
-def test_format_parity_small_workloads(name):
+@pytest.mark.parametrize("bpt", [8, 16])
+def test_format_parity_small_workloads(name, bpt):
     mats = [m for _, m in SMALL_WORKLOADS[name]()]
-    check_format_parity(mats)
-
-
-@pytest.mark.parametrize("tpc", [128, 256, 512])
-def test_format_parity_layouts(tpc):
-    mats = [m for _, m in workloads.llama_block(1001, scale_div=128)]
-    check_format_parity(mats, threads_per_chunk=tpc)
+    check_format_parity(mats, bytes_per_thread=bpt)
 
 
 @pytest.mark.parametrize("cap", [8, 9, 12, 15, 16])
@@ -139,21 +136,23 @@ def test_all_bf16_patterns_and_tiny_sizes():
     allw = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     check_format_parity([allw])
     for n in (1, 2, 7, 8, 9, 15, 16, 17):
-        check_format_parity([allw[12345: 12345 + n]])
+        for bpt in (8, 16):
+            check_format_parity([allw[12345: 12345 + n]], bytes_per_thread=bpt)
     # several matrices, including a one-element one, in caller order
     check_format_parity([allw[:5], allw[40000:40001], allw[100:1100]])
 
 
 @pytest.mark.parametrize("delta", [-1, 0, 1])
-def test_chunk_boundary(delta):
-    """Stream lengths one bit under, at and over a whole chunk (256 x 64 bits)."""
-    chunk_bits = 256 * 64
+@pytest.mark.parametrize("bpt", [8, 16])
+def test_chunk_boundary(delta, bpt):
+    """Stream lengths one bit under, at and over a whole chunk (32 slices)."""
+    chunk_bits = 32 * 8 * bpt
     # two symbols of 1 bit each: total bits == element count
     n = chunk_bits + delta
     rng = np.random.default_rng(7)
     e = np.where(rng.random(n) < 0.5, 0x7A, 0x7B).astype(np.uint16)
     w = (e << np.uint16(7)) | rng.integers(0, 128, n).astype(np.uint16)
-    cb, hb, ob = check_format_parity([w])
+    cb, hb, ob = check_format_parity([w], bytes_per_thread=bpt)
     assert hb.header.total_bits == n
     assert hb.header.n_chunks == (1 if delta <= 0 else 2)
 
@@ -189,18 +188,19 @@ def test_compress_errors():
     with pytest.raises(df11.DF11Error) as ei:               # different data
         df11.compress(cb, [w[::-1].copy() ^ np.uint16(0x0080)])
     assert ei.value.status == 1
-    for tpc in (0, 64, 300, 1024):
+    for tpc in (0, 16, 64, 128, 256, 300):
         with pytest.raises(df11.DF11Error):
             df11.compress(cb, [w], threads_per_chunk=tpc)
-    with pytest.raises(df11.DF11Error):
-        df11.compress(cb, [w], bytes_per_thread=4)
+    for bpt in (0, 4, 12, 32):
+        with pytest.raises(df11.DF11Error):
+            df11.compress(cb, [w], bytes_per_thread=bpt)
     # a buffer one entry short
     hb = df11.compress(cb, [w])
     blk = hb.c_struct()
     blk.chunk_pos_count -= 1
     lib = df11.load_library()
     arrs, ptrs, numel = binding._mats_args([w])
-    ly = binding.Layout(256, 8)
+    ly = binding.Layout(32, 8)
     assert lib.df11_compress(ctypes.byref(cb), ctypes.byref(ly), ptrs, numel, 1,
                              ctypes.byref(blk)) == 2
 
@@ -267,10 +267,15 @@ def test_decompress_rejects_bad_arguments_before_any_cuda_call():
     assert call(dev_block(chunk_pos_count=hb.chunk_pos.size - 1)) == 1
     assert call(dev_block(lut_entries=hb.lut.size - 1)) == 1
     assert call(dev_block(exp_stream=fake + 4)) == 1               # misaligned
+    assert call(dev_block(gaps=fake + 8)) == 1
+    assert call(dev_block(signmant=fake + 8)) == 1
     assert call(dev_block(), out=fake + 2) == 1
     assert call(dev_block(), err=fake + 1) == 1
     h = binding.Header.from_buffer_copy(hb.header)
     h.threads_per_chunk = 64
+    assert call(dev_block(hdr=h)) == 1
+    h = binding.Header.from_buffer_copy(hb.header)
+    h.bytes_per_thread = 4
     assert call(dev_block(hdr=h)) == 1
     h = binding.Header.from_buffer_copy(hb.header)
     h.n_chunks += 1
