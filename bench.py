@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--bytes-per-thread", type=int, default=8, choices=[8, 16],
                     help="stream bytes each decoding thread owns (format layout)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.WORKLOADS),
+                    help="block to decode (the headline number is llama8b_block)")
     ap.add_argument("--scale-div", type=int, default=1,
                     help="divide every row count of the block (smaller case for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=20,
@@ -90,8 +92,12 @@ def profiled_traffic(n_weights: int):
     return float(d["dram_bytes_per_weight"]) * n_weights
 
 
-def make_block(seed: int, scale_div: int = 1):
-    return [m for _, m in workloads.llama_block(seed, scale_div=scale_div)]
+def make_block(seed: int, scale_div: int = 1, workload: str = WORKLOAD):
+    if workload == "llama8b_block":
+        return [m for _, m in workloads.llama_block(seed, scale_div=scale_div)]
+    if workload == "flux_dit_block":
+        return [m for _, m in workloads.flux_block(5000 + (seed - 1000), scale_div=scale_div)]
+    return [m for _, m in workloads.WORKLOADS[workload]()]
 
 
 # ----------------------------------------------------------- clocks
@@ -247,7 +253,7 @@ def run_b200(args):
                                 device_id=dev)
 
     seed = 1000 + rank
-    mats = make_block(seed, args.scale_div)
+    mats = make_block(seed, args.scale_div, args.workload)
     t0 = time.perf_counter()
     cb = df11.build_codebook(mats)
     hb = df11.compress(cb, mats, 32, args.bytes_per_thread)
@@ -362,7 +368,7 @@ def run_b200(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "u8", "data": "synthetic",
-        "config": {"workload": WORKLOAD if args.scale_div == 1 else f"{WORKLOAD}/rows{args.scale_div}",
+        "config": {"workload": args.workload if args.scale_div == 1 else f"{args.workload}/rows{args.scale_div}",
                    "n_weights": n, "n_matrices": len(mats),
                    "seed": seed, "threads_per_chunk": 32, "bytes_per_thread": args.bytes_per_thread,
                    "bits_per_weight": round(8 + cb.total_bits / n, 4),

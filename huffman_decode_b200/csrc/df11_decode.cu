@@ -40,7 +40,6 @@ constexpr uint32_t kLutNoCode = 0x4000u | (1u << 8);
 constexpr int kWindowBits = 10;                    // multi-code table index width
 constexpr int kMultiEntries = 1 << kWindowBits;
 constexpr int kMaxCodesPerEntry = 3;
-constexpr int kPrefetchGroups = 4;                 // 8-byte sign|mantissa groups per lane
 
 struct DecodeParams {
     const uint8_t *stream;
@@ -66,6 +65,7 @@ struct Geometry {
     static constexpr int kSlotBytes = kSlotRows * 32 * 4; // per warp
     static constexpr int kEbufBytes = 32 * kMaxCodes + 16; // per warp, multiple of 16
     static constexpr int kWords = W / 4 + 1;              // stream words per lane incl. halo
+    static constexpr int kPrefetch = W / 2;               // 8-byte sign|mantissa groups per lane
 };
 
 template <int W, int WARPS>
@@ -190,14 +190,16 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
                             pos1 - pos0 <= (uint32_t)(32 * G::kMaxCodes);
         const uint32_t head = pos0 & 7u;
         const uint64_t base = (uint64_t)pos0 - head;           // 8-element aligned
-        const uint32_t groups = pos_ok ? (head + (pos1 - pos0) + 7) >> 3 : 0u;
+        // whole 8-element groups of the chunk: local [gfirst*8, gend*8)
+        const uint32_t gfirst = head ? 1u : 0u;
+        const uint32_t gend = pos_ok ? (head + (pos1 - pos0)) >> 3 : 0u;
 
         // ---- loads for later: sign|mantissa of this chunk, next slice -------
-        uint2 pre[kPrefetchGroups];
+        uint2 pre[G::kPrefetch];
 #pragma unroll
-        for (int j = 0; j < kPrefetchGroups; ++j) {
-            const uint32_t i = lane + 32 * j;
-            if (i < groups)
+        for (int j = 0; j < G::kPrefetch; ++j) {
+            const uint32_t i = gfirst + lane + 32 * j;
+            if (i < gend)
                 pre[j] = __ldg(reinterpret_cast<const uint2 *>(p.signmant + base + 8ull * i));
             else
                 pre[j] = make_uint2(0u, 0u);
@@ -234,7 +236,6 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
                 accl |= (uint32_t)s;
                 acch |= (uint32_t)(s >> 32);
                 nb += n;
-                count += n;
                 if (nb >= 4) {
                     slots[row * 32 + lane] = accl;
                     ++row;
@@ -266,14 +267,21 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
                     append(r);
                 }
             }
+            // the last code starts: in a full slice they lie in the last word
+            // pair; only the stream's final slice can end earlier
+            const bool full_slice = end == G::kSliceBits;
             while (bitpos < end) {
-                const int h = bitpos >> 5;
-                uint32_t hi = w[0], lo = w[1];
+                uint32_t hi = w[G::kWords - 2], lo = w[G::kWords - 1];
+                if (!full_slice) {
+                    const int h = bitpos >> 5;
+                    hi = w[0];
+                    lo = w[1];
 #pragma unroll
-                for (int k = 1; k < G::kWords - 1; ++k) {
-                    if (h == k) {
-                        hi = w[k];
-                        lo = w[k + 1];
+                    for (int k = 1; k < G::kWords - 1; ++k) {
+                        if (h == k) {
+                            hi = w[k];
+                            lo = w[k + 1];
+                        }
                     }
                 }
                 const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
@@ -286,6 +294,7 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
             }
             if (nb)
                 slots[row * 32 + lane] = accl;
+            count = row * 4 + nb;
             if (seen & 0x4000u)
                 err |= DF11_DEVERR_BAD_CODE;
 
@@ -304,69 +313,89 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
             const uint32_t n_write = min(total, pos1 - pos0);
 
             // ---- compaction into the exponent buffer ------------------------
-            for (int i = lane; i < G::kEbufBytes / 16; i += 32)
-                reinterpret_cast<uint4 *>(ebuf)[i] = make_uint4(0u, 0u, 0u, 0u);
-            __syncwarp();
+            // Lane bytes go to ebuf[head + off, head + off + nbytes).  Words the
+            // lane covers entirely are plain stores; the first and last word
+            // may be shared with neighbouring lanes: zeroed, then ORed.
             const uint32_t nbytes = off < n_write ? min(count, n_write - off) : 0u;
+            const uint32_t a = head + off;
+            const uint32_t sh = (a & 3u) * 8;
+            const uint32_t first = a >> 2;
+            const uint32_t last = (a + nbytes - 1) >> 2;
+            const bool head_shared = sh != 0;
+            const bool tail_shared = ((a + nbytes) & 3u) != 0;
+            const uint32_t nwords = (nbytes + 3) >> 2;
             if (nbytes) {
-                const uint32_t a = head + off;                 // byte address in ebuf
-                const uint32_t sh = (a & 3u) * 8;
-                const uint32_t first = a >> 2;
-                const uint32_t last = (a + nbytes - 1) >> 2;
-                const bool end_partial = ((a + nbytes) & 3u) != 0;
-                const uint32_t nwords = (nbytes + 3) >> 2;
-                const uint32_t tail_mask = (nbytes & 3u) ? (1u << (8 * (nbytes & 3u))) - 1 : ~0u;
-                uint32_t prev = 0;
-                for (uint32_t j = 0; j <= last - first; ++j) {
-                    uint32_t cur = 0;
-                    if (j < nwords) {
-                        cur = slots[j * 32 + lane];
-                        if (j == nwords - 1)
-                            cur &= tail_mask;
-                    }
-                    const uint32_t v = __funnelshift_l(prev, cur, sh);
+                if (head_shared)
+                    ebuf32[first] = 0u;
+                if (tail_shared)
+                    ebuf32[last] = 0u;
+                if (nbytes != count && (nbytes & 3u))   // clamped: clear bytes past nbytes
+                    slots[(nwords - 1) * 32 + lane] &= (1u << (8 * (nbytes & 3u))) - 1;
+            }
+            __syncwarp();
+            if (nbytes) {
+                uint32_t prev = slots[lane];
+                uint32_t v = prev << sh;
+                if (head_shared || (first == last && tail_shared))
+                    atomicOr(ebuf32 + first, v);
+                else
+                    ebuf32[first] = v;
+                uint32_t j = 1;
+                for (; first + j < last; ++j) {
+                    const uint32_t cur = slots[j * 32 + lane];
+                    ebuf32[first + j] = __funnelshift_l(prev, cur, sh);
                     prev = cur;
-                    const bool shared = (j == 0 && sh != 0) || (first + j == last && end_partial);
-                    if (shared)
-                        atomicOr(ebuf32 + first + j, v);
+                }
+                if (first + j == last) {
+                    const uint32_t cur = j < nwords ? slots[j * 32 + lane] : 0u;
+                    v = __funnelshift_l(prev, cur, sh);
+                    if (tail_shared)
+                        atomicOr(ebuf32 + last, v);
                     else
-                        ebuf32[first + j] = v;
+                        ebuf32[last] = v;
                 }
             }
             __syncwarp();
 
             // ---- merge with sign|mantissa and store -------------------------
+            // Whole groups: 8 exponents + 8 sign|mantissa bytes -> one 16-byte
+            // store per lane.  The partial groups at both ends (<= 7 elements
+            // each) take one element per lane on lanes 0..15.
             const uint32_t span = head + n_write;
-            const uint32_t mgroups = (span + 7) >> 3;
+            const uint32_t mend = span >> 3;                   // whole groups end
             auto merge_group = [&](uint32_t i, uint2 s8) {
                 const uint32_t l0 = 8 * i;
-                const uint64_t g0 = base + l0;
-                if (l0 >= head && l0 + 8 <= span) {
-                    const uint2 e8 = *reinterpret_cast<const uint2 *>(ebuf + l0);
-                    uint4 o;
-                    o.x = join2(__byte_perm(s8.x, e8.x, 0x5140));
-                    o.y = join2(__byte_perm(s8.x, e8.x, 0x7362));
-                    o.z = join2(__byte_perm(s8.y, e8.y, 0x5140));
-                    o.w = join2(__byte_perm(s8.y, e8.y, 0x7362));
-                    *reinterpret_cast<uint4 *>(p.out + g0) = o;
-                } else {
-                    for (uint32_t k = 0; k < 8; ++k) {
-                        const uint32_t l = l0 + k;
-                        if (l >= head && l < span) {
-                            const uint32_t sb = ((k < 4 ? s8.x : s8.y) >> (8 * (k & 3))) & 0xFFu;
-                            p.out[base + l] = join1(ebuf[l], sb);
-                        }
-                    }
-                }
+                const uint2 e8 = *reinterpret_cast<const uint2 *>(ebuf + l0);
+                uint4 o;
+                o.x = join2(__byte_perm(s8.x, e8.x, 0x5140));
+                o.y = join2(__byte_perm(s8.x, e8.x, 0x7362));
+                o.z = join2(__byte_perm(s8.y, e8.y, 0x5140));
+                o.w = join2(__byte_perm(s8.y, e8.y, 0x7362));
+                *reinterpret_cast<uint4 *>(p.out + base + l0) = o;
             };
 #pragma unroll
-            for (int j = 0; j < kPrefetchGroups; ++j) {
-                const uint32_t i = lane + 32 * j;
-                if (i < mgroups)
+            for (int j = 0; j < G::kPrefetch; ++j) {
+                const uint32_t i = gfirst + lane + 32 * j;
+                if (i < mend)
                     merge_group(i, pre[j]);
             }
-            for (uint32_t i = lane + 32 * kPrefetchGroups; i < mgroups; i += 32)
+            for (uint32_t i = gfirst + lane + 32 * G::kPrefetch; i < mend; i += 32)
                 merge_group(i, __ldg(reinterpret_cast<const uint2 *>(p.signmant + base + 8ull * i)));
+            {
+                const uint32_t fs = gfirst * 8;                    // first whole-group element
+                const uint32_t hend = min(fs, span);               // head part: [head, hend)
+                const uint32_t tbeg = max(mend * 8, fs);           // tail part: [tbeg, span)
+                uint32_t l = 0xFFFFFFFFu;
+                if (lane < 8) {
+                    if (head + lane < hend)
+                        l = head + lane;
+                } else if (lane < 16) {
+                    if (tbeg + (lane - 8) < span)
+                        l = tbeg + (lane - 8);
+                }
+                if (l != 0xFFFFFFFFu)
+                    p.out[base + l] = join1(ebuf[l], p.signmant[base + l]);
+            }
             __syncwarp();
         }
 
