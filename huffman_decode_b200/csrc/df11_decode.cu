@@ -61,7 +61,7 @@ template <int W>
 struct Geometry {
     static constexpr int kSliceBits = 8 * W;              // 64 or 128
     static constexpr int kMaxCodes = kSliceBits;          // 1-bit codes at most
-    static constexpr int kSlotRows = kMaxCodes / 4;
+    static constexpr int kSlotRows = kMaxCodes / 4 + 1;   // + codes past the slice end
     static constexpr int kSlotBytes = kSlotRows * 32 * 4; // per warp
     static constexpr int kEbufBytes = 32 * kMaxCodes + 16; // per warp, multiple of 16
     static constexpr int kWords = W / 4 + 1;              // stream words per lane incl. halo
@@ -72,7 +72,7 @@ template <int W, int WARPS>
 constexpr size_t smem_bytes_for(uint32_t n_tables)
 {
     using G = Geometry<W>;
-    return (size_t)kMultiEntries * 4 + (size_t)WARPS * (G::kSlotBytes + G::kEbufBytes) +
+    return (size_t)kMultiEntries * 4 + 256 + (size_t)WARPS * (G::kSlotBytes + G::kEbufBytes) +
            (size_t)n_tables * 512;
 }
 
@@ -118,7 +118,8 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
     using G = Geometry<W>;
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t *multi = reinterpret_cast<uint32_t *>(smem);
-    uint8_t *warp_area = smem + kMultiEntries * 4;
+    uint8_t *len_of = smem + kMultiEntries * 4;                 // code length by exponent
+    uint8_t *warp_area = len_of + 256;
     uint16_t *lut = reinterpret_cast<uint16_t *>(warp_area + WARPS * (G::kSlotBytes + G::kEbufBytes));
 
     const int tid = threadIdx.x;
@@ -139,6 +140,8 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
             const uint32_t l = (e >> 8) & 0x1Fu;
             if ((e & 0x4000u) || l == 0 || l > 16)
                 e = kLutNoCode;
+            else
+                len_of[e & 0xFFu] = (uint8_t)l;   // every leaf of a symbol holds its length
         }
         lut[i] = (uint16_t)e;
     }
@@ -179,31 +182,39 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
         return;
 
     uint32_t err = 0;
+    // Per chunk: positions valid?  Whole 8-element groups [gfirst, gend) of
+    // the chunk's output (relative to the 8-aligned base) get their
+    // sign|mantissa bytes loaded ahead into registers.
+    auto positions_ok = [&](uint32_t a, uint32_t b) {
+        return a <= b && (uint64_t)b <= p.out_limit && b - a <= (uint32_t)(32 * G::kMaxCodes);
+    };
+    auto prefetch = [&](uint32_t a, uint32_t b, bool ok, uint2 (&dst)[G::kPrefetch]) {
+        const uint32_t hd = a & 7u;
+        const uint64_t bs = (uint64_t)a - hd;
+        const uint32_t g0 = hd ? 1u : 0u;
+        const uint32_t g1 = ok ? (hd + (b - a)) >> 3 : 0u;
+#pragma unroll
+        for (int j = 0; j < G::kPrefetch; ++j) {
+            const uint32_t i = g0 + lane + 32 * j;
+            dst[j] = i < g1 ? __ldg(reinterpret_cast<const uint2 *>(p.signmant + bs + 8ull * i))
+                            : make_uint2(0u, 0u);
+        }
+    };
+
     uint32_t w[G::kWords];
     uint32_t gap;
     load_slice<W>(p, chunk * 32 + lane, w, gap);
     uint32_t pos0 = p.chunk_pos[chunk], pos1 = p.chunk_pos[chunk + 1];
+    bool pos_ok = positions_ok(pos0, pos1);
+    uint2 pre[G::kPrefetch];
+    prefetch(pos0, pos1, pos_ok, pre);
 
     for (;;) {
-        // ---- positions of this chunk (warp-uniform) ------------------------
-        const bool pos_ok = pos0 <= pos1 && (uint64_t)pos1 <= p.out_limit &&
-                            pos1 - pos0 <= (uint32_t)(32 * G::kMaxCodes);
         const uint32_t head = pos0 & 7u;
         const uint64_t base = (uint64_t)pos0 - head;           // 8-element aligned
-        // whole 8-element groups of the chunk: local [gfirst*8, gend*8)
         const uint32_t gfirst = head ? 1u : 0u;
-        const uint32_t gend = pos_ok ? (head + (pos1 - pos0)) >> 3 : 0u;
 
-        // ---- loads for later: sign|mantissa of this chunk, next slice -------
-        uint2 pre[G::kPrefetch];
-#pragma unroll
-        for (int j = 0; j < G::kPrefetch; ++j) {
-            const uint32_t i = gfirst + lane + 32 * j;
-            if (i < gend)
-                pre[j] = __ldg(reinterpret_cast<const uint2 *>(p.signmant + base + 8ull * i));
-            else
-                pre[j] = make_uint2(0u, 0u);
-        }
+        // ---- the next chunk's slice and positions, loaded ahead -------------
         const uint64_t next = chunk + stride;
         const bool has_next = next < p.n_chunks;
         uint32_t nw[G::kWords];
@@ -214,89 +225,82 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
             npos1 = p.chunk_pos[next + 1];
         }
 
+        uint2 npre[G::kPrefetch];
+        bool npos_ok = false;
         if (!pos_ok) {
             err |= DF11_DEVERR_BAD_POS;
+            if (has_next) {
+                npos_ok = positions_ok(npos0, npos1);
+                prefetch(npos0, npos1, npos_ok, npre);
+            }
         } else {
             // ---- decode this lane's slice ----------------------------------
-            // Codes starting in [gap, end) belong to this lane.  While at
-            // least kWindowBits bits remain before `end`, every code a table
-            // entry returns starts inside the slice; the last few bits go
-            // through the checked tail loop.
+            // Codes starting in [gap, end) belong to this lane.  The loop
+            // runs while bitpos < end; the last table entry may also hold
+            // codes that start at or past `end` -- they are dropped below.
             const uint64_t bit0 = (chunk * 32 + lane) * (uint64_t)G::kSliceBits;
             const int end = bit0 >= p.total_bits
                                 ? 0
                                 : (int)min((uint64_t)G::kSliceBits, p.total_bits - bit0);
             int bitpos = (int)gap;
             uint32_t count = 0, nb = 0, row = 0, accl = 0, acch = 0, seen = 0;
-            // appends the codes of entry r (symbols in bytes 0..2, count in
-            // bits 24..25) to the lane's packed slot column
-            auto append = [&](uint32_t r) {
-                const uint32_t n = (r >> 24) & 3u;
-                const uint64_t s = (uint64_t)(r & 0xFFFFFFu) << (8 * nb);
-                accl |= (uint32_t)s;
-                acch |= (uint32_t)(s >> 32);
-                nb += n;
-                if (nb >= 4) {
-                    slots[row * 32 + lane] = accl;
-                    ++row;
-                    accl = acch;
-                    acch = 0;
-                    nb -= 4;
-                }
-            };
-            // one code through the two-level tables, as an entry with count 1
-            auto single = [&](uint32_t win, uint32_t &adv) -> uint32_t {
-                uint32_t e = lut[win >> 24];
-                if (e & kLutPointer)
-                    e = lut[((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)];
-                seen |= e;
-                adv = (e >> 8) & 0x1Fu;
-                return (e & 0xFFu) | (1u << 24);
-            };
+            uint32_t r = 0, adv = 0;                 // last entry and its length
 #pragma unroll
             for (int h = 0; h < G::kWords - 1; ++h) {
                 const uint32_t hi = w[h], lo = w[h + 1];
-                const int lim = min(end - kWindowBits, 32 * (h + 1));
+                const int lim = min(end, 32 * (h + 1));
                 while (bitpos < lim) {
                     const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
-                    uint32_t r = multi[win >> (32 - kWindowBits)];
-                    uint32_t adv = r >> 28;
-                    if (r < (1u << 28))
-                        r = single(win, adv);
+                    r = multi[win >> (32 - kWindowBits)];
+                    adv = r >> 28;
+                    if (r < (1u << 28)) {
+                        // first code longer than the window: two-level tables
+                        uint32_t e = lut[win >> 24];
+                        if (e & kLutPointer)
+                            e = lut[((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)];
+                        seen |= e;
+                        r = (e & 0xFFu) | (1u << 24);
+                        adv = (e >> 8) & 0x1Fu;
+                    }
                     bitpos += (int)adv;
-                    append(r);
-                }
-            }
-            // the last code starts: in a full slice they lie in the last word
-            // pair; only the stream's final slice can end earlier
-            const bool full_slice = end == G::kSliceBits;
-            while (bitpos < end) {
-                uint32_t hi = w[G::kWords - 2], lo = w[G::kWords - 1];
-                if (!full_slice) {
-                    const int h = bitpos >> 5;
-                    hi = w[0];
-                    lo = w[1];
-#pragma unroll
-                    for (int k = 1; k < G::kWords - 1; ++k) {
-                        if (h == k) {
-                            hi = w[k];
-                            lo = w[k + 1];
-                        }
+                    const uint32_t n = (r >> 24) & 3u;
+                    const uint64_t sv = (uint64_t)(r & 0xFFFFFFu) << (8 * nb);
+                    accl |= (uint32_t)sv;
+                    acch |= (uint32_t)(sv >> 32);
+                    nb += n;
+                    if (nb >= 4) {
+                        slots[row * 32 + lane] = accl;
+                        ++row;
+                        accl = acch;
+                        acch = 0;
+                        nb -= 4;
                     }
                 }
-                const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
-                uint32_t r = multi[win >> (32 - kWindowBits)];
-                uint32_t adv = r >> 28;
-                if (r < (1u << 28) || bitpos + (int)adv > end)
-                    r = single(win, adv);
-                bitpos += (int)adv;
-                append(r);
             }
             if (nb)
                 slots[row * 32 + lane] = accl;
             count = row * 4 + nb;
+            if (count) {
+                // codes of the last entry that start at or past `end`
+                const uint32_t n = (r >> 24) & 3u;
+                const int p_last = bitpos - (int)adv;
+                uint32_t keep = 1;
+                if (n >= 2) {
+                    const int c1 = p_last + len_of[r & 0xFFu];
+                    keep += c1 < end;
+                    if (n == 3)
+                        keep += c1 + len_of[(r >> 8) & 0xFFu] < end;
+                }
+                count -= n - keep;
+            }
             if (seen & 0x4000u)
                 err |= DF11_DEVERR_BAD_CODE;
+
+            // ---- sign|mantissa of the next chunk, loaded ahead -------------
+            if (has_next) {
+                npos_ok = positions_ok(npos0, npos1);
+                prefetch(npos0, npos1, npos_ok, npre);
+            }
 
             // ---- warp scan of the counts ------------------------------------
             uint32_t incl = count;
@@ -329,7 +333,7 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
                     ebuf32[first] = 0u;
                 if (tail_shared)
                     ebuf32[last] = 0u;
-                if (nbytes != count && (nbytes & 3u))   // clamped: clear bytes past nbytes
+                if (nbytes & 3u)                        // clear bytes past nbytes
                     slots[(nwords - 1) * 32 + lane] &= (1u << (8 * (nbytes & 3u))) - 1;
             }
             __syncwarp();
@@ -341,6 +345,7 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
                 else
                     ebuf32[first] = v;
                 uint32_t j = 1;
+#pragma unroll 4
                 for (; first + j < last; ++j) {
                     const uint32_t cur = slots[j * 32 + lane];
                     ebuf32[first + j] = __funnelshift_l(prev, cur, sh);
@@ -405,9 +410,13 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
 #pragma unroll
         for (int k = 0; k < G::kWords; ++k)
             w[k] = nw[k];
+#pragma unroll
+        for (int j = 0; j < G::kPrefetch; ++j)
+            pre[j] = npre[j];
         gap = ngap;
         pos0 = npos0;
         pos1 = npos1;
+        pos_ok = npos_ok;
     }
     if (err && p.err)
         atomicOr(p.err, err);
