@@ -78,11 +78,19 @@ constexpr size_t smem_bytes_for(uint32_t n_tables)
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
-// Two BF16 words from v = [s0 e0 s1 e1] (bytes, low first): per 16-bit half,
-// exponent -> bits 14..7, sign -> bit 15, mantissa -> bits 6..0.
-__device__ __forceinline__ uint32_t join2(uint32_t v)
+// Four BF16 values from four exponent bytes (e) and four sign|mantissa bytes
+// (s), element k in byte k.  BF16 = sign (bit 15) | exponent (14..7) |
+// mantissa (6..0), so its low byte is (exponent bit 0) << 7 | mantissa and
+// its high byte is sign << 7 | exponent >> 1.  Both are built for all four
+// elements with one shift and one bit-select each, then interleaved.
+__device__ __forceinline__ uint2 join4(uint32_t e, uint32_t s)
 {
-    return ((v >> 1) & 0x7F807F80u) | ((v & 0x00800080u) << 8) | (v & 0x007F007Fu);
+    uint32_t lo, hi;
+    // lo = (e << 7) where mask 0x80808080, else s
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(lo) : "r"(e << 7), "r"(s), "r"(0x80808080u));
+    // hi = s where mask 0x80808080, else (e >> 1)
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(hi) : "r"(s), "r"(e >> 1), "r"(0x80808080u));
+    return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
 __device__ __forceinline__ uint16_t join1(uint32_t e, uint32_t s)
@@ -368,15 +376,13 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
             // each) take one element per lane on lanes 0..15.
             const uint32_t span = head + n_write;
             const uint32_t mend = span >> 3;                   // whole groups end
+            uint4 *const out16 = reinterpret_cast<uint4 *>(p.out + base);   // group i -> out16[i]
+            const uint2 *const e64 = reinterpret_cast<const uint2 *>(ebuf);
             auto merge_group = [&](uint32_t i, uint2 s8) {
-                const uint32_t l0 = 8 * i;
-                const uint2 e8 = *reinterpret_cast<const uint2 *>(ebuf + l0);
-                uint4 o;
-                o.x = join2(__byte_perm(s8.x, e8.x, 0x5140));
-                o.y = join2(__byte_perm(s8.x, e8.x, 0x7362));
-                o.z = join2(__byte_perm(s8.y, e8.y, 0x5140));
-                o.w = join2(__byte_perm(s8.y, e8.y, 0x7362));
-                *reinterpret_cast<uint4 *>(p.out + base + l0) = o;
+                const uint2 e8 = e64[i];
+                const uint2 a = join4(e8.x, s8.x);
+                const uint2 b = join4(e8.y, s8.y);
+                out16[i] = make_uint4(a.x, a.y, b.x, b.y);
             };
 #pragma unroll
             for (int j = 0; j < G::kPrefetch; ++j) {
