@@ -23,6 +23,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -41,7 +42,7 @@ UNIT = "GB/s"
 WORKLOAD = "llama8b_block"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SRC = os.path.join(ROOT, "huffman_decode_b200", "csrc", "df11_decode.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_llama8b_block.md")
 
 
 def parse_args():
@@ -50,7 +51,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--bytes-per-thread", type=int, default=8, choices=[8, 16],
+    ap.add_argument("--bytes-per-thread", type=int, default=16, choices=[8, 16],
                     help="stream bytes each decoding thread owns (format layout)")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.WORKLOADS),
                     help="block to decode (the headline number is llama8b_block)")
@@ -80,16 +81,18 @@ def kernel_hash() -> str:
 
 
 def profiled_traffic(n_weights: int):
-    """DRAM bytes per launch from the committed ncu summary, scaled to this
-    launch's weights, or None when the kernel changed since it was taken."""
+    """DRAM bytes per launch from the committed ncu summary (its
+    `dram_bytes_per_weight` line), scaled to this launch's weights, or None
+    when the kernel source changed since the counters were taken."""
     try:
         with open(TRAFFIC_FILE) as f:
-            d = json.load(f)
-    except Exception:
+            text = f.read()
+    except OSError:
         return None
-    if d.get("kernel_sha256_16") != kernel_hash():
+    fields = dict(re.findall(r"^([a-z0-9_]+): ([0-9a-f.]+)$", text, re.M))
+    if fields.get("kernel_source_sha256_16") != kernel_hash() or "dram_bytes_per_weight" not in fields:
         return None
-    return float(d["dram_bytes_per_weight"]) * n_weights
+    return round(float(fields["dram_bytes_per_weight"]) * n_weights)
 
 
 def make_block(seed: int, scale_div: int = 1, workload: str = WORKLOAD):

@@ -5,7 +5,7 @@ the decode in the sm_100a kernel.  torch is used for device memory and
 streams; numpy for host buffers.  Names follow the C calls:
 
     cb  = build_codebook(mats, max_code_len=16)
-    hb  = compress(cb, mats, bytes_per_thread=8)
+    hb  = compress(cb, mats)               # 32 threads x 16 bytes per chunk
     validate(hb)
     db  = hb.to_device("cuda")
     decompress_async(db, out, error=None, stream=None)
@@ -33,7 +33,7 @@ DEVERR_BAD_POS = 0x4
 MAX_CODE_LEN = 16
 STREAM_PAD = 16
 THREADS_PER_CHUNK = 32
-BYTES_PER_THREAD = 8
+BYTES_PER_THREAD = 16           # 128-bit slices: fastest layout on B200
 LAYOUTS = ((32, 8), (32, 16))   # (threads_per_chunk, bytes_per_thread) this build decodes
 
 EXPORTED_SYMBOLS = (

@@ -188,21 +188,22 @@ def test_no_code_window_sets_bad_code_bit():
     assert np.all(got[hb.n_elements:] == 0x5A5A)
 
 
-def _thread_counts(stream, lengths, gap, total_bits, chunk, tpc):
+def _thread_counts(stream, lengths, gap, total_bits, chunk, tpc, slice_bits):
     """Codes each thread of `chunk` decodes, by the oracle's bit-by-bit decode
     under the kernel's contract (codes starting in the slice, from its gap)."""
     n = 0
     for t in range(tpc):
         g = chunk * tpc + t
-        p = 64 * g + int(gap[g])
-        end = min(64 * (g + 1), total_bits)
+        p = slice_bits * g + int(gap[g])
+        end = min(slice_bits * (g + 1), total_bits)
         while p < end:
             _, p = oracle.decode(stream, 1, lengths, start_bit=p)
             n += 1
     return n
 
 
-def test_flipped_bit_detected_when_chunk_count_changes():
+@pytest.mark.parametrize("bpt", BPT)
+def test_flipped_bit_detected_when_chunk_count_changes(bpt):
     """A flipped stream bit desyncs only the thread(s) that read it; the
     kernel reports it whenever that changes the chunk's code count."""
     mats = [m for _, m in workloads.single_matrix(0, shape=(64, 512))]
@@ -211,16 +212,17 @@ def test_flipped_bit_detected_when_chunk_count_changes():
     rng = np.random.default_rng(99)
     flagged = 0
     for trial in range(12):
-        hb = df11.compress(cb, mats)
+        hb = df11.compress(cb, mats, 32, bpt)
         gaps = np.empty(hb.gaps.size * 2, np.uint8)
         gaps[0::2], gaps[1::2] = hb.gaps & 15, hb.gaps >> 4
         bit = int(rng.integers(0, hb.header.total_bits))
         hb.exp_stream[bit // 8] ^= np.uint8(0x80 >> (bit % 8))
-        chunk = bit // (32 * 64)
+        chunk = bit // (32 * 8 * bpt)
         changed = False
         for c in {max(chunk - 1, 0), chunk}:
             want = int(hb.chunk_pos[c + 1] - hb.chunk_pos[c])
-            changed |= _thread_counts(hb.exp_stream, L, gaps, hb.header.total_bits, c, 32) != want
+            changed |= _thread_counts(hb.exp_stream, L, gaps, hb.header.total_bits, c, 32,
+                                      8 * bpt) != want
         _, err = gpu_decode(hb)
         assert bool(err & df11.DEVERR_COUNT) == changed
         flagged += changed

@@ -220,7 +220,7 @@ def test_validate_flags_corruption():
     assert df11.validate(bad) == 4
     bad = _fresh_block()                       # a gap past the end of the stream
     g = bad.gaps.size * 2 - 1
-    assert 64 * g >= bad.header.total_bits
+    assert 8 * bad.header.bytes_per_thread * g >= bad.header.total_bits
     bad.gaps[g // 2] |= 0x50
     assert df11.validate(bad) == 4
     bad = _fresh_block(); bad.gaps[0] |= 0x01  # thread 0 always starts at bit 0
