@@ -19,11 +19,14 @@
 //     (row k holds word k of every lane: conflict-free stores), then moved
 //     into a contiguous, 8-element-aligned exponent buffer with funnel-shifted
 //     word stores (shared-memory OR only on words two lanes share);
-//   * the sign|mantissa bytes of the chunk and the next chunk's stream words
-//     are loaded into registers before decoding, so their latency hides
-//     behind the decode;
-//   * the merge joins 8 exponents with 8 sign|mantissa bytes per lane and
-//     writes one 16-byte BF16 vector per lane;
+//   * the chunk's sign|mantissa bytes are staged into shared memory by one
+//     TMA bulk copy (cp.async.bulk + mbarrier) issued before decoding; the
+//     next chunk's stream words are loaded into registers a chunk ahead;
+//   * per-warp buffers are sized by the codebook's shortest code (the kernel
+//     rejects table entries shorter than it), so blocks whose codes are at
+//     least 2 bits long fit twice as many warps per SM;
+//   * the merge builds four BF16 values with two bit-selects and two byte
+//     permutes and writes one 16-byte vector per lane and group;
 //   * persistent CTAs: grid = resident CTAs per SM x SM count.
 // No tensor cores: this is integer decode, bounded by HBM traffic and issue.
 #include "df11.h"
@@ -36,10 +39,11 @@
 namespace {
 
 constexpr uint32_t kLutPointer = 0x8000u;
-constexpr uint32_t kLutNoCode = 0x4000u | (1u << 8);
 constexpr int kWindowBits = 10;                    // multi-code table index width
 constexpr int kMultiEntries = 1 << kWindowBits;
 constexpr int kMaxCodesPerEntry = 3;
+constexpr int kMaxWarpsPerCta = 16;
+constexpr uint32_t kWaitLimit = 1u << 22;          // bounded mbarrier polls
 
 struct DecodeParams {
     const uint8_t *stream;
@@ -53,27 +57,33 @@ struct DecodeParams {
     uint64_t n_chunks;
     uint64_t out_limit;   // min(n_elements, out_capacity)
     uint32_t n_tables;
+    uint32_t min_len;     // shortest legal code; shorter table entries are corrupt
 };
 
-// Shared-memory layout per CTA: multi-code table, per-warp slot columns and
-// exponent buffers, then the two-level tables.
-template <int W>
+// Per-warp buffers for W stream bytes per lane and codes of at least MINLEN
+// bits: slot columns, the contiguous exponent buffer, the staged
+// sign|mantissa bytes.
+template <int W, int MINLEN>
 struct Geometry {
-    static constexpr int kSliceBits = 8 * W;              // 64 or 128
-    static constexpr int kMaxCodes = kSliceBits;          // 1-bit codes at most
-    static constexpr int kSlotRows = kMaxCodes / 4 + 1;   // + codes past the slice end
-    static constexpr int kSlotBytes = kSlotRows * 32 * 4; // per warp
-    static constexpr int kEbufBytes = 32 * kMaxCodes + 16; // per warp, multiple of 16
-    static constexpr int kWords = W / 4 + 1;              // stream words per lane incl. halo
-    static constexpr int kPrefetch = W / 2;               // 8-byte sign|mantissa groups per lane
+    static constexpr int kSliceBits = 8 * W;                         // 64 or 128
+    static constexpr int kMaxCodes = (kSliceBits + MINLEN - 1) / MINLEN;  // per lane
+    static constexpr int kSlotRows = (kMaxCodes + 2 + 3) / 4;        // + codes past the end
+    static constexpr int kSlotBytes = kSlotRows * 32 * 4;
+    static constexpr int kEbufBytes = 32 * kMaxCodes + 16;           // multiple of 16
+    static constexpr int kSbufBytes = 32 * kMaxCodes + 32;           // 16-aligned copy range
+    static constexpr int kWarpBytes = kSlotBytes + kEbufBytes + kSbufBytes;
+    static constexpr int kWords = W / 4 + 1;                         // stream words incl. halo
+    static_assert(kWarpBytes % 16 == 0, "per-warp area must keep 16-byte alignment");
 };
 
-template <int W, int WARPS>
-constexpr size_t smem_bytes_for(uint32_t n_tables)
+// Shared memory: mbarriers | multi-code table | code lengths | per-warp areas
+// | two-level tables.
+constexpr size_t kHeadBytes = kMaxWarpsPerCta * 8 + kMultiEntries * 4 + 256;
+
+template <int W, int MINLEN>
+constexpr size_t smem_bytes_for(int warps, uint32_t n_tables)
 {
-    using G = Geometry<W>;
-    return (size_t)kMultiEntries * 4 + 256 + (size_t)WARPS * (G::kSlotBytes + G::kEbufBytes) +
-           (size_t)n_tables * 512;
+    return kHeadBytes + (size_t)warps * Geometry<W, MINLEN>::kWarpBytes + (size_t)n_tables * 512;
 }
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
@@ -98,9 +108,53 @@ __device__ __forceinline__ uint16_t join1(uint32_t e, uint32_t s)
     return (uint16_t)(((s & 0x80u) << 8) | (e << 7) | (s & 0x7Fu));
 }
 
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// ---- mbarrier + bulk copy (TMA) helpers ------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint32_t bar)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+
+// Copies `bytes` (multiple of 16, 16-byte aligned ends) from global to shared
+// memory; completion is signalled on `bar` (one arrival carrying the bytes).
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t bar)
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Waits until the barrier completes the phase with the given parity; gives up
+// after kWaitLimit polls and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+{
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.b32 %0, 1, 0, p; }"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done)
+            return true;
+    }
+    return false;
+}
+
 // Loads lane's stream words (big-endian, MSB-first bit order) and gap.
 template <int W>
-__device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, uint32_t (&w)[Geometry<W>::kWords],
+__device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, uint32_t (&w)[W / 4 + 1],
                                            uint32_t &gap)
 {
     const uint8_t *src = p.stream + (uint64_t)W * g;
@@ -120,46 +174,56 @@ __device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, ui
     gap = (p.gaps[g >> 1] >> ((g & 1) * 4)) & 0xFu;
 }
 
-template <int W, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
+template <int W, int MINLEN>
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(DecodeParams p)
 {
-    using G = Geometry<W>;
+    using G = Geometry<W, MINLEN>;
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t *multi = reinterpret_cast<uint32_t *>(smem);
-    uint8_t *len_of = smem + kMultiEntries * 4;                 // code length by exponent
-    uint8_t *warp_area = len_of + 256;
-    uint16_t *lut = reinterpret_cast<uint16_t *>(warp_area + WARPS * (G::kSlotBytes + G::kEbufBytes));
+    const int warps = blockDim.x >> 5;
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(smem);
+    uint32_t *multi = reinterpret_cast<uint32_t *>(smem + kMaxWarpsPerCta * 8);
+    uint8_t *len_of = smem + kMaxWarpsPerCta * 8 + kMultiEntries * 4;   // code length by exponent
+    uint8_t *warp_area = smem + kHeadBytes;
+    uint16_t *lut = reinterpret_cast<uint16_t *>(warp_area + (size_t)warps * G::kWarpBytes);
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const uint32_t n_tables = p.n_tables;
+    const uint32_t min_len = p.min_len;
+    // "no code" in shared memory: flagged, and as long as the shortest code,
+    // so every decode step advances by at least min_len bits
+    const uint32_t no_code = 0x4000u | (min_len << 8);
 
     // ---- prologue: two-level tables, sanitised ------------------------------
-    // Anything malformed becomes "no code" (length 1), so decoding always
-    // advances and never indexes outside the tables.
-    for (uint32_t i = tid; i < n_tables * 256u; i += WARPS * 32) {
+    // Anything malformed (bad pointer, bad length, shorter than the shortest
+    // code) becomes "no code", so decoding never indexes outside the tables
+    // and a lane never produces more codes than its buffers hold.
+    for (uint32_t i = tid; i < n_tables * 256u; i += blockDim.x) {
         uint32_t e = p.lut[i];
         if (e & kLutPointer) {
             const uint32_t to = e & 0xFFu;
             if (i >= 256u || to == 0 || to >= n_tables || (e & 0x7F00u))
-                e = kLutNoCode;
+                e = no_code;
         } else {
             const uint32_t l = (e >> 8) & 0x1Fu;
-            if ((e & 0x4000u) || l == 0 || l > 16)
-                e = kLutNoCode;
+            if ((e & 0x4000u) || l < min_len || l > 16)
+                e = no_code;
             else
                 len_of[e & 0xFFu] = (uint8_t)l;   // every leaf of a symbol holds its length
         }
         lut[i] = (uint16_t)e;
     }
+    if (lane == 0)
+        mbar_init(smem_addr(&mbar[warp]));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
     // ---- prologue: multi-code table -----------------------------------------
     // Entry for a 10-bit window: the whole codes it starts with (at most 3),
     // as symbols in bytes 0..2, their count in bits 24..25 and their total
     // length in bits 28..31.  0 when the first code is longer than the window
     // (or is no code): the decoder then takes the two-level path.
-    for (int idx = tid; idx < kMultiEntries; idx += WARPS * 32) {
+    for (int idx = tid; idx < kMultiEntries; idx += blockDim.x) {
         const uint32_t win = (uint32_t)idx << (32 - kWindowBits);
         uint32_t t = 0, n = 0, syms = 0;
         while (n < kMaxCodesPerEntry) {
@@ -180,47 +244,38 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
     }
     __syncthreads();
 
-    uint32_t *slots = reinterpret_cast<uint32_t *>(warp_area + warp * (G::kSlotBytes + G::kEbufBytes));
-    uint8_t *ebuf = warp_area + warp * (G::kSlotBytes + G::kEbufBytes) + G::kSlotBytes;
+    uint8_t *area = warp_area + (size_t)warp * G::kWarpBytes;
+    uint32_t *slots = reinterpret_cast<uint32_t *>(area);
+    uint8_t *ebuf = area + G::kSlotBytes;
     uint32_t *ebuf32 = reinterpret_cast<uint32_t *>(ebuf);
+    uint8_t *sbuf = ebuf + G::kEbufBytes;
+    const uint32_t bar = smem_addr(&mbar[warp]);
+    uint32_t parity = 0;
 
-    const uint64_t stride = (uint64_t)gridDim.x * WARPS;
-    uint64_t chunk = (uint64_t)blockIdx.x * WARPS + warp;
+    const uint64_t stride = (uint64_t)gridDim.x * warps;
+    uint64_t chunk = (uint64_t)blockIdx.x * warps + warp;
     if (chunk >= p.n_chunks)
         return;
 
     uint32_t err = 0;
-    // Per chunk: positions valid?  Whole 8-element groups [gfirst, gend) of
-    // the chunk's output (relative to the 8-aligned base) get their
-    // sign|mantissa bytes loaded ahead into registers.
-    auto positions_ok = [&](uint32_t a, uint32_t b) {
-        return a <= b && (uint64_t)b <= p.out_limit && b - a <= (uint32_t)(32 * G::kMaxCodes);
-    };
-    auto prefetch = [&](uint32_t a, uint32_t b, bool ok, uint2 (&dst)[G::kPrefetch]) {
-        const uint32_t hd = a & 7u;
-        const uint64_t bs = (uint64_t)a - hd;
-        const uint32_t g0 = hd ? 1u : 0u;
-        const uint32_t g1 = ok ? (hd + (b - a)) >> 3 : 0u;
-#pragma unroll
-        for (int j = 0; j < G::kPrefetch; ++j) {
-            const uint32_t i = g0 + lane + 32 * j;
-            dst[j] = i < g1 ? __ldg(reinterpret_cast<const uint2 *>(p.signmant + bs + 8ull * i))
-                            : make_uint2(0u, 0u);
-        }
-    };
-
+    bool stalled = false;      // a staged copy did not arrive in time
     uint32_t w[G::kWords];
     uint32_t gap;
     load_slice<W>(p, chunk * 32 + lane, w, gap);
     uint32_t pos0 = p.chunk_pos[chunk], pos1 = p.chunk_pos[chunk + 1];
-    bool pos_ok = positions_ok(pos0, pos1);
-    uint2 pre[G::kPrefetch];
-    prefetch(pos0, pos1, pos_ok, pre);
 
     for (;;) {
+        // ---- positions (warp-uniform) and the staged sign|mantissa copy -----
+        const bool pos_ok = pos0 <= pos1 && (uint64_t)pos1 <= p.out_limit &&
+                            pos1 - pos0 <= (uint32_t)(32 * G::kMaxCodes);
         const uint32_t head = pos0 & 7u;
         const uint64_t base = (uint64_t)pos0 - head;           // 8-element aligned
         const uint32_t gfirst = head ? 1u : 0u;
+        // copy [pos0 & ~15, ceil16(pos1)) -> sbuf; group i is at sbuf + (pos0 & 8) + 8i
+        const uint64_t cp_lo = (uint64_t)pos0 & ~15ull;
+        const uint32_t cp_bytes = pos_ok ? (uint32_t)((((uint64_t)pos1 + 15) & ~15ull) - cp_lo) : 0u;
+        if (cp_bytes && lane == 0)
+            bulk_copy_g2s(smem_addr(sbuf), p.signmant + cp_lo, cp_bytes, bar);
 
         // ---- the next chunk's slice and positions, loaded ahead -------------
         const uint64_t next = chunk + stride;
@@ -233,14 +288,8 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
             npos1 = p.chunk_pos[next + 1];
         }
 
-        uint2 npre[G::kPrefetch];
-        bool npos_ok = false;
         if (!pos_ok) {
             err |= DF11_DEVERR_BAD_POS;
-            if (has_next) {
-                npos_ok = positions_ok(npos0, npos1);
-                prefetch(npos0, npos1, npos_ok, npre);
-            }
         } else {
             // ---- decode this lane's slice ----------------------------------
             // Codes starting in [gap, end) belong to this lane.  The loop
@@ -304,12 +353,6 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
             if (seen & 0x4000u)
                 err |= DF11_DEVERR_BAD_CODE;
 
-            // ---- sign|mantissa of the next chunk, loaded ahead -------------
-            if (has_next) {
-                npos_ok = positions_ok(npos0, npos1);
-                prefetch(npos0, npos1, npos_ok, npre);
-            }
-
             // ---- warp scan of the counts ------------------------------------
             uint32_t incl = count;
 #pragma unroll
@@ -370,29 +413,34 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
             }
             __syncwarp();
 
+            // ---- wait for the staged sign|mantissa bytes --------------------
+            if (cp_bytes) {
+                if (!mbar_wait(bar, parity)) {
+                    err |= DF11_DEVERR_TIMEOUT;
+                    stalled = true;
+                }
+                parity ^= 1u;
+            }
+
             // ---- merge with sign|mantissa and store -------------------------
             // Whole groups: 8 exponents + 8 sign|mantissa bytes -> one 16-byte
             // store per lane.  The partial groups at both ends (<= 7 elements
             // each) take one element per lane on lanes 0..15.
-            const uint32_t span = head + n_write;
-            const uint32_t mend = span >> 3;                   // whole groups end
-            uint4 *const out16 = reinterpret_cast<uint4 *>(p.out + base);   // group i -> out16[i]
-            const uint2 *const e64 = reinterpret_cast<const uint2 *>(ebuf);
-            auto merge_group = [&](uint32_t i, uint2 s8) {
-                const uint2 e8 = e64[i];
-                const uint2 a = join4(e8.x, s8.x);
-                const uint2 b = join4(e8.y, s8.y);
-                out16[i] = make_uint4(a.x, a.y, b.x, b.y);
-            };
-#pragma unroll
-            for (int j = 0; j < G::kPrefetch; ++j) {
-                const uint32_t i = gfirst + lane + 32 * j;
-                if (i < mend)
-                    merge_group(i, pre[j]);
-            }
-            for (uint32_t i = gfirst + lane + 32 * G::kPrefetch; i < mend; i += 32)
-                merge_group(i, __ldg(reinterpret_cast<const uint2 *>(p.signmant + base + 8ull * i)));
-            {
+            if (!stalled) {
+                const uint32_t span = head + n_write;
+                const uint32_t mend = span >> 3;                   // whole groups end
+                const uint8_t *sgrp = sbuf + (pos0 & 8u);          // group 0 of the chunk
+                uint4 *const out16 = reinterpret_cast<uint4 *>(p.out + base);
+                const uint2 *const e64 = reinterpret_cast<const uint2 *>(ebuf);
+                const uint2 *const s64 = reinterpret_cast<const uint2 *>(sgrp);
+#pragma unroll 2
+                for (uint32_t i = gfirst + lane; i < mend; i += 32) {
+                    const uint2 e8 = e64[i];
+                    const uint2 s8 = s64[i];
+                    const uint2 x = join4(e8.x, s8.x);
+                    const uint2 y = join4(e8.y, s8.y);
+                    out16[i] = make_uint4(x.x, x.y, y.x, y.y);
+                }
                 const uint32_t fs = gfirst * 8;                    // first whole-group element
                 const uint32_t hend = min(fs, span);               // head part: [head, hend)
                 const uint32_t tbeg = max(mend * 8, fs);           // tail part: [tbeg, span)
@@ -405,25 +453,23 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
                         l = tbeg + (lane - 8);
                 }
                 if (l != 0xFFFFFFFFu)
-                    p.out[base + l] = join1(ebuf[l], p.signmant[base + l]);
+                    p.out[base + l] = join1(ebuf[l], sgrp[l]);
             }
             __syncwarp();
         }
 
-        if (!has_next)
+        if (!has_next || stalled)
             break;
         chunk = next;
 #pragma unroll
         for (int k = 0; k < G::kWords; ++k)
             w[k] = nw[k];
-#pragma unroll
-        for (int j = 0; j < G::kPrefetch; ++j)
-            pre[j] = npre[j];
         gap = ngap;
         pos0 = npos0;
         pos1 = npos1;
-        pos_ok = npos_ok;
     }
+    if (stalled)   // let the late copy land before this CTA's shared memory is released
+        mbar_wait(bar, parity ^ 1u);
     if (err && p.err)
         atomicOr(p.err, err);
 }
@@ -431,21 +477,26 @@ __global__ void __launch_bounds__(WARPS * 32) df11_decode_kernel(DecodeParams p)
 // ------------------------------------------------------------ launch
 
 constexpr int kMaxDevices = 64;
-constexpr int kWarpsPerCta = 8;
-// resident CTAs per SM, by device, slice width and table count
-std::atomic<int> g_occupancy[kMaxDevices][2][257];
+constexpr size_t kSmemLimit = 227 * 1024;
+// resident CTAs per SM, by device, kernel variant and table count
+std::atomic<int> g_occupancy[kMaxDevices][4][257];
 std::atomic<int> g_sm_count[kMaxDevices];
-std::atomic<int> g_attr_done[kMaxDevices][2];
+std::atomic<int> g_attr_done[kMaxDevices][4];
 
-template <int W>
+template <int W, int MINLEN>
 df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream)
 {
-    constexpr int v = W == 8 ? 0 : 1;
-    auto kernel = df11_decode_kernel<W, kWarpsPerCta>;
-    const size_t smem = smem_bytes_for<W, kWarpsPerCta>(prm.n_tables);
+    constexpr int v = (W == 8 ? 0 : 2) + (MINLEN == 1 ? 0 : 1);
+    auto kernel = df11_decode_kernel<W, MINLEN>;
+    int warps = kMaxWarpsPerCta;
+    while (warps > 1 && smem_bytes_for<W, MINLEN>(warps, prm.n_tables) > kSmemLimit)
+        warps /= 2;
+    const size_t smem = smem_bytes_for<W, MINLEN>(warps, prm.n_tables);
+    if (smem > kSmemLimit)
+        return DF11_ERR_INVALID_ARGUMENT;
     if (!g_attr_done[dev][v].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem_bytes_for<W, kWarpsPerCta>(256)) != cudaSuccess)
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit) !=
+            cudaSuccess)
             return DF11_ERR_CUDA;
         g_attr_done[dev][v].store(1, std::memory_order_release);
     }
@@ -457,18 +508,16 @@ df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream)
     }
     int occ = g_occupancy[dev][v][prm.n_tables].load(std::memory_order_relaxed);
     if (occ == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kWarpsPerCta * 32, smem) !=
-            cudaSuccess)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, warps * 32, smem) != cudaSuccess)
             return DF11_ERR_CUDA;
         if (occ < 1)
             return DF11_ERR_CUDA;
         g_occupancy[dev][v][prm.n_tables].store(occ, std::memory_order_relaxed);
     }
-    const uint64_t warps_needed = prm.n_chunks;
-    const uint64_t ctas_needed = (warps_needed + kWarpsPerCta - 1) / kWarpsPerCta;
+    const uint64_t ctas_needed = (prm.n_chunks + warps - 1) / warps;
     const uint64_t resident = (uint64_t)occ * (uint64_t)sms;
     const unsigned grid = (unsigned)(ctas_needed < resident ? ctas_needed : resident);
-    kernel<<<grid, kWarpsPerCta * 32, smem, stream>>>(prm);
+    kernel<<<grid, warps * 32, smem, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
@@ -487,7 +536,8 @@ extern "C" df11_status df11_decompress_async(const df11_device_block *blk, uint1
     if (h.threads_per_chunk != DF11_THREADS_PER_CHUNK || (W != 8 && W != 16))
         return DF11_ERR_INVALID_ARGUMENT;
     if (h.n_elements == 0 || h.n_elements >= (1ull << 32) || h.n_tables < 1 || h.n_tables > 256 ||
-        h.total_bits == 0 || out_capacity < h.n_elements)
+        h.total_bits == 0 || out_capacity < h.n_elements || h.min_code_len < 1 ||
+        h.min_code_len > DF11_MAX_CODE_LEN)
         return DF11_ERR_INVALID_ARGUMENT;
     const uint64_t chunk_bits = (uint64_t)DF11_THREADS_PER_CHUNK * 8 * W;
     if (h.n_chunks != (h.total_bits + chunk_bits - 1) / chunk_bits)
@@ -521,6 +571,9 @@ extern "C" df11_status df11_decompress_async(const df11_device_block *blk, uint1
     prm.n_chunks = h.n_chunks;
     prm.out_limit = h.n_elements < out_capacity ? h.n_elements : out_capacity;
     prm.n_tables = h.n_tables;
+    prm.min_len = h.min_code_len;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return W == 8 ? launch<8>(prm, dev, s) : launch<16>(prm, dev, s);
+    if (W == 8)
+        return h.min_code_len >= 2 ? launch<8, 2>(prm, dev, s) : launch<8, 1>(prm, dev, s);
+    return h.min_code_len >= 2 ? launch<16, 2>(prm, dev, s) : launch<16, 1>(prm, dev, s);
 }

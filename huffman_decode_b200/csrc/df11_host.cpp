@@ -481,6 +481,11 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
     out->hdr.threads_per_chunk = T;
     out->hdr.bytes_per_thread = layout->bytes_per_thread;
     out->hdr.n_tables = cb->n_tables;
+    out->hdr.min_code_len = DF11_MAX_CODE_LEN;
+    for (int s = 0; s < 256; ++s)
+        if (cb->code_len[s] && cb->code_len[s] < out->hdr.min_code_len)
+            out->hdr.min_code_len = cb->code_len[s];
+    out->hdr.reserved = 0;
     out->hdr.total_bits = total_bits;
     out->hdr.n_elements = N;
     out->hdr.n_chunks = z.n_chunks;
@@ -495,6 +500,7 @@ df11_status df11_validate(const df11_host_block *b)
     df11_layout ly{h.threads_per_chunk, h.bytes_per_thread};
     if (!layout_ok(&ly) || h.max_code_len < 1 || h.max_code_len > DF11_MAX_CODE_LEN ||
         h.n_tables < 1 || h.n_tables > 256 || h.n_elements == 0 ||
+        h.min_code_len < 1 || h.min_code_len > h.max_code_len ||
         h.n_elements >= (1ull << 32) || h.total_bits < h.n_elements ||
         h.total_bits > h.n_elements * h.max_code_len)
         return DF11_ERR_CORRUPT;
@@ -533,9 +539,11 @@ df11_status df11_validate(const df11_host_block *b)
                 if (t != 0 || to == 0 || to >= h.n_tables || (e & 0x7F00))
                     return DF11_ERR_CORRUPT;
             } else if (e & 0x4000) {
-                if (e != kLutNoCode || t != 0)
+                if (e != kLutNoCode || t != 0 || h.min_code_len != 1)
                     return DF11_ERR_CORRUPT;
             } else if (t == 0 ? (l < 1 || l > 8) : (l < 9 || l > h.max_code_len)) {
+                return DF11_ERR_CORRUPT;
+            } else if (l < h.min_code_len) {
                 return DF11_ERR_CORRUPT;
             }
         }

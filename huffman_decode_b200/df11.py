@@ -30,6 +30,7 @@ STATUS_NAMES = {
 DEVERR_COUNT = 0x1
 DEVERR_BAD_CODE = 0x2
 DEVERR_BAD_POS = 0x4
+DEVERR_TIMEOUT = 0x8
 MAX_CODE_LEN = 16
 STREAM_PAD = 16
 THREADS_PER_CHUNK = 32
@@ -94,6 +95,7 @@ class Header(ctypes.Structure):
     _fields_ = [
         ("max_code_len", ctypes.c_uint32), ("threads_per_chunk", ctypes.c_uint32),
         ("bytes_per_thread", ctypes.c_uint32), ("n_tables", ctypes.c_uint32),
+        ("min_code_len", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
         ("total_bits", ctypes.c_uint64), ("n_elements", ctypes.c_uint64),
         ("n_chunks", ctypes.c_uint64),
     ]

@@ -68,7 +68,7 @@ typedef enum {
     DF11_ERR_OVERFLOW = 3,         /* element count >= 2^32                     */
     DF11_ERR_CORRUPT = 4,          /* artifact fails a structural check         */
     DF11_ERR_CUDA = 5,             /* a CUDA runtime call failed                */
-    DF11_ERR_TIMEOUT = 6           /* reserved for bounded device waits         */
+    DF11_ERR_TIMEOUT = 6           /* reserved (device waits report DF11_DEVERR_TIMEOUT) */
 } df11_status;
 
 /* Bits the decoder ORs into the caller's device error word. */
@@ -78,6 +78,8 @@ typedef enum {
                                      entry (corrupt stream or table)           */
 #define DF11_DEVERR_BAD_POS 0x4u  /* chunk_pos not monotone or beyond
                                      out_capacity; that chunk writes nothing   */
+#define DF11_DEVERR_TIMEOUT 0x8u  /* a bounded wait for a staged copy ran out;
+                                     that chunk's output is not trustworthy    */
 
 #define DF11_MAX_CODE_LEN 16u     /* longest code the format allows           */
 #define DF11_MIN_CODE_LEN_CAP 8u  /* smallest cap accepted by build_codebook  */
@@ -117,12 +119,17 @@ typedef struct {
     uint64_t lut_entries;       /* n_tables * 256 (uint16 entries)             */
 } df11_sizes;
 
-/* Header fields shared by the host and device views of a block. */
+/* Header fields shared by the host and device views of a block.
+ * min_code_len is the shortest code in the codebook; the decoder treats any
+ * table entry shorter than it as corrupt, which bounds the codes per slice
+ * and so the decoder's per-warp buffers. */
 typedef struct {
     uint32_t max_code_len;
     uint32_t threads_per_chunk;
     uint32_t bytes_per_thread;
     uint32_t n_tables;
+    uint32_t min_code_len;
+    uint32_t reserved;          /* 0 */
     uint64_t total_bits;
     uint64_t n_elements;
     uint64_t n_chunks;

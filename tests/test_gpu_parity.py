@@ -188,6 +188,34 @@ def test_no_code_window_sets_bad_code_bit():
     assert np.all(got[hb.n_elements:] == 0x5A5A)
 
 
+@pytest.mark.parametrize("bpt", BPT)
+def test_header_claiming_longer_shortest_code_is_caught(bpt):
+    """A header whose min_code_len is larger than the codes in the tables
+    makes the kernel treat the short codes as corrupt: it reports it and
+    still writes nothing outside the block."""
+    mats = [m for _, m in workloads.llama_block(31, scale_div=512)]
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats, 32, bpt)
+    assert hb.header.min_code_len == 2
+    hb.header.min_code_len = 3
+    got, err = gpu_decode(hb, guard=64)
+    assert err & (df11.DEVERR_BAD_CODE | df11.DEVERR_COUNT)
+    assert np.all(got[hb.n_elements:] == 0x5A5A)
+
+
+@pytest.mark.parametrize("bpt", BPT)
+def test_header_claiming_shorter_shortest_code_still_decodes(bpt):
+    """min_code_len smaller than the real shortest code only enlarges the
+    kernel's buffers; the output stays exact."""
+    mats = [m for _, m in workloads.llama_block(32, scale_div=512)]
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats, 32, bpt)
+    hb.header.min_code_len = 1
+    got, err = gpu_decode(hb, guard=8)
+    assert err == 0
+    assert np.array_equal(got[: hb.n_elements], _flat(mats))
+
+
 def _thread_counts(stream, lengths, gap, total_bits, chunk, tpc, slice_bits):
     """Codes each thread of `chunk` decodes, by the oracle's bit-by-bit decode
     under the kernel's contract (codes starting in the slice, from its gap)."""

@@ -233,6 +233,23 @@ def test_validate_flags_corruption():
     assert df11.validate(bad) == 4
     bad = _fresh_block(); bad.header.total_bits = bad.header.n_elements - 1
     assert df11.validate(bad) == 4
+    # the header claims a shortest code longer than one the tables hold
+    bad = _fresh_block()
+    assert bad.header.min_code_len == 2
+    bad.header.min_code_len = 3
+    assert df11.validate(bad) == 4
+    bad = _fresh_block(); bad.header.min_code_len = 0
+    assert df11.validate(bad) == 4
+
+
+def test_header_min_code_len_matches_codebook():
+    for mats in ([m for _, m in workloads.llama_block(1002, scale_div=256)],
+                 [m for _, m in workloads.single_exponent(4002, (64, 64))],
+                 [m for _, m in workloads.uniform_bits(4003, (64, 64))]):
+        cb = df11.build_codebook(mats)
+        hb = df11.compress(cb, mats)
+        L = cb.lengths()
+        assert hb.header.min_code_len == int(L[L > 0].min())
 
 
 def test_decompress_rejects_bad_arguments_before_any_cuda_call():
@@ -283,3 +300,7 @@ def test_decompress_rejects_bad_arguments_before_any_cuda_call():
     h = binding.Header.from_buffer_copy(hb.header)
     h.n_tables = 0
     assert call(dev_block(hdr=h)) == 1
+    for bad_min in (0, 17):
+        h = binding.Header.from_buffer_copy(hb.header)
+        h.min_code_len = bad_min
+        assert call(dev_block(hdr=h)) == 1
