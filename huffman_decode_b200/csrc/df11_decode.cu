@@ -113,6 +113,56 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p)
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// ---- 32-bit shared-window accesses -----------------------------------------
+// The hot loops address shared memory with 32-bit shared-window offsets.
+// Table reads (read-only after the prologue) may be scheduled freely; reads
+// of data written during a chunk are ordered with "memory".
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a)
+{
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a)
+{
+    unsigned short v;
+    asm("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a)
+{
+    uint32_t v;
+    asm("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u32_m(uint32_t a)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u8_m(uint32_t a)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint2 lds_v2_m(uint32_t a)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v)
+{
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_or_u32(uint32_t a, uint32_t v)
+{
+    asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
 // ---- mbarrier + bulk copy (TMA) helpers ------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint32_t bar)
@@ -244,11 +294,15 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
     }
     __syncthreads();
 
-    uint8_t *area = warp_area + (size_t)warp * G::kWarpBytes;
-    uint32_t *slots = reinterpret_cast<uint32_t *>(area);
-    uint8_t *ebuf = area + G::kSlotBytes;
-    uint32_t *ebuf32 = reinterpret_cast<uint32_t *>(ebuf);
-    uint8_t *sbuf = ebuf + G::kEbufBytes;
+    // shared-window addresses (bytes)
+    const uint32_t smem_base = smem_addr(smem);
+    const uint32_t multi_a = smem_base + kMaxWarpsPerCta * 8;
+    const uint32_t len_a = multi_a + kMultiEntries * 4;
+    const uint32_t lut_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warps * G::kWarpBytes);
+    const uint32_t slots_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warp * G::kWarpBytes);
+    const uint32_t slot_lane_a = slots_a + 4u * lane;      // row 0 of this lane's column
+    const uint32_t ebuf_a = slots_a + G::kSlotBytes;
+    const uint32_t sbuf_a = ebuf_a + G::kEbufBytes;
     const uint32_t bar = smem_addr(&mbar[warp]);
     uint32_t parity = 0;
 
@@ -275,7 +329,7 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
         const uint64_t cp_lo = (uint64_t)pos0 & ~15ull;
         const uint32_t cp_bytes = pos_ok ? (uint32_t)((((uint64_t)pos1 + 15) & ~15ull) - cp_lo) : 0u;
         if (cp_bytes && lane == 0)
-            bulk_copy_g2s(smem_addr(sbuf), p.signmant + cp_lo, cp_bytes, bar);
+            bulk_copy_g2s(sbuf_a, p.signmant + cp_lo, cp_bytes, bar);
 
         // ---- the next chunk's slice and positions, loaded ahead -------------
         const uint64_t next = chunk + stride;
@@ -300,7 +354,8 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
                                 ? 0
                                 : (int)min((uint64_t)G::kSliceBits, p.total_bits - bit0);
             int bitpos = (int)gap;
-            uint32_t count = 0, nb = 0, row = 0, accl = 0, acch = 0, seen = 0;
+            uint32_t count = 0, nb = 0, accl = 0, acch = 0, seen = 0;
+            uint32_t sp = slot_lane_a;               // next slot word of this lane
             uint32_t r = 0, adv = 0;                 // last entry and its length
 #pragma unroll
             for (int h = 0; h < G::kWords - 1; ++h) {
@@ -308,13 +363,13 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
                 const int lim = min(end, 32 * (h + 1));
                 while (bitpos < lim) {
                     const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
-                    r = multi[win >> (32 - kWindowBits)];
+                    r = lds_u32(multi_a + ((win >> (32 - kWindowBits)) << 2));
                     adv = r >> 28;
                     if (r < (1u << 28)) {
                         // first code longer than the window: two-level tables
-                        uint32_t e = lut[win >> 24];
+                        uint32_t e = lds_u16(lut_a + ((win >> 24) << 1));
                         if (e & kLutPointer)
-                            e = lut[((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)];
+                            e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)) << 1));
                         seen |= e;
                         r = (e & 0xFFu) | (1u << 24);
                         adv = (e >> 8) & 0x1Fu;
@@ -326,8 +381,8 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
                     acch |= (uint32_t)(sv >> 32);
                     nb += n;
                     if (nb >= 4) {
-                        slots[row * 32 + lane] = accl;
-                        ++row;
+                        sts_u32(sp, accl);
+                        sp += 128;
                         accl = acch;
                         acch = 0;
                         nb -= 4;
@@ -335,18 +390,18 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
                 }
             }
             if (nb)
-                slots[row * 32 + lane] = accl;
-            count = row * 4 + nb;
+                sts_u32(sp, accl);
+            count = ((sp - slot_lane_a) >> 5) + nb;      // 4 codes per 128-byte row
             if (count) {
                 // codes of the last entry that start at or past `end`
                 const uint32_t n = (r >> 24) & 3u;
                 const int p_last = bitpos - (int)adv;
                 uint32_t keep = 1;
                 if (n >= 2) {
-                    const int c1 = p_last + len_of[r & 0xFFu];
+                    const int c1 = p_last + (int)lds_u8(len_a + (r & 0xFFu));
                     keep += c1 < end;
                     if (n == 3)
-                        keep += c1 + len_of[(r >> 8) & 0xFFu] < end;
+                        keep += c1 + (int)lds_u8(len_a + ((r >> 8) & 0xFFu)) < end;
                 }
                 count -= n - keep;
             }
@@ -379,36 +434,40 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             const bool head_shared = sh != 0;
             const bool tail_shared = ((a + nbytes) & 3u) != 0;
             const uint32_t nwords = (nbytes + 3) >> 2;
+            const uint32_t first_a = ebuf_a + 4u * first;
+            const uint32_t last_a = ebuf_a + 4u * last;
             if (nbytes) {
                 if (head_shared)
-                    ebuf32[first] = 0u;
+                    sts_u32(first_a, 0u);
                 if (tail_shared)
-                    ebuf32[last] = 0u;
-                if (nbytes & 3u)                        // clear bytes past nbytes
-                    slots[(nwords - 1) * 32 + lane] &= (1u << (8 * (nbytes & 3u))) - 1;
+                    sts_u32(last_a, 0u);
+                if (nbytes & 3u) {                       // clear bytes past nbytes
+                    const uint32_t ta = slot_lane_a + (nwords - 1) * 128;
+                    sts_u32(ta, lds_u32_m(ta) & ((1u << (8 * (nbytes & 3u))) - 1));
+                }
             }
             __syncwarp();
             if (nbytes) {
-                uint32_t prev = slots[lane];
+                uint32_t prev = lds_u32_m(slot_lane_a);
                 uint32_t v = prev << sh;
                 if (head_shared || (first == last && tail_shared))
-                    atomicOr(ebuf32 + first, v);
+                    red_or_u32(first_a, v);
                 else
-                    ebuf32[first] = v;
-                uint32_t j = 1;
+                    sts_u32(first_a, v);
+                uint32_t src = slot_lane_a + 128, dst = first_a + 4;
 #pragma unroll 4
-                for (; first + j < last; ++j) {
-                    const uint32_t cur = slots[j * 32 + lane];
-                    ebuf32[first + j] = __funnelshift_l(prev, cur, sh);
+                for (; dst < last_a; src += 128, dst += 4) {
+                    const uint32_t cur = lds_u32_m(src);
+                    sts_u32(dst, __funnelshift_l(prev, cur, sh));
                     prev = cur;
                 }
-                if (first + j == last) {
-                    const uint32_t cur = j < nwords ? slots[j * 32 + lane] : 0u;
+                if (dst == last_a) {
+                    const uint32_t cur = src < slot_lane_a + nwords * 128 ? lds_u32_m(src) : 0u;
                     v = __funnelshift_l(prev, cur, sh);
                     if (tail_shared)
-                        atomicOr(ebuf32 + last, v);
+                        red_or_u32(last_a, v);
                     else
-                        ebuf32[last] = v;
+                        sts_u32(last_a, v);
                 }
             }
             __syncwarp();
@@ -429,14 +488,12 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             if (!stalled) {
                 const uint32_t span = head + n_write;
                 const uint32_t mend = span >> 3;                   // whole groups end
-                const uint8_t *sgrp = sbuf + (pos0 & 8u);          // group 0 of the chunk
+                const uint32_t sgrp_a = sbuf_a + (pos0 & 8u);     // group 0 of the chunk
                 uint4 *const out16 = reinterpret_cast<uint4 *>(p.out + base);
-                const uint2 *const e64 = reinterpret_cast<const uint2 *>(ebuf);
-                const uint2 *const s64 = reinterpret_cast<const uint2 *>(sgrp);
 #pragma unroll 2
                 for (uint32_t i = gfirst + lane; i < mend; i += 32) {
-                    const uint2 e8 = e64[i];
-                    const uint2 s8 = s64[i];
+                    const uint2 e8 = lds_v2_m(ebuf_a + 8u * i);
+                    const uint2 s8 = lds_v2_m(sgrp_a + 8u * i);
                     const uint2 x = join4(e8.x, s8.x);
                     const uint2 y = join4(e8.y, s8.y);
                     out16[i] = make_uint4(x.x, x.y, y.x, y.y);
@@ -453,7 +510,7 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
                         l = tbeg + (lane - 8);
                 }
                 if (l != 0xFFFFFFFFu)
-                    p.out[base + l] = join1(ebuf[l], sgrp[l]);
+                    p.out[base + l] = join1(lds_u8_m(ebuf_a + l), lds_u8_m(sgrp_a + l));
             }
             __syncwarp();
         }
