@@ -58,6 +58,7 @@ struct DecodeParams {
     uint64_t out_limit;   // min(n_elements, out_capacity)
     uint32_t n_tables;
     uint32_t min_len;     // shortest legal code; shorter table entries are corrupt
+    uint32_t full_chunks; // chunks lying wholly below total_bits (every slice full)
 };
 
 // Per-warp buffers for W stream bytes per lane and codes of at least MINLEN
@@ -87,6 +88,13 @@ constexpr size_t smem_bytes_for(int warps, uint32_t n_tables)
 }
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
+
+// A compile-time int that converts like a runtime one (lets one code path be
+// instantiated with a constant slice end).
+template <int V>
+struct ConstInt {
+    __device__ constexpr operator int() const { return V; }
+};
 
 // Four BF16 values from four exponent bytes (e) and four sign|mantissa bytes
 // (s), element k in byte k.  BF16 = sign (bit 15) | exponent (14..7) |
@@ -349,61 +357,72 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             // Codes starting in [gap, end) belong to this lane.  The loop
             // runs while bitpos < end; the last table entry may also hold
             // codes that start at or past `end` -- they are dropped below.
-            const uint64_t bit0 = (chunk * 32 + lane) * (uint64_t)G::kSliceBits;
-            const int end = bit0 >= p.total_bits
-                                ? 0
-                                : (int)min((uint64_t)G::kSliceBits, p.total_bits - bit0);
-            int bitpos = (int)gap;
-            uint32_t count = 0, nb = 0, accl = 0, acch = 0, seen = 0;
-            uint32_t sp = slot_lane_a;               // next slot word of this lane
-            uint32_t r = 0, adv = 0;                 // last entry and its length
+            // Chunks below the last are full: end is the constant slice width.
+            uint32_t seen = 0;
+            auto decode = [&](auto end_arg) -> uint32_t {
+                const int end = end_arg;
+                int bitpos = (int)gap;
+                uint32_t nb = 0, accl = 0, acch = 0;
+                uint32_t sp = slot_lane_a;           // next slot word of this lane
+                uint32_t r = 0, adv = 0;             // last entry and its length
 #pragma unroll
-            for (int h = 0; h < G::kWords - 1; ++h) {
-                const uint32_t hi = w[h], lo = w[h + 1];
-                const int lim = min(end, 32 * (h + 1));
-                while (bitpos < lim) {
-                    const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
-                    r = lds_u32(multi_a + ((win >> (32 - kWindowBits)) << 2));
-                    adv = r >> 28;
-                    if (r < (1u << 28)) {
-                        // first code longer than the window: two-level tables
-                        uint32_t e = lds_u16(lut_a + ((win >> 24) << 1));
-                        if (e & kLutPointer)
-                            e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)) << 1));
-                        seen |= e;
-                        r = (e & 0xFFu) | (1u << 24);
-                        adv = (e >> 8) & 0x1Fu;
+                for (int h = 0; h < G::kWords - 1; ++h) {
+                    const uint32_t hi = w[h], lo = w[h + 1];
+                    const int lim = min(end, 32 * (h + 1));
+                    while (bitpos < lim) {
+                        const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
+                        r = lds_u32(multi_a + ((win >> (32 - kWindowBits)) << 2));
+                        adv = r >> 28;
+                        if (r < (1u << 28)) {
+                            // first code longer than the window: two-level tables
+                            uint32_t e = lds_u16(lut_a + ((win >> 24) << 1));
+                            if (e & kLutPointer)
+                                e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)) << 1));
+                            seen |= e;
+                            r = (e & 0xFFu) | (1u << 24);
+                            adv = (e >> 8) & 0x1Fu;
+                        }
+                        bitpos += (int)adv;
+                        const uint32_t n = (r >> 24) & 3u;
+                        const uint64_t sv = (uint64_t)(r & 0xFFFFFFu) << (8 * nb);
+                        accl |= (uint32_t)sv;
+                        acch |= (uint32_t)(sv >> 32);
+                        nb += n;
+                        if (nb >= 4) {
+                            sts_u32(sp, accl);
+                            sp += 128;
+                            accl = acch;
+                            acch = 0;
+                            nb -= 4;
+                        }
                     }
-                    bitpos += (int)adv;
+                }
+                if (nb)
+                    sts_u32(sp, accl);
+                uint32_t cnt = ((sp - slot_lane_a) >> 5) + nb;   // 4 codes per 128-byte row
+                if (cnt) {
+                    // codes of the last entry that start at or past `end`
                     const uint32_t n = (r >> 24) & 3u;
-                    const uint64_t sv = (uint64_t)(r & 0xFFFFFFu) << (8 * nb);
-                    accl |= (uint32_t)sv;
-                    acch |= (uint32_t)(sv >> 32);
-                    nb += n;
-                    if (nb >= 4) {
-                        sts_u32(sp, accl);
-                        sp += 128;
-                        accl = acch;
-                        acch = 0;
-                        nb -= 4;
+                    const int p_last = bitpos - (int)adv;
+                    uint32_t keep = 1;
+                    if (n >= 2) {
+                        const int c1 = p_last + (int)lds_u8(len_a + (r & 0xFFu));
+                        keep += c1 < end;
+                        if (n == 3)
+                            keep += c1 + (int)lds_u8(len_a + ((r >> 8) & 0xFFu)) < end;
                     }
+                    cnt -= n - keep;
                 }
-            }
-            if (nb)
-                sts_u32(sp, accl);
-            count = ((sp - slot_lane_a) >> 5) + nb;      // 4 codes per 128-byte row
-            if (count) {
-                // codes of the last entry that start at or past `end`
-                const uint32_t n = (r >> 24) & 3u;
-                const int p_last = bitpos - (int)adv;
-                uint32_t keep = 1;
-                if (n >= 2) {
-                    const int c1 = p_last + (int)lds_u8(len_a + (r & 0xFFu));
-                    keep += c1 < end;
-                    if (n == 3)
-                        keep += c1 + (int)lds_u8(len_a + ((r >> 8) & 0xFFu)) < end;
-                }
-                count -= n - keep;
+                return cnt;
+            };
+            uint32_t count;
+            if (chunk < p.full_chunks) {
+                count = decode(ConstInt<G::kSliceBits>{});
+            } else {
+                const uint64_t bit0 = ((uint64_t)chunk * 32 + lane) * (uint64_t)G::kSliceBits;
+                count = decode(bit0 >= p.total_bits
+                                   ? 0
+                                   : (int)min((uint64_t)G::kSliceBits, p.total_bits - bit0));
             }
             if (seen & 0x4000u)
                 err |= DF11_DEVERR_BAD_CODE;
@@ -629,6 +648,7 @@ extern "C" df11_status df11_decompress_async(const df11_device_block *blk, uint1
     prm.out_limit = h.n_elements < out_capacity ? h.n_elements : out_capacity;
     prm.n_tables = h.n_tables;
     prm.min_len = h.min_code_len;
+    prm.full_chunks = (uint32_t)(h.total_bits / chunk_bits);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (W == 8)
         return h.min_code_len >= 2 ? launch<8, 2>(prm, dev, s) : launch<8, 1>(prm, dev, s);
