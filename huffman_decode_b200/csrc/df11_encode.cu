@@ -1,0 +1,453 @@
+// df11_encode.cu -- GPU-side DF11 compressor (sm_100a).
+//
+// The pages compress on the CPU only ("DFloat11: lossless BFloat16
+// compression", section "How to develop with it": single-thread compression
+// per transformer block, minutes per block).  This file does the same work
+// on the GPU for one block already in device memory:
+//   1. df11_histogram_device   -- 256-bin exponent histogram (per-CTA shared
+//                                 histograms, one global add per bin and CTA);
+//   2. (host) df11_build_codebook_from_histogram -- code lengths, canonical
+//                                 codes and tables from that histogram;
+//   3. df11_compress_device    -- bit count per segment of 8192 elements,
+//      a scan of the segment counts, then one encode pass in which every
+//      thread knows its first bit: it appends its codes MSB-first into
+//      32-bit stream words (words shared with a neighbouring thread are
+//      ORed), records the gap of every slice whose first code it owns and
+//      the output position of every chunk that starts in such a slice, and
+//      writes its sign|mantissa bytes.
+// The result is byte-identical to df11_compress (host) for the same
+// codebook and layout ("How it works": canonical codes, MSB-first encode;
+// "Architecture": Gaps and per-chunk output positions).
+#include "df11.h"
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+namespace {
+
+constexpr int kEncThreads = 256;
+constexpr int kElemsPerThread = 32;
+constexpr int kSegElems = kEncThreads * kElemsPerThread;   // 8192 elements per segment
+constexpr int kScanThreads = 1024;
+
+// Code table passed by value: entry s = code | (length << 24); length 0 = absent.
+struct CodeTable {
+    uint32_t e[256];
+};
+
+struct EncodeParams {
+    const uint16_t *in;
+    uint8_t *stream;
+    uint8_t *gaps;
+    uint32_t *chunk_pos;
+    uint8_t *signmant;
+    uint32_t *seg_bits;     // scratch: bits per segment
+    uint64_t *seg_start;    // scratch: first bit per segment (exclusive scan)
+    uint32_t *err;          // optional device error word
+    uint64_t n;
+    uint64_t n_seg;
+    uint64_t total_bits;    // what the codebook promises
+    uint64_t n_threads;     // decoding threads (slices)
+    uint32_t slice_shift;   // log2(bits per slice)
+    uint32_t threads_per_chunk;
+};
+
+__device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
+
+// ---- histogram ---------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) histogram_kernel(const uint16_t *in, uint64_t n, uint64_t *hist)
+{
+    __shared__ uint32_t h[256];
+    h[threadIdx.x] = 0;
+    __syncthreads();
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x * 8;
+    const uint64_t n8 = n & ~7ull;
+    for (uint64_t i = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < n8; i += stride) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(in + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            atomicAdd(&h[(w[k] >> 7) & 0xFFu], 1u);
+            atomicAdd(&h[(w[k] >> 23) & 0xFFu], 1u);
+        }
+    }
+    if (blockIdx.x == 0)
+        for (uint64_t i = n8 + threadIdx.x; i < n; i += blockDim.x)
+            atomicAdd(&h[(in[i] >> 7) & 0xFFu], 1u);
+    __syncthreads();
+    if (h[threadIdx.x])
+        atomicAdd(reinterpret_cast<unsigned long long *>(&hist[threadIdx.x]),
+                  (unsigned long long)h[threadIdx.x]);
+}
+
+// ---- encode: per-thread code lengths -----------------------------------------
+
+// Loads this thread's up to 32 elements (zero past n) and returns their
+// bits; *bad is set when an element's exponent has no code.
+__device__ __forceinline__ uint32_t load_elems(const EncodeParams &p, const uint32_t *len_tab,
+                                               uint64_t e0, uint32_t (&w)[16], bool &bad)
+{
+    if (e0 + kElemsPerThread <= p.n) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.in + e0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = src[q];
+            w[4 * q] = v.x;
+            w[4 * q + 1] = v.y;
+            w[4 * q + 2] = v.z;
+            w[4 * q + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const uint64_t i = e0 + 2 * k;
+            const uint32_t a = i < p.n ? p.in[i] : 0u;
+            const uint32_t b = i + 1 < p.n ? p.in[i + 1] : 0u;
+            w[k] = a | (b << 16);
+        }
+    }
+    uint32_t bits = 0;
+#pragma unroll
+    for (int k = 0; k < kElemsPerThread; ++k) {
+        if (e0 + k < p.n) {
+            const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+            const uint32_t l = len_tab[(x >> 7) & 0xFFu];
+            bad |= l == 0;
+            bits += l;
+        }
+    }
+    return bits;
+}
+
+// Block-wide exclusive scan of one value per thread (256 threads).
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_tot, uint32_t &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d)
+            incl += y;
+    }
+    if (lane == 31)
+        warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t t = lane < kEncThreads / 32 ? warp_tot[lane] : 0u;
+        uint32_t ti = t;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, ti, d);
+            if (lane >= d)
+                ti += y;
+        }
+        if (lane < kEncThreads / 32)
+            warp_tot[lane] = ti - t;
+        if (lane == 31)
+            warp_tot[kEncThreads / 32] = ti;
+    }
+    __syncthreads();
+    total = warp_tot[kEncThreads / 32];
+    return warp_tot[warp] + incl - v;
+}
+
+__global__ void __launch_bounds__(kEncThreads) segment_bits_kernel(EncodeParams p, CodeTable ct)
+{
+    __shared__ uint32_t len_tab[256];
+    __shared__ uint32_t warp_tot[kEncThreads / 32 + 1];
+    len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
+    __syncthreads();
+    const uint64_t seg = blockIdx.x;
+    const uint64_t e0 = seg * kSegElems + (uint64_t)threadIdx.x * kElemsPerThread;
+    uint32_t w[16];
+    bool bad = false;
+    const uint32_t bits = load_elems(p, len_tab, e0, w, bad);
+    uint32_t total;
+    block_exclusive_scan(bits, warp_tot, total);
+    if (threadIdx.x == 0)
+        p.seg_bits[seg] = total;
+    if (bad && p.err)
+        atomicOr(p.err, DF11_DEVERR_MISMATCH);
+}
+
+// Exclusive scan of the segment bit counts (one CTA); checks the total.
+__global__ void __launch_bounds__(kScanThreads) segment_scan_kernel(EncodeParams p)
+{
+    __shared__ unsigned long long warp_tot[kScanThreads / 32];
+    __shared__ unsigned long long carry;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0)
+        carry = 0;
+    __syncthreads();
+    for (uint64_t base = 0; base < p.n_seg; base += kScanThreads) {
+        const uint64_t i = base + threadIdx.x;
+        const unsigned long long v = i < p.n_seg ? p.seg_bits[i] : 0ull;
+        unsigned long long incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d)
+                incl += y;
+        }
+        if (lane == 31)
+            warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const unsigned long long t = warp_tot[lane];
+            unsigned long long ti = t;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, ti, d);
+                if (lane >= d)
+                    ti += y;
+            }
+            warp_tot[lane] = ti - t;
+        }
+        __syncthreads();
+        const unsigned long long c = carry;
+        if (i < p.n_seg)
+            p.seg_start[i] = c + warp_tot[warp] + incl - v;
+        __syncthreads();
+        if (threadIdx.x == kScanThreads - 1)
+            carry = c + warp_tot[warp] + incl;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0 && carry != p.total_bits && p.err)
+        atomicOr(p.err, DF11_DEVERR_MISMATCH);
+}
+
+// Zeroes the stream, gaps and sign|mantissa tail; fills chunk positions with n.
+__global__ void prepare_kernel(EncodeParams p, uint64_t stream_words, uint64_t gap_words,
+                               uint64_t n_chunks, uint64_t sm_bytes)
+{
+    const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    uint32_t *s32 = reinterpret_cast<uint32_t *>(p.stream);
+    for (uint64_t i = tid; i < stream_words; i += stride)
+        s32[i] = 0;
+    uint32_t *g32 = reinterpret_cast<uint32_t *>(p.gaps);
+    for (uint64_t i = tid; i < gap_words; i += stride)
+        g32[i] = 0;
+    for (uint64_t i = tid; i <= n_chunks; i += stride)
+        p.chunk_pos[i] = (uint32_t)p.n;
+    for (uint64_t i = p.n + tid; i < sm_bytes; i += stride)
+        p.signmant[i] = 0;
+}
+
+__device__ __forceinline__ void or_word(uint8_t *stream, uint64_t word, uint32_t v_be)
+{
+    atomicOr(reinterpret_cast<uint32_t *>(stream) + word, bswap32(v_be));
+}
+
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, CodeTable ct)
+{
+    __shared__ uint32_t code_tab[256];
+    __shared__ uint32_t len_tab[256];
+    __shared__ uint32_t warp_tot[kEncThreads / 32 + 1];
+    code_tab[threadIdx.x] = ct.e[threadIdx.x] & 0xFFFFFFu;
+    len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
+    __syncthreads();
+
+    const uint64_t seg = blockIdx.x;
+    const uint64_t e0 = seg * kSegElems + (uint64_t)threadIdx.x * kElemsPerThread;
+    uint32_t w[16];
+    bool bad = false;
+    const uint32_t bits = load_elems(p, len_tab, e0, w, bad);
+    uint32_t seg_total;
+    const uint32_t off = block_exclusive_scan(bits, warp_tot, seg_total);
+    if (e0 >= p.n)
+        return;
+    uint64_t bitpos = p.seg_start[seg] + off;
+
+    // slice of the previous code start (none for element 0)
+    uint64_t prev_slice = ~0ull;
+    if (e0 > 0) {
+        const uint32_t lp = len_tab[(p.in[e0 - 1] >> 7) & 0xFFu];
+        prev_slice = (bitpos - lp) >> p.slice_shift;
+    }
+    const uint32_t T = p.threads_per_chunk;
+
+    uint64_t word = bitpos >> 5;        // stream word being filled
+    uint64_t acc = 0;                   // pending bits, right-aligned
+    uint32_t filled = (uint32_t)(bitpos & 31);   // bits of `word` already set (earlier threads)
+    bool first_word = true;
+    const uint32_t cnt = (uint32_t)min((uint64_t)kElemsPerThread, p.n - e0);
+#pragma unroll
+    for (uint32_t k = 0; k < kElemsPerThread; ++k) {
+        if (k >= cnt)
+            break;
+        const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+        const uint32_t s = (x >> 7) & 0xFFu;
+        const uint32_t l = len_tab[s];
+        // metadata: first code of its slice
+        const uint64_t g = bitpos >> p.slice_shift;
+        if (g != prev_slice) {
+            const uint32_t gapv = (uint32_t)(bitpos - (g << p.slice_shift));
+            atomicOr(reinterpret_cast<uint32_t *>(p.gaps) + (g >> 3),
+                     (gapv & 0xFu) << (((g >> 1) & 3u) * 8 + (g & 1u) * 4));
+            if (g % T == 0)
+                p.chunk_pos[g / T] = (uint32_t)(e0 + k);
+            prev_slice = g;
+        }
+        // the code, MSB-first
+        acc = (acc << l) | code_tab[s];
+        filled += l;
+        bitpos += l;
+        if (filled >= 32) {
+            const uint32_t v = (uint32_t)(acc >> (filled - 32));
+            if (first_word)
+                or_word(p.stream, word, v);
+            else
+                reinterpret_cast<uint32_t *>(p.stream)[word] = bswap32(v);
+            first_word = false;
+            ++word;
+            filled -= 32;
+            acc &= (filled ? ((1ull << filled) - 1) : 0ull);
+        }
+    }
+    if (filled)
+        or_word(p.stream, word, (uint32_t)(acc << (32 - filled)));
+    // the end of the stream counts as a code start for the gap of its slice
+    if (e0 + cnt == p.n) {
+        const uint64_t g = bitpos >> p.slice_shift;
+        if (g < p.n_threads && g != prev_slice) {
+            const uint32_t gapv = (uint32_t)(bitpos - (g << p.slice_shift));
+            atomicOr(reinterpret_cast<uint32_t *>(p.gaps) + (g >> 3),
+                     (gapv & 0xFu) << (((g >> 1) & 3u) * 8 + (g & 1u) * 4));
+        }
+    }
+    // sign|mantissa bytes
+    if (cnt == kElemsPerThread) {
+        uint32_t sm[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const uint32_t a = w[2 * q], b = w[2 * q + 1];
+            // element bytes: (x >> 8) & 0x80 | x & 0x7F for 4 elements
+            const uint32_t lo = __byte_perm(a, b, 0x6420);   // low bytes of the 4 elements
+            const uint32_t hi = __byte_perm(a, b, 0x7531);   // high bytes
+            sm[q] = (lo & 0x7F7F7F7Fu) | (hi & 0x80808080u);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(p.signmant + e0);
+        dst[0] = make_uint4(sm[0], sm[1], sm[2], sm[3]);
+        dst[1] = make_uint4(sm[4], sm[5], sm[6], sm[7]);
+    } else {
+#pragma unroll
+        for (uint32_t k = 0; k < kElemsPerThread; ++k) {
+            if (k < cnt) {
+                const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+                p.signmant[e0 + k] = (uint8_t)(((x >> 8) & 0x80u) | (x & 0x7Fu));
+            }
+        }
+    }
+    if (bad && p.err)
+        atomicOr(p.err, DF11_DEVERR_MISMATCH);
+}
+
+bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+uint64_t n_segments(uint64_t n) { return (n + kSegElems - 1) / kSegElems; }
+
+}  // namespace
+
+extern "C" {
+
+df11_status df11_histogram_device(const uint16_t *d_in, uint64_t n, uint64_t *d_hist, void *stream)
+{
+    if (!d_in || !d_hist || n == 0 || !aligned(d_in, 16) || !aligned(d_hist, 8))
+        return DF11_ERR_INVALID_ARGUMENT;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DF11_ERR_CUDA;
+    const uint64_t want = (n + 256 * 8 - 1) / (256 * 8);
+    const uint64_t cap = (uint64_t)sms * 8;
+    const unsigned grid = (unsigned)(want < cap ? (want ? want : 1) : cap);
+    histogram_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(d_in, n, d_hist);
+    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+uint64_t df11_compress_device_scratch_bytes(uint64_t n_elements)
+{
+    const uint64_t ns = n_segments(n_elements);
+    return ns * 8 + ((ns * 4 + 15) & ~15ull);
+}
+
+df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *layout,
+                                 const uint16_t *d_in, uint64_t n, df11_device_block *out,
+                                 void *d_scratch, uint64_t scratch_bytes, uint32_t *d_error,
+                                 void *stream)
+{
+    if (!cb || !layout || !d_in || !out || !d_scratch)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if (n == 0 || n != cb->n_elements)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if (n >= (1ull << 32))
+        return DF11_ERR_OVERFLOW;
+    df11_sizes z;
+    df11_status st = df11_compress_sizes(cb, layout, &z);
+    if (st != DF11_OK)
+        return st;
+    if (scratch_bytes < df11_compress_device_scratch_bytes(n))
+        return DF11_ERR_BUFFER_TOO_SMALL;
+    if (!out->exp_stream || !out->gaps || !out->chunk_pos || !out->signmant)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if (out->exp_stream_bytes < z.exp_stream_bytes || out->gaps_bytes < z.gaps_bytes ||
+        out->chunk_pos_count < z.chunk_pos_count || out->signmant_bytes < z.signmant_bytes)
+        return DF11_ERR_BUFFER_TOO_SMALL;
+    if (!aligned(d_in, 16) || !aligned(out->exp_stream, 16) || !aligned(out->gaps, 16) ||
+        !aligned(out->chunk_pos, 16) || !aligned(out->signmant, 16) || !aligned(d_scratch, 16) ||
+        !aligned(d_error, 4))
+        return DF11_ERR_INVALID_ARGUMENT;
+
+    EncodeParams p;
+    p.in = d_in;
+    // the arrays are written through the const-qualified device view
+    p.stream = const_cast<uint8_t *>(out->exp_stream);
+    p.gaps = const_cast<uint8_t *>(out->gaps);
+    p.chunk_pos = const_cast<uint32_t *>(out->chunk_pos);
+    p.signmant = const_cast<uint8_t *>(out->signmant);
+    p.n_seg = n_segments(n);
+    p.seg_start = reinterpret_cast<uint64_t *>(d_scratch);
+    p.seg_bits = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(d_scratch) + p.n_seg * 8);
+    p.err = d_error;
+    p.n = n;
+    p.total_bits = cb->total_bits;
+    p.n_threads = z.n_threads;
+    p.slice_shift = layout->bytes_per_thread == 16 ? 7u : 6u;
+    p.threads_per_chunk = layout->threads_per_chunk;
+    CodeTable ct;
+    for (int s = 0; s < 256; ++s)
+        ct.e[s] = cb->code_len[s] ? (cb->code[s] | ((uint32_t)cb->code_len[s] << 24)) : 0u;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DF11_ERR_CUDA;
+    prepare_kernel<<<sms * 4, 256, 0, s>>>(p, z.exp_stream_bytes / 4, (z.gaps_bytes + 3) / 4,
+                                            z.n_chunks, z.signmant_bytes);
+    segment_bits_kernel<<<(unsigned)p.n_seg, kEncThreads, 0, s>>>(p, ct);
+    segment_scan_kernel<<<1, kScanThreads, 0, s>>>(p);
+    encode_kernel<<<(unsigned)p.n_seg, kEncThreads, 0, s>>>(p, ct);
+    if (cudaGetLastError() != cudaSuccess)
+        return DF11_ERR_CUDA;
+    out->hdr.max_code_len = cb->max_code_len;
+    out->hdr.threads_per_chunk = layout->threads_per_chunk;
+    out->hdr.bytes_per_thread = layout->bytes_per_thread;
+    out->hdr.n_tables = cb->n_tables;
+    out->hdr.min_code_len = DF11_MAX_CODE_LEN;
+    for (int k = 0; k < 256; ++k)
+        if (cb->code_len[k] && cb->code_len[k] < out->hdr.min_code_len)
+            out->hdr.min_code_len = cb->code_len[k];
+    out->hdr.reserved = 0;
+    out->hdr.total_bits = cb->total_bits;
+    out->hdr.n_elements = n;
+    out->hdr.n_chunks = z.n_chunks;
+    return DF11_OK;
+}
+
+}  // extern "C"

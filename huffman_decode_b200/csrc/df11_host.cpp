@@ -313,14 +313,33 @@ df11_status df11_build_codebook(const uint16_t *const *mats, const uint64_t *num
         return DF11_ERR_INVALID_ARGUMENT;
     if (v.total >= (1ull << 32))
         return DF11_ERR_OVERFLOW;
+    uint64_t h[256];
+    histogram(v, h);
+    return df11_build_codebook_from_histogram(h, max_code_len, out);
+}
+
+df11_status df11_build_codebook_from_histogram(const uint64_t hist[256], uint32_t max_code_len,
+                                               df11_codebook *out)
+{
+    if (!hist || !out)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if (max_code_len < DF11_MIN_CODE_LEN_CAP || max_code_len > DF11_MAX_CODE_LEN)
+        return DF11_ERR_INVALID_ARGUMENT;
+    uint64_t total = 0;
+    for (int s = 0; s < 256; ++s)
+        total += hist[s];
+    if (total == 0)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if (total >= (1ull << 32))
+        return DF11_ERR_OVERFLOW;
     std::memset(out, 0, sizeof(*out));
-    histogram(v, out->histogram);
+    std::memcpy(out->histogram, hist, sizeof(out->histogram));
     if (!optimal_lengths(out->histogram, max_code_len, out->code_len))
         return DF11_ERR_INVALID_ARGUMENT;
     canonical_codes(out->code_len, out->code);
     out->n_tables = build_lut(out->code_len, out->code, out->lut);
     out->max_code_len = max_code_len;
-    out->n_elements = v.total;
+    out->n_elements = total;
     for (int s = 0; s < 256; ++s) {
         if (out->code_len[s]) {
             out->n_symbols += 1;

@@ -31,6 +31,7 @@ DEVERR_COUNT = 0x1
 DEVERR_BAD_CODE = 0x2
 DEVERR_BAD_POS = 0x4
 DEVERR_TIMEOUT = 0x8
+DEVERR_MISMATCH = 0x10
 MAX_CODE_LEN = 16
 STREAM_PAD = 16
 THREADS_PER_CHUNK = 32
@@ -38,8 +39,9 @@ BYTES_PER_THREAD = 16           # 128-bit slices: fastest layout on B200
 LAYOUTS = ((32, 8), (32, 16))   # (threads_per_chunk, bytes_per_thread) this build decodes
 
 EXPORTED_SYMBOLS = (
-    "df11_build_codebook", "df11_compress_sizes", "df11_compress", "df11_validate",
-    "df11_decompress_async", "df11_status_string",
+    "df11_build_codebook", "df11_build_codebook_from_histogram", "df11_compress_sizes",
+    "df11_compress", "df11_validate", "df11_decompress_async", "df11_status_string",
+    "df11_histogram_device", "df11_compress_device_scratch_bytes", "df11_compress_device",
 )
 
 
@@ -137,6 +139,10 @@ def load_library(path: str | None = None):
         ("df11_validate", S, [P]),
         ("df11_decompress_async", S, [P, P, U64, P, P]),
         ("df11_status_string", ctypes.c_char_p, [S]),
+        ("df11_build_codebook_from_histogram", S, [P, U32, P]),
+        ("df11_histogram_device", S, [P, U64, P, P]),
+        ("df11_compress_device_scratch_bytes", U64, [U64]),
+        ("df11_compress_device", S, [P, P, P, U64, P, P, U64, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -310,3 +316,71 @@ def decompress_async(db: DeviceBlock, out, error=None, stream=None, c_block=None
     cap = out.numel() if capacity is None else min(int(capacity), out.numel())
     _check(load_library().df11_decompress_async(ctypes.byref(blk), out.data_ptr(), cap,
                                                 err_ptr, handle), "df11_decompress_async")
+
+
+# ------------------------------------------------------- GPU-side compressor
+
+def _stream_handle(stream, device):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def build_codebook_from_histogram(hist, max_code_len: int = MAX_CODE_LEN) -> Codebook:
+    """df11_build_codebook_from_histogram (host) from 256 exponent counts."""
+    h = np.ascontiguousarray(np.asarray(hist).reshape(-1)[:256], dtype=np.uint64)
+    if h.size != 256:
+        raise ValueError("histogram needs 256 bins")
+    cb = Codebook()
+    _check(load_library().df11_build_codebook_from_histogram(h.ctypes.data, max_code_len,
+                                                              ctypes.byref(cb)),
+           "df11_build_codebook_from_histogram")
+    return cb
+
+
+def histogram_device(d_in, stream=None):
+    """df11_histogram_device: exponent histogram of a contiguous CUDA tensor of
+    16-bit elements; returns an int64 CUDA tensor of 256 counts."""
+    import torch
+    if d_in.element_size() != 2 or not d_in.is_cuda or not d_in.is_contiguous():
+        raise ValueError("d_in must be a contiguous CUDA tensor of 16-bit elements")
+    hist = torch.zeros(256, dtype=torch.int64, device=d_in.device)
+    _check(load_library().df11_histogram_device(d_in.data_ptr(), d_in.numel(), hist.data_ptr(),
+                                                _stream_handle(stream, d_in.device)),
+           "df11_histogram_device")
+    return hist
+
+
+def compress_device_scratch_bytes(n_elements: int) -> int:
+    return int(load_library().df11_compress_device_scratch_bytes(n_elements))
+
+
+def compress_device(cb: Codebook, d_in, threads_per_chunk: int = THREADS_PER_CHUNK,
+                    bytes_per_thread: int = BYTES_PER_THREAD, stream=None, error=None,
+                    scratch=None) -> DeviceBlock:
+    """df11_compress_device: encodes a contiguous CUDA tensor of BF16 bit
+    patterns (the block's matrices concatenated) into freshly allocated device
+    arrays; the codebook's tables are copied into the block's lut array."""
+    import torch
+    if d_in.element_size() != 2 or not d_in.is_cuda or not d_in.is_contiguous():
+        raise ValueError("d_in must be a contiguous CUDA tensor of 16-bit elements")
+    dev = d_in.device
+    z = compress_sizes(cb, threads_per_chunk, bytes_per_thread)
+    sizes = {"exp_stream": z.exp_stream_bytes, "gaps": z.gaps_bytes,
+             "chunk_pos": z.chunk_pos_count * 4, "signmant": z.signmant_bytes,
+             "lut": z.lut_entries * 2}
+    t = {name: torch.empty(nbytes, dtype=torch.uint8, device=dev) for name, nbytes in sizes.items()}
+    t["lut"].copy_(torch.from_numpy(cb.tables().view(np.uint8)))
+    if scratch is None:
+        scratch = torch.empty(max(compress_device_scratch_bytes(d_in.numel()), 16),
+                              dtype=torch.uint8, device=dev)
+    db = DeviceBlock(header=Header(), tensors=t, sizes=sizes, matrix_numel=[d_in.numel()])
+    blk = db.c_struct()
+    ly = Layout(threads_per_chunk, bytes_per_thread)
+    _check(load_library().df11_compress_device(
+        ctypes.byref(cb), ctypes.byref(ly), d_in.data_ptr(), d_in.numel(), ctypes.byref(blk),
+        scratch.data_ptr(), scratch.numel(), error.data_ptr() if error is not None else None,
+        _stream_handle(stream, dev)), "df11_compress_device")
+    db.header = blk.hdr
+    return db

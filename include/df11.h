@@ -80,6 +80,8 @@ typedef enum {
                                      out_capacity; that chunk writes nothing   */
 #define DF11_DEVERR_TIMEOUT 0x8u  /* a bounded wait for a staged copy ran out;
                                      that chunk's output is not trustworthy    */
+#define DF11_DEVERR_MISMATCH 0x10u /* GPU compressor: an exponent without a code,
+                                     or a bit total other than the codebook's  */
 
 #define DF11_MAX_CODE_LEN 16u     /* longest code the format allows           */
 #define DF11_MIN_CODE_LEN_CAP 8u  /* smallest cap accepted by build_codebook  */
@@ -170,6 +172,13 @@ df11_status df11_build_codebook(const uint16_t *const *mats, const uint64_t *num
                                 uint32_t n_mats, uint32_t max_code_len,
                                 df11_codebook *out);
 
+/* Host.  The codebook for a given 256-bin exponent histogram (for example
+ * one df11_histogram_device computed): the same lengths, codes and tables
+ * df11_build_codebook would build from the data.  Errors as for
+ * df11_build_codebook. */
+df11_status df11_build_codebook_from_histogram(const uint64_t histogram[256], uint32_t max_code_len,
+                                               df11_codebook *out);
+
 /* Host.  Sizes of every array df11_compress fills for this codebook and
  * layout, from the histogram alone (no pass over the data).
  * Errors: INVALID_ARGUMENT for an unsupported layout or an empty codebook. */
@@ -207,6 +216,39 @@ df11_status df11_validate(const df11_host_block *blk);
 df11_status df11_decompress_async(const df11_device_block *blk, uint16_t *out_bf16,
                                   uint64_t out_capacity, uint32_t *d_error,
                                   void *stream);
+
+/* ---- GPU-side compressor --------------------------------------------------
+ * The pages compress on the CPU only ("DFloat11: lossless BFloat16
+ * compression", "How to develop with it": minutes per block on one thread).
+ * These calls do the same on the GPU for a block already in device memory,
+ * producing exactly the arrays df11_compress produces for the same codebook.
+ */
+
+/* GPU.  Adds the exponent histogram of d_in[0 .. n) (device, BF16 bit
+ * patterns, 16-byte aligned) into d_hist (device uint64[256], 8-byte
+ * aligned; the caller zeroes it).  One launch on `stream`.  Errors:
+ * INVALID_ARGUMENT for null/misaligned pointers or n == 0, CUDA. */
+df11_status df11_histogram_device(const uint16_t *d_in, uint64_t n, uint64_t *d_hist, void *stream);
+
+/* Scratch bytes df11_compress_device needs for n elements (12 bytes per
+ * 8192 elements, rounded up). */
+uint64_t df11_compress_device_scratch_bytes(uint64_t n_elements);
+
+/* GPU.  Encodes d_in[0 .. n) (device, the block's matrices concatenated,
+ * 16-byte aligned) with the codebook cb (host) into the device arrays of
+ * `out` (exp_stream, gaps, chunk_pos, signmant; sized by
+ * df11_compress_sizes, 16-byte aligned) and fills out->hdr.  out->lut is not
+ * touched: the caller copies cb->lut (n_tables * 256 entries) into it.
+ * d_scratch (device, 16-byte aligned, >= df11_compress_device_scratch_bytes)
+ * is caller-owned work space.  Four kernel launches on `stream`; nothing is
+ * allocated and nothing synchronises.  Data that disagree with the codebook
+ * (an exponent without a code, another bit total) OR DF11_DEVERR_MISMATCH
+ * into *d_error (device, may be NULL).  Errors: INVALID_ARGUMENT (pointers,
+ * alignment, n != cb->n_elements, layout), BUFFER_TOO_SMALL, OVERFLOW, CUDA. */
+df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *layout,
+                                 const uint16_t *d_in, uint64_t n, df11_device_block *out,
+                                 void *d_scratch, uint64_t scratch_bytes, uint32_t *d_error,
+                                 void *stream);
 
 /* Human-readable name of a status code (static string). */
 const char *df11_status_string(df11_status s);

@@ -23,7 +23,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def _declared_functions():
     src = open(os.path.join(ROOT, "include", "df11.h")).read()
-    return sorted(set(re.findall(r"^(?:df11_status|const char \*)\s*(df11_\w+)\s*\(", src, re.M)))
+    return sorted(set(re.findall(r"^(?:df11_status|const char \*|uint64_t)\s*(df11_\w+)\s*\(", src, re.M)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -304,3 +304,63 @@ def test_decompress_rejects_bad_arguments_before_any_cuda_call():
         h = binding.Header.from_buffer_copy(hb.header)
         h.min_code_len = bad_min
         assert call(dev_block(hdr=h)) == 1
+
+
+# ------------------------------------------- codebook from a histogram
+
+@pytest.mark.parametrize("name", ["single_1024x1024", "heavy_tail_512", "uniform_bits_512",
+                                  "single_exponent_512"])
+def test_codebook_from_histogram_equals_data_pass(name):
+    """The histogram entry point (used with the GPU histogram) builds exactly
+    the codebook the data pass builds."""
+    mats = [m for _, m in SMALL_WORKLOADS[name]()]
+    a = df11.build_codebook(mats)
+    counts = oracle.histogram(oracle.split(_flat(mats))[0])
+    b = df11.build_codebook_from_histogram(counts)
+    assert bytes(a) == bytes(b)
+
+
+def test_codebook_from_histogram_errors():
+    with pytest.raises(df11.DF11Error):
+        df11.build_codebook_from_histogram(np.zeros(256, np.uint64))
+    h = np.zeros(256, np.uint64); h[3] = 5
+    with pytest.raises(df11.DF11Error):
+        df11.build_codebook_from_histogram(h, 7)
+    h[4] = 1 << 32
+    with pytest.raises(df11.DF11Error) as ei:
+        df11.build_codebook_from_histogram(h)
+    assert ei.value.status == 3
+
+
+def test_compress_device_rejects_bad_arguments_before_any_cuda_call():
+    mats = [m for _, m in workloads.llama_block(1002, scale_div=256)]
+    cb = df11.build_codebook(mats)
+    lib = df11.load_library()
+    n = int(cb.n_elements)
+    ly = binding.Layout(32, 16)
+    z = df11.compress_sizes(cb)
+    fake = 1 << 20
+    b = binding._Block()
+    for name in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut"):
+        setattr(b, name, fake)
+    b.exp_stream_bytes, b.gaps_bytes = z.exp_stream_bytes, z.gaps_bytes
+    b.chunk_pos_count, b.signmant_bytes, b.lut_entries = z.chunk_pos_count, z.signmant_bytes, z.lut_entries
+    scratch = df11.compress_device_scratch_bytes(n)
+    assert scratch >= 12 * ((n + 8191) // 8192)
+    call = lambda **kw: lib.df11_compress_device(
+        ctypes.byref(cb), ctypes.byref(kw.get("ly", ly)), kw.get("inp", fake), kw.get("n", n),
+        ctypes.byref(kw.get("blk", b)), kw.get("scr", fake), kw.get("scrn", scratch),
+        kw.get("err", None), None)
+    assert call(inp=None) == 1
+    assert call(n=n + 1) == 1
+    assert call(scr=None) == 1
+    assert call(scrn=scratch - 1) == 2
+    assert call(inp=fake + 2) == 1
+    assert call(err=fake + 2) == 1
+    assert call(ly=binding.Layout(32, 4)) == 1
+    short = binding._Block.from_buffer_copy(b)
+    short.gaps_bytes -= 1
+    assert call(blk=short) == 2
+    assert lib.df11_histogram_device(None, n, fake, None) == 1
+    assert lib.df11_histogram_device(fake, 0, fake, None) == 1
+    assert lib.df11_histogram_device(fake + 2, n, fake, None) == 1
