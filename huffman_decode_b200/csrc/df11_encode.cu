@@ -22,6 +22,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -451,3 +452,54 @@ df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *lay
 }
 
 }  // extern "C"
+
+// ---- allocation-free variant -------------------------------------------------
+// Some callers cannot let a library allocate device memory: a serving runtime
+// or framework that reserves the whole GPU for its own memory pool up front
+// (cudaMalloc then fails, or bypasses the pool's accounting), or code that
+// must not call cudaFree, which synchronises the device.  For them,
+// df11_compress_device_noalloc takes its work space from the fixed array
+// below instead of from the caller.
+
+namespace {
+
+constexpr uint64_t kNoAllocScratchBytes = DF11_NOALLOC_SCRATCH_BYTES;
+constexpr int kNoAllocMaxDevices = 64;
+
+// Segment bit counts and starts of the last call.  Every call writes all the
+// entries it reads before reading them, so nothing needs clearing.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, per device (0 = not looked up yet).
+std::atomic<uintptr_t> g_noalloc_addr[kNoAllocMaxDevices];
+
+}  // namespace
+
+extern "C" df11_status df11_compress_device_noalloc(const df11_codebook *cb,
+                                                    const df11_layout *layout,
+                                                    const uint16_t *d_in, uint64_t n,
+                                                    df11_device_block *out, uint32_t *d_error,
+                                                    void *stream)
+{
+    if (!cb || !layout || !d_in || !out)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if (n > DF11_NOALLOC_MAX_ELEMENTS)
+        return DF11_ERR_BUFFER_TOO_SMALL;       // the fixed work space is too small
+    if (df11_compress_device_scratch_bytes(n) > kNoAllocScratchBytes)
+        return DF11_ERR_BUFFER_TOO_SMALL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+        return DF11_ERR_CUDA;
+    uintptr_t addr = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (addr == 0) {
+        // host code only knows a stand-in for the array: ask the runtime for
+        // its address on the current device (once per device)
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+            return DF11_ERR_CUDA;
+        addr = reinterpret_cast<uintptr_t>(ptr);
+        g_noalloc_addr[dev].store(addr, std::memory_order_release);
+    }
+    return df11_compress_device(cb, layout, d_in, n, out, reinterpret_cast<void *>(addr),
+                                kNoAllocScratchBytes, d_error, stream);
+}

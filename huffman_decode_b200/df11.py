@@ -42,7 +42,10 @@ EXPORTED_SYMBOLS = (
     "df11_build_codebook", "df11_build_codebook_from_histogram", "df11_compress_sizes",
     "df11_compress", "df11_validate", "df11_decompress_async", "df11_status_string",
     "df11_histogram_device", "df11_compress_device_scratch_bytes", "df11_compress_device",
+    "df11_compress_device_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 1 << 20
+NOALLOC_MAX_ELEMENTS = 715816960
 
 
 class DF11Error(RuntimeError):
@@ -143,6 +146,7 @@ def load_library(path: str | None = None):
         ("df11_histogram_device", S, [P, U64, P, P]),
         ("df11_compress_device_scratch_bytes", U64, [U64]),
         ("df11_compress_device", S, [P, P, P, U64, P, P, U64, P, P]),
+        ("df11_compress_device_noalloc", S, [P, P, P, U64, P, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -382,5 +386,35 @@ def compress_device(cb: Codebook, d_in, threads_per_chunk: int = THREADS_PER_CHU
         ctypes.byref(cb), ctypes.byref(ly), d_in.data_ptr(), d_in.numel(), ctypes.byref(blk),
         scratch.data_ptr(), scratch.numel(), error.data_ptr() if error is not None else None,
         _stream_handle(stream, dev)), "df11_compress_device")
+    db.header = blk.hdr
+    return db
+
+
+def compress_device_noalloc(cb: Codebook, d_in, threads_per_chunk: int = THREADS_PER_CHUNK,
+                            bytes_per_thread: int = BYTES_PER_THREAD, stream=None,
+                            error=None) -> DeviceBlock:
+    """df11_compress_device_noalloc: the GPU compressor for callers that cannot
+    let a library allocate device memory (a runtime that reserves the GPU for
+    its own pool, code that must not call cudaFree).  Its work space is one
+    fixed device array inside the library, shared by every call, so calls
+    must not overlap on the GPU.  The output arrays here are still allocated
+    by this Python wrapper through torch; a C caller passes its own."""
+    import torch
+    if d_in.element_size() != 2 or not d_in.is_cuda or not d_in.is_contiguous():
+        raise ValueError("d_in must be a contiguous CUDA tensor of 16-bit elements")
+    dev = d_in.device
+    z = compress_sizes(cb, threads_per_chunk, bytes_per_thread)
+    sizes = {"exp_stream": z.exp_stream_bytes, "gaps": z.gaps_bytes,
+             "chunk_pos": z.chunk_pos_count * 4, "signmant": z.signmant_bytes,
+             "lut": z.lut_entries * 2}
+    t = {name: torch.empty(nbytes, dtype=torch.uint8, device=dev) for name, nbytes in sizes.items()}
+    t["lut"].copy_(torch.from_numpy(cb.tables().view(np.uint8)))
+    db = DeviceBlock(header=Header(), tensors=t, sizes=sizes, matrix_numel=[d_in.numel()])
+    blk = db.c_struct()
+    ly = Layout(threads_per_chunk, bytes_per_thread)
+    _check(load_library().df11_compress_device_noalloc(
+        ctypes.byref(cb), ctypes.byref(ly), d_in.data_ptr(), d_in.numel(), ctypes.byref(blk),
+        error.data_ptr() if error is not None else None, _stream_handle(stream, dev)),
+        "df11_compress_device_noalloc")
     db.header = blk.hdr
     return db

@@ -250,6 +250,31 @@ df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *lay
                                  void *d_scratch, uint64_t scratch_bytes, uint32_t *d_error,
                                  void *stream);
 
+/* ---- allocation-free compressor (no counterpart on the pages) -------------
+ * The same GPU compression as df11_compress_device, for callers that cannot
+ * let a library allocate device memory -- a serving runtime or framework that
+ * reserves the whole GPU for its own pool (cudaMalloc would fail or escape
+ * its accounting), or code that must not call cudaFree, which synchronises
+ * the device.  Instead of caller scratch it uses one fixed device array of
+ * DF11_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads
+ * it, until the process exits.
+ *   - Blocks of more than DF11_NOALLOC_MAX_ELEMENTS elements are rejected
+ *     with DF11_ERR_BUFFER_TOO_SMALL; nothing is launched.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current); make that first call
+ *     before any stream capture.  Later calls reuse the address.
+ *   - Every call shares the one array, which keeps the last call's contents;
+ *     each call writes all it reads, so nothing needs clearing.  Calls whose
+ *     work overlaps on the GPU (another stream, another host thread) race on
+ *     the array: order them on one stream or synchronise between them.
+ *   - Nothing is allocated or freed.  Arguments, outputs, error behaviour and
+ *     results are those of df11_compress_device. */
+#define DF11_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define DF11_NOALLOC_MAX_ELEMENTS 715816960ull   /* 87380 segments of 8192 */
+df11_status df11_compress_device_noalloc(const df11_codebook *cb, const df11_layout *layout,
+                                         const uint16_t *d_in, uint64_t n, df11_device_block *out,
+                                         uint32_t *d_error, void *stream);
+
 /* Human-readable name of a status code (static string). */
 const char *df11_status_string(df11_status s);
 
