@@ -53,8 +53,12 @@ def parse_args():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--bytes-per-thread", type=int, default=16, choices=[8, 16],
                     help="stream bytes each decoding thread owns (format layout)")
-    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.WORKLOADS),
-                    help="block to decode (the headline number is llama8b_block)")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=sorted(workloads.WORKLOADS) + ["llama8b_model"],
+                    help="block to decode (the headline number is llama8b_block); "
+                         "llama8b_model = 32 Llama-3.1-8B blocks, each with its own "
+                         "codebook, decoded one after another into one buffer")
+    ap.add_argument("--blocks", type=int, default=32, help="blocks of llama8b_model")
     ap.add_argument("--scale-div", type=int, default=1,
                     help="divide every row count of the block (smaller case for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=20,
@@ -399,10 +403,135 @@ def run_b200(args):
     return 0
 
 
+def run_model_stream(args):
+    """The 8B-scale stream: n_blocks Llama-3.1-8B-shaped blocks (seed 1000 +
+    block, drawn on the GPU), each histogrammed, given its own codebook and
+    compressed on the GPU, all resident in HBM; one step decodes every block
+    in turn into one reused BF16 buffer on one stream."""
+    import torch
+    import torch.distributed as dist
+
+    import huffman_decode_b200 as df11
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    stream = torch.cuda.current_stream(dev)
+    bpt = args.bytes_per_thread
+    blocks = []
+    out = None
+    cerr = torch.zeros(1, dtype=torch.int32, device=dev)
+    derr = torch.zeros(1, dtype=torch.int32, device=dev)
+    gpu_ms = []
+    host_cb_s = 0.0
+    n_weights = 0
+    for b in range(args.blocks):
+        seed = 1000 + b + rank * args.blocks
+        d_in = workloads.llama_block_device(seed, dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        hist = df11.histogram_device(d_in)
+        ev[1].record(stream)
+        t0 = time.perf_counter()
+        cb = df11.build_codebook_from_histogram(hist.cpu().numpy().astype(np.uint64))
+        host_cb_s += time.perf_counter() - t0
+        ev[2].record(stream)
+        db = df11.compress_device(cb, d_in, 32, bpt, error=cerr)
+        ev[3].record(stream)
+        if out is None:
+            out = torch.empty(d_in.numel(), dtype=torch.bfloat16, device=dev)
+        df11.decompress_async(db, out, derr, stream=stream)
+        torch.cuda.synchronize()
+        gpu_ms.append(ev[0].elapsed_time(ev[1]) + ev[2].elapsed_time(ev[3]))
+        if int(cerr.item()) or int(derr.item()) or not torch.equal(out.view(torch.int16), d_in):
+            raise RuntimeError(f"block {b}: GPU compress/decode is not bit-exact")
+        n_weights += d_in.numel()
+        del d_in, hist
+        blocks.append((db, db.c_struct(), db.compressed_bytes() + 2 * db.n_elements))
+    step_bytes = sum(x[2] for x in blocks)
+
+    def step():
+        for db, cblk, _ in blocks:
+            df11.decompress_async(db, out, derr, stream=stream, c_block=cblk)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    end.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = start.elapsed_time(end)
+    if int(derr.item()):
+        raise RuntimeError("device error word set during the timed decode")
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        bsum = torch.tensor([float(step_bytes), float(n_weights)], dtype=torch.float64, device=dev)
+        dist.all_reduce(bsum, op=dist.ReduceOp.SUM)
+        ms_max, job_bytes, job_weights = float(t[0]), float(bsum[0]), float(bsum[1])
+        dist.barrier()
+        dist.destroy_process_group()
+    else:
+        ms_max, job_bytes, job_weights = ms, float(step_bytes), float(n_weights)
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_peaks()
+    launches = args.steps * len(blocks)
+    achieved = step_bytes / (ms / args.steps * 1e-3) / 1e9
+    value = job_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    bf16_in = 2.0 * n_weights / len(blocks)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8", "data": "synthetic (GPU-drawn, torch CUDA generator)",
+        "config": {"workload": "llama8b_model", "blocks": len(blocks), "n_weights": n_weights,
+                   "threads_per_chunk": 32, "bytes_per_thread": bpt,
+                   "bytes_per_step": step_bytes, "seeds": f"1000..{999 + len(blocks)}",
+                   "l2": "inputs larger than L2, no flush",
+                   "parallelism": f"replicas x{world}, own blocks per GPU, no collective"},
+        "gweights_per_s": round(job_weights * args.steps / (ms_max * 1e-3) / 1e9, 2),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "bit_exact": True,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(n_weights // len(blocks)),
+                     "algorithmic_bytes_per_launch": step_bytes // len(blocks)},
+        "clocks": clocks,
+        "gpu_launches": launches,
+        "gpu_compress": {"ms_per_block_mean": round(statistics.mean(gpu_ms), 4),
+                         "ms_per_block_min": round(min(gpu_ms), 4),
+                         "bf16_gb_per_s": round(bf16_in / (min(gpu_ms) * 1e-3) / 1e9, 1),
+                         "host_codebook_ms_per_block": round(1e3 * host_cb_s / len(blocks), 3),
+                         "what": "device histogram + device encode per block (CUDA events); "
+                                 "codebook from the histogram on the host"},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "llama8b_model":
+        return run_model_stream(args)
     return run_b200(args)
 
 

@@ -137,6 +137,26 @@ def uniform_bits(seed: int = 4003, shape=(4096, 4096)):
     return [("uniform_bits", w.reshape(shape))]
 
 
+def llama_block_device(seed: int, device="cuda", scale_div: int = 1):
+    """The Llama-3.1-8B-shaped block drawn on the GPU with torch's CUDA
+    generator (seeded), for streams of many blocks where host generation is
+    too slow: sigma_i = uniform(0.01, 0.04) for the 7 matrices first, then
+    float32 normals; BF16 by torch's round-to-nearest-even cast.  Returns one
+    contiguous int16 tensor of BF16 bit patterns (matrices in order).  Not the
+    same numbers as llama_block(seed): a different generator."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    sig = torch.rand(len(LLAMA8B_BLOCK_SHAPES), generator=g, device=device, dtype=torch.float64)
+    sig = (0.01 + 0.03 * sig).tolist()
+    parts = []
+    for (name, (r, c)), s in zip(LLAMA8B_BLOCK_SHAPES, sig):
+        x = torch.randn(max(1, r // scale_div) * c, generator=g, device=device, dtype=torch.float32)
+        x.mul_(s)
+        parts.append(x.to(torch.bfloat16).view(torch.int16))
+    return torch.cat(parts)
+
+
 # The five workloads by name; each returns a list of (name, uint16 array).
 WORKLOADS = {
     "single_1024x1024": lambda: single_matrix(0),
