@@ -13,8 +13,11 @@
 //     with no block-wide barrier after the prologue;
 //   * single decode pass with a multi-code table: a 10-bit window indexes a
 //     1024-entry table (built in shared memory from the format's two-level
-//     16-bit tables) that yields up to three whole codes per lookup; longer
+//     16-bit tables) that yields up to four whole codes per lookup; longer
 //     codes fall back to the two-level tables;
+//   * exponents travel rotated right by one bit (bit 0 on top), which is
+//     where the BF16 halves want them: the merge is two bit-selects and two
+//     byte permutes per four weights, with no shifts;
 //   * decoded exponents are packed four per word into a per-warp slot column
 //     (row k holds word k of every lane: conflict-free stores), then moved
 //     into a contiguous, 8-element-aligned exponent buffer with funnel-shifted
@@ -41,7 +44,8 @@ namespace {
 constexpr uint32_t kLutPointer = 0x8000u;
 constexpr int kWindowBits = 10;                    // multi-code table index width
 constexpr int kMultiEntries = 1 << kWindowBits;
-constexpr int kMaxCodesPerEntry = 3;
+constexpr int kMaxCodesPerEntry = 4;
+constexpr int kEntryBytes = 8;                     // multi-code entry: symbols | step
 constexpr int kMaxWarpsPerCta = 16;
 constexpr uint32_t kWaitLimit = 1u << 22;          // bounded mbarrier polls
 
@@ -68,7 +72,7 @@ template <int W, int MINLEN>
 struct Geometry {
     static constexpr int kSliceBits = 8 * W;                         // 64 or 128
     static constexpr int kMaxCodes = (kSliceBits + MINLEN - 1) / MINLEN;  // per lane
-    static constexpr int kSlotRows = (kMaxCodes + 2 + 3) / 4;        // + codes past the end
+    static constexpr int kSlotRows = (kMaxCodes + 3 + 3) / 4;        // + codes past the end
     static constexpr int kSlotBytes = kSlotRows * 32 * 4;
     static constexpr int kEbufBytes = 32 * kMaxCodes + 16;           // multiple of 16
     static constexpr int kSbufBytes = 32 * kMaxCodes + 32;           // 16-aligned copy range
@@ -79,7 +83,7 @@ struct Geometry {
 
 // Shared memory: mbarriers | multi-code table | code lengths | per-warp areas
 // | two-level tables.
-constexpr size_t kHeadBytes = kMaxWarpsPerCta * 8 + kMultiEntries * 4 + 256;
+constexpr size_t kHeadBytes = kMaxWarpsPerCta * 8 + kMultiEntries * kEntryBytes + 256;
 
 template <int W, int MINLEN>
 constexpr size_t smem_bytes_for(int warps, uint32_t n_tables)
@@ -96,24 +100,27 @@ struct ConstInt {
     __device__ constexpr operator int() const { return V; }
 };
 
-// Four BF16 values from four exponent bytes (e) and four sign|mantissa bytes
-// (s), element k in byte k.  BF16 = sign (bit 15) | exponent (14..7) |
-// mantissa (6..0), so its low byte is (exponent bit 0) << 7 | mantissa and
-// its high byte is sign << 7 | exponent >> 1.  Both are built for all four
-// elements with one shift and one bit-select each, then interleaved.
-__device__ __forceinline__ uint2 join4(uint32_t e, uint32_t s)
+// Exponent byte rotated right by one bit: bit 0 moves to bit 7.
+__host__ __device__ __forceinline__ uint32_t rot_exp(uint32_t e) { return (e >> 1) | ((e & 1u) << 7); }
+
+// Four BF16 values from four rotated exponent bytes (r) and four
+// sign|mantissa bytes (s), element k in byte k.  BF16 = sign (bit 15) |
+// exponent (14..7) | mantissa (6..0), so its low byte is (exponent bit 0) << 7
+// | mantissa and its high byte is sign << 7 | exponent >> 1: each is one
+// bit-select of r and s under the mask 0x80, then the halves interleave.
+__device__ __forceinline__ uint2 join4(uint32_t r, uint32_t s)
 {
     uint32_t lo, hi;
-    // lo = (e << 7) where mask 0x80808080, else s
-    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(lo) : "r"(e << 7), "r"(s), "r"(0x80808080u));
-    // hi = s where mask 0x80808080, else (e >> 1)
-    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(hi) : "r"(s), "r"(e >> 1), "r"(0x80808080u));
+    // lo = r where mask 0x80808080, else s
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(lo) : "r"(r), "r"(s), "r"(0x80808080u));
+    // hi = s where mask 0x80808080, else r
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(hi) : "r"(s), "r"(r), "r"(0x80808080u));
     return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
-__device__ __forceinline__ uint16_t join1(uint32_t e, uint32_t s)
+__device__ __forceinline__ uint16_t join1(uint32_t r, uint32_t s)
 {
-    return (uint16_t)(((s & 0x80u) << 8) | (e << 7) | (s & 0x7Fu));
+    return (uint16_t)((((s & 0x80u) | (r & 0x7Fu)) << 8) | (r & 0x80u) | (s & 0x7Fu));
 }
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -126,12 +133,6 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p)
 // Table reads (read-only after the prologue) may be scheduled freely; reads
 // of data written during a chunk are ordered with "memory".
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t a)
-{
-    uint32_t v;
-    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
 __device__ __forceinline__ uint32_t lds_u16(uint32_t a)
 {
     unsigned short v;
@@ -142,6 +143,12 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t a)
 {
     uint32_t v;
     asm("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t a)
+{
+    uint2 v;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
 __device__ __forceinline__ uint32_t lds_u32_m(uint32_t a)
@@ -239,8 +246,8 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
     extern __shared__ __align__(16) uint8_t smem[];
     const int warps = blockDim.x >> 5;
     uint64_t *mbar = reinterpret_cast<uint64_t *>(smem);
-    uint32_t *multi = reinterpret_cast<uint32_t *>(smem + kMaxWarpsPerCta * 8);
-    uint8_t *len_of = smem + kMaxWarpsPerCta * 8 + kMultiEntries * 4;   // code length by exponent
+    uint2 *multi = reinterpret_cast<uint2 *>(smem + kMaxWarpsPerCta * 8);
+    uint8_t *len_of = smem + kMaxWarpsPerCta * 8 + kMultiEntries * kEntryBytes;   // by rotated exponent
     uint8_t *warp_area = smem + kHeadBytes;
     uint16_t *lut = reinterpret_cast<uint16_t *>(warp_area + (size_t)warps * G::kWarpBytes);
 
@@ -268,7 +275,7 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             if ((e & 0x4000u) || l < min_len || l > 16)
                 e = no_code;
             else
-                len_of[e & 0xFFu] = (uint8_t)l;   // every leaf of a symbol holds its length
+                len_of[rot_exp(e & 0xFFu)] = (uint8_t)l;   // every leaf of a symbol holds its length
         }
         lut[i] = (uint16_t)e;
     }
@@ -277,10 +284,11 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
     // ---- prologue: multi-code table -----------------------------------------
-    // Entry for a 10-bit window: the whole codes it starts with (at most 3),
-    // as symbols in bytes 0..2, their count in bits 24..25 and their total
-    // length in bits 28..31.  0 when the first code is longer than the window
-    // (or is no code): the decoder then takes the two-level path.
+    // Entry for a 10-bit window: x = the whole codes it starts with (at most
+    // 4), as rotated exponents in bytes 0..3 (unused bytes 0); y = the step
+    // 8 * count | total length << 8.  y = 0 when the first code is longer
+    // than the window (or is no code): the decoder then takes the two-level
+    // path.
     for (int idx = tid; idx < kMultiEntries; idx += blockDim.x) {
         const uint32_t win = (uint32_t)idx << (32 - kWindowBits);
         uint32_t t = 0, n = 0, syms = 0;
@@ -294,18 +302,18 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             const uint32_t l = (e >> 8) & 0x1Fu;
             if (t + l > (uint32_t)kWindowBits)
                 break;
-            syms |= (e & 0xFFu) << (8 * n);
+            syms |= rot_exp(e & 0xFFu) << (8 * n);
             ++n;
             t += l;
         }
-        multi[idx] = n ? (syms | (n << 24) | (t << 28)) : 0u;
+        multi[idx] = make_uint2(syms, n ? (8u * n) | (t << 8) : 0u);
     }
     __syncthreads();
 
     // shared-window addresses (bytes)
     const uint32_t smem_base = smem_addr(smem);
     const uint32_t multi_a = smem_base + kMaxWarpsPerCta * 8;
-    const uint32_t len_a = multi_a + kMultiEntries * 4;
+    const uint32_t len_a = multi_a + kMultiEntries * kEntryBytes;
     const uint32_t lut_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warps * G::kWarpBytes);
     const uint32_t slots_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warp * G::kWarpBytes);
     const uint32_t slot_lane_a = slots_a + 4u * lane;      // row 0 of this lane's column
@@ -361,55 +369,53 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             uint32_t seen = 0;
             auto decode = [&](auto end_arg) -> uint32_t {
                 const int end = end_arg;
-                int bitpos = (int)gap;
-                uint32_t nb = 0, accl = 0, acch = 0;
+                // X = bit position << 8 | fill of the slot word in bits
+                // (0..24 between lookups).  Both shifts below use the low
+                // five bits of their amount, so X feeds the word assembly
+                // directly; an entry's step adds 8 * count and length << 8.
+                uint32_t X = gap << 8;
+                uint32_t accl = 0, acch = 0;
                 uint32_t sp = slot_lane_a;           // next slot word of this lane
-                uint32_t r = 0, adv = 0;             // last entry and its length
+                uint2 r = make_uint2(0u, 0u);        // last entry
 #pragma unroll
                 for (int h = 0; h < G::kWords - 1; ++h) {
                     const uint32_t hi = w[h], lo = w[h + 1];
-                    const int lim = min(end, 32 * (h + 1));
-                    while (bitpos < lim) {
-                        const uint32_t win = __funnelshift_l(lo, hi, (uint32_t)bitpos);
-                        r = lds_u32(multi_a + ((win >> (32 - kWindowBits)) << 2));
-                        adv = r >> 28;
-                        if (r < (1u << 28)) {
+                    const uint32_t lim = (uint32_t)min(end, 32 * (h + 1)) << 8;
+                    while (X < lim) {
+                        const uint32_t win = __funnelshift_l(lo, hi, X >> 8);
+                        r = lds_v2(multi_a + ((win >> (32 - kWindowBits - 3)) & ((kMultiEntries - 1) << 3)));
+                        if (r.y == 0) {
                             // first code longer than the window: two-level tables
                             uint32_t e = lds_u16(lut_a + ((win >> 24) << 1));
                             if (e & kLutPointer)
                                 e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)) << 1));
                             seen |= e;
-                            r = (e & 0xFFu) | (1u << 24);
-                            adv = (e >> 8) & 0x1Fu;
+                            r = make_uint2(rot_exp(e & 0xFFu), 8u | (e & 0x1F00u));
                         }
-                        bitpos += (int)adv;
-                        const uint32_t n = (r >> 24) & 3u;
-                        const uint64_t sv = (uint64_t)(r & 0xFFFFFFu) << (8 * nb);
-                        accl |= (uint32_t)sv;
-                        acch |= (uint32_t)(sv >> 32);
-                        nb += n;
-                        if (nb >= 4) {
+                        accl |= __funnelshift_l(0u, r.x, X);   // r.x << fill
+                        acch = __funnelshift_l(r.x, 0u, X);    // bytes past the word
+                        X += r.y;
+                        if (X & 32u) {                        // word full
                             sts_u32(sp, accl);
                             sp += 128;
                             accl = acch;
-                            acch = 0;
-                            nb -= 4;
+                            X -= 32u;
                         }
                     }
                 }
-                if (nb)
+                const uint32_t fill = X & 0xFFu;
+                if (fill)
                     sts_u32(sp, accl);
-                uint32_t cnt = ((sp - slot_lane_a) >> 5) + nb;   // 4 codes per 128-byte row
+                uint32_t cnt = ((sp - slot_lane_a) >> 5) + (fill >> 3);   // 4 codes per 128-byte row
                 if (cnt) {
                     // codes of the last entry that start at or past `end`
-                    const uint32_t n = (r >> 24) & 3u;
-                    const int p_last = bitpos - (int)adv;
+                    const uint32_t n = (r.y & 0xFFu) >> 3;
+                    int c = (int)(X >> 8) - (int)(r.y >> 8);   // start of the entry's first code
                     uint32_t keep = 1;
-                    if (n >= 2) {
-                        const int c1 = p_last + (int)lds_u8(len_a + (r & 0xFFu));
-                        keep += c1 < end;
-                        if (n == 3)
-                            keep += c1 + (int)lds_u8(len_a + ((r >> 8) & 0xFFu)) < end;
+#pragma unroll
+                    for (uint32_t k = 1; k < (uint32_t)kMaxCodesPerEntry; ++k) {
+                        c += (int)lds_u8(len_a + ((r.x >> (8 * (k - 1))) & 0xFFu));
+                        keep += (k < n && c < end) ? 1u : 0u;
                     }
                     cnt -= n - keep;
                 }
