@@ -46,6 +46,7 @@ constexpr int kWindowBits = 10;                    // multi-code table index wid
 constexpr int kMultiEntries = 1 << kWindowBits;
 constexpr int kMaxCodesPerEntry = 4;
 constexpr int kEntryBytes = 8;                     // multi-code entry: symbols | step
+constexpr uint32_t kLongStep = 0x80000000u;        // step of an entry whose first code is long
 constexpr int kMaxWarpsPerCta = 16;
 constexpr uint32_t kWaitLimit = 1u << 22;          // bounded mbarrier polls
 
@@ -145,12 +146,6 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t a)
     asm("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
-__device__ __forceinline__ uint2 lds_v2(uint32_t a)
-{
-    uint2 v;
-    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-    return v;
-}
 __device__ __forceinline__ uint32_t lds_u32_m(uint32_t a)
 {
     uint32_t v;
@@ -173,9 +168,58 @@ __device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v)
 {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
+__device__ __forceinline__ void sts_u32_if(bool p, uint32_t a, uint32_t v)
+{
+    asm volatile("{ .reg .pred q; setp.ne.u32 q, %2, 0; @q st.shared.u32 [%0], %1; }" ::"r"(a), "r"(v),
+                 "r"((uint32_t)p)
+                 : "memory");
+}
 __device__ __forceinline__ void red_or_u32(uint32_t a, uint32_t v)
 {
     asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
+static_assert(kWindowBits == 10 && kEntryBytes == 8, "lookup_step hard-codes the index mask and scale");
+
+// Lane decode state X: bit position in bits 0..15, fill of the slot word (in
+// bits, 0..24 between lookups) in bits 16..21; kLongStep (bit 31) is added by
+// an entry whose first code is longer than the window.
+constexpr uint32_t kFillOne = 1u << 16;          // X units of one fill bit
+constexpr uint32_t kPosMask = 0xFFFFu | kLongStep;
+
+// One multi-code lookup for window `win` (the upcoming stream bits, first
+// lowest): appends the entry's symbols to the slot word at the fill, steps X,
+// computes the next window from the stream words lo:hi, and stores the word
+// (then carries the overflow) when it is full.  One predicated block, so the
+// store is not a branch; the next window is formed before the store so it
+// waits only on the step.
+__device__ __forceinline__ void lookup_step(uint32_t &X, uint32_t &win, uint32_t &accl, uint32_t &sp,
+                                            uint2 &r, uint32_t lo, uint32_t hi, uint32_t multi_a)
+{
+    asm volatile(
+        "{\n\t"
+        ".reg .b32 a, f, t, z, c;\n\t"
+        ".reg .pred p;\n\t"
+        "mov.b32 z, 0;\n\t"
+        "and.b32 a, %1, 1023;\n\t"
+        "mad.lo.u32 a, a, 8, %8;\n\t"
+        "ld.shared.v2.u32 {%4, %5}, [a];\n\t"
+        "shr.b32 f, %0, 16;\n\t"
+        "shf.l.wrap.b32 t, z, %4, f;\n\t"       // symbols << fill
+        "or.b32 %2, %2, t;\n\t"
+        "shf.l.wrap.b32 c, %4, z, f;\n\t"       // symbols past the word
+        "add.u32 %0, %0, %5;\n\t"
+        "shf.r.wrap.b32 %1, %6, %7, %0;\n\t"    // next window: (hi:lo) >> bit position
+        "and.b32 t, %0, 2097152;\n\t"           // fill >= 32
+        "setp.ne.u32 p, t, 0;\n\t"
+        "@p st.shared.u32 [%3], %2;\n\t"
+        "@p add.u32 %3, %3, 128;\n\t"
+        "@p mov.b32 %2, c;\n\t"
+        "@p sub.u32 %0, %0, 2097152;\n\t"
+        "}"
+        : "+r"(X), "+r"(win), "+r"(accl), "+r"(sp), "=r"(r.x), "=r"(r.y)
+        : "r"(lo), "r"(hi), "r"(multi_a)
+        : "memory");
 }
 
 // ---- mbarrier + bulk copy (TMA) helpers ------------------------------------
@@ -217,7 +261,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
     return false;
 }
 
-// Loads lane's stream words (big-endian, MSB-first bit order) and gap.
+// Loads the lane's stream words and gap.  Words are bit-reversed: stream bit
+// 32k + i (MSB-first in the bytes) is bit i of word k, so a right funnel
+// shift by the bit position leaves the upcoming bits, first bit lowest.
 template <int W>
 __device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, uint32_t (&w)[W / 4 + 1],
                                            uint32_t &gap)
@@ -225,16 +271,16 @@ __device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, ui
     const uint8_t *src = p.stream + (uint64_t)W * g;
     if constexpr (W == 8) {
         const uint2 a = *reinterpret_cast<const uint2 *>(src);
-        w[0] = bswap32(a.x);
-        w[1] = bswap32(a.y);
-        w[2] = bswap32(*reinterpret_cast<const uint32_t *>(src + 8));
+        w[0] = __brev(bswap32(a.x));
+        w[1] = __brev(bswap32(a.y));
+        w[2] = __brev(bswap32(*reinterpret_cast<const uint32_t *>(src + 8)));
     } else {
         const uint4 a = *reinterpret_cast<const uint4 *>(src);
-        w[0] = bswap32(a.x);
-        w[1] = bswap32(a.y);
-        w[2] = bswap32(a.z);
-        w[3] = bswap32(a.w);
-        w[4] = bswap32(*reinterpret_cast<const uint32_t *>(src + 16));
+        w[0] = __brev(bswap32(a.x));
+        w[1] = __brev(bswap32(a.y));
+        w[2] = __brev(bswap32(a.z));
+        w[3] = __brev(bswap32(a.w));
+        w[4] = __brev(bswap32(*reinterpret_cast<const uint32_t *>(src + 16)));
     }
     gap = (p.gaps[g >> 1] >> ((g & 1) * 4)) & 0xFu;
 }
@@ -284,13 +330,15 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
     // ---- prologue: multi-code table -----------------------------------------
-    // Entry for a 10-bit window: x = the whole codes it starts with (at most
-    // 4), as rotated exponents in bytes 0..3 (unused bytes 0); y = the step
-    // 8 * count | total length << 8.  y = 0 when the first code is longer
-    // than the window (or is no code): the decoder then takes the two-level
-    // path.
+    // Entry for a 10-bit window, stored at the window's bit-reversed value
+    // (first stream bit lowest, as the decoder reads it): x = the whole codes
+    // the window starts with (at most 4), as rotated exponents in bytes 0..3
+    // (unused bytes 0); y = the step total length | 8 * count << 16.  When
+    // the first code is longer than the window (or is no code) the entry is
+    // x = 0, y = kLongStep: adding it ends the lookup loop, and the decoder
+    // takes the two-level path.
     for (int idx = tid; idx < kMultiEntries; idx += blockDim.x) {
-        const uint32_t win = (uint32_t)idx << (32 - kWindowBits);
+        const uint32_t win = (uint32_t)idx << (32 - kWindowBits);   // MSB-first window
         uint32_t t = 0, n = 0, syms = 0;
         while (n < kMaxCodesPerEntry) {
             const uint32_t v = win << t;
@@ -306,7 +354,7 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             ++n;
             t += l;
         }
-        multi[idx] = make_uint2(syms, n ? (8u * n) | (t << 8) : 0u);
+        multi[__brev((uint32_t)idx) >> (32 - kWindowBits)] = make_uint2(syms, n ? t | (8u * n << 16) : kLongStep);
     }
     __syncthreads();
 
@@ -369,48 +417,50 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             uint32_t seen = 0;
             auto decode = [&](auto end_arg) -> uint32_t {
                 const int end = end_arg;
-                // X = bit position << 8 | fill of the slot word in bits
-                // (0..24 between lookups).  Both shifts below use the low
-                // five bits of their amount, so X feeds the word assembly
-                // directly; an entry's step adds 8 * count and length << 8.
-                uint32_t X = gap << 8;
-                uint32_t accl = 0, acch = 0;
+                uint32_t X = gap;
+                uint32_t accl = 0;
                 uint32_t sp = slot_lane_a;           // next slot word of this lane
                 uint2 r = make_uint2(0u, 0u);        // last entry
 #pragma unroll
                 for (int h = 0; h < G::kWords - 1; ++h) {
-                    const uint32_t hi = w[h], lo = w[h + 1];
-                    const uint32_t lim = (uint32_t)min(end, 32 * (h + 1)) << 8;
-                    while (X < lim) {
-                        const uint32_t win = __funnelshift_l(lo, hi, X >> 8);
-                        r = lds_v2(multi_a + ((win >> (32 - kWindowBits - 3)) & ((kMultiEntries - 1) << 3)));
-                        if (r.y == 0) {
-                            // first code longer than the window: two-level tables
-                            uint32_t e = lds_u16(lut_a + ((win >> 24) << 1));
-                            if (e & kLutPointer)
-                                e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((win >> 16) & 0xFFu)) << 1));
-                            seen |= e;
-                            r = make_uint2(rot_exp(e & 0xFFu), 8u | (e & 0x1F00u));
-                        }
-                        accl |= __funnelshift_l(0u, r.x, X);   // r.x << fill
-                        acch = __funnelshift_l(r.x, 0u, X);    // bytes past the word
+                    const uint32_t lo = w[h], hi = w[h + 1];
+                    const uint32_t lim = (uint32_t)min(end, 32 * (h + 1));
+                    uint32_t win = __funnelshift_r(lo, hi, X);
+                    for (;;) {
+                        while ((X & kPosMask) < lim)
+                            lookup_step(X, win, accl, sp, r, lo, hi, multi_a);
+                        if (X < kLongStep)
+                            break;
+                        // the first code is longer than the window: take it
+                        // from the two-level tables (MSB-first window)
+                        X -= kLongStep;
+                        const uint32_t wm = __brev(win);
+                        uint32_t e = lds_u16(lut_a + ((wm >> 24) << 1));
+                        if (e & kLutPointer)
+                            e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((wm >> 16) & 0xFFu)) << 1));
+                        seen |= e;
+                        r = make_uint2(rot_exp(e & 0xFFu), ((e >> 8) & 0x1Fu) | (8u * kFillOne));
+                        const uint32_t f = X >> 16;
+                        accl |= __funnelshift_l(0u, r.x, f);
+                        const uint32_t acch = __funnelshift_l(r.x, 0u, f);
                         X += r.y;
-                        if (X & 32u) {                        // word full
+                        if (X & (32u * kFillOne)) {
                             sts_u32(sp, accl);
                             sp += 128;
                             accl = acch;
-                            X -= 32u;
+                            X -= 32u * kFillOne;
                         }
+                        win = __funnelshift_r(lo, hi, X);
                     }
                 }
-                const uint32_t fill = X & 0xFFu;
+                const uint32_t fill = X >> 16;
                 if (fill)
                     sts_u32(sp, accl);
                 uint32_t cnt = ((sp - slot_lane_a) >> 5) + (fill >> 3);   // 4 codes per 128-byte row
                 if (cnt) {
                     // codes of the last entry that start at or past `end`
-                    const uint32_t n = (r.y & 0xFFu) >> 3;
-                    int c = (int)(X >> 8) - (int)(r.y >> 8);   // start of the entry's first code
+                    const uint32_t n = r.y >> 19;
+                    int c = (int)(X & 0xFFFFu) - (int)(r.y & 0xFFFFu);   // start of the entry's first code
                     uint32_t keep = 1;
 #pragma unroll
                     for (uint32_t k = 1; k < (uint32_t)kMaxCodesPerEntry; ++k) {
@@ -473,26 +523,40 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             }
             __syncwarp();
             if (nbytes) {
-                uint32_t prev = lds_u32_m(slot_lane_a);
-                uint32_t v = prev << sh;
+                // first word: slot word 0 shifted into place
+                const uint32_t v = lds_u32_m(slot_lane_a) << sh;
                 if (head_shared || (first == last && tail_shared))
                     red_or_u32(first_a, v);
                 else
                     sts_u32(first_a, v);
-                uint32_t src = slot_lane_a + 128, dst = first_a + 4;
-#pragma unroll 4
-                for (; dst < last_a; src += 128, dst += 4) {
-                    const uint32_t cur = lds_u32_m(src);
-                    sts_u32(dst, __funnelshift_l(prev, cur, sh));
-                    prev = cur;
-                }
-                if (dst == last_a) {
-                    const uint32_t cur = src < slot_lane_a + nwords * 128 ? lds_u32_m(src) : 0u;
-                    v = __funnelshift_l(prev, cur, sh);
+                // last word, when it is not the first
+                if (last > first) {
+                    const uint32_t L = last - first;
+                    const uint32_t prev = lds_u32_m(slot_lane_a + 128 * (L - 1));
+                    const uint32_t cur = L < nwords ? lds_u32_m(slot_lane_a + 128 * L) : 0u;
+                    const uint32_t t = __funnelshift_l(prev, cur, sh);
                     if (tail_shared)
-                        red_or_u32(last_a, v);
+                        red_or_u32(last_a, t);
                     else
-                        sts_u32(last_a, v);
+                        sts_u32(last_a, t);
+                }
+            }
+            {
+                // middle words first+1 .. last-1, wholly this lane's: a
+                // warp-uniform trip count, four words a step, stores
+                // predicated per lane.  Rows past a lane's last slot word
+                // are read but never stored (they lie at most two rows past
+                // the slot columns, inside the warp's exponent buffer).
+                const uint32_t m = (nbytes && last > first) ? last - first - 1 : 0u;
+                const uint32_t mmax = __reduce_max_sync(0xFFFFFFFFu, m);
+                uint32_t prev = lds_u32_m(slot_lane_a);
+                for (uint32_t k = 1; k <= mmax; k += 4) {
+#pragma unroll
+                    for (uint32_t u = 0; u < 4; ++u) {
+                        const uint32_t cur = lds_u32_m(slot_lane_a + 128 * (k + u));
+                        sts_u32_if(k + u <= m, first_a + 4 * (k + u), __funnelshift_l(prev, cur, sh));
+                        prev = cur;
+                    }
                 }
             }
             __syncwarp();
