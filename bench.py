@@ -54,11 +54,25 @@ def parse_args():
     ap.add_argument("--bytes-per-thread", type=int, default=16, choices=[8, 16],
                     help="stream bytes each decoding thread owns (format layout)")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=sorted(workloads.WORKLOADS) + ["llama8b_model"],
+                    choices=sorted(workloads.WORKLOADS) + ["llama8b_model", "llama8b_overlap",
+                                                           "llama8b_offload"],
                     help="block to decode (the headline number is llama8b_block); "
                          "llama8b_model = 32 Llama-3.1-8B blocks, each with its own "
-                         "codebook, decoded one after another into one buffer")
-    ap.add_argument("--blocks", type=int, default=32, help="blocks of llama8b_model")
+                         "codebook, decoded one after another into one buffer; "
+                         "llama8b_overlap = those blocks decoded while the previous "
+                         "block's matrix products run; llama8b_offload = blocks held "
+                         "compressed in pinned host memory, uploaded and decoded in a "
+                         "pipeline")
+    ap.add_argument("--blocks", type=int, default=None,
+                    help="blocks of the llama8b_model/overlap/offload streams "
+                         "(default 32, 8 for offload)")
+    ap.add_argument("--tokens", default="1,256,2048,8192",
+                    help="llama8b_overlap: comma-separated token counts of the activations")
+    ap.add_argument("--max-ctas", default="0,1184",
+                    help="llama8b_overlap: comma-separated decode CTA counts (0 = one resident "
+                         "wave; large = one short-lived CTA per 16 chunks)")
+    ap.add_argument("--consumer-priority", type=int, default=-1,
+                    help="llama8b_overlap: CUDA priority of the consumer stream (lower = higher)")
     ap.add_argument("--scale-div", type=int, default=1,
                     help="divide every row count of the block (smaller case for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=20,
@@ -403,6 +417,45 @@ def run_b200(args):
     return 0
 
 
+def gpu_compressed_blocks(n_blocks, seed0, dev, bpt, verify_into=None):
+    """n_blocks Llama-3.1-8B-shaped blocks drawn on the GPU (seeds seed0..),
+    each histogrammed, given its own codebook and compressed on the GPU.
+    Every block is decoded once and compared with its input (bit-exact or an
+    exception).  Returns (device blocks, per-block GPU compress ms, host
+    codebook seconds)."""
+    import torch
+
+    import huffman_decode_b200 as df11
+    stream = torch.cuda.current_stream(dev)
+    cerr = torch.zeros(1, dtype=torch.int32, device=dev)
+    derr = torch.zeros(1, dtype=torch.int32, device=dev)
+    blocks, gpu_ms, host_cb_s = [], [], 0.0
+    out = verify_into
+    for b in range(n_blocks):
+        d_in = workloads.llama_block_device(seed0 + b, dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        hist = df11.histogram_device(d_in)
+        ev[1].record(stream)
+        t0 = time.perf_counter()
+        cb = df11.build_codebook_from_histogram(hist.cpu().numpy().astype(np.uint64))
+        host_cb_s += time.perf_counter() - t0
+        ev[2].record(stream)
+        db = df11.compress_device(cb, d_in, 32, bpt, error=cerr)
+        ev[3].record(stream)
+        if out is None or out.numel() < d_in.numel():
+            out = torch.empty(d_in.numel(), dtype=torch.bfloat16, device=dev)
+        df11.decompress_async(db, out, derr, stream=stream)
+        torch.cuda.synchronize()
+        gpu_ms.append(ev[0].elapsed_time(ev[1]) + ev[2].elapsed_time(ev[3]))
+        if int(cerr.item()) or int(derr.item()) or not torch.equal(
+                out[: d_in.numel()].view(torch.int16), d_in):
+            raise RuntimeError(f"block {b}: GPU compress/decode is not bit-exact")
+        del d_in, hist
+        blocks.append(db)
+    return blocks, gpu_ms, host_cb_s
+
+
 def run_model_stream(args):
     """The 8B-scale stream: n_blocks Llama-3.1-8B-shaped blocks (seed 1000 +
     block, drawn on the GPU), each histogrammed, given its own codebook and
@@ -422,36 +475,12 @@ def run_model_stream(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     stream = torch.cuda.current_stream(dev)
     bpt = args.bytes_per_thread
-    blocks = []
-    out = None
-    cerr = torch.zeros(1, dtype=torch.int32, device=dev)
+    n_blocks = args.blocks or 32
     derr = torch.zeros(1, dtype=torch.int32, device=dev)
-    gpu_ms = []
-    host_cb_s = 0.0
-    n_weights = 0
-    for b in range(args.blocks):
-        seed = 1000 + b + rank * args.blocks
-        d_in = workloads.llama_block_device(seed, dev)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        ev[0].record(stream)
-        hist = df11.histogram_device(d_in)
-        ev[1].record(stream)
-        t0 = time.perf_counter()
-        cb = df11.build_codebook_from_histogram(hist.cpu().numpy().astype(np.uint64))
-        host_cb_s += time.perf_counter() - t0
-        ev[2].record(stream)
-        db = df11.compress_device(cb, d_in, 32, bpt, error=cerr)
-        ev[3].record(stream)
-        if out is None:
-            out = torch.empty(d_in.numel(), dtype=torch.bfloat16, device=dev)
-        df11.decompress_async(db, out, derr, stream=stream)
-        torch.cuda.synchronize()
-        gpu_ms.append(ev[0].elapsed_time(ev[1]) + ev[2].elapsed_time(ev[3]))
-        if int(cerr.item()) or int(derr.item()) or not torch.equal(out.view(torch.int16), d_in):
-            raise RuntimeError(f"block {b}: GPU compress/decode is not bit-exact")
-        n_weights += d_in.numel()
-        del d_in, hist
-        blocks.append((db, db.c_struct(), db.compressed_bytes() + 2 * db.n_elements))
+    dbs, gpu_ms, host_cb_s = gpu_compressed_blocks(n_blocks, 1000 + rank * n_blocks, dev, bpt)
+    out = torch.empty(max(db.n_elements for db in dbs), dtype=torch.bfloat16, device=dev)
+    blocks = [(db, db.c_struct(), db.compressed_bytes() + 2 * db.n_elements) for db in dbs]
+    n_weights = sum(db.n_elements for db in dbs)
     step_bytes = sum(x[2] for x in blocks)
 
     def step():
@@ -526,12 +555,253 @@ def run_model_stream(args):
     return 0
 
 
+def _events(n):
+    import torch
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def run_overlap(args):
+    """Decode overlapped with consumption (1 GPU): n blocks resident
+    compressed in HBM; the consumer runs each block's seven linear layers
+    (cuBLAS BF16 GEMMs, Y = X W^T) on activations of T tokens.  Timed on the
+    device with CUDA events:
+      decode  - every block decoded back to back;
+      gemm    - every block's products on already-decoded weights;
+      serial  - per block, decode then its products, one stream (the pages'
+                order: decode just before the block runs);
+      overlap - the pipeline: block i+1 decodes on its own stream while the
+                products of block i run, two output slots.
+    hidden = (serial - overlap) / decode: the share of decode time hidden."""
+    import torch
+
+    import huffman_decode_b200 as df11
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    n_blocks = args.blocks or 32
+    dbs, _, _ = gpu_compressed_blocks(n_blocks, 1000, dev, args.bytes_per_thread)
+    n = dbs[0].n_elements
+    shapes = [s for _, s in workloads.LLAMA8B_BLOCK_SHAPES]
+    offs = np.cumsum([0] + [r * c for r, c in shapes])
+    slots = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    cblk = [db.c_struct() for db in dbs]
+    s_dec = torch.cuda.Stream(dev)
+    s_use = torch.cuda.Stream(dev, priority=args.consumer_priority)
+    results = []
+    token_list = [int(t) for t in args.tokens.split(",") if t]
+    cap_list = [int(c) for c in args.max_ctas.split(",") if c != ""]
+    for T in token_list:
+        g = torch.Generator(device=dev)
+        g.manual_seed(T)
+        x_in = {k: torch.randn(T, k, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+                for k in (4096, 14336)}
+        y = [torch.empty(T, r, dtype=torch.bfloat16, device=dev) for r, _ in shapes]
+
+        def weights(buf):
+            return [buf[offs[i]:offs[i + 1]].view(r, c) for i, (r, c) in enumerate(shapes)]
+
+        wv = [weights(sl) for sl in slots]
+
+        def products(slot):
+            for i, (r, c) in enumerate(shapes):
+                torch.mm(x_in[c], wv[slot][i].t(), out=y[i])
+
+        def decode(i, slot, stream, max_ctas=0):
+            df11.decompress_async(dbs[i], slots[slot], err, stream=stream, c_block=cblk[i],
+                                  max_ctas=max_ctas)
+
+        def timed(fn, reps=1):
+            for _ in range(max(args.warmup, 1)):
+                fn()
+            torch.cuda.synchronize()
+            e = _events(2)
+            e[0].record(torch.cuda.current_stream(dev))
+            for _ in range(reps):
+                fn()
+            e[1].record(torch.cuda.current_stream(dev))
+            torch.cuda.synchronize()
+            return e[0].elapsed_time(e[1]) / reps
+
+        cur = torch.cuda.current_stream(dev)
+
+        def run_decode():
+            for i in range(n_blocks):
+                decode(i, 0, cur)
+
+        def run_gemm():
+            for i in range(n_blocks):
+                products(0)
+
+        def run_serial():
+            for i in range(n_blocks):
+                decode(i, i % 2, cur)
+                products(i % 2)
+
+        def run_overlap_cap(max_ctas):
+            def fn():
+                with df11.Pipeline(2) as pipe:
+                    s_dec.wait_stream(cur)
+                    s_use.wait_stream(cur)
+                    for i in range(n_blocks):
+                        slot = i % 2
+                        pipe.decode(slot, dbs[i], slots[slot], err, s_dec, max_ctas=max_ctas)
+                        pipe.acquire(slot, s_use)
+                        with torch.cuda.stream(s_use):
+                            products(slot)
+                        pipe.release(slot, s_use)
+                    cur.wait_stream(s_use)
+                    cur.wait_stream(s_dec)
+            return fn
+
+        reps = max(1, args.steps)
+        t_dec = timed(run_decode, reps)
+        t_gemm = timed(run_gemm, reps)
+        t_ser = timed(run_serial, reps)
+        ref = [t.clone() for t in y]
+        row = {"tokens": T, "decode_ms": round(t_dec, 4), "gemm_ms": round(t_gemm, 4),
+               "serial_ms": round(t_ser, 4), "overlap": []}
+        for cap in cap_list:
+            t_ov = timed(run_overlap_cap(cap), reps)
+            same = all(torch.equal(a, b) for a, b in zip(ref, y))
+            row["overlap"].append({
+                "max_ctas": cap, "overlap_ms": round(t_ov, 4),
+                "hidden_frac": round((t_ser - t_ov) / t_dec, 4),
+                "overhead_vs_bf16": round(t_ov / t_gemm, 4),
+                "outputs_equal_serial": bool(same)})
+        flops = 2.0 * T * offs[-1] * n_blocks
+        row["gemm_tflops"] = round(flops / (t_gemm * 1e-3) / 1e12, 1)
+        results.append(row)
+    if int(err.item()):
+        raise RuntimeError("device error word set")
+    best = {r["tokens"]: max(r["overlap"], key=lambda o: o["hidden_frac"]) for r in results}
+    line = {
+        "metric": "decode hidden behind the block's matrix products (fraction of decode time)",
+        "value": None, "unit": "fraction", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic (GPU-drawn weights and activations)",
+        "config": {"workload": "llama8b_overlap", "blocks": n_blocks, "n_weights_per_block": n,
+                   "bytes_per_thread": args.bytes_per_thread,
+                   "consumer_stream_priority": args.consumer_priority,
+                   "consumer": "7 cuBLAS BF16 GEMMs per block (Y = X W^T), torch.mm"},
+        "results": results,
+        "best_hidden_frac": {str(k): v["hidden_frac"] for k, v in best.items()},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_offload(args):
+    """Offload streaming (1 GPU): n blocks held compressed in pinned host
+    memory; a step uploads every block over PCIe into one of two staging
+    slots and decodes it into one of two BF16 slots (the pipeline: upload of
+    block i+1 overlaps the decode of block i).  Reported beside it, on the
+    same box: the pinned host->device copy bandwidth of the compressed arrays
+    alone, and of plain BF16 weights (offloading without DF11)."""
+    import torch
+
+    import huffman_decode_b200 as df11
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    n_blocks = args.blocks or 8
+    dbs, _, _ = gpu_compressed_blocks(n_blocks, 1000, dev, args.bytes_per_thread)
+    # the blocks move to pinned host memory; the device copies are dropped
+    hosts = []
+    for db in dbs:
+        t = {k: v.to("cpu").pin_memory() for k, v in db.tensors.items()}
+        hosts.append(df11.PinnedHostBlock(header=db.header, tensors=t, sizes=dict(db.sizes)))
+    last_n = dbs[-1].n_elements
+    last_ref = torch.empty(last_n, dtype=torch.bfloat16, device=dev)
+    df11.decompress_async(dbs[-1], last_ref)
+    torch.cuda.synchronize()
+    del dbs
+    torch.cuda.empty_cache()
+    sizes = {k: max(h.sizes[k] for h in hosts) for k in hosts[0].sizes}
+    staging = [df11.DeviceBlock.staging(sizes, dev) for _ in range(2)]
+    n_max = max(h.n_elements for h in hosts)
+    slots = [torch.empty(n_max, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    s_copy, s_dec = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cur = torch.cuda.current_stream(dev)
+    comp_bytes = sum(h.compressed_bytes() for h in hosts)
+    bf16_bytes = sum(2 * h.n_elements for h in hosts)
+
+    def step():
+        with df11.Pipeline(2) as pipe:
+            s_copy.wait_stream(cur)
+            s_dec.wait_stream(cur)
+            for i, h in enumerate(hosts):
+                slot = i % 2
+                pipe.upload(slot, h, staging[slot], s_copy)
+                pipe.decode(slot, staging[slot], slots[slot], err, s_dec)
+                pipe.acquire(slot, cur)
+                pipe.release(slot, cur)
+            cur.wait_stream(s_dec)
+
+    def copies_only():
+        for i, h in enumerate(hosts):
+            for k, t in h.tensors.items():
+                staging[i % 2].tensors[k][: t.numel()].copy_(t, non_blocking=True)
+
+    bf16_host = torch.empty(n_max, dtype=torch.int16).pin_memory()
+
+    def bf16_copies():
+        for h in hosts:
+            slots[0][: h.n_elements].view(torch.int16).copy_(bf16_host[: h.n_elements],
+                                                             non_blocking=True)
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 1)):
+            fn()
+        torch.cuda.synchronize()
+        e = _events(2)
+        e[0].record(cur)
+        for _ in range(args.steps):
+            fn()
+        e[1].record(cur)
+        torch.cuda.synchronize()
+        return e[0].elapsed_time(e[1]) / args.steps
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    t_pipe = timed(step)
+    clocks = sampler.stop()
+    ok = int(err.item()) == 0 and torch.equal(slots[(n_blocks - 1) % 2][:last_n], last_ref)
+    t_copy = timed(copies_only)
+    t_bf16 = timed(bf16_copies)
+    h2d = comp_bytes / (t_copy * 1e-3) / 1e9
+    line = {
+        "metric": "offload stream: BF16 weights delivered per second (pinned host DF11 -> GPU BF16)",
+        "value": round(bf16_bytes / (t_pipe * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t_pipe, 4), "higher_is_better": True, "dtype": "u8",
+        "data": "synthetic (GPU-drawn, GPU-compressed, then pinned host)",
+        "config": {"workload": "llama8b_offload", "blocks": n_blocks,
+                   "bytes_per_thread": args.bytes_per_thread, "slots": 2,
+                   "compressed_bytes_per_step": comp_bytes, "bf16_bytes_per_step": bf16_bytes},
+        "compressed_h2d_gbs_in_pipeline": round(comp_bytes / (t_pipe * 1e-3) / 1e9, 2),
+        "h2d_copy_only": {"ms": round(t_copy, 4), "gbs": round(h2d, 2)},
+        "pcie_frac": round((comp_bytes / (t_pipe * 1e-3) / 1e9) / h2d, 4),
+        "bf16_offload": {"ms": round(t_bf16, 4),
+                         "gbs": round(bf16_bytes / (t_bf16 * 1e-3) / 1e9, 2)},
+        "speedup_vs_bf16_offload": round(t_bf16 / t_pipe, 3),
+        "bit_exact_last_block": bool(ok),
+        "clocks": clocks,
+        "gpu_launches": n_blocks * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0 if ok else 1
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "llama8b_model":
         return run_model_stream(args)
+    if args.workload == "llama8b_overlap":
+        return run_overlap(args)
+    if args.workload == "llama8b_offload":
+        return run_offload(args)
     return run_b200(args)
 
 

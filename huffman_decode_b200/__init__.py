@@ -7,7 +7,7 @@ happens in libdf11.so (C ABI in include/df11.h); this package only binds it.
 """
 from .df11 import (  # noqa: F401
     DEVERR_BAD_CODE, DEVERR_BAD_POS, DEVERR_COUNT, DEVERR_MISMATCH, DEVERR_TIMEOUT, DF11Error,
-    DeviceBlock, EXPORTED_SYMBOLS, LAYOUTS, HostBlock, build_codebook,
+    DeviceBlock, EXPORTED_SYMBOLS, LAYOUTS, HostBlock, PinnedHostBlock, Pipeline, build_codebook,
     build_codebook_from_histogram, compress, compress_device, compress_device_noalloc,
     compress_device_scratch_bytes,
     compress_sizes, decompress_async, histogram_device, library_path, load_library, validate,

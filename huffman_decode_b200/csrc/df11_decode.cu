@@ -630,7 +630,7 @@ std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_attr_done[kMaxDevices][4];
 
 template <int W, int MINLEN>
-df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream)
+df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32_t max_ctas)
 {
     constexpr int v = (W == 8 ? 0 : 2) + (MINLEN == 1 ? 0 : 1);
     auto kernel = df11_decode_kernel<W, MINLEN>;
@@ -662,8 +662,12 @@ df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream)
     }
     const uint64_t ctas_needed = (prm.n_chunks + warps - 1) / warps;
     const uint64_t resident = (uint64_t)occ * (uint64_t)sms;
-    const unsigned grid = (unsigned)(ctas_needed < resident ? ctas_needed : resident);
-    kernel<<<grid, warps * 32, smem, stream>>>(prm);
+    // default: one wave of resident CTAs, each looping over chunks; a given
+    // count may be smaller (SMs left to other streams) or larger (waves of
+    // short-lived CTAs that free their SM as each one finishes)
+    const uint64_t want = max_ctas ? (uint64_t)max_ctas : resident;
+    const uint64_t grid = ctas_needed < want ? ctas_needed : want;
+    kernel<<<(unsigned)grid, warps * 32, smem, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
@@ -674,6 +678,13 @@ bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>
 extern "C" df11_status df11_decompress_async(const df11_device_block *blk, uint16_t *out_bf16,
                                              uint64_t out_capacity, uint32_t *d_error,
                                              void *stream)
+{
+    return df11_decompress_async_ctas(blk, out_bf16, out_capacity, d_error, 0, stream);
+}
+
+extern "C" df11_status df11_decompress_async_ctas(const df11_device_block *blk, uint16_t *out_bf16,
+                                                  uint64_t out_capacity, uint32_t *d_error,
+                                                  uint32_t max_ctas, void *stream)
 {
     if (!blk || !out_bf16)
         return DF11_ERR_INVALID_ARGUMENT;
@@ -721,6 +732,6 @@ extern "C" df11_status df11_decompress_async(const df11_device_block *blk, uint1
     prm.full_chunks = (uint32_t)(h.total_bits / chunk_bits);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (W == 8)
-        return h.min_code_len >= 2 ? launch<8, 2>(prm, dev, s) : launch<8, 1>(prm, dev, s);
-    return h.min_code_len >= 2 ? launch<16, 2>(prm, dev, s) : launch<16, 1>(prm, dev, s);
+        return h.min_code_len >= 2 ? launch<8, 2>(prm, dev, s, max_ctas) : launch<8, 1>(prm, dev, s, max_ctas);
+    return h.min_code_len >= 2 ? launch<16, 2>(prm, dev, s, max_ctas) : launch<16, 1>(prm, dev, s, max_ctas);
 }

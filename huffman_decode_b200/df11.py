@@ -42,7 +42,9 @@ EXPORTED_SYMBOLS = (
     "df11_build_codebook", "df11_build_codebook_from_histogram", "df11_compress_sizes",
     "df11_compress", "df11_validate", "df11_decompress_async", "df11_status_string",
     "df11_histogram_device", "df11_compress_device_scratch_bytes", "df11_compress_device",
-    "df11_compress_device_noalloc",
+    "df11_compress_device_noalloc", "df11_decompress_async_ctas", "df11_pipeline_create",
+    "df11_pipeline_destroy", "df11_pipeline_upload", "df11_pipeline_decode", "df11_pipeline_acquire",
+    "df11_pipeline_release",
 )
 NOALLOC_SCRATCH_BYTES = 1 << 20
 NOALLOC_MAX_ELEMENTS = 715816960
@@ -147,6 +149,13 @@ def load_library(path: str | None = None):
         ("df11_compress_device_scratch_bytes", U64, [U64]),
         ("df11_compress_device", S, [P, P, P, U64, P, P, U64, P, P]),
         ("df11_compress_device_noalloc", S, [P, P, P, U64, P, P, P]),
+        ("df11_decompress_async_ctas", S, [P, P, U64, P, U32, P]),
+        ("df11_pipeline_create", S, [U32, P]),
+        ("df11_pipeline_destroy", S, [P]),
+        ("df11_pipeline_upload", S, [P, U32, P, P, P]),
+        ("df11_pipeline_decode", S, [P, U32, P, P, U64, P, U32, P]),
+        ("df11_pipeline_acquire", S, [P, U32, P]),
+        ("df11_pipeline_release", S, [P, U32, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -228,6 +237,16 @@ class HostBlock:
     def arrays(self):
         return {n: getattr(self, n) for n in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")}
 
+    def pinned(self) -> "PinnedHostBlock":
+        """A copy of the block in page-locked host memory (torch pinned
+        tensors), so host -> device copies of it run asynchronously."""
+        import torch
+        t = {n: torch.from_numpy(a.view(np.uint8).reshape(-1)).pin_memory()
+             for n, a in self.arrays().items()}
+        return PinnedHostBlock(header=self.header, tensors=t,
+                               sizes={n: a.nbytes for n, a in self.arrays().items()},
+                               matrix_numel=list(self.matrix_numel))
+
     def to_device(self, device="cuda", pin: bool = False) -> "DeviceBlock":
         import torch
         t = {}
@@ -239,6 +258,38 @@ class HostBlock:
         return DeviceBlock(header=self.header, tensors=t,
                            sizes={n: a.nbytes for n, a in self.arrays().items()},
                            matrix_numel=list(self.matrix_numel))
+
+
+def _struct_from_tensors(header, tensors, sizes) -> _Block:
+    b = _Block()
+    b.hdr = header
+    for name, t in tensors.items():
+        setattr(b, name, t.data_ptr())
+    b.exp_stream_bytes = sizes["exp_stream"]
+    b.gaps_bytes = sizes["gaps"]
+    b.chunk_pos_count = sizes["chunk_pos"] // 4
+    b.signmant_bytes = sizes["signmant"]
+    b.lut_entries = sizes["lut"] // 2
+    return b
+
+
+@dataclass
+class PinnedHostBlock:
+    """A compressed block whose arrays are pinned host (uint8) tensors."""
+    header: Header
+    tensors: dict
+    sizes: dict
+    matrix_numel: list = field(default_factory=list)
+
+    def c_struct(self) -> _Block:
+        return _struct_from_tensors(self.header, self.tensors, self.sizes)
+
+    @property
+    def n_elements(self) -> int:
+        return int(self.header.n_elements)
+
+    def compressed_bytes(self) -> int:
+        return int(sum(self.sizes.values()))
 
 
 def compress(cb: Codebook, mats, threads_per_chunk: int = THREADS_PER_CHUNK,
@@ -280,16 +331,7 @@ class DeviceBlock:
     matrix_numel: list = field(default_factory=list)
 
     def c_struct(self) -> _Block:
-        b = _Block()
-        b.hdr = self.header
-        for name, t in self.tensors.items():
-            setattr(b, name, t.data_ptr())
-        b.exp_stream_bytes = self.sizes["exp_stream"]
-        b.gaps_bytes = self.sizes["gaps"]
-        b.chunk_pos_count = self.sizes["chunk_pos"] // 4
-        b.signmant_bytes = self.sizes["signmant"]
-        b.lut_entries = self.sizes["lut"] // 2
-        return b
+        return _struct_from_tensors(self.header, self.tensors, self.sizes)
 
     @property
     def n_elements(self) -> int:
@@ -298,14 +340,24 @@ class DeviceBlock:
     def compressed_bytes(self) -> int:
         return int(sum(self.sizes.values()))
 
+    @staticmethod
+    def staging(sizes: dict, device="cuda") -> "DeviceBlock":
+        """Empty device arrays of the given byte sizes (a pipeline slot's
+        staging area); the header is filled by the upload that uses it."""
+        import torch
+        t = {n: torch.empty(max(int(b), 16), dtype=torch.uint8, device=device)
+             for n, b in sizes.items()}
+        return DeviceBlock(header=Header(), tensors=t, sizes={n: int(b) for n, b in sizes.items()})
+
 
 def decompress_async(db: DeviceBlock, out, error=None, stream=None, c_block=None,
-                     capacity: int | None = None) -> None:
+                     capacity: int | None = None, max_ctas: int = 0) -> None:
     """df11_decompress_async: one kernel launch decoding the whole block into
     `out` (a CUDA tensor of >= n_elements 16-bit elements, e.g. bfloat16 or
     int16) on `stream` (torch.cuda.Stream, raw handle, or the current stream).
     `error` is an optional int32 CUDA tensor the kernel ORs error bits into;
-    `capacity` (default out.numel()) is the element count the kernel may write."""
+    `capacity` (default out.numel()) is the element count the kernel may write;
+    `max_ctas` > 0 caps the launch (df11_decompress_async_ctas)."""
     import torch
     if stream is None:
         handle = torch.cuda.current_stream(out.device).cuda_stream
@@ -318,8 +370,13 @@ def decompress_async(db: DeviceBlock, out, error=None, stream=None, c_block=None
     blk = c_block if c_block is not None else db.c_struct()
     err_ptr = error.data_ptr() if error is not None else None
     cap = out.numel() if capacity is None else min(int(capacity), out.numel())
-    _check(load_library().df11_decompress_async(ctypes.byref(blk), out.data_ptr(), cap,
-                                                err_ptr, handle), "df11_decompress_async")
+    if max_ctas:
+        _check(load_library().df11_decompress_async_ctas(ctypes.byref(blk), out.data_ptr(), cap,
+                                                         err_ptr, int(max_ctas), handle),
+               "df11_decompress_async_ctas")
+    else:
+        _check(load_library().df11_decompress_async(ctypes.byref(blk), out.data_ptr(), cap,
+                                                    err_ptr, handle), "df11_decompress_async")
 
 
 # ------------------------------------------------------- GPU-side compressor
@@ -418,3 +475,71 @@ def compress_device_noalloc(cb: Codebook, d_in, threads_per_chunk: int = THREADS
         "df11_compress_device_noalloc")
     db.header = blk.hdr
     return db
+
+
+# ------------------------------------------------------- streamed decoding
+
+class Pipeline:
+    """df11_pipeline_*: event ordering of upload -> decode -> consume over
+    caller streams and `n_slots` slots (see include/df11.h).  The pipeline
+    owns CUDA events only; staging blocks and outputs belong to the caller."""
+
+    def __init__(self, n_slots: int = 2):
+        self._lib = load_library()
+        h = ctypes.c_void_p()
+        _check(self._lib.df11_pipeline_create(int(n_slots), ctypes.byref(h)), "df11_pipeline_create")
+        self._h = h
+        self.n_slots = int(n_slots)
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            _check(self._lib.df11_pipeline_destroy(self._h), "df11_pipeline_destroy")
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def upload(self, slot: int, src, dst: "DeviceBlock", stream) -> None:
+        """Host -> device copies of `src` (HostBlock or PinnedHostBlock) into
+        the staging block `dst`; dst takes src's header."""
+        s, d = src.c_struct(), dst.c_struct()
+        _check(self._lib.df11_pipeline_upload(self._h, int(slot), ctypes.byref(s), ctypes.byref(d),
+                                              _raw_stream(stream)), "df11_pipeline_upload")
+        dst.header = src.header
+        dst.matrix_numel = list(src.matrix_numel)
+        dst._keep = src   # the copy reads src after this call returns
+
+    def decode(self, slot: int, blk: "DeviceBlock", out, error=None, stream=None,
+               max_ctas: int = 0) -> None:
+        if out.element_size() != 2 or not out.is_cuda or not out.is_contiguous():
+            raise ValueError("out must be a contiguous CUDA tensor of 16-bit elements")
+        b = blk.c_struct()
+        err_ptr = error.data_ptr() if error is not None else None
+        _check(self._lib.df11_pipeline_decode(self._h, int(slot), ctypes.byref(b), out.data_ptr(),
+                                              out.numel(), err_ptr, int(max_ctas),
+                                              _raw_stream(stream, out.device)),
+               "df11_pipeline_decode")
+
+    def acquire(self, slot: int, stream) -> None:
+        _check(self._lib.df11_pipeline_acquire(self._h, int(slot), _raw_stream(stream)),
+               "df11_pipeline_acquire")
+
+    def release(self, slot: int, stream) -> None:
+        _check(self._lib.df11_pipeline_release(self._h, int(slot), _raw_stream(stream)),
+               "df11_pipeline_release")
+
+
+def _raw_stream(stream, device=None):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream(device).cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream

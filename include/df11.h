@@ -217,6 +217,20 @@ df11_status df11_decompress_async(const df11_device_block *blk, uint16_t *out_bf
                                   uint64_t out_capacity, uint32_t *d_error,
                                   void *stream);
 
+/* GPU.  df11_decompress_async launching max_ctas CTAs (at most one per 16
+ * chunks; 0 = one wave of resident CTAs on every SM).  Decode CTAs loop over
+ * the block's chunks, so any count decodes the whole block: fewer than a
+ * wave leave SMs to work on other streams, more than a wave run as waves of
+ * short-lived CTAs that each free their SM when done, which lets kernels of
+ * a higher-priority stream (such as the matrix products consuming the
+ * previous block) take SMs between them ("Architecture": decode runs before
+ * each block's forward pass; overlapping it with the previous block's
+ * compute is this library's addition).  Same checks and errors as
+ * df11_decompress_async. */
+df11_status df11_decompress_async_ctas(const df11_device_block *blk, uint16_t *out_bf16,
+                                       uint64_t out_capacity, uint32_t *d_error,
+                                       uint32_t max_ctas, void *stream);
+
 /* ---- GPU-side compressor --------------------------------------------------
  * The pages compress on the CPU only ("DFloat11: lossless BFloat16
  * compression", "How to develop with it": minutes per block on one thread).
@@ -276,6 +290,63 @@ df11_status df11_compress_device_noalloc(const df11_codebook *cb, const df11_lay
                                          uint32_t *d_error, void *stream);
 
 /* Human-readable name of a status code (static string). */
+/* ---- Streamed decoding: upload -> decode -> consume ----------------------
+ * The pages decode each transformer block right before its matrix products
+ * and discard the BF16 copy afterwards ("DFloat11: lossless BFloat16
+ * compression", "Architecture": block-level batching); the upstream README
+ * adds CPU offloading with one block on the GPU at a time ("DFloat11:
+ * Lossless Compression of LLMs and Diffusion Models for Efficient GPU
+ * Inference", news "Efficient CPU Offloading Now Supported!").  A pipeline
+ * orders those stages on the caller's streams so that uploading block i+1,
+ * decoding it and consuming block i overlap.
+ *
+ * A pipeline has n_slots slots; slot s pairs a caller-owned device staging
+ * block (for uploaded compressed arrays) with a caller-owned output buffer.
+ * It owns only CUDA events (three per slot), never device memory, and never
+ * blocks the host.  Ordering per slot:
+ *   upload  (copy stream)     waits until the slot's previous decode ran;
+ *   decode  (decode stream)   waits for the slot's last upload and for the
+ *                             consumer's release of the slot's output;
+ *   acquire (consumer stream) waits for the slot's last decode;
+ *   release (consumer stream) marks the slot's output free.
+ * A slot used without upload (block already in HBM) skips the first wait.
+ * Each wait refers to the event's most recent record when the call is made,
+ * so enqueue the stages in block order: a slot's next upload after its
+ * previous decode, its next decode after the consumer's release.  Calls
+ * must come from one host thread per pipeline, on the device that was
+ * current at creation (else INVALID_ARGUMENT). */
+typedef struct df11_pipeline df11_pipeline;
+
+/* Host.  Creates a pipeline of n_slots (1..64) slots.  Errors:
+ * INVALID_ARGUMENT, CUDA (no device or event creation failed). */
+df11_status df11_pipeline_create(uint32_t n_slots, df11_pipeline **out);
+
+/* Host.  Destroys the pipeline's events (work already enqueued still runs). */
+df11_status df11_pipeline_destroy(df11_pipeline *p);
+
+/* Copy stage.  Enqueues on copy_stream the host -> device copies of src's
+ * five arrays into dst's arrays (sizes from src; src should be pinned host
+ * memory for the copies to overlap with kernels).  dst->hdr is not written:
+ * the caller decodes with src->hdr.  Errors: INVALID_ARGUMENT (null
+ * pointers, slot out of range, wrong device), BUFFER_TOO_SMALL (a dst array
+ * smaller than its src, checked before anything is enqueued), CUDA. */
+df11_status df11_pipeline_upload(df11_pipeline *p, uint32_t slot, const df11_host_block *src,
+                                 const df11_device_block *dst, void *copy_stream);
+
+/* Decode stage.  Enqueues on decode_stream the slot's waits and
+ * df11_decompress_async_ctas(blk, out_bf16, out_capacity, d_error, max_ctas),
+ * then marks the slot decoded.  Errors: those of the decode call, and
+ * INVALID_ARGUMENT for a bad pipeline, slot or device. */
+df11_status df11_pipeline_decode(df11_pipeline *p, uint32_t slot, const df11_device_block *blk,
+                                 uint16_t *out_bf16, uint64_t out_capacity, uint32_t *d_error,
+                                 uint32_t max_ctas, void *decode_stream);
+
+/* Consume stage.  acquire: consumer_stream waits for the slot's last
+ * decode.  release: records that the consumer is done with the slot's
+ * output (enqueue it after the last kernel that reads it). */
+df11_status df11_pipeline_acquire(df11_pipeline *p, uint32_t slot, void *consumer_stream);
+df11_status df11_pipeline_release(df11_pipeline *p, uint32_t slot, void *consumer_stream);
+
 const char *df11_status_string(df11_status s);
 
 #ifdef __cplusplus

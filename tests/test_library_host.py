@@ -304,6 +304,27 @@ def test_decompress_rejects_bad_arguments_before_any_cuda_call():
         h = binding.Header.from_buffer_copy(hb.header)
         h.min_code_len = bad_min
         assert call(dev_block(hdr=h)) == 1
+    # the CTA-capped entry point runs the same checks
+    capped = lambda b, cap=n: lib.df11_decompress_async_ctas(ctypes.byref(b), fake, cap, None, 8, None)
+    assert lib.df11_decompress_async_ctas(None, fake, n, None, 8, None) == 1
+    assert capped(dev_block(), cap=n - 1) == 1
+    assert capped(dev_block(signmant=fake + 8)) == 1
+
+
+def test_pipeline_rejects_bad_arguments_before_any_cuda_call():
+    """df11_pipeline_*: argument checks that need no CUDA runtime."""
+    lib = df11.load_library()
+    h = ctypes.c_void_p()
+    assert lib.df11_pipeline_create(0, ctypes.byref(h)) == 1
+    assert lib.df11_pipeline_create(65, ctypes.byref(h)) == 1
+    assert lib.df11_pipeline_create(2, None) == 1
+    assert lib.df11_pipeline_destroy(None) == 1
+    fake = 1 << 20
+    b = binding._Block()
+    assert lib.df11_pipeline_upload(None, 0, ctypes.byref(b), ctypes.byref(b), None) == 1
+    assert lib.df11_pipeline_decode(None, 0, ctypes.byref(b), fake, 16, None, 0, None) == 1
+    assert lib.df11_pipeline_acquire(None, 0, None) == 1
+    assert lib.df11_pipeline_release(None, 0, None) == 1
 
 
 # ------------------------------------------- codebook from a histogram
