@@ -704,6 +704,21 @@ def run_offload(args):
     dev = torch.device("cuda", 0)
     n_blocks = args.blocks or 8
     dbs, _, _ = gpu_compressed_blocks(n_blocks, 1000, dev, args.bytes_per_thread)
+    # checksum lists (kept on the device for the verify stage) and the
+    # checksum kernel's own throughput on a resident block
+    crcs = [df11.checksum_device(db) for db in dbs]
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream(dev)
+    e = _events(2)
+    for _ in range(3):
+        df11.checksum_device(dbs[0])
+    e[0].record(cur)
+    for _ in range(20):
+        df11.checksum_device(dbs[0])
+    e[1].record(cur)
+    torch.cuda.synchronize()
+    crc_ms = e[0].elapsed_time(e[1]) / 20
+    crc_gbs = dbs[0].compressed_bytes() / (crc_ms * 1e-3) / 1e9
     # the blocks move to pinned host memory; the device copies are dropped
     hosts = []
     for db in dbs:
@@ -713,7 +728,7 @@ def run_offload(args):
     last_ref = torch.empty(last_n, dtype=torch.bfloat16, device=dev)
     df11.decompress_async(dbs[-1], last_ref)
     torch.cuda.synchronize()
-    del dbs
+    del dbs, e
     torch.cuda.empty_cache()
     sizes = {k: max(h.sizes[k] for h in hosts) for k in hosts[0].sizes}
     staging = [df11.DeviceBlock.staging(sizes, dev) for _ in range(2)]
@@ -725,17 +740,21 @@ def run_offload(args):
     comp_bytes = sum(h.compressed_bytes() for h in hosts)
     bf16_bytes = sum(2 * h.n_elements for h in hosts)
 
-    def step():
-        with df11.Pipeline(2) as pipe:
-            s_copy.wait_stream(cur)
-            s_dec.wait_stream(cur)
-            for i, h in enumerate(hosts):
-                slot = i % 2
-                pipe.upload(slot, h, staging[slot], s_copy)
-                pipe.decode(slot, staging[slot], slots[slot], err, s_dec)
-                pipe.acquire(slot, cur)
-                pipe.release(slot, cur)
-            cur.wait_stream(s_dec)
+    def make_step(verify):
+        def step():
+            with df11.Pipeline(2) as pipe:
+                s_copy.wait_stream(cur)
+                s_dec.wait_stream(cur)
+                for i, h in enumerate(hosts):
+                    slot = i % 2
+                    pipe.upload(slot, h, staging[slot], s_copy)
+                    if verify:
+                        pipe.verify(slot, staging[slot], crcs[i], err, stream=s_dec)
+                    pipe.decode(slot, staging[slot], slots[slot], err, s_dec)
+                    pipe.acquire(slot, cur)
+                    pipe.release(slot, cur)
+                cur.wait_stream(s_dec)
+        return step
 
     def copies_only():
         for i, h in enumerate(hosts):
@@ -763,9 +782,11 @@ def run_offload(args):
 
     sampler = ClockSampler(0)
     sampler.start()
-    t_pipe = timed(step)
+    t_pipe = timed(make_step(False))
     clocks = sampler.stop()
     ok = int(err.item()) == 0 and torch.equal(slots[(n_blocks - 1) % 2][:last_n], last_ref)
+    t_pipe_verify = timed(make_step(True))
+    ok = ok and int(err.item()) == 0
     t_copy = timed(copies_only)
     t_bf16 = timed(bf16_copies)
     h2d = comp_bytes / (t_copy * 1e-3) / 1e9
@@ -784,6 +805,11 @@ def run_offload(args):
         "bf16_offload": {"ms": round(t_bf16, 4),
                          "gbs": round(bf16_bytes / (t_bf16 * 1e-3) / 1e9, 2)},
         "speedup_vs_bf16_offload": round(t_bf16 / t_pipe, 3),
+        "with_checksum_verify": {"ms": round(t_pipe_verify, 4),
+                                 "overhead": round(t_pipe_verify / t_pipe - 1, 4)},
+        "checksum_kernel": {"ms_per_block": round(crc_ms, 4), "gbs": round(crc_gbs, 1),
+                            "what": "df11_checksum_device_async over one resident block's "
+                                    "compressed arrays"},
         "bit_exact_last_block": bool(ok),
         "clocks": clocks,
         "gpu_launches": n_blocks * args.steps,

@@ -6,7 +6,8 @@ and one GPU launch per block rebuilds the bit-exact BF16 matrices.  The work
 happens in libdf11.so (C ABI in include/df11.h); this package only binds it.
 """
 from .df11 import (  # noqa: F401
-    DEVERR_BAD_CODE, DEVERR_BAD_POS, DEVERR_COUNT, DEVERR_MISMATCH, DEVERR_TIMEOUT, DF11Error,
+    CRC_SEGMENT_BYTES, DEVERR_BAD_CODE, DEVERR_BAD_POS, DEVERR_CHECKSUM, DEVERR_COUNT, DEVERR_MISMATCH,
+    DEVERR_TIMEOUT, DF11Error, checksum, checksum_count, checksum_device, crc32c, verify_device,
     DeviceBlock, EXPORTED_SYMBOLS, LAYOUTS, HostBlock, PinnedHostBlock, Pipeline, build_codebook,
     build_codebook_from_histogram, compress, compress_device, compress_device_noalloc,
     compress_device_scratch_bytes,

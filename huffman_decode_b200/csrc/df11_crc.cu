@@ -1,0 +1,309 @@
+// df11_crc.cu -- CRC-32C checksums of a DF11 artifact, on the host and on
+// the GPU.
+//
+// The pages warn that one flipped bit in the exponent stream silently
+// rewrites most of a tensor and tell users to checksum DF11 artifacts on
+// download and after every copy ("DFloat11: lossless BFloat16 compression",
+// sections "How to run it in production" and "Failure modes"; the
+// corruption test in "How it works: the core algorithm").  Here the checksum
+// is a list: the CRC-32C (Castagnoli; reflected polynomial 0x82F63B78,
+// initial value and final XOR 0xFFFFFFFF) of every 4096-byte segment of the
+// block's five arrays, in the order exp_stream, gaps, chunk_pos, signmant,
+// lut (the last segment of an array is shorter).  Segments make the GPU
+// check embarrassingly parallel and locate damage.
+//
+// GPU method: one warp per segment, lane l covers bytes [128 l, 128 l + 128)
+// of it.  A lane folds its bytes four at a time (x = crc ^ word; crc = x
+// advanced over four zero bytes, which is linear in x: four 256-entry table
+// lookups), then advances its partial CRC over the bytes after its run, and
+// the warp XORs the 32 partials: CRC is linear, and crc(A || B) = crc(A)
+// advanced over |B| zero bytes, XOR crc(B).  "Advance over 2^j zero bytes"
+// is a table operator S_j (4 x 256 words) built in shared memory by
+// squaring S_{j-1}.  The initial value enters the same way: the standard CRC
+// of n bytes is the zero-initialised one XOR (0xFFFFFFFF advanced over n
+// bytes) XOR 0xFFFFFFFF.
+#include "df11.h"
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstring>
+
+namespace {
+
+constexpr uint32_t kPolyReflected = 0x82F63B78u;
+constexpr uint64_t kSeg = DF11_CRC_SEGMENT_BYTES;
+constexpr int kLaneBytes = (int)(kSeg / 32);     // 128
+constexpr int kShiftOps = 13;                    // advance by 2^0 .. 2^12 bytes
+constexpr int kCrcThreads = 256;
+constexpr size_t kCrcSmem = (256 + (size_t)kShiftOps * 1024) * 4;
+
+static_assert(kSeg == 4096, "one warp of 32 lanes x 128 bytes per segment");
+
+struct ArrayView {
+    const uint8_t *ptr[5];
+    uint64_t len[5];
+    uint64_t first[6];   // first segment index of each array; first[5] = total
+};
+
+ArrayView view_of(const uint8_t *p0, uint64_t l0, const uint8_t *p1, uint64_t l1, const uint8_t *p2,
+                  uint64_t l2, const uint8_t *p3, uint64_t l3, const uint8_t *p4, uint64_t l4)
+{
+    ArrayView v;
+    const uint8_t *ps[5] = {p0, p1, p2, p3, p4};
+    const uint64_t ls[5] = {l0, l1, l2, l3, l4};
+    v.first[0] = 0;
+    for (int a = 0; a < 5; ++a) {
+        v.ptr[a] = ps[a];
+        v.len[a] = ls[a];
+        v.first[a + 1] = v.first[a] + (ls[a] + kSeg - 1) / kSeg;
+    }
+    return v;
+}
+
+ArrayView view_of(const df11_host_block *b)
+{
+    return view_of(b->exp_stream, b->exp_stream_bytes, b->gaps, b->gaps_bytes,
+                   reinterpret_cast<const uint8_t *>(b->chunk_pos), b->chunk_pos_count * 4, b->signmant,
+                   b->signmant_bytes, reinterpret_cast<const uint8_t *>(b->lut), b->lut_entries * 2);
+}
+
+ArrayView view_of(const df11_device_block *b)
+{
+    return view_of(b->exp_stream, b->exp_stream_bytes, b->gaps, b->gaps_bytes,
+                   reinterpret_cast<const uint8_t *>(b->chunk_pos), b->chunk_pos_count * 4, b->signmant,
+                   b->signmant_bytes, reinterpret_cast<const uint8_t *>(b->lut), b->lut_entries * 2);
+}
+
+// ---- host ------------------------------------------------------------------
+
+struct ByteTable {
+    uint32_t v[256];
+    ByteTable()
+    {
+        for (uint32_t i = 0; i < 256; ++i) {
+            uint32_t c = i;
+            for (int k = 0; k < 8; ++k)
+                c = (c >> 1) ^ (kPolyReflected & (0u - (c & 1u)));
+            v[i] = c;
+        }
+    }
+};
+
+uint32_t crc_bytes_table(uint32_t c, const uint8_t *p, uint64_t n)
+{
+    static const ByteTable t;   // built once, thread-safe
+    for (uint64_t i = 0; i < n; ++i)
+        c = (c >> 8) ^ t.v[(c ^ p[i]) & 0xFFu];
+    return c;
+}
+
+#if defined(__x86_64__)
+// The SSE4.2 crc32 instruction computes exactly this CRC (Castagnoli,
+// reflected) without the initial value and final XOR.
+__attribute__((target("sse4.2"))) uint32_t crc_bytes_sse42(uint32_t c, const uint8_t *p, uint64_t n)
+{
+    uint64_t c64 = c;
+    while (n >= 8) {
+        uint64_t w;
+        std::memcpy(&w, p, 8);
+        c64 = __builtin_ia32_crc32di(c64, w);
+        p += 8;
+        n -= 8;
+    }
+    c = (uint32_t)c64;
+    while (n--)
+        c = __builtin_ia32_crc32qi(c, *p++);
+    return c;
+}
+
+bool have_sse42()
+{
+    static const bool ok = __builtin_cpu_supports("sse4.2");
+    return ok;
+}
+#endif
+
+uint32_t crc32c_host(const uint8_t *p, uint64_t n)
+{
+#if defined(__x86_64__)
+    if (have_sse42())
+        return ~crc_bytes_sse42(0xFFFFFFFFu, p, n);
+#endif
+    return ~crc_bytes_table(0xFFFFFFFFu, p, n);
+}
+
+// ---- device ----------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t advance(const uint32_t *op, uint32_t c)
+{
+    return op[c & 0xFFu] ^ op[256 + ((c >> 8) & 0xFFu)] ^ op[512 + ((c >> 16) & 0xFFu)] ^ op[768 + (c >> 24)];
+}
+
+// Advance c over m zero bytes (m < 2^kShiftOps) with the squaring operators.
+__device__ __forceinline__ uint32_t advance_by(const uint32_t *ops, uint32_t c, uint32_t m)
+{
+#pragma unroll
+    for (int j = 0; j < kShiftOps; ++j)
+        if ((m >> j) & 1u)
+            c = advance(ops + j * 1024, c);
+    return c;
+}
+
+__device__ __forceinline__ uint32_t fold_word(const uint32_t *ops, uint32_t c, uint32_t w)
+{
+    return advance(ops + 2 * 1024, c ^ w);   // four bytes = operator S_2
+}
+
+__global__ void __launch_bounds__(kCrcThreads) crc_kernel(ArrayView av, uint32_t *out, const uint32_t *expected,
+                                                          uint32_t *err, unsigned long long *first_bad)
+{
+    extern __shared__ uint32_t tab[];
+    uint32_t *t0 = tab;          // one-byte step table
+    uint32_t *ops = tab + 256;   // S_j[k][v] = (v << 8k) advanced over 2^j zero bytes
+    const int tid = threadIdx.x;
+    for (int i = tid; i < 256; i += blockDim.x) {
+        uint32_t c = (uint32_t)i;
+        for (int k = 0; k < 8; ++k)
+            c = (c >> 1) ^ (kPolyReflected & (0u - (c & 1u)));
+        t0[i] = c;
+    }
+    __syncthreads();
+    for (int i = tid; i < 1024; i += blockDim.x) {
+        const uint32_t c = (uint32_t)(i & 255) << (8 * (i >> 8));
+        ops[i] = (c >> 8) ^ t0[c & 0xFFu];
+    }
+    __syncthreads();
+    for (int j = 1; j < kShiftOps; ++j) {
+        for (int i = tid; i < 1024; i += blockDim.x)
+            ops[j * 1024 + i] = advance(ops + (j - 1) * 1024, ops[(j - 1) * 1024 + i]);
+        __syncthreads();
+    }
+
+    const int lane = tid & 31;
+    const uint64_t warps = blockDim.x >> 5;
+    const uint64_t total = av.first[5];
+    for (uint64_t seg = blockIdx.x * warps + (tid >> 5); seg < total; seg += gridDim.x * warps) {
+        int a = 0;
+        while (seg >= av.first[a + 1])
+            ++a;
+        const uint64_t local = seg - av.first[a];
+        const uint8_t *base = av.ptr[a] + local * kSeg;
+        const uint64_t rem = av.len[a] - local * kSeg;
+        const uint32_t n = (uint32_t)(rem < kSeg ? rem : kSeg);
+        const uint32_t beg = (uint32_t)(kLaneBytes * lane);
+        const uint32_t end = beg < n ? min(n, beg + (uint32_t)kLaneBytes) : beg;
+        uint32_t c = 0;
+        uint32_t q = beg;
+        for (; q + 16 <= end; q += 16) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + q));
+            c = fold_word(ops, c, v.x);
+            c = fold_word(ops, c, v.y);
+            c = fold_word(ops, c, v.z);
+            c = fold_word(ops, c, v.w);
+        }
+        for (; q < end; ++q)
+            c = (c >> 8) ^ t0[(c ^ base[q]) & 0xFFu];
+        c = advance_by(ops, c, end > beg ? n - end : 0u);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            c ^= __shfl_xor_sync(0xFFFFFFFFu, c, o);
+        if (lane == 0) {
+            const uint32_t crc = c ^ advance_by(ops, 0xFFFFFFFFu, n) ^ 0xFFFFFFFFu;
+            if (out)
+                out[seg] = crc;
+            if (expected && expected[seg] != crc) {
+                atomicOr(err, DF11_DEVERR_CHECKSUM);
+                if (first_bad)
+                    atomicMin(first_bad, (unsigned long long)seg);
+            }
+        }
+    }
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+df11_status launch_crc(const df11_device_block *blk, uint32_t *d_out, const uint32_t *d_expected,
+                       uint64_t n_crc, uint32_t *d_error, uint64_t *d_first_bad, void *stream)
+{
+    if (!blk || !blk->exp_stream || !blk->gaps || !blk->chunk_pos || !blk->signmant || !blk->lut)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if (!aligned16(blk->exp_stream) || !aligned16(blk->gaps) || !aligned16(blk->chunk_pos) ||
+        !aligned16(blk->signmant) || !aligned16(blk->lut))
+        return DF11_ERR_INVALID_ARGUMENT;
+    const ArrayView av = view_of(blk);
+    if (n_crc != av.first[5] || av.first[5] == 0)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if ((reinterpret_cast<uintptr_t>(d_out) & 3u) || (reinterpret_cast<uintptr_t>(d_expected) & 3u) ||
+        (reinterpret_cast<uintptr_t>(d_error) & 3u) || (reinterpret_cast<uintptr_t>(d_first_bad) & 7u))
+        return DF11_ERR_INVALID_ARGUMENT;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DF11_ERR_CUDA;
+    static std::atomic<int> attr_done[64];
+    if (dev < 0 || dev >= 64)
+        return DF11_ERR_CUDA;
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(crc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCrcSmem) !=
+            cudaSuccess)
+            return DF11_ERR_CUDA;
+        attr_done[dev].store(1, std::memory_order_release);
+    }
+    const uint64_t warps = kCrcThreads / 32;
+    const uint64_t need = (av.first[5] + warps - 1) / warps;
+    const uint64_t cap = 4ull * (uint64_t)sms;
+    const unsigned grid = (unsigned)(need < cap ? need : cap);
+    crc_kernel<<<grid, kCrcThreads, kCrcSmem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        av, d_out, d_expected, d_error, reinterpret_cast<unsigned long long *>(d_first_bad));
+    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" uint64_t df11_checksum_count(const df11_host_block *blk)
+{
+    if (!blk)
+        return 0;
+    return view_of(blk).first[5];
+}
+
+extern "C" df11_status df11_checksum(const df11_host_block *blk, uint32_t *crc, uint64_t n_crc)
+{
+    if (!blk || !crc || !blk->exp_stream || !blk->gaps || !blk->chunk_pos || !blk->signmant || !blk->lut)
+        return DF11_ERR_INVALID_ARGUMENT;
+    const ArrayView av = view_of(blk);
+    if (n_crc != av.first[5])
+        return DF11_ERR_INVALID_ARGUMENT;
+    for (int a = 0; a < 5; ++a)
+        for (uint64_t s = 0; s < av.first[a + 1] - av.first[a]; ++s) {
+            const uint64_t off = s * kSeg;
+            const uint64_t n = av.len[a] - off < kSeg ? av.len[a] - off : kSeg;
+            crc[av.first[a] + s] = crc32c_host(av.ptr[a] + off, n);
+        }
+    return DF11_OK;
+}
+
+extern "C" uint32_t df11_crc32c(const void *data, uint64_t n)
+{
+    if (!data && n)
+        return 0;
+    return crc32c_host(static_cast<const uint8_t *>(data), n);
+}
+
+extern "C" df11_status df11_checksum_device_async(const df11_device_block *blk, uint32_t *d_crc, uint64_t n_crc,
+                                                  void *stream)
+{
+    if (!d_crc)
+        return DF11_ERR_INVALID_ARGUMENT;
+    return launch_crc(blk, d_crc, nullptr, n_crc, nullptr, nullptr, stream);
+}
+
+extern "C" df11_status df11_verify_device_async(const df11_device_block *blk, const uint32_t *d_expected,
+                                                uint64_t n_crc, uint32_t *d_error, uint64_t *d_first_bad,
+                                                void *stream)
+{
+    if (!d_expected || !d_error)
+        return DF11_ERR_INVALID_ARGUMENT;
+    return launch_crc(blk, nullptr, d_expected, n_crc, d_error, d_first_bad, stream);
+}

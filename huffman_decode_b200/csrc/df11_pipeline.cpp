@@ -169,6 +169,20 @@ extern "C" df11_status df11_pipeline_decode(df11_pipeline *p, uint32_t slot, con
     return cudaEventRecord(p->decoded[slot], s) == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
+extern "C" df11_status df11_pipeline_verify(df11_pipeline *p, uint32_t slot, const df11_device_block *blk,
+                                            const uint32_t *d_expected, uint64_t n_crc, uint32_t *d_error,
+                                            uint64_t *d_first_bad, void *stream)
+{
+    if (!p || !blk || slot >= p->n_slots)
+        return DF11_ERR_INVALID_ARGUMENT;
+    if (!on_device(p))
+        return DF11_ERR_INVALID_ARGUMENT;
+    const cudaStream_t s = as_stream(stream);
+    if (cudaStreamWaitEvent(s, p->uploaded[slot], 0) != cudaSuccess)
+        return DF11_ERR_CUDA;
+    return df11_verify_device_async(blk, d_expected, n_crc, d_error, d_first_bad, s);
+}
+
 extern "C" df11_status df11_pipeline_acquire(df11_pipeline *p, uint32_t slot, void *consumer_stream)
 {
     if (!p || slot >= p->n_slots)

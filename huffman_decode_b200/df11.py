@@ -32,6 +32,7 @@ DEVERR_BAD_CODE = 0x2
 DEVERR_BAD_POS = 0x4
 DEVERR_TIMEOUT = 0x8
 DEVERR_MISMATCH = 0x10
+DEVERR_CHECKSUM = 0x20
 MAX_CODE_LEN = 16
 STREAM_PAD = 16
 THREADS_PER_CHUNK = 32
@@ -44,8 +45,10 @@ EXPORTED_SYMBOLS = (
     "df11_histogram_device", "df11_compress_device_scratch_bytes", "df11_compress_device",
     "df11_compress_device_noalloc", "df11_decompress_async_ctas", "df11_pipeline_create",
     "df11_pipeline_destroy", "df11_pipeline_upload", "df11_pipeline_decode", "df11_pipeline_acquire",
-    "df11_pipeline_release",
+    "df11_pipeline_release", "df11_checksum_count", "df11_crc32c", "df11_checksum",
+    "df11_checksum_device_async", "df11_verify_device_async", "df11_pipeline_verify",
 )
+CRC_SEGMENT_BYTES = 4096
 NOALLOC_SCRATCH_BYTES = 1 << 20
 NOALLOC_MAX_ELEMENTS = 715816960
 
@@ -156,6 +159,12 @@ def load_library(path: str | None = None):
         ("df11_pipeline_decode", S, [P, U32, P, P, U64, P, U32, P]),
         ("df11_pipeline_acquire", S, [P, U32, P]),
         ("df11_pipeline_release", S, [P, U32, P]),
+        ("df11_checksum_count", U64, [P]),
+        ("df11_crc32c", U32, [P, U64]),
+        ("df11_checksum", S, [P, P, U64]),
+        ("df11_checksum_device_async", S, [P, P, U64, P]),
+        ("df11_verify_device_async", S, [P, P, U64, P, P, P]),
+        ("df11_pipeline_verify", S, [P, U32, P, P, U64, P, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -511,10 +520,14 @@ class Pipeline:
     def upload(self, slot: int, src, dst: "DeviceBlock", stream) -> None:
         """Host -> device copies of `src` (HostBlock or PinnedHostBlock) into
         the staging block `dst`; dst takes src's header."""
-        s, d = src.c_struct(), dst.c_struct()
+        s = src.c_struct()
+        # the destination offers its whole capacity; afterwards it describes
+        # the uploaded block (its header and array sizes)
+        d = _struct_from_tensors(dst.header, dst.tensors, {n: t.numel() for n, t in dst.tensors.items()})
         _check(self._lib.df11_pipeline_upload(self._h, int(slot), ctypes.byref(s), ctypes.byref(d),
                                               _raw_stream(stream)), "df11_pipeline_upload")
         dst.header = src.header
+        dst.sizes = dict(src.sizes)
         dst.matrix_numel = list(src.matrix_numel)
         dst._keep = src   # the copy reads src after this call returns
 
@@ -533,6 +546,16 @@ class Pipeline:
         _check(self._lib.df11_pipeline_acquire(self._h, int(slot), _raw_stream(stream)),
                "df11_pipeline_acquire")
 
+    def verify(self, slot: int, blk: "DeviceBlock", expected, error, first_bad=None,
+               stream=None) -> None:
+        """Checksum check of the slot's staging block after its upload, on
+        `stream` (put it on the decode stream before decode)."""
+        b = blk.c_struct()
+        fb = first_bad.data_ptr() if first_bad is not None else None
+        _check(self._lib.df11_pipeline_verify(self._h, int(slot), ctypes.byref(b), expected.data_ptr(),
+                                              expected.numel(), error.data_ptr(), fb,
+                                              _raw_stream(stream)), "df11_pipeline_verify")
+
     def release(self, slot: int, stream) -> None:
         _check(self._lib.df11_pipeline_release(self._h, int(slot), _raw_stream(stream)),
                "df11_pipeline_release")
@@ -543,3 +566,55 @@ def _raw_stream(stream, device=None):
         import torch
         return torch.cuda.current_stream(device).cuda_stream
     return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+# ------------------------------------------------------------- integrity
+
+def crc32c(data) -> int:
+    """df11_crc32c of a bytes-like object or numpy array (its raw bytes)."""
+    a = np.ascontiguousarray(np.frombuffer(data, np.uint8) if isinstance(data, (bytes, bytearray))
+                             else np.asarray(data)).view(np.uint8).reshape(-1)
+    return int(load_library().df11_crc32c(a.ctypes.data if a.size else None, a.size))
+
+
+def checksum_count(blk) -> int:
+    """Checksum values of a block (HostBlock, PinnedHostBlock or DeviceBlock):
+    one per 4096-byte segment of each array."""
+    b = blk.c_struct()
+    return int(load_library().df11_checksum_count(ctypes.byref(b)))
+
+
+def checksum(hb: HostBlock) -> np.ndarray:
+    """df11_checksum: the block's CRC-32C list, computed on the host."""
+    n = checksum_count(hb)
+    out = np.empty(n, np.uint32)
+    b = hb.c_struct()
+    _check(load_library().df11_checksum(ctypes.byref(b), out.ctypes.data, n), "df11_checksum")
+    return out
+
+
+def checksum_device(db: "DeviceBlock", stream=None):
+    """df11_checksum_device_async into a new int32 CUDA tensor (the uint32
+    values' bit patterns)."""
+    import torch
+    dev = next(iter(db.tensors.values())).device
+    n = checksum_count(db)
+    out = torch.empty(n, dtype=torch.int32, device=dev)
+    b = db.c_struct()
+    _check(load_library().df11_checksum_device_async(ctypes.byref(b), out.data_ptr(), n,
+                                                     _raw_stream(stream, dev)),
+           "df11_checksum_device_async")
+    return out
+
+
+def verify_device(db: "DeviceBlock", expected, error, first_bad=None, stream=None) -> None:
+    """df11_verify_device_async: ORs DEVERR_CHECKSUM into `error` (int32
+    CUDA tensor) if any segment differs from `expected` (int32 CUDA tensor of
+    the checksum list); `first_bad` (int64 CUDA tensor, preset to -1, i.e.
+    UINT64_MAX) receives the lowest bad segment index."""
+    b = db.c_struct()
+    fb = first_bad.data_ptr() if first_bad is not None else None
+    _check(load_library().df11_verify_device_async(ctypes.byref(b), expected.data_ptr(),
+                                                   expected.numel(), error.data_ptr(), fb,
+                                                   _raw_stream(stream, error.device)),
+           "df11_verify_device_async")

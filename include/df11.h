@@ -82,6 +82,8 @@ typedef enum {
                                      that chunk's output is not trustworthy    */
 #define DF11_DEVERR_MISMATCH 0x10u /* GPU compressor: an exponent without a code,
                                      or a bit total other than the codebook's  */
+#define DF11_DEVERR_CHECKSUM 0x20u /* df11_verify_device_async: a segment's
+                                     CRC-32C differs from the expected value   */
 
 #define DF11_MAX_CODE_LEN 16u     /* longest code the format allows           */
 #define DF11_MIN_CODE_LEN_CAP 8u  /* smallest cap accepted by build_codebook  */
@@ -290,6 +292,51 @@ df11_status df11_compress_device_noalloc(const df11_codebook *cb, const df11_lay
                                          uint32_t *d_error, void *stream);
 
 /* Human-readable name of a status code (static string). */
+/* ---- Integrity: CRC-32C per 4096-byte segment -----------------------------
+ * One flipped bit in the exponent stream desyncs the Huffman decoder and
+ * silently rewrites most of a tensor; the pages tell users to checksum DF11
+ * artifacts on download and after every copy ("DFloat11: lossless BFloat16
+ * compression", "How to run it in production" and "Failure modes").  The
+ * checksum of a block is a list of CRC-32C values (Castagnoli: reflected
+ * polynomial 0x82F63B78, initial value and final XOR 0xFFFFFFFF; the
+ * iSCSI / SSE4.2 CRC), one per DF11_CRC_SEGMENT_BYTES-byte segment of each
+ * array, arrays in the order exp_stream, gaps, chunk_pos (little-endian
+ * bytes), signmant, lut (little-endian bytes), each over the array sizes in
+ * the block struct; an array's last segment may be shorter.  Segments let
+ * the GPU check run in parallel and point at the damaged region.  The
+ * decoder itself flags desynchronised chunks (DF11_DEVERR_COUNT), but not a
+ * flipped sign or mantissa bit: only the checksum covers those. */
+#define DF11_CRC_SEGMENT_BYTES 4096u
+
+/* Host.  Number of checksum values of a block (0 for NULL). */
+uint64_t df11_checksum_count(const df11_host_block *blk);
+
+/* Host.  The CRC-32C of data[0 .. n) (the standard check value of the
+ * nine bytes "123456789" is 0xE3069283). */
+uint32_t df11_crc32c(const void *data, uint64_t n);
+
+/* Host.  Writes the block's checksum list into crc[0 .. n_crc);
+ * n_crc must equal df11_checksum_count(blk).  INVALID_ARGUMENT otherwise or
+ * for null pointers. */
+df11_status df11_checksum(const df11_host_block *blk, uint32_t *crc, uint64_t n_crc);
+
+/* GPU.  Computes the same list for a block in device memory into d_crc
+ * (device, 4-byte aligned, n_crc values = the count of the matching host
+ * block).  One launch on `stream`.  INVALID_ARGUMENT for null or
+ * misaligned pointers (arrays must be 16-byte aligned) or a wrong n_crc;
+ * CUDA when the launch fails. */
+df11_status df11_checksum_device_async(const df11_device_block *blk, uint32_t *d_crc, uint64_t n_crc,
+                                       void *stream);
+
+/* GPU.  Recomputes the list and compares it with d_expected (device): each
+ * mismatching segment ORs DF11_DEVERR_CHECKSUM into *d_error and, when
+ * d_first_bad (device uint64, 8-byte aligned, set to UINT64_MAX by the
+ * caller) is given, lowers it to the segment's index.  Same argument errors
+ * as df11_checksum_device_async; d_error must not be NULL. */
+df11_status df11_verify_device_async(const df11_device_block *blk, const uint32_t *d_expected,
+                                     uint64_t n_crc, uint32_t *d_error, uint64_t *d_first_bad,
+                                     void *stream);
+
 /* ---- Streamed decoding: upload -> decode -> consume ----------------------
  * The pages decode each transformer block right before its matrix products
  * and discard the BF16 copy afterwards ("DFloat11: lossless BFloat16
@@ -340,6 +387,15 @@ df11_status df11_pipeline_upload(df11_pipeline *p, uint32_t slot, const df11_hos
 df11_status df11_pipeline_decode(df11_pipeline *p, uint32_t slot, const df11_device_block *blk,
                                  uint16_t *out_bf16, uint64_t out_capacity, uint32_t *d_error,
                                  uint32_t max_ctas, void *decode_stream);
+
+/* Verify stage (optional, "after every copy").  Enqueues on `stream`,
+ * after the slot's last upload, df11_verify_device_async(blk, d_expected,
+ * n_crc, d_error, d_first_bad); enqueue it on the decode stream before
+ * df11_pipeline_decode so the decode follows it.  Errors: those of the
+ * verify call, INVALID_ARGUMENT for a bad pipeline, slot or device. */
+df11_status df11_pipeline_verify(df11_pipeline *p, uint32_t slot, const df11_device_block *blk,
+                                 const uint32_t *d_expected, uint64_t n_crc, uint32_t *d_error,
+                                 uint64_t *d_first_bad, void *stream);
 
 /* Consume stage.  acquire: consumer_stream waits for the slot's last
  * decode.  release: records that the consumer is done with the slot's

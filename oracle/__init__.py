@@ -2,7 +2,8 @@
 
 A plain, slow, single-threaded restatement of the method on the page
 "DFloat11: lossless BFloat16 compression" (sections "What it is",
-"Architecture" and "How it works: the core algorithm").  The arithmetic lives
+"Architecture" and "How it works: the core algorithm"; the artifact checksum
+of "How to run it in production").  The arithmetic lives
 in ``df11_oracle.c`` (plain C, compiled here with gcc); this module only
 marshals numpy arrays.  Only the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg may import it.  It shares no code with the
@@ -65,6 +66,8 @@ def _load():
         "orc_decode": (I, [P, U64, U64, U64, P, P, P]),
         "orc_first_code_table": (I, [P, P, P]),
         "orc_metadata": (I, [P, U64, P, U32, U32, U64, P, P]),
+        "orc_crc32c": (U32, [P, U64]),
+        "orc_segment_crcs": (U64, [P, U64, U64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -259,3 +262,30 @@ def decode_block(stream: np.ndarray, n_elements: int, lengths: np.ndarray,
     """Serial bit-by-bit decode of a whole block, joined back into BF16."""
     e, _ = decode(stream, n_elements, lengths)
     return join(e, _u8(signmant)[:n_elements])
+
+
+# ------------------------------------------------------------- checksum
+
+CRC_SEGMENT = 4096
+
+
+def crc32c(data) -> int:
+    """CRC-32C of the raw bytes of `data` (bytes or numpy array), bit by bit."""
+    a = _u8(np.frombuffer(bytes(data), np.uint8) if isinstance(data, (bytes, bytearray))
+            else np.ascontiguousarray(data).view(np.uint8).reshape(-1))
+    return int(_load().orc_crc32c(_ptr(a) if a.size else None, a.size))
+
+
+def segment_crcs(data, seg: int = CRC_SEGMENT) -> np.ndarray:
+    """CRC-32C of every `seg`-byte segment of the raw bytes of `data`."""
+    a = _u8(np.ascontiguousarray(data).view(np.uint8).reshape(-1))
+    out = np.empty(max(1, (a.size + seg - 1) // seg), np.uint32)
+    k = _load().orc_segment_crcs(_ptr(a) if a.size else None, a.size, seg, _ptr(out))
+    return out[:k]
+
+
+def block_checksums(exp_stream, gaps, chunk_pos, signmant, lut, seg: int = CRC_SEGMENT) -> np.ndarray:
+    """The checksum list of a block: segment CRCs of its five arrays in the
+    order exp_stream, gaps, chunk_pos, signmant, lut (raw little-endian
+    bytes of each array as given)."""
+    return np.concatenate([segment_crcs(a, seg) for a in (exp_stream, gaps, chunk_pos, signmant, lut)])

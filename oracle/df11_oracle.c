@@ -461,3 +461,30 @@ int orc_metadata(const uint8_t *exp, uint64_t n, const uint8_t len[256],
     }
     return 0;
 }
+
+
+/* ---- checksum ----------------------------------------------------------- */
+
+uint32_t orc_crc32c(const uint8_t *data, uint64_t n)
+{
+    const uint32_t poly = 0x82F63B78u;   /* the generator, bit-reversed */
+    uint32_t reg = 0xFFFFFFFFu;
+    for (uint64_t i = 0; i < n; ++i) {
+        reg ^= data[i];
+        for (int b = 0; b < 8; ++b) {
+            if (reg & 1u)
+                reg = (reg >> 1) ^ poly;
+            else
+                reg >>= 1;
+        }
+    }
+    return ~reg;
+}
+
+uint64_t orc_segment_crcs(const uint8_t *data, uint64_t n, uint64_t seg, uint32_t *out)
+{
+    uint64_t k = 0;
+    for (uint64_t off = 0; off < n; off += seg, ++k)
+        out[k] = orc_crc32c(data + off, n - off < seg ? n - off : seg);
+    return k;
+}

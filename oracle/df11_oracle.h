@@ -13,7 +13,8 @@
  *   [DF11-page] "DFloat11: lossless BFloat16 compression" (ai-infrastructure.net),
  *               sections "What it is", "Architecture" and
  *               "How it works: the core algorithm" (executed numpy sketch and
- *               its printed output).
+ *               its printed output); "How to run it in production" and
+ *               "Failure modes" (checksum every artifact).
  *
  * Every function below names the passage it follows.  All functions return 0
  * on success and a negative value on a detected error.
@@ -101,6 +102,20 @@ int orc_first_code_table(const uint8_t len[256], int16_t *sym_out, uint8_t *len_
 int orc_metadata(const uint8_t *exp, uint64_t n, const uint8_t len[256],
                  uint32_t threads_per_chunk, uint32_t bytes_per_thread,
                  uint64_t n_chunks, uint8_t *gap, uint32_t *pos);
+
+/* [DF11-page] "How to run it in production": checksum every artifact.  The
+ * checksum is CRC-32C (Castagnoli), written here bit by bit from its
+ * definition: the generator x^32 + x^28 + x^27 + x^26 + x^25 + x^23 + x^22 +
+ * x^20 + x^19 + x^18 + x^14 + x^13 + x^11 + x^10 + x^9 + x^8 + x^6 + 1,
+ * message bits taken least-significant first in every byte (a reflected
+ * register, so the generator appears as 0x82F63B78), register preset to all
+ * ones, result complemented.  No tables. */
+uint32_t orc_crc32c(const uint8_t *data, uint64_t n);
+
+/* The checksum list of one array: the CRC-32C of every `seg`-byte segment
+ * of data[0 .. n) in order (the last one may be shorter); returns the
+ * number of values written to out (ceil(n / seg)). */
+uint64_t orc_segment_crcs(const uint8_t *data, uint64_t n, uint64_t seg, uint32_t *out);
 
 #ifdef __cplusplus
 }

@@ -23,7 +23,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def _declared_functions():
     src = open(os.path.join(ROOT, "include", "df11.h")).read()
-    return sorted(set(re.findall(r"^(?:df11_status|const char \*|uint64_t)\s*(df11_\w+)\s*\(", src, re.M)))
+    return sorted(set(re.findall(r"^(?:df11_status|const char \*|uint64_t|uint32_t)\s*(df11_\w+)\s*\(", src, re.M)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -385,3 +385,58 @@ def test_compress_device_rejects_bad_arguments_before_any_cuda_call():
     assert lib.df11_histogram_device(None, n, fake, None) == 1
     assert lib.df11_histogram_device(fake, 0, fake, None) == 1
     assert lib.df11_histogram_device(fake + 2, n, fake, None) == 1
+
+
+# ------------------------------------------------------------- checksums
+# "DFloat11: lossless BFloat16 compression", "How to run it in production":
+# checksum every artifact.  The library's CRC-32C list must equal the
+# oracle's bit-by-bit CRC of every 4096-byte segment of every array.
+
+def _oracle_list(hb):
+    return oracle.block_checksums(hb.exp_stream, hb.gaps, hb.chunk_pos, hb.signmant, hb.lut)
+
+
+@pytest.mark.parametrize("name", ["single_1024x1024", "heavy_tail_512", "single_exponent_512"])
+def test_checksum_list_equals_oracle(name):
+    mats = [m for _, m in SMALL_WORKLOADS[name]()]
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats)
+    got = df11.checksum(hb)
+    ref = _oracle_list(hb)
+    assert df11.checksum_count(hb) == ref.size
+    assert np.array_equal(got, ref)
+
+
+def test_crc32c_equals_oracle_any_length_and_offset():
+    rng = np.random.default_rng(11)
+    buf = rng.integers(0, 256, 20000, dtype=np.uint8)
+    for start in (0, 1, 3, 7, 8, 13):
+        for n in (0, 1, 2, 7, 8, 9, 15, 16, 17, 4095, 4096, 4097, 12345):
+            d = buf[start:start + n]
+            assert df11.crc32c(d) == oracle.crc32c(d), (start, n)
+
+
+def test_checksum_rejects_bad_arguments():
+    hb = _fresh_block()
+    lib = df11.load_library()
+    b = hb.c_struct()
+    n = df11.checksum_count(hb)
+    out = np.empty(n + 1, np.uint32)
+    assert lib.df11_checksum(ctypes.byref(b), out.ctypes.data, n + 1) == 1
+    assert lib.df11_checksum(ctypes.byref(b), None, n) == 1
+    assert lib.df11_checksum(None, out.ctypes.data, n) == 1
+    assert lib.df11_checksum_count(None) == 0
+    fake = 1 << 20
+    d = binding._Block()
+    d.hdr = hb.header
+    for name in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut"):
+        setattr(d, name, fake)
+    d.exp_stream_bytes, d.gaps_bytes = hb.exp_stream.nbytes, hb.gaps.nbytes
+    d.chunk_pos_count, d.signmant_bytes, d.lut_entries = hb.chunk_pos.size, hb.signmant.nbytes, hb.lut.size
+    # host-side checks of the GPU calls, before any CUDA call
+    assert lib.df11_checksum_device_async(ctypes.byref(d), fake, n + 1, None) == 1
+    assert lib.df11_checksum_device_async(ctypes.byref(d), None, n, None) == 1
+    assert lib.df11_verify_device_async(ctypes.byref(d), fake, n, None, None, None) == 1
+    assert lib.df11_verify_device_async(ctypes.byref(d), fake, n, fake, fake + 4, None) == 1
+    d.signmant = fake + 8
+    assert lib.df11_checksum_device_async(ctypes.byref(d), fake, n, None) == 1

@@ -388,3 +388,72 @@ def test_metadata_brute_force_and_thread_decode(seed, T, W):
                 got += 1
         assert got == int(pos[ch + 1] - pos[ch])
     assert out == e.tolist()
+
+
+# ------------------------------------------------------------- checksum
+# "DFloat11: lossless BFloat16 compression", "How to run it in production":
+# checksum every artifact.  The oracle's CRC-32C is pinned to published check
+# values and to the definition as a polynomial remainder, computed here with
+# Python integers (no register loop, no reflection trick in the arithmetic).
+
+def _crc32c_by_division(data: bytes) -> int:
+    """CRC-32C as the remainder of (M(x) x^32 + (x^31 + ... + 1) x^n) by the
+    Castagnoli generator, where M's coefficients are the n message bits in
+    order, least significant bit of each byte first; the remainder's
+    coefficients are then read lowest degree first and complemented."""
+    bits = [(b >> i) & 1 for b in data for i in range(8)]
+    n = len(bits)
+    m = 0
+    for bit in bits:
+        m = (m << 1) | bit
+    v = (m << 32) ^ (0xFFFFFFFF << n)
+    g = 0x11EDC6F41
+    for sh in range(v.bit_length() - 33, -1, -1):
+        if (v >> (sh + 32)) & 1:
+            v ^= g << sh
+    return int(f"{v:032b}"[::-1], 2) ^ 0xFFFFFFFF
+
+
+def test_crc32c_published_vectors():
+    from conftest import read_golden
+    g = read_golden("crc32c_vectors.txt")
+    msgs = {
+        "check_123456789": b"123456789",
+        "zeros_32": bytes(32),
+        "ones_32": bytes([0xFF] * 32),
+        "incrementing_32": bytes(range(32)),
+        "decrementing_32": bytes(range(31, -1, -1)),
+    }
+    for k, m in msgs.items():
+        assert oracle.crc32c(m) == int(g[k], 16), k
+        assert _crc32c_by_division(m) == int(g[k], 16), k
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_crc32c_equals_polynomial_remainder(seed):
+    rng = np.random.default_rng(seed)
+    for n in (0, 1, 2, 3, 4, 5, 15, 16, 17, 63, 64, 65, 300):
+        d = rng.integers(0, 256, n, dtype=np.uint8).tobytes()
+        assert oracle.crc32c(d) == _crc32c_by_division(d), n
+
+
+def test_crc32c_detects_every_single_bit_flip():
+    """A CRC with a generator of more than one term catches every one-bit
+    error: the flip's error polynomial x^k is not a multiple of g."""
+    d = bytearray(np.random.default_rng(7).integers(0, 256, 64, dtype=np.uint8).tobytes())
+    base = oracle.crc32c(bytes(d))
+    for i in range(len(d) * 8):
+        d[i // 8] ^= 1 << (i % 8)
+        assert oracle.crc32c(bytes(d)) != base
+        d[i // 8] ^= 1 << (i % 8)
+
+
+def test_segment_crcs_split_and_ragged_tail():
+    rng = np.random.default_rng(3)
+    a = rng.integers(0, 256, 3 * 4096 + 123, dtype=np.uint8)
+    s = oracle.segment_crcs(a)
+    assert s.size == 4
+    for k in range(4):
+        assert s[k] == _crc32c_by_division(a[4096 * k: 4096 * (k + 1)].tobytes())
+    assert oracle.segment_crcs(np.zeros(0, np.uint8)).size == 0
+    assert oracle.segment_crcs(np.zeros(4096, np.uint8)).size == 1
