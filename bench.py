@@ -121,6 +121,35 @@ def make_block(seed: int, scale_div: int = 1, workload: str = WORKLOAD):
     return [m for _, m in workloads.WORKLOADS[workload]()]
 
 
+# ------------------------------------------------------ ranks (replicas)
+
+def rank_seed(rank: int, base: int = 1000, per_rank: int = 1) -> int:
+    """First block seed of a rank: ranks decode disjoint, independent blocks
+    (replicas, no data exchange)."""
+    return base + rank * per_rank
+
+
+def reduce_over_ranks(maxima, sums, device=None):
+    """Max-reduce `maxima` (timings) and sum-reduce `sums` (bytes, weights)
+    over all ranks; identity without an initialised process group.  Works on
+    NCCL (device tensors) and gloo (CPU tensors)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in maxima], [float(x) for x in sums]
+    t = torch.tensor([float(x) for x in maxima], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    c = torch.tensor([float(x) for x in sums], dtype=torch.float64, device=device)
+    dist.all_reduce(c, op=dist.ReduceOp.SUM)
+    return t.tolist(), c.tolist()
+
+
+def job_rate(job_units: float, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's device time (units per second / 1e9)."""
+    return job_units * steps / (ms_max * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -273,7 +302,7 @@ def run_b200(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    seed = 1000 + rank
+    seed = rank_seed(rank)
     mats = make_block(seed, args.scale_div, args.workload)
     t0 = time.perf_counter()
     cb = df11.build_codebook(mats)
@@ -354,18 +383,8 @@ def run_b200(args):
         e2e = {"ms": e2e_ms, "k": k, "h2d": h2d, "d2h": d2h}
 
     # ---- max over ranks, bytes summed over ranks
-    if world > 1:
-        t = torch.tensor([ms, e2e["ms"] / e2e["k"] if e2e else 0.0], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        b = torch.tensor([bytes_per_step, n], dtype=torch.float64, device=dev)
-        dist.all_reduce(b, op=dist.ReduceOp.SUM)
-        ms_max = float(t[0])
-        e2e_ms_per_step = float(t[1])
-        job_bytes, job_weights = float(b[0]), float(b[1])
-    else:
-        ms_max = ms
-        e2e_ms_per_step = e2e["ms"] / e2e["k"] if e2e else 0.0
-        job_bytes, job_weights = float(bytes_per_step), float(n)
+    (ms_max, e2e_ms_per_step), (job_bytes, job_weights) = reduce_over_ranks(
+        [ms, e2e["ms"] / e2e["k"] if e2e else 0.0], [bytes_per_step, n], dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -379,7 +398,7 @@ def run_b200(args):
         return 0
 
     ms_per_step = ms_max / args.steps
-    value = job_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    value = job_rate(job_bytes, args.steps, ms_max)
     peak, peak_kind = measured_peaks()
     launch_s = ms / args.steps * 1e-3              # this rank's own kernel time per launch
     achieved = bytes_per_step / launch_s / 1e9
@@ -397,7 +416,7 @@ def run_b200(args):
                    "l2": "inputs larger than L2 (%.2f GB touched per step vs 126 MB L2), no flush"
                          % (bytes_per_step / 1e9),
                    "parallelism": f"replicas x{world}, one block per GPU, no collective"},
-        "gweights_per_s": round(job_weights * args.steps / (ms_max * 1e-3) / 1e9, 2),
+        "gweights_per_s": round(job_rate(job_weights, args.steps, ms_max), 2),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "bit_exact": bit_exact,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
@@ -477,7 +496,7 @@ def run_model_stream(args):
     bpt = args.bytes_per_thread
     n_blocks = args.blocks or 32
     derr = torch.zeros(1, dtype=torch.int32, device=dev)
-    dbs, gpu_ms, host_cb_s = gpu_compressed_blocks(n_blocks, 1000 + rank * n_blocks, dev, bpt)
+    dbs, gpu_ms, host_cb_s = gpu_compressed_blocks(n_blocks, rank_seed(rank, per_rank=n_blocks), dev, bpt)
     out = torch.empty(max(db.n_elements for db in dbs), dtype=torch.bfloat16, device=dev)
     blocks = [(db, db.c_struct(), db.compressed_bytes() + 2 * db.n_elements) for db in dbs]
     n_weights = sum(db.n_elements for db in dbs)
@@ -508,22 +527,16 @@ def run_model_stream(args):
     ms = start.elapsed_time(end)
     if int(derr.item()):
         raise RuntimeError("device error word set during the timed decode")
+    (ms_max,), (job_bytes, job_weights) = reduce_over_ranks([ms], [step_bytes, n_weights], dev)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        bsum = torch.tensor([float(step_bytes), float(n_weights)], dtype=torch.float64, device=dev)
-        dist.all_reduce(bsum, op=dist.ReduceOp.SUM)
-        ms_max, job_bytes, job_weights = float(t[0]), float(bsum[0]), float(bsum[1])
         dist.barrier()
         dist.destroy_process_group()
-    else:
-        ms_max, job_bytes, job_weights = ms, float(step_bytes), float(n_weights)
     if rank != 0:
         return 0
     peak, peak_kind = measured_peaks()
     launches = args.steps * len(blocks)
     achieved = step_bytes / (ms / args.steps * 1e-3) / 1e9
-    value = job_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    value = job_rate(job_bytes, args.steps, ms_max)
     bf16_in = 2.0 * n_weights / len(blocks)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -535,7 +548,7 @@ def run_model_stream(args):
                    "bytes_per_step": step_bytes, "seeds": f"1000..{999 + len(blocks)}",
                    "l2": "inputs larger than L2, no flush",
                    "parallelism": f"replicas x{world}, own blocks per GPU, no collective"},
-        "gweights_per_s": round(job_weights * args.steps / (ms_max * 1e-3) / 1e9, 2),
+        "gweights_per_s": round(job_rate(job_weights, args.steps, ms_max), 2),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "bit_exact": True,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
