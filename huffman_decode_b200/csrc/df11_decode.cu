@@ -11,8 +11,8 @@
 //   * one warp = one chunk: output positions are stored per 32 threads, so
 //     every warp decodes, scans (shuffles), compacts and stores on its own,
 //     with no block-wide barrier after the prologue;
-//   * single decode pass with a multi-code table: a 10-bit window indexes a
-//     1024-entry table (built in shared memory from the format's two-level
+//   * single decode pass with a multi-code table: an 11-bit window indexes a
+//     2048-entry table (built in shared memory from the format's two-level
 //     16-bit tables) that yields up to four whole codes per lookup; longer
 //     codes fall back to the two-level tables;
 //   * exponents travel rotated right by one bit (bit 0 on top), which is
@@ -30,7 +30,9 @@
 //     least 2 bits long fit twice as many warps per SM;
 //   * the merge builds four BF16 values with two bit-selects and two byte
 //     permutes and writes one 16-byte vector per lane and group;
-//   * persistent CTAs: grid = resident CTAs per SM x SM count.
+//   * persistent CTAs of up to 32 warps (as many as shared memory holds;
+//     one CTA per SM for typical blocks, so all warps of an SM share one
+//     copy of the tables): grid = resident CTAs per SM x SM count.
 // No tensor cores: this is integer decode, bounded by HBM traffic and issue.
 #include "df11.h"
 
@@ -42,12 +44,12 @@
 namespace {
 
 constexpr uint32_t kLutPointer = 0x8000u;
-constexpr int kWindowBits = 10;                    // multi-code table index width
+constexpr int kWindowBits = 11;                    // multi-code table index width
 constexpr int kMultiEntries = 1 << kWindowBits;
 constexpr int kMaxCodesPerEntry = 4;
 constexpr int kEntryBytes = 8;                     // multi-code entry: symbols | step
 constexpr uint32_t kLongStep = 0x80000000u;        // step of an entry whose first code is long
-constexpr int kMaxWarpsPerCta = 16;
+constexpr int kMaxWarpsPerCta = 32;
 constexpr uint32_t kWaitLimit = 1u << 22;          // bounded mbarrier polls
 
 struct DecodeParams {
@@ -179,7 +181,7 @@ __device__ __forceinline__ void red_or_u32(uint32_t a, uint32_t v)
     asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
-static_assert(kWindowBits == 10 && kEntryBytes == 8, "lookup_step hard-codes the index mask and scale");
+static_assert(kEntryBytes == 8, "lookup_step scales the table index by 8");
 
 // Lane decode state X: bit position in bits 0..15, fill of the slot word (in
 // bits, 0..24 between lookups) in bits 16..21; kLongStep (bit 31) is added by
@@ -201,7 +203,7 @@ __device__ __forceinline__ void lookup_step(uint32_t &X, uint32_t &win, uint32_t
         ".reg .b32 a, f, t, z, c;\n\t"
         ".reg .pred p;\n\t"
         "mov.b32 z, 0;\n\t"
-        "and.b32 a, %1, 1023;\n\t"
+        "and.b32 a, %1, %9;\n\t"
         "mad.lo.u32 a, a, 8, %8;\n\t"
         "ld.shared.v2.u32 {%4, %5}, [a];\n\t"
         "shr.b32 f, %0, 16;\n\t"
@@ -218,7 +220,7 @@ __device__ __forceinline__ void lookup_step(uint32_t &X, uint32_t &win, uint32_t
         "@p sub.u32 %0, %0, 2097152;\n\t"
         "}"
         : "+r"(X), "+r"(win), "+r"(accl), "+r"(sp), "=r"(r.x), "=r"(r.y)
-        : "r"(lo), "r"(hi), "r"(multi_a)
+        : "r"(lo), "r"(hi), "r"(multi_a), "n"(kMultiEntries - 1)
         : "memory");
 }
 
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
     // ---- prologue: multi-code table -----------------------------------------
-    // Entry for a 10-bit window, stored at the window's bit-reversed value
+    // Entry for an 11-bit window, stored at the window's bit-reversed value
     // (first stream bit lowest, as the decoder reads it): x = the whole codes
     // the window starts with (at most 4), as rotated exponents in bytes 0..3
     // (unused bytes 0); y = the step total length | 8 * count << 16.  When
@@ -634,9 +636,9 @@ df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32
 {
     constexpr int v = (W == 8 ? 0 : 2) + (MINLEN == 1 ? 0 : 1);
     auto kernel = df11_decode_kernel<W, MINLEN>;
-    int warps = kMaxWarpsPerCta;
+    int warps = kMaxWarpsPerCta;   // as many warps as shared memory holds
     while (warps > 1 && smem_bytes_for<W, MINLEN>(warps, prm.n_tables) > kSmemLimit)
-        warps /= 2;
+        --warps;
     const size_t smem = smem_bytes_for<W, MINLEN>(warps, prm.n_tables);
     if (smem > kSmemLimit)
         return DF11_ERR_INVALID_ARGUMENT;
