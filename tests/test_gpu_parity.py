@@ -118,6 +118,17 @@ def test_codes_crossing_slice_ends(bpt):
     check_block([w], bytes_per_thread=bpt)
 
 
+@pytest.mark.parametrize("bpt", BPT)
+def test_many_tables_fewer_warps_per_cta(bpt):
+    """128 decode tables (64 KB in shared memory): the launch fits fewer warps
+    per CTA and every element must still match the oracle; one code is a
+    single bit (shortest code 1)."""
+    mats = [m for _, m in workloads.many_tables()]
+    cb, hb = check_block(mats, bytes_per_thread=bpt)
+    assert cb.n_tables >= 100
+    assert hb.header.min_code_len == 1
+
+
 def test_many_matrices_keep_caller_order():
     rng = np.random.default_rng(5)
     mats = [workloads.to_bf16((rng.standard_normal(int(k)) * s).astype(np.float32))

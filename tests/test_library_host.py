@@ -97,6 +97,7 @@ SMALL_WORKLOADS = {
     "heavy_tail_512": lambda: workloads.heavy_tail(4001, (512, 512)),
     "single_exponent_512": lambda: workloads.single_exponent(4002, (512, 512)),
     "uniform_bits_512": lambda: workloads.uniform_bits(4003, (512, 512)),
+    "many_tables_1m": lambda: workloads.many_tables(4004, 1 << 20),
 }
 
 

@@ -157,6 +157,22 @@ def llama_block_device(seed: int, device="cuda", scale_div: int = 1):
     return torch.cat(parts)
 
 
+def many_tables(seed: int = 4004, n: int = 1 << 21, rare_fraction: float = 1 / 64):
+    """One exponent (0x79) almost everywhere and the other 255 exponents
+    uniformly rare, random sign and mantissa: the dominant exponent gets a
+    1-bit code and the rare ones 8-9-bit codes spread over ~128 second-level
+    tables (a block whose decode tables fill a large part of shared memory)."""
+    rng = np.random.default_rng(seed)
+    e = np.full(n, 0x79, dtype=np.uint16)
+    k = int(n * rare_fraction)
+    pos = rng.choice(n, size=k, replace=False)
+    others = np.array([x for x in range(256) if x != 0x79], dtype=np.uint16)
+    e[pos] = others[rng.integers(0, others.size, k)]
+    sm = rng.integers(0, 256, n, dtype=np.uint16)
+    w = ((sm >> 7) << 15) | (e << 7) | (sm & 0x7F)
+    return [("many_tables", w.astype(np.uint16).reshape(1024, -1))]
+
+
 # The five workloads by name; each returns a list of (name, uint16 array).
 WORKLOADS = {
     "single_1024x1024": lambda: single_matrix(0),
