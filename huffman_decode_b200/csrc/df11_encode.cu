@@ -8,13 +8,16 @@
 //                                 histograms, one global add per bin and CTA);
 //   2. (host) df11_build_codebook_from_histogram -- code lengths, canonical
 //                                 codes and tables from that histogram;
-//   3. df11_compress_device    -- bit count per segment of 8192 elements,
-//      a scan of the segment counts, then one encode pass in which every
-//      thread knows its first bit: it appends its codes MSB-first into
-//      32-bit stream words (words shared with a neighbouring thread are
-//      ORed), records the gap of every slice whose first code it owns and
-//      the output position of every chunk that starts in such a slice, and
-//      writes its sign|mantissa bytes.
+//   3. df11_compress_device    -- bit count per segment of 8192 elements
+//      (one warp per segment), a scan of the segment counts, then one
+//      encode pass in which every thread knows its first bit: it appends its
+//      codes MSB-first into the segment's stream words staged in shared
+//      memory (words shared with a neighbouring thread are ORed), records
+//      the gap of every slice whose first code it owns (staged too) and the
+//      output position of every chunk that starts in such a slice, and
+//      writes its sign|mantissa bytes; the staged words then go to global
+//      memory with plain stores, ORing only the two words a segment may
+//      share with its neighbours.
 // The result is byte-identical to df11_compress (host) for the same
 // codebook and layout ("How it works": canonical codes, MSB-first encode;
 // "Architecture": Gaps and per-chunk output positions).
@@ -156,68 +159,94 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
     return warp_tot[warp] + incl - v;
 }
 
-__global__ void __launch_bounds__(kEncThreads) segment_bits_kernel(EncodeParams p, CodeTable ct)
+// Bits of every segment: one warp per segment (lane l sums the code lengths
+// of elements [256 l, 256 l + 256) of it), then a warp sum.
+__global__ void __launch_bounds__(256) segment_bits_kernel(EncodeParams p, CodeTable ct)
 {
     __shared__ uint32_t len_tab[256];
-    __shared__ uint32_t warp_tot[kEncThreads / 32 + 1];
     len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
     __syncthreads();
-    const uint64_t seg = blockIdx.x;
-    const uint64_t e0 = seg * kSegElems + (uint64_t)threadIdx.x * kElemsPerThread;
-    uint32_t w[16];
+    const int lane = threadIdx.x & 31;
+    const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x >> 5);
     bool bad = false;
-    const uint32_t bits = load_elems(p, len_tab, e0, w, bad);
-    uint32_t total;
-    block_exclusive_scan(bits, warp_tot, total);
-    if (threadIdx.x == 0)
-        p.seg_bits[seg] = total;
+    for (uint64_t seg = (uint64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); seg < p.n_seg;
+         seg += warps) {
+        const uint64_t e0 = seg * kSegElems + (uint64_t)lane * (kSegElems / 32);
+        uint32_t bits = 0;
+        if (e0 + kSegElems / 32 <= p.n) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.in + e0);
+#pragma unroll 8
+            for (int q = 0; q < kSegElems / 32 / 8; ++q) {
+                const uint4 v = src[q];
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t a = len_tab[(w4[k] >> 7) & 0xFFu];
+                    const uint32_t b = len_tab[(w4[k] >> 23) & 0xFFu];
+                    bad |= (a == 0) | (b == 0);
+                    bits += a + b;
+                }
+            }
+        } else {
+            for (uint64_t i = e0; i < e0 + kSegElems / 32 && i < p.n; ++i) {
+                const uint32_t l = len_tab[(p.in[i] >> 7) & 0xFFu];
+                bad |= l == 0;
+                bits += l;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            bits += __shfl_xor_sync(0xFFFFFFFFu, bits, o);
+        if (lane == 0)
+            p.seg_bits[seg] = bits;
+    }
     if (bad && p.err)
         atomicOr(p.err, DF11_DEVERR_MISMATCH);
 }
 
-// Exclusive scan of the segment bit counts (one CTA); checks the total.
+// Exclusive scan of the segment bit counts (one CTA): thread t sums a run of
+// consecutive segments, the CTA scans the run totals, then every thread
+// writes its run's starts.  Checks the grand total against the codebook.
 __global__ void __launch_bounds__(kScanThreads) segment_scan_kernel(EncodeParams p)
 {
-    __shared__ unsigned long long warp_tot[kScanThreads / 32];
-    __shared__ unsigned long long carry;
+    __shared__ unsigned long long warp_tot[kScanThreads / 32 + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0)
-        carry = 0;
+    const uint64_t per = (p.n_seg + kScanThreads - 1) / kScanThreads;
+    const uint64_t lo = (uint64_t)threadIdx.x * per;
+    const uint64_t hi = lo + per < p.n_seg ? lo + per : p.n_seg;
+    unsigned long long run = 0;
+    for (uint64_t i = lo; i < hi; ++i)
+        run += p.seg_bits[i];
+    unsigned long long incl = run;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d)
+            incl += y;
+    }
+    if (lane == 31)
+        warp_tot[warp] = incl;
     __syncthreads();
-    for (uint64_t base = 0; base < p.n_seg; base += kScanThreads) {
-        const uint64_t i = base + threadIdx.x;
-        const unsigned long long v = i < p.n_seg ? p.seg_bits[i] : 0ull;
-        unsigned long long incl = v;
+    if (warp == 0) {
+        const unsigned long long t = warp_tot[lane];
+        unsigned long long ti = t;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, ti, d);
             if (lane >= d)
-                incl += y;
+                ti += y;
         }
+        warp_tot[lane] = ti - t;
         if (lane == 31)
-            warp_tot[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            const unsigned long long t = warp_tot[lane];
-            unsigned long long ti = t;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, ti, d);
-                if (lane >= d)
-                    ti += y;
-            }
-            warp_tot[lane] = ti - t;
-        }
-        __syncthreads();
-        const unsigned long long c = carry;
-        if (i < p.n_seg)
-            p.seg_start[i] = c + warp_tot[warp] + incl - v;
-        __syncthreads();
-        if (threadIdx.x == kScanThreads - 1)
-            carry = c + warp_tot[warp] + incl;
-        __syncthreads();
+            warp_tot[kScanThreads / 32] = ti;
     }
-    if (threadIdx.x == 0 && carry != p.total_bits && p.err)
+    __syncthreads();
+    unsigned long long start = warp_tot[warp] + incl - run;
+    for (uint64_t i = lo; i < hi; ++i) {
+        p.seg_start[i] = start;
+        start += p.seg_bits[i];
+    }
+    if (threadIdx.x == 0 && warp_tot[kScanThreads / 32] != p.total_bits && p.err)
         atomicOr(p.err, DF11_DEVERR_MISMATCH);
 }
 
@@ -239,18 +268,42 @@ __global__ void prepare_kernel(EncodeParams p, uint64_t stream_words, uint64_t g
         p.signmant[i] = 0;
 }
 
-__device__ __forceinline__ void or_word(uint8_t *stream, uint64_t word, uint32_t v_be)
+__device__ __forceinline__ void red_or_shared_if(bool p, uint32_t a, uint32_t v)
 {
-    atomicOr(reinterpret_cast<uint32_t *>(stream) + word, bswap32(v_be));
+    asm volatile("{ .reg .pred q; setp.ne.u32 q, %0, 0; @q red.shared.or.b32 [%1], %2; }" ::"r"((uint32_t)p), "r"(a),
+                 "r"(v)
+                 : "memory");
 }
+
+// Stores v to the staged word at a when `full`: ORed in when `first` (the
+// word is shared with the previous thread), plainly otherwise.
+__device__ __forceinline__ void store_word_if(bool full, bool first, uint32_t a, uint32_t v)
+{
+    asm volatile(
+        "{ .reg .pred f, q, r; setp.ne.u32 f, %0, 0; setp.ne.u32 q, %1, 0; and.pred r, f, q;"
+        " @r red.shared.or.b32 [%2], %3; and.pred r, f, !q; @r st.shared.u32 [%2], %3; }" ::"r"((uint32_t)full),
+        "r"((uint32_t)first), "r"(a), "r"(v)
+        : "memory");
+}
+
+// Shared staging of one segment's output: stream words in bit order (bit 31
+// = first bit), and gap words (8 nibbles each, as in the gaps array).
+constexpr int kStageWords = kSegElems * 16 / 32 + 2;          // 16-bit codes at most
+constexpr int kGapStageWords = kSegElems * 16 / 64 / 8 + 2;   // 64-bit slices at the finest
 
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, CodeTable ct)
 {
     __shared__ uint32_t code_tab[256];
     __shared__ uint32_t len_tab[256];
     __shared__ uint32_t warp_tot[kEncThreads / 32 + 1];
+    __shared__ uint32_t sw[kStageWords];
+    __shared__ uint32_t sg[kGapStageWords];
     code_tab[threadIdx.x] = ct.e[threadIdx.x] & 0xFFFFFFu;
     len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
+    for (int i = threadIdx.x; i < kStageWords; i += kEncThreads)
+        sw[i] = 0;
+    for (int i = threadIdx.x; i < kGapStageWords; i += kEncThreads)
+        sg[i] = 0;
     __syncthreads();
 
     const uint64_t seg = blockIdx.x;
@@ -260,92 +313,136 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
     const uint32_t bits = load_elems(p, len_tab, e0, w, bad);
     uint32_t seg_total;
     const uint32_t off = block_exclusive_scan(bits, warp_tot, seg_total);
-    if (e0 >= p.n)
-        return;
-    uint64_t bitpos = p.seg_start[seg] + off;
+    const uint64_t S = p.seg_start[seg];                  // first bit of the segment
+    const uint64_t wbase = S >> 5;                        // stream word of sw[0]
+    const uint32_t sh = p.slice_shift;
+    const uint64_t gS = S >> sh;                          // slice of the segment's first bit
+    const uint64_t gbase = gS >> 3;                       // gap word of sg[0]
+    // Positions below are local: lb = bit - (gS << sh), so the slice of a
+    // local bit is gS + (lb >> sh) and its staged gap word ((lb >> sh) + (gS & 7)) >> 3.
+    const uint32_t lb0 = (uint32_t)(S - (gS << sh));
 
-    // slice of the previous code start (none for element 0)
-    uint64_t prev_slice = ~0ull;
-    if (e0 > 0) {
-        const uint32_t lp = len_tab[(p.in[e0 - 1] >> 7) & 0xFFu];
-        prev_slice = (bitpos - lp) >> p.slice_shift;
-    }
-    const uint32_t T = p.threads_per_chunk;
-
-    uint64_t word = bitpos >> 5;        // stream word being filled
-    uint64_t acc = 0;                   // pending bits, right-aligned
-    uint32_t filled = (uint32_t)(bitpos & 31);   // bits of `word` already set (earlier threads)
-    bool first_word = true;
-    const uint32_t cnt = (uint32_t)min((uint64_t)kElemsPerThread, p.n - e0);
+    if (e0 < p.n) {
+        uint32_t lb = lb0 + off;                          // local bit of the next code
+        // local slice of the previous code start (none for element 0)
+        int32_t prev_gl = -0x40000000;
+        if (e0 > 0) {
+            const uint32_t lp = len_tab[(p.in[e0 - 1] >> 7) & 0xFFu];
+            prev_gl = (int32_t)((int64_t)((int64_t)lb - lp) >> sh);   // may be -1
+        }
+        const uint32_t goff = (uint32_t)(gS & 7u);
+        uint32_t j = (uint32_t)(((S + off) >> 5) - wbase);   // staging word being filled
+        uint32_t fill = (uint32_t)((S + off) & 31);          // its bits already placed
+        uint32_t cur = 0;
+        bool first_word = true;
+        const uint32_t cnt = (uint32_t)min((uint64_t)kElemsPerThread, p.n - e0);
+        const uint32_t sw_a = (uint32_t)__cvta_generic_to_shared(sw);
+        const uint32_t sg_a = (uint32_t)__cvta_generic_to_shared(sg);
+        uint32_t prev = prev_gl < 0 ? 0xFFFFFFFFu : (uint32_t)prev_gl;
+        // One element: gap nibble of a slice its code opens, then the code
+        // MSB-first at bit `fill` of staged word j.  Branch-free apart from
+        // the rare chunk start; stores are predicated.
+        auto step = [&](uint32_t k) {
+            const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+            const uint32_t sy = (x >> 7) & 0xFFu;
+            const uint32_t l = len_tab[sy];
+            const uint32_t c = code_tab[sy];
+            const uint32_t gl = lb >> sh;
+            const bool opens = gl != prev;
+            const uint32_t gi = gl + goff;                 // slice index relative to gbase * 8
+            red_or_shared_if(opens, sg_a + 4u * (gi >> 3), ((lb - (gl << sh)) & 0xFu) << ((gi & 7u) * 4));
+            if (opens && ((gS + gl) & (DF11_THREADS_PER_CHUNK - 1)) == 0)
+                p.chunk_pos[(gS + gl) / DF11_THREADS_PER_CHUNK] = (uint32_t)(e0 + k);
+            prev = gl;
+            lb += l;
+            const uint32_t t = fill + l;
+            const uint64_t add = (uint64_t)c << ((64u - t) & 63u);
+            cur |= (uint32_t)(add >> 32);
+            const bool full = t >= 32;
+            store_word_if(full, first_word, sw_a + 4u * j, cur);   // the first is shared: ORed
+            cur = full ? (uint32_t)add : cur;
+            j += full ? 1u : 0u;
+            fill = full ? t - 32 : t;
+            first_word = first_word && !full;
+        };
+        if (cnt == kElemsPerThread) {
 #pragma unroll
-    for (uint32_t k = 0; k < kElemsPerThread; ++k) {
-        if (k >= cnt)
-            break;
-        const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
-        const uint32_t s = (x >> 7) & 0xFFu;
-        const uint32_t l = len_tab[s];
-        // metadata: first code of its slice
-        const uint64_t g = bitpos >> p.slice_shift;
-        if (g != prev_slice) {
-            const uint32_t gapv = (uint32_t)(bitpos - (g << p.slice_shift));
-            atomicOr(reinterpret_cast<uint32_t *>(p.gaps) + (g >> 3),
-                     (gapv & 0xFu) << (((g >> 1) & 3u) * 8 + (g & 1u) * 4));
-            if (g % T == 0)
-                p.chunk_pos[g / T] = (uint32_t)(e0 + k);
-            prev_slice = g;
-        }
-        // the code, MSB-first
-        acc = (acc << l) | code_tab[s];
-        filled += l;
-        bitpos += l;
-        if (filled >= 32) {
-            const uint32_t v = (uint32_t)(acc >> (filled - 32));
-            if (first_word)
-                or_word(p.stream, word, v);
-            else
-                reinterpret_cast<uint32_t *>(p.stream)[word] = bswap32(v);
-            first_word = false;
-            ++word;
-            filled -= 32;
-            acc &= (filled ? ((1ull << filled) - 1) : 0ull);
-        }
-    }
-    if (filled)
-        or_word(p.stream, word, (uint32_t)(acc << (32 - filled)));
-    // the end of the stream counts as a code start for the gap of its slice
-    if (e0 + cnt == p.n) {
-        const uint64_t g = bitpos >> p.slice_shift;
-        if (g < p.n_threads && g != prev_slice) {
-            const uint32_t gapv = (uint32_t)(bitpos - (g << p.slice_shift));
-            atomicOr(reinterpret_cast<uint32_t *>(p.gaps) + (g >> 3),
-                     (gapv & 0xFu) << (((g >> 1) & 3u) * 8 + (g & 1u) * 4));
-        }
-    }
-    // sign|mantissa bytes
-    if (cnt == kElemsPerThread) {
-        uint32_t sm[8];
+            for (uint32_t k = 0; k < kElemsPerThread; ++k)
+                step(k);
+        } else {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const uint32_t a = w[2 * q], b = w[2 * q + 1];
-            // element bytes: (x >> 8) & 0x80 | x & 0x7F for 4 elements
-            const uint32_t lo = __byte_perm(a, b, 0x6420);   // low bytes of the 4 elements
-            const uint32_t hi = __byte_perm(a, b, 0x7531);   // high bytes
-            sm[q] = (lo & 0x7F7F7F7Fu) | (hi & 0x80808080u);
+            for (uint32_t k = 0; k < kElemsPerThread; ++k) {
+                if (k >= cnt)
+                    break;
+                step(k);
+            }
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(p.signmant + e0);
-        dst[0] = make_uint4(sm[0], sm[1], sm[2], sm[3]);
-        dst[1] = make_uint4(sm[4], sm[5], sm[6], sm[7]);
-    } else {
+        const int32_t prev_gl_end = prev == 0xFFFFFFFFu ? -1 : (int32_t)prev;
+        if (fill)
+            atomicOr(&sw[j], cur);                                // shared with the next thread
+        // the end of the stream counts as a code start for the gap of its slice
+        if (e0 + cnt == p.n) {
+            const int32_t gl = (int32_t)(lb >> sh);
+            if (gS + (uint64_t)gl < p.n_threads && gl != prev_gl_end) {
+                const uint32_t gapv = lb - ((uint32_t)gl << sh);
+                const uint32_t gi = (uint32_t)gl + goff;
+                atomicOr(&sg[gi >> 3], (gapv & 0xFu) << ((gi & 7u) * 4));
+            }
+        }
+        // sign|mantissa bytes
+        if (cnt == kElemsPerThread) {
+            uint32_t sm[8];
 #pragma unroll
-        for (uint32_t k = 0; k < kElemsPerThread; ++k) {
-            if (k < cnt) {
-                const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
-                p.signmant[e0 + k] = (uint8_t)(((x >> 8) & 0x80u) | (x & 0x7Fu));
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t a = w[2 * q], b = w[2 * q + 1];
+                // element bytes: (x >> 8) & 0x80 | x & 0x7F for 4 elements
+                const uint32_t lo = __byte_perm(a, b, 0x6420);   // low bytes of the 4 elements
+                const uint32_t hi = __byte_perm(a, b, 0x7531);   // high bytes
+                sm[q] = (lo & 0x7F7F7F7Fu) | (hi & 0x80808080u);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(p.signmant + e0);
+            dst[0] = make_uint4(sm[0], sm[1], sm[2], sm[3]);
+            dst[1] = make_uint4(sm[4], sm[5], sm[6], sm[7]);
+        } else {
+#pragma unroll
+            for (uint32_t k = 0; k < kElemsPerThread; ++k) {
+                if (k < cnt) {
+                    const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+                    p.signmant[e0 + k] = (uint8_t)(((x >> 8) & 0x80u) | (x & 0x7Fu));
+                }
             }
         }
     }
     if (bad && p.err)
         atomicOr(p.err, DF11_DEVERR_MISMATCH);
+    __syncthreads();
+
+    // ---- staged words -> global: words that may be shared with the
+    // neighbouring segments (the first and the last) are ORed in
+    const uint64_t end_bit = S + seg_total;
+    if (seg_total) {
+        const uint32_t nw = (uint32_t)(((end_bit + 31) >> 5) - wbase);
+        uint32_t *g32 = reinterpret_cast<uint32_t *>(p.stream) + wbase;
+        for (uint32_t i = threadIdx.x; i < nw; i += kEncThreads) {
+            const uint32_t v = bswap32(sw[i]);
+            if (i == 0 || i == nw - 1)
+                atomicOr(g32 + i, v);
+            else
+                g32[i] = v;
+        }
+    }
+    {
+        const uint64_t glast = (end_bit >> p.slice_shift) >> 3;   // the end may open a slice
+        const uint32_t ng = (uint32_t)(glast - gbase + 1);
+        const uint64_t gwords = p.n_threads / 8;                  // gaps array length in words
+        uint32_t *gg = reinterpret_cast<uint32_t *>(p.gaps) + gbase;
+        for (uint32_t i = threadIdx.x; i < ng && gbase + i < gwords; i += kEncThreads) {
+            if (i == 0 || i == ng - 1)
+                atomicOr(gg + i, sg[i]);
+            else
+                gg[i] = sg[i];
+        }
+    }
 }
 
 bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
@@ -431,7 +528,8 @@ df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *lay
         return DF11_ERR_CUDA;
     prepare_kernel<<<sms * 4, 256, 0, s>>>(p, z.exp_stream_bytes / 4, (z.gaps_bytes + 3) / 4,
                                             z.n_chunks, z.signmant_bytes);
-    segment_bits_kernel<<<(unsigned)p.n_seg, kEncThreads, 0, s>>>(p, ct);
+    segment_bits_kernel<<<(unsigned)((p.n_seg + 7) / 8 < (uint64_t)sms * 8 ? (p.n_seg + 7) / 8 : (uint64_t)sms * 8),
+                          256, 0, s>>>(p, ct);
     segment_scan_kernel<<<1, kScanThreads, 0, s>>>(p);
     encode_kernel<<<(unsigned)p.n_seg, kEncThreads, 0, s>>>(p, ct);
     if (cudaGetLastError() != cudaSuccess)
