@@ -86,7 +86,11 @@ struct Geometry {
 
 // Shared memory: mbarriers | multi-code table | code lengths | per-warp areas
 // | two-level tables.
-constexpr size_t kHeadBytes = kMaxWarpsPerCta * 8 + kMultiEntries * kEntryBytes + 256;
+constexpr size_t kBarBytes = (kMaxWarpsPerCta * 8 + 15) / 16 * 16;   // one mbarrier per warp
+constexpr size_t kHeadBytes = kBarBytes + kMultiEntries * kEntryBytes + 256;
+// per-warp areas and the tables after them keep 16-byte alignment (TMA
+// destinations, 8- and 16-byte shared accesses)
+static_assert(kHeadBytes % 16 == 0, "shared-memory head must keep 16-byte alignment");
 
 template <int W, int MINLEN>
 constexpr size_t smem_bytes_for(int warps, uint32_t n_tables)
@@ -294,8 +298,8 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
     extern __shared__ __align__(16) uint8_t smem[];
     const int warps = blockDim.x >> 5;
     uint64_t *mbar = reinterpret_cast<uint64_t *>(smem);
-    uint2 *multi = reinterpret_cast<uint2 *>(smem + kMaxWarpsPerCta * 8);
-    uint8_t *len_of = smem + kMaxWarpsPerCta * 8 + kMultiEntries * kEntryBytes;   // by rotated exponent
+    uint2 *multi = reinterpret_cast<uint2 *>(smem + kBarBytes);
+    uint8_t *len_of = smem + kBarBytes + kMultiEntries * kEntryBytes;   // by rotated exponent
     uint8_t *warp_area = smem + kHeadBytes;
     uint16_t *lut = reinterpret_cast<uint16_t *>(warp_area + (size_t)warps * G::kWarpBytes);
 
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
 
     // shared-window addresses (bytes)
     const uint32_t smem_base = smem_addr(smem);
-    const uint32_t multi_a = smem_base + kMaxWarpsPerCta * 8;
+    const uint32_t multi_a = smem_base + (uint32_t)kBarBytes;
     const uint32_t len_a = multi_a + kMultiEntries * kEntryBytes;
     const uint32_t lut_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warps * G::kWarpBytes);
     const uint32_t slots_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warp * G::kWarpBytes);
