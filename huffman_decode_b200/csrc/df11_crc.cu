@@ -15,7 +15,8 @@
 // GPU method: one warp per segment, lane l covers bytes [128 l, 128 l + 128)
 // of it.  A lane folds its bytes four at a time (x = crc ^ word; crc = x
 // advanced over four zero bytes, which is linear in x: four 256-entry table
-// lookups), then advances its partial CRC over the bytes after its run, and
+// lookups in a copy of the tables private to the lane, so the 32 lanes of a
+// warp never meet on a shared-memory bank), then advances its partial CRC over the bytes after its run, and
 // the warp XORs the 32 partials: CRC is linear, and crc(A || B) = crc(A)
 // advanced over |B| zero bytes, XOR crc(B).  "Advance over 2^j zero bytes"
 // is a table operator S_j (4 x 256 words) built in shared memory by
@@ -35,8 +36,11 @@ constexpr uint32_t kPolyReflected = 0x82F63B78u;
 constexpr uint64_t kSeg = DF11_CRC_SEGMENT_BYTES;
 constexpr int kLaneBytes = (int)(kSeg / 32);     // 128
 constexpr int kShiftOps = 13;                    // advance by 2^0 .. 2^12 bytes
-constexpr int kCrcThreads = 256;
-constexpr size_t kCrcSmem = (256 + (size_t)kShiftOps * 1024) * 4;
+constexpr int kCrcThreads = 1024;
+// shared: byte table | S_0..S_12 | a lane-private copy of S_2 (the four-byte
+// fold), entry e of lane l at word 32 e + l, so every lane reads its own bank
+constexpr size_t kPrivWords = 1024 * 32;
+constexpr size_t kCrcSmem = (256 + (size_t)kShiftOps * 1024 + kPrivWords) * 4;
 
 static_assert(kSeg == 4096, "one warp of 32 lanes x 128 bytes per segment");
 
@@ -150,9 +154,13 @@ __device__ __forceinline__ uint32_t advance_by(const uint32_t *ops, uint32_t c, 
     return c;
 }
 
-__device__ __forceinline__ uint32_t fold_word(const uint32_t *ops, uint32_t c, uint32_t w)
+// c advanced over the four bytes of w (operator S_2), from the lane's
+// private copy: lane_priv points at word `lane` of it.
+__device__ __forceinline__ uint32_t fold_word(const uint32_t *lane_priv, uint32_t c, uint32_t w)
 {
-    return advance(ops + 2 * 1024, c ^ w);   // four bytes = operator S_2
+    const uint32_t x = c ^ w;
+    return lane_priv[32 * (x & 0xFFu)] ^ lane_priv[32 * (256 + ((x >> 8) & 0xFFu))] ^
+           lane_priv[32 * (512 + ((x >> 16) & 0xFFu))] ^ lane_priv[32 * (768 + (x >> 24))];
 }
 
 __global__ void __launch_bounds__(kCrcThreads) crc_kernel(ArrayView av, uint32_t *out, const uint32_t *expected,
@@ -179,28 +187,56 @@ __global__ void __launch_bounds__(kCrcThreads) crc_kernel(ArrayView av, uint32_t
             ops[j * 1024 + i] = advance(ops + (j - 1) * 1024, ops[(j - 1) * 1024 + i]);
         __syncthreads();
     }
+    uint32_t *priv = ops + kShiftOps * 1024;
+    for (int i = tid; i < (int)kPrivWords; i += blockDim.x)
+        priv[i] = ops[2 * 1024 + (i >> 5)];
+    __syncthreads();
 
     const int lane = tid & 31;
+    const uint32_t *lane_priv = priv + lane;
     const uint64_t warps = blockDim.x >> 5;
     const uint64_t total = av.first[5];
     for (uint64_t seg = blockIdx.x * warps + (tid >> 5); seg < total; seg += gridDim.x * warps) {
-        int a = 0;
-        while (seg >= av.first[a + 1])
-            ++a;
-        const uint64_t local = seg - av.first[a];
-        const uint8_t *base = av.ptr[a] + local * kSeg;
-        const uint64_t rem = av.len[a] - local * kSeg;
+        // the array holding the segment: the last one whose first segment is
+        // <= seg (empty arrays share their first index with the next one)
+        const uint8_t *aptr = av.ptr[0];
+        uint64_t alen = av.len[0], afirst = 0;
+#pragma unroll
+        for (int k = 1; k < 5; ++k)
+            if (seg >= av.first[k]) {
+                aptr = av.ptr[k];
+                alen = av.len[k];
+                afirst = av.first[k];
+            }
+        const uint64_t local = seg - afirst;
+        const uint8_t *base = aptr + local * kSeg;
+        const uint64_t rem = alen - local * kSeg;
         const uint32_t n = (uint32_t)(rem < kSeg ? rem : kSeg);
         const uint32_t beg = (uint32_t)(kLaneBytes * lane);
         const uint32_t end = beg < n ? min(n, beg + (uint32_t)kLaneBytes) : beg;
         uint32_t c = 0;
         uint32_t q = beg;
+        if (end - beg == (uint32_t)kLaneBytes) {
+            // a full run: all eight loads in flight before folding
+            uint4 v[kLaneBytes / 16];
+#pragma unroll
+            for (int i = 0; i < kLaneBytes / 16; ++i)
+                v[i] = __ldg(reinterpret_cast<const uint4 *>(base + beg) + i);
+#pragma unroll
+            for (int i = 0; i < kLaneBytes / 16; ++i) {
+                c = fold_word(lane_priv, c, v[i].x);
+                c = fold_word(lane_priv, c, v[i].y);
+                c = fold_word(lane_priv, c, v[i].z);
+                c = fold_word(lane_priv, c, v[i].w);
+            }
+            q = end;
+        }
         for (; q + 16 <= end; q += 16) {
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + q));
-            c = fold_word(ops, c, v.x);
-            c = fold_word(ops, c, v.y);
-            c = fold_word(ops, c, v.z);
-            c = fold_word(ops, c, v.w);
+            c = fold_word(lane_priv, c, v.x);
+            c = fold_word(lane_priv, c, v.y);
+            c = fold_word(lane_priv, c, v.z);
+            c = fold_word(lane_priv, c, v.w);
         }
         for (; q < end; ++q)
             c = (c >> 8) ^ t0[(c ^ base[q]) & 0xFFu];
@@ -252,7 +288,7 @@ df11_status launch_crc(const df11_device_block *blk, uint32_t *d_out, const uint
     }
     const uint64_t warps = kCrcThreads / 32;
     const uint64_t need = (av.first[5] + warps - 1) / warps;
-    const uint64_t cap = 4ull * (uint64_t)sms;
+    const uint64_t cap = (uint64_t)sms;   // one 32-warp CTA per SM (the private table fills shared memory)
     const unsigned grid = (unsigned)(need < cap ? need : cap);
     crc_kernel<<<grid, kCrcThreads, kCrcSmem, reinterpret_cast<cudaStream_t>(stream)>>>(
         av, d_out, d_expected, d_error, reinterpret_cast<unsigned long long *>(d_first_bad));
