@@ -68,6 +68,26 @@ struct DecodeParams {
     uint32_t full_chunks; // chunks lying wholly below total_bits (every slice full)
 };
 
+// Decode fused with a matrix-vector product: every matrix of the block is
+// multiplied by n_tokens activation rows as it is decoded, and the BF16
+// weights never reach HBM.
+constexpr int kGemvMaxMats = 128;
+
+struct GemvMat {
+    uint32_t start;    // first element of the matrix in the block
+    uint32_t cols;     // row length, a multiple of 8
+    uint32_t rows;
+    uint32_t pad;
+    const uint16_t *x; // n_tokens x cols BF16, token-major
+    float *y;          // n_tokens x rows FP32, accumulated into
+};
+
+struct GemvParams {
+    uint32_t n_mats;
+    uint32_t n_tokens;
+    GemvMat m[kGemvMaxMats];
+};
+
 // Per-warp buffers for W stream bytes per lane and codes of at least MINLEN
 // bits: slot columns, the contiguous exponent buffer, the staged
 // sign|mantissa bytes.
@@ -291,8 +311,143 @@ __device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, ui
     gap = (p.gaps[g >> 1] >> ((g & 1) * 4)) & 0xFu;
 }
 
-template <int W, int MINLEN>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(DecodeParams p)
+// Matrix of block element e: the last one whose start is <= e.
+__device__ __forceinline__ int gemv_matrix_of(const GemvParams *gp, uint32_t e)
+{
+    int lo = 0, hi = (int)gp->n_mats - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (gp->m[mid].start <= e)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Adds the chunk's products to y: whole 8-element groups go lane by lane
+// (group gfirst + lane + 32k), each lane keeping one partial sum per token
+// for its current row and adding it to y when the row changes; the partial
+// groups at both ends take one element per lane on lanes 0..15.  ebuf holds
+// the chunk's rotated exponents, sgrp its sign|mantissa bytes (group 0 of
+// the chunk at offset 0 of both).
+template <int TT>
+__device__ __forceinline__ void gemv_chunk(const GemvParams *gp, uint32_t head, uint32_t n_write, uint64_t base,
+                                           uint32_t gfirst, int lane, uint32_t ebuf_a, uint32_t sgrp_a)
+{
+    const uint32_t nt = gp->n_tokens;
+    const uint32_t span = head + n_write;
+    const uint32_t mend = span >> 3;
+    uint32_t i = gfirst + lane;
+    if (i < mend) {
+        uint32_t e = (uint32_t)base + 8u * i;               // block element of the group
+        int m = gemv_matrix_of(gp, e);
+        uint32_t cols = gp->m[m].cols, rows = gp->m[m].rows;
+        uint32_t mlast = gp->m[m].start + rows * cols;      // one past the matrix
+        uint32_t off = e - gp->m[m].start;
+        uint32_t r = off / cols, c = off - r * cols;
+        const uint16_t *x = gp->m[m].x;
+        float *y = gp->m[m].y;
+        float acc[TT];
+#pragma unroll
+        for (int t = 0; t < TT; ++t)
+            acc[t] = 0.f;
+        for (;;) {
+            const uint2 e8 = lds_v2_m(ebuf_a + 8u * i);
+            const uint2 s8 = lds_v2_m(sgrp_a + 8u * i);
+            const uint2 wa = join4(e8.x, s8.x);
+            const uint2 wb = join4(e8.y, s8.y);
+            const float w0 = bf16_lo(wa.x), w1 = bf16_hi(wa.x), w2 = bf16_lo(wa.y), w3 = bf16_hi(wa.y);
+            const float w4 = bf16_lo(wb.x), w5 = bf16_hi(wb.x), w6 = bf16_lo(wb.y), w7 = bf16_hi(wb.y);
+#pragma unroll
+            for (int t = 0; t < TT; ++t) {
+                if (t < (int)nt) {
+                    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * cols + c));
+                    float a = acc[t];
+                    a = fmaf(w0, bf16_lo(xv.x), a);
+                    a = fmaf(w1, bf16_hi(xv.x), a);
+                    a = fmaf(w2, bf16_lo(xv.y), a);
+                    a = fmaf(w3, bf16_hi(xv.y), a);
+                    a = fmaf(w4, bf16_lo(xv.z), a);
+                    a = fmaf(w5, bf16_hi(xv.z), a);
+                    a = fmaf(w6, bf16_lo(xv.w), a);
+                    a = fmaf(w7, bf16_hi(xv.w), a);
+                    acc[t] = a;
+                }
+            }
+            i += 32;
+            const bool more = i < mend;
+            // the next group: same row, a later row, or another matrix
+            uint32_t ne = e + 256u, nr = r, nc = c + 256u;
+            int nm = m;
+            if (more) {
+                if (ne >= mlast) {
+                    nm = gemv_matrix_of(gp, ne);
+                    const uint32_t o = ne - gp->m[nm].start;
+                    nr = o / gp->m[nm].cols;
+                    nc = o - nr * gp->m[nm].cols;
+                } else {
+                    while (nc >= cols) {
+                        nc -= cols;
+                        ++nr;
+                    }
+                }
+            }
+            if (!more || nm != m || nr != r) {
+#pragma unroll
+                for (int t = 0; t < TT; ++t) {
+                    if (t < (int)nt)
+                        atomicAdd(y + (size_t)t * rows + r, acc[t]);
+                    acc[t] = 0.f;
+                }
+            }
+            if (!more)
+                break;
+            if (nm != m) {
+                m = nm;
+                cols = gp->m[m].cols;
+                rows = gp->m[m].rows;
+                mlast = gp->m[m].start + rows * cols;
+                x = gp->m[m].x;
+                y = gp->m[m].y;
+            }
+            e = ne;
+            r = nr;
+            c = nc;
+        }
+    }
+    // partial groups at both ends, one element per lane
+    const uint32_t fs = gfirst * 8;
+    const uint32_t hend = min(fs, span);
+    const uint32_t tbeg = max(mend * 8, fs);
+    uint32_t l = 0xFFFFFFFFu;
+    if (lane < 8) {
+        if (head + lane < hend)
+            l = head + lane;
+    } else if (lane < 16) {
+        if (tbeg + (lane - 8) < span)
+            l = tbeg + (lane - 8);
+    }
+    if (l != 0xFFFFFFFFu) {
+        const uint32_t e = (uint32_t)base + l;
+        const int m = gemv_matrix_of(gp, e);
+        const uint32_t cols = gp->m[m].cols;
+        const uint32_t o = e - gp->m[m].start;
+        const uint32_t r = o / cols, c = o - r * cols;
+        const float wv = __uint_as_float((uint32_t)join1(lds_u8_m(ebuf_a + l), lds_u8_m(sgrp_a + l)) << 16);
+        for (uint32_t t = 0; t < nt; ++t)
+            atomicAdd(gp->m[m].y + (size_t)t * gp->m[m].rows + r,
+                      wv * __uint_as_float((uint32_t)gp->m[m].x[(size_t)t * cols + c] << 16));
+    }
+}
+
+// The chunk body.  TT = 0: BF16 output; TT > 0: fused matrix-vector product
+// for up to TT tokens (gp != nullptr).
+template <int W, int MINLEN, int TT>
+__device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvParams *gp)
 {
     using G = Geometry<W, MINLEN>;
     extern __shared__ __align__(16) uint8_t smem[];
@@ -580,7 +735,7 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
             // Whole groups: 8 exponents + 8 sign|mantissa bytes -> one 16-byte
             // store per lane.  The partial groups at both ends (<= 7 elements
             // each) take one element per lane on lanes 0..15.
-            if (!stalled) {
+            if (!stalled && TT == 0) {
                 const uint32_t span = head + n_write;
                 const uint32_t mend = span >> 3;                   // whole groups end
                 const uint32_t sgrp_a = sbuf_a + (pos0 & 8u);     // group 0 of the chunk
@@ -607,6 +762,10 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
                 if (l != 0xFFFFFFFFu)
                     p.out[base + l] = join1(lds_u8_m(ebuf_a + l), lds_u8_m(sgrp_a + l));
             }
+            if constexpr (TT > 0) {
+                if (!stalled)
+                    gemv_chunk<TT>(gp, head, n_write, base, gfirst, lane, ebuf_a, sbuf_a + (pos0 & 8u));
+            }
             __syncwarp();
         }
 
@@ -626,21 +785,45 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(Decod
         atomicOr(p.err, err);
 }
 
+template <int W, int MINLEN>
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(DecodeParams p)
+{
+    decode_body<W, MINLEN, 0>(p, nullptr);
+}
+
+template <int W, int MINLEN, int TT>
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_gemv_kernel(DecodeParams p,
+                                                                         const __grid_constant__ GemvParams gp)
+{
+    decode_body<W, MINLEN, TT>(p, &gp);
+}
+
 // ------------------------------------------------------------ launch
 
 constexpr int kMaxDevices = 64;
 constexpr size_t kSmemLimit = 227 * 1024;
+// kernel variants: (slice width, shortest code) x (store, products for 1, 2,
+// 4, 8 tokens)
+constexpr int kVariants = 4 * 5;
 // resident CTAs per SM, by device, kernel variant and table count
-std::atomic<int> g_occupancy[kMaxDevices][4][257];
+std::atomic<int> g_occupancy[kMaxDevices][kVariants][257];
 std::atomic<int> g_sm_count[kMaxDevices];
-std::atomic<int> g_attr_done[kMaxDevices][4];
+std::atomic<int> g_attr_done[kMaxDevices][kVariants];
 
-template <int W, int MINLEN>
-df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32_t max_ctas)
+struct LaunchShape {
+    int warps;
+    size_t smem;
+    unsigned grid;
+};
+
+// Warps per CTA (as many as shared memory holds), shared memory, and the
+// grid (one wave of resident CTAs by default; max_ctas overrides it) for
+// one kernel variant; sets the shared-memory attribute once per device.
+template <int W, int MINLEN, typename Kernel>
+df11_status shape_launch(Kernel kernel, int v, const DecodeParams &prm, int dev, uint32_t max_ctas,
+                         LaunchShape &ls)
 {
-    constexpr int v = (W == 8 ? 0 : 2) + (MINLEN == 1 ? 0 : 1);
-    auto kernel = df11_decode_kernel<W, MINLEN>;
-    int warps = kMaxWarpsPerCta;   // as many warps as shared memory holds
+    int warps = kMaxWarpsPerCta;
     while (warps > 1 && smem_bytes_for<W, MINLEN>(warps, prm.n_tables) > kSmemLimit)
         --warps;
     const size_t smem = smem_bytes_for<W, MINLEN>(warps, prm.n_tables);
@@ -672,9 +855,53 @@ df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32
     // count may be smaller (SMs left to other streams) or larger (waves of
     // short-lived CTAs that free their SM as each one finishes)
     const uint64_t want = max_ctas ? (uint64_t)max_ctas : resident;
-    const uint64_t grid = ctas_needed < want ? ctas_needed : want;
-    kernel<<<(unsigned)grid, warps * 32, smem, stream>>>(prm);
+    ls.warps = warps;
+    ls.smem = smem;
+    ls.grid = (unsigned)(ctas_needed < want ? ctas_needed : want);
+    return DF11_OK;
+}
+
+template <int W, int MINLEN>
+constexpr int variant_base()
+{
+    return ((W == 8 ? 0 : 2) + (MINLEN == 1 ? 0 : 1)) * 5;
+}
+
+template <int W, int MINLEN>
+df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32_t max_ctas)
+{
+    auto kernel = df11_decode_kernel<W, MINLEN>;
+    LaunchShape ls;
+    const df11_status st = shape_launch<W, MINLEN>(kernel, variant_base<W, MINLEN>(), prm, dev, max_ctas, ls);
+    if (st != DF11_OK)
+        return st;
+    kernel<<<ls.grid, ls.warps * 32, ls.smem, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+template <int W, int MINLEN, int TT>
+df11_status launch_gemv(const DecodeParams &prm, const GemvParams &gp, int dev, cudaStream_t stream)
+{
+    auto kernel = df11_gemv_kernel<W, MINLEN, TT>;
+    constexpr int v = variant_base<W, MINLEN>() + (TT == 1 ? 1 : TT == 2 ? 2 : TT == 4 ? 3 : 4);
+    LaunchShape ls;
+    const df11_status st = shape_launch<W, MINLEN>(kernel, v, prm, dev, 0, ls);
+    if (st != DF11_OK)
+        return st;
+    kernel<<<ls.grid, ls.warps * 32, ls.smem, stream>>>(prm, gp);
+    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+template <int W, int MINLEN>
+df11_status launch_gemv_tokens(const DecodeParams &prm, const GemvParams &gp, int dev, cudaStream_t stream)
+{
+    if (gp.n_tokens <= 1)
+        return launch_gemv<W, MINLEN, 1>(prm, gp, dev, stream);
+    if (gp.n_tokens <= 2)
+        return launch_gemv<W, MINLEN, 2>(prm, gp, dev, stream);
+    if (gp.n_tokens <= 4)
+        return launch_gemv<W, MINLEN, 4>(prm, gp, dev, stream);
+    return launch_gemv<W, MINLEN, 8>(prm, gp, dev, stream);
 }
 
 bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
@@ -688,18 +915,20 @@ extern "C" df11_status df11_decompress_async(const df11_device_block *blk, uint1
     return df11_decompress_async_ctas(blk, out_bf16, out_capacity, d_error, 0, stream);
 }
 
-extern "C" df11_status df11_decompress_async_ctas(const df11_device_block *blk, uint16_t *out_bf16,
-                                                  uint64_t out_capacity, uint32_t *d_error,
-                                                  uint32_t max_ctas, void *stream)
+namespace {
+
+// Host-side checks of a device block and the decode parameters for it.
+df11_status block_params(const df11_device_block *blk, uint16_t *out_bf16, uint64_t out_limit, uint32_t *d_error,
+                         DecodeParams &prm, int &dev)
 {
-    if (!blk || !out_bf16)
+    if (!blk)
         return DF11_ERR_INVALID_ARGUMENT;
     const df11_header &h = blk->hdr;
     const uint32_t W = h.bytes_per_thread;
     if (h.threads_per_chunk != DF11_THREADS_PER_CHUNK || (W != 8 && W != 16))
         return DF11_ERR_INVALID_ARGUMENT;
     if (h.n_elements == 0 || h.n_elements >= (1ull << 32) || h.n_tables < 1 || h.n_tables > 256 ||
-        h.total_bits == 0 || out_capacity < h.n_elements || h.min_code_len < 1 ||
+        h.total_bits == 0 || out_limit < h.n_elements || h.min_code_len < 1 ||
         h.min_code_len > DF11_MAX_CODE_LEN)
         return DF11_ERR_INVALID_ARGUMENT;
     const uint64_t chunk_bits = (uint64_t)DF11_THREADS_PER_CHUNK * 8 * W;
@@ -717,12 +946,8 @@ extern "C" df11_status df11_decompress_async_ctas(const df11_device_block *blk, 
         !aligned(blk->signmant, 16) || !aligned(blk->gaps, 16) || !aligned(out_bf16, 16) ||
         !aligned(d_error, 4))
         return DF11_ERR_INVALID_ARGUMENT;
-
-    int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return DF11_ERR_CUDA;
-
-    DecodeParams prm;
     prm.stream = blk->exp_stream;
     prm.gaps = blk->gaps;
     prm.chunk_pos = blk->chunk_pos;
@@ -732,12 +957,71 @@ extern "C" df11_status df11_decompress_async_ctas(const df11_device_block *blk, 
     prm.err = d_error;
     prm.total_bits = h.total_bits;
     prm.n_chunks = h.n_chunks;
-    prm.out_limit = h.n_elements < out_capacity ? h.n_elements : out_capacity;
+    prm.out_limit = h.n_elements < out_limit ? h.n_elements : out_limit;
     prm.n_tables = h.n_tables;
     prm.min_len = h.min_code_len;
     prm.full_chunks = (uint32_t)(h.total_bits / chunk_bits);
+    return DF11_OK;
+}
+
+}  // namespace
+
+extern "C" df11_status df11_decompress_async_ctas(const df11_device_block *blk, uint16_t *out_bf16,
+                                                  uint64_t out_capacity, uint32_t *d_error,
+                                                  uint32_t max_ctas, void *stream)
+{
+    if (!out_bf16)
+        return DF11_ERR_INVALID_ARGUMENT;
+    DecodeParams prm;
+    int dev = 0;
+    const df11_status st = block_params(blk, out_bf16, out_capacity, d_error, prm, dev);
+    if (st != DF11_OK)
+        return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (W == 8)
-        return h.min_code_len >= 2 ? launch<8, 2>(prm, dev, s, max_ctas) : launch<8, 1>(prm, dev, s, max_ctas);
-    return h.min_code_len >= 2 ? launch<16, 2>(prm, dev, s, max_ctas) : launch<16, 1>(prm, dev, s, max_ctas);
+    if (blk->hdr.bytes_per_thread == 8)
+        return prm.min_len >= 2 ? launch<8, 2>(prm, dev, s, max_ctas) : launch<8, 1>(prm, dev, s, max_ctas);
+    return prm.min_len >= 2 ? launch<16, 2>(prm, dev, s, max_ctas) : launch<16, 1>(prm, dev, s, max_ctas);
+}
+
+extern "C" df11_status df11_decode_gemv_async(const df11_device_block *blk, const df11_gemv_matrix *mats,
+                                              uint32_t n_mats, uint32_t n_tokens, uint32_t *d_error,
+                                              void *stream)
+{
+    if (!blk || !mats || n_mats == 0 || n_mats > (uint32_t)kGemvMaxMats || n_tokens == 0 || n_tokens > 8)
+        return DF11_ERR_INVALID_ARGUMENT;
+    GemvParams gp;
+    gp.n_mats = n_mats;
+    gp.n_tokens = n_tokens;
+    uint64_t start = 0;
+    for (uint32_t i = 0; i < n_mats; ++i) {
+        const df11_gemv_matrix &m = mats[i];
+        if (m.rows == 0 || m.cols == 0 || (m.cols & 7u) || !m.x || !m.y || !aligned(m.x, 16) ||
+            !aligned(m.y, 4))
+            return DF11_ERR_INVALID_ARGUMENT;
+        if (m.rows >= (1ull << 32) || m.cols >= (1ull << 32))
+            return DF11_ERR_INVALID_ARGUMENT;
+        gp.m[i].start = (uint32_t)start;
+        gp.m[i].cols = (uint32_t)m.cols;
+        gp.m[i].rows = (uint32_t)m.rows;
+        gp.m[i].pad = 0;
+        gp.m[i].x = m.x;
+        gp.m[i].y = m.y;
+        start += m.rows * m.cols;
+        if (start >= (1ull << 32))
+            return DF11_ERR_INVALID_ARGUMENT;
+    }
+    if (start != blk->hdr.n_elements)
+        return DF11_ERR_INVALID_ARGUMENT;
+    DecodeParams prm;
+    int dev = 0;
+    // no BF16 output: a dummy aligned pointer satisfies the checks and is never written
+    const df11_status st =
+        block_params(blk, reinterpret_cast<uint16_t *>(16), blk->hdr.n_elements, d_error, prm, dev);
+    if (st != DF11_OK)
+        return st;
+    prm.out = nullptr;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (blk->hdr.bytes_per_thread == 8)
+        return prm.min_len >= 2 ? launch_gemv_tokens<8, 2>(prm, gp, dev, s) : launch_gemv_tokens<8, 1>(prm, gp, dev, s);
+    return prm.min_len >= 2 ? launch_gemv_tokens<16, 2>(prm, gp, dev, s) : launch_gemv_tokens<16, 1>(prm, gp, dev, s);
 }

@@ -47,6 +47,7 @@ EXPORTED_SYMBOLS = (
     "df11_pipeline_destroy", "df11_pipeline_upload", "df11_pipeline_decode", "df11_pipeline_acquire",
     "df11_pipeline_release", "df11_checksum_count", "df11_crc32c", "df11_checksum",
     "df11_checksum_device_async", "df11_verify_device_async", "df11_pipeline_verify",
+    "df11_decode_gemv_async",
 )
 CRC_SEGMENT_BYTES = 4096
 NOALLOC_SCRATCH_BYTES = 1 << 20
@@ -165,6 +166,7 @@ def load_library(path: str | None = None):
         ("df11_checksum_device_async", S, [P, P, U64, P]),
         ("df11_verify_device_async", S, [P, P, U64, P, P, P]),
         ("df11_pipeline_verify", S, [P, U32, P, P, U64, P, P, P]),
+        ("df11_decode_gemv_async", S, [P, P, U32, U32, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -618,3 +620,33 @@ def verify_device(db: "DeviceBlock", expected, error, first_bad=None, stream=Non
                                                    expected.numel(), error.data_ptr(), fb,
                                                    _raw_stream(stream, error.device)),
            "df11_verify_device_async")
+
+
+# ------------------------------------------------ decode fused with products
+
+class GemvMatrix(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_uint64), ("cols", ctypes.c_uint64),
+                ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+
+
+def decode_gemv_async(db: "DeviceBlock", shapes, xs, ys, error=None, stream=None) -> None:
+    """df11_decode_gemv_async: for matrix i of the block, shapes[i] = (rows,
+    cols), adds xs[i] (n_tokens x cols, 16-bit CUDA tensor of BF16 bits)
+    times W_i^T into ys[i] (n_tokens x rows, float32 CUDA tensor, zeroed by
+    the caller), decoding the block once and never writing it in BF16."""
+    n = len(shapes)
+    if len(xs) != n or len(ys) != n or n == 0:
+        raise ValueError("one x and one y per matrix")
+    n_tokens = int(xs[0].shape[0])
+    arr = (GemvMatrix * n)()
+    for i, ((r, c), x, y) in enumerate(zip(shapes, xs, ys)):
+        if x.element_size() != 2 or not x.is_contiguous() or tuple(x.shape) != (n_tokens, c):
+            raise ValueError(f"x[{i}] must be a contiguous {n_tokens} x {c} 16-bit tensor")
+        if y.dtype.itemsize != 4 or not y.is_contiguous() or tuple(y.shape) != (n_tokens, r):
+            raise ValueError(f"y[{i}] must be a contiguous {n_tokens} x {r} float32 tensor")
+        arr[i] = GemvMatrix(int(r), int(c), x.data_ptr(), y.data_ptr())
+    b = db.c_struct()
+    err_ptr = error.data_ptr() if error is not None else None
+    _check(load_library().df11_decode_gemv_async(ctypes.byref(b), arr, n, n_tokens, err_ptr,
+                                                 _raw_stream(stream, xs[0].device)),
+           "df11_decode_gemv_async")

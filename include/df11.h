@@ -233,6 +233,34 @@ df11_status df11_decompress_async_ctas(const df11_device_block *blk, uint16_t *o
                                        uint64_t out_capacity, uint32_t *d_error,
                                        uint32_t max_ctas, void *stream);
 
+/* ---- Decode fused with its consumer: matrix-vector products --------------
+ * The pages decode a block into a BF16 buffer and then run its matrix
+ * products ("DFloat11: lossless BFloat16 compression", "Architecture":
+ * decode, block matmuls, discard).  For a few tokens the products are
+ * matrix-vector work bound by reading the weights, so this call multiplies
+ * each weight as it is decoded and never writes the BF16 block to HBM
+ * (this library's addition).  Matrix i of the block (mats[i], in block
+ * order, rows x cols row-major, cols a multiple of 8) gets
+ *     y[t][r] += sum_c W[r][c] * x[t][c],   t < n_tokens (1..8),
+ * with x device BF16 (n_tokens x cols, token-major, 16-byte aligned) and y
+ * device FP32 (n_tokens x rows, 4-byte aligned, zeroed by the caller: the
+ * kernel accumulates into it with atomic adds, so the summation order and
+ * the last bits of y vary between runs).  Products and sums are FP32. */
+typedef struct {
+    uint64_t rows;
+    uint64_t cols;
+    const uint16_t *x;
+    float *y;
+} df11_gemv_matrix;
+
+/* GPU.  One launch on `stream`.  Errors: INVALID_ARGUMENT (the block checks
+ * of df11_decompress_async, n_mats outside 1..128, n_tokens outside 1..8,
+ * a matrix with cols not a multiple of 8 or misaligned pointers, or
+ * matrices that do not add up to the block's elements), CUDA.  Device
+ * errors go to *d_error as for df11_decompress_async. */
+df11_status df11_decode_gemv_async(const df11_device_block *blk, const df11_gemv_matrix *mats,
+                                   uint32_t n_mats, uint32_t n_tokens, uint32_t *d_error, void *stream);
+
 /* ---- GPU-side compressor --------------------------------------------------
  * The pages compress on the CPU only ("DFloat11: lossless BFloat16
  * compression", "How to develop with it": minutes per block on one thread).

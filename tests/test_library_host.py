@@ -441,3 +441,37 @@ def test_checksum_rejects_bad_arguments():
     assert lib.df11_verify_device_async(ctypes.byref(d), fake, n, fake, fake + 4, None) == 1
     d.signmant = fake + 8
     assert lib.df11_checksum_device_async(ctypes.byref(d), fake, n, None) == 1
+
+
+def test_decode_gemv_rejects_bad_arguments_before_any_cuda_call():
+    """df11_decode_gemv_async: matrix table and token checks need no GPU."""
+    hb = _fresh_block()
+    lib = df11.load_library()
+    fake = 1 << 20
+    d = binding._Block()
+    d.hdr = hb.header
+    for name in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut"):
+        setattr(d, name, fake)
+    d.exp_stream_bytes, d.gaps_bytes = hb.exp_stream.nbytes, hb.gaps.nbytes
+    d.chunk_pos_count, d.signmant_bytes, d.lut_entries = hb.chunk_pos.size, hb.signmant.nbytes, hb.lut.size
+    shapes = [m.shape for _, m in workloads.llama_block(1002, scale_div=256)]
+
+    def table(shp, x=fake, y=fake):
+        arr = (binding.GemvMatrix * len(shp))()
+        for i, (r, c) in enumerate(shp):
+            arr[i] = binding.GemvMatrix(r, c, x, y)
+        return arr
+
+    call = lambda arr, n, t: lib.df11_decode_gemv_async(ctypes.byref(d), arr, n, t, None, None)
+    good = table(shapes)
+    assert sum(r * c for r, c in shapes) == hb.n_elements
+    assert call(good, len(shapes), 0) == 1                      # no tokens
+    assert call(good, len(shapes), 9) == 1                      # more than 8
+    assert call(good, 0, 1) == 1
+    assert call(good, len(shapes) - 1, 1) == 1                  # does not cover the block
+    assert call(table(shapes, x=fake + 8), len(shapes), 1) == 1 # misaligned activations
+    assert call(table(shapes, y=fake + 2), len(shapes), 1) == 1
+    bad = list(shapes)
+    bad[0] = (bad[0][0] * 2, bad[0][1] // 2 + 4)                # cols not a multiple of 8
+    assert call(table(bad), len(bad), 1) == 1
+    assert lib.df11_decode_gemv_async(None, good, len(shapes), 1, None, None) == 1

@@ -157,20 +157,38 @@ def llama_block_device(seed: int, device="cuda", scale_div: int = 1):
     return torch.cat(parts)
 
 
-def many_tables(seed: int = 4004, n: int = 1 << 21, rare_fraction: float = 1 / 64):
-    """One exponent (0x79) almost everywhere and the other 255 exponents
-    uniformly rare, random sign and mantissa: the dominant exponent gets a
-    1-bit code and the rare ones 8-9-bit codes spread over ~128 second-level
-    tables (a block whose decode tables fill a large part of shared memory)."""
+def many_tables(seed: int = 4004, n: int = 1 << 21, rare_fraction: float = 1 / 64,
+                rare_exponents=range(256)):
+    """One exponent (0x79) almost everywhere and the other exponents of
+    rare_exponents (default: all 255 others) uniformly rare, random sign and
+    mantissa: the dominant exponent gets a 1-bit code and the rare ones
+    long codes spread over many second-level tables (with all 255: ~128
+    tables, a block whose decode tables fill a large part of shared
+    memory)."""
     rng = np.random.default_rng(seed)
     e = np.full(n, 0x79, dtype=np.uint16)
     k = int(n * rare_fraction)
     pos = rng.choice(n, size=k, replace=False)
-    others = np.array([x for x in range(256) if x != 0x79], dtype=np.uint16)
+    others = np.array([x for x in rare_exponents if x != 0x79], dtype=np.uint16)
     e[pos] = others[rng.integers(0, others.size, k)]
     sm = rng.integers(0, 256, n, dtype=np.uint16)
     w = ((sm >> 7) << 15) | (e << 7) | (sm & 0x7F)
     return [("many_tables", w.astype(np.uint16).reshape(1024, -1))]
+
+
+def activations(seed: int, n_tokens: int, cols: int, sigma: float = 1.0):
+    """Activation rows for the fused matrix-vector products: n_tokens x cols
+    float32 N(0, sigma) rounded to BF16 (uint16 bit patterns)."""
+    rng = np.random.default_rng(seed)
+    return _normal_bf16(rng, (n_tokens, cols), sigma)
+
+
+def small_cols_block(seed: int = 6000):
+    """Matrices with rows shorter than 256 elements (and one of 8), so one
+    step of 256 elements crosses several rows: 512x64, 64x8, 8x1024, 100x16."""
+    rng = np.random.default_rng(seed)
+    return [(f"m{i}", _normal_bf16(rng, shape, 0.02))
+            for i, shape in enumerate([(512, 64), (64, 8), (8, 1024), (100, 16)])]
 
 
 # The five workloads by name; each returns a list of (name, uint16 array).
