@@ -55,7 +55,7 @@ def parse_args():
                     help="stream bytes each decoding thread owns (format layout)")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=sorted(workloads.WORKLOADS) + ["llama8b_model", "llama8b_overlap",
-                                                           "llama8b_offload"],
+                                                           "llama8b_offload", "llama8b_gemv"],
                     help="block to decode (the headline number is llama8b_block); "
                          "llama8b_model = 32 Llama-3.1-8B blocks, each with its own "
                          "codebook, decoded one after another into one buffer; "
@@ -66,8 +66,9 @@ def parse_args():
     ap.add_argument("--blocks", type=int, default=None,
                     help="blocks of the llama8b_model/overlap/offload streams "
                          "(default 32, 8 for offload)")
-    ap.add_argument("--tokens", default="1,256,2048,8192",
-                    help="llama8b_overlap: comma-separated token counts of the activations")
+    ap.add_argument("--tokens", default=None,
+                    help="comma-separated token counts of the activations (llama8b_overlap: "
+                         "default 1,256,2048,8192; llama8b_gemv: default 1,4,8)")
     ap.add_argument("--max-ctas", default="0,1184",
                     help="llama8b_overlap: comma-separated decode CTA counts (0 = one resident "
                          "wave; large = one short-lived CTA per 16 chunks)")
@@ -601,7 +602,7 @@ def run_overlap(args):
     s_dec = torch.cuda.Stream(dev)
     s_use = torch.cuda.Stream(dev, priority=args.consumer_priority)
     results = []
-    token_list = [int(t) for t in args.tokens.split(",") if t]
+    token_list = [int(t) for t in (args.tokens or "1,256,2048,8192").split(",") if t]
     cap_list = [int(c) for c in args.max_ctas.split(",") if c != ""]
     for T in token_list:
         g = torch.Generator(device=dev)
@@ -831,6 +832,113 @@ def run_offload(args):
     return 0 if ok else 1
 
 
+def run_gemv(args):
+    """Decode fused with its consumer at small token counts (1 GPU): n
+    blocks resident compressed in HBM; per block the seven Llama-3.1-8B
+    matrices multiply T activation rows.  Timed on the device:
+      fused   - df11_decode_gemv_async, one launch per block (the BF16 block
+                never reaches HBM), plus zeroing the block's outputs;
+      serial  - decode to a BF16 buffer, then seven cuBLAS products
+                (torch.mm), the pages' order;
+      bf16    - seven cuBLAS products on resident BF16 weights (no DF11).
+    The fused launch's roofline is HBM: it reads the compressed block (and
+    the activations) and writes the outputs."""
+    import torch
+
+    import huffman_decode_b200 as df11
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    n_blocks = args.blocks or 16
+    dbs, _, _ = gpu_compressed_blocks(n_blocks, 1000, dev, args.bytes_per_thread)
+    shapes = [s for _, s in workloads.LLAMA8B_BLOCK_SHAPES]
+    offs = np.cumsum([0] + [r * c for r, c in shapes])
+    n = int(offs[-1])
+    buf = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    wres = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    df11.decompress_async(dbs[0], wres)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    cur = torch.cuda.current_stream(dev)
+    peak, peak_kind = measured_peaks()
+    results = []
+    for T in [int(t) for t in (args.tokens or "1,4,8").split(",") if t]:
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 + T)
+        xs = [torch.randn(T, c, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+              for _, c in shapes]
+        xs16 = [x.view(torch.int16) for x in xs]
+        ybuf = torch.zeros(sum(T * r for r, _ in shapes), dtype=torch.float32, device=dev)
+        ys, o = [], 0
+        for r, _ in shapes:
+            ys.append(ybuf[o:o + T * r].view(T, r))
+            o += T * r
+        yb = [torch.empty(T, r, dtype=torch.bfloat16, device=dev) for r, _ in shapes]
+
+        def fused():
+            for db in dbs:
+                ybuf.zero_()
+                df11.decode_gemv_async(db, shapes, xs16, ys, err)
+
+        def mm(wbuf):
+            for i, (r, c) in enumerate(shapes):
+                torch.mm(xs[i], wbuf[offs[i]:offs[i + 1]].view(r, c).t(), out=yb[i])
+
+        def serial():
+            for db in dbs:
+                df11.decompress_async(db, buf, err)
+                mm(buf)
+
+        def bf16():
+            for _ in dbs:
+                mm(wres)
+
+        def timed(fn):
+            for _ in range(max(args.warmup, 1)):
+                fn()
+            torch.cuda.synchronize()
+            e = _events(2)
+            e[0].record(cur)
+            for _ in range(args.steps):
+                fn()
+            e[1].record(cur)
+            torch.cuda.synchronize()
+            return e[0].elapsed_time(e[1]) / args.steps / n_blocks
+
+        t_f, t_s, t_b = timed(fused), timed(serial), timed(bf16)
+        # the last block's fused products against decode + cuBLAS (FP32 from BF16 outputs)
+        ybuf.zero_()
+        df11.decode_gemv_async(dbs[-1], shapes, xs16, ys, err)
+        df11.decompress_async(dbs[-1], buf, err)
+        mm(buf)
+        torch.cuda.synchronize()
+        rel = max(float(((ys[i] - yb[i].float()).abs().max() / (yb[i].float().abs().max() + 1e-30)))
+                  for i in range(len(shapes)))
+        comp = dbs[0].compressed_bytes()
+        moved = comp + 2 * T * sum(c for _, c in shapes) + 4 * T * sum(r for r, _ in shapes)
+        gbs = moved / (t_f * 1e-3) / 1e9
+        results.append({
+            "tokens": T, "fused_ms_per_block": round(t_f, 4), "serial_ms_per_block": round(t_s, 4),
+            "bf16_ms_per_block": round(t_b, 4), "fused_vs_serial": round(t_s / t_f, 3),
+            "fused_vs_bf16": round(t_b / t_f, 3),
+            "fused_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                               "peak_source": peak_kind, "frac": round(gbs / peak, 4),
+                               "bytes_per_block": moved},
+            "max_rel_diff_vs_cublas_bf16_out": rel})
+    if int(err.item()):
+        raise RuntimeError("device error word set")
+    line = {
+        "metric": "decode fused with matrix-vector products: ms per Llama-3.1-8B block",
+        "value": None, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": False, "dtype": "fp32 accumulate, bf16 in",
+        "data": "synthetic (GPU-drawn weights and activations)",
+        "config": {"workload": "llama8b_gemv", "blocks": n_blocks, "n_weights_per_block": n,
+                   "bytes_per_thread": args.bytes_per_thread},
+        "results": results,
+        "gpu_launches": n_blocks * args.steps * 2,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -841,6 +949,8 @@ def main():
         return run_overlap(args)
     if args.workload == "llama8b_offload":
         return run_offload(args)
+    if args.workload == "llama8b_gemv":
+        return run_gemv(args)
     return run_b200(args)
 
 

@@ -172,6 +172,12 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t a)
     asm("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
+__device__ __forceinline__ uint2 lds_v2(uint32_t a)
+{
+    uint2 v;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
 __device__ __forceinline__ uint32_t lds_u32_m(uint32_t a)
 {
     uint32_t v;
@@ -328,119 +334,121 @@ __device__ __forceinline__ int gemv_matrix_of(const GemvParams *gp, uint32_t e)
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// Adds the chunk's products to y: whole 8-element groups go lane by lane
-// (group gfirst + lane + 32k), each lane keeping one partial sum per token
-// for its current row and adding it to y when the row changes; the partial
-// groups at both ends take one element per lane on lanes 0..15.  ebuf holds
-// the chunk's rotated exponents, sgrp its sign|mantissa bytes (group 0 of
-// the chunk at offset 0 of both).
+// Adds the chunk's products to y.  The groups of 8 elements that touch
+// the chunk's range [head, head + n_write) (relative to base, 8-aligned)
+// are taken one row segment at a time: a segment is the groups of one row
+// of one matrix (groups never straddle rows because rows and matrices
+// start at multiples of 8).  The lanes share a segment's groups, keep one
+// partial sum per token, and a warp sum adds each token's total to y with
+// one atomic add.  Matrix and row are located once per chunk and then
+// stepped.  In the first and last groups only the chunk's own elements
+// count.  ebuf holds the chunk's rotated exponents, sgrp its
+// sign|mantissa bytes (group 0 of the chunk at offset 0 of both).
 template <int TT>
 __device__ __forceinline__ void gemv_chunk(const GemvParams *gp, uint32_t head, uint32_t n_write, uint64_t base,
-                                           uint32_t gfirst, int lane, uint32_t ebuf_a, uint32_t sgrp_a)
+                                           int lane, uint32_t ebuf_a, uint32_t sgrp_a)
 {
     const uint32_t nt = gp->n_tokens;
     const uint32_t span = head + n_write;
-    const uint32_t mend = span >> 3;
-    uint32_t i = gfirst + lane;
-    if (i < mend) {
-        uint32_t e = (uint32_t)base + 8u * i;               // block element of the group
-        int m = gemv_matrix_of(gp, e);
-        uint32_t cols = gp->m[m].cols, rows = gp->m[m].rows;
-        uint32_t mlast = gp->m[m].start + rows * cols;      // one past the matrix
-        uint32_t off = e - gp->m[m].start;
-        uint32_t r = off / cols, c = off - r * cols;
-        const uint16_t *x = gp->m[m].x;
-        float *y = gp->m[m].y;
+    const uint32_t ngroups = (span + 7) >> 3;
+    if (ngroups == 0)
+        return;
+    // matrix, row and column of group 0
+    int m = gemv_matrix_of(gp, (uint32_t)base);
+    uint32_t cols = gp->m[m].cols, rows = gp->m[m].rows;
+    uint32_t r, c;
+    {
+        const uint32_t o = (uint32_t)base - gp->m[m].start;
+        r = o / cols;
+        c = o - r * cols;
+    }
+    const uint16_t *xm = gp->m[m].x;
+    float *ym = gp->m[m].y;
+    uint32_t g = 0;
+    for (;;) {
+        const uint32_t gend = min(ngroups, g + ((cols - c) >> 3));
+        const uint16_t *xr = xm + c;                        // activations at the segment's first column
         float acc[TT];
 #pragma unroll
         for (int t = 0; t < TT; ++t)
             acc[t] = 0.f;
-        for (;;) {
-            const uint2 e8 = lds_v2_m(ebuf_a + 8u * i);
-            const uint2 s8 = lds_v2_m(sgrp_a + 8u * i);
-            const uint2 wa = join4(e8.x, s8.x);
-            const uint2 wb = join4(e8.y, s8.y);
+        // The buffers were filled before the warp's last __syncwarp, which
+        // orders these plain shared loads; the activation loads go first so
+        // their latency overlaps the weight assembly.
+#pragma unroll(TT <= 2 ? 2 : 1)
+        for (uint32_t i = g + lane; i < gend; i += 32) {
+            const uint32_t dc = 8u * (i - g);               // column offset within the segment
+            constexpr int TP = TT < 2 ? TT : 2;             // tokens whose rows are loaded together
+            uint4 xv[TP];
+#pragma unroll
+            for (int t = 0; t < TP; ++t)
+                xv[t] = t < (int)nt ? __ldg(reinterpret_cast<const uint4 *>(xr + (size_t)t * cols + dc))
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            const uint2 e8 = lds_v2(ebuf_a + 8u * i);
+            const uint2 s8 = lds_v2(sgrp_a + 8u * i);
+            uint2 wa = join4(e8.x, s8.x);
+            uint2 wb = join4(e8.y, s8.y);
+            if (i == 0 || i + 1 == ngroups) {
+                // a group at an end of the chunk: zero the weights outside it
+                const uint32_t lo = i == 0 ? head : 0u;
+                const uint32_t hi = min(8u, span - 8u * i);
+                const uint32_t keep = (0xFFu >> (8 - hi)) & (0xFFu << lo);   // element mask
+                wa.x &= ((keep & 1u) ? 0x0000FFFFu : 0u) | ((keep & 2u) ? 0xFFFF0000u : 0u);
+                wa.y &= ((keep & 4u) ? 0x0000FFFFu : 0u) | ((keep & 8u) ? 0xFFFF0000u : 0u);
+                wb.x &= ((keep & 16u) ? 0x0000FFFFu : 0u) | ((keep & 32u) ? 0xFFFF0000u : 0u);
+                wb.y &= ((keep & 64u) ? 0x0000FFFFu : 0u) | ((keep & 128u) ? 0xFFFF0000u : 0u);
+            }
             const float w0 = bf16_lo(wa.x), w1 = bf16_hi(wa.x), w2 = bf16_lo(wa.y), w3 = bf16_hi(wa.y);
             const float w4 = bf16_lo(wb.x), w5 = bf16_hi(wb.x), w6 = bf16_lo(wb.y), w7 = bf16_hi(wb.y);
 #pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                if (t < (int)nt) {
-                    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * cols + c));
-                    float a = acc[t];
-                    a = fmaf(w0, bf16_lo(xv.x), a);
-                    a = fmaf(w1, bf16_hi(xv.x), a);
-                    a = fmaf(w2, bf16_lo(xv.y), a);
-                    a = fmaf(w3, bf16_hi(xv.y), a);
-                    a = fmaf(w4, bf16_lo(xv.z), a);
-                    a = fmaf(w5, bf16_hi(xv.z), a);
-                    a = fmaf(w6, bf16_lo(xv.w), a);
-                    a = fmaf(w7, bf16_hi(xv.w), a);
-                    acc[t] = a;
+            for (int t0 = 0; t0 < TT; t0 += TP) {
+#pragma unroll
+                for (int u = 0; u < TP; ++u) {
+                    const int t = t0 + u;
+                    if (t0 > 0 && t < (int)nt)                 // later token blocks load here
+                        xv[u] = __ldg(reinterpret_cast<const uint4 *>(xr + (size_t)t * cols + dc));
                 }
-            }
-            i += 32;
-            const bool more = i < mend;
-            // the next group: same row, a later row, or another matrix
-            uint32_t ne = e + 256u, nr = r, nc = c + 256u;
-            int nm = m;
-            if (more) {
-                if (ne >= mlast) {
-                    nm = gemv_matrix_of(gp, ne);
-                    const uint32_t o = ne - gp->m[nm].start;
-                    nr = o / gp->m[nm].cols;
-                    nc = o - nr * gp->m[nm].cols;
-                } else {
-                    while (nc >= cols) {
-                        nc -= cols;
-                        ++nr;
+#pragma unroll
+                for (int u = 0; u < TP; ++u) {
+                    const int t = t0 + u;
+                    if (t < (int)nt) {
+                        const uint4 xv_t = xv[u];
+                        float a = acc[t];
+                        a = fmaf(w0, bf16_lo(xv_t.x), a);
+                        a = fmaf(w1, bf16_hi(xv_t.x), a);
+                        a = fmaf(w2, bf16_lo(xv_t.y), a);
+                        a = fmaf(w3, bf16_hi(xv_t.y), a);
+                        a = fmaf(w4, bf16_lo(xv_t.z), a);
+                        a = fmaf(w5, bf16_hi(xv_t.z), a);
+                        a = fmaf(w6, bf16_lo(xv_t.w), a);
+                        a = fmaf(w7, bf16_hi(xv_t.w), a);
+                        acc[t] = a;
                     }
                 }
             }
-            if (!more || nm != m || nr != r) {
-#pragma unroll
-                for (int t = 0; t < TT; ++t) {
-                    if (t < (int)nt)
-                        atomicAdd(y + (size_t)t * rows + r, acc[t]);
-                    acc[t] = 0.f;
-                }
-            }
-            if (!more)
-                break;
-            if (nm != m) {
-                m = nm;
-                cols = gp->m[m].cols;
-                rows = gp->m[m].rows;
-                mlast = gp->m[m].start + rows * cols;
-                x = gp->m[m].x;
-                y = gp->m[m].y;
-            }
-            e = ne;
-            r = nr;
-            c = nc;
         }
-    }
-    // partial groups at both ends, one element per lane
-    const uint32_t fs = gfirst * 8;
-    const uint32_t hend = min(fs, span);
-    const uint32_t tbeg = max(mend * 8, fs);
-    uint32_t l = 0xFFFFFFFFu;
-    if (lane < 8) {
-        if (head + lane < hend)
-            l = head + lane;
-    } else if (lane < 16) {
-        if (tbeg + (lane - 8) < span)
-            l = tbeg + (lane - 8);
-    }
-    if (l != 0xFFFFFFFFu) {
-        const uint32_t e = (uint32_t)base + l;
-        const int m = gemv_matrix_of(gp, e);
-        const uint32_t cols = gp->m[m].cols;
-        const uint32_t o = e - gp->m[m].start;
-        const uint32_t r = o / cols, c = o - r * cols;
-        const float wv = __uint_as_float((uint32_t)join1(lds_u8_m(ebuf_a + l), lds_u8_m(sgrp_a + l)) << 16);
-        for (uint32_t t = 0; t < nt; ++t)
-            atomicAdd(gp->m[m].y + (size_t)t * gp->m[m].rows + r,
-                      wv * __uint_as_float((uint32_t)gp->m[m].x[(size_t)t * cols + c] << 16));
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+            float a = acc[t];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
+            if (lane == 0 && t < (int)nt)
+                atomicAdd(ym + (size_t)t * rows + r, a);
+        }
+        if (gend >= ngroups)
+            break;
+        // the next row, or the first row of the next matrix
+        g = gend;
+        c = 0;
+        if (++r == rows) {
+            ++m;
+            cols = gp->m[m].cols;
+            rows = gp->m[m].rows;
+            xm = gp->m[m].x;
+            ym = gp->m[m].y;
+            r = 0;
+        }
     }
 }
 
@@ -764,7 +772,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             }
             if constexpr (TT > 0) {
                 if (!stalled)
-                    gemv_chunk<TT>(gp, head, n_write, base, gfirst, lane, ebuf_a, sbuf_a + (pos0 & 8u));
+                    gemv_chunk<TT>(gp, head, n_write, base, lane, ebuf_a, sbuf_a + (pos0 & 8u));
             }
             __syncwarp();
         }

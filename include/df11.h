@@ -245,7 +245,10 @@ df11_status df11_decompress_async_ctas(const df11_device_block *blk, uint16_t *o
  * with x device BF16 (n_tokens x cols, token-major, 16-byte aligned) and y
  * device FP32 (n_tokens x rows, 4-byte aligned, zeroed by the caller: the
  * kernel accumulates into it with atomic adds, so the summation order and
- * the last bits of y vary between runs).  Products and sums are FP32. */
+ * the last bits of y vary between runs).  Products and sums are FP32.  The
+ * activations should be finite: a chunk's end groups multiply the
+ * neighbouring chunk's columns by +0, so an infinite x entry can turn an
+ * infinite y into NaN. */
 typedef struct {
     uint64_t rows;
     uint64_t cols;
