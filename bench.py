@@ -80,6 +80,9 @@ def parse_args():
                     help="steps of the end-to-end measurement (capped at --steps)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 256 MB buffer before every timed launch and time each launch "
+                         "alone (for blocks whose working set fits in the 126 MB L2)")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -340,16 +343,31 @@ def run_b200(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    end.record(stream)
-    end.synchronize()
+    if args.flush_l2:
+        # every launch starts from an L2 holding none of its data; only the
+        # launches are timed (one event pair each)
+        scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            scrub.fill_(1)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs)
+        del scrub
+    else:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        end.synchronize()
+        ms = start.elapsed_time(end)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    ms = start.elapsed_time(end)
 
     # ---- end to end: pinned host arrays -> device, decode, BF16 -> host
     e2e = None
@@ -414,8 +432,11 @@ def run_b200(args):
                    "seed": seed, "threads_per_chunk": 32, "bytes_per_thread": args.bytes_per_thread,
                    "bits_per_weight": round(8 + cb.total_bits / n, 4),
                    "compressed_bytes": comp_bytes, "bytes_per_step": bytes_per_step,
-                   "l2": "inputs larger than L2 (%.2f GB touched per step vs 126 MB L2), no flush"
-                         % (bytes_per_step / 1e9),
+                   "l2": ("L2 flushed (256 MB written) before every timed launch, launches timed alone"
+                          if args.flush_l2 else
+                          "%s (%.3f GB touched per step vs 126 MB L2), no flush"
+                          % ("inputs larger than L2" if bytes_per_step > 126e6 else
+                             "working set fits in L2: an L2-resident figure", bytes_per_step / 1e9)),
                    "parallelism": f"replicas x{world}, one block per GPU, no collective"},
         "gweights_per_s": round(job_rate(job_weights, args.steps, ms_max), 2),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
