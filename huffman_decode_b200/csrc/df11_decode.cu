@@ -32,7 +32,14 @@
 //     permutes and writes one 16-byte vector per lane and group;
 //   * persistent CTAs of up to 32 warps (as many as shared memory holds;
 //     one CTA per SM for typical blocks, so all warps of an SM share one
-//     copy of the tables): grid = resident CTAs per SM x SM count.
+//     copy of the tables): grid = resident CTAs per SM x SM count;
+//   * with a scheduling workspace, the last few rounds of chunks are not
+//     dealt out but claimed one at a time from four global counters (each
+//     warp claims a chunk ahead, so the atomic's latency hides behind a
+//     decode): warps and SMs that ran slower take fewer of them and all
+//     finish within about one chunk of each other.  Claiming only the tail
+//     keeps the atomics off the memory system for most of the launch.  The
+//     last CTA out resets the counters.
 // No tensor cores: this is integer decode, bounded by HBM traffic and issue.
 #include "df11.h"
 
@@ -66,7 +73,16 @@ struct DecodeParams {
     uint32_t n_tables;
     uint32_t min_len;     // shortest legal code; shorter table entries are corrupt
     uint32_t full_chunks; // chunks lying wholly below total_bits (every slice full)
+    uint32_t *sched;      // scheduling workspace, zero between launches; or null
 };
+// Scheduling workspace: claim counter q at word q * kSchedStride (pools on
+// separate 256-byte stretches, so on different L2 lines), CTAs done at word
+// kSchedDoneWord.
+constexpr int kSchedPools = 4;
+constexpr int kSchedStride = 64;
+constexpr int kSchedDoneWord = kSchedPools * kSchedStride;
+constexpr int kSchedTailRounds = 3;   // rounds of chunks left to claiming
+static_assert((kSchedDoneWord + 1) * 4 <= DF11_SCHED_WORKSPACE_BYTES, "workspace too small");
 
 // Decode fused with a matrix-vector product: every matrix of the block is
 // multiplied by n_tokens activation rows as it is decoded, and the BF16
@@ -475,6 +491,33 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     // so every decode step advances by at least min_len bits
     const uint32_t no_code = 0x4000u | (min_len << 8);
 
+    // ---- this warp's first chunk: its loads overlap the table build ---------
+    const uint64_t n_warps = (uint64_t)gridDim.x * warps;
+    const uint64_t gw = (uint64_t)blockIdx.x * warps + warp;
+    uint64_t chunk = gw;
+    // Rounds below r_static are dealt out: chunk gw + k n_warps is this
+    // warp's k-th.  With a workspace, chunks from d0 on are claimed: pool q
+    // holds d0 + q, d0 + q + 4, ..., and warp gw claims from pool gw % 4.
+    // Blocks of fewer rounds keep the plain deal: their imbalance is the
+    // rounding of chunks to warps, which claiming cannot remove.
+    const uint64_t rounds = p.n_chunks / n_warps;
+    const uint64_t r_static = rounds - kSchedTailRounds;
+    const uint64_t d0 = r_static * n_warps;
+    const bool dyn = p.sched != nullptr && rounds >= (uint64_t)kSchedTailRounds + 2;
+    const uint32_t q = (uint32_t)(gw % kSchedPools);
+    uint32_t *const pool = p.sched + q * kSchedStride;
+    uint32_t claim = 0;   // lane 0: the last claim's result
+    uint32_t w[G::kWords];
+    uint32_t gap = 0, pos0 = 0, pos1 = 0;
+#pragma unroll
+    for (int k = 0; k < G::kWords; ++k)
+        w[k] = 0;
+    if (chunk < p.n_chunks) {
+        load_slice<W>(p, chunk * 32 + lane, w, gap);
+        pos0 = p.chunk_pos[chunk];
+        pos1 = p.chunk_pos[chunk + 1];
+    }
+
     // ---- prologue: two-level tables, sanitised ------------------------------
     // Anything malformed (bad pointer, bad length, shorter than the shortest
     // code) becomes "no code", so decoding never indexes outside the tables
@@ -506,8 +549,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     // the first code is longer than the window (or is no code) the entry is
     // x = 0, y = kLongStep: adding it ends the lookup loop, and the decoder
     // takes the two-level path.
-    for (int idx = tid; idx < kMultiEntries; idx += blockDim.x) {
-        const uint32_t win = (uint32_t)idx << (32 - kWindowBits);   // MSB-first window
+    for (int slot = tid; slot < kMultiEntries; slot += blockDim.x) {
+        // consecutive threads fill consecutive entries (conflict-free stores)
+        const uint32_t idx = __brev((uint32_t)slot) >> (32 - kWindowBits);
+        const uint32_t win = idx << (32 - kWindowBits);   // MSB-first window
         uint32_t t = 0, n = 0, syms = 0;
         while (n < kMaxCodesPerEntry) {
             const uint32_t v = win << t;
@@ -523,7 +568,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             ++n;
             t += l;
         }
-        multi[__brev((uint32_t)idx) >> (32 - kWindowBits)] = make_uint2(syms, n ? t | (8u * n << 16) : kLongStep);
+        multi[slot] = make_uint2(syms, n ? t | (8u * n << 16) : kLongStep);
     }
     __syncthreads();
 
@@ -539,17 +584,12 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     const uint32_t bar = smem_addr(&mbar[warp]);
     uint32_t parity = 0;
 
-    const uint64_t stride = (uint64_t)gridDim.x * warps;
-    uint64_t chunk = (uint64_t)blockIdx.x * warps + warp;
-    if (chunk >= p.n_chunks)
+    if (chunk >= p.n_chunks)   // (never with the dynamic schedule)
         return;
 
     uint32_t err = 0;
     bool stalled = false;      // a staged copy did not arrive in time
-    uint32_t w[G::kWords];
-    uint32_t gap;
-    load_slice<W>(p, chunk * 32 + lane, w, gap);
-    uint32_t pos0 = p.chunk_pos[chunk], pos1 = p.chunk_pos[chunk + 1];
+    uint64_t k = 0;            // chunks this warp has finished
 
     for (;;) {
         // ---- positions (warp-uniform) and the staged sign|mantissa copy -----
@@ -565,7 +605,16 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             bulk_copy_g2s(sbuf_a, p.signmant + cp_lo, cp_bytes, bar);
 
         // ---- the next chunk's slice and positions, loaded ahead -------------
-        const uint64_t next = chunk + stride;
+        uint64_t next;
+        if (!dyn || k + 1 < r_static) {
+            next = chunk + n_warps;
+            if (dyn && k + 2 == r_static && lane == 0)
+                claim = atomicAdd(pool, 1u);      // the first claimed chunk, a chunk ahead
+        } else {
+            next = d0 + q + (uint64_t)kSchedPools * __shfl_sync(0xFFFFFFFFu, claim, 0);
+            if (lane == 0 && next < p.n_chunks)
+                claim = atomicAdd(pool, 1u);      // the chunk after next
+        }
         const bool has_next = next < p.n_chunks;
         uint32_t nw[G::kWords];
         uint32_t ngap = 0, npos0 = 0, npos1 = 0;
@@ -777,6 +826,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             __syncwarp();
         }
 
+        ++k;
         if (!has_next || stalled)
             break;
         chunk = next;
@@ -791,6 +841,23 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
         mbar_wait(bar, parity ^ 1u);
     if (err && p.err)
         atomicOr(p.err, err);
+    if (dyn) {
+        // a claim still in flight (after a stall) must land before the CTA
+        // counts itself out: the and waits for its result
+        uint32_t z = 0;
+        if (lane == 0)
+            asm volatile("and.b32 %0, %1, 0;" : "=r"(z) : "r"(claim));
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && atomicAdd(p.sched + kSchedDoneWord, 1u + z) == gridDim.x - 1) {
+            // every other CTA is out: ready for the next launch
+#pragma unroll
+            for (int i = 0; i < kSchedPools; ++i)
+                p.sched[i * kSchedStride] = 0;
+            p.sched[kSchedDoneWord] = 0;
+            __threadfence();
+        }
+    }
 }
 
 template <int W, int MINLEN>
@@ -969,6 +1036,7 @@ df11_status block_params(const df11_device_block *blk, uint16_t *out_bf16, uint6
     prm.n_tables = h.n_tables;
     prm.min_len = h.min_code_len;
     prm.full_chunks = (uint32_t)(h.total_bits / chunk_bits);
+    prm.sched = nullptr;
     return DF11_OK;
 }
 
@@ -978,13 +1046,21 @@ extern "C" df11_status df11_decompress_async_ctas(const df11_device_block *blk, 
                                                   uint64_t out_capacity, uint32_t *d_error,
                                                   uint32_t max_ctas, void *stream)
 {
-    if (!out_bf16)
+    return df11_decompress_async_ws(blk, out_bf16, out_capacity, d_error, max_ctas, nullptr, stream);
+}
+
+extern "C" df11_status df11_decompress_async_ws(const df11_device_block *blk, uint16_t *out_bf16,
+                                                uint64_t out_capacity, uint32_t *d_error,
+                                                uint32_t max_ctas, void *workspace, void *stream)
+{
+    if (!out_bf16 || !aligned(workspace, 16))
         return DF11_ERR_INVALID_ARGUMENT;
     DecodeParams prm;
     int dev = 0;
     const df11_status st = block_params(blk, out_bf16, out_capacity, d_error, prm, dev);
     if (st != DF11_OK)
         return st;
+    prm.sched = static_cast<uint32_t *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (blk->hdr.bytes_per_thread == 8)
         return prm.min_len >= 2 ? launch<8, 2>(prm, dev, s, max_ctas) : launch<8, 1>(prm, dev, s, max_ctas);
@@ -993,9 +1069,10 @@ extern "C" df11_status df11_decompress_async_ctas(const df11_device_block *blk, 
 
 extern "C" df11_status df11_decode_gemv_async(const df11_device_block *blk, const df11_gemv_matrix *mats,
                                               uint32_t n_mats, uint32_t n_tokens, uint32_t *d_error,
-                                              void *stream)
+                                              void *workspace, void *stream)
 {
-    if (!blk || !mats || n_mats == 0 || n_mats > (uint32_t)kGemvMaxMats || n_tokens == 0 || n_tokens > 8)
+    if (!blk || !mats || n_mats == 0 || n_mats > (uint32_t)kGemvMaxMats || n_tokens == 0 || n_tokens > 8 ||
+        !aligned(workspace, 16))
         return DF11_ERR_INVALID_ARGUMENT;
     GemvParams gp;
     gp.n_mats = n_mats;
@@ -1028,6 +1105,7 @@ extern "C" df11_status df11_decode_gemv_async(const df11_device_block *blk, cons
     if (st != DF11_OK)
         return st;
     prm.out = nullptr;
+    prm.sched = static_cast<uint32_t *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (blk->hdr.bytes_per_thread == 8)
         return prm.min_len >= 2 ? launch_gemv_tokens<8, 2>(prm, gp, dev, s) : launch_gemv_tokens<8, 1>(prm, gp, dev, s);

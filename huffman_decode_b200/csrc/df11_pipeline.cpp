@@ -33,6 +33,7 @@ struct df11_pipeline {
     cudaEvent_t *uploaded;
     cudaEvent_t *decoded;
     cudaEvent_t *released;
+    uint8_t *sched;   // one decode scheduling workspace per slot (zeroed)
 };
 
 namespace {
@@ -101,12 +102,23 @@ extern "C" df11_status df11_pipeline_create(uint32_t n_slots, df11_pipeline **ou
     p->uploaded = create_events(n_slots);
     p->decoded = p->uploaded ? create_events(n_slots) : nullptr;
     p->released = p->decoded ? create_events(n_slots) : nullptr;
-    if (!p->released) {
+    // decodes of one slot are ordered by its events; different slots may
+    // decode concurrently, so each has its own workspace
+    void *ws = nullptr;
+    if (p->released && (cudaMalloc(&ws, (size_t)n_slots * DF11_SCHED_WORKSPACE_BYTES) != cudaSuccess ||
+                        cudaMemset(ws, 0, (size_t)n_slots * DF11_SCHED_WORKSPACE_BYTES) != cudaSuccess)) {
+        if (ws)
+            cudaFree(ws);
+        ws = nullptr;
+    }
+    if (!ws) {
         destroy_events(p->uploaded, n_slots);
         destroy_events(p->decoded, n_slots);
+        destroy_events(p->released, n_slots);
         delete p;
         return DF11_ERR_CUDA;
     }
+    p->sched = static_cast<uint8_t *>(ws);
     *out = p;
     return DF11_OK;
 }
@@ -118,6 +130,7 @@ extern "C" df11_status df11_pipeline_destroy(df11_pipeline *p)
     destroy_events(p->uploaded, p->n_slots);
     destroy_events(p->decoded, p->n_slots);
     destroy_events(p->released, p->n_slots);
+    cudaFree(p->sched);
     delete p;
     return DF11_OK;
 }
@@ -163,7 +176,8 @@ extern "C" df11_status df11_pipeline_decode(df11_pipeline *p, uint32_t slot, con
     if (cudaStreamWaitEvent(s, p->uploaded[slot], 0) != cudaSuccess ||
         cudaStreamWaitEvent(s, p->released[slot], 0) != cudaSuccess)
         return DF11_ERR_CUDA;
-    const df11_status st = df11_decompress_async_ctas(blk, out_bf16, out_capacity, d_error, max_ctas, s);
+    const df11_status st = df11_decompress_async_ws(blk, out_bf16, out_capacity, d_error, max_ctas,
+                                                    p->sched + (size_t)slot * DF11_SCHED_WORKSPACE_BYTES, s);
     if (st != DF11_OK)
         return st;
     return cudaEventRecord(p->decoded[slot], s) == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;

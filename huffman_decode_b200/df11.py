@@ -47,8 +47,9 @@ EXPORTED_SYMBOLS = (
     "df11_pipeline_destroy", "df11_pipeline_upload", "df11_pipeline_decode", "df11_pipeline_acquire",
     "df11_pipeline_release", "df11_checksum_count", "df11_crc32c", "df11_checksum",
     "df11_checksum_device_async", "df11_verify_device_async", "df11_pipeline_verify",
-    "df11_decode_gemv_async",
+    "df11_decode_gemv_async", "df11_decompress_async_ws",
 )
+SCHED_WORKSPACE_BYTES = 2048
 CRC_SEGMENT_BYTES = 4096
 NOALLOC_SCRATCH_BYTES = 1 << 20
 NOALLOC_MAX_ELEMENTS = 715816960
@@ -166,7 +167,8 @@ def load_library(path: str | None = None):
         ("df11_checksum_device_async", S, [P, P, U64, P]),
         ("df11_verify_device_async", S, [P, P, U64, P, P, P]),
         ("df11_pipeline_verify", S, [P, U32, P, P, U64, P, P, P]),
-        ("df11_decode_gemv_async", S, [P, P, U32, U32, P, P]),
+        ("df11_decode_gemv_async", S, [P, P, U32, U32, P, P, P]),
+        ("df11_decompress_async_ws", S, [P, P, U64, P, U32, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -361,33 +363,55 @@ class DeviceBlock:
         return DeviceBlock(header=Header(), tensors=t, sizes={n: int(b) for n, b in sizes.items()})
 
 
-def decompress_async(db: DeviceBlock, out, error=None, stream=None, c_block=None,
-                     capacity: int | None = None, max_ctas: int = 0) -> None:
-    """df11_decompress_async: one kernel launch decoding the whole block into
-    `out` (a CUDA tensor of >= n_elements 16-bit elements, e.g. bfloat16 or
-    int16) on `stream` (torch.cuda.Stream, raw handle, or the current stream).
-    `error` is an optional int32 CUDA tensor the kernel ORs error bits into;
-    `capacity` (default out.numel()) is the element count the kernel may write;
-    `max_ctas` > 0 caps the launch (df11_decompress_async_ctas)."""
+_WORKSPACES: dict = {}
+
+
+def sched_workspace(device, stream_handle: int):
+    """The scheduling workspace this module uses for launches on one stream
+    (DF11_SCHED_WORKSPACE_BYTES of zeroed device memory, created on first
+    use).  Launches on one stream run one after another, so they can share
+    it; launches on different streams get different workspaces."""
     import torch
-    if stream is None:
-        handle = torch.cuda.current_stream(out.device).cuda_stream
-    elif isinstance(stream, int):
-        handle = stream
-    else:
-        handle = stream.cuda_stream
+    dev = torch.device(device)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device(), int(stream_handle))
+    ws = _WORKSPACES.get(key)
+    if ws is None:
+        ws = torch.zeros(SCHED_WORKSPACE_BYTES, dtype=torch.uint8, device=torch.device("cuda", key[0]))
+        _WORKSPACES[key] = ws
+    return ws
+
+
+def _workspace_ptr(workspace, device, handle):
+    """True: this stream's workspace; False/None: static chunk schedule; a
+    tensor: that workspace."""
+    if workspace is True:
+        return sched_workspace(device, handle).data_ptr()
+    if workspace is None or workspace is False:
+        return None
+    if workspace.numel() * workspace.element_size() < SCHED_WORKSPACE_BYTES or not workspace.is_cuda:
+        raise ValueError(f"workspace must be >= {SCHED_WORKSPACE_BYTES} bytes of CUDA memory")
+    return workspace.data_ptr()
+
+
+def decompress_async(db: DeviceBlock, out, error=None, stream=None, c_block=None,
+                     capacity: int | None = None, max_ctas: int = 0, workspace=True) -> None:
+    """df11_decompress_async_ws: one kernel launch decoding the whole block
+    into `out` (a CUDA tensor of >= n_elements 16-bit elements, e.g. bfloat16
+    or int16) on `stream` (torch.cuda.Stream, raw handle, or the current
+    stream).  `error` is an optional int32 CUDA tensor the kernel ORs error
+    bits into; `capacity` (default out.numel()) is the element count the
+    kernel may write; `max_ctas` > 0 caps the launch; `workspace` (default:
+    one per stream) selects the dynamic chunk schedule, False the static
+    one."""
     if out.element_size() != 2 or not out.is_cuda or not out.is_contiguous():
         raise ValueError("out must be a contiguous CUDA tensor of 16-bit elements")
+    handle = _raw_stream(stream, out.device)
     blk = c_block if c_block is not None else db.c_struct()
     err_ptr = error.data_ptr() if error is not None else None
     cap = out.numel() if capacity is None else min(int(capacity), out.numel())
-    if max_ctas:
-        _check(load_library().df11_decompress_async_ctas(ctypes.byref(blk), out.data_ptr(), cap,
-                                                         err_ptr, int(max_ctas), handle),
-               "df11_decompress_async_ctas")
-    else:
-        _check(load_library().df11_decompress_async(ctypes.byref(blk), out.data_ptr(), cap,
-                                                    err_ptr, handle), "df11_decompress_async")
+    _check(load_library().df11_decompress_async_ws(ctypes.byref(blk), out.data_ptr(), cap, err_ptr,
+                                                   int(max_ctas), _workspace_ptr(workspace, out.device, handle),
+                                                   handle), "df11_decompress_async_ws")
 
 
 # ------------------------------------------------------- GPU-side compressor
@@ -629,11 +653,12 @@ class GemvMatrix(ctypes.Structure):
                 ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
 
 
-def decode_gemv_async(db: "DeviceBlock", shapes, xs, ys, error=None, stream=None) -> None:
+def decode_gemv_async(db: "DeviceBlock", shapes, xs, ys, error=None, stream=None, workspace=True) -> None:
     """df11_decode_gemv_async: for matrix i of the block, shapes[i] = (rows,
     cols), adds xs[i] (n_tokens x cols, 16-bit CUDA tensor of BF16 bits)
     times W_i^T into ys[i] (n_tokens x rows, float32 CUDA tensor, zeroed by
-    the caller), decoding the block once and never writing it in BF16."""
+    the caller), decoding the block once and never writing it in BF16.
+    `workspace` as for decompress_async."""
     n = len(shapes)
     if len(xs) != n or len(ys) != n or n == 0:
         raise ValueError("one x and one y per matrix")
@@ -647,6 +672,7 @@ def decode_gemv_async(db: "DeviceBlock", shapes, xs, ys, error=None, stream=None
         arr[i] = GemvMatrix(int(r), int(c), x.data_ptr(), y.data_ptr())
     b = db.c_struct()
     err_ptr = error.data_ptr() if error is not None else None
+    handle = _raw_stream(stream, xs[0].device)
     _check(load_library().df11_decode_gemv_async(ctypes.byref(b), arr, n, n_tokens, err_ptr,
-                                                 _raw_stream(stream, xs[0].device)),
+                                                 _workspace_ptr(workspace, xs[0].device, handle), handle),
            "df11_decode_gemv_async")

@@ -233,6 +233,28 @@ df11_status df11_decompress_async_ctas(const df11_device_block *blk, uint16_t *o
                                        uint64_t out_capacity, uint32_t *d_error,
                                        uint32_t max_ctas, void *stream);
 
+/* Bytes of a scheduling workspace. */
+#define DF11_SCHED_WORKSPACE_BYTES 2048u
+
+/* GPU.  df11_decompress_async_ctas with a scheduling workspace: device
+ * memory of DF11_SCHED_WORKSPACE_BYTES, 16-byte aligned, all zero before
+ * its first use (cudaMemset once); the kernel leaves it zero when it
+ * completes.  Without one (NULL) warp k of the grid's W warps decodes
+ * chunks k, k + W, k + 2W, ...; with one, in a block of at least five such
+ * rounds the chunks of the last three are instead claimed one at a time by
+ * whichever warps get there first, so warps and SMs that ran faster take
+ * more of them and the launch ends within about one chunk time of its last
+ * claim.  Output is identical either way.
+ * (The pages leave the split of chunks over thread blocks open,
+ * "Architecture"; this is the library's choice.)  A workspace serves one
+ * launch at a time: launches that may run concurrently (different streams,
+ * or graphs replayed on different streams) need different workspaces, as
+ * with a cuBLAS workspace.  Same checks and errors as df11_decompress_async,
+ * plus INVALID_ARGUMENT for a misaligned workspace. */
+df11_status df11_decompress_async_ws(const df11_device_block *blk, uint16_t *out_bf16,
+                                     uint64_t out_capacity, uint32_t *d_error,
+                                     uint32_t max_ctas, void *workspace, void *stream);
+
 /* ---- Decode fused with its consumer: matrix-vector products --------------
  * The pages decode a block into a BF16 buffer and then run its matrix
  * products ("DFloat11: lossless BFloat16 compression", "Architecture":
@@ -256,13 +278,16 @@ typedef struct {
     float *y;
 } df11_gemv_matrix;
 
-/* GPU.  One launch on `stream`.  Errors: INVALID_ARGUMENT (the block checks
- * of df11_decompress_async, n_mats outside 1..128, n_tokens outside 1..8,
- * a matrix with cols not a multiple of 8 or misaligned pointers, or
- * matrices that do not add up to the block's elements), CUDA.  Device
- * errors go to *d_error as for df11_decompress_async. */
+/* GPU.  One launch on `stream`.  `workspace` is a scheduling workspace as
+ * for df11_decompress_async_ws, or NULL.  Errors: INVALID_ARGUMENT (the
+ * block checks of df11_decompress_async, n_mats outside 1..128, n_tokens
+ * outside 1..8, a matrix with cols not a multiple of 8 or misaligned
+ * pointers, matrices that do not add up to the block's elements, a
+ * misaligned workspace), CUDA.  Device errors go to *d_error as for
+ * df11_decompress_async. */
 df11_status df11_decode_gemv_async(const df11_device_block *blk, const df11_gemv_matrix *mats,
-                                   uint32_t n_mats, uint32_t n_tokens, uint32_t *d_error, void *stream);
+                                   uint32_t n_mats, uint32_t n_tokens, uint32_t *d_error,
+                                   void *workspace, void *stream);
 
 /* ---- GPU-side compressor --------------------------------------------------
  * The pages compress on the CPU only ("DFloat11: lossless BFloat16
@@ -395,11 +420,14 @@ df11_status df11_verify_device_async(const df11_device_block *blk, const uint32_
  * current at creation (else INVALID_ARGUMENT). */
 typedef struct df11_pipeline df11_pipeline;
 
-/* Host.  Creates a pipeline of n_slots (1..64) slots.  Errors:
- * INVALID_ARGUMENT, CUDA (no device or event creation failed). */
+/* Host.  Creates a pipeline of n_slots (1..64) slots, each with its own
+ * decode scheduling workspace (device memory, DF11_SCHED_WORKSPACE_BYTES a
+ * slot).  Errors: INVALID_ARGUMENT, CUDA (no device, or event creation or
+ * allocation failed). */
 df11_status df11_pipeline_create(uint32_t n_slots, df11_pipeline **out);
 
-/* Host.  Destroys the pipeline's events (work already enqueued still runs). */
+/* Host.  Destroys the pipeline's events and frees its workspaces; the free
+ * (cudaFree) waits for work already enqueued on the device. */
 df11_status df11_pipeline_destroy(df11_pipeline *p);
 
 /* Copy stage.  Enqueues on copy_stream the host -> device copies of src's
@@ -412,8 +440,8 @@ df11_status df11_pipeline_upload(df11_pipeline *p, uint32_t slot, const df11_hos
                                  const df11_device_block *dst, void *copy_stream);
 
 /* Decode stage.  Enqueues on decode_stream the slot's waits and
- * df11_decompress_async_ctas(blk, out_bf16, out_capacity, d_error, max_ctas),
- * then marks the slot decoded.  Errors: those of the decode call, and
+ * df11_decompress_async_ws(blk, out_bf16, out_capacity, d_error, max_ctas,
+ * the slot's workspace), then marks the slot decoded.  Errors: those of the decode call, and
  * INVALID_ARGUMENT for a bad pipeline, slot or device. */
 df11_status df11_pipeline_decode(df11_pipeline *p, uint32_t slot, const df11_device_block *blk,
                                  uint16_t *out_bf16, uint64_t out_capacity, uint32_t *d_error,

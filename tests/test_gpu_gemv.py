@@ -38,7 +38,7 @@ def _f64(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def run_and_check(mats, n_tokens, bytes_per_thread=16, seed=77):
+def run_and_check(mats, n_tokens, bytes_per_thread=16, seed=77, workspace=True):
     cb = df11.build_codebook(mats)
     hb = df11.compress(cb, mats, 32, bytes_per_thread)
     flat = np.concatenate([m.reshape(-1) for m in mats])
@@ -51,7 +51,7 @@ def run_and_check(mats, n_tokens, bytes_per_thread=16, seed=77):
     xs = [torch.from_numpy(x.view(np.int16)).cuda() for x in xs_host]
     ys = [torch.zeros(n_tokens, r, dtype=torch.float32, device="cuda") for r, _ in shapes]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    df11.decode_gemv_async(db, shapes, xs, ys, err)
+    df11.decode_gemv_async(db, shapes, xs, ys, err, workspace=workspace)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     for i, (m, x) in enumerate(zip(mats, xs_host)):
@@ -73,6 +73,14 @@ def run_and_check(mats, n_tokens, bytes_per_thread=16, seed=77):
 def test_llama_block_products(n_tokens, bpt):
     mats = [m for _, m in workloads.llama_block(3000, scale_div=64)]
     run_and_check(mats, n_tokens, bpt)
+
+
+@pytest.mark.parametrize("workspace", [True, False])
+def test_products_under_both_chunk_schedules(workspace):
+    """A block of over five rounds of chunks for a full wave of warps, so
+    with a workspace the last rounds really are claimed."""
+    mats = [m for _, m in workloads.llama_block(3002, scale_div=4)]
+    run_and_check(mats, 2, workspace=workspace)
 
 
 def test_flux_block_69_matrices():

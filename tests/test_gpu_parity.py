@@ -28,23 +28,23 @@ def _flat(mats):
     return np.concatenate([np.ascontiguousarray(m, dtype=np.uint16).reshape(-1) for m in mats])
 
 
-def gpu_decode(hb, capacity=None, guard=0, stream=None):
+def gpu_decode(hb, capacity=None, guard=0, stream=None, workspace=True):
     """Decode on cuda:0 into a buffer with `guard` extra elements set to a
     sentinel; returns (output incl. guard as uint16, error word)."""
     db = hb.to_device("cuda")
     n = hb.n_elements
     out = torch.full((n + guard,), 0x5A5A, dtype=torch.int16, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    df11.decompress_async(db, out, err, stream=stream, capacity=capacity)
+    df11.decompress_async(db, out, err, stream=stream, capacity=capacity, workspace=workspace)
     torch.cuda.synchronize()
     return out.cpu().numpy().view(np.uint16), int(err.item())
 
 
-def check_block(mats, bytes_per_thread=8, oracle_decode=True):
+def check_block(mats, bytes_per_thread=8, oracle_decode=True, workspace=True):
     w = _flat(mats)
     cb = df11.build_codebook(mats)
     hb = df11.compress(cb, mats, 32, bytes_per_thread)
-    got, err = gpu_decode(hb, guard=8)
+    got, err = gpu_decode(hb, guard=8, workspace=workspace)
     assert err == 0
     assert np.all(got[w.size:] == 0x5A5A), "wrote past the block"
     got = got[: w.size]
@@ -75,8 +75,58 @@ BPT = [8, 16]
 
 @pytest.mark.parametrize("name", sorted(SMALL))
 @pytest.mark.parametrize("bpt", BPT)
-def test_small_workloads(name, bpt):
-    check_block([m for _, m in SMALL[name]()], bytes_per_thread=bpt)
+@pytest.mark.parametrize("schedule", ["dynamic", "static"])
+def test_small_workloads(name, bpt, schedule):
+    check_block([m for _, m in SMALL[name]()], bytes_per_thread=bpt, workspace=schedule == "dynamic")
+
+
+# ------------------------------------------------------- chunk schedules
+
+@pytest.mark.parametrize("max_ctas", [0, 1, 7, 148, 1 << 20])
+def test_dynamic_schedule_leaves_workspace_zero(max_ctas):
+    """With a workspace, warps past their first chunk claim chunks from a
+    counter; every launch must decode every chunk exactly right and leave
+    the workspace zero for the next launch (any grid: one CTA, a partial
+    wave, waves of short-lived CTAs).  The block has over five rounds of
+    chunks for a full wave, so every grid but the largest claims chunks."""
+    mats = [m for _, m in workloads.llama_block(1000, scale_div=4)]
+    w = _flat(mats)
+    hb = df11.compress(df11.build_codebook(mats), mats)
+    db = hb.to_device("cuda")
+    ws = torch.zeros(df11.SCHED_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    out = torch.empty(hb.n_elements, dtype=torch.int16, device="cuda")
+    for rep in range(3):
+        out.fill_(0x5A5A)
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        df11.decompress_async(db, out, err, max_ctas=max_ctas, workspace=ws)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        assert np.array_equal(out.cpu().numpy().view(np.uint16), w), rep
+        assert int(ws.count_nonzero().item()) == 0, rep
+
+
+def test_schedules_agree_on_the_full_block():
+    mats = [m for _, m in workloads.llama_block(1000)]
+    w = _flat(mats)
+    hb = df11.compress(df11.build_codebook(mats), mats)
+    for workspace in (True, False):
+        got, err = gpu_decode(hb, workspace=workspace)
+        assert err == 0 and np.array_equal(got, w), workspace
+
+
+def test_dynamic_schedule_with_a_corrupt_block_still_resets():
+    """A block with a wrong chunk position: the error bit is set and the
+    workspace still ends zero, so the next (clean) launch is exact."""
+    mats = [m for _, m in workloads.llama_block(22, scale_div=4)]
+    hb = df11.compress(df11.build_codebook(mats), mats)
+    ws = torch.zeros(df11.SCHED_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    bad = df11.compress(df11.build_codebook(mats), mats)
+    bad.chunk_pos[bad.chunk_pos.size // 2] += 3
+    _, err = gpu_decode(bad, workspace=ws)
+    assert err & df11.DEVERR_COUNT
+    assert int(ws.count_nonzero().item()) == 0
+    got, err = gpu_decode(hb, workspace=ws)
+    assert err == 0 and np.array_equal(got, _flat(mats))
 
 
 @pytest.mark.parametrize("bpt", BPT)

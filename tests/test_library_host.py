@@ -310,6 +310,13 @@ def test_decompress_rejects_bad_arguments_before_any_cuda_call():
     assert lib.df11_decompress_async_ctas(None, fake, n, None, 8, None) == 1
     assert capped(dev_block(), cap=n - 1) == 1
     assert capped(dev_block(signmant=fake + 8)) == 1
+    # and so does the entry point with a scheduling workspace, which must
+    # also be 16-byte aligned
+    with_ws = lambda b, ws, cap=n: lib.df11_decompress_async_ws(ctypes.byref(b), fake, cap, None, 0, ws, None)
+    assert lib.df11_decompress_async_ws(None, fake, n, None, 0, fake, None) == 1
+    assert with_ws(dev_block(), fake + 4) == 1
+    assert with_ws(dev_block(), fake, cap=n - 1) == 1
+    assert with_ws(dev_block(exp_stream=fake + 8), fake) == 1
 
 
 def test_pipeline_rejects_bad_arguments_before_any_cuda_call():
@@ -462,7 +469,7 @@ def test_decode_gemv_rejects_bad_arguments_before_any_cuda_call():
             arr[i] = binding.GemvMatrix(r, c, x, y)
         return arr
 
-    call = lambda arr, n, t: lib.df11_decode_gemv_async(ctypes.byref(d), arr, n, t, None, None)
+    call = lambda arr, n, t, ws=None: lib.df11_decode_gemv_async(ctypes.byref(d), arr, n, t, None, ws, None)
     good = table(shapes)
     assert sum(r * c for r, c in shapes) == hb.n_elements
     assert call(good, len(shapes), 0) == 1                      # no tokens
@@ -474,4 +481,5 @@ def test_decode_gemv_rejects_bad_arguments_before_any_cuda_call():
     bad = list(shapes)
     bad[0] = (bad[0][0] * 2, bad[0][1] // 2 + 4)                # cols not a multiple of 8
     assert call(table(bad), len(bad), 1) == 1
-    assert lib.df11_decode_gemv_async(None, good, len(shapes), 1, None, None) == 1
+    assert lib.df11_decode_gemv_async(None, good, len(shapes), 1, None, None, None) == 1
+    assert call(good, len(shapes), 1, ws=fake + 8) == 1         # misaligned workspace
