@@ -49,6 +49,7 @@ struct EncodeParams {
     uint8_t *signmant;
     uint32_t *seg_bits;     // scratch: bits per segment
     uint64_t *seg_start;    // scratch: first bit per segment (exclusive scan)
+    uint16_t *grp_bits;     // scratch: bits per 32 elements of full segments, or null
     uint32_t *err;          // optional device error word
     uint64_t n;
     uint64_t n_seg;
@@ -90,10 +91,17 @@ __global__ void __launch_bounds__(256) histogram_kernel(const uint16_t *in, uint
 // ---- encode: per-thread code lengths -----------------------------------------
 
 // Loads this thread's up to 32 elements (zero past n) and returns their
-// bits; *bad is set when an element's exponent has no code.
+// bits: counted in the bit-count pass for a full segment when the scratch
+// holds the group counts, else here (*bad is then set when an element's
+// exponent has no code).
 __device__ __forceinline__ uint32_t load_elems(const EncodeParams &p, const uint32_t *len_tab,
                                                uint64_t e0, uint32_t (&w)[16], bool &bad)
 {
+    const uint64_t seg = e0 / kSegElems;
+    const bool counted = p.grp_bits != nullptr && (seg + 1) * kSegElems <= p.n;
+    uint32_t counted_bits = 0;
+    if (counted)
+        counted_bits = p.grp_bits[e0 / kElemsPerThread];
     if (e0 + kElemsPerThread <= p.n) {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.in + e0);
 #pragma unroll
@@ -113,6 +121,8 @@ __device__ __forceinline__ uint32_t load_elems(const EncodeParams &p, const uint
             w[k] = a | (b << 16);
         }
     }
+    if (counted)
+        return counted_bits;
     uint32_t bits = 0;
 #pragma unroll
     for (int k = 0; k < kElemsPerThread; ++k) {
@@ -159,8 +169,9 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
     return warp_tot[warp] + incl - v;
 }
 
-// Bits of every segment: one warp per segment (lane l sums the code lengths
-// of elements [256 l, 256 l + 256) of it), then a warp sum.
+// Bits of every segment: one warp per segment, whose lanes read it 512
+// contiguous bytes at a time (lane l takes bytes [16 l, 16 l + 16) of each),
+// then a warp sum.
 __global__ void __launch_bounds__(256) segment_bits_kernel(EncodeParams p, CodeTable ct)
 {
     __shared__ uint32_t len_tab[256];
@@ -171,24 +182,33 @@ __global__ void __launch_bounds__(256) segment_bits_kernel(EncodeParams p, CodeT
     bool bad = false;
     for (uint64_t seg = (uint64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); seg < p.n_seg;
          seg += warps) {
-        const uint64_t e0 = seg * kSegElems + (uint64_t)lane * (kSegElems / 32);
+        const uint64_t s0 = seg * kSegElems;
         uint32_t bits = 0;
-        if (e0 + kSegElems / 32 <= p.n) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.in + e0);
+        if (s0 + kSegElems <= p.n) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.in + s0) + lane;
 #pragma unroll 8
             for (int q = 0; q < kSegElems / 32 / 8; ++q) {
-                const uint4 v = src[q];
+                const uint4 v = src[32 * q];
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                uint32_t part = 0;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const uint32_t a = len_tab[(w4[k] >> 7) & 0xFFu];
                     const uint32_t b = len_tab[(w4[k] >> 23) & 0xFFu];
                     bad |= (a == 0) | (b == 0);
-                    bits += a + b;
+                    part += a + b;
+                }
+                bits += part;
+                if (p.grp_bits) {
+                    // lanes 4m .. 4m + 3 hold the 32 elements of group 8q + m
+                    part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
+                    part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
+                    if ((lane & 3) == 0)
+                        p.grp_bits[seg * (kSegElems / kElemsPerThread) + 8 * q + (lane >> 2)] = (uint16_t)part;
                 }
             }
         } else {
-            for (uint64_t i = e0; i < e0 + kSegElems / 32 && i < p.n; ++i) {
+            for (uint64_t i = s0 + lane; i < s0 + kSegElems && i < p.n; i += 32) {
                 const uint32_t l = len_tab[(p.in[i] >> 7) & 0xFFu];
                 bad |= l == 0;
                 bits += l;
@@ -275,17 +295,6 @@ __device__ __forceinline__ void red_or_shared_if(bool p, uint32_t a, uint32_t v)
                  : "memory");
 }
 
-// Stores v to the staged word at a when `full`: ORed in when `first` (the
-// word is shared with the previous thread), plainly otherwise.
-__device__ __forceinline__ void store_word_if(bool full, bool first, uint32_t a, uint32_t v)
-{
-    asm volatile(
-        "{ .reg .pred f, q, r; setp.ne.u32 f, %0, 0; setp.ne.u32 q, %1, 0; and.pred r, f, q;"
-        " @r red.shared.or.b32 [%2], %3; and.pred r, f, !q; @r st.shared.u32 [%2], %3; }" ::"r"((uint32_t)full),
-        "r"((uint32_t)first), "r"(a), "r"(v)
-        : "memory");
-}
-
 // Shared staging of one segment's output: stream words in bit order (bit 31
 // = first bit), and gap words (8 nibbles each, as in the gaps array).
 constexpr int kStageWords = kSegElems * 16 / 32 + 2;          // 16-bit codes at most
@@ -293,12 +302,12 @@ constexpr int kGapStageWords = kSegElems * 16 / 64 / 8 + 2;   // 64-bit slices a
 
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, CodeTable ct)
 {
-    __shared__ uint32_t code_tab[256];
+    __shared__ uint32_t code_tab[256];   // code | length << 24
     __shared__ uint32_t len_tab[256];
     __shared__ uint32_t warp_tot[kEncThreads / 32 + 1];
     __shared__ uint32_t sw[kStageWords];
     __shared__ uint32_t sg[kGapStageWords];
-    code_tab[threadIdx.x] = ct.e[threadIdx.x] & 0xFFFFFFu;
+    code_tab[threadIdx.x] = ct.e[threadIdx.x];
     len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
     for (int i = threadIdx.x; i < kStageWords; i += kEncThreads)
         sw[i] = 0;
@@ -324,69 +333,79 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
 
     if (e0 < p.n) {
         uint32_t lb = lb0 + off;                          // local bit of the next code
-        // local slice of the previous code start (none for element 0)
-        int32_t prev_gl = -0x40000000;
+        // First local bit of the slice after the one holding the previous
+        // code start (0 for element 0, or when that start lies before the
+        // segment's first slice): a code starting at or past it opens a slice.
+        uint32_t next_open = 0;
         if (e0 > 0) {
             const uint32_t lp = len_tab[(p.in[e0 - 1] >> 7) & 0xFFu];
-            prev_gl = (int32_t)((int64_t)((int64_t)lb - lp) >> sh);   // may be -1
+            if (lb >= lp)
+                next_open = (((lb - lp) >> sh) + 1) << sh;
         }
         const uint32_t goff = (uint32_t)(gS & 7u);
+        const uint32_t slice_mask = (1u << sh) - 1;
         uint32_t j = (uint32_t)(((S + off) >> 5) - wbase);   // staging word being filled
         uint32_t fill = (uint32_t)((S + off) & 31);          // its bits already placed
         uint32_t cur = 0;
-        bool first_word = true;
         const uint32_t cnt = (uint32_t)min((uint64_t)kElemsPerThread, p.n - e0);
         const uint32_t sw_a = (uint32_t)__cvta_generic_to_shared(sw);
-        const uint32_t sg_a = (uint32_t)__cvta_generic_to_shared(sg);
-        uint32_t prev = prev_gl < 0 ? 0xFFFFFFFFu : (uint32_t)prev_gl;
-        // One element: gap nibble of a slice its code opens, then the code
-        // MSB-first at bit `fill` of staged word j.  Branch-free apart from
-        // the rare chunk start; stores are predicated.
-        auto step = [&](uint32_t k) {
-            const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
-            const uint32_t sy = (x >> 7) & 0xFFu;
-            const uint32_t l = len_tab[sy];
-            const uint32_t c = code_tab[sy];
-            const uint32_t gl = lb >> sh;
-            const bool opens = gl != prev;
-            const uint32_t gi = gl + goff;                 // slice index relative to gbase * 8
-            red_or_shared_if(opens, sg_a + 4u * (gi >> 3), ((lb - (gl << sh)) & 0xFu) << ((gi & 7u) * 4));
-            if (opens && ((gS + gl) & (DF11_THREADS_PER_CHUNK - 1)) == 0)
-                p.chunk_pos[(gS + gl) / DF11_THREADS_PER_CHUNK] = (uint32_t)(e0 + k);
-            prev = gl;
+        // Two elements k, k + 1 (the second may be absent past the end):
+        // their codes joined into one of at most 32 bits, appended MSB-first
+        // at bit `fill` of staged word j (a full word is ORed into the
+        // staging: its first bits may be the previous thread's).  A slice one
+        // of the codes opens gets its gap nibble, and a chunk that starts
+        // there its output position (rare: a branch).  At most one of the
+        // two opens a slice: an opening code starts within 15 bits of its
+        // slice's start, so the next one starts within 31, short of the
+        // next slice (at least 64 bits on).
+        auto pair = [&](uint32_t k, bool second) {
+            const uint32_t x = w[k >> 1];                  // element k low, k + 1 high
+            const uint32_t ce1 = code_tab[(x >> 7) & 0xFFu];
+            const uint32_t ce2 = second ? code_tab[(x >> 23) & 0xFFu] : 0u;
+            const uint32_t l1 = ce1 >> 24, l2 = ce2 >> 24;
+            const uint32_t lb2 = lb + l1;                  // start of the second code
+            if ((second ? lb2 : lb) >= next_open) {
+                const bool by_first = lb >= next_open;
+                const uint32_t ob = by_first ? lb : lb2;
+                const uint32_t gl = ob >> sh;
+                const uint32_t gi = gl + goff;             // slice index relative to gbase * 8
+                atomicOr(&sg[gi >> 3], (ob & slice_mask & 0xFu) << ((gi & 7u) * 4));
+                if (((gS + gl) & (DF11_THREADS_PER_CHUNK - 1)) == 0)
+                    p.chunk_pos[(gS + gl) / DF11_THREADS_PER_CHUNK] = (uint32_t)(e0 + k + (by_first ? 0u : 1u));
+                next_open = (gl + 1) << sh;
+            }
+            const uint32_t l = l1 + l2;
             lb += l;
-            const uint32_t t = fill + l;
-            const uint64_t add = (uint64_t)c << ((64u - t) & 63u);
+            const uint32_t code = ((ce1 & 0xFFFFu) << l2) | (ce2 & 0xFFFFu);
+            const uint32_t t = fill + l;                   // <= 63: one word fills at most
+            const uint64_t add = (uint64_t)code << (64u - t);
             cur |= (uint32_t)(add >> 32);
             const bool full = t >= 32;
-            store_word_if(full, first_word, sw_a + 4u * j, cur);   // the first is shared: ORed
+            red_or_shared_if(full, sw_a + 4u * j, cur);
             cur = full ? (uint32_t)add : cur;
             j += full ? 1u : 0u;
             fill = full ? t - 32 : t;
-            first_word = first_word && !full;
         };
         if (cnt == kElemsPerThread) {
 #pragma unroll
-            for (uint32_t k = 0; k < kElemsPerThread; ++k)
-                step(k);
+            for (uint32_t k = 0; k < kElemsPerThread; k += 2)
+                pair(k, true);
         } else {
 #pragma unroll
-            for (uint32_t k = 0; k < kElemsPerThread; ++k) {
+            for (uint32_t k = 0; k < kElemsPerThread; k += 2) {
                 if (k >= cnt)
                     break;
-                step(k);
+                pair(k, k + 1 < cnt);
             }
         }
-        const int32_t prev_gl_end = prev == 0xFFFFFFFFu ? -1 : (int32_t)prev;
         if (fill)
             atomicOr(&sw[j], cur);                                // shared with the next thread
         // the end of the stream counts as a code start for the gap of its slice
         if (e0 + cnt == p.n) {
-            const int32_t gl = (int32_t)(lb >> sh);
-            if (gS + (uint64_t)gl < p.n_threads && gl != prev_gl_end) {
-                const uint32_t gapv = lb - ((uint32_t)gl << sh);
-                const uint32_t gi = (uint32_t)gl + goff;
-                atomicOr(&sg[gi >> 3], (gapv & 0xFu) << ((gi & 7u) * 4));
+            const uint32_t gl = lb >> sh;
+            if (gS + (uint64_t)gl < p.n_threads && lb >= next_open) {
+                const uint32_t gi = gl + goff;
+                atomicOr(&sg[gi >> 3], (lb & slice_mask & 0xFu) << ((gi & 7u) * 4));
             }
         }
         // sign|mantissa bytes
@@ -449,6 +468,19 @@ bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>
 
 uint64_t n_segments(uint64_t n) { return (n + kSegElems - 1) / kSegElems; }
 
+// Scratch: segment starts (8 bytes per segment) | segment bits (4 bytes per
+// segment, rounded to 16) | group bits (2 bytes per 32 elements of every
+// segment).  The allocation-free path goes without the group bits.
+uint64_t segment_scratch_bytes(uint64_t n)
+{
+    const uint64_t ns = n_segments(n);
+    return ns * 8 + ((ns * 4 + 15) & ~15ull);
+}
+
+df11_status compress_device_impl(const df11_codebook *cb, const df11_layout *layout, const uint16_t *d_in,
+                                 uint64_t n, df11_device_block *out, void *d_scratch, uint64_t scratch_bytes,
+                                 bool group_bits, uint32_t *d_error, void *stream);
+
 }  // namespace
 
 extern "C" {
@@ -470,14 +502,24 @@ df11_status df11_histogram_device(const uint16_t *d_in, uint64_t n, uint64_t *d_
 
 uint64_t df11_compress_device_scratch_bytes(uint64_t n_elements)
 {
-    const uint64_t ns = n_segments(n_elements);
-    return ns * 8 + ((ns * 4 + 15) & ~15ull);
+    return segment_scratch_bytes(n_elements) + n_segments(n_elements) * (kSegElems / kElemsPerThread) * 2;
 }
 
 df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *layout,
                                  const uint16_t *d_in, uint64_t n, df11_device_block *out,
                                  void *d_scratch, uint64_t scratch_bytes, uint32_t *d_error,
                                  void *stream)
+{
+    return compress_device_impl(cb, layout, d_in, n, out, d_scratch, scratch_bytes, true, d_error, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+df11_status compress_device_impl(const df11_codebook *cb, const df11_layout *layout, const uint16_t *d_in,
+                                 uint64_t n, df11_device_block *out, void *d_scratch, uint64_t scratch_bytes,
+                                 bool group_bits, uint32_t *d_error, void *stream)
 {
     if (!cb || !layout || !d_in || !out || !d_scratch)
         return DF11_ERR_INVALID_ARGUMENT;
@@ -489,7 +531,7 @@ df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *lay
     df11_status st = df11_compress_sizes(cb, layout, &z);
     if (st != DF11_OK)
         return st;
-    if (scratch_bytes < df11_compress_device_scratch_bytes(n))
+    if (scratch_bytes < (group_bits ? df11_compress_device_scratch_bytes(n) : segment_scratch_bytes(n)))
         return DF11_ERR_BUFFER_TOO_SMALL;
     if (!out->exp_stream || !out->gaps || !out->chunk_pos || !out->signmant)
         return DF11_ERR_INVALID_ARGUMENT;
@@ -511,6 +553,9 @@ df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *lay
     p.n_seg = n_segments(n);
     p.seg_start = reinterpret_cast<uint64_t *>(d_scratch);
     p.seg_bits = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(d_scratch) + p.n_seg * 8);
+    p.grp_bits = group_bits ? reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(d_scratch) +
+                                                           segment_scratch_bytes(n))
+                            : nullptr;
     p.err = d_error;
     p.n = n;
     p.total_bits = cb->total_bits;
@@ -549,7 +594,7 @@ df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *lay
     return DF11_OK;
 }
 
-}  // extern "C"
+}  // namespace
 
 // ---- allocation-free variant -------------------------------------------------
 // Some callers cannot let a library allocate device memory: a serving runtime
@@ -583,7 +628,7 @@ extern "C" df11_status df11_compress_device_noalloc(const df11_codebook *cb,
         return DF11_ERR_INVALID_ARGUMENT;
     if (n > DF11_NOALLOC_MAX_ELEMENTS)
         return DF11_ERR_BUFFER_TOO_SMALL;       // the fixed work space is too small
-    if (df11_compress_device_scratch_bytes(n) > kNoAllocScratchBytes)
+    if (segment_scratch_bytes(n) > kNoAllocScratchBytes)
         return DF11_ERR_BUFFER_TOO_SMALL;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
@@ -598,6 +643,6 @@ extern "C" df11_status df11_compress_device_noalloc(const df11_codebook *cb,
         addr = reinterpret_cast<uintptr_t>(ptr);
         g_noalloc_addr[dev].store(addr, std::memory_order_release);
     }
-    return df11_compress_device(cb, layout, d_in, n, out, reinterpret_cast<void *>(addr),
-                                kNoAllocScratchBytes, d_error, stream);
+    return compress_device_impl(cb, layout, d_in, n, out, reinterpret_cast<void *>(addr), kNoAllocScratchBytes,
+                                false, d_error, stream);
 }

@@ -302,8 +302,9 @@ df11_status df11_decode_gemv_async(const df11_device_block *blk, const df11_gemv
  * INVALID_ARGUMENT for null/misaligned pointers or n == 0, CUDA. */
 df11_status df11_histogram_device(const uint16_t *d_in, uint64_t n, uint64_t *d_hist, void *stream);
 
-/* Scratch bytes df11_compress_device needs for n elements (12 bytes per
- * 8192 elements, rounded up). */
+/* Scratch bytes df11_compress_device needs for n elements: 12 bytes per
+ * 8192 elements (rounded up) for the segment bit counts and starts, and 2
+ * bytes per 32 elements for the bit counts the encode pass reuses. */
 uint64_t df11_compress_device_scratch_bytes(uint64_t n_elements);
 
 /* GPU.  Encodes d_in[0 .. n) (device, the block's matrices concatenated,
