@@ -306,13 +306,14 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
     __shared__ uint32_t len_tab[256];
     __shared__ uint32_t warp_tot[kEncThreads / 32 + 1];
     __shared__ uint32_t sw[kStageWords];
-    __shared__ uint32_t sg[kGapStageWords];
+    __shared__ uint32_t sg[kGapStageWords * 2];   // one byte per slice's gap (plain byte stores)
     code_tab[threadIdx.x] = ct.e[threadIdx.x];
     len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
     for (int i = threadIdx.x; i < kStageWords; i += kEncThreads)
         sw[i] = 0;
-    for (int i = threadIdx.x; i < kGapStageWords; i += kEncThreads)
+    for (int i = threadIdx.x; i < kGapStageWords * 2; i += kEncThreads)
         sg[i] = 0;
+    uint8_t *const sgb = reinterpret_cast<uint8_t *>(sg);
     __syncthreads();
 
     const uint64_t seg = blockIdx.x;
@@ -326,9 +327,9 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
     const uint64_t wbase = S >> 5;                        // stream word of sw[0]
     const uint32_t sh = p.slice_shift;
     const uint64_t gS = S >> sh;                          // slice of the segment's first bit
-    const uint64_t gbase = gS >> 3;                       // gap word of sg[0]
+    const uint64_t gbase = gS >> 3;                       // gap word of staged slice 0
     // Positions below are local: lb = bit - (gS << sh), so the slice of a
-    // local bit is gS + (lb >> sh) and its staged gap word ((lb >> sh) + (gS & 7)) >> 3.
+    // local bit is gS + (lb >> sh) and its staged gap byte (lb >> sh) + (gS & 7).
     const uint32_t lb0 = (uint32_t)(S - (gS << sh));
 
     if (e0 < p.n) {
@@ -369,7 +370,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
                 const uint32_t ob = by_first ? lb : lb2;
                 const uint32_t gl = ob >> sh;
                 const uint32_t gi = gl + goff;             // slice index relative to gbase * 8
-                atomicOr(&sg[gi >> 3], (ob & slice_mask & 0xFu) << ((gi & 7u) * 4));
+                sgb[gi] = (uint8_t)(ob & slice_mask & 0xFu);
                 if (((gS + gl) & (DF11_THREADS_PER_CHUNK - 1)) == 0)
                     p.chunk_pos[(gS + gl) / DF11_THREADS_PER_CHUNK] = (uint32_t)(e0 + k + (by_first ? 0u : 1u));
                 next_open = (gl + 1) << sh;
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
             const uint32_t gl = lb >> sh;
             if (gS + (uint64_t)gl < p.n_threads && lb >= next_open) {
                 const uint32_t gi = gl + goff;
-                atomicOr(&sg[gi >> 3], (lb & slice_mask & 0xFu) << ((gi & 7u) * 4));
+                sgb[gi] = (uint8_t)(lb & slice_mask & 0xFu);
             }
         }
         // sign|mantissa bytes
@@ -456,10 +457,18 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
         const uint64_t gwords = p.n_threads / 8;                  // gaps array length in words
         uint32_t *gg = reinterpret_cast<uint32_t *>(p.gaps) + gbase;
         for (uint32_t i = threadIdx.x; i < ng && gbase + i < gwords; i += kEncThreads) {
+            // eight gap bytes (each < 16) -> eight nibbles, slice 8i + k at bits 4k
+            uint32_t v = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t x = sg[2 * i + h];
+                const uint32_t y = x | (x >> 4);                 // bytes 0, 2: two nibbles each
+                v |= ((y & 0xFFu) | ((y >> 8) & 0xFF00u)) << (16 * h);
+            }
             if (i == 0 || i == ng - 1)
-                atomicOr(gg + i, sg[i]);
+                atomicOr(gg + i, v);
             else
-                gg[i] = sg[i];
+                gg[i] = v;
         }
     }
 }
