@@ -16,9 +16,9 @@
 // of it.  A lane folds its bytes four at a time (x = crc ^ word; crc = x
 // advanced over four zero bytes, which is linear in x: four 256-entry table
 // lookups in a copy of the tables private to the lane, so the 32 lanes of a
-// warp never meet on a shared-memory bank), then advances its partial CRC over the bytes after its run, and
-// the warp XORs the 32 partials: CRC is linear, and crc(A || B) = crc(A)
-// advanced over |B| zero bytes, XOR crc(B).  "Advance over 2^j zero bytes"
+// warp never meet on a shared-memory bank).  The 32 partial CRCs are joined
+// in a five-level tree: CRC is linear, and crc(A || B) = crc(A) advanced
+// over |B| zero bytes, XOR crc(B).  "Advance over 2^j zero bytes"
 // is a table operator S_j (4 x 256 words) built in shared memory by
 // squaring S_{j-1}.  The initial value enters the same way: the standard CRC
 // of n bytes is the zero-initialised one XOR (0xFFFFFFFF advanced over n
@@ -194,6 +194,8 @@ __global__ void __launch_bounds__(kCrcThreads) crc_kernel(ArrayView av, uint32_t
 
     const int lane = tid & 31;
     const uint32_t *lane_priv = priv + lane;
+    // the initial value's part of a full segment's CRC
+    const uint32_t init_full = advance(ops + 12 * 1024, 0xFFFFFFFFu);
     const uint64_t warps = blockDim.x >> 5;
     const uint64_t total = av.first[5];
     for (uint64_t seg = blockIdx.x * warps + (tid >> 5); seg < total; seg += gridDim.x * warps) {
@@ -212,16 +214,16 @@ __global__ void __launch_bounds__(kCrcThreads) crc_kernel(ArrayView av, uint32_t
         const uint8_t *base = aptr + local * kSeg;
         const uint64_t rem = alen - local * kSeg;
         const uint32_t n = (uint32_t)(rem < kSeg ? rem : kSeg);
-        const uint32_t beg = (uint32_t)(kLaneBytes * lane);
-        const uint32_t end = beg < n ? min(n, beg + (uint32_t)kLaneBytes) : beg;
         uint32_t c = 0;
-        uint32_t q = beg;
-        if (end - beg == (uint32_t)kLaneBytes) {
-            // a full run: all eight loads in flight before folding
+        if (n == (uint32_t)kSeg) {
+            // a full segment: lane l folds bytes [128 l, 128 l + 128), all
+            // eight loads in flight first; then a five-level tree in which
+            // lanes 2^(j+1) i join the CRC of the 128 * 2^j bytes after
+            // their own (lane 0 ends with the segment's)
             uint4 v[kLaneBytes / 16];
 #pragma unroll
             for (int i = 0; i < kLaneBytes / 16; ++i)
-                v[i] = __ldg(reinterpret_cast<const uint4 *>(base + beg) + i);
+                v[i] = __ldg(reinterpret_cast<const uint4 *>(base + kLaneBytes * lane) + i);
 #pragma unroll
             for (int i = 0; i < kLaneBytes / 16; ++i) {
                 c = fold_word(lane_priv, c, v[i].x);
@@ -229,23 +231,33 @@ __global__ void __launch_bounds__(kCrcThreads) crc_kernel(ArrayView av, uint32_t
                 c = fold_word(lane_priv, c, v[i].z);
                 c = fold_word(lane_priv, c, v[i].w);
             }
-            q = end;
-        }
-        for (; q + 16 <= end; q += 16) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + q));
-            c = fold_word(lane_priv, c, v.x);
-            c = fold_word(lane_priv, c, v.y);
-            c = fold_word(lane_priv, c, v.z);
-            c = fold_word(lane_priv, c, v.w);
-        }
-        for (; q < end; ++q)
-            c = (c >> 8) ^ t0[(c ^ base[q]) & 0xFFu];
-        c = advance_by(ops, c, end > beg ? n - end : 0u);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            c ^= __shfl_xor_sync(0xFFFFFFFFu, c, o);
+            for (int j = 0; j < 5; ++j) {
+                const uint32_t right = __shfl_down_sync(0xFFFFFFFFu, c, 1 << j);
+                c = advance(ops + (7 + j) * 1024, c) ^ right;   // S_{7+j}: over 128 * 2^j zero bytes
+            }
+        } else {
+            // the short last segment of an array: lanes fold what they have,
+            // advance over the bytes after their run, and the warp XORs
+            const uint32_t beg = (uint32_t)(kLaneBytes * lane);
+            const uint32_t end = beg < n ? min(n, beg + (uint32_t)kLaneBytes) : beg;
+            uint32_t q = beg;
+            for (; q + 16 <= end; q += 16) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + q));
+                c = fold_word(lane_priv, c, v.x);
+                c = fold_word(lane_priv, c, v.y);
+                c = fold_word(lane_priv, c, v.z);
+                c = fold_word(lane_priv, c, v.w);
+            }
+            for (; q < end; ++q)
+                c = (c >> 8) ^ t0[(c ^ base[q]) & 0xFFu];
+            c = advance_by(ops, c, end > beg ? n - end : 0u);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                c ^= __shfl_xor_sync(0xFFFFFFFFu, c, o);
+        }
         if (lane == 0) {
-            const uint32_t crc = c ^ advance_by(ops, 0xFFFFFFFFu, n) ^ 0xFFFFFFFFu;
+            const uint32_t crc = c ^ (n == (uint32_t)kSeg ? init_full : advance_by(ops, 0xFFFFFFFFu, n)) ^ 0xFFFFFFFFu;
             if (out)
                 out[seg] = crc;
             if (expected && expected[seg] != crc) {
