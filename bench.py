@@ -55,14 +55,16 @@ def parse_args():
                     help="stream bytes each decoding thread owns (format layout)")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=sorted(workloads.WORKLOADS) + ["llama8b_model", "llama8b_overlap",
-                                                           "llama8b_offload", "llama8b_gemv"],
+                                                           "llama8b_offload", "llama8b_gemv",
+                                                           "llama8b_compress", "llama8b_verify"],
                     help="block to decode (the headline number is llama8b_block); "
                          "llama8b_model = 32 Llama-3.1-8B blocks, each with its own "
                          "codebook, decoded one after another into one buffer; "
                          "llama8b_overlap = those blocks decoded while the previous "
                          "block's matrix products run; llama8b_offload = blocks held "
                          "compressed in pinned host memory, uploaded and decoded in a "
-                         "pipeline")
+                         "pipeline; llama8b_compress = the GPU compressor on the block; "
+                         "llama8b_verify = the CRC-32C check of a resident block")
     ap.add_argument("--blocks", type=int, default=None,
                     help="blocks of the llama8b_model/overlap/offload streams "
                          "(default 32, 8 for offload)")
@@ -960,6 +962,150 @@ def run_gemv(args):
     return 0
 
 
+def _timed_steps(step, steps, warmup, stream, local):
+    """Warm-up, then `steps` back-to-back steps between two events on
+    `stream`, with clocks sampled meanwhile.  Returns (ms, clocks)."""
+    import torch
+    for _ in range(max(warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    e = _events(2)
+    sampler.start()
+    e[0].record(stream)
+    for _ in range(steps):
+        step()
+    e[1].record(stream)
+    e[1].synchronize()
+    clocks = sampler.stop()
+    return e[0].elapsed_time(e[1]), clocks
+
+
+def run_compress(args):
+    """The GPU compressor (1 GPU): one step is df11_histogram_device +
+    df11_compress_device of the Llama-3.1-8B-shaped block, drawn on the GPU and
+    resident in HBM.  The codebook comes from the histogram on the host (its
+    time is reported beside, not in the step; the pages build it on the CPU
+    too).  The output is checked byte for byte against the host compressor
+    and by a decode round trip.  Roofline: the method must read the BF16
+    block and write the compressed arrays (2 + ~1.33 B/weight)."""
+    import torch
+
+    import huffman_decode_b200 as df11
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    d_in = workloads.llama_block_device(1000, dev, scale_div=args.scale_div)
+    n = d_in.numel()
+    hist = df11.histogram_device(d_in)
+    t0 = time.perf_counter()
+    cb = df11.build_codebook_from_histogram(hist.cpu().numpy().astype(np.uint64))
+    cb_ms = 1e3 * (time.perf_counter() - t0)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    scratch = torch.empty(df11.compress_device_scratch_bytes(n), dtype=torch.uint8, device=dev)
+    db = df11.compress_device(cb, d_in, 32, args.bytes_per_thread, error=err, scratch=scratch)
+    out = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    df11.decompress_async(db, out)
+    torch.cuda.synchronize()
+    ok = int(err.item()) == 0 and bool(torch.equal(out.view(torch.int16), d_in))
+    hb = df11.compress(cb, [d_in.cpu().numpy().view(np.uint16)], 32, args.bytes_per_thread)
+    for name in ("exp_stream", "gaps", "chunk_pos", "signmant"):
+        a = db.tensors[name][: db.sizes[name]].cpu().numpy().view(np.uint8)
+        h = getattr(hb, name).view(np.uint8)
+        ok = ok and np.array_equal(a[: h.size], h) and not a[h.size:].any()
+    if not ok:
+        raise RuntimeError("GPU compressor output differs from the host compressor")
+    del out, hb
+
+    def step():
+        df11.histogram_device(d_in)
+        df11.compress_device(cb, d_in, 32, args.bytes_per_thread, error=err, scratch=scratch)
+
+    ms, clocks = _timed_steps(step, args.steps, args.warmup, stream, 0)
+    if int(err.item()):
+        raise RuntimeError("device error word set during the timed compression")
+    peak, peak_kind = measured_peaks()
+    comp = db.compressed_bytes()
+    alg = 2 * n + comp
+    step_s = ms / args.steps * 1e-3
+    line = {
+        "metric": "GPU compression of BF16 weights to DF11 (histogram + encode), BF16 GB/s in",
+        "value": round(2 * n / step_s / 1e9, 2), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8", "data": "synthetic (GPU-drawn, torch CUDA generator)",
+        "config": {"workload": "llama8b_compress", "n_weights": n, "seed": 1000,
+                   "threads_per_chunk": 32, "bytes_per_thread": args.bytes_per_thread,
+                   "compressed_bytes": comp, "l2": "inputs larger than L2, no flush"},
+        "byte_identical_to_host_compressor": True,
+        "host_codebook_ms": round(cb_ms, 3),
+        "roofline": {"bound": "hbm", "achieved": round(alg / step_s / 1e9, 2), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s",
+                     "frac": round(alg / step_s / 1e9 / peak, 4), "traffic": None,
+                     "algorithmic_bytes_per_step": alg},
+        "clocks": clocks,
+        "gpu_launches": 5 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_verify(args):
+    """The integrity check (1 GPU): one step is df11_verify_device_async over a
+    resident GPU-compressed Llama-3.1-8B-shaped block: the CRC-32C of every
+    4096-byte segment of its five arrays against the expected list.  The
+    list is checked against the host's (SSE4.2) list first.  Roofline: the
+    compressed bytes must be read once."""
+    import torch
+
+    import huffman_decode_b200 as df11
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    (db,), _, _ = gpu_compressed_blocks(1, 1000, dev, args.bytes_per_thread)
+    expected = df11.checksum_device(db)
+    names = ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")
+    host = {a: db.tensors[a][: db.sizes[a]].cpu().numpy() for a in names}
+    hb = df11.HostBlock(header=db.header, exp_stream=host["exp_stream"], gaps=host["gaps"],
+                        chunk_pos=host["chunk_pos"].view(np.uint32), signmant=host["signmant"],
+                        lut=host["lut"].view(np.uint16))
+    t0 = time.perf_counter()
+    host_list = df11.checksum(hb)
+    host_s = time.perf_counter() - t0
+    if not np.array_equal(expected.cpu().numpy().view(np.uint32), host_list):
+        raise RuntimeError("device checksum list differs from the host's")
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        df11.verify_device(db, expected, err, stream=stream)
+
+    ms, clocks = _timed_steps(step, args.steps, args.warmup, stream, 0)
+    if int(err.item()):
+        raise RuntimeError("verification failed on an intact block")
+    peak, peak_kind = measured_peaks()
+    comp = db.compressed_bytes()
+    step_s = ms / args.steps * 1e-3
+    line = {
+        "metric": "CRC-32C verification of a resident DF11 block (compressed GB/s checked)",
+        "value": round(comp / step_s / 1e9, 2), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8", "data": "synthetic (GPU-drawn, GPU-compressed)",
+        "config": {"workload": "llama8b_verify", "n_weights": db.n_elements, "seed": 1000,
+                   "segments": int(expected.numel()), "compressed_bytes": comp,
+                   "l2": "inputs larger than L2, no flush"},
+        "host_sse42_gbs": round(comp / host_s / 1e9, 2),
+        "roofline": {"bound": "hbm", "achieved": round(comp / step_s / 1e9, 2), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s",
+                     "frac": round(comp / step_s / 1e9 / peak, 4), "traffic": None,
+                     "algorithmic_bytes_per_step": comp},
+        "clocks": clocks,
+        "gpu_launches": args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -972,6 +1118,10 @@ def main():
         return run_offload(args)
     if args.workload == "llama8b_gemv":
         return run_gemv(args)
+    if args.workload == "llama8b_compress":
+        return run_compress(args)
+    if args.workload == "llama8b_verify":
+        return run_verify(args)
     return run_b200(args)
 
 
