@@ -460,7 +460,7 @@ def run_b200(args):
     return 0
 
 
-def gpu_compressed_blocks(n_blocks, seed0, dev, bpt, verify_into=None):
+def gpu_compressed_blocks(n_blocks, seed0, dev, bpt, verify_into=None, scale_div=1):
     """n_blocks Llama-3.1-8B-shaped blocks drawn on the GPU (seeds seed0..),
     each histogrammed, given its own codebook and compressed on the GPU.
     Every block is decoded once and compared with its input (bit-exact or an
@@ -475,7 +475,7 @@ def gpu_compressed_blocks(n_blocks, seed0, dev, bpt, verify_into=None):
     blocks, gpu_ms, host_cb_s = [], [], 0.0
     out = verify_into
     for b in range(n_blocks):
-        d_in = workloads.llama_block_device(seed0 + b, dev)
+        d_in = workloads.llama_block_device(seed0 + b, dev, scale_div=scale_div)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         ev[0].record(stream)
         hist = df11.histogram_device(d_in)
@@ -1062,7 +1062,7 @@ def run_verify(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
-    (db,), _, _ = gpu_compressed_blocks(1, 1000, dev, args.bytes_per_thread)
+    (db,), _, _ = gpu_compressed_blocks(1, 1000, dev, args.bytes_per_thread, scale_div=args.scale_div)
     expected = df11.checksum_device(db)
     names = ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")
     host = {a: db.tensors[a][: db.sizes[a]].cpu().numpy() for a in names}
