@@ -9,7 +9,7 @@ from .df11 import (  # noqa: F401
     CRC_SEGMENT_BYTES, DEVERR_BAD_CODE, DEVERR_BAD_POS, DEVERR_CHECKSUM, DEVERR_COUNT, DEVERR_MISMATCH,
     DEVERR_TIMEOUT, DF11Error, checksum, checksum_count, checksum_device, crc32c, verify_device,
     DeviceBlock, EXPORTED_SYMBOLS, LAYOUTS, HostBlock, PinnedHostBlock, Pipeline, build_codebook,
-    decode_gemv_async, SCHED_WORKSPACE_BYTES, sched_workspace,
+    decode_gemv_async, SCHED_WORKSPACE_BYTES, sched_workspace, decompress_range_async,
     build_codebook_from_histogram, compress, compress_device, compress_device_noalloc,
     compress_device_scratch_bytes,
     compress_sizes, decompress_async, histogram_device, library_path, load_library, validate,

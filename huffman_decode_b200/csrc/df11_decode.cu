@@ -1067,6 +1067,37 @@ extern "C" df11_status df11_decompress_async_ws(const df11_device_block *blk, ui
     return prm.min_len >= 2 ? launch<16, 2>(prm, dev, s, max_ctas) : launch<16, 1>(prm, dev, s, max_ctas);
 }
 
+extern "C" df11_status df11_decompress_range_async(const df11_device_block *blk, uint64_t chunk_begin,
+                                                   uint64_t chunk_end, uint16_t *out_bf16, uint64_t out_capacity,
+                                                   uint32_t *d_error, void *workspace, void *stream)
+{
+    if (!blk || !out_bf16 || !aligned(workspace, 16) || chunk_begin >= chunk_end ||
+        chunk_end > blk->hdr.n_chunks)
+        return DF11_ERR_INVALID_ARGUMENT;
+    DecodeParams prm;
+    int dev = 0;
+    const df11_status st = block_params(blk, out_bf16, out_capacity, d_error, prm, dev);
+    if (st != DF11_OK)
+        return st;
+    // The same launch over a block that starts at chunk_begin: chunks are
+    // independent given their gaps and positions, and positions (hence the
+    // sign|mantissa and output offsets) stay absolute.
+    const uint32_t W = blk->hdr.bytes_per_thread;
+    const uint64_t chunk_bits = (uint64_t)DF11_THREADS_PER_CHUNK * 8 * W;
+    prm.stream += chunk_begin * DF11_THREADS_PER_CHUNK * W;
+    prm.gaps += chunk_begin * (DF11_THREADS_PER_CHUNK / 2);
+    prm.chunk_pos += chunk_begin;
+    prm.total_bits -= chunk_begin * chunk_bits;
+    prm.n_chunks = chunk_end - chunk_begin;
+    const uint64_t full = prm.total_bits / chunk_bits;
+    prm.full_chunks = (uint32_t)(full < prm.n_chunks ? full : prm.n_chunks);
+    prm.sched = static_cast<uint32_t *>(workspace);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (W == 8)
+        return prm.min_len >= 2 ? launch<8, 2>(prm, dev, s, 0) : launch<8, 1>(prm, dev, s, 0);
+    return prm.min_len >= 2 ? launch<16, 2>(prm, dev, s, 0) : launch<16, 1>(prm, dev, s, 0);
+}
+
 extern "C" df11_status df11_decode_gemv_async(const df11_device_block *blk, const df11_gemv_matrix *mats,
                                               uint32_t n_mats, uint32_t n_tokens, uint32_t *d_error,
                                               void *workspace, void *stream)

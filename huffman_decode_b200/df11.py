@@ -47,7 +47,7 @@ EXPORTED_SYMBOLS = (
     "df11_pipeline_destroy", "df11_pipeline_upload", "df11_pipeline_decode", "df11_pipeline_acquire",
     "df11_pipeline_release", "df11_checksum_count", "df11_crc32c", "df11_checksum",
     "df11_checksum_device_async", "df11_verify_device_async", "df11_pipeline_verify",
-    "df11_decode_gemv_async", "df11_decompress_async_ws",
+    "df11_decode_gemv_async", "df11_decompress_async_ws", "df11_decompress_range_async",
 )
 SCHED_WORKSPACE_BYTES = 2048
 CRC_SEGMENT_BYTES = 4096
@@ -169,6 +169,7 @@ def load_library(path: str | None = None):
         ("df11_pipeline_verify", S, [P, U32, P, P, U64, P, P, P]),
         ("df11_decode_gemv_async", S, [P, P, U32, U32, P, P, P]),
         ("df11_decompress_async_ws", S, [P, P, U64, P, U32, P, P]),
+        ("df11_decompress_range_async", S, [P, U64, U64, P, U64, P, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -412,6 +413,22 @@ def decompress_async(db: DeviceBlock, out, error=None, stream=None, c_block=None
     _check(load_library().df11_decompress_async_ws(ctypes.byref(blk), out.data_ptr(), cap, err_ptr,
                                                    int(max_ctas), _workspace_ptr(workspace, out.device, handle),
                                                    handle), "df11_decompress_async_ws")
+
+
+def decompress_range_async(db: DeviceBlock, chunk_begin: int, chunk_end: int, out, error=None,
+                           stream=None, c_block=None, workspace=True) -> None:
+    """df11_decompress_range_async: decodes chunks [chunk_begin, chunk_end) of
+    the block into their part of `out` (the whole block's output buffer,
+    16-bit CUDA tensor); `workspace` as for decompress_async."""
+    if out.element_size() != 2 or not out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CUDA tensor of 16-bit elements")
+    handle = _raw_stream(stream, out.device)
+    blk = c_block if c_block is not None else db.c_struct()
+    err_ptr = error.data_ptr() if error is not None else None
+    _check(load_library().df11_decompress_range_async(ctypes.byref(blk), int(chunk_begin), int(chunk_end),
+                                                      out.data_ptr(), out.numel(), err_ptr,
+                                                      _workspace_ptr(workspace, out.device, handle), handle),
+           "df11_decompress_range_async")
 
 
 # ------------------------------------------------------- GPU-side compressor

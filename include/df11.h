@@ -255,6 +255,28 @@ df11_status df11_decompress_async_ws(const df11_device_block *blk, uint16_t *out
                                      uint64_t out_capacity, uint32_t *d_error,
                                      uint32_t max_ctas, void *workspace, void *stream);
 
+/* GPU.  Decodes only chunks [chunk_begin, chunk_end) of the block (chunk c =
+ * threads 32c .. 32c + 31, DF11_THREADS_PER_CHUNK * bytes_per_thread bytes of
+ * exp_stream): out_bf16[chunk_pos[chunk_begin] .. chunk_pos[chunk_end]) and
+ * nothing else.  Chunks are independent given their gaps and output
+ * positions ("Architecture": each thread block decodes its chunk alone), so
+ * a block can be decoded piece by piece as it arrives, for instance while
+ * the next piece is copied in and the last one copied out.  One launch reads
+ * only:
+ *   - exp_stream bytes [32 W chunk_begin, 32 W chunk_end + DF11_STREAM_PAD)
+ *     (W = bytes_per_thread);
+ *   - gaps bytes [16 chunk_begin, 16 chunk_end);
+ *   - chunk_pos[chunk_begin .. chunk_end];
+ *   - signmant bytes [p0 & ~15, (p1 + 15) & ~15), with p0 and p1 the
+ *     positions of chunk_begin and chunk_end;
+ *   - the tables.
+ * `workspace` as for df11_decompress_async_ws (may be NULL).  Errors: those
+ * of df11_decompress_async, and INVALID_ARGUMENT for an empty range or one
+ * past n_chunks, or a misaligned workspace. */
+df11_status df11_decompress_range_async(const df11_device_block *blk, uint64_t chunk_begin,
+                                        uint64_t chunk_end, uint16_t *out_bf16, uint64_t out_capacity,
+                                        uint32_t *d_error, void *workspace, void *stream);
+
 /* ---- Decode fused with its consumer: matrix-vector products --------------
  * The pages decode a block into a BF16 buffer and then run its matrix
  * products ("DFloat11: lossless BFloat16 compression", "Architecture":

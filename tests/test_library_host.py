@@ -317,6 +317,18 @@ def test_decompress_rejects_bad_arguments_before_any_cuda_call():
     assert with_ws(dev_block(), fake + 4) == 1
     assert with_ws(dev_block(), fake, cap=n - 1) == 1
     assert with_ws(dev_block(exp_stream=fake + 8), fake) == 1
+    # the chunk-range entry point: the same checks, and a non-empty range
+    # inside the block, all before any CUDA call
+    nch = int(hb.header.n_chunks)
+    rng = lambda b, c0, c1, ws=None: lib.df11_decompress_range_async(ctypes.byref(b), c0, c1, fake, n, None,
+                                                                     ws, None)
+    assert lib.df11_decompress_range_async(None, 0, 1, fake, n, None, None, None) == 1
+    assert rng(dev_block(), 0, 0) == 1
+    assert rng(dev_block(), 3, 2) == 1
+    assert rng(dev_block(), 0, nch + 1) == 1
+    assert rng(dev_block(), nch, nch + 1) == 1
+    assert rng(dev_block(), 0, 1, ws=fake + 8) == 1
+    assert rng(dev_block(exp_stream=fake + 8), 0, 1) == 1
 
 
 def test_pipeline_rejects_bad_arguments_before_any_cuda_call():
