@@ -81,6 +81,10 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=20,
                     help="steps of the end-to-end measurement (capped at --steps)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-pieces", type=int, default=8,
+                    help="end-to-end measurement: the block moves in this many chunk ranges, so "
+                         "the copy in of one overlaps the decode and the copy out of others "
+                         "(1 = copy everything in, decode, copy everything out)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 256 MB buffer before every timed launch and time each launch "
@@ -253,6 +257,60 @@ def cpu_baseline(oracle, hb, cb, bytes_per_weight, seconds):
                       f"{total_t:.1f} s"}
 
 
+def e2e_pipeline(df11, db, hb, host, out, host_out, err, host_err, pieces, stream, dev):
+    """One end-to-end step as a pipeline over `pieces` chunk ranges: range k
+    is copied in (its stream words, gaps, positions and sign|mantissa bytes)
+    on a copy-in stream, decoded on `stream` (df11_decompress_range_async)
+    and its BF16 output copied out on a copy-out stream, so the two PCIe
+    directions and the decode overlap.  The step ends on `stream`.  Returns
+    (step, host->device bytes, device->host bytes) per step."""
+    import torch
+    n_chunks = int(hb.header.n_chunks)
+    pieces = min(pieces, n_chunks)
+    W = 32 * int(hb.header.bytes_per_thread)
+    pos = hb.chunk_pos.astype(np.int64)
+    cuts = [n_chunks * i // pieces for i in range(pieces + 1)]
+    c_in, c_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cblk = db.c_struct()
+    plan = []
+    for c0, c1 in zip(cuts[:-1], cuts[1:]):
+        p0, p1 = int(pos[c0]), int(pos[c1])
+        spans = [("exp_stream", W * c0, min(W * c1 + 16, host["exp_stream"].numel())),
+                 ("gaps", 16 * c0, 16 * c1),
+                 ("chunk_pos", 4 * c0, 4 * (c1 + 1)),
+                 ("signmant", p0 & ~15, min((p1 + 15) & ~15, host["signmant"].numel()))]
+        plan.append((c0, c1, p0, p1, spans))
+    h2d = host["lut"].numel() + sum(b - a for *_, spans in plan for _, a, b in spans)
+    d2h = 2 * int(pos[-1]) + 4
+    ev_in = [torch.cuda.Event() for _ in plan]
+    ev_dec = [torch.cuda.Event() for _ in plan]
+    ev_start, ev_end = torch.cuda.Event(), torch.cuda.Event()
+
+    def step():
+        ev_start.record(stream)              # after the previous step, on every stream
+        c_in.wait_event(ev_start)
+        c_out.wait_event(ev_start)
+        with torch.cuda.stream(c_in):
+            db.tensors["lut"].copy_(host["lut"], non_blocking=True)
+            for i, (_, _, _, _, spans) in enumerate(plan):
+                for name, a, b in spans:
+                    db.tensors[name][a:b].copy_(host[name][a:b], non_blocking=True)
+                ev_in[i].record(c_in)
+        for i, (c0, c1, _, _, _) in enumerate(plan):
+            stream.wait_event(ev_in[i])
+            df11.decompress_range_async(db, c0, c1, out, err, stream=stream, c_block=cblk)
+            ev_dec[i].record(stream)
+        with torch.cuda.stream(c_out):
+            for i, (_, _, p0, p1, _) in enumerate(plan):
+                c_out.wait_event(ev_dec[i])
+                host_out[p0:p1].copy_(out[p0:p1], non_blocking=True)
+            host_err.copy_(err, non_blocking=True)
+            ev_end.record(c_out)
+        stream.wait_event(ev_end)
+
+    return step, h2d, d2h
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -323,7 +381,8 @@ def run_b200(args):
     db = hb.to_device(dev)
     out = torch.empty(n, dtype=torch.bfloat16, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    want = torch.from_numpy(np.concatenate([m.reshape(-1) for m in mats]).view(np.int16)).to(dev)
+    hb_bits = np.concatenate([m.reshape(-1) for m in mats]).view(np.int16)
+    want = torch.from_numpy(hb_bits).to(dev)
     stream = torch.cuda.current_stream(dev)
     cblk = db.c_struct()
 
@@ -377,19 +436,13 @@ def run_b200(args):
         k = max(1, min(args.e2e_steps, args.steps))
         host = {name: torch.from_numpy(a.view(np.uint8)).pin_memory() for name, a in hb.arrays().items()}
         host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
-        h2d = sum(t.numel() for t in host.values())
-        d2h = host_out.numel() * 2 + 4
         host_err = torch.empty(1, dtype=torch.int32, pin_memory=True)
-
-        def e2e_step():
-            for name, t in host.items():
-                db.tensors[name].copy_(t, non_blocking=True)
-            step()
-            host_out.copy_(out, non_blocking=True)
-            host_err.copy_(err, non_blocking=True)
-
+        e2e_step, h2d, d2h = e2e_pipeline(df11, db, hb, host, out, host_out, err, host_err,
+                                          max(1, args.e2e_pieces), stream, dev)
         e2e_step()
         torch.cuda.synchronize()
+        if not torch.equal(host_out.view(torch.int16), torch.from_numpy(hb_bits)) or int(host_err.item()):
+            raise RuntimeError("end-to-end decode is not bit-exact")
         s2 = torch.cuda.Event(enable_timing=True)
         e2 = torch.cuda.Event(enable_timing=True)
         if world > 1:
@@ -453,7 +506,10 @@ def run_b200(args):
     if e2e:
         line["e2e"] = {"value": round(job_bytes / (e2e_ms_per_step * 1e-3) / 1e9, 2), "unit": UNIT,
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                       "ms_per_step": round(e2e_ms_per_step, 4), "steps": e2e["k"]}
+                       "ms_per_step": round(e2e_ms_per_step, 4), "steps": e2e["k"],
+                       "pieces": max(1, args.e2e_pieces),
+                       "what": "pinned host arrays -> device, decode, BF16 + error word -> pinned host, "
+                               "as a pipeline over chunk ranges (df11_decompress_range_async)"}
     if cpu:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
