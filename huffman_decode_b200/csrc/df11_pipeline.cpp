@@ -33,7 +33,6 @@ struct df11_pipeline {
     cudaEvent_t *uploaded;
     cudaEvent_t *decoded;
     cudaEvent_t *released;
-    uint8_t *sched;   // one decode scheduling workspace per slot (zeroed)
 };
 
 namespace {
@@ -102,23 +101,12 @@ extern "C" df11_status df11_pipeline_create(uint32_t n_slots, df11_pipeline **ou
     p->uploaded = create_events(n_slots);
     p->decoded = p->uploaded ? create_events(n_slots) : nullptr;
     p->released = p->decoded ? create_events(n_slots) : nullptr;
-    // decodes of one slot are ordered by its events; different slots may
-    // decode concurrently, so each has its own workspace
-    void *ws = nullptr;
-    if (p->released && (cudaMalloc(&ws, (size_t)n_slots * DF11_SCHED_WORKSPACE_BYTES) != cudaSuccess ||
-                        cudaMemset(ws, 0, (size_t)n_slots * DF11_SCHED_WORKSPACE_BYTES) != cudaSuccess)) {
-        if (ws)
-            cudaFree(ws);
-        ws = nullptr;
-    }
-    if (!ws) {
+    if (!p->released) {
         destroy_events(p->uploaded, n_slots);
         destroy_events(p->decoded, n_slots);
-        destroy_events(p->released, n_slots);
         delete p;
         return DF11_ERR_CUDA;
     }
-    p->sched = static_cast<uint8_t *>(ws);
     *out = p;
     return DF11_OK;
 }
@@ -130,7 +118,6 @@ extern "C" df11_status df11_pipeline_destroy(df11_pipeline *p)
     destroy_events(p->uploaded, p->n_slots);
     destroy_events(p->decoded, p->n_slots);
     destroy_events(p->released, p->n_slots);
-    cudaFree(p->sched);
     delete p;
     return DF11_OK;
 }
@@ -166,7 +153,7 @@ extern "C" df11_status df11_pipeline_upload(df11_pipeline *p, uint32_t slot, con
 
 extern "C" df11_status df11_pipeline_decode(df11_pipeline *p, uint32_t slot, const df11_device_block *blk,
                                             uint16_t *out_bf16, uint64_t out_capacity, uint32_t *d_error,
-                                            uint32_t max_ctas, void *decode_stream)
+                                            uint32_t max_ctas, void *workspace, void *decode_stream)
 {
     if (!p || !blk || !out_bf16 || slot >= p->n_slots)
         return DF11_ERR_INVALID_ARGUMENT;
@@ -176,8 +163,7 @@ extern "C" df11_status df11_pipeline_decode(df11_pipeline *p, uint32_t slot, con
     if (cudaStreamWaitEvent(s, p->uploaded[slot], 0) != cudaSuccess ||
         cudaStreamWaitEvent(s, p->released[slot], 0) != cudaSuccess)
         return DF11_ERR_CUDA;
-    const df11_status st = df11_decompress_async_ws(blk, out_bf16, out_capacity, d_error, max_ctas,
-                                                    p->sched + (size_t)slot * DF11_SCHED_WORKSPACE_BYTES, s);
+    const df11_status st = df11_decompress_async_ws(blk, out_bf16, out_capacity, d_error, max_ctas, workspace, s);
     if (st != DF11_OK)
         return st;
     return cudaEventRecord(p->decoded[slot], s) == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;

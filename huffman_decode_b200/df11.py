@@ -158,7 +158,7 @@ def load_library(path: str | None = None):
         ("df11_pipeline_create", S, [U32, P]),
         ("df11_pipeline_destroy", S, [P]),
         ("df11_pipeline_upload", S, [P, U32, P, P, P]),
-        ("df11_pipeline_decode", S, [P, U32, P, P, U64, P, U32, P]),
+        ("df11_pipeline_decode", S, [P, U32, P, P, U64, P, U32, P, P]),
         ("df11_pipeline_acquire", S, [P, U32, P]),
         ("df11_pipeline_release", S, [P, U32, P]),
         ("df11_checksum_count", U64, [P]),
@@ -371,14 +371,23 @@ def sched_workspace(device, stream_handle: int):
     """The scheduling workspace this module uses for launches on one stream
     (DF11_SCHED_WORKSPACE_BYTES of zeroed device memory, created on first
     use).  Launches on one stream run one after another, so they can share
-    it; launches on different streams get different workspaces."""
+    it; launches on different streams get different workspaces.  Creation
+    waits for the zero fill (it runs on torch's current stream, the launches
+    on theirs), so make the first launch on a stream outside graph capture."""
     import torch
     dev = torch.device(device)
     key = (dev.index if dev.index is not None else torch.cuda.current_device(), int(stream_handle))
     ws = _WORKSPACES.get(key)
     if ws is None:
-        ws = torch.zeros(SCHED_WORKSPACE_BYTES, dtype=torch.uint8, device=torch.device("cuda", key[0]))
+        ws = _zeroed_workspace(torch.device("cuda", key[0]))
         _WORKSPACES[key] = ws
+    return ws
+
+
+def _zeroed_workspace(device):
+    import torch
+    ws = torch.zeros(SCHED_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+    torch.cuda.synchronize(device)
     return ws
 
 
@@ -533,8 +542,10 @@ def compress_device_noalloc(cb: Codebook, d_in, threads_per_chunk: int = THREADS
 
 class Pipeline:
     """df11_pipeline_*: event ordering of upload -> decode -> consume over
-    caller streams and `n_slots` slots (see include/df11.h).  The pipeline
-    owns CUDA events only; staging blocks and outputs belong to the caller."""
+    caller streams and `n_slots` slots (see include/df11.h).  The C pipeline
+    owns CUDA events only; this object also keeps one decode scheduling
+    workspace per slot (device memory, allocated on the first decode of the
+    slot); staging blocks and outputs belong to the caller."""
 
     def __init__(self, n_slots: int = 2):
         self._lib = load_library()
@@ -542,6 +553,7 @@ class Pipeline:
         _check(self._lib.df11_pipeline_create(int(n_slots), ctypes.byref(h)), "df11_pipeline_create")
         self._h = h
         self.n_slots = int(n_slots)
+        self._ws = {}
 
     def close(self):
         if self._h is not None and self._h.value:
@@ -580,8 +592,12 @@ class Pipeline:
             raise ValueError("out must be a contiguous CUDA tensor of 16-bit elements")
         b = blk.c_struct()
         err_ptr = error.data_ptr() if error is not None else None
+        ws = self._ws.get(int(slot))
+        if ws is None:
+            ws = _zeroed_workspace(out.device)
+            self._ws[int(slot)] = ws
         _check(self._lib.df11_pipeline_decode(self._h, int(slot), ctypes.byref(b), out.data_ptr(),
-                                              out.numel(), err_ptr, int(max_ctas),
+                                              out.numel(), err_ptr, int(max_ctas), ws.data_ptr(),
                                               _raw_stream(stream, out.device)),
                "df11_pipeline_decode")
 

@@ -443,14 +443,11 @@ df11_status df11_verify_device_async(const df11_device_block *blk, const uint32_
  * current at creation (else INVALID_ARGUMENT). */
 typedef struct df11_pipeline df11_pipeline;
 
-/* Host.  Creates a pipeline of n_slots (1..64) slots, each with its own
- * decode scheduling workspace (device memory, DF11_SCHED_WORKSPACE_BYTES a
- * slot).  Errors: INVALID_ARGUMENT, CUDA (no device, or event creation or
- * allocation failed). */
+/* Host.  Creates a pipeline of n_slots (1..64) slots.  Errors:
+ * INVALID_ARGUMENT, CUDA (no device or event creation failed). */
 df11_status df11_pipeline_create(uint32_t n_slots, df11_pipeline **out);
 
-/* Host.  Destroys the pipeline's events and frees its workspaces; the free
- * (cudaFree) waits for work already enqueued on the device. */
+/* Host.  Destroys the pipeline's events (work already enqueued still runs). */
 df11_status df11_pipeline_destroy(df11_pipeline *p);
 
 /* Copy stage.  Enqueues on copy_stream the host -> device copies of src's
@@ -464,11 +461,14 @@ df11_status df11_pipeline_upload(df11_pipeline *p, uint32_t slot, const df11_hos
 
 /* Decode stage.  Enqueues on decode_stream the slot's waits and
  * df11_decompress_async_ws(blk, out_bf16, out_capacity, d_error, max_ctas,
- * the slot's workspace), then marks the slot decoded.  Errors: those of the decode call, and
+ * workspace), then marks the slot decoded.  Decodes of one slot are ordered
+ * by its events, so a slot can keep one workspace; slots whose decodes may
+ * overlap (other decode streams) need different ones.  NULL = the static
+ * chunk schedule.  Errors: those of the decode call, and
  * INVALID_ARGUMENT for a bad pipeline, slot or device. */
 df11_status df11_pipeline_decode(df11_pipeline *p, uint32_t slot, const df11_device_block *blk,
                                  uint16_t *out_bf16, uint64_t out_capacity, uint32_t *d_error,
-                                 uint32_t max_ctas, void *decode_stream);
+                                 uint32_t max_ctas, void *workspace, void *decode_stream);
 
 /* Verify stage (optional, "after every copy").  Enqueues on `stream`,
  * after the slot's last upload, df11_verify_device_async(blk, d_expected,

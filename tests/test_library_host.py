@@ -342,7 +342,7 @@ def test_pipeline_rejects_bad_arguments_before_any_cuda_call():
     fake = 1 << 20
     b = binding._Block()
     assert lib.df11_pipeline_upload(None, 0, ctypes.byref(b), ctypes.byref(b), None) == 1
-    assert lib.df11_pipeline_decode(None, 0, ctypes.byref(b), fake, 16, None, 0, None) == 1
+    assert lib.df11_pipeline_decode(None, 0, ctypes.byref(b), fake, 16, None, 0, None, None) == 1
     assert lib.df11_pipeline_acquire(None, 0, None) == 1
     assert lib.df11_pipeline_release(None, 0, None) == 1
 
