@@ -37,7 +37,7 @@ MAX_CODE_LEN = 16
 STREAM_PAD = 16
 THREADS_PER_CHUNK = 32
 BYTES_PER_THREAD = 16           # 128-bit slices: fastest layout on B200
-LAYOUTS = ((32, 8), (32, 16))   # (threads_per_chunk, bytes_per_thread) this build decodes
+LAYOUTS = ((32, 8), (32, 16))   # (threads_per_chunk, bytes_per_thread) the library decodes
 
 EXPORTED_SYMBOLS = (
     "df11_build_codebook", "df11_build_codebook_from_histogram", "df11_compress_sizes",

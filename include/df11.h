@@ -105,7 +105,7 @@ typedef struct {
 } df11_codebook;
 
 /* Compress-time layout: threads per chunk and bytes of stream per thread.
- * This build uses threads_per_chunk == 32 (one warp) and bytes_per_thread in
+ * The library decodes threads_per_chunk == 32 (one warp) and bytes_per_thread in
  * {8, 16} (64- or 128-bit slices; the pages use 8). */
 typedef struct {
     uint32_t threads_per_chunk;
