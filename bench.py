@@ -236,22 +236,61 @@ def time_oracle_decode(oracle, ob, plan_item):
     return dt, w
 
 
+def host_cpu():
+    """The host's CPU model and logical core count."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "host_logical_cpus": os.cpu_count()}
+
+
+def pinned_to_one_core(fn):
+    """Runs fn() with this process pinned to one core it may use (restoring
+    the affinity afterwards); returns (result, core or None)."""
+    try:
+        old = os.sched_getaffinity(0)
+    except (AttributeError, OSError):
+        return fn(), None
+    core = max(old)
+    try:
+        os.sched_setaffinity(0, {core})
+        return fn(), core
+    except OSError:
+        return fn(), None
+    finally:
+        try:
+            os.sched_setaffinity(0, old)
+        except OSError:
+            pass
+
+
 def cpu_baseline(oracle, hb, cb, bytes_per_weight, seconds):
     """The oracle's serial decode of the whole block (repeated until about
-    `seconds` of CPU time, at most 4 passes), one core."""
-    total_w = 0
-    total_t = 0.0
-    passes = 0
-    while passes < 4 and (passes == 0 or total_t < seconds):
-        t0 = time.perf_counter()
-        e, _ = oracle.decode(hb.exp_stream, hb.n_elements, cb.lengths())
-        oracle.join(e, hb.signmant[: hb.n_elements])
-        total_t += time.perf_counter() - t0
-        total_w += hb.n_elements
-        passes += 1
+    `seconds` of CPU time, at most 4 passes), on one core (pinned)."""
+    def run():
+        total_w = 0
+        total_t = 0.0
+        passes = 0
+        while passes < 4 and (passes == 0 or total_t < seconds):
+            t0 = time.perf_counter()
+            e, _ = oracle.decode(hb.exp_stream, hb.n_elements, cb.lengths())
+            oracle.join(e, hb.signmant[: hb.n_elements])
+            total_t += time.perf_counter() - t0
+            total_w += hb.n_elements
+            passes += 1
+        return total_w, total_t, passes
+
+    (total_w, total_t, passes), core = pinned_to_one_core(run)
     return {"value": round(total_w * bytes_per_weight / total_t / 1e9, 4), "unit": UNIT,
             "cores": 1, "kind": "oracle",
             "gweights_per_s": round(total_w / total_t / 1e9, 5),
+            "pinned_core": core, **host_cpu(),
             "sample": f"{passes} full serial decode pass(es) of the llama8b_block "
                       f"({hb.n_elements} weights each) by the oracle, one thread, "
                       f"{total_t:.1f} s"}
@@ -322,14 +361,19 @@ def run_reference(args):
     comp_bytes = ob.stream.nbytes + ob.gap.size // 2 + ob.pos.nbytes + (n + 15) // 16 * 16
     bytes_per_weight = (comp_bytes + 2 * n) / n
     plan = oracle_sample_plan(ob, 64)
-    for i in range(args.warmup):
-        time_oracle_decode(oracle, ob, plan[i % len(plan)])
-    total_t = 0.0
-    total_w = 0
-    for i in range(args.steps):
-        dt, _ = time_oracle_decode(oracle, ob, plan[i % len(plan)])
-        total_t += dt
-        total_w += plan[i % len(plan)][2]
+
+    def run():
+        for i in range(args.warmup):
+            time_oracle_decode(oracle, ob, plan[i % len(plan)])
+        total_t = 0.0
+        total_w = 0
+        for i in range(args.steps):
+            dt, _ = time_oracle_decode(oracle, ob, plan[i % len(plan)])
+            total_t += dt
+            total_w += plan[i % len(plan)][2]
+        return total_t, total_w
+
+    (total_t, total_w), core = pinned_to_one_core(run)
     value = total_w * bytes_per_weight / total_t / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
@@ -339,6 +383,7 @@ def run_reference(args):
         "config": {"workload": WORKLOAD, "n_weights": n, "seed": 1000,
                    "sample_per_step": "1/64 of the block's chunks, decoded serially"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "pinned_core": core, **host_cpu(),
                          "sample": f"each step decodes 1/64 of the llama8b_block "
                                    f"(~{n // 64} weights) serially, one thread"},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
