@@ -296,6 +296,28 @@ def cpu_baseline(oracle, hb, cb, bytes_per_weight, seconds):
                       f"{total_t:.1f} s"}
 
 
+def e2e_plan(hb, pieces):
+    """The chunk ranges of a piecewise end-to-end step and, for each, the
+    byte spans of the arrays its range decode reads (df11_decompress_range_async:
+    stream words plus the 16-byte pad, gaps, positions incl. the next one,
+    sign|mantissa rounded out to 16 bytes).  Returns [(c0, c1, p0, p1,
+    [(array, begin, end), ...]), ...] with p0, p1 the output range."""
+    n_chunks = int(hb.header.n_chunks)
+    pieces = max(1, min(pieces, n_chunks))
+    W = 32 * int(hb.header.bytes_per_thread)
+    pos = hb.chunk_pos.astype(np.int64)
+    cuts = [n_chunks * i // pieces for i in range(pieces + 1)]
+    plan = []
+    for c0, c1 in zip(cuts[:-1], cuts[1:]):
+        p0, p1 = int(pos[c0]), int(pos[c1])
+        spans = [("exp_stream", W * c0, min(W * c1 + 16, hb.exp_stream.nbytes)),
+                 ("gaps", 16 * c0, 16 * c1),
+                 ("chunk_pos", 4 * c0, 4 * (c1 + 1)),
+                 ("signmant", p0 & ~15, min((p1 + 15) & ~15, hb.signmant.nbytes))]
+        plan.append((c0, c1, p0, p1, spans))
+    return plan
+
+
 def e2e_pipeline(df11, db, hb, host, out, host_out, err, host_err, pieces, stream, dev):
     """One end-to-end step as a pipeline over `pieces` chunk ranges: range k
     is copied in (its stream words, gaps, positions and sign|mantissa bytes)
@@ -304,23 +326,11 @@ def e2e_pipeline(df11, db, hb, host, out, host_out, err, host_err, pieces, strea
     directions and the decode overlap.  The step ends on `stream`.  Returns
     (step, host->device bytes, device->host bytes) per step."""
     import torch
-    n_chunks = int(hb.header.n_chunks)
-    pieces = min(pieces, n_chunks)
-    W = 32 * int(hb.header.bytes_per_thread)
-    pos = hb.chunk_pos.astype(np.int64)
-    cuts = [n_chunks * i // pieces for i in range(pieces + 1)]
     c_in, c_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     cblk = db.c_struct()
-    plan = []
-    for c0, c1 in zip(cuts[:-1], cuts[1:]):
-        p0, p1 = int(pos[c0]), int(pos[c1])
-        spans = [("exp_stream", W * c0, min(W * c1 + 16, host["exp_stream"].numel())),
-                 ("gaps", 16 * c0, 16 * c1),
-                 ("chunk_pos", 4 * c0, 4 * (c1 + 1)),
-                 ("signmant", p0 & ~15, min((p1 + 15) & ~15, host["signmant"].numel()))]
-        plan.append((c0, c1, p0, p1, spans))
+    plan = e2e_plan(hb, pieces)
     h2d = host["lut"].numel() + sum(b - a for *_, spans in plan for _, a, b in spans)
-    d2h = 2 * int(pos[-1]) + 4
+    d2h = 2 * int(hb.chunk_pos[-1]) + 4
     ev_in = [torch.cuda.Event() for _ in plan]
     ev_dec = [torch.cuda.Event() for _ in plan]
     ev_start, ev_end = torch.cuda.Event(), torch.cuda.Event()

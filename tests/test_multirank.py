@@ -70,3 +70,4 @@ def test_single_process_is_identity():
 @pytest.mark.parametrize("units,steps,ms,want", [(300e9, 10, 1000.0, 3000.0), (1e9, 1, 1.0, 1000.0)])
 def test_job_rate(units, steps, ms, want):
     assert bench.job_rate(units, steps, ms) == pytest.approx(want)
+
