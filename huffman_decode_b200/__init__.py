@@ -10,6 +10,7 @@ from .df11 import (  # noqa: F401
     DEVERR_TIMEOUT, DF11Error, checksum, checksum_count, checksum_device, crc32c, verify_device,
     DeviceBlock, EXPORTED_SYMBOLS, LAYOUTS, HostBlock, PinnedHostBlock, Pipeline, build_codebook,
     decode_gemv_async, SCHED_WORKSPACE_BYTES, sched_workspace, decompress_range_async,
+    selftest_bounded_wait,
     build_codebook_from_histogram, compress, compress_device, compress_device_noalloc,
     compress_device_scratch_bytes,
     compress_sizes, decompress_async, histogram_device, library_path, load_library, validate,

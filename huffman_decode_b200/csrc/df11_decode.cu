@@ -58,6 +58,7 @@ constexpr int kEntryBytes = 8;                     // multi-code entry: symbols 
 constexpr uint32_t kLongStep = 0x80000000u;        // step of an entry whose first code is long
 constexpr int kMaxWarpsPerCta = 32;
 constexpr uint32_t kWaitLimit = 1u << 22;          // bounded mbarrier polls
+constexpr uint32_t kWaitHintNs = 2000;              // longest suspension of one poll (so <= 8.4 s in all)
 
 struct DecodeParams {
     const uint8_t *stream;
@@ -293,15 +294,16 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uin
 }
 
 // Waits until the barrier completes the phase with the given parity; gives up
-// after kWaitLimit polls and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+// after `limit` polls (each suspends the thread for at most kWaitHintNs)
+// and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit = kWaitLimit)
 {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    for (uint32_t i = 0; i < limit; ++i) {
         uint32_t done;
         asm volatile(
-            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.b32 %0, 1, 0, p; }"
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.b32 %0, 1, 0, p; }"
             : "=r"(done)
-            : "r"(bar), "r"(parity)
+            : "r"(bar), "r"(parity), "n"(kWaitHintNs)
             : "memory");
         if (done)
             return true;
@@ -860,6 +862,21 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     }
 }
 
+// The bounded wait's give-up path, on its own: one warp waits on a barrier
+// that nothing arrives on, and reports what the decode would report.
+__global__ void bounded_wait_kernel(uint32_t polls, uint32_t *status)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t a = smem_addr(&bar);
+    if (threadIdx.x == 0)
+        mbar_init(a);   // one arrival expected; none comes
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncwarp();
+    const bool done = mbar_wait(a, 0u, polls);
+    if (threadIdx.x == 0)
+        *status = done ? 0u : DF11_DEVERR_TIMEOUT;
+}
+
 template <int W, int MINLEN>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(DecodeParams p)
 {
@@ -1065,6 +1082,14 @@ extern "C" df11_status df11_decompress_async_ws(const df11_device_block *blk, ui
     if (blk->hdr.bytes_per_thread == 8)
         return prm.min_len >= 2 ? launch<8, 2>(prm, dev, s, max_ctas) : launch<8, 1>(prm, dev, s, max_ctas);
     return prm.min_len >= 2 ? launch<16, 2>(prm, dev, s, max_ctas) : launch<16, 1>(prm, dev, s, max_ctas);
+}
+
+extern "C" df11_status df11_selftest_bounded_wait(uint32_t polls, uint32_t *d_status, void *stream)
+{
+    if (!d_status || !aligned(d_status, 4) || polls == 0 || polls > 4096)
+        return DF11_ERR_INVALID_ARGUMENT;
+    bounded_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(polls, d_status);
+    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
 extern "C" df11_status df11_decompress_range_async(const df11_device_block *blk, uint64_t chunk_begin,

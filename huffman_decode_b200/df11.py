@@ -48,6 +48,7 @@ EXPORTED_SYMBOLS = (
     "df11_pipeline_release", "df11_checksum_count", "df11_crc32c", "df11_checksum",
     "df11_checksum_device_async", "df11_verify_device_async", "df11_pipeline_verify",
     "df11_decode_gemv_async", "df11_decompress_async_ws", "df11_decompress_range_async",
+    "df11_selftest_bounded_wait",
 )
 SCHED_WORKSPACE_BYTES = 2048
 CRC_SEGMENT_BYTES = 4096
@@ -170,6 +171,7 @@ def load_library(path: str | None = None):
         ("df11_decode_gemv_async", S, [P, P, U32, U32, P, P, P]),
         ("df11_decompress_async_ws", S, [P, P, U64, P, U32, P, P]),
         ("df11_decompress_range_async", S, [P, U64, U64, P, U64, P, P, P]),
+        ("df11_selftest_bounded_wait", S, [U32, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -422,6 +424,15 @@ def decompress_async(db: DeviceBlock, out, error=None, stream=None, c_block=None
     _check(load_library().df11_decompress_async_ws(ctypes.byref(blk), out.data_ptr(), cap, err_ptr,
                                                    int(max_ctas), _workspace_ptr(workspace, out.device, handle),
                                                    handle), "df11_decompress_async_ws")
+
+
+def selftest_bounded_wait(polls: int, status, stream=None) -> None:
+    """df11_selftest_bounded_wait: one warp polls a barrier nothing arrives
+    on `polls` times and writes the timeout status into `status` (int32 CUDA
+    tensor)."""
+    _check(load_library().df11_selftest_bounded_wait(int(polls), status.data_ptr(),
+                                                     _raw_stream(stream, status.device)),
+           "df11_selftest_bounded_wait")
 
 
 def decompress_range_async(db: DeviceBlock, chunk_begin: int, chunk_end: int, out, error=None,

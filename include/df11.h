@@ -277,6 +277,14 @@ df11_status df11_decompress_range_async(const df11_device_block *blk, uint64_t c
                                         uint64_t chunk_end, uint16_t *out_bf16, uint64_t out_capacity,
                                         uint32_t *d_error, void *workspace, void *stream);
 
+/* GPU, diagnostic.  Runs the decode kernel's bounded barrier wait on a
+ * barrier that nothing arrives on: one warp polls it `polls` times (1..4096),
+ * gives up and writes DF11_DEVERR_TIMEOUT to *d_status (device uint32) --
+ * what a decode whose staged copy never lands ORs into its error word.
+ * Shows that a wait that runs out returns a status instead of hanging, with
+ * no fault and the context still usable.  Errors: INVALID_ARGUMENT, CUDA. */
+df11_status df11_selftest_bounded_wait(uint32_t polls, uint32_t *d_status, void *stream);
+
 /* ---- Decode fused with its consumer: matrix-vector products --------------
  * The pages decode a block into a BF16 buffer and then run its matrix
  * products ("DFloat11: lossless BFloat16 compression", "Architecture":

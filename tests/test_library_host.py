@@ -329,6 +329,11 @@ def test_decompress_rejects_bad_arguments_before_any_cuda_call():
     assert rng(dev_block(), nch, nch + 1) == 1
     assert rng(dev_block(), 0, 1, ws=fake + 8) == 1
     assert rng(dev_block(exp_stream=fake + 8), 0, 1) == 1
+    # the bounded-wait self-test checks its arguments before launching
+    assert lib.df11_selftest_bounded_wait(0, fake, None) == 1
+    assert lib.df11_selftest_bounded_wait(4097, fake, None) == 1
+    assert lib.df11_selftest_bounded_wait(16, None, None) == 1
+    assert lib.df11_selftest_bounded_wait(16, fake + 2, None) == 1
 
 
 def test_pipeline_rejects_bad_arguments_before_any_cuda_call():
