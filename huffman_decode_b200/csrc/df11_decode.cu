@@ -591,7 +591,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
 
     uint32_t err = 0;
     bool stalled = false;      // a staged copy did not arrive in time
-    uint64_t k = 0;            // chunks this warp has finished
+    uint64_t n_done = 0;       // chunks this warp has finished
 
     for (;;) {
         // ---- positions (warp-uniform) and the staged sign|mantissa copy -----
@@ -608,9 +608,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
 
         // ---- the next chunk's slice and positions, loaded ahead -------------
         uint64_t next;
-        if (!dyn || k + 1 < r_static) {
+        if (!dyn || n_done + 1 < r_static) {
             next = chunk + n_warps;
-            if (dyn && k + 2 == r_static && lane == 0)
+            if (dyn && n_done + 2 == r_static && lane == 0)
                 claim = atomicAdd(pool, 1u);      // the first claimed chunk, a chunk ahead
         } else {
             next = d0 + q + (uint64_t)kSchedPools * __shfl_sync(0xFFFFFFFFu, claim, 0);
@@ -828,7 +828,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             __syncwarp();
         }
 
-        ++k;
+        ++n_done;
         if (!has_next || stalled)
             break;
         chunk = next;
