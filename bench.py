@@ -785,14 +785,15 @@ def run_overlap(args):
                 decode(i, i % 2, cur)
                 products(i % 2)
 
-        def run_overlap_cap(max_ctas):
+        def run_overlap_cap(max_ctas, claimed):
             def fn():
                 with df11.Pipeline(2) as pipe:
                     s_dec.wait_stream(cur)
                     s_use.wait_stream(cur)
                     for i in range(n_blocks):
                         slot = i % 2
-                        pipe.decode(slot, dbs[i], slots[slot], err, s_dec, max_ctas=max_ctas)
+                        pipe.decode(slot, dbs[i], slots[slot], err, s_dec, max_ctas=max_ctas,
+                                    workspace=claimed)
                         pipe.acquire(slot, s_use)
                         with torch.cuda.stream(s_use):
                             products(slot)
@@ -808,11 +809,12 @@ def run_overlap(args):
         ref = [t.clone() for t in y]
         row = {"tokens": T, "decode_ms": round(t_dec, 4), "gemm_ms": round(t_gemm, 4),
                "serial_ms": round(t_ser, 4), "overlap": []}
-        for cap in cap_list:
-            t_ov = timed(run_overlap_cap(cap), reps)
+        for cap, claimed in [(c, w) for c in cap_list for w in (True, False)]:
+            t_ov = timed(run_overlap_cap(cap, claimed), reps)
             same = all(torch.equal(a, b) for a, b in zip(ref, y))
             row["overlap"].append({
-                "max_ctas": cap, "overlap_ms": round(t_ov, 4),
+                "max_ctas": cap, "schedule": "claimed tail" if claimed else "static",
+                "overlap_ms": round(t_ov, 4),
                 "hidden_frac": round((t_ser - t_ov) / t_dec, 4),
                 "overhead_vs_bf16": round(t_ov / t_gemm, 4),
                 "outputs_equal_serial": bool(same)})

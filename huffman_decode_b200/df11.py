@@ -598,17 +598,22 @@ class Pipeline:
         dst._keep = src   # the copy reads src after this call returns
 
     def decode(self, slot: int, blk: "DeviceBlock", out, error=None, stream=None,
-               max_ctas: int = 0) -> None:
+               max_ctas: int = 0, workspace=True) -> None:
+        """Decode stage of `slot`; `workspace` True = the slot's own
+        scheduling workspace (claimed tail), False = the static schedule."""
         if out.element_size() != 2 or not out.is_cuda or not out.is_contiguous():
             raise ValueError("out must be a contiguous CUDA tensor of 16-bit elements")
         b = blk.c_struct()
         err_ptr = error.data_ptr() if error is not None else None
-        ws = self._ws.get(int(slot))
-        if ws is None:
-            ws = _zeroed_workspace(out.device)
-            self._ws[int(slot)] = ws
+        ws_ptr = None
+        if workspace:
+            ws = self._ws.get(int(slot))
+            if ws is None:
+                ws = _zeroed_workspace(out.device)
+                self._ws[int(slot)] = ws
+            ws_ptr = ws.data_ptr()
         _check(self._lib.df11_pipeline_decode(self._h, int(slot), ctypes.byref(b), out.data_ptr(),
-                                              out.numel(), err_ptr, int(max_ctas), ws.data_ptr(),
+                                              out.numel(), err_ptr, int(max_ctas), ws_ptr,
                                               _raw_stream(stream, out.device)),
                "df11_pipeline_decode")
 
