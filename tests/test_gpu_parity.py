@@ -82,13 +82,14 @@ def test_small_workloads(name, bpt, schedule):
 
 # ------------------------------------------------------- chunk schedules
 
-@pytest.mark.parametrize("max_ctas", [0, 1, 7, 148, 1 << 20])
+@pytest.mark.parametrize("max_ctas", [0, 1, 7, 148, 200, 1 << 20])
 def test_dynamic_schedule_leaves_workspace_zero(max_ctas):
-    """With a workspace, warps past their first chunk claim chunks from a
-    counter; every launch must decode every chunk exactly right and leave
+    """With a workspace, warps past their first rounds claim chunks from
+    counters; every launch must decode every chunk exactly right and leave
     the workspace zero for the next launch (any grid: one CTA, a partial
-    wave, waves of short-lived CTAs).  The block has over five rounds of
-    chunks for a full wave, so every grid but the largest claims chunks."""
+    wave, two waves of CTAs, one short-lived CTA per 32 chunks).  The block
+    has over five rounds of chunks for every grid but the largest, so all
+    the others claim chunks."""
     mats = [m for _, m in workloads.llama_block(1000, scale_div=4)]
     w = _flat(mats)
     hb = df11.compress(df11.build_codebook(mats), mats)

@@ -105,6 +105,26 @@ def test_a_range_reads_and_writes_only_its_own_bytes(bpt):
         assert np.all(got[:p0] == SENTINEL) and np.all(got[p1:] == SENTINEL), (c0, c1)
 
 
+def test_full_size_block_in_two_claimed_pieces():
+    """Two halves of the Llama-3.1-8B-shaped block: each has over five
+    rounds of chunks for a full wave of warps, so each range launch claims
+    its last rounds from the (per-stream) scheduling workspace."""
+    mats = [m for _, m in workloads.llama_block(1001)]
+    w = np.concatenate([m.reshape(-1) for m in mats])
+    hb = df11.compress(df11.build_codebook(mats), mats)
+    db = hb.to_device("cuda")
+    n_chunks = int(hb.header.n_chunks)
+    out = torch.full((hb.n_elements,), SENTINEL, dtype=torch.int16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(df11.SCHED_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    for c0, c1 in ((n_chunks // 2, n_chunks), (0, n_chunks // 2)):
+        df11.decompress_range_async(db, c0, c1, out, err, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert int(ws.count_nonzero().item()) == 0
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), w)
+
+
 def test_full_size_block_in_pieces():
     """The Llama-3.1-8B-shaped block in 8 pieces on two streams, against the
     input bits (the oracle's whole-block parity at this size is in
