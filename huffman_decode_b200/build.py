@@ -18,7 +18,8 @@ CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libdf11.so")
 
-SOURCES = [os.path.join(CSRC, f) for f in ("df11_host.cpp", "df11_decode.cu", "df11_encode.cu", "df11_pipeline.cpp", "df11_crc.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("df11_host.cpp", "df11_decode.cu", "df11_encode.cu", "df11_pipeline.cpp", "df11_crc.cu",
+                                                 "df11_io.cpp")]
 HEADERS = [os.path.join(INCLUDE, "df11.h")]
 
 NVCC_FLAGS = [

@@ -23,6 +23,9 @@ from . import build as _build
 # ------------------------------------------------------------ constants
 
 DF11_OK = 0
+DF11_ERR_INVALID_ARGUMENT = 1
+DF11_ERR_BUFFER_TOO_SMALL = 2
+DF11_ERR_CORRUPT = 4
 STATUS_NAMES = {
     0: "DF11_OK", 1: "DF11_ERR_INVALID_ARGUMENT", 2: "DF11_ERR_BUFFER_TOO_SMALL",
     3: "DF11_ERR_OVERFLOW", 4: "DF11_ERR_CORRUPT", 5: "DF11_ERR_CUDA", 6: "DF11_ERR_TIMEOUT",
@@ -48,7 +51,7 @@ EXPORTED_SYMBOLS = (
     "df11_pipeline_release", "df11_checksum_count", "df11_crc32c", "df11_checksum",
     "df11_checksum_device_async", "df11_verify_device_async", "df11_pipeline_verify",
     "df11_decode_gemv_async", "df11_decompress_async_ws", "df11_decompress_range_async",
-    "df11_selftest_bounded_wait",
+    "df11_selftest_bounded_wait", "df11_serialized_bytes", "df11_serialize", "df11_deserialize",
 )
 SCHED_WORKSPACE_BYTES = 2048
 CRC_SEGMENT_BYTES = 4096
@@ -172,6 +175,9 @@ def load_library(path: str | None = None):
         ("df11_decompress_async_ws", S, [P, P, U64, P, U32, P, P]),
         ("df11_decompress_range_async", S, [P, U64, U64, P, U64, P, P, P]),
         ("df11_selftest_bounded_wait", S, [U32, P, P]),
+        ("df11_serialized_bytes", U64, [P]),
+        ("df11_serialize", S, [P, P, U64]),
+        ("df11_deserialize", S, [P, U64, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -252,6 +258,57 @@ class HostBlock:
 
     def arrays(self):
         return {n: getattr(self, n) for n in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")}
+
+    def to_bytes(self) -> bytes:
+        """df11_serialize: the block as one flat buffer (header, the five
+        arrays, the CRC-32C checksum list).  matrix_numel is not stored."""
+        lib = load_library()
+        b = self.c_struct()
+        n = int(lib.df11_serialized_bytes(ctypes.byref(b)))
+        if n == 0:
+            raise DF11Error(DF11_ERR_INVALID_ARGUMENT, "df11_serialized_bytes")
+        buf = np.empty(n, dtype=np.uint8)
+        _check(lib.df11_serialize(ctypes.byref(b), buf.ctypes.data, n), "df11_serialize")
+        return buf.tobytes()
+
+    @staticmethod
+    def from_bytes(data) -> "HostBlock":
+        """df11_deserialize: checks the header, sizes, every segment checksum
+        and the block's structure, then copies the arrays out.  Raises
+        DF11Error (with .first_bad_segment, or None) when anything is off."""
+        src = np.frombuffer(data, dtype=np.uint8)
+        store = np.zeros(max(1, src.size), dtype=np.uint8)   # a real pointer even when empty
+        store[: src.size] = src
+        buf = store[: src.size]
+        blk = _Block()
+        first = ctypes.c_uint64(0)
+        st = load_library().df11_deserialize(store.ctypes.data, src.size, ctypes.byref(blk),
+                                             ctypes.byref(first))
+        if st != DF11_OK:
+            e = DF11Error(st, "df11_deserialize")
+            e.first_bad_segment = None if first.value == (1 << 64) - 1 else int(first.value)
+            raise e
+        base = store.ctypes.data
+
+        def take(ptr, nbytes, dtype):
+            off = int(ptr) - base
+            return buf[off:off + nbytes].view(dtype).copy()
+
+        return HostBlock(header=Header.from_buffer_copy(blk.hdr),
+                         exp_stream=take(blk.exp_stream, blk.exp_stream_bytes, np.uint8),
+                         gaps=take(blk.gaps, blk.gaps_bytes, np.uint8),
+                         chunk_pos=take(blk.chunk_pos, 4 * blk.chunk_pos_count, np.uint32),
+                         signmant=take(blk.signmant, blk.signmant_bytes, np.uint8),
+                         lut=take(blk.lut, 2 * blk.lut_entries, np.uint16))
+
+    def save(self, path) -> None:
+        with open(path, "wb") as f:
+            f.write(self.to_bytes())
+
+    @staticmethod
+    def load(path) -> "HostBlock":
+        with open(path, "rb") as f:
+            return HostBlock.from_bytes(f.read())
 
     def pinned(self) -> "PinnedHostBlock":
         """A copy of the block in page-locked host memory (torch pinned

@@ -493,6 +493,35 @@ df11_status df11_pipeline_verify(df11_pipeline *p, uint32_t slot, const df11_dev
 df11_status df11_pipeline_acquire(df11_pipeline *p, uint32_t slot, void *consumer_stream);
 df11_status df11_pipeline_release(df11_pipeline *p, uint32_t slot, void *consumer_stream);
 
+/* ---- One block as a flat byte buffer (files) -------------------------------
+ * The pages keep DF11 models in safetensors files and tell users to checksum
+ * artifacts on download and after every copy ("DFloat11: lossless BFloat16
+ * compression", "How to run it in production", "Failure modes").  The
+ * library's own container for one block: a 128-byte header (magic
+ * "DF11BLK\0", version 1, the block header, the five array lengths, the
+ * checksum count, the CRC-32C of those header bytes), the five arrays in
+ * the order exp_stream, gaps, chunk_pos, signmant, lut, each at a 16-byte
+ * aligned offset, then the checksum list of df11_checksum.  Little-endian.
+ */
+
+/* Host.  Bytes df11_serialize writes for blk (0 for NULL or absurd sizes). */
+uint64_t df11_serialized_bytes(const df11_host_block *blk);
+
+/* Host.  Writes blk into buf[0 .. df11_serialized_bytes(blk)).  Errors:
+ * INVALID_ARGUMENT (null pointers), BUFFER_TOO_SMALL. */
+df11_status df11_serialize(const df11_host_block *blk, void *buf, uint64_t buf_bytes);
+
+/* Host.  Reads a buffer written by df11_serialize (buf_bytes must be its
+ * exact length): checks the magic, version and header CRC, the sizes,
+ * that all padding is zero, every segment checksum and the block's
+ * structure (df11_validate), so that every byte is checked, then
+ * fills *blk with pointers INTO buf (no copy; buf must outlive blk).
+ * *first_bad (may be NULL) receives the index of the first segment whose
+ * checksum differs, else UINT64_MAX.  Errors: INVALID_ARGUMENT (null
+ * pointers), CORRUPT (anything that does not check out; *blk untouched). */
+df11_status df11_deserialize(const void *buf, uint64_t buf_bytes, df11_host_block *blk,
+                             uint64_t *first_bad);
+
 const char *df11_status_string(df11_status s);
 
 #ifdef __cplusplus

@@ -355,3 +355,16 @@ def test_model_stream_blocks_into_one_reused_buffer():
             assert np.array_equal(got, ref)
         assert np.array_equal(got, _flat(mats))
         del db
+
+
+def test_a_block_read_back_from_its_file_decodes_exactly(tmp_path):
+    """The flat container (df11_serialize) written to a file, read back and
+    checked (df11_deserialize), then decoded on the GPU."""
+    mats = [m for _, m in workloads.llama_block(1006, scale_div=32)]
+    hb = df11.compress(df11.build_codebook(mats), mats)
+    path = tmp_path / "block.df11"
+    hb.save(path)
+    got, err = gpu_decode(df11.HostBlock.load(path), guard=8)
+    assert err == 0
+    w = _flat(mats)
+    assert np.array_equal(got[: w.size], w) and np.all(got[w.size:] == 0x5A5A)
