@@ -41,6 +41,7 @@ METRIC = "DF11 decode GB/s (compressed in + BF16 out), Gweights/s, % of B200 HBM
 UNIT = "GB/s"
 WORKLOAD = "llama8b_block"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 7700.0      # B200 HBM3e, the HGX data-sheet figure (context only)
 KERNEL_SRC = os.path.join(ROOT, "huffman_decode_b200", "csrc", "df11_decode.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_llama8b_block.md")
 
@@ -550,6 +551,7 @@ def run_b200(args):
                    "parallelism": f"replicas x{world}, one block per GPU, no collective"},
         "gweights_per_s": round(job_rate(job_weights, args.steps, ms_max), 2),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "pct_of_nominal_hbm": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "bit_exact": bit_exact,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
