@@ -6,7 +6,7 @@ and one GPU launch per block rebuilds the bit-exact BF16 matrices.  The work
 happens in libdf11.so (C ABI in include/df11.h); this package only binds it.
 """
 from .df11 import (  # noqa: F401
-    CRC_SEGMENT_BYTES, DEVERR_BAD_CODE, DEVERR_BAD_POS, DEVERR_CHECKSUM, DEVERR_COUNT, DEVERR_MISMATCH,
+    CRC_SEGMENT_BYTES, DEVERR_BOUNDS, DEVERR_BAD_CODE, DEVERR_BAD_POS, DEVERR_CHECKSUM, DEVERR_COUNT, DEVERR_MISMATCH,
     DEVERR_TIMEOUT, DF11Error, checksum, checksum_count, checksum_device, crc32c, verify_device,
     DeviceBlock, EXPORTED_SYMBOLS, LAYOUTS, HostBlock, PinnedHostBlock, Pipeline, build_codebook,
     decode_gemv_async, SCHED_WORKSPACE_BYTES, sched_workspace, decompress_range_async,

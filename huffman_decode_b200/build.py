@@ -3,7 +3,9 @@
     python -m huffman_decode_b200.build        # or build() from Python
 
 Output: huffman_decode_b200/_lib/libdf11.so, exporting the C ABI declared in
-include/df11.h.  nvcc cross-compiles for sm_100a without a GPU present.
+include/df11.h, and libdf11_checked.so, the same library built with
+-DDF11_CHECKED (run-time bound checks in the decode kernel; the binding loads
+it when DF11_CHECKED=1).  nvcc cross-compiles for sm_100a without a GPU.
 """
 from __future__ import annotations
 
@@ -17,6 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libdf11.so")
+CHECKED_LIB_PATH = os.path.join(LIB_DIR, "libdf11_checked.so")
 
 SOURCES = [os.path.join(CSRC, f) for f in ("df11_host.cpp", "df11_decode.cu", "df11_encode.cu", "df11_pipeline.cpp", "df11_crc.cu",
                                                  "df11_io.cpp")]
@@ -37,26 +40,35 @@ def nvcc_path() -> str:
     return "nvcc"
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB_PATH):
+def is_stale(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return True
-    built = os.path.getmtime(LIB_PATH)
+    built = os.path.getmtime(path)
     return any(os.path.getmtime(f) > built for f in SOURCES + HEADERS + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the library if a source is newer than it (or force)."""
-    if not force and not is_stale():
-        return LIB_PATH
+def _compile(path: str, extra, verbose: bool) -> None:
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
-    cmd = [nvcc_path(), *NVCC_FLAGS, f"-I{INCLUDE}", *SOURCES, "-o", tmp]
+    tmp = path + f".tmp{os.getpid()}"
+    cmd = [nvcc_path(), *NVCC_FLAGS, *extra, f"-I{INCLUDE}", *SOURCES, "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+
+
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Compile the library (checked=True: the bound-checked one) if a source
+    is newer than it (or force); returns its path."""
+    path = CHECKED_LIB_PATH if checked else LIB_PATH
+    if force or is_stale(path):
+        _compile(path, ["-DDF11_CHECKED"] if checked else [], verbose)
+    return path
+
+
+def build_all(force: bool = False, verbose: bool = False) -> list:
+    return [build(force, verbose, checked=False), build(force, verbose, checked=True)]
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build_all(force="--force" in sys.argv, verbose=True))

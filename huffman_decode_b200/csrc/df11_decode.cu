@@ -57,6 +57,15 @@ constexpr int kMaxCodesPerEntry = 4;
 constexpr int kEntryBytes = 8;                     // multi-code entry: symbols | step
 constexpr uint32_t kLongStep = 0x80000000u;        // step of an entry whose first code is long
 constexpr int kMaxWarpsPerCta = 32;
+// A checked build (-DDF11_CHECKED, libdf11_checked.so) verifies at run time
+// the invariants that keep every access in bounds, ORs DF11_DEVERR_BOUNDS
+// and skips the access when one fails.  The normal build compiles the checks
+// away.
+#ifdef DF11_CHECKED
+#define DF11_CHECK(err, cond) ((cond) ? true : ((err) |= DF11_DEVERR_BOUNDS, false))
+#else
+#define DF11_CHECK(err, cond) true
+#endif
 constexpr uint32_t kWaitLimit = 1u << 22;          // bounded mbarrier polls
 constexpr uint32_t kWaitHintNs = 2000;              // longest suspension of one poll (so <= 8.4 s in all)
 
@@ -602,7 +611,12 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
         const uint32_t gfirst = head ? 1u : 0u;
         // copy [pos0 & ~15, ceil16(pos1)) -> sbuf; group i is at sbuf + (pos0 & 8) + 8i
         const uint64_t cp_lo = (uint64_t)pos0 & ~15ull;
-        const uint32_t cp_bytes = pos_ok ? (uint32_t)((((uint64_t)pos1 + 15) & ~15ull) - cp_lo) : 0u;
+        uint32_t cp_bytes = pos_ok ? (uint32_t)((((uint64_t)pos1 + 15) & ~15ull) - cp_lo) : 0u;
+        // (warp-uniform) the copy stays inside the block's sign|mantissa
+        // bytes and the warp's buffer
+        if (cp_bytes && !DF11_CHECK(err, cp_bytes <= (uint32_t)G::kSbufBytes &&
+                                             cp_lo + cp_bytes <= ((p.out_limit + 15) & ~15ull)))
+            cp_bytes = 0;
         if (cp_bytes && lane == 0)
             bulk_copy_g2s(sbuf_a, p.signmant + cp_lo, cp_bytes, bar);
 
@@ -674,6 +688,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                     }
                 }
                 const uint32_t fill = X >> 16;
+                // the lane's slot words stayed inside its column
+                (void)DF11_CHECK(err, sp - slot_lane_a < 128u * (uint32_t)G::kSlotRows);
                 if (fill)
                     sts_u32(sp, accl);
                 uint32_t cnt = ((sp - slot_lane_a) >> 5) + (fill >> 3);   // 4 codes per 128-byte row
@@ -721,7 +737,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             // Lane bytes go to ebuf[head + off, head + off + nbytes).  Words the
             // lane covers entirely are plain stores; the first and last word
             // may be shared with neighbouring lanes: zeroed, then ORed.
-            const uint32_t nbytes = off < n_write ? min(count, n_write - off) : 0u;
+            uint32_t nbytes = off < n_write ? min(count, n_write - off) : 0u;
+            if (!DF11_CHECK(err, head + off + nbytes <= (uint32_t)G::kEbufBytes))
+                nbytes = 0;
             const uint32_t a = head + off;
             const uint32_t sh = (a & 3u) * 8;
             const uint32_t first = a >> 2;
@@ -794,7 +812,11 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             // Whole groups: 8 exponents + 8 sign|mantissa bytes -> one 16-byte
             // store per lane.  The partial groups at both ends (<= 7 elements
             // each) take one element per lane on lanes 0..15.
-            if (!stalled && TT == 0) {
+            // the merge's groups lie inside the output range and the staged bytes
+            const bool merge_ok =
+                DF11_CHECK(err, (uint64_t)pos0 + n_write <= p.out_limit &&
+                                    (pos0 & 8u) + 8u * ((head + n_write + 7) >> 3) <= (uint32_t)G::kSbufBytes);
+            if (!stalled && TT == 0 && merge_ok) {
                 const uint32_t span = head + n_write;
                 const uint32_t mend = span >> 3;                   // whole groups end
                 const uint32_t sgrp_a = sbuf_a + (pos0 & 8u);     // group 0 of the chunk
@@ -822,7 +844,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                     p.out[base + l] = join1(lds_u8_m(ebuf_a + l), lds_u8_m(sgrp_a + l));
             }
             if constexpr (TT > 0) {
-                if (!stalled)
+                if (!stalled && merge_ok)
                     gemv_chunk<TT>(gp, head, n_write, base, lane, ebuf_a, sbuf_a + (pos0 & 8u));
             }
             __syncwarp();

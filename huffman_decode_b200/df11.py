@@ -36,6 +36,7 @@ DEVERR_BAD_POS = 0x4
 DEVERR_TIMEOUT = 0x8
 DEVERR_MISMATCH = 0x10
 DEVERR_CHECKSUM = 0x20
+DEVERR_BOUNDS = 0x40
 MAX_CODE_LEN = 16
 STREAM_PAD = 16
 THREADS_PER_CHUNK = 32
@@ -134,13 +135,15 @@ _lib = None
 
 
 def load_library(path: str | None = None):
-    """Loads libdf11.so (building it first if a source is newer).  Raises if
-    the library cannot be built or loaded: there is no fallback path."""
+    """Loads libdf11.so -- or libdf11_checked.so, the build whose decode
+    kernel checks its bounds at run time, when the environment has
+    DF11_CHECKED=1 -- building it first if a source is newer.  Raises if the
+    library cannot be built or loaded: there is no fallback path."""
     global _lib
     if _lib is not None and path is None:
         return _lib
     if path is None:
-        path = _build.build()
+        path = _build.build(checked=os.environ.get("DF11_CHECKED") == "1")
     lib = ctypes.CDLL(path)
     P = ctypes.c_void_p
     U32 = ctypes.c_uint32
@@ -188,7 +191,9 @@ def load_library(path: str | None = None):
 
 
 def library_path() -> str:
-    return _build.LIB_PATH
+    """Path of the library this process uses (the checked one when
+    DF11_CHECKED=1)."""
+    return _build.CHECKED_LIB_PATH if os.environ.get("DF11_CHECKED") == "1" else _build.LIB_PATH
 
 
 def _check(status: int, call: str):

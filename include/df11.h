@@ -84,6 +84,9 @@ typedef enum {
                                      or a bit total other than the codebook's  */
 #define DF11_DEVERR_CHECKSUM 0x20u /* df11_verify_device_async: a segment's
                                      CRC-32C differs from the expected value   */
+#define DF11_DEVERR_BOUNDS 0x40u   /* checked build (libdf11_checked.so) only: an
+                                     invariant that keeps an access in bounds
+                                     failed; the access was skipped            */
 
 #define DF11_MAX_CODE_LEN 16u     /* longest code the format allows           */
 #define DF11_MIN_CODE_LEN_CAP 8u  /* smallest cap accepted by build_codebook  */
