@@ -10,7 +10,8 @@
 // B200 design (differs from the page's two-phase kernel):
 //   * one warp = one chunk: output positions are stored per 32 threads, so
 //     every warp decodes, scans (shuffles), compacts and stores on its own,
-//     with no block-wide barrier after the prologue;
+//     with no block-wide barrier after the prologue (the claimed schedule
+//     below adds one at the very end, to count the CTA out);
 //   * single decode pass with a multi-code table: an 11-bit window indexes a
 //     2048-entry table (built in shared memory from the format's two-level
 //     16-bit tables) that yields up to four whole codes per lookup; longer
@@ -40,6 +41,9 @@
 //     finish within about one chunk of each other.  Claiming only the tail
 //     keeps the atomics off the memory system for most of the launch.  The
 //     last CTA out resets the counters.
+// Also here: decoding a chunk range alone (df11_decompress_range_async), the
+// fused matrix-vector products (df11_decode_gemv_async), the bounded-wait
+// self-test, and the run-time bound checks of the checked build.
 // No tensor cores: this is integer decode, bounded by HBM traffic and issue.
 #include "df11.h"
 
