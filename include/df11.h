@@ -285,7 +285,9 @@ df11_status df11_decompress_range_async(const df11_device_block *blk, uint64_t c
  * gives up and writes DF11_DEVERR_TIMEOUT to *d_status (device uint32) --
  * what a decode whose staged copy never lands ORs into its error word.
  * Shows that a wait that runs out returns a status instead of hanging, with
- * no fault and the context still usable.  Errors: INVALID_ARGUMENT, CUDA. */
+ * no fault and the context still usable.  (No counterpart on the pages,
+ * whose kernel neither stages copies nor reports errors; "Failure modes"
+ * only warns that corruption is silent.)  Errors: INVALID_ARGUMENT, CUDA. */
 df11_status df11_selftest_bounded_wait(uint32_t polls, uint32_t *d_status, void *stream);
 
 /* ---- Decode fused with its consumer: matrix-vector products --------------
