@@ -23,11 +23,14 @@
 // "Architecture": Gaps and per-chunk output positions).
 #include "df11.h"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
+#include <utility>
 
 namespace {
 
@@ -622,8 +625,47 @@ constexpr int kNoAllocMaxDevices = 64;
 // entries it reads before reading them, so nothing needs clearing.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch, per device (0 = not looked up yet).
-std::atomic<uintptr_t> g_noalloc_addr[kNoAllocMaxDevices];
+// The array's device address belongs to the module as loaded into one CUDA
+// context: a context made after cudaDeviceReset, or another driver context
+// on the same device, loads the module again at another address.  So the
+// address is cached per device together with the identity of the context it
+// was looked up in (the driver's context ID, reached through the runtime's
+// entry-point query so the library needs no link to the driver library),
+// and looked up again whenever the current context differs.
+struct NoAllocSlot {
+    unsigned long long ctx_id = 0;   // 0 = nothing cached
+    uintptr_t addr = 0;
+};
+NoAllocSlot g_noalloc_slot[kNoAllocMaxDevices];
+std::mutex g_noalloc_mutex;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// ID of the context current on this thread, or 0 when it cannot be had.
+unsigned long long current_context_id()
+{
+    static const auto fns = [] {
+        std::pair<CtxGetCurrentFn, CtxGetIdFn> f{nullptr, nullptr};
+        void *a = nullptr, *b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            f.first = reinterpret_cast<CtxGetCurrentFn>(a);
+            f.second = reinterpret_cast<CtxGetIdFn>(b);
+        }
+        return f;
+    }();
+    if (!fns.first || !fns.second)
+        return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (fns.first(&ctx) != CUDA_SUCCESS || ctx == nullptr || fns.second(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
 
 }  // namespace
 
@@ -642,15 +684,23 @@ extern "C" df11_status df11_compress_device_noalloc(const df11_codebook *cb,
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
         return DF11_ERR_CUDA;
-    uintptr_t addr = g_noalloc_addr[dev].load(std::memory_order_acquire);
-    if (addr == 0) {
-        // host code only knows a stand-in for the array: ask the runtime for
-        // its address on the current device (once per device)
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
-            return DF11_ERR_CUDA;
-        addr = reinterpret_cast<uintptr_t>(ptr);
-        g_noalloc_addr[dev].store(addr, std::memory_order_release);
+    unsigned long long ctx = current_context_id();   // 0 before the runtime made one current
+    uintptr_t addr = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        NoAllocSlot &slot = g_noalloc_slot[dev];
+        if (ctx != 0 && slot.ctx_id == ctx) {
+            addr = slot.addr;
+        } else {
+            // host code only knows a stand-in for the array: ask the runtime
+            // for its address in the current context
+            void *ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+                return DF11_ERR_CUDA;
+            addr = reinterpret_cast<uintptr_t>(ptr);
+            slot.ctx_id = current_context_id();   // the lookup made a context current
+            slot.addr = addr;
+        }
     }
     return compress_device_impl(cb, layout, d_in, n, out, reinterpret_cast<void *>(addr), kNoAllocScratchBytes,
                                 false, d_error, stream);

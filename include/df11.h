@@ -370,7 +370,10 @@ df11_status df11_compress_device(const df11_codebook *cb, const df11_layout *lay
  *     with DF11_ERR_BUFFER_TOO_SMALL; nothing is launched.
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (with that device current); make that first call
- *     before any stream capture.  Later calls reuse the address.
+ *     before any stream capture.  Later calls in the same CUDA context reuse
+ *     the address; a call in another context (a new primary context after
+ *     cudaDeviceReset, or a driver context of the caller's) looks it up
+ *     again, so make the first call in each context before capturing too.
  *   - Every call shares the one array, which keeps the last call's contents;
  *     each call writes all it reads, so nothing needs clearing.  Calls whose
  *     work overlaps on the GPU (another stream, another host thread) race on

@@ -1,9 +1,10 @@
 """GPU-side compressor (histogram + encode kernels, through the C ABI)
-against the host compressor, which the oracle pins byte for byte.
+against the oracle's artifact and the host compressor.
 
 The artifact a block compresses to on the GPU must equal, array by array and
-byte by byte, the one the host library writes for the same codebook; the GPU
-decode of it must give back the input.  Page: "DFloat11: lossless BFloat16
+byte by byte, the oracle's own (oracle.compress_block with the codebook's
+code lengths) and the one the host library writes for the same codebook;
+the GPU decode of it must give back the input.  Page: "DFloat11: lossless BFloat16
 compression" ("How to develop with it": compression; "Architecture": the
 format's Gaps and output positions).
 """
@@ -34,6 +35,31 @@ def _dev(w):
     return torch.from_numpy(w.view(np.int16)).cuda()
 
 
+def check_against_oracle(mats, cb, db, bpt):
+    """The GPU arrays against the oracle's own artifact for the same code
+    lengths: the MSB-first stream, every thread's gap (the offset of the
+    first code starting in its slice), every chunk's output position and the
+    sign|mantissa bytes, byte for byte ("Architecture": Gaps and
+    BlockOutputPos; "How it works": encode)."""
+    ob = oracle.compress_block(mats, lengths=cb.lengths(), threads_per_chunk=32, bytes_per_thread=bpt)
+    assert db.header.total_bits == ob.total_bits and db.header.n_chunks == ob.n_chunks
+    stream = db.tensors["exp_stream"].cpu().numpy()
+    assert stream.size == ob.stream.size
+    bad = np.nonzero(stream != ob.stream)[0]
+    assert bad.size == 0, f"stream: {bad.size} bytes differ from the oracle, first at {bad[:8]}"
+    packed = db.tensors["gaps"].cpu().numpy()
+    gaps = np.empty(packed.size * 2, np.uint8)
+    gaps[0::2], gaps[1::2] = packed & 15, packed >> 4
+    assert gaps.size == ob.gap.size
+    bad = np.nonzero(gaps != ob.gap)[0]
+    assert bad.size == 0, f"gaps: {bad.size} threads differ from the oracle, first at {bad[:8]}"
+    pos = db.tensors["chunk_pos"].cpu().numpy().view(np.uint32)
+    assert np.array_equal(pos, ob.pos)
+    sm = db.tensors["signmant"].cpu().numpy()
+    assert np.array_equal(sm[: ob.signmant.size], ob.signmant)
+    assert not sm[ob.signmant.size:].any()
+
+
 def check_gpu_compress(mats, bpt=16):
     w = _flat(mats)
     d_in = _dev(w)
@@ -53,6 +79,7 @@ def check_gpu_compress(mats, bpt=16):
         want = a.view(np.uint8)
         bad = np.nonzero(got != want)[0]
         assert bad.size == 0, f"{name}: {bad.size} bytes differ, first at {bad[:8]}"
+    check_against_oracle(mats, cb, db, bpt)
     out = torch.empty(w.size, dtype=torch.int16, device="cuda")
     derr = torch.zeros(1, dtype=torch.int32, device="cuda")
     df11.decompress_async(db, out, derr)

@@ -9,6 +9,8 @@ Every generator is deterministic in its seed.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 # --------------------------------------------------------------- rounding
@@ -85,6 +87,29 @@ def llama_block(seed: int = 1000, scale_div: int = 1):
 def llama_model_seeds(n_blocks: int = 32, first_seed: int = 1000):
     """Seeds of the blocks of the 8B-scale stream (block i uses first_seed+i)."""
     return [first_seed + i for i in range(n_blocks)]
+
+
+def _llama_block_flat(args):
+    seed, scale_div = args
+    return seed, np.concatenate([m.reshape(-1) for _, m in llama_block(seed, scale_div=scale_div)])
+
+
+def llama_model_blocks(seeds, scale_div: int = 1, processes: int | None = None):
+    """Yields (seed, flat uint16 BF16 bits of llama_block(seed)) in seed
+    order, the blocks drawn by a pool of worker processes (numpy draws one
+    block on one core; a 32-block stream would take minutes serially).  The
+    pool uses the spawn start method, so it is safe in a process that has
+    already initialised CUDA.  Same numbers as llama_block(seed)."""
+    import multiprocessing as mp
+    seeds = list(seeds)
+    if processes is None:
+        processes = max(1, min(8, (os.cpu_count() or 2) - 1, len(seeds)))
+    if processes <= 1 or len(seeds) <= 1:
+        for sd in seeds:
+            yield _llama_block_flat((sd, scale_div))
+        return
+    with mp.get_context("spawn").Pool(processes) as pool:
+        yield from pool.imap(_llama_block_flat, [(sd, scale_div) for sd in seeds])
 
 
 def flux_block(seed: int = 5000, scale_div: int = 1):
