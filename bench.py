@@ -300,7 +300,8 @@ def cpu_baseline(oracle, hb, cb, bytes_per_weight, seconds):
 def e2e_plan(hb, pieces):
     """The chunk ranges of a piecewise end-to-end step and, for each, the
     byte spans of the arrays its range decode reads (df11_decompress_range_async:
-    stream words plus the 16-byte pad, gaps, positions incl. the next one,
+    stream words plus the 16-byte pad, gaps incl. the next thread's, counts,
+    positions incl. the next one,
     sign|mantissa rounded out to 16 bytes).  Returns [(c0, c1, p0, p1,
     [(array, begin, end), ...]), ...] with p0, p1 the output range."""
     n_chunks = int(hb.header.n_chunks)
@@ -312,7 +313,8 @@ def e2e_plan(hb, pieces):
     for c0, c1 in zip(cuts[:-1], cuts[1:]):
         p0, p1 = int(pos[c0]), int(pos[c1])
         spans = [("exp_stream", W * c0, min(W * c1 + 16, hb.exp_stream.nbytes)),
-                 ("gaps", 16 * c0, 16 * c1),
+                 ("gaps", 16 * c0, min(16 * c1 + 1, hb.gaps.nbytes)),
+                 ("counts", 32 * c0, 32 * c1),
                  ("chunk_pos", 4 * c0, 4 * (c1 + 1)),
                  ("signmant", p0 & ~15, min((p1 + 15) & ~15, hb.signmant.nbytes))]
         plan.append((c0, c1, p0, p1, spans))
@@ -369,7 +371,8 @@ def run_reference(args):
     mats = make_block(1000)
     n = int(sum(m.size for m in mats))
     ob = oracle.compress_block(mats)
-    comp_bytes = ob.stream.nbytes + ob.gap.size // 2 + ob.pos.nbytes + (n + 15) // 16 * 16
+    comp_bytes = (ob.stream.nbytes + ob.gap.size // 2 + ob.thread_count.size + ob.pos.nbytes
+                  + (n + 15) // 16 * 16)
     bytes_per_weight = (comp_bytes + 2 * n) / n
     plan = oracle_sample_plan(ob, 64)
 
@@ -1124,7 +1127,7 @@ def run_compress(args):
     torch.cuda.synchronize()
     ok = int(err.item()) == 0 and bool(torch.equal(out.view(torch.int16), d_in))
     hb = df11.compress(cb, [d_in.cpu().numpy().view(np.uint16)], 32, args.bytes_per_thread)
-    for name in ("exp_stream", "gaps", "chunk_pos", "signmant"):
+    for name in ("exp_stream", "gaps", "counts", "chunk_pos", "signmant"):
         a = db.tensors[name][: db.sizes[name]].cpu().numpy().view(np.uint8)
         h = getattr(hb, name).view(np.uint8)
         ok = ok and np.array_equal(a[: h.size], h) and not a[h.size:].any()
@@ -1179,10 +1182,10 @@ def run_verify(args):
     stream = torch.cuda.current_stream(dev)
     (db,), _, _ = gpu_compressed_blocks(1, 1000, dev, args.bytes_per_thread, scale_div=args.scale_div)
     expected = df11.checksum_device(db)
-    names = ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")
-    host = {a: db.tensors[a][: db.sizes[a]].cpu().numpy() for a in names}
+    host = {a: db.tensors[a][: db.sizes[a]].cpu().numpy() for a in ("exp_stream", "gaps", "counts", "chunk_pos",
+                                                                     "signmant", "lut")}
     hb = df11.HostBlock(header=db.header, exp_stream=host["exp_stream"], gaps=host["gaps"],
-                        chunk_pos=host["chunk_pos"].view(np.uint32), signmant=host["signmant"],
+                        counts=host["counts"], chunk_pos=host["chunk_pos"].view(np.uint32), signmant=host["signmant"],
                         lut=host["lut"].view(np.uint16))
     t0 = time.perf_counter()
     host_list = df11.checksum(hb)

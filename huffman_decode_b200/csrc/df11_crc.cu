@@ -8,8 +8,8 @@
 // corruption test in "How it works: the core algorithm").  Here the checksum
 // is a list: the CRC-32C (Castagnoli; reflected polynomial 0x82F63B78,
 // initial value and final XOR 0xFFFFFFFF) of every 4096-byte segment of the
-// block's five arrays, in the order exp_stream, gaps, chunk_pos, signmant,
-// lut (the last segment of an array is shorter).  Segments make the GPU
+// block's six arrays, in the order exp_stream, gaps, counts, chunk_pos,
+// signmant, lut (the last segment of an array is shorter).  Segments make the GPU
 // check embarrassingly parallel and locate damage.
 //
 // GPU method: one warp per segment, lane l covers bytes [128 l, 128 l + 128)
@@ -44,20 +44,25 @@ constexpr size_t kCrcSmem = (256 + (size_t)kShiftOps * 1024 + kPrivWords) * 4;
 
 static_assert(kSeg == 4096, "one warp of 32 lanes x 128 bytes per segment");
 
+constexpr int kArrays = 6;
+
 struct ArrayView {
-    const uint8_t *ptr[5];
-    uint64_t len[5];
-    uint64_t first[6];   // first segment index of each array; first[5] = total
+    const uint8_t *ptr[kArrays];
+    uint64_t len[kArrays];
+    uint64_t first[kArrays + 1];   // first segment index of each array; first[kArrays] = total
 };
 
-ArrayView view_of(const uint8_t *p0, uint64_t l0, const uint8_t *p1, uint64_t l1, const uint8_t *p2,
-                  uint64_t l2, const uint8_t *p3, uint64_t l3, const uint8_t *p4, uint64_t l4)
+template <class Block>
+ArrayView view_of(const Block *b)
 {
     ArrayView v;
-    const uint8_t *ps[5] = {p0, p1, p2, p3, p4};
-    const uint64_t ls[5] = {l0, l1, l2, l3, l4};
+    const uint8_t *ps[kArrays] = {b->exp_stream, b->gaps, b->counts,
+                                  reinterpret_cast<const uint8_t *>(b->chunk_pos), b->signmant,
+                                  reinterpret_cast<const uint8_t *>(b->lut)};
+    const uint64_t ls[kArrays] = {b->exp_stream_bytes, b->gaps_bytes, b->counts_bytes, b->chunk_pos_count * 4,
+                                  b->signmant_bytes, b->lut_entries * 2};
     v.first[0] = 0;
-    for (int a = 0; a < 5; ++a) {
+    for (int a = 0; a < kArrays; ++a) {
         v.ptr[a] = ps[a];
         v.len[a] = ls[a];
         v.first[a + 1] = v.first[a] + (ls[a] + kSeg - 1) / kSeg;
@@ -65,19 +70,6 @@ ArrayView view_of(const uint8_t *p0, uint64_t l0, const uint8_t *p1, uint64_t l1
     return v;
 }
 
-ArrayView view_of(const df11_host_block *b)
-{
-    return view_of(b->exp_stream, b->exp_stream_bytes, b->gaps, b->gaps_bytes,
-                   reinterpret_cast<const uint8_t *>(b->chunk_pos), b->chunk_pos_count * 4, b->signmant,
-                   b->signmant_bytes, reinterpret_cast<const uint8_t *>(b->lut), b->lut_entries * 2);
-}
-
-ArrayView view_of(const df11_device_block *b)
-{
-    return view_of(b->exp_stream, b->exp_stream_bytes, b->gaps, b->gaps_bytes,
-                   reinterpret_cast<const uint8_t *>(b->chunk_pos), b->chunk_pos_count * 4, b->signmant,
-                   b->signmant_bytes, reinterpret_cast<const uint8_t *>(b->lut), b->lut_entries * 2);
-}
 
 // ---- host ------------------------------------------------------------------
 
@@ -197,14 +189,14 @@ __global__ void __launch_bounds__(kCrcThreads) crc_kernel(ArrayView av, uint32_t
     // the initial value's part of a full segment's CRC
     const uint32_t init_full = advance(ops + 12 * 1024, 0xFFFFFFFFu);
     const uint64_t warps = blockDim.x >> 5;
-    const uint64_t total = av.first[5];
+    const uint64_t total = av.first[kArrays];
     for (uint64_t seg = blockIdx.x * warps + (tid >> 5); seg < total; seg += gridDim.x * warps) {
         // the array holding the segment: the last one whose first segment is
         // <= seg (empty arrays share their first index with the next one)
         const uint8_t *aptr = av.ptr[0];
         uint64_t alen = av.len[0], afirst = 0;
 #pragma unroll
-        for (int k = 1; k < 5; ++k)
+        for (int k = 1; k < kArrays; ++k)
             if (seg >= av.first[k]) {
                 aptr = av.ptr[k];
                 alen = av.len[k];
@@ -274,13 +266,13 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 df11_status launch_crc(const df11_device_block *blk, uint32_t *d_out, const uint32_t *d_expected,
                        uint64_t n_crc, uint32_t *d_error, uint64_t *d_first_bad, void *stream)
 {
-    if (!blk || !blk->exp_stream || !blk->gaps || !blk->chunk_pos || !blk->signmant || !blk->lut)
+    if (!blk || !blk->exp_stream || !blk->gaps || !blk->counts || !blk->chunk_pos || !blk->signmant || !blk->lut)
         return DF11_ERR_INVALID_ARGUMENT;
-    if (!aligned16(blk->exp_stream) || !aligned16(blk->gaps) || !aligned16(blk->chunk_pos) ||
+    if (!aligned16(blk->exp_stream) || !aligned16(blk->gaps) || !aligned16(blk->counts) || !aligned16(blk->chunk_pos) ||
         !aligned16(blk->signmant) || !aligned16(blk->lut))
         return DF11_ERR_INVALID_ARGUMENT;
     const ArrayView av = view_of(blk);
-    if (n_crc != av.first[5] || av.first[5] == 0)
+    if (n_crc != av.first[kArrays] || av.first[kArrays] == 0)
         return DF11_ERR_INVALID_ARGUMENT;
     if ((reinterpret_cast<uintptr_t>(d_out) & 3u) || (reinterpret_cast<uintptr_t>(d_expected) & 3u) ||
         (reinterpret_cast<uintptr_t>(d_error) & 3u) || (reinterpret_cast<uintptr_t>(d_first_bad) & 7u))
@@ -299,7 +291,7 @@ df11_status launch_crc(const df11_device_block *blk, uint32_t *d_out, const uint
         attr_done[dev].store(1, std::memory_order_release);
     }
     const uint64_t warps = kCrcThreads / 32;
-    const uint64_t need = (av.first[5] + warps - 1) / warps;
+    const uint64_t need = (av.first[kArrays] + warps - 1) / warps;
     const uint64_t cap = (uint64_t)sms;   // one 32-warp CTA per SM (the private table fills shared memory)
     const unsigned grid = (unsigned)(need < cap ? need : cap);
     crc_kernel<<<grid, kCrcThreads, kCrcSmem, reinterpret_cast<cudaStream_t>(stream)>>>(
@@ -313,17 +305,17 @@ extern "C" uint64_t df11_checksum_count(const df11_host_block *blk)
 {
     if (!blk)
         return 0;
-    return view_of(blk).first[5];
+    return view_of(blk).first[kArrays];
 }
 
 extern "C" df11_status df11_checksum(const df11_host_block *blk, uint32_t *crc, uint64_t n_crc)
 {
-    if (!blk || !crc || !blk->exp_stream || !blk->gaps || !blk->chunk_pos || !blk->signmant || !blk->lut)
+    if (!blk || !crc || !blk->exp_stream || !blk->gaps || !blk->counts || !blk->chunk_pos || !blk->signmant || !blk->lut)
         return DF11_ERR_INVALID_ARGUMENT;
     const ArrayView av = view_of(blk);
-    if (n_crc != av.first[5])
+    if (n_crc != av.first[kArrays])
         return DF11_ERR_INVALID_ARGUMENT;
-    for (int a = 0; a < 5; ++a)
+    for (int a = 0; a < kArrays; ++a)
         for (uint64_t s = 0; s < av.first[a + 1] - av.first[a]; ++s) {
             const uint64_t off = s * kSeg;
             const uint64_t n = av.len[a] - off < kSeg ? av.len[a] - off : kSeg;

@@ -7,22 +7,26 @@
 // bytes and written with coalesced stores; one launch covers every matrix of
 // a block (block-level batching).
 //
-// B200 design (differs from the page's two-phase kernel):
+// B200 design (differs from the page's kernel):
 //   * one warp = one chunk: output positions are stored per 32 threads, so
-//     every warp decodes, scans (shuffles), compacts and stores on its own,
+//     every warp counts, scans (shuffles), decodes and stores on its own,
 //     with no block-wide barrier after the prologue (the claimed schedule
 //     below adds one at the very end, to count the CTA out);
-//   * single decode pass with a multi-code table: an 11-bit window indexes a
+//   * two passes over the lane's slice, as on the page (count, then decode
+//     and write), both with a multi-code table: an 11-bit window indexes a
 //     2048-entry table (built in shared memory from the format's two-level
 //     16-bit tables) that yields up to four whole codes per lookup; longer
 //     codes fall back to the two-level tables;
+//   * the second pass writes each lane's exponents straight to their place
+//     in a contiguous, 8-element-aligned per-warp exponent buffer: four per
+//     word, ORed into the zeroed buffer, since a lane's first and last words
+//     are shared with its neighbours.  A lane's last lookup may also decode
+//     the next lane's first codes; they come from the same bit position, so
+//     ORing them again changes nothing.  No staging columns, no compaction:
+//     a warp needs 4.1 KB of shared memory instead of 6.3 KB;
 //   * exponents travel rotated right by one bit (bit 0 on top), which is
 //     where the BF16 halves want them: the merge is two bit-selects and two
 //     byte permutes per four weights, with no shifts;
-//   * decoded exponents are packed four per word into a per-warp slot column
-//     (row k holds word k of every lane: conflict-free stores), then moved
-//     into a contiguous, 8-element-aligned exponent buffer with funnel-shifted
-//     word stores (shared-memory OR only on words two lanes share);
 //   * the chunk's sign|mantissa bytes are staged into shared memory by one
 //     TMA bulk copy (cp.async.bulk + mbarrier) issued before decoding; the
 //     next chunk's stream words are loaded into registers a chunk ahead;
@@ -31,9 +35,9 @@
 //     least 2 bits long fit twice as many warps per SM;
 //   * the merge builds four BF16 values with two bit-selects and two byte
 //     permutes and writes one 16-byte vector per lane and group;
-//   * persistent CTAs of up to 32 warps (as many as shared memory holds;
-//     one CTA per SM for typical blocks, so all warps of an SM share one
-//     copy of the tables): grid = resident CTAs per SM x SM count;
+//   * persistent CTAs, grid = resident CTAs per SM x SM count: one CTA of up
+//     to 32 warps per SM, or two of up to 23 (a 40-register build), whichever
+//     keeps more warps resident -- two 23-warp CTAs for typical blocks;
 //   * with a scheduling workspace, the last few rounds of chunks are not
 //     dealt out but claimed one at a time from four global counters (each
 //     warp claims a chunk ahead, so the atomic's latency hides behind a
@@ -58,6 +62,8 @@ constexpr uint32_t kLutPointer = 0x8000u;
 constexpr int kWindowBits = 11;                    // multi-code table index width
 constexpr int kMultiEntries = 1 << kWindowBits;
 constexpr int kMaxCodesPerEntry = 4;
+static_assert(kWindowBits == DF11_DECODE_TABLE_WINDOW_BITS && kMultiEntries == DF11_DECODE_TABLE_ENTRIES,
+              "the host-built decode table has the kernel's shape");
 constexpr int kEntryBytes = 8;                     // multi-code entry: symbols | step
 constexpr uint32_t kLongStep = 0x80000000u;        // step of an entry whose first code is long
 constexpr int kMaxWarpsPerCta = 32;
@@ -76,6 +82,7 @@ constexpr uint32_t kWaitHintNs = 2000;              // longest suspension of one
 struct DecodeParams {
     const uint8_t *stream;
     const uint8_t *gaps;
+    const uint8_t *counts;
     const uint32_t *chunk_pos;
     const uint8_t *signmant;
     const uint16_t *lut;
@@ -87,7 +94,9 @@ struct DecodeParams {
     uint32_t n_tables;
     uint32_t min_len;     // shortest legal code; shorter table entries are corrupt
     uint32_t full_chunks; // chunks lying wholly below total_bits (every slice full)
+    uint64_t gaps_limit;  // gap bytes readable from `gaps` (the next thread's gap after the last chunk)
     uint32_t *sched;      // scheduling workspace, zero between launches; or null
+    const uint2 *multi_src;   // the multi-code table built on the host, or null
 };
 // Scheduling workspace: claim counter q at word q * kSchedStride (pools on
 // separate 256-byte stretches, so on different L2 lines), CTAs done at word
@@ -119,19 +128,22 @@ struct GemvParams {
 };
 
 // Per-warp buffers for W stream bytes per lane and codes of at least MINLEN
-// bits: slot columns, the contiguous exponent buffer, the staged
-// sign|mantissa bytes.
+// bits: the contiguous exponent buffer and the staged sign|mantissa bytes.
+// A lane writes its codes to the exponent buffer at its output offset head
+// (< 8) + off, off + count <= 32 kMaxCodes.  A corrupt stream can make the
+// lane's main loop write up to kMaxCodes + 1 codes whatever its count (every
+// code that starts below end - 10 + 11), so the buffer has that much slack.
 template <int W, int MINLEN>
 struct Geometry {
     static constexpr int kSliceBits = 8 * W;                         // 64 or 128
     static constexpr int kMaxCodes = (kSliceBits + MINLEN - 1) / MINLEN;  // per lane
-    static constexpr int kSlotRows = (kMaxCodes + 3 + 3) / 4;        // + codes past the end
-    static constexpr int kSlotBytes = kSlotRows * 32 * 4;
-    static constexpr int kEbufBytes = 32 * kMaxCodes + 16;           // multiple of 16
+    static constexpr int kEbufBytes = 33 * kMaxCodes + 16;           // multiple of 16
     static constexpr int kSbufBytes = 32 * kMaxCodes + 32;           // 16-aligned copy range
-    static constexpr int kWarpBytes = kSlotBytes + kEbufBytes + kSbufBytes;
+    static constexpr int kWarpBytes = kEbufBytes + kSbufBytes;
     static constexpr int kWords = W / 4 + 1;                         // stream words incl. halo
     static_assert(kWarpBytes % 16 == 0, "per-warp area must keep 16-byte alignment");
+    static_assert(kMaxCodes % 16 == 0, "buffer sizes keep 16-byte alignment");
+    static_assert(7 + (32 * kMaxCodes - 1) + (kMaxCodes + 1) + 3 <= kEbufBytes, "exponent buffer too small");
 };
 
 // Shared memory: mbarriers | multi-code table | code lengths | per-warp areas
@@ -208,12 +220,6 @@ __device__ __forceinline__ uint2 lds_v2(uint32_t a)
     asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
-__device__ __forceinline__ uint32_t lds_u32_m(uint32_t a)
-{
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-    return v;
-}
 __device__ __forceinline__ uint32_t lds_u8_m(uint32_t a)
 {
     uint32_t v;
@@ -226,38 +232,60 @@ __device__ __forceinline__ uint2 lds_v2_m(uint32_t a)
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
     return v;
 }
-__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v)
-{
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-__device__ __forceinline__ void sts_u32_if(bool p, uint32_t a, uint32_t v)
-{
-    asm volatile("{ .reg .pred q; setp.ne.u32 q, %2, 0; @q st.shared.u32 [%0], %1; }" ::"r"(a), "r"(v),
-                 "r"((uint32_t)p)
-                 : "memory");
-}
 __device__ __forceinline__ void red_or_u32(uint32_t a, uint32_t v)
 {
     asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v)
+{
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
 
 static_assert(kEntryBytes == 8, "lookup_step scales the table index by 8");
 
-// Lane decode state X: bit position in bits 0..15, fill of the slot word (in
-// bits, 0..24 between lookups) in bits 16..21; kLongStep (bit 31) is added by
-// an entry whose first code is longer than the window.
+// Lane decode state X: bit position in bits 0..15, fill of the word being
+// filled (in bits, 0..24 between lookups) in bits 16..21; kLongStep (bit 31)
+// is added by an entry whose first code is longer than the window.
 constexpr uint32_t kFillOne = 1u << 16;          // X units of one fill bit
 constexpr uint32_t kPosMask = 0xFFFFu | kLongStep;
 
 // One multi-code lookup for window `win` (the upcoming stream bits, first
-// lowest): appends the entry's symbols to the slot word at the fill, steps X,
-// computes the next window from the stream words lo:hi, and stores the word
-// (then carries the overflow) when it is full.  One predicated block, so the
-// store is not a branch; the next window is formed before the store so it
-// waits only on the step.
+// lowest): appends the entry's symbols to the word being filled at the
+// fill, steps X, computes the next window from the stream words lo:hi, and
+// stores the word to the exponent buffer (then carries the overflow) when
+// it is full (OR: ORs it into a zeroed buffer).  One predicated block, so
+// the store is not a branch; the next window is formed before the store so
+// it waits only on the step.
+template <bool OR>
 __device__ __forceinline__ void lookup_step(uint32_t &X, uint32_t &win, uint32_t &accl, uint32_t &sp,
                                             uint2 &r, uint32_t lo, uint32_t hi, uint32_t multi_a)
 {
+    if constexpr (OR)
+        asm volatile(
+        "{\n\t"
+        ".reg .b32 a, f, t, z, c;\n\t"
+        ".reg .pred p;\n\t"
+        "mov.b32 z, 0;\n\t"
+        "and.b32 a, %1, %9;\n\t"
+        "mad.lo.u32 a, a, 8, %8;\n\t"
+        "ld.shared.v2.u32 {%4, %5}, [a];\n\t"
+        "shr.b32 f, %0, 16;\n\t"
+        "shf.l.wrap.b32 t, z, %4, f;\n\t"
+        "or.b32 %2, %2, t;\n\t"
+        "shf.l.wrap.b32 c, %4, z, f;\n\t"
+        "add.u32 %0, %0, %5;\n\t"
+        "shf.r.wrap.b32 %1, %6, %7, %0;\n\t"
+        "and.b32 t, %0, 2097152;\n\t"
+        "setp.ne.u32 p, t, 0;\n\t"
+        "@p red.shared.or.b32 [%3], %2;\n\t"
+        "@p add.u32 %3, %3, 4;\n\t"
+        "@p mov.b32 %2, c;\n\t"
+        "@p sub.u32 %0, %0, 2097152;\n\t"
+        "}"
+        : "+r"(X), "+r"(win), "+r"(accl), "+r"(sp), "=r"(r.x), "=r"(r.y)
+        : "r"(lo), "r"(hi), "r"(multi_a), "n"(kMultiEntries - 1)
+        : "memory");
+    else
     asm volatile(
         "{\n\t"
         ".reg .b32 a, f, t, z, c;\n\t"
@@ -275,7 +303,7 @@ __device__ __forceinline__ void lookup_step(uint32_t &X, uint32_t &win, uint32_t
         "and.b32 t, %0, 2097152;\n\t"           // fill >= 32
         "setp.ne.u32 p, t, 0;\n\t"
         "@p st.shared.u32 [%3], %2;\n\t"
-        "@p add.u32 %3, %3, 128;\n\t"
+        "@p add.u32 %3, %3, 4;\n\t"
         "@p mov.b32 %2, c;\n\t"
         "@p sub.u32 %0, %0, 2097152;\n\t"
         "}"
@@ -324,13 +352,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
     return false;
 }
 
-// Loads the lane's stream words and gap.  Words are bit-reversed: stream bit
-// 32k + i (MSB-first in the bytes) is bit i of word k, so a right funnel
-// shift by the bit position leaves the upcoming bits, first bit lowest.
+// Loads the lane's stream words and its thread metadata: meta = gap |
+// next thread's gap << 4 (lane 31 only; the other lanes take it from their
+// neighbour) | count << 8.  Words are bit-reversed: stream bit 32k + i
+// (MSB-first in the bytes) is bit i of word k, so a right funnel shift by the
+// bit position leaves the upcoming bits, first bit lowest.
 template <int W>
-__device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, uint32_t (&w)[W / 4 + 1],
-                                           uint32_t &gap)
+__device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t chunk, int lane,
+                                           uint32_t (&w)[W / 4 + 1], uint32_t &meta)
 {
+    const uint64_t g = chunk * 32 + lane;
     const uint8_t *src = p.stream + (uint64_t)W * g;
     if constexpr (W == 8) {
         const uint2 a = *reinterpret_cast<const uint2 *>(src);
@@ -345,7 +376,9 @@ __device__ __forceinline__ void load_slice(const DecodeParams &p, uint64_t g, ui
         w[3] = __brev(bswap32(a.w));
         w[4] = __brev(bswap32(*reinterpret_cast<const uint32_t *>(src + 16)));
     }
-    gap = (p.gaps[g >> 1] >> ((g & 1) * 4)) & 0xFu;
+    meta = ((p.gaps[g >> 1] >> ((g & 1) * 4)) & 0xFu) | ((uint32_t)p.counts[g] << 8);
+    if (lane == 31 && 16 * (chunk + 1) < p.gaps_limit)
+        meta |= (p.gaps[16 * (chunk + 1)] & 0xFu) << 4;
 }
 
 // Matrix of block element e: the last one whose start is <= e.
@@ -483,6 +516,130 @@ __device__ __forceinline__ void gemv_chunk(const GemvParams *gp, uint32_t head, 
     }
 }
 
+// Two-level table lookup of the code at the front of window `win` (first
+// stream bit lowest): the entry as the multi-code table would hold it for
+// that one code (rotated exponent; length | 8 << 16).
+__device__ __forceinline__ uint2 long_code(uint32_t win, uint32_t lut_a, uint32_t &seen)
+{
+    const uint32_t wm = __brev(win);
+    uint32_t e = lds_u16(lut_a + ((wm >> 24) << 1));
+    if (e & kLutPointer)
+        e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((wm >> 16) & 0xFFu)) << 1));
+    seen |= e;
+    return make_uint2(rot_exp(e & 0xFFu), ((e >> 8) & 0x1Fu) | (8u * kFillOne));
+}
+
+// Decodes the codes of a full slice (every lane of the chunk has one) into
+// the exponent buffer: this lane's codes go to bytes a, a + 1, ... (a =
+// offset within the buffer at shared-window address ebuf_a), four per word,
+// and each word is stored as it fills (the fill starts at byte a's place in
+// its word).  Its last lookup may also decode the first codes of the next
+// lane: they come from the same bit position, so they are the next lane's
+// own bytes.  A word two lanes share (the word a lane's run ends in, when
+// the next lane's run starts inside it) is stored by both: by the next lane
+// when it fills its first word (zeros below its first byte), and by this
+// lane when the next lane's first codes, decoded at its end, complete the
+// word.  The next lane fills its first word within its first 64 bits (at
+// most three codes from bit 15); this lane completes the word only in the
+// lookup that crosses the slice end, so a warp barrier after the first two
+// stream words puts the complete word last.  A last word still part-filled
+// at the end is left in accl at address sp (fill in X) for the caller to OR
+// in.  Returns X: bit position after the last lookup (bits 0..15), fill
+// (bits 16..21); r holds the last table entry.
+template <int W>
+__device__ __forceinline__ uint32_t decode_full_slice(const uint32_t (&w)[W / 4 + 1], uint32_t gap, uint32_t a,
+                                                      uint32_t ebuf_a, uint32_t multi_a, uint32_t lut_a,
+                                                      uint32_t &seen, uint32_t &sp, uint32_t &accl, uint2 &r)
+{
+    constexpr int kWords = W / 4 + 1;
+    constexpr int kSliceBits = 8 * W;
+    // 128-bit slices: plain stores, ordered as above; 64-bit slices are too
+    // short for that order, so their words are ORed into a zeroed buffer
+    constexpr bool kOr = kSliceBits - (kWindowBits - 1) <= 64;
+    uint32_t X = gap | ((a & 3u) << 19);
+    sp = ebuf_a + (a & ~3u);
+    accl = 0;
+    r = make_uint2(0u, 0u);
+#pragma unroll
+    for (int h = 0; h < kWords - 1; ++h) {
+        if (!kOr && h == 2)
+            __syncwarp();   // every lane's first word is stored by now
+        const uint32_t lo = w[h], hi = w[h + 1];
+        const uint32_t lim = (uint32_t)min(kSliceBits, 32 * (h + 1));
+        uint32_t win = __funnelshift_r(lo, hi, X);
+        for (;;) {
+            while ((X & kPosMask) < lim)
+                lookup_step<kOr>(X, win, accl, sp, r, lo, hi, multi_a);
+            if (X < kLongStep)
+                break;
+            // the first code is longer than the window: take it from the
+            // two-level tables
+            X -= kLongStep;
+            r = long_code(win, lut_a, seen);
+            const uint32_t f = X >> 16;
+            accl |= __funnelshift_l(0u, r.x, f);
+            const uint32_t acch = __funnelshift_l(r.x, 0u, f);
+            X += r.y;
+            if (X & (32u * kFillOne)) {
+                if constexpr (kOr)
+                    red_or_u32(sp, accl);
+                else
+                    sts_u32(sp, accl);
+                sp += 4;
+                accl = acch;
+                X -= 32u * kFillOne;
+            }
+            win = __funnelshift_r(lo, hi, X);
+        }
+    }
+    return X;
+}
+
+// The slice of a lane in the block's last chunk, whose slices may end at
+// the end of the stream (end < slice width) or lie past it: one code at a
+// time, one byte store per code, exactly `cnt` codes.  Returns the number of
+// codes that start in [gap, end), or cnt + 1 when there are more than cnt,
+// and the bit position after the last code counted in *after.
+template <int W>
+__device__ __forceinline__ uint32_t decode_last_slice(const uint32_t (&w)[W / 4 + 1], uint32_t gap, uint32_t cnt,
+                                                      int end, uint32_t a, uint32_t ebuf_a, uint32_t multi_a,
+                                                      uint32_t lut_a, uint32_t len_a, uint32_t &seen,
+                                                      uint32_t &after)
+{
+    constexpr int kWords = W / 4 + 1;
+    uint32_t X = gap, k = 0;
+    while ((int)X < end && k <= cnt) {
+        const uint32_t hw = min(X >> 5, (uint32_t)(kWords - 2));
+        uint32_t lo = w[0], hi = w[1];
+#pragma unroll
+        for (int i = 1; i < kWords - 1; ++i)
+            if (hw == (uint32_t)i) {
+                lo = w[i];
+                hi = w[i + 1];
+            }
+        const uint32_t win = __funnelshift_r(lo, hi, X);
+        uint2 e = lds_v2(multi_a + (win & (kMultiEntries - 1)) * kEntryBytes);
+        uint32_t sym, len;
+        if (e.y == kLongStep) {
+            e = long_code(win, lut_a, seen);
+            sym = e.x;
+            len = e.y & 0xFFFFu;
+        } else {
+            sym = e.x & 0xFFu;
+            len = lds_u8(len_a + sym);
+        }
+        if (k < cnt) {
+            asm volatile("st.shared.u8 [%0], %1;" ::"r"(ebuf_a + a + k), "r"(sym) : "memory");
+            after = X + len;
+        }
+        X += len;
+        ++k;
+    }
+    if (k == 0)
+        after = gap;
+    return k;
+}
+
 // The chunk body.  TT = 0: BF16 output; TT > 0: fused matrix-vector product
 // for up to TT tokens (gp != nullptr).
 template <int W, int MINLEN, int TT>
@@ -507,28 +664,31 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     const uint32_t no_code = 0x4000u | (min_len << 8);
 
     // ---- this warp's first chunk: its loads overlap the table build ---------
-    const uint64_t n_warps = (uint64_t)gridDim.x * warps;
-    const uint64_t gw = (uint64_t)blockIdx.x * warps + warp;
-    uint64_t chunk = gw;
+    // (chunk indices fit in 32 bits: a block has fewer than 2^32 elements,
+    // and a chunk holds at least 32 slices of 64 bits)
+    const uint32_t n_chunks = (uint32_t)p.n_chunks;
+    const uint32_t n_warps = gridDim.x * (uint32_t)warps;
+    const uint32_t gw = blockIdx.x * (uint32_t)warps + (uint32_t)warp;
+    uint32_t chunk = gw;
     // Rounds below r_static are dealt out: chunk gw + k n_warps is this
     // warp's k-th.  With a workspace, chunks from d0 on are claimed: pool q
     // holds d0 + q, d0 + q + 4, ..., and warp gw claims from pool gw % 4.
     // Blocks of fewer rounds keep the plain deal: their imbalance is the
     // rounding of chunks to warps, which claiming cannot remove.
-    const uint64_t rounds = p.n_chunks / n_warps;
-    const uint64_t r_static = rounds - kSchedTailRounds;
-    const uint64_t d0 = r_static * n_warps;
-    const bool dyn = p.sched != nullptr && rounds >= (uint64_t)kSchedTailRounds + 2;
-    const uint32_t q = (uint32_t)(gw % kSchedPools);
+    const uint32_t rounds = n_chunks / n_warps;
+    const uint32_t r_static = rounds - kSchedTailRounds;
+    const uint32_t d0 = r_static * n_warps;
+    const bool dyn = p.sched != nullptr && rounds >= (uint32_t)kSchedTailRounds + 2;
+    const uint32_t q = gw % kSchedPools;
     uint32_t *const pool = p.sched + q * kSchedStride;
     uint32_t claim = 0;   // lane 0: the last claim's result
     uint32_t w[G::kWords];
-    uint32_t gap = 0, pos0 = 0, pos1 = 0;
+    uint32_t meta = 0, pos0 = 0, pos1 = 0;
 #pragma unroll
     for (int k = 0; k < G::kWords; ++k)
         w[k] = 0;
-    if (chunk < p.n_chunks) {
-        load_slice<W>(p, chunk * 32 + lane, w, gap);
+    if (chunk < n_chunks) {
+        load_slice<W>(p, chunk, lane, w, meta);
         pos0 = p.chunk_pos[chunk];
         pos1 = p.chunk_pos[chunk + 1];
     }
@@ -564,26 +724,44 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     // the first code is longer than the window (or is no code) the entry is
     // x = 0, y = kLongStep: adding it ends the lookup loop, and the decoder
     // takes the two-level path.
-    for (int slot = tid; slot < kMultiEntries; slot += blockDim.x) {
-        // consecutive threads fill consecutive entries (conflict-free stores)
-        const uint32_t idx = __brev((uint32_t)slot) >> (32 - kWindowBits);
-        const uint32_t win = idx << (32 - kWindowBits);   // MSB-first window
-        uint32_t t = 0, n = 0, syms = 0;
-        while (n < kMaxCodesPerEntry) {
-            const uint32_t v = win << t;
-            uint32_t e = lut[v >> 24];
-            if (e & kLutPointer)
-                e = lut[((e & 0xFFu) << 8) | ((v >> 16) & 0xFFu)];
-            if (e & 0x4000u)
-                break;
-            const uint32_t l = (e >> 8) & 0x1Fu;
-            if (t + l > (uint32_t)kWindowBits)
-                break;
-            syms |= rot_exp(e & 0xFFu) << (8 * n);
-            ++n;
-            t += l;
+    if (p.multi_src) {
+        // built once on the host (df11_build_decode_table): copied, and any
+        // entry whose count and length no table of this block could hold
+        // becomes the long-code marker, so a lane still advances at least
+        // min_len bits per code and never writes more codes than its buffer
+        // holds
+        for (int slot = tid; slot < kMultiEntries; slot += blockDim.x) {
+            uint2 v = __ldg(p.multi_src + slot);
+            const uint32_t n = v.y >> 19, t = v.y & 0xFFFFu;
+            if (v.y != (t | (n << 19)) || n < 1 || n > (uint32_t)kMaxCodesPerEntry ||
+                t > (uint32_t)kWindowBits || t < n * min_len)
+                v = make_uint2(0u, kLongStep);
+            else if (n < 4)
+                v.x &= (1u << (8 * n)) - 1u;
+            multi[slot] = v;
         }
-        multi[slot] = make_uint2(syms, n ? t | (8u * n << 16) : kLongStep);
+    } else {
+        for (int slot = tid; slot < kMultiEntries; slot += blockDim.x) {
+            // consecutive threads fill consecutive entries (conflict-free stores)
+            const uint32_t idx = __brev((uint32_t)slot) >> (32 - kWindowBits);
+            const uint32_t win = idx << (32 - kWindowBits);   // MSB-first window
+            uint32_t t = 0, n = 0, syms = 0;
+            while (n < kMaxCodesPerEntry) {
+                const uint32_t v = win << t;
+                uint32_t e = lut[v >> 24];
+                if (e & kLutPointer)
+                    e = lut[((e & 0xFFu) << 8) | ((v >> 16) & 0xFFu)];
+                if (e & 0x4000u)
+                    break;
+                const uint32_t l = (e >> 8) & 0x1Fu;
+                if (t + l > (uint32_t)kWindowBits)
+                    break;
+                syms |= rot_exp(e & 0xFFu) << (8 * n);
+                ++n;
+                t += l;
+            }
+            multi[slot] = make_uint2(syms, n ? t | (8u * n << 16) : kLongStep);
+        }
     }
     __syncthreads();
 
@@ -592,19 +770,17 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     const uint32_t multi_a = smem_base + (uint32_t)kBarBytes;
     const uint32_t len_a = multi_a + kMultiEntries * kEntryBytes;
     const uint32_t lut_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warps * G::kWarpBytes);
-    const uint32_t slots_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warp * G::kWarpBytes);
-    const uint32_t slot_lane_a = slots_a + 4u * lane;      // row 0 of this lane's column
-    const uint32_t ebuf_a = slots_a + G::kSlotBytes;
+    const uint32_t ebuf_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warp * G::kWarpBytes);
     const uint32_t sbuf_a = ebuf_a + G::kEbufBytes;
     const uint32_t bar = smem_addr(&mbar[warp]);
     uint32_t parity = 0;
 
-    if (chunk >= p.n_chunks)   // (never with the dynamic schedule)
+    if (chunk >= n_chunks)   // (never with the dynamic schedule)
         return;
 
     uint32_t err = 0;
     bool stalled = false;      // a staged copy did not arrive in time
-    uint64_t n_done = 0;       // chunks this warp has finished
+    uint32_t n_done = 0;       // chunks this warp has finished
 
     for (;;) {
         // ---- positions (warp-uniform) and the staged sign|mantissa copy -----
@@ -625,182 +801,124 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             bulk_copy_g2s(sbuf_a, p.signmant + cp_lo, cp_bytes, bar);
 
         // ---- the next chunk's slice and positions, loaded ahead -------------
-        uint64_t next;
+        uint32_t next;
         if (!dyn || n_done + 1 < r_static) {
             next = chunk + n_warps;
             if (dyn && n_done + 2 == r_static && lane == 0)
                 claim = atomicAdd(pool, 1u);      // the first claimed chunk, a chunk ahead
         } else {
-            next = d0 + q + (uint64_t)kSchedPools * __shfl_sync(0xFFFFFFFFu, claim, 0);
-            if (lane == 0 && next < p.n_chunks)
+            next = d0 + q + kSchedPools * __shfl_sync(0xFFFFFFFFu, claim, 0);
+            if (lane == 0 && next < n_chunks)
                 claim = atomicAdd(pool, 1u);      // the chunk after next
         }
-        const bool has_next = next < p.n_chunks;
+        const bool has_next = next < n_chunks;
         uint32_t nw[G::kWords];
-        uint32_t ngap = 0, npos0 = 0, npos1 = 0;
+        uint32_t nmeta = 0, npos0 = 0, npos1 = 0;
         if (has_next) {
-            load_slice<W>(p, next * 32 + lane, nw, ngap);
+            load_slice<W>(p, next, lane, nw, nmeta);
             npos0 = p.chunk_pos[next];
             npos1 = p.chunk_pos[next + 1];
         }
 
+        // thread metadata: gap, count and the next thread's gap
+        const uint32_t gap = meta & 0xFu;
+        const uint32_t cnt = meta >> 8;
+        const uint32_t gap_up = __shfl_down_sync(0xFFFFFFFFu, gap, 1);
+        const uint32_t gnext = lane == 31 ? (meta >> 4) & 0xFu : gap_up;
+        // ---- warp scan of the stored counts: each lane's output offset -----
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d)
+                incl += y;
+        }
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const uint32_t off = incl - cnt;
+        const bool counts_ok = !__any_sync(0xFFFFFFFFu, cnt > (uint32_t)G::kMaxCodes) && total == pos1 - pos0;
         if (!pos_ok) {
             err |= DF11_DEVERR_BAD_POS;
+        } else if (!counts_ok) {
+            err |= DF11_DEVERR_COUNT;
         } else {
-            // ---- decode this lane's slice ----------------------------------
-            // Codes starting in [gap, end) belong to this lane.  The loop
-            // runs while bitpos < end; the last table entry may also hold
-            // codes that start at or past `end` -- they are dropped below.
-            // Chunks below the last are full: end is the constant slice width.
+            const uint32_t n_write = total;
+            // The lane's codes start in [gap, end): end is the slice width,
+            // or the end of the stream in the block's last chunk; the next
+            // code (the next thread's first, or the end of the stream) must
+            // start where they end.
+
+            // ---- decode this lane's codes straight into place ---------------
+            // Lane bytes go to ebuf[head + off, head + off + cnt).
+            const uint32_t a = head + off;
+            // (checked build) every word the lane may store lies in the
+            // buffer: at most kMaxCodes + 3 codes from a
+            const bool write_ok =
+                __all_sync(0xFFFFFFFFu, DF11_CHECK(err, a + G::kMaxCodes + 8 <= (uint32_t)G::kEbufBytes));
             uint32_t seen = 0;
-            auto decode = [&](auto end_arg) -> uint32_t {
-                const int end = end_arg;
-                uint32_t X = gap;
-                uint32_t accl = 0;
-                uint32_t sp = slot_lane_a;           // next slot word of this lane
-                uint2 r = make_uint2(0u, 0u);        // last entry
-#pragma unroll
-                for (int h = 0; h < G::kWords - 1; ++h) {
-                    const uint32_t lo = w[h], hi = w[h + 1];
-                    const uint32_t lim = (uint32_t)min(end, 32 * (h + 1));
-                    uint32_t win = __funnelshift_r(lo, hi, X);
-                    for (;;) {
-                        while ((X & kPosMask) < lim)
-                            lookup_step(X, win, accl, sp, r, lo, hi, multi_a);
-                        if (X < kLongStep)
-                            break;
-                        // the first code is longer than the window: take it
-                        // from the two-level tables (MSB-first window)
-                        X -= kLongStep;
-                        const uint32_t wm = __brev(win);
-                        uint32_t e = lds_u16(lut_a + ((wm >> 24) << 1));
-                        if (e & kLutPointer)
-                            e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((wm >> 16) & 0xFFu)) << 1));
-                        seen |= e;
-                        r = make_uint2(rot_exp(e & 0xFFu), ((e >> 8) & 0x1Fu) | (8u * kFillOne));
-                        const uint32_t f = X >> 16;
-                        accl |= __funnelshift_l(0u, r.x, f);
-                        const uint32_t acch = __funnelshift_l(r.x, 0u, f);
-                        X += r.y;
-                        if (X & (32u * kFillOne)) {
-                            sts_u32(sp, accl);
-                            sp += 128;
-                            accl = acch;
-                            X -= 32u * kFillOne;
-                        }
-                        win = __funnelshift_r(lo, hi, X);
-                    }
-                }
-                const uint32_t fill = X >> 16;
-                // the lane's slot words stayed inside its column
-                (void)DF11_CHECK(err, sp - slot_lane_a < 128u * (uint32_t)G::kSlotRows);
-                if (fill)
-                    sts_u32(sp, accl);
-                uint32_t cnt = ((sp - slot_lane_a) >> 5) + (fill >> 3);   // 4 codes per 128-byte row
-                if (cnt) {
-                    // codes of the last entry that start at or past `end`
-                    const uint32_t n = r.y >> 19;
-                    int c = (int)(X & 0xFFFFu) - (int)(r.y & 0xFFFFu);   // start of the entry's first code
-                    uint32_t keep = 1;
-#pragma unroll
-                    for (uint32_t k = 1; k < (uint32_t)kMaxCodesPerEntry; ++k) {
-                        c += (int)lds_u8(len_a + ((r.x >> (8 * (k - 1))) & 0xFFu));
-                        keep += (k < n && c < end) ? 1u : 0u;
-                    }
-                    cnt -= n - keep;
-                }
-                return cnt;
-            };
-            uint32_t count;
+            bool lane_bad = false;
             if (chunk < p.full_chunks) {
-                count = decode(ConstInt<G::kSliceBits>{});
+                constexpr bool kOr = G::kSliceBits - (kWindowBits - 1) <= 64;
+                if constexpr (kOr) {
+                    // zero the words the lanes OR into (up to the next
+                    // lane's first codes after the last lane's run)
+                    const uint32_t zend = min((uint32_t)G::kEbufBytes, (head + total + 6u + 15u) & ~15u);
+                    for (uint32_t i = 16u * lane; i < zend; i += 512u)
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(ebuf_a + i), "r"(0u)
+                                     : "memory");
+                    __syncwarp();
+                }
+                uint32_t sp = 0, accl = 0;
+                uint2 r = make_uint2(0u, 0u);
+                uint32_t X = 0;
+                if (write_ok)
+                    X = decode_full_slice<W>(w, gap, a, ebuf_a, multi_a, lut_a, seen, sp, accl, r);
+                // codes of the last entry that start at or past the slice
+                // end are the next lane's; the first of them (or the end of
+                // the entry) is where the next code starts
+                const uint32_t emitted = sp - ebuf_a + ((X >> 19) & 7u) - a;
+                const uint32_t n = r.y >> 19;
+                int c = (int)(X & 0xFFFFu) - (int)(r.y & 0xFFFFu);   // start of the entry's first code
+                uint32_t keep = n ? 1u : 0u;
+                int next_start = (int)(X & 0xFFFFu);
+#pragma unroll
+                for (uint32_t k = 1; k < (uint32_t)kMaxCodesPerEntry; ++k) {
+                    c += (int)lds_u8(len_a + ((r.x >> (8 * (k - 1))) & 0xFFu));
+                    if (k < n && c < G::kSliceBits)
+                        ++keep;
+                    else if (k == keep && k < n)
+                        next_start = c;
+                }
+                // a full chunk's next code starts at the next slice's gap
+                // (the end of the stream when that is the slice end)
+                lane_bad = emitted - (n - keep) != cnt || next_start != G::kSliceBits + (int)gnext;
+                __syncwarp();
+                // the part-filled last word: ORed over the next lane's first
+                // word (zeros below its first byte); the last lane's is its own
+                if (write_ok && (X >> 16)) {
+                    if (kOr || lane < 31)
+                        red_or_u32(sp, accl);
+                    else
+                        sts_u32(sp, accl);
+                }
             } else {
+                // the block's last chunk: slices end at the end of the stream
                 const uint64_t bit0 = ((uint64_t)chunk * 32 + lane) * (uint64_t)G::kSliceBits;
-                count = decode(bit0 >= p.total_bits
-                                   ? 0
-                                   : (int)min((uint64_t)G::kSliceBits, p.total_bits - bit0));
+                int end = G::kSliceBits;
+                int expect = G::kSliceBits + (int)gnext;
+                if (bit0 + G::kSliceBits >= p.total_bits) {
+                    end = bit0 >= p.total_bits ? 0 : (int)(p.total_bits - bit0);
+                    expect = end;
+                }
+                uint32_t after = 0;
+                const uint32_t k = write_ok ? decode_last_slice<W>(w, gap, cnt, end, a, ebuf_a, multi_a, lut_a,
+                                                                   len_a, seen, after)
+                                            : cnt;
+                lane_bad = k != cnt || (cnt && (int)after != expect);
             }
+            if (lane_bad)
+                err |= DF11_DEVERR_COUNT;
             if (seen & 0x4000u)
                 err |= DF11_DEVERR_BAD_CODE;
-
-            // ---- warp scan of the counts ------------------------------------
-            uint32_t incl = count;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-                if (lane >= d)
-                    incl += y;
-            }
-            const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-            const uint32_t off = incl - count;
-            if (total != pos1 - pos0)
-                err |= DF11_DEVERR_COUNT;
-            const uint32_t n_write = min(total, pos1 - pos0);
-
-            // ---- compaction into the exponent buffer ------------------------
-            // Lane bytes go to ebuf[head + off, head + off + nbytes).  Words the
-            // lane covers entirely are plain stores; the first and last word
-            // may be shared with neighbouring lanes: zeroed, then ORed.
-            uint32_t nbytes = off < n_write ? min(count, n_write - off) : 0u;
-            if (!DF11_CHECK(err, head + off + nbytes <= (uint32_t)G::kEbufBytes))
-                nbytes = 0;
-            const uint32_t a = head + off;
-            const uint32_t sh = (a & 3u) * 8;
-            const uint32_t first = a >> 2;
-            const uint32_t last = (a + nbytes - 1) >> 2;
-            const bool head_shared = sh != 0;
-            const bool tail_shared = ((a + nbytes) & 3u) != 0;
-            const uint32_t nwords = (nbytes + 3) >> 2;
-            const uint32_t first_a = ebuf_a + 4u * first;
-            const uint32_t last_a = ebuf_a + 4u * last;
-            if (nbytes) {
-                if (head_shared)
-                    sts_u32(first_a, 0u);
-                if (tail_shared)
-                    sts_u32(last_a, 0u);
-                if (nbytes & 3u) {                       // clear bytes past nbytes
-                    const uint32_t ta = slot_lane_a + (nwords - 1) * 128;
-                    sts_u32(ta, lds_u32_m(ta) & ((1u << (8 * (nbytes & 3u))) - 1));
-                }
-            }
-            __syncwarp();
-            if (nbytes) {
-                // first word: slot word 0 shifted into place
-                const uint32_t v = lds_u32_m(slot_lane_a) << sh;
-                if (head_shared || (first == last && tail_shared))
-                    red_or_u32(first_a, v);
-                else
-                    sts_u32(first_a, v);
-                // last word, when it is not the first
-                if (last > first) {
-                    const uint32_t L = last - first;
-                    const uint32_t prev = lds_u32_m(slot_lane_a + 128 * (L - 1));
-                    const uint32_t cur = L < nwords ? lds_u32_m(slot_lane_a + 128 * L) : 0u;
-                    const uint32_t t = __funnelshift_l(prev, cur, sh);
-                    if (tail_shared)
-                        red_or_u32(last_a, t);
-                    else
-                        sts_u32(last_a, t);
-                }
-            }
-            {
-                // middle words first+1 .. last-1, wholly this lane's: a
-                // warp-uniform trip count, four words a step, stores
-                // predicated per lane.  Rows past a lane's last slot word
-                // are read but never stored (they lie at most two rows past
-                // the slot columns, inside the warp's exponent buffer).
-                const uint32_t m = (nbytes && last > first) ? last - first - 1 : 0u;
-                const uint32_t mmax = __reduce_max_sync(0xFFFFFFFFu, m);
-                uint32_t prev = lds_u32_m(slot_lane_a);
-                for (uint32_t k = 1; k <= mmax; k += 4) {
-#pragma unroll
-                    for (uint32_t u = 0; u < 4; ++u) {
-                        const uint32_t cur = lds_u32_m(slot_lane_a + 128 * (k + u));
-                        sts_u32_if(k + u <= m, first_a + 4 * (k + u), __funnelshift_l(prev, cur, sh));
-                        prev = cur;
-                    }
-                }
-            }
             __syncwarp();
 
             // ---- wait for the staged sign|mantissa bytes --------------------
@@ -861,7 +979,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
 #pragma unroll
         for (int k = 0; k < G::kWords; ++k)
             w[k] = nw[k];
-        gap = ngap;
+        meta = nmeta;
         pos0 = npos0;
         pos1 = npos1;
     }
@@ -903,8 +1021,16 @@ __global__ void bounded_wait_kernel(uint32_t polls, uint32_t *status)
         *status = done ? 0u : DF11_DEVERR_TIMEOUT;
 }
 
-template <int W, int MINLEN>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_decode_kernel(DecodeParams p)
+// A decode kernel is compiled for one resident CTA per SM (up to 32 warps)
+// or two (up to 23 warps each): with two, the register cap is 40 per thread
+// (11.5 warps per SM sub-partition), and two 23-warp CTAs fill the SM's
+// shared memory with 46 warps instead of 32.  Each CTA holds its own copy
+// of the tables.
+template <int CPS>
+constexpr int kCtaWarps = CPS == 1 ? kMaxWarpsPerCta : 23;
+
+template <int W, int MINLEN, int CPS>
+__global__ void __launch_bounds__(kCtaWarps<CPS> * 32, CPS) df11_decode_kernel(DecodeParams p)
 {
     decode_body<W, MINLEN, 0>(p, nullptr);
 }
@@ -919,45 +1045,74 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_gemv_kernel(DecodeP
 // ------------------------------------------------------------ launch
 
 constexpr int kMaxDevices = 64;
-constexpr size_t kSmemLimit = 227 * 1024;
-// kernel variants: (slice width, shortest code) x (store, products for 1, 2,
-// 4, 8 tokens)
-constexpr int kVariants = 4 * 5;
+// kernel variants: (slice width, shortest code) x (store with one CTA per
+// SM, products for 1, 2, 4, 8 tokens, store with two CTAs per SM)
+constexpr int kVariantsPerLayout = 6;
+constexpr int kVariants = 4 * kVariantsPerLayout;
 // resident CTAs per SM, by device, kernel variant and table count
 std::atomic<int> g_occupancy[kMaxDevices][kVariants][257];
-std::atomic<int> g_sm_count[kMaxDevices];
 std::atomic<int> g_attr_done[kMaxDevices][kVariants];
+
+// Per-device properties the launch shapes need (read once).
+struct DeviceProps {
+    int sms;
+    int smem_per_sm;      // shared memory of one SM
+    int smem_reserved;    // shared memory the system reserves per CTA
+    int smem_optin;       // largest dynamic shared memory of one CTA
+};
+std::atomic<int> g_props_done[kMaxDevices];
+DeviceProps g_props[kMaxDevices];
+
+df11_status device_props(int dev, DeviceProps &out)
+{
+    if (!g_props_done[dev].load(std::memory_order_acquire)) {
+        DeviceProps d;
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return DF11_ERR_CUDA;
+        g_props[dev] = d;   // identical values if two threads race here
+        g_props_done[dev].store(1, std::memory_order_release);
+    }
+    out = g_props[dev];
+    return DF11_OK;
+}
 
 struct LaunchShape {
     int warps;
     size_t smem;
     unsigned grid;
+    int resident_warps;   // warps resident per SM
 };
 
-// Warps per CTA (as many as shared memory holds), shared memory, and the
-// grid (one wave of resident CTAs by default; max_ctas overrides it) for
-// one kernel variant; sets the shared-memory attribute once per device.
+// Warps per CTA (as many as shared memory holds for `cps` CTAs per SM, at
+// most max_warps), shared memory, and the grid (one wave of resident CTAs
+// by default; max_ctas overrides it) for one kernel variant; sets the
+// shared-memory attribute once per device.
 template <int W, int MINLEN, typename Kernel>
 df11_status shape_launch(Kernel kernel, int v, const DecodeParams &prm, int dev, uint32_t max_ctas,
-                         LaunchShape &ls)
+                         int max_warps, int cps, LaunchShape &ls)
 {
-    int warps = kMaxWarpsPerCta;
-    while (warps > 1 && smem_bytes_for<W, MINLEN>(warps, prm.n_tables) > kSmemLimit)
+    DeviceProps d;
+    if (device_props(dev, d) != DF11_OK)
+        return DF11_ERR_CUDA;
+    const size_t limit = (size_t)min(d.smem_optin, d.smem_per_sm / cps - d.smem_reserved);
+    int warps = max_warps;
+    while (warps > 1 && smem_bytes_for<W, MINLEN>(warps, prm.n_tables) > limit)
         --warps;
     const size_t smem = smem_bytes_for<W, MINLEN>(warps, prm.n_tables);
-    if (smem > kSmemLimit)
+    if (smem > limit)
         return DF11_ERR_INVALID_ARGUMENT;
     if (!g_attr_done[dev][v].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return DF11_ERR_CUDA;
         g_attr_done[dev][v].store(1, std::memory_order_release);
-    }
-    int sms = g_sm_count[dev].load(std::memory_order_relaxed);
-    if (sms == 0) {
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return DF11_ERR_CUDA;
-        g_sm_count[dev].store(sms, std::memory_order_relaxed);
     }
     int occ = g_occupancy[dev][v][prm.n_tables].load(std::memory_order_relaxed);
     if (occ == 0) {
@@ -968,7 +1123,7 @@ df11_status shape_launch(Kernel kernel, int v, const DecodeParams &prm, int dev,
         g_occupancy[dev][v][prm.n_tables].store(occ, std::memory_order_relaxed);
     }
     const uint64_t ctas_needed = (prm.n_chunks + warps - 1) / warps;
-    const uint64_t resident = (uint64_t)occ * (uint64_t)sms;
+    const uint64_t resident = (uint64_t)occ * (uint64_t)d.sms;
     // default: one wave of resident CTAs, each looping over chunks; a given
     // count may be smaller (SMs left to other streams) or larger (waves of
     // short-lived CTAs that free their SM as each one finishes)
@@ -976,24 +1131,34 @@ df11_status shape_launch(Kernel kernel, int v, const DecodeParams &prm, int dev,
     ls.warps = warps;
     ls.smem = smem;
     ls.grid = (unsigned)(ctas_needed < want ? ctas_needed : want);
+    ls.resident_warps = occ * warps;
     return DF11_OK;
 }
 
 template <int W, int MINLEN>
 constexpr int variant_base()
 {
-    return ((W == 8 ? 0 : 2) + (MINLEN == 1 ? 0 : 1)) * 5;
+    return ((W == 8 ? 0 : 2) + (MINLEN == 1 ? 0 : 1)) * kVariantsPerLayout;
 }
 
+// Launches the store kernel shaped for one or two CTAs per SM, whichever
+// keeps more warps resident (one on a tie: fewer table copies to build).
 template <int W, int MINLEN>
 df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32_t max_ctas)
 {
-    auto kernel = df11_decode_kernel<W, MINLEN>;
-    LaunchShape ls;
-    const df11_status st = shape_launch<W, MINLEN>(kernel, variant_base<W, MINLEN>(), prm, dev, max_ctas, ls);
-    if (st != DF11_OK)
-        return st;
-    kernel<<<ls.grid, ls.warps * 32, ls.smem, stream>>>(prm);
+    auto k1 = df11_decode_kernel<W, MINLEN, 1>;
+    auto k2 = df11_decode_kernel<W, MINLEN, 2>;
+    LaunchShape s1, s2;
+    const df11_status st1 =
+        shape_launch<W, MINLEN>(k1, variant_base<W, MINLEN>(), prm, dev, max_ctas, kCtaWarps<1>, 1, s1);
+    const df11_status st2 =
+        shape_launch<W, MINLEN>(k2, variant_base<W, MINLEN>() + 5, prm, dev, max_ctas, kCtaWarps<2>, 2, s2);
+    if (st1 != DF11_OK && st2 != DF11_OK)
+        return st1;
+    if (st2 == DF11_OK && (st1 != DF11_OK || s2.resident_warps > s1.resident_warps))
+        k2<<<s2.grid, s2.warps * 32, s2.smem, stream>>>(prm);
+    else
+        k1<<<s1.grid, s1.warps * 32, s1.smem, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
@@ -1003,7 +1168,7 @@ df11_status launch_gemv(const DecodeParams &prm, const GemvParams &gp, int dev, 
     auto kernel = df11_gemv_kernel<W, MINLEN, TT>;
     constexpr int v = variant_base<W, MINLEN>() + (TT == 1 ? 1 : TT == 2 ? 2 : TT == 4 ? 3 : 4);
     LaunchShape ls;
-    const df11_status st = shape_launch<W, MINLEN>(kernel, v, prm, dev, 0, ls);
+    const df11_status st = shape_launch<W, MINLEN>(kernel, v, prm, dev, 0, kMaxWarpsPerCta, 1, ls);
     if (st != DF11_OK)
         return st;
     kernel<<<ls.grid, ls.warps * 32, ls.smem, stream>>>(prm, gp);
@@ -1053,21 +1218,25 @@ df11_status block_params(const df11_device_block *blk, uint16_t *out_bf16, uint6
     if (h.n_chunks != (h.total_bits + chunk_bits - 1) / chunk_bits)
         return DF11_ERR_INVALID_ARGUMENT;
     const uint64_t n_threads = h.n_chunks * DF11_THREADS_PER_CHUNK;
-    if (!blk->exp_stream || !blk->gaps || !blk->chunk_pos || !blk->signmant || !blk->lut)
+    if (!blk->exp_stream || !blk->gaps || !blk->counts || !blk->chunk_pos || !blk->signmant || !blk->lut)
         return DF11_ERR_INVALID_ARGUMENT;
     if (blk->exp_stream_bytes < n_threads * W + DF11_STREAM_PAD || blk->gaps_bytes < n_threads / 2 ||
+        blk->counts_bytes < n_threads ||
         blk->chunk_pos_count < h.n_chunks + 1 ||
         blk->signmant_bytes < (h.n_elements + 15) / 16 * 16 ||
         blk->lut_entries < (uint64_t)h.n_tables * 256)
         return DF11_ERR_INVALID_ARGUMENT;
     if (!aligned(blk->exp_stream, 16) || !aligned(blk->chunk_pos, 16) || !aligned(blk->lut, 16) ||
-        !aligned(blk->signmant, 16) || !aligned(blk->gaps, 16) || !aligned(out_bf16, 16) ||
-        !aligned(d_error, 4))
+        !aligned(blk->signmant, 16) || !aligned(blk->gaps, 16) || !aligned(blk->counts, 16) ||
+        !aligned(out_bf16, 16) ||
+        !aligned(d_error, 4) || !aligned(blk->decode_table, 16))
         return DF11_ERR_INVALID_ARGUMENT;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return DF11_ERR_CUDA;
     prm.stream = blk->exp_stream;
     prm.gaps = blk->gaps;
+    prm.counts = blk->counts;
+    prm.gaps_limit = n_threads / 2;
     prm.chunk_pos = blk->chunk_pos;
     prm.signmant = blk->signmant;
     prm.lut = blk->lut;
@@ -1080,6 +1249,7 @@ df11_status block_params(const df11_device_block *blk, uint16_t *out_bf16, uint6
     prm.min_len = h.min_code_len;
     prm.full_chunks = (uint32_t)(h.total_bits / chunk_bits);
     prm.sched = nullptr;
+    prm.multi_src = reinterpret_cast<const uint2 *>(blk->decode_table);
     return DF11_OK;
 }
 
@@ -1137,6 +1307,8 @@ extern "C" df11_status df11_decompress_range_async(const df11_device_block *blk,
     const uint64_t chunk_bits = (uint64_t)DF11_THREADS_PER_CHUNK * 8 * W;
     prm.stream += chunk_begin * DF11_THREADS_PER_CHUNK * W;
     prm.gaps += chunk_begin * (DF11_THREADS_PER_CHUNK / 2);
+    prm.gaps_limit -= chunk_begin * (DF11_THREADS_PER_CHUNK / 2);   // the thread after the range included
+    prm.counts += chunk_begin * DF11_THREADS_PER_CHUNK;
     prm.chunk_pos += chunk_begin;
     prm.total_bits -= chunk_begin * chunk_bits;
     prm.n_chunks = chunk_end - chunk_begin;

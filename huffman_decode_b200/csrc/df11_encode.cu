@@ -14,10 +14,12 @@
 //      codes MSB-first into the segment's stream words staged in shared
 //      memory (words shared with a neighbouring thread are ORed), records
 //      the gap of every slice whose first code it owns (staged too) and the
-//      output position of every chunk that starts in such a slice, and
-//      writes its sign|mantissa bytes; the staged words then go to global
-//      memory with plain stores, ORing only the two words a segment may
-//      share with its neighbours.
+//      output position of every chunk that starts in such a slice, adds the
+//      number of its codes that start in each slice to a staged per-slice
+//      count, and writes its sign|mantissa bytes; the staged words then go
+//      to global memory with plain stores, ORing only the two words a
+//      segment may share with its neighbours, and the staged counts are
+//      added into the (zeroed) counts array, four per word.
 // The result is byte-identical to df11_compress (host) for the same
 // codebook and layout ("How it works": canonical codes, MSB-first encode;
 // "Architecture": Gaps and per-chunk output positions).
@@ -48,6 +50,7 @@ struct EncodeParams {
     const uint16_t *in;
     uint8_t *stream;
     uint8_t *gaps;
+    uint8_t *counts;
     uint32_t *chunk_pos;
     uint8_t *signmant;
     uint32_t *seg_bits;     // scratch: bits per segment
@@ -273,7 +276,8 @@ __global__ void __launch_bounds__(kScanThreads) segment_scan_kernel(EncodeParams
         atomicOr(p.err, DF11_DEVERR_MISMATCH);
 }
 
-// Zeroes the stream, gaps and sign|mantissa tail; fills chunk positions with n.
+// Zeroes the stream, gaps, counts and sign|mantissa tail; fills chunk
+// positions with n.
 __global__ void prepare_kernel(EncodeParams p, uint64_t stream_words, uint64_t gap_words,
                                uint64_t n_chunks, uint64_t sm_bytes)
 {
@@ -285,6 +289,9 @@ __global__ void prepare_kernel(EncodeParams p, uint64_t stream_words, uint64_t g
     uint32_t *g32 = reinterpret_cast<uint32_t *>(p.gaps);
     for (uint64_t i = tid; i < gap_words; i += stride)
         g32[i] = 0;
+    uint32_t *c32 = reinterpret_cast<uint32_t *>(p.counts);
+    for (uint64_t i = tid; i < p.n_threads / 4; i += stride)
+        c32[i] = 0;
     for (uint64_t i = tid; i <= n_chunks; i += stride)
         p.chunk_pos[i] = (uint32_t)p.n;
     for (uint64_t i = p.n + tid; i < sm_bytes; i += stride)
@@ -310,12 +317,15 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
     __shared__ uint32_t warp_tot[kEncThreads / 32 + 1];
     __shared__ uint32_t sw[kStageWords];
     __shared__ uint32_t sg[kGapStageWords * 2];   // one byte per slice's gap (plain byte stores)
+    __shared__ uint32_t sc[kGapStageWords * 8];   // one count per slice (shared atomic adds)
     code_tab[threadIdx.x] = ct.e[threadIdx.x];
     len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
     for (int i = threadIdx.x; i < kStageWords; i += kEncThreads)
         sw[i] = 0;
     for (int i = threadIdx.x; i < kGapStageWords * 2; i += kEncThreads)
         sg[i] = 0;
+    for (int i = threadIdx.x; i < kGapStageWords * 8; i += kEncThreads)
+        sc[i] = 0;
     uint8_t *const sgb = reinterpret_cast<uint8_t *>(sg);
     __syncthreads();
 
@@ -353,6 +363,10 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
         uint32_t cur = 0;
         const uint32_t cnt = (uint32_t)min((uint64_t)kElemsPerThread, p.n - e0);
         const uint32_t sw_a = (uint32_t)__cvta_generic_to_shared(sw);
+        // this thread's codes from element run_k on start in staged slice
+        // cur_gi (its first code's slice to begin with)
+        uint32_t cur_gi = (lb >> sh) + goff;
+        uint32_t run_k = 0;
         // Two elements k, k + 1 (the second may be absent past the end):
         // their codes joined into one of at most 32 bits, appended MSB-first
         // at bit `fill` of staged word j (a full word is ORed into the
@@ -374,8 +388,13 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
                 const uint32_t gl = ob >> sh;
                 const uint32_t gi = gl + goff;             // slice index relative to gbase * 8
                 sgb[gi] = (uint8_t)(ob & slice_mask & 0xFu);
+                const uint32_t k_open = k + (by_first ? 0u : 1u);
                 if (((gS + gl) & (DF11_THREADS_PER_CHUNK - 1)) == 0)
-                    p.chunk_pos[(gS + gl) / DF11_THREADS_PER_CHUNK] = (uint32_t)(e0 + k + (by_first ? 0u : 1u));
+                    p.chunk_pos[(gS + gl) / DF11_THREADS_PER_CHUNK] = (uint32_t)(e0 + k_open);
+                if (k_open > run_k)
+                    atomicAdd(&sc[cur_gi], k_open - run_k);
+                cur_gi = gi;
+                run_k = k_open;
                 next_open = (gl + 1) << sh;
             }
             const uint32_t l = l1 + l2;
@@ -404,6 +423,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
         }
         if (fill)
             atomicOr(&sw[j], cur);                                // shared with the next thread
+        atomicAdd(&sc[cur_gi], cnt - run_k);
         // the end of the stream counts as a code start for the gap of its slice
         if (e0 + cnt == p.n) {
             const uint32_t gl = lb >> sh;
@@ -472,6 +492,16 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
                 atomicOr(gg + i, v);
             else
                 gg[i] = v;
+        }
+        // counts: staged slice 4i + k at byte k of word i; slices this
+        // segment shares with its neighbours get all their contributions
+        // added (a count is at most 128, so bytes never carry)
+        uint32_t *cc = reinterpret_cast<uint32_t *>(p.counts) + 2 * gbase;
+        const uint64_t cwords = p.n_threads / 4;
+        for (uint32_t i = threadIdx.x; i < 2 * ng && 2 * gbase + i < cwords; i += kEncThreads) {
+            const uint32_t v = sc[4 * i] | (sc[4 * i + 1] << 8) | (sc[4 * i + 2] << 16) | (sc[4 * i + 3] << 24);
+            if (v)
+                atomicAdd(cc + i, v);
         }
     }
 }
@@ -545,12 +575,14 @@ df11_status compress_device_impl(const df11_codebook *cb, const df11_layout *lay
         return st;
     if (scratch_bytes < (group_bits ? df11_compress_device_scratch_bytes(n) : segment_scratch_bytes(n)))
         return DF11_ERR_BUFFER_TOO_SMALL;
-    if (!out->exp_stream || !out->gaps || !out->chunk_pos || !out->signmant)
+    if (!out->exp_stream || !out->gaps || !out->counts || !out->chunk_pos || !out->signmant)
         return DF11_ERR_INVALID_ARGUMENT;
     if (out->exp_stream_bytes < z.exp_stream_bytes || out->gaps_bytes < z.gaps_bytes ||
-        out->chunk_pos_count < z.chunk_pos_count || out->signmant_bytes < z.signmant_bytes)
+        out->counts_bytes < z.counts_bytes || out->chunk_pos_count < z.chunk_pos_count ||
+        out->signmant_bytes < z.signmant_bytes)
         return DF11_ERR_BUFFER_TOO_SMALL;
     if (!aligned(d_in, 16) || !aligned(out->exp_stream, 16) || !aligned(out->gaps, 16) ||
+        !aligned(out->counts, 16) ||
         !aligned(out->chunk_pos, 16) || !aligned(out->signmant, 16) || !aligned(d_scratch, 16) ||
         !aligned(d_error, 4))
         return DF11_ERR_INVALID_ARGUMENT;
@@ -560,6 +592,7 @@ df11_status compress_device_impl(const df11_codebook *cb, const df11_layout *lay
     // the arrays are written through the const-qualified device view
     p.stream = const_cast<uint8_t *>(out->exp_stream);
     p.gaps = const_cast<uint8_t *>(out->gaps);
+    p.counts = const_cast<uint8_t *>(out->counts);
     p.chunk_pos = const_cast<uint32_t *>(out->chunk_pos);
     p.signmant = const_cast<uint8_t *>(out->signmant);
     p.n_seg = n_segments(n);

@@ -275,6 +275,7 @@ df11_sizes sizes_for(uint64_t total_bits, uint64_t n_elements, uint32_t n_tables
     z.n_threads = z.n_chunks * ly->threads_per_chunk;
     z.exp_stream_bytes = z.n_threads * ly->bytes_per_thread + DF11_STREAM_PAD;
     z.gaps_bytes = z.n_threads / 2;
+    z.counts_bytes = z.n_threads;
     z.chunk_pos_count = z.n_chunks + 1;
     z.signmant_bytes = (n_elements + 15) / 16 * 16;
     z.lut_entries = (uint64_t)n_tables * 256;
@@ -366,7 +367,7 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
 {
     if (!cb || !out || !layout_ok(layout) || !check_mats(mats, numel, n_mats))
         return DF11_ERR_INVALID_ARGUMENT;
-    if (!out->exp_stream || !out->gaps || !out->chunk_pos || !out->signmant || !out->lut)
+    if (!out->exp_stream || !out->gaps || !out->counts || !out->chunk_pos || !out->signmant || !out->lut)
         return DF11_ERR_INVALID_ARGUMENT;
     ElementView v(mats, numel, n_mats);
     if (v.total == 0 || v.total != cb->n_elements)
@@ -378,8 +379,8 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
     if (st != DF11_OK)
         return st;
     if (out->exp_stream_bytes < z.exp_stream_bytes || out->gaps_bytes < z.gaps_bytes ||
-        out->chunk_pos_count < z.chunk_pos_count || out->signmant_bytes < z.signmant_bytes ||
-        out->lut_entries < z.lut_entries)
+        out->counts_bytes < z.counts_bytes || out->chunk_pos_count < z.chunk_pos_count ||
+        out->signmant_bytes < z.signmant_bytes || out->lut_entries < z.lut_entries)
         return DF11_ERR_BUFFER_TOO_SMALL;
 
     uint64_t h[256];
@@ -415,6 +416,9 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
     const uint64_t used_bytes = (total_bits + 7) / 8;
     std::memset(stream + used_bytes, 0, z.exp_stream_bytes - used_bytes);
     std::vector<uint8_t> gap_tmp(z.n_threads, 0);
+    // element index of the first code starting in each slice (N for slices
+    // no code starts in); a slice's count is the difference to the next one
+    std::vector<uint32_t> first_elem(z.n_threads + 1, (uint32_t)N);
     std::vector<uint8_t> first_byte(nseg, 0);
     uint32_t *pos = out->chunk_pos;
     std::memset(pos, 0, sizeof(uint32_t) * z.chunk_pos_count);
@@ -448,6 +452,7 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
             uint64_t g = bit / kSliceBits;
             if (g != prev_slice) {
                 gap_tmp[g] = (uint8_t)(bit - g * kSliceBits);
+                first_elem[g] = (uint32_t)k;
                 if (g % T == 0)
                     pos[g / T] = (uint32_t)k;
                 prev_slice = g;
@@ -485,6 +490,8 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
     }
     for (uint64_t j = 0; j < z.gaps_bytes; ++j)
         out->gaps[j] = (uint8_t)((gap_tmp[2 * j] & 0xF) | ((gap_tmp[2 * j + 1] & 0xF) << 4));
+    for (uint64_t g = 0; g < z.n_threads; ++g)
+        out->counts[g] = (uint8_t)(first_elem[g + 1] - first_elem[g]);
 
     parallel_for(nw, [&](unsigned w) {
         uint64_t lo = N * w / nw, hi = N * (w + 1) / nw;
@@ -513,7 +520,7 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
 
 df11_status df11_validate(const df11_host_block *b)
 {
-    if (!b || !b->exp_stream || !b->gaps || !b->chunk_pos || !b->signmant || !b->lut)
+    if (!b || !b->exp_stream || !b->gaps || !b->counts || !b->chunk_pos || !b->signmant || !b->lut)
         return DF11_ERR_INVALID_ARGUMENT;
     const df11_header &h = b->hdr;
     df11_layout ly{h.threads_per_chunk, h.bytes_per_thread};
@@ -525,7 +532,8 @@ df11_status df11_validate(const df11_host_block *b)
         return DF11_ERR_CORRUPT;
     df11_sizes z = sizes_for(h.total_bits, h.n_elements, h.n_tables, &ly);
     if (h.n_chunks != z.n_chunks || b->exp_stream_bytes < z.exp_stream_bytes ||
-        b->gaps_bytes < z.gaps_bytes || b->chunk_pos_count < z.chunk_pos_count ||
+        b->gaps_bytes < z.gaps_bytes || b->counts_bytes < z.counts_bytes ||
+        b->chunk_pos_count < z.chunk_pos_count ||
         b->signmant_bytes < h.n_elements || b->lut_entries < z.lut_entries)
         return DF11_ERR_CORRUPT;
     // output positions: 0 .. n_elements, monotone, at most one code per bit
@@ -547,6 +555,21 @@ df11_status df11_validate(const df11_host_block *b)
     }
     if ((b->gaps[0] & 0xF) != 0)
         return DF11_ERR_CORRUPT;
+    // counts: a chunk's add up to its output range; none above what the
+    // shortest code allows in a slice, none past the end of the stream
+    for (uint64_t c = 0; c < h.n_chunks; ++c) {
+        uint64_t sum = 0;
+        for (uint64_t t = 0; t < h.threads_per_chunk; ++t) {
+            const uint64_t g = c * h.threads_per_chunk + t;
+            const uint32_t n = b->counts[g];
+            if (n > (kSliceBits + h.min_code_len - 1) / h.min_code_len ||
+                (g * kSliceBits >= h.total_bits && n != 0))
+                return DF11_ERR_CORRUPT;
+            sum += n;
+        }
+        if (sum != (uint64_t)b->chunk_pos[c + 1] - b->chunk_pos[c])
+            return DF11_ERR_CORRUPT;
+    }
     // tables: root leaves <= 8 bits, pointers to existing sub-tables, each
     // sub-table entry a leaf of 9..cap bits
     for (uint32_t t = 0; t < h.n_tables; ++t) {
@@ -566,6 +589,60 @@ df11_status df11_validate(const df11_host_block *b)
                 return DF11_ERR_CORRUPT;
             }
         }
+    }
+    return DF11_OK;
+}
+
+df11_status df11_build_decode_table(const uint16_t *lut, uint32_t n_tables, uint32_t min_code_len,
+                                    uint64_t *table)
+{
+    if (!lut || !table || n_tables < 1 || n_tables > 256 || min_code_len < 1 ||
+        min_code_len > DF11_MAX_CODE_LEN)
+        return DF11_ERR_INVALID_ARGUMENT;
+    // the tables as the decoder sanitises them: a malformed entry, or one
+    // shorter than the shortest code, reads as "no code"
+    const uint16_t no_code = (uint16_t)(0x4000u | (min_code_len << 8));
+    std::vector<uint16_t> t((size_t)n_tables * 256);
+    for (uint32_t i = 0; i < n_tables * 256u; ++i) {
+        uint32_t e = lut[i];
+        if (e & kLutPointer) {
+            const uint32_t to = e & 0xFFu;
+            if (i >= 256u || to == 0 || to >= n_tables || (e & 0x7F00u))
+                e = no_code;
+        } else {
+            const uint32_t l = (e >> 8) & 0x1Fu;
+            if ((e & 0x4000u) || l < min_code_len || l > DF11_MAX_CODE_LEN)
+                e = no_code;
+        }
+        t[i] = (uint16_t)e;
+    }
+    // entry k serves the window whose first stream bit is bit 0 of k:
+    // the whole codes the window starts with, at most four, as rotated
+    // exponents (bit 0 moved to bit 7) in bytes 0..3, and their total
+    // length | 8 x count << 16; a first code longer than the window (or
+    // none) gives the marker 0x80000000 << 32
+    for (uint32_t k = 0; k < DF11_DECODE_TABLE_ENTRIES; ++k) {
+        uint32_t win = 0;   // MSB-first: first stream bit at bit 31
+        for (uint32_t b = 0; b < DF11_DECODE_TABLE_WINDOW_BITS; ++b)
+            win |= ((k >> b) & 1u) << (31 - b);
+        uint32_t used = 0, n = 0, syms = 0;
+        while (n < 4) {
+            const uint32_t v = win << used;
+            uint32_t e = t[v >> 24];
+            if (e & kLutPointer)
+                e = t[((e & 0xFFu) << 8) | ((v >> 16) & 0xFFu)];
+            if (e & 0x4000u)
+                break;
+            const uint32_t l = (e >> 8) & 0x1Fu;
+            if (used + l > DF11_DECODE_TABLE_WINDOW_BITS)
+                break;
+            const uint32_t x = e & 0xFFu;
+            syms |= (((x >> 1) | ((x & 1u) << 7)) & 0xFFu) << (8 * n);
+            ++n;
+            used += l;
+        }
+        const uint32_t y = n ? used | (8u * n << 16) : 0x80000000u;
+        table[k] = (uint64_t)syms | ((uint64_t)y << 32);
     }
     return DF11_OK;
 }

@@ -127,14 +127,15 @@ extern "C" df11_status df11_pipeline_upload(df11_pipeline *p, uint32_t slot, con
 {
     if (!p || !src || !dst || slot >= p->n_slots)
         return DF11_ERR_INVALID_ARGUMENT;
-    if (!src->exp_stream || !src->gaps || !src->chunk_pos || !src->signmant || !src->lut ||
-        !dst->exp_stream || !dst->gaps || !dst->chunk_pos || !dst->signmant || !dst->lut)
+    if (!src->exp_stream || !src->gaps || !src->counts || !src->chunk_pos || !src->signmant || !src->lut ||
+        !dst->exp_stream || !dst->gaps || !dst->counts || !dst->chunk_pos || !dst->signmant || !dst->lut)
         return DF11_ERR_INVALID_ARGUMENT;
     if (!on_device(p))
         return DF11_ERR_INVALID_ARGUMENT;
     // every staging array must hold its source before anything is enqueued
     if (src->exp_stream_bytes > dst->exp_stream_bytes || src->gaps_bytes > dst->gaps_bytes ||
-        src->chunk_pos_count > dst->chunk_pos_count || src->signmant_bytes > dst->signmant_bytes ||
+        src->counts_bytes > dst->counts_bytes || src->chunk_pos_count > dst->chunk_pos_count ||
+        src->signmant_bytes > dst->signmant_bytes ||
         src->lut_entries > dst->lut_entries)
         return DF11_ERR_BUFFER_TOO_SMALL;
     const cudaStream_t s = as_stream(copy_stream);
@@ -144,6 +145,7 @@ extern "C" df11_status df11_pipeline_upload(df11_pipeline *p, uint32_t slot, con
     df11_status st;
     if ((st = copy_array(dst->exp_stream, src->exp_stream, src->exp_stream_bytes, s)) != DF11_OK ||
         (st = copy_array(dst->gaps, src->gaps, src->gaps_bytes, s)) != DF11_OK ||
+        (st = copy_array(dst->counts, src->counts, src->counts_bytes, s)) != DF11_OK ||
         (st = copy_array(dst->chunk_pos, src->chunk_pos, src->chunk_pos_count * 4, s)) != DF11_OK ||
         (st = copy_array(dst->signmant, src->signmant, src->signmant_bytes, s)) != DF11_OK ||
         (st = copy_array(dst->lut, src->lut, src->lut_entries * 2, s)) != DF11_OK)

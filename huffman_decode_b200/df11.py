@@ -42,6 +42,7 @@ STREAM_PAD = 16
 THREADS_PER_CHUNK = 32
 BYTES_PER_THREAD = 16           # 128-bit slices: fastest layout on B200
 LAYOUTS = ((32, 8), (32, 16))   # (threads_per_chunk, bytes_per_thread) the library decodes
+ARRAYS = ("exp_stream", "gaps", "counts", "chunk_pos", "signmant", "lut")   # artifact order
 
 EXPORTED_SYMBOLS = (
     "df11_build_codebook", "df11_build_codebook_from_histogram", "df11_compress_sizes",
@@ -53,11 +54,14 @@ EXPORTED_SYMBOLS = (
     "df11_checksum_device_async", "df11_verify_device_async", "df11_pipeline_verify",
     "df11_decode_gemv_async", "df11_decompress_async_ws", "df11_decompress_range_async",
     "df11_selftest_bounded_wait", "df11_serialized_bytes", "df11_serialize", "df11_deserialize",
+    "df11_build_decode_table",
 )
 SCHED_WORKSPACE_BYTES = 2048
 CRC_SEGMENT_BYTES = 4096
 NOALLOC_SCRATCH_BYTES = 1 << 20
 NOALLOC_MAX_ELEMENTS = 715816960
+DECODE_TABLE_ENTRIES = 2048
+DECODE_TABLE_WINDOW_BITS = 11
 
 
 class DF11Error(RuntimeError):
@@ -103,6 +107,7 @@ class Sizes(ctypes.Structure):
     _fields_ = [
         ("n_chunks", ctypes.c_uint64), ("n_threads", ctypes.c_uint64),
         ("exp_stream_bytes", ctypes.c_uint64), ("gaps_bytes", ctypes.c_uint64),
+        ("counts_bytes", ctypes.c_uint64),
         ("chunk_pos_count", ctypes.c_uint64), ("signmant_bytes", ctypes.c_uint64),
         ("lut_entries", ctypes.c_uint64),
     ]
@@ -123,9 +128,11 @@ class _Block(ctypes.Structure):
         ("hdr", Header),
         ("exp_stream", ctypes.c_void_p), ("exp_stream_bytes", ctypes.c_uint64),
         ("gaps", ctypes.c_void_p), ("gaps_bytes", ctypes.c_uint64),
+        ("counts", ctypes.c_void_p), ("counts_bytes", ctypes.c_uint64),
         ("chunk_pos", ctypes.c_void_p), ("chunk_pos_count", ctypes.c_uint64),
         ("signmant", ctypes.c_void_p), ("signmant_bytes", ctypes.c_uint64),
         ("lut", ctypes.c_void_p), ("lut_entries", ctypes.c_uint64),
+        ("decode_table", ctypes.c_void_p),   # df11_device_block only (host calls ignore it)
     ]
 
 
@@ -181,6 +188,7 @@ def load_library(path: str | None = None):
         ("df11_serialized_bytes", U64, [P]),
         ("df11_serialize", S, [P, P, U64]),
         ("df11_deserialize", S, [P, U64, P, P]),
+        ("df11_build_decode_table", S, [P, U32, U32, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -234,6 +242,7 @@ class HostBlock:
     header: Header
     exp_stream: np.ndarray
     gaps: np.ndarray
+    counts: np.ndarray
     chunk_pos: np.ndarray
     signmant: np.ndarray
     lut: np.ndarray
@@ -242,11 +251,12 @@ class HostBlock:
     def c_struct(self) -> _Block:
         b = _Block()
         b.hdr = self.header
-        for name in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut"):
+        for name in ARRAYS:
             a = getattr(self, name)
             setattr(b, name, a.ctypes.data)
         b.exp_stream_bytes = self.exp_stream.nbytes
         b.gaps_bytes = self.gaps.nbytes
+        b.counts_bytes = self.counts.nbytes
         b.chunk_pos_count = self.chunk_pos.size
         b.signmant_bytes = self.signmant.nbytes
         b.lut_entries = self.lut.size
@@ -257,15 +267,15 @@ class HostBlock:
         return int(self.header.n_elements)
 
     def compressed_bytes(self) -> int:
-        """Bytes a decode reads: stream, gaps, positions, sign|mantissa, tables."""
-        return int(self.exp_stream.nbytes + self.gaps.nbytes + self.chunk_pos.nbytes
-                   + self.signmant.nbytes + self.lut.nbytes)
+        """Bytes a decode reads: stream, gaps, counts, positions,
+        sign|mantissa, tables."""
+        return int(sum(getattr(self, n).nbytes for n in ARRAYS))
 
     def arrays(self):
-        return {n: getattr(self, n) for n in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")}
+        return {n: getattr(self, n) for n in ARRAYS}
 
     def to_bytes(self) -> bytes:
-        """df11_serialize: the block as one flat buffer (header, the five
+        """df11_serialize: the block as one flat buffer (header, the six
         arrays, the CRC-32C checksum list).  matrix_numel is not stored."""
         lib = load_library()
         b = self.c_struct()
@@ -302,6 +312,7 @@ class HostBlock:
         return HostBlock(header=Header.from_buffer_copy(blk.hdr),
                          exp_stream=take(blk.exp_stream, blk.exp_stream_bytes, np.uint8),
                          gaps=take(blk.gaps, blk.gaps_bytes, np.uint8),
+                         counts=take(blk.counts, blk.counts_bytes, np.uint8),
                          chunk_pos=take(blk.chunk_pos, 4 * blk.chunk_pos_count, np.uint32),
                          signmant=take(blk.signmant, blk.signmant_bytes, np.uint8),
                          lut=take(blk.lut, 2 * blk.lut_entries, np.uint16))
@@ -325,7 +336,11 @@ class HostBlock:
                                sizes={n: a.nbytes for n, a in self.arrays().items()},
                                matrix_numel=list(self.matrix_numel))
 
-    def to_device(self, device="cuda", pin: bool = False) -> "DeviceBlock":
+    def to_device(self, device="cuda", pin: bool = False, decode_table: bool = True) -> "DeviceBlock":
+        """The block's arrays copied to the GPU, plus (decode_table=True) the
+        decoder's multi-code table built from its lookup tables
+        (df11_build_decode_table), so decode launches copy it instead of
+        building it in every CTA."""
         import torch
         t = {}
         for name, a in self.arrays().items():
@@ -333,18 +348,35 @@ class HostBlock:
             if pin:
                 src = src.pin_memory()
             t[name] = src.to(device, non_blocking=pin)
-        return DeviceBlock(header=self.header, tensors=t,
-                           sizes={n: a.nbytes for n, a in self.arrays().items()},
-                           matrix_numel=list(self.matrix_numel))
+        db = DeviceBlock(header=self.header, tensors=t,
+                         sizes={n: a.nbytes for n, a in self.arrays().items()},
+                         matrix_numel=list(self.matrix_numel))
+        if decode_table:
+            db.attach_decode_table(self.lut)
+        return db
 
 
-def _struct_from_tensors(header, tensors, sizes) -> _Block:
+def build_decode_table(lut, n_tables: int, min_code_len: int) -> np.ndarray:
+    """df11_build_decode_table: the decoder's 2048-entry multi-code table
+    (uint64 entries) for a block's lookup tables."""
+    lut = np.ascontiguousarray(lut, dtype=np.uint16)
+    if lut.size < int(n_tables) * 256:
+        raise ValueError("lut holds fewer than n_tables * 256 entries")
+    out = np.empty(DECODE_TABLE_ENTRIES, np.uint64)
+    _check(load_library().df11_build_decode_table(lut.ctypes.data, int(n_tables), int(min_code_len),
+                                                  out.ctypes.data), "df11_build_decode_table")
+    return out
+
+
+def _struct_from_tensors(header, tensors, sizes, decode_table=None) -> _Block:
     b = _Block()
     b.hdr = header
+    b.decode_table = decode_table.data_ptr() if decode_table is not None else None
     for name, t in tensors.items():
         setattr(b, name, t.data_ptr())
     b.exp_stream_bytes = sizes["exp_stream"]
     b.gaps_bytes = sizes["gaps"]
+    b.counts_bytes = sizes["counts"]
     b.chunk_pos_count = sizes["chunk_pos"] // 4
     b.signmant_bytes = sizes["signmant"]
     b.lut_entries = sizes["lut"] // 2
@@ -379,6 +411,7 @@ def compress(cb: Codebook, mats, threads_per_chunk: int = THREADS_PER_CHUNK,
         header=Header(),
         exp_stream=np.empty(z.exp_stream_bytes, np.uint8),
         gaps=np.empty(z.gaps_bytes, np.uint8),
+        counts=np.empty(z.counts_bytes, np.uint8),
         chunk_pos=np.empty(z.chunk_pos_count, np.uint32),
         signmant=np.empty(z.signmant_bytes, np.uint8),
         lut=np.empty(z.lut_entries, np.uint16),
@@ -402,14 +435,25 @@ def validate(hb: HostBlock) -> int:
 
 @dataclass
 class DeviceBlock:
-    """The block's arrays as uint8 torch tensors on one GPU."""
+    """The block's arrays as uint8 torch tensors on one GPU, and optionally
+    the decoder's multi-code table (a uint8 tensor of 16 KB; not part of the
+    artifact, built from its tables)."""
     header: Header
     tensors: dict
     sizes: dict
     matrix_numel: list = field(default_factory=list)
+    decode_table: object = None
 
     def c_struct(self) -> _Block:
-        return _struct_from_tensors(self.header, self.tensors, self.sizes)
+        return _struct_from_tensors(self.header, self.tensors, self.sizes, self.decode_table)
+
+    def attach_decode_table(self, lut) -> None:
+        """Builds the multi-code table for this block's header and host
+        copy of its tables, and keeps it on the block's device."""
+        import torch
+        tab = build_decode_table(lut, self.header.n_tables, self.header.min_code_len)
+        dev = self.tensors["lut"].device
+        self.decode_table = torch.from_numpy(tab.view(np.uint8)).to(dev)
 
     @property
     def n_elements(self) -> int:
@@ -562,7 +606,7 @@ def compress_device(cb: Codebook, d_in, threads_per_chunk: int = THREADS_PER_CHU
         raise ValueError("d_in must be a contiguous CUDA tensor of 16-bit elements")
     dev = d_in.device
     z = compress_sizes(cb, threads_per_chunk, bytes_per_thread)
-    sizes = {"exp_stream": z.exp_stream_bytes, "gaps": z.gaps_bytes,
+    sizes = {"exp_stream": z.exp_stream_bytes, "gaps": z.gaps_bytes, "counts": z.counts_bytes,
              "chunk_pos": z.chunk_pos_count * 4, "signmant": z.signmant_bytes,
              "lut": z.lut_entries * 2}
     t = {name: torch.empty(nbytes, dtype=torch.uint8, device=dev) for name, nbytes in sizes.items()}
@@ -578,6 +622,7 @@ def compress_device(cb: Codebook, d_in, threads_per_chunk: int = THREADS_PER_CHU
         scratch.data_ptr(), scratch.numel(), error.data_ptr() if error is not None else None,
         _stream_handle(stream, dev)), "df11_compress_device")
     db.header = blk.hdr
+    db.attach_decode_table(cb.tables())
     return db
 
 
@@ -595,7 +640,7 @@ def compress_device_noalloc(cb: Codebook, d_in, threads_per_chunk: int = THREADS
         raise ValueError("d_in must be a contiguous CUDA tensor of 16-bit elements")
     dev = d_in.device
     z = compress_sizes(cb, threads_per_chunk, bytes_per_thread)
-    sizes = {"exp_stream": z.exp_stream_bytes, "gaps": z.gaps_bytes,
+    sizes = {"exp_stream": z.exp_stream_bytes, "gaps": z.gaps_bytes, "counts": z.counts_bytes,
              "chunk_pos": z.chunk_pos_count * 4, "signmant": z.signmant_bytes,
              "lut": z.lut_entries * 2}
     t = {name: torch.empty(nbytes, dtype=torch.uint8, device=dev) for name, nbytes in sizes.items()}
@@ -608,6 +653,7 @@ def compress_device_noalloc(cb: Codebook, d_in, threads_per_chunk: int = THREADS
         error.data_ptr() if error is not None else None, _stream_handle(stream, dev)),
         "df11_compress_device_noalloc")
     db.header = blk.hdr
+    db.attach_decode_table(cb.tables())
     return db
 
 

@@ -31,6 +31,15 @@
  *                  slice (the end of the stream counts as a start; slices at
  *                  or past the end hold 0).  Two per byte, thread 2j in the
  *                  low nibble of byte j.
+ *   counts         uint8 per thread: the number of codes that start in its
+ *                  slice (0 past the end of the stream; at most
+ *                  ceil(8 * bytes_per_thread / min_code_len), so at most 128).  The
+ *                  pages store no per-thread count: their decoder's first
+ *                  phase decodes every slice once only to count its codes.
+ *                  Stored, the counts give each thread its output offset
+ *                  from one warp prefix sum before it decodes, so the slice
+ *                  is decoded once, straight into place; they cost one byte
+ *                  per slice (about 1.5% of a compressed LLM block).
  *   chunk_pos      uint32[n_chunks+1]: chunk c (threads_per_chunk = 32
  *                  threads, one warp) writes elements [chunk_pos[c],
  *                  chunk_pos[c+1]); the last entry is n_elements.  (The pages
@@ -72,8 +81,12 @@ typedef enum {
 } df11_status;
 
 /* Bits the decoder ORs into the caller's device error word. */
-#define DF11_DEVERR_COUNT 0x1u    /* a chunk decoded a different number of codes
-                                     than chunk_pos says (corrupt stream/gaps) */
+#define DF11_DEVERR_COUNT 0x1u    /* a chunk's counts disagree with chunk_pos, a
+                                     count is impossible, or a thread's codes
+                                     do not end where the next thread's first
+                                     code starts (corrupt stream, gaps or
+                                     counts); a chunk whose counts disagree
+                                     with chunk_pos writes nothing */
 #define DF11_DEVERR_BAD_CODE 0x2u /* a window hit a "no code" or bad pointer
                                      entry (corrupt stream or table)           */
 #define DF11_DEVERR_BAD_POS 0x4u  /* chunk_pos not monotone or beyond
@@ -121,6 +134,7 @@ typedef struct {
     uint64_t n_threads;         /* n_chunks * threads_per_chunk                */
     uint64_t exp_stream_bytes;  /* n_threads * bytes_per_thread + STREAM_PAD   */
     uint64_t gaps_bytes;        /* n_threads / 2                               */
+    uint64_t counts_bytes;      /* n_threads                                   */
     uint64_t chunk_pos_count;   /* n_chunks + 1 (uint32 entries)               */
     uint64_t signmant_bytes;    /* n_elements rounded up to a multiple of 16   */
     uint64_t lut_entries;       /* n_tables * 256 (uint16 entries)             */
@@ -148,21 +162,26 @@ typedef struct {
     df11_header hdr;
     uint8_t *exp_stream;  uint64_t exp_stream_bytes;
     uint8_t *gaps;        uint64_t gaps_bytes;
+    uint8_t *counts;      uint64_t counts_bytes;
     uint32_t *chunk_pos;  uint64_t chunk_pos_count;
     uint8_t *signmant;    uint64_t signmant_bytes;
     uint16_t *lut;        uint64_t lut_entries;
 } df11_host_block;
 
 /* The same block after the caller copied each array to the GPU (device
- * pointers).  exp_stream, chunk_pos and lut must be 16-byte aligned, signmant
- * 8-byte aligned (any cudaMalloc / torch allocation is). */
+ * pointers).  Every array must be 16-byte aligned (any cudaMalloc / torch
+ * allocation is).  decode_table is optional: NULL, or the
+ * DF11_DECODE_TABLE_ENTRIES entries df11_build_decode_table made from this
+ * block's tables, copied to the GPU (see there). */
 typedef struct {
     df11_header hdr;
     const uint8_t *exp_stream;  uint64_t exp_stream_bytes;
     const uint8_t *gaps;        uint64_t gaps_bytes;
+    const uint8_t *counts;      uint64_t counts_bytes;
     const uint32_t *chunk_pos;  uint64_t chunk_pos_count;
     const uint8_t *signmant;    uint64_t signmant_bytes;
     const uint16_t *lut;        uint64_t lut_entries;
+    const uint64_t *decode_table;
 } df11_device_block;
 
 /* Host.  Histograms the exponents of n_mats BF16 matrices (bit patterns,
@@ -205,6 +224,32 @@ df11_status df11_compress(const df11_codebook *cb, const df11_layout *layout,
  * code-length cap, every table entry well formed.  Returns CORRUPT on the
  * first failure, INVALID_ARGUMENT for null pointers. */
 df11_status df11_validate(const df11_host_block *blk);
+
+/* Host.  The decoder's multi-code table for a block's lookup tables
+ * (lut: n_tables * 256 entries, as df11_compress writes them; min_code_len
+ * from the block header).  The decode kernel indexes it with the next
+ * DF11_DECODE_TABLE_WINDOW_BITS stream bits and takes up to four whole
+ * codes per lookup; it is a function of the tables alone, so it is built
+ * once per block (like the tables, at compress or load time) and kept on
+ * the GPU beside the block (df11_device_block.decode_table).  Without it,
+ * every decode CTA builds the same table in its prologue.  Entry k (a
+ * uint64) serves the window whose first stream bit is bit 0 of k: bits
+ * 0..31 hold the whole codes the window starts with (at most four), as
+ * exponents rotated right by one bit (bit 0 moved to bit 7), one per byte,
+ * unused bytes zero; bits 32..63 hold their total length | (8 x count) << 16,
+ * or 0x80000000 when the first code is longer than the window.  Entries are
+ * read as malformed tables are: the decoder treats bad entries of `lut`
+ * (and shorter than min_code_len) as "no code" before building.  A table
+ * that is not this block's gives wrong output, never an access out of
+ * bounds: the kernel replaces entries whose length and count are impossible
+ * by the long-code marker, and masks unused symbol bytes.
+ * ("Architecture", hierarchical lookup tables kept in SRAM.)
+ * Errors: INVALID_ARGUMENT for null pointers, n_tables outside 1..256 or
+ * min_code_len outside 1..16. */
+#define DF11_DECODE_TABLE_WINDOW_BITS 11u
+#define DF11_DECODE_TABLE_ENTRIES 2048u   /* 16 KB */
+df11_status df11_build_decode_table(const uint16_t *lut, uint32_t n_tables, uint32_t min_code_len,
+                                    uint64_t *table);
 
 /* GPU.  Enqueues ONE kernel launch on `stream` (a cudaStream_t; NULL = the
  * legacy default stream) that decodes every element of the block into
@@ -268,7 +313,10 @@ df11_status df11_decompress_async_ws(const df11_device_block *blk, uint16_t *out
  * only:
  *   - exp_stream bytes [32 W chunk_begin, 32 W chunk_end + DF11_STREAM_PAD)
  *     (W = bytes_per_thread);
- *   - gaps bytes [16 chunk_begin, 16 chunk_end);
+ *   - gaps bytes [16 chunk_begin, 16 chunk_end + 1) (the low nibble of the
+ *     last one, the gap of the thread after the range, when chunk_end <
+ *     n_chunks);
+ *   - counts bytes [32 chunk_begin, 32 chunk_end);
  *   - chunk_pos[chunk_begin .. chunk_end];
  *   - signmant bytes [p0 & ~15, (p1 + 15) & ~15), with p0 and p1 the
  *     positions of chunk_begin and chunk_end;
@@ -344,7 +392,7 @@ uint64_t df11_compress_device_scratch_bytes(uint64_t n_elements);
 
 /* GPU.  Encodes d_in[0 .. n) (device, the block's matrices concatenated,
  * 16-byte aligned) with the codebook cb (host) into the device arrays of
- * `out` (exp_stream, gaps, chunk_pos, signmant; sized by
+ * `out` (exp_stream, gaps, counts, chunk_pos, signmant; sized by
  * df11_compress_sizes, 16-byte aligned) and fills out->hdr.  out->lut is not
  * touched: the caller copies cb->lut (n_tables * 256 entries) into it.
  * d_scratch (device, 16-byte aligned, >= df11_compress_device_scratch_bytes)
@@ -395,8 +443,9 @@ df11_status df11_compress_device_noalloc(const df11_codebook *cb, const df11_lay
  * checksum of a block is a list of CRC-32C values (Castagnoli: reflected
  * polynomial 0x82F63B78, initial value and final XOR 0xFFFFFFFF; the
  * iSCSI / SSE4.2 CRC), one per DF11_CRC_SEGMENT_BYTES-byte segment of each
- * array, arrays in the order exp_stream, gaps, chunk_pos (little-endian
- * bytes), signmant, lut (little-endian bytes), each over the array sizes in
+ * array, arrays in the order exp_stream, gaps, counts, chunk_pos
+ * (little-endian bytes), signmant, lut (little-endian bytes), each over the
+ * array sizes in
  * the block struct; an array's last segment may be shorter.  Segments let
  * the GPU check run in parallel and point at the damaged region.  The
  * decoder itself flags desynchronised chunks (DF11_DEVERR_COUNT), but not a
@@ -467,7 +516,7 @@ df11_status df11_pipeline_create(uint32_t n_slots, df11_pipeline **out);
 df11_status df11_pipeline_destroy(df11_pipeline *p);
 
 /* Copy stage.  Enqueues on copy_stream the host -> device copies of src's
- * five arrays into dst's arrays (sizes from src; src should be pinned host
+ * six arrays into dst's arrays (sizes from src; src should be pinned host
  * memory for the copies to overlap with kernels).  dst->hdr is not written:
  * the caller decodes with src->hdr.  Errors: INVALID_ARGUMENT (null
  * pointers, slot out of range, wrong device), BUFFER_TOO_SMALL (a dst array
@@ -506,10 +555,11 @@ df11_status df11_pipeline_release(df11_pipeline *p, uint32_t slot, void *consume
  * artifacts on download and after every copy ("DFloat11: lossless BFloat16
  * compression", "How to run it in production", "Failure modes").  The
  * library's own container for one block: a 128-byte header (magic
- * "DF11BLK\0", version 1, the block header, the five array lengths, the
- * checksum count, the CRC-32C of those header bytes), the five arrays in
- * the order exp_stream, gaps, chunk_pos, signmant, lut, each at a 16-byte
- * aligned offset, then the checksum list of df11_checksum.  Little-endian.
+ * "DF11BLK\0", version 2, the block header, the six array lengths, the
+ * checksum count, the CRC-32C of those header bytes), the six arrays in
+ * the order exp_stream, gaps, counts, chunk_pos, signmant, lut, each at a
+ * 16-byte aligned offset, then the checksum list of df11_checksum.
+ * Little-endian.
  */
 
 /* Host.  Bytes df11_serialize writes for blk (0 for NULL or absurd sizes). */

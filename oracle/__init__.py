@@ -65,7 +65,7 @@ def _load():
         "orc_encode": (I, [P, U64, P, P, P, U64, P]),
         "orc_decode": (I, [P, U64, U64, U64, P, P, P]),
         "orc_first_code_table": (I, [P, P, P]),
-        "orc_metadata": (I, [P, U64, P, U32, U32, U64, P, P]),
+        "orc_metadata": (I, [P, U64, P, U32, U32, U64, P, P, P]),
         "orc_crc32c": (U32, [P, U64]),
         "orc_segment_crcs": (U64, [P, U64, U64, P]),
     }
@@ -203,17 +203,19 @@ def first_code_table(lengths: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 
 
 def metadata(exp: np.ndarray, lengths: np.ndarray, threads_per_chunk: int,
-             bytes_per_thread: int, n_chunks: int) -> tuple[np.ndarray, np.ndarray]:
-    """(per-thread gap, unpacked; per-chunk output positions incl. the end)."""
+             bytes_per_thread: int, n_chunks: int) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(per-thread gap, per-thread code count, both unpacked; per-chunk output
+    positions incl. the end)."""
     exp = _u8(exp).reshape(-1)
     gap = np.zeros(n_chunks * threads_per_chunk, np.uint8)
+    count = np.zeros(n_chunks * threads_per_chunk, np.uint8)
     pos = np.zeros(n_chunks + 1, np.uint32)
     rc = _load().orc_metadata(_ptr(exp) if exp.size else 0, exp.size, _ptr(_u8(lengths)),
                               threads_per_chunk, bytes_per_thread, n_chunks,
-                              _ptr(gap), _ptr(pos))
+                              _ptr(gap), _ptr(count), _ptr(pos))
     if rc != 0:
         raise ValueError("metadata failed")
-    return gap, pos
+    return gap, count, pos
 
 
 # ----------------------------------------------------- whole-block helpers
@@ -229,6 +231,7 @@ class OracleBlock:
     n_chunks: int
     stream: np.ndarray       # uint8, zero padded to n_chunks*T*W + pad bytes
     gap: np.ndarray          # uint8 per thread (unpacked)
+    thread_count: np.ndarray  # uint8 per thread: codes starting in its slice
     pos: np.ndarray          # uint32[n_chunks + 1]
     signmant: np.ndarray     # uint8[n_elements]
 
@@ -251,10 +254,10 @@ def compress_block(mats, cap: int = 16, threads_per_chunk: int = 32,
     stream_bytes = n_chunks * threads_per_chunk * bytes_per_thread + pad_bytes
     stream, tb2 = encode(e, lengths, codes, stream_bytes)
     assert tb2 == tb
-    gap, pos = metadata(e, lengths, threads_per_chunk, bytes_per_thread, n_chunks)
+    gap, thread_count, pos = metadata(e, lengths, threads_per_chunk, bytes_per_thread, n_chunks)
     return OracleBlock(lengths=lengths, codes=codes, counts=counts, total_bits=tb,
                        n_elements=w.size, n_chunks=n_chunks, stream=stream, gap=gap,
-                       pos=pos, signmant=s)
+                       thread_count=thread_count, pos=pos, signmant=s)
 
 
 def decode_block(stream: np.ndarray, n_elements: int, lengths: np.ndarray,
@@ -284,8 +287,8 @@ def segment_crcs(data, seg: int = CRC_SEGMENT) -> np.ndarray:
     return out[:k]
 
 
-def block_checksums(exp_stream, gaps, chunk_pos, signmant, lut, seg: int = CRC_SEGMENT) -> np.ndarray:
-    """The checksum list of a block: segment CRCs of its five arrays in the
-    order exp_stream, gaps, chunk_pos, signmant, lut (raw little-endian
-    bytes of each array as given)."""
-    return np.concatenate([segment_crcs(a, seg) for a in (exp_stream, gaps, chunk_pos, signmant, lut)])
+def block_checksums(exp_stream, gaps, counts, chunk_pos, signmant, lut, seg: int = CRC_SEGMENT) -> np.ndarray:
+    """The checksum list of a block: segment CRCs of its six arrays in the
+    order exp_stream, gaps, counts, chunk_pos, signmant, lut (raw
+    little-endian bytes of each array as given)."""
+    return np.concatenate([segment_crcs(a, seg) for a in (exp_stream, gaps, counts, chunk_pos, signmant, lut)])

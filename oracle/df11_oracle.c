@@ -420,7 +420,7 @@ int orc_first_code_table(const uint8_t len[256], int16_t *sym_out, uint8_t *len_
 
 int orc_metadata(const uint8_t *exp, uint64_t n, const uint8_t len[256],
                  uint32_t threads_per_chunk, uint32_t bytes_per_thread,
-                 uint64_t n_chunks, uint8_t *gap, uint32_t *pos)
+                 uint64_t n_chunks, uint8_t *gap, uint8_t *count, uint32_t *pos)
 {
     if (n >= ((uint64_t)1 << 32) || threads_per_chunk == 0 || bytes_per_thread == 0)
         return -1;
@@ -446,6 +446,18 @@ int orc_metadata(const uint8_t *exp, uint64_t n, const uint8_t len[256],
         if (d > 255)
             return -1;
         gap[g] = (uint8_t)d;
+    }
+
+    /* per-thread counts: every code start s_k < total lands in slice s_k / B */
+    for (uint64_t g = 0; g < n_threads; ++g)
+        count[g] = 0;
+    s = 0;
+    for (k = 0; k < n; ++k) {
+        uint64_t g = s / slice_bits;
+        if (g >= n_threads || count[g] == 255)
+            return -1;
+        count[g] += 1;
+        s += len[exp[k]];
     }
 
     /* chunk output positions */

@@ -97,11 +97,15 @@ int orc_first_code_table(const uint8_t len[256], int16_t *sym_out, uint8_t *len_
  * s_k = sum_{j<k} len(exp_j); s_n = total_bits is counted as a start so a
  * slice whose codes all began earlier still points at the end.
  *   gap[g]   = min{ s_k >= B*g } - B*g for slices with B*g < total_bits, else 0
+ *   count[g] = #{ k < n : B*g <= s_k < B*(g+1) }   (codes starting in slice g)
  *   pos[c]   = #{ k < n : s_k < c*T*B },  c = 0..n_chunks  (B = 8*bytes_per_thread)
- * gap is unpacked (one byte per thread, n_threads = n_chunks*T entries). */
+ * gap and count are unpacked (one byte per thread, n_threads = n_chunks*T
+ * entries).  count is what the page's first decode phase computes for each
+ * thread ("Architecture", the two-phase kernel); the library's format stores
+ * it. */
 int orc_metadata(const uint8_t *exp, uint64_t n, const uint8_t len[256],
                  uint32_t threads_per_chunk, uint32_t bytes_per_thread,
-                 uint64_t n_chunks, uint8_t *gap, uint32_t *pos);
+                 uint64_t n_chunks, uint8_t *gap, uint8_t *count, uint32_t *pos);
 
 /* [DF11-page] "How to run it in production": checksum every artifact.  The
  * checksum is CRC-32C (Castagnoli), written here bit by bit from its

@@ -26,14 +26,16 @@ def test_e2e_plan_covers_every_byte_a_range_reads(pieces, bpt):
     assert all(c0 < c1 for c0, c1, *_ in plan)
     W = 32 * bpt
     pos = hb.chunk_pos.astype(np.int64)
-    covered = {n: np.zeros(getattr(hb, n).nbytes, bool) for n in ("exp_stream", "gaps", "chunk_pos", "signmant")}
+    covered = {n: np.zeros(getattr(hb, n).nbytes, bool)
+               for n in ("exp_stream", "gaps", "counts", "chunk_pos", "signmant")}
     out_prev = 0
     for c0, c1, p0, p1, spans in plan:
         assert (p0, p1) == (pos[c0], pos[c1]) and p0 == out_prev
         out_prev = p1
         got = {n: (a, b) for n, a, b in spans}
         need = {"exp_stream": (W * c0, min(W * c1 + 16, hb.exp_stream.nbytes)),
-                "gaps": (16 * c0, 16 * c1),
+                "gaps": (16 * c0, min(16 * c1 + 1, hb.gaps.nbytes)),
+                "counts": (32 * c0, 32 * c1),
                 "chunk_pos": (4 * c0, 4 * (c1 + 1)),
                 "signmant": (p0 & ~15, min((p1 + 15) & ~15, hb.signmant.nbytes))}
         for n, (a, b) in need.items():
@@ -44,6 +46,7 @@ def test_e2e_plan_covers_every_byte_a_range_reads(pieces, bpt):
     # together the pieces move every byte of the stream words, gaps, positions
     # and sign|mantissa bytes a whole-block decode reads
     assert covered["gaps"][: 16 * n_chunks].all()
+    assert covered["counts"][: 32 * n_chunks].all()
     assert covered["chunk_pos"][: 4 * (n_chunks + 1)].all()
     assert covered["exp_stream"][: W * n_chunks].all()
     assert covered["signmant"][: hb.n_elements].all()

@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
 
-ARRAYS = ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")
+ARRAYS = ("exp_stream", "gaps", "counts", "chunk_pos", "signmant", "lut")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -30,7 +30,7 @@ def _cuda():
 
 
 def _oracle_list(hb):
-    return oracle.block_checksums(hb.exp_stream, hb.gaps, hb.chunk_pos, hb.signmant, hb.lut)
+    return oracle.block_checksums(hb.exp_stream, hb.gaps, hb.counts, hb.chunk_pos, hb.signmant, hb.lut)
 
 
 def _block(name):
@@ -108,7 +108,7 @@ def test_full_block_device_checksum():
     got = df11.checksum_device(db).cpu().numpy().view(np.uint32)
     host = {a: db.tensors[a][: db.sizes[a]].cpu().numpy() for a in ARRAYS}
     hb = df11.HostBlock(header=db.header, exp_stream=host["exp_stream"], gaps=host["gaps"],
-                        chunk_pos=host["chunk_pos"].view(np.uint32), signmant=host["signmant"],
+                        counts=host["counts"], chunk_pos=host["chunk_pos"].view(np.uint32), signmant=host["signmant"],
                         lut=host["lut"].view(np.uint16))
     assert np.array_equal(got, df11.checksum(hb))
     rng = np.random.default_rng(9)

@@ -28,10 +28,12 @@ def _flat(mats):
     return np.concatenate([np.ascontiguousarray(m, dtype=np.uint16).reshape(-1) for m in mats])
 
 
-def gpu_decode(hb, capacity=None, guard=0, stream=None, workspace=True):
+def gpu_decode(hb, capacity=None, guard=0, stream=None, workspace=True, decode_table=True):
     """Decode on cuda:0 into a buffer with `guard` extra elements set to a
-    sentinel; returns (output incl. guard as uint16, error word)."""
-    db = hb.to_device("cuda")
+    sentinel; returns (output incl. guard as uint16, error word).
+    decode_table: the multi-code table built on the host (else every CTA
+    builds it)."""
+    db = hb.to_device("cuda", decode_table=decode_table)
     n = hb.n_elements
     out = torch.full((n + guard,), 0x5A5A, dtype=torch.int16, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -40,11 +42,11 @@ def gpu_decode(hb, capacity=None, guard=0, stream=None, workspace=True):
     return out.cpu().numpy().view(np.uint16), int(err.item())
 
 
-def check_block(mats, bytes_per_thread=8, oracle_decode=True, workspace=True):
+def check_block(mats, bytes_per_thread=8, oracle_decode=True, workspace=True, decode_table=True):
     w = _flat(mats)
     cb = df11.build_codebook(mats)
     hb = df11.compress(cb, mats, 32, bytes_per_thread)
-    got, err = gpu_decode(hb, guard=8, workspace=workspace)
+    got, err = gpu_decode(hb, guard=8, workspace=workspace, decode_table=decode_table)
     assert err == 0
     assert np.all(got[w.size:] == 0x5A5A), "wrote past the block"
     got = got[: w.size]
@@ -76,8 +78,40 @@ BPT = [8, 16]
 @pytest.mark.parametrize("name", sorted(SMALL))
 @pytest.mark.parametrize("bpt", BPT)
 @pytest.mark.parametrize("schedule", ["dynamic", "static"])
-def test_small_workloads(name, bpt, schedule):
-    check_block([m for _, m in SMALL[name]()], bytes_per_thread=bpt, workspace=schedule == "dynamic")
+@pytest.mark.parametrize("table", ["prebuilt", "per_cta"])
+def test_small_workloads(name, bpt, schedule, table):
+    check_block([m for _, m in SMALL[name]()], bytes_per_thread=bpt, workspace=schedule == "dynamic",
+                decode_table=table == "prebuilt")
+
+
+def test_garbage_decode_table_stays_in_bounds():
+    """A decode table that is not the block's (random words, and one with
+    impossible lengths and counts) gives wrong output or error bits, but
+    every write stays inside the output buffer: the kernel turns entries no
+    table could hold into the long-code marker and masks unused symbol
+    bytes."""
+    mats = [m for _, m in workloads.llama_block(1000, scale_div=64)]
+    hb = df11.compress(df11.build_codebook(mats), mats)
+    n = hb.n_elements
+    rng = np.random.default_rng(7)
+    good = df11.build_decode_table(hb.lut, hb.header.n_tables, hb.header.min_code_len)
+    tables = [rng.integers(0, 1 << 63, good.size, dtype=np.uint64),
+              good ^ np.uint64(0x0000_0001_0000_0000),                 # lengths one off
+              (good & np.uint64(0xFFFFFFFF)) | np.uint64((1 | 4 << 19) << 32),   # 4 codes in 1 bit
+              good.copy()]
+    tables[3][::3] = np.uint64(0)                                       # zero entries
+    for tab in tables:
+        db = hb.to_device("cuda", decode_table=False)
+        db.decode_table = torch.from_numpy(tab.view(np.uint8).copy()).cuda()
+        out = torch.full((n + 64,), 0x5A5A, dtype=torch.int16, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        df11.decompress_async(db, out, err, capacity=n)
+        torch.cuda.synchronize()
+        got = out.cpu().numpy().view(np.uint16)
+        assert np.all(got[n:] == 0x5A5A), "wrote past the output"
+    # the block's own table again: exact
+    got, err = gpu_decode(hb, guard=8)
+    assert err == 0 and np.array_equal(got[:n], _flat(mats))
 
 
 # ------------------------------------------------------- chunk schedules
@@ -215,14 +249,19 @@ def _small_block(seed=21):
 
 
 def test_wrong_chunk_position_sets_count_bit():
+    """A position that disagrees with its chunks' counts: both chunks it
+    bounds report it and write nothing; the other chunks stay exact."""
     mats, cb, hb = _small_block()
     assert hb.header.n_chunks >= 3
     hb.chunk_pos[1] += 1
     got, err = gpu_decode(hb, guard=64)
     assert err & df11.DEVERR_COUNT
-    assert np.all(got[hb.n_elements:] == 0x5A5A)
+    n = hb.n_elements
+    assert np.all(got[n:] == 0x5A5A)
     w = _flat(mats)
-    assert np.array_equal(got[: hb.chunk_pos[1] - 1], w[: hb.chunk_pos[1] - 1])
+    p2 = int(hb.chunk_pos[2])
+    assert np.all(got[:p2] == 0x5A5A)
+    assert np.array_equal(got[p2:n], w[p2:])
 
 
 def test_non_monotone_and_out_of_range_positions_write_nothing_outside():
@@ -278,45 +317,84 @@ def test_header_claiming_shorter_shortest_code_still_decodes(bpt):
     assert np.array_equal(got[: hb.n_elements], _flat(mats))
 
 
-def _thread_counts(stream, lengths, gap, total_bits, chunk, tpc, slice_bits):
-    """Codes each thread of `chunk` decodes, by the oracle's bit-by-bit decode
-    under the kernel's contract (codes starting in the slice, from its gap)."""
-    n = 0
+def _chunk_breaks_contract(stream, lengths, gap, count, total_bits, chunk, tpc, slice_bits):
+    """The per-thread contract the kernel checks, by the oracle's bit-by-bit
+    decode: thread g decodes the codes that start in [gap, end) of its
+    slice (end = the slice end, or the end of the stream); there must be
+    count[g] of them, and the next code must start where they end (the next
+    thread's first code, B (g + 1) + gap[g + 1], or the end of the stream).
+    True when some thread of `chunk` breaks it."""
     for t in range(tpc):
         g = chunk * tpc + t
-        p = slice_bits * g + int(gap[g])
-        end = min(slice_bits * (g + 1), total_bits)
+        b0 = slice_bits * g
+        if b0 >= total_bits:
+            continue
+        p = b0 + int(gap[g])
+        end = min(b0 + slice_bits, total_bits)
+        n = 0
         while p < end:
             _, p = oracle.decode(stream, 1, lengths, start_bit=p)
             n += 1
-    return n
+        nb = b0 + slice_bits
+        expect = nb + int(gap[g + 1]) if nb < total_bits else total_bits
+        if n != int(count[g]) or (n and p != expect):
+            return True
+    return False
 
 
 @pytest.mark.parametrize("bpt", BPT)
-def test_flipped_bit_detected_when_chunk_count_changes(bpt):
+def test_flipped_bit_detected_exactly_when_a_thread_breaks_its_contract(bpt):
     """A flipped stream bit desyncs only the thread(s) that read it; the
-    kernel reports it whenever that changes the chunk's code count."""
+    kernel sets the count bit exactly when the oracle says a thread of the
+    chunk no longer decodes its stored count of codes ending where the next
+    thread's first code starts."""
     mats = [m for _, m in workloads.single_matrix(0, shape=(64, 512))]
     cb = df11.build_codebook(mats)
     L = cb.lengths()
     rng = np.random.default_rng(99)
     flagged = 0
-    for trial in range(12):
+    for trial in range(24):
         hb = df11.compress(cb, mats, 32, bpt)
         gaps = np.empty(hb.gaps.size * 2, np.uint8)
         gaps[0::2], gaps[1::2] = hb.gaps & 15, hb.gaps >> 4
         bit = int(rng.integers(0, hb.header.total_bits))
         hb.exp_stream[bit // 8] ^= np.uint8(0x80 >> (bit % 8))
         chunk = bit // (32 * 8 * bpt)
-        changed = False
+        broken = False
         for c in {max(chunk - 1, 0), chunk}:
-            want = int(hb.chunk_pos[c + 1] - hb.chunk_pos[c])
-            changed |= _thread_counts(hb.exp_stream, L, gaps, hb.header.total_bits, c, 32,
-                                      8 * bpt) != want
+            broken |= _chunk_breaks_contract(hb.exp_stream, L, gaps, hb.counts, hb.header.total_bits, c, 32,
+                                             8 * bpt)
         _, err = gpu_decode(hb)
-        assert bool(err & df11.DEVERR_COUNT) == changed
-        flagged += changed
+        assert bool(err & df11.DEVERR_COUNT) == broken, (trial, bit)
+        flagged += broken
     assert flagged > 0
+
+
+def test_corrupt_counts_are_caught_and_stay_in_bounds():
+    """Counts that disagree with the positions, exceed what a slice can hold,
+    or move codes between threads: the count bit is set and nothing is
+    written outside the output."""
+    mats = [m for _, m in workloads.llama_block(1000, scale_div=64)]
+    hb0 = df11.compress(df11.build_codebook(mats), mats)
+    n = hb0.n_elements
+    rng = np.random.default_rng(5)
+    for kind in ("plus_one", "max", "swap", "zero"):
+        hb = df11.compress(df11.build_codebook(mats), mats)
+        g = int(rng.integers(0, hb.counts.size - 40))
+        g -= g % 32
+        if kind == "plus_one":
+            hb.counts[g + 3] += 1
+        elif kind == "max":
+            hb.counts[g + 5] = 255
+        elif kind == "swap":            # same chunk total, codes moved between threads
+            hb.counts[g + 7] += 2
+            hb.counts[g + 8] -= 2
+        else:
+            hb.counts[g + 9] = 0
+            hb.counts[g + 10] += hb0.counts[g + 9]
+        got, err = gpu_decode(hb, guard=64)
+        assert err & df11.DEVERR_COUNT, kind
+        assert np.all(got[n:] == 0x5A5A), kind
 
 
 # --------------------------------------------------------- full workloads

@@ -84,13 +84,15 @@ def test_a_range_reads_and_writes_only_its_own_bytes(bpt):
         spans.append((a, b))
     for c0, c1 in spans:
         # poison every array, then restore only what the range may read
-        for name in ("exp_stream", "gaps", "chunk_pos", "signmant"):
+        for name in ("exp_stream", "gaps", "counts", "chunk_pos", "signmant"):
             db.tensors[name].fill_(0xA5)
         src = {n: torch.from_numpy(getattr(hb, n).view(np.uint8)).cuda()
-               for n in ("exp_stream", "gaps", "chunk_pos", "signmant")}
+               for n in ("exp_stream", "gaps", "counts", "chunk_pos", "signmant")}
         s0, s1 = W * c0, min(W * c1 + STREAM_PAD, hb.exp_stream.nbytes)
         db.tensors["exp_stream"][s0:s1] = src["exp_stream"][s0:s1]
-        db.tensors["gaps"][16 * c0:16 * c1] = src["gaps"][16 * c0:16 * c1]
+        g1 = min(16 * c1 + 1, hb.gaps.nbytes)       # and the gap of the thread after the range
+        db.tensors["gaps"][16 * c0:g1] = src["gaps"][16 * c0:g1]
+        db.tensors["counts"][32 * c0:32 * c1] = src["counts"][32 * c0:32 * c1]
         db.tensors["chunk_pos"][4 * c0:4 * (c1 + 1)] = src["chunk_pos"][4 * c0:4 * (c1 + 1)]
         p0, p1 = int(pos[c0]), int(pos[c1])
         m0, m1 = p0 & ~15, min((p1 + 15) & ~15, hb.signmant.nbytes)

@@ -65,6 +65,7 @@ def check_format_parity(mats, bytes_per_thread=8, cap=16):
     gaps = np.empty(hb.gaps.size * 2, np.uint8)
     gaps[0::2], gaps[1::2] = hb.gaps & 15, hb.gaps >> 4
     assert np.array_equal(gaps, ob.gap)
+    assert np.array_equal(hb.counts, ob.thread_count)
     assert np.array_equal(hb.chunk_pos, ob.pos)
     assert np.array_equal(hb.signmant[: w.size], ob.signmant)
     assert not hb.signmant[w.size:].any()
@@ -387,9 +388,9 @@ def test_compress_device_rejects_bad_arguments_before_any_cuda_call():
     z = df11.compress_sizes(cb)
     fake = 1 << 20
     b = binding._Block()
-    for name in ("exp_stream", "gaps", "chunk_pos", "signmant", "lut"):
+    for name in binding.ARRAYS:
         setattr(b, name, fake)
-    b.exp_stream_bytes, b.gaps_bytes = z.exp_stream_bytes, z.gaps_bytes
+    b.exp_stream_bytes, b.gaps_bytes, b.counts_bytes = z.exp_stream_bytes, z.gaps_bytes, z.counts_bytes
     b.chunk_pos_count, b.signmant_bytes, b.lut_entries = z.chunk_pos_count, z.signmant_bytes, z.lut_entries
     scratch = df11.compress_device_scratch_bytes(n)
     assert scratch >= 12 * ((n + 8191) // 8192)
@@ -407,6 +408,12 @@ def test_compress_device_rejects_bad_arguments_before_any_cuda_call():
     short = binding._Block.from_buffer_copy(b)
     short.gaps_bytes -= 1
     assert call(blk=short) == 2
+    short = binding._Block.from_buffer_copy(b)
+    short.counts_bytes -= 1
+    assert call(blk=short) == 2
+    nocounts = binding._Block.from_buffer_copy(b)
+    nocounts.counts = None
+    assert call(blk=nocounts) == 1
     assert lib.df11_histogram_device(None, n, fake, None) == 1
     assert lib.df11_histogram_device(fake, 0, fake, None) == 1
     assert lib.df11_histogram_device(fake + 2, n, fake, None) == 1
@@ -418,7 +425,7 @@ def test_compress_device_rejects_bad_arguments_before_any_cuda_call():
 # oracle's bit-by-bit CRC of every 4096-byte segment of every array.
 
 def _oracle_list(hb):
-    return oracle.block_checksums(hb.exp_stream, hb.gaps, hb.chunk_pos, hb.signmant, hb.lut)
+    return oracle.block_checksums(hb.exp_stream, hb.gaps, hb.counts, hb.chunk_pos, hb.signmant, hb.lut)
 
 
 @pytest.mark.parametrize("name", ["single_1024x1024", "heavy_tail_512", "single_exponent_512"])
@@ -500,3 +507,78 @@ def test_decode_gemv_rejects_bad_arguments_before_any_cuda_call():
     assert call(table(bad), len(bad), 1) == 1
     assert lib.df11_decode_gemv_async(None, good, len(shapes), 1, None, None, None) == 1
     assert call(good, len(shapes), 1, ws=fake + 8) == 1         # misaligned workspace
+
+
+# ------------------------------------------------ decoder's multi-code table
+
+def _oracle_multi_entry(k, sym, ln, window_bits=11):
+    """The entry for window k (first stream bit = bit 0 of k) from the
+    oracle's first-code table: the whole codes the window starts with, at
+    most four, as rotated exponents and their total length | 8 x count << 16."""
+    m = 0
+    for b in range(window_bits):
+        m |= ((k >> b) & 1) << (window_bits - 1 - b)        # MSB-first window
+    used = n = syms = 0
+    while n < 4:
+        v = ((m << used) << (16 - window_bits)) & 0xFFFF     # unknown bits read as 0
+        s, l = int(sym[v]), int(ln[v])
+        if s < 0 or used + l > window_bits:
+            break
+        syms |= (((s >> 1) | ((s & 1) << 7)) & 0xFF) << (8 * n)
+        n += 1
+        used += l
+    y = used | (8 * n << 16) if n else 0x80000000
+    return syms | (y << 32)
+
+
+@pytest.mark.parametrize("name", ["single_1024x1024", "heavy_tail_1024", "uniform_bits_1024",
+                                  "single_exponent_1024", "many_tables"])
+def test_decode_table_equals_oracle_walk(name):
+    """df11_build_decode_table: every one of the 2048 entries equals a walk
+    of the window with the oracle's canonical first-code table (the codes
+    the window starts with and their lengths), for codebooks with short and
+    long codes, many sub-tables and a single symbol ("Architecture":
+    hierarchical lookup tables; "How it works": canonical codes)."""
+    mats = {
+        "single_1024x1024": lambda: workloads.single_matrix(0),
+        "heavy_tail_1024": lambda: workloads.heavy_tail(4001, (1024, 1024)),
+        "uniform_bits_1024": lambda: workloads.uniform_bits(4003, (1024, 1024)),
+        "single_exponent_1024": lambda: workloads.single_exponent(4002, (1024, 1024)),
+        "many_tables": lambda: workloads.many_tables(),
+    }[name]()
+    mats = [m for _, m in mats]
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats)
+    tab = df11.build_decode_table(hb.lut, hb.header.n_tables, hb.header.min_code_len)
+    sym, ln = oracle.first_code_table(cb.lengths())
+    want = np.array([_oracle_multi_entry(k, sym, ln) for k in range(2048)], np.uint64)
+    bad = np.nonzero(tab != want)[0]
+    assert bad.size == 0, f"{bad.size} entries differ, first {bad[:4]}: {tab[bad[:4]]} vs {want[bad[:4]]}"
+
+
+def test_decode_table_reads_malformed_tables_as_no_code():
+    """Entries the decoder sanitises (a pointer inside a sub-table, a
+    pointer to a missing table, a leaf shorter than the shortest code) end
+    the walk exactly where a "no code" entry would; bad arguments are
+    refused."""
+    mats = [m for _, m in workloads.heavy_tail(4001, (1024, 1024))]
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats)
+    nt, ml = hb.header.n_tables, hb.header.min_code_len
+    good = df11.build_decode_table(hb.lut, nt, ml)
+    lut = hb.lut.copy()
+    root = int(np.nonzero(lut[:256] & 0x8000)[0][0])          # a root pointer
+    lut[root] = 0x8000 | nt                                   # to a table that does not exist
+    bad = df11.build_decode_table(lut, nt, ml)
+    # windows whose first 8 bits are that prefix now start with no code
+    for k in range(2048):
+        first8 = int(''.join(str((k >> b) & 1) for b in range(8)), 2)
+        if first8 == root:
+            assert bad[k] == np.uint64(0x80000000 << 32)
+    assert np.any(bad != good)
+    with pytest.raises(df11.DF11Error):
+        df11.build_decode_table(hb.lut, 0, ml)
+    with pytest.raises(df11.DF11Error):
+        df11.build_decode_table(hb.lut, nt, 0)
+    with pytest.raises(df11.DF11Error):
+        df11.build_decode_table(hb.lut, nt, 17)

@@ -345,16 +345,19 @@ def _brute_metadata(lens_per_symbol, T, W, n_chunks):
         else:
             gap.append(min(s for s in starts if s >= B * g) - B * g)
     pos = [sum(1 for s in starts[:-1] if s < c * T * B) for c in range(n_chunks + 1)]
-    return gap, pos
+    count = [sum(1 for s in starts[:-1] if B * g <= s < B * (g + 1)) for g in range(n_chunks * T)]
+    return gap, count, pos
 
 
 @pytest.mark.parametrize("seed", range(8))
 @pytest.mark.parametrize("T,W", [(2, 1), (4, 2), (8, 8), (4, 8)])
 def test_metadata_brute_force_and_thread_decode(seed, T, W):
-    """Gaps and chunk positions against their definitions, and the property
-    the two-phase kernel rests on: every thread decoding the codes that start
-    in its slice, from its gap, reproduces the serial decode, and each chunk
-    yields exactly pos[c+1]-pos[c] symbols."""
+    """Gaps, per-thread counts and chunk positions against their
+    definitions, and the properties the decoder rests on: every thread
+    decoding the codes that start in its slice, from its gap, reproduces the
+    serial decode; it decodes exactly count[g] codes, and they end where the
+    next thread's first code starts (or at the end of the stream); each
+    chunk yields exactly pos[c+1]-pos[c] symbols, the sum of its counts."""
     rng = np.random.default_rng(seed)
     n_sym = int(rng.integers(1, 9))
     syms = rng.choice(256, n_sym, replace=False)
@@ -369,9 +372,9 @@ def test_metadata_brute_force_and_thread_decode(seed, T, W):
     tb = sum(lens_seq)
     B = 8 * W
     n_chunks = (tb + T * B - 1) // (T * B)
-    gap, pos = oracle.metadata(e, L, T, W, n_chunks)
-    bg, bp = _brute_metadata(lens_seq, T, W, n_chunks)
-    assert gap.tolist() == bg and pos.tolist() == bp
+    gap, count, pos = oracle.metadata(e, L, T, W, n_chunks)
+    bg, bc, bp = _brute_metadata(lens_seq, T, W, n_chunks)
+    assert gap.tolist() == bg and pos.tolist() == bp and count.tolist() == bc
     assert int(gap.max()) < max(int(L.max()), 1) or tb == 0
     stream, _ = oracle.encode(e, L, codes, n_chunks * T * W + 16)
     out = []
@@ -381,12 +384,18 @@ def test_metadata_brute_force_and_thread_decode(seed, T, W):
             g = ch * T + t
             p0 = B * g + int(gap[g])
             end = min(B * (g + 1), tb)
+            mine = 0
             while p0 < end:
                 d, nxt = oracle.decode(stream, 1, L, start_bit=p0)
                 out.append(int(d[0]))
                 p0 = nxt
                 got += 1
-        assert got == int(pos[ch + 1] - pos[ch])
+                mine += 1
+            assert mine == int(count[g])
+            nxt_start = B * (g + 1) + int(gap[g + 1]) if g + 1 < gap.size and B * (g + 1) < tb else tb
+            if mine:
+                assert p0 == nxt_start
+        assert got == int(pos[ch + 1] - pos[ch]) == int(count[ch * T:(ch + 1) * T].sum())
     assert out == e.tolist()
 
 

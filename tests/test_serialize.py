@@ -1,6 +1,6 @@
 """A block as one flat buffer (df11_serialize / df11_deserialize), CPU only.
 
-The container holds the block header, the five arrays and the CRC-32C of
+The container holds the block header, the six arrays and the CRC-32C of
 every 4096-byte segment of them ("DFloat11: lossless BFloat16 compression",
 "How to run it in production": checksum artifacts on download and after
 every copy).  Checks: a round trip gives back every array byte for byte and
@@ -17,7 +17,7 @@ import workloads
 import huffman_decode_b200 as df11
 from huffman_decode_b200 import df11 as binding
 
-ARRAYS = ("exp_stream", "gaps", "chunk_pos", "signmant", "lut")
+ARRAYS = binding.ARRAYS
 BLOCKS = {
     "llama_div256": lambda: workloads.llama_block(1003, scale_div=256),
     "heavy_tail_256": lambda: workloads.heavy_tail(4001, (256, 256)),
@@ -109,7 +109,7 @@ def test_truncated_padded_or_foreign_buffers_are_refused():
         _refused(data[:cut])
     _refused(data + b"\0" * 4)
     buf = bytearray(data)
-    buf[8] = 2                  # another version (header CRC recomputed below)
+    buf[8] = 1                  # another version (the header CRC no longer matches)
     _refused(buf)
     _refused(b"NOTDF11!" + data[8:])
 
