@@ -65,7 +65,7 @@ constexpr int kMaxCodesPerEntry = 4;
 static_assert(kWindowBits == DF11_DECODE_TABLE_WINDOW_BITS && kMultiEntries == DF11_DECODE_TABLE_ENTRIES,
               "the host-built decode table has the kernel's shape");
 constexpr int kEntryBytes = 8;                     // multi-code entry: symbols | step
-constexpr uint32_t kLongStep = 0x80000000u;        // step of an entry whose first code is long
+constexpr uint32_t kLongStep = 0x4000u;            // step of an entry whose first code is long
 constexpr int kMaxWarpsPerCta = 32;
 // A checked build (-DDF11_CHECKED, libdf11_checked.so) verifies at run time
 // the invariants that keep every access in bounds, ORs DF11_DEVERR_BOUNDS
@@ -243,73 +243,77 @@ __device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v)
 
 static_assert(kEntryBytes == 8, "lookup_step scales the table index by 8");
 
-// Lane decode state X: bit position in bits 0..15, fill of the word being
-// filled (in bits, 0..24 between lookups) in bits 16..21; kLongStep (bit 31)
-// is added by an entry whose first code is longer than the window.
-constexpr uint32_t kFillOne = 1u << 16;          // X units of one fill bit
-constexpr uint32_t kPosMask = 0xFFFFu | kLongStep;
+// Lane decode state X: bit position in bits 0..13; kLongStep (bit 14) is
+// added by an entry whose first code is longer than the window (it ends the
+// lookup loop); fill of the word being filled (in bits, 0..24 between
+// lookups) in bits 26..31, so a full word (fill >= 32) is X >= 2^31.  A table
+// entry's step y = total length | 8 x count << 26 advances both fields with
+// one add.
+constexpr int kFillShift = 26;
+constexpr uint32_t kFillOne = 1u << kFillShift;   // X units of one fill bit
+constexpr uint32_t kWordFull = 32u * kFillOne;    // fill >= 32
+constexpr uint32_t kPosMask = 0xFFFFu;            // bit position and the long marker
+
+// y of a table entry holding n codes of total length t
+__host__ __device__ constexpr uint32_t entry_step(uint32_t t, uint32_t n) { return t | (8u * n << kFillShift); }
+// codes of a table entry's y
+__device__ __forceinline__ uint32_t entry_codes(uint32_t y) { return y >> (kFillShift + 3); }
 
 // One multi-code lookup for window `win` (the upcoming stream bits, first
 // lowest): appends the entry's symbols to the word being filled at the
 // fill, steps X, computes the next window from the stream words lo:hi, and
-// stores the word to the exponent buffer (then carries the overflow) when
-// it is full (OR: ORs it into a zeroed buffer).  One predicated block, so
-// the store is not a branch; the next window is formed before the store so
-// it waits only on the step.
+// when the word is full stores it to the exponent buffer (OR: ORs it into a
+// zeroed buffer) and starts the next word with the symbols past it.  One
+// predicated block, so the store is not a branch; the next window is formed
+// before the store so it waits only on the step.
 template <bool OR>
 __device__ __forceinline__ void lookup_step(uint32_t &X, uint32_t &win, uint32_t &accl, uint32_t &sp,
                                             uint2 &r, uint32_t lo, uint32_t hi, uint32_t multi_a)
 {
     if constexpr (OR)
         asm volatile(
-        "{\n\t"
-        ".reg .b32 a, f, t, z, c;\n\t"
-        ".reg .pred p;\n\t"
-        "mov.b32 z, 0;\n\t"
-        "and.b32 a, %1, %9;\n\t"
-        "mad.lo.u32 a, a, 8, %8;\n\t"
-        "ld.shared.v2.u32 {%4, %5}, [a];\n\t"
-        "shr.b32 f, %0, 16;\n\t"
-        "shf.l.wrap.b32 t, z, %4, f;\n\t"
-        "or.b32 %2, %2, t;\n\t"
-        "shf.l.wrap.b32 c, %4, z, f;\n\t"
-        "add.u32 %0, %0, %5;\n\t"
-        "shf.r.wrap.b32 %1, %6, %7, %0;\n\t"
-        "and.b32 t, %0, 2097152;\n\t"
-        "setp.ne.u32 p, t, 0;\n\t"
-        "@p red.shared.or.b32 [%3], %2;\n\t"
-        "@p add.u32 %3, %3, 4;\n\t"
-        "@p mov.b32 %2, c;\n\t"
-        "@p sub.u32 %0, %0, 2097152;\n\t"
-        "}"
-        : "+r"(X), "+r"(win), "+r"(accl), "+r"(sp), "=r"(r.x), "=r"(r.y)
-        : "r"(lo), "r"(hi), "r"(multi_a), "n"(kMultiEntries - 1)
-        : "memory");
+            "{\n\t"
+            ".reg .b32 a, f, t;\n\t"
+            ".reg .pred p;\n\t"
+            "and.b32 a, %1, %9;\n\t"
+            "mad.lo.u32 a, a, 8, %8;\n\t"
+            "ld.shared.v2.u32 {%4, %5}, [a];\n\t"
+            "shr.b32 f, %0, 26;\n\t"
+            "shf.l.wrap.b32 t, %10, %4, f;\n\t"
+            "or.b32 %2, %2, t;\n\t"
+            "add.u32 %0, %0, %5;\n\t"
+            "shf.r.wrap.b32 %1, %6, %7, %0;\n\t"
+            "setp.ge.u32 p, %0, %11;\n\t"
+            "@p red.shared.or.b32 [%3], %2;\n\t"
+            "@p shf.l.wrap.b32 %2, %4, %10, f;\n\t"
+            "@p add.u32 %3, %3, 4;\n\t"
+            "@p sub.u32 %0, %0, %11;\n\t"
+            "}"
+            : "+r"(X), "+r"(win), "+r"(accl), "+r"(sp), "=r"(r.x), "=r"(r.y)
+            : "r"(lo), "r"(hi), "r"(multi_a), "n"(kMultiEntries - 1), "r"(0u), "n"(kWordFull)
+            : "memory");
     else
-    asm volatile(
-        "{\n\t"
-        ".reg .b32 a, f, t, z, c;\n\t"
-        ".reg .pred p;\n\t"
-        "mov.b32 z, 0;\n\t"
-        "and.b32 a, %1, %9;\n\t"
-        "mad.lo.u32 a, a, 8, %8;\n\t"
-        "ld.shared.v2.u32 {%4, %5}, [a];\n\t"
-        "shr.b32 f, %0, 16;\n\t"
-        "shf.l.wrap.b32 t, z, %4, f;\n\t"       // symbols << fill
-        "or.b32 %2, %2, t;\n\t"
-        "shf.l.wrap.b32 c, %4, z, f;\n\t"       // symbols past the word
-        "add.u32 %0, %0, %5;\n\t"
-        "shf.r.wrap.b32 %1, %6, %7, %0;\n\t"    // next window: (hi:lo) >> bit position
-        "and.b32 t, %0, 2097152;\n\t"           // fill >= 32
-        "setp.ne.u32 p, t, 0;\n\t"
-        "@p st.shared.u32 [%3], %2;\n\t"
-        "@p add.u32 %3, %3, 4;\n\t"
-        "@p mov.b32 %2, c;\n\t"
-        "@p sub.u32 %0, %0, 2097152;\n\t"
-        "}"
-        : "+r"(X), "+r"(win), "+r"(accl), "+r"(sp), "=r"(r.x), "=r"(r.y)
-        : "r"(lo), "r"(hi), "r"(multi_a), "n"(kMultiEntries - 1)
-        : "memory");
+        asm volatile(
+            "{\n\t"
+            ".reg .b32 a, f, t;\n\t"
+            ".reg .pred p;\n\t"
+            "and.b32 a, %1, %9;\n\t"
+            "mad.lo.u32 a, a, 8, %8;\n\t"
+            "ld.shared.v2.u32 {%4, %5}, [a];\n\t"
+            "shr.b32 f, %0, 26;\n\t"                // fill
+            "shf.l.wrap.b32 t, %10, %4, f;\n\t"     // symbols << fill
+            "or.b32 %2, %2, t;\n\t"
+            "add.u32 %0, %0, %5;\n\t"
+            "shf.r.wrap.b32 %1, %6, %7, %0;\n\t"    // next window: (hi:lo) >> bit position
+            "setp.ge.u32 p, %0, %11;\n\t"           // the word is full
+            "@p st.shared.u32 [%3], %2;\n\t"
+            "@p shf.l.wrap.b32 %2, %4, %10, f;\n\t" // the next word: symbols past this one
+            "@p add.u32 %3, %3, 4;\n\t"
+            "@p sub.u32 %0, %0, %11;\n\t"
+            "}"
+            : "+r"(X), "+r"(win), "+r"(accl), "+r"(sp), "=r"(r.x), "=r"(r.y)
+            : "r"(lo), "r"(hi), "r"(multi_a), "n"(kMultiEntries - 1), "r"(0u), "n"(kWordFull)
+            : "memory");
 }
 
 // ---- mbarrier + bulk copy (TMA) helpers ------------------------------------
@@ -526,7 +530,7 @@ __device__ __forceinline__ uint2 long_code(uint32_t win, uint32_t lut_a, uint32_
     if (e & kLutPointer)
         e = lds_u16(lut_a + ((((e & 0xFFu) << 8) | ((wm >> 16) & 0xFFu)) << 1));
     seen |= e;
-    return make_uint2(rot_exp(e & 0xFFu), ((e >> 8) & 0x1Fu) | (8u * kFillOne));
+    return make_uint2(rot_exp(e & 0xFFu), entry_step((e >> 8) & 0x1Fu, 1));
 }
 
 // Decodes the codes of a full slice (every lane of the chunk has one) into
@@ -556,7 +560,7 @@ __device__ __forceinline__ uint32_t decode_full_slice(const uint32_t (&w)[W / 4 
     // 128-bit slices: plain stores, ordered as above; 64-bit slices are too
     // short for that order, so their words are ORed into a zeroed buffer
     constexpr bool kOr = kSliceBits - (kWindowBits - 1) <= 64;
-    uint32_t X = gap | ((a & 3u) << 19);
+    uint32_t X = gap | ((a & 3u) * 8u * kFillOne);
     sp = ebuf_a + (a & ~3u);
     accl = 0;
     r = make_uint2(0u, 0u);
@@ -570,24 +574,24 @@ __device__ __forceinline__ uint32_t decode_full_slice(const uint32_t (&w)[W / 4 
         for (;;) {
             while ((X & kPosMask) < lim)
                 lookup_step<kOr>(X, win, accl, sp, r, lo, hi, multi_a);
-            if (X < kLongStep)
+            if (!(X & kLongStep))
                 break;
             // the first code is longer than the window: take it from the
             // two-level tables
             X -= kLongStep;
             r = long_code(win, lut_a, seen);
-            const uint32_t f = X >> 16;
+            const uint32_t f = X >> kFillShift;
             accl |= __funnelshift_l(0u, r.x, f);
             const uint32_t acch = __funnelshift_l(r.x, 0u, f);
             X += r.y;
-            if (X & (32u * kFillOne)) {
+            if (X >= kWordFull) {
                 if constexpr (kOr)
                     red_or_u32(sp, accl);
                 else
                     sts_u32(sp, accl);
                 sp += 4;
                 accl = acch;
-                X -= 32u * kFillOne;
+                X -= kWordFull;
             }
             win = __funnelshift_r(lo, hi, X);
         }
@@ -732,12 +736,17 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
         // holds
         for (int slot = tid; slot < kMultiEntries; slot += blockDim.x) {
             uint2 v = __ldg(p.multi_src + slot);
+            // (the host table's y is length | 8 x count << 16; the long-code
+            // marker 2^31)
             const uint32_t n = v.y >> 19, t = v.y & 0xFFFFu;
             if (v.y != (t | (n << 19)) || n < 1 || n > (uint32_t)kMaxCodesPerEntry ||
-                t > (uint32_t)kWindowBits || t < n * min_len)
+                t > (uint32_t)kWindowBits || t < n * min_len) {
                 v = make_uint2(0u, kLongStep);
-            else if (n < 4)
-                v.x &= (1u << (8 * n)) - 1u;
+            } else {
+                if (n < 4)
+                    v.x &= (1u << (8 * n)) - 1u;
+                v.y = entry_step(t, n);
+            }
             multi[slot] = v;
         }
     } else {
@@ -760,7 +769,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                 ++n;
                 t += l;
             }
-            multi[slot] = make_uint2(syms, n ? t | (8u * n << 16) : kLongStep);
+            multi[slot] = make_uint2(syms, n ? entry_step(t, n) : kLongStep);
         }
     }
     __syncthreads();
@@ -875,8 +884,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                 // codes of the last entry that start at or past the slice
                 // end are the next lane's; the first of them (or the end of
                 // the entry) is where the next code starts
-                const uint32_t emitted = sp - ebuf_a + ((X >> 19) & 7u) - a;
-                const uint32_t n = r.y >> 19;
+                const uint32_t emitted = sp - ebuf_a + (X >> (kFillShift + 3)) - a;
+                const uint32_t n = entry_codes(r.y);
                 int c = (int)(X & 0xFFFFu) - (int)(r.y & 0xFFFFu);   // start of the entry's first code
                 uint32_t keep = n ? 1u : 0u;
                 int next_start = (int)(X & 0xFFFFu);
@@ -894,7 +903,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                 __syncwarp();
                 // the part-filled last word: ORed over the next lane's first
                 // word (zeros below its first byte); the last lane's is its own
-                if (write_ok && (X >> 16)) {
+                if (write_ok && (X >> kFillShift)) {
                     if (kOr || lane < 31)
                         red_or_u32(sp, accl);
                     else
