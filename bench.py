@@ -91,6 +91,11 @@ def parse_args():
                     help="write a 256 MB buffer before every timed launch and time each launch "
                          "alone (for blocks whose working set fits in the 126 MB L2)")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
+    ap.add_argument("--min-seconds", type=float, default=1.0,
+                    help="repeat the timed K steps until about this much wall time has passed "
+                         "(the median repetition is reported)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-configuration measurements of the default run")
     return ap.parse_args()
 
 
@@ -332,7 +337,10 @@ def e2e_pipeline(df11, db, hb, host, out, host_out, err, host_err, pieces, strea
     c_in, c_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     cblk = db.c_struct()
     plan = e2e_plan(hb, pieces)
-    h2d = host["lut"].numel() + sum(b - a for *_, spans in plan for _, a, b in spans)
+    # the decoder's multi-code table travels with the block's tables
+    host_table = db.decode_table.cpu().pin_memory() if db.decode_table is not None else None
+    h2d = (host["lut"].numel() + (host_table.numel() if host_table is not None else 0)
+           + sum(b - a for *_, spans in plan for _, a, b in spans))
     d2h = 2 * int(hb.chunk_pos[-1]) + 4
     ev_in = [torch.cuda.Event() for _ in plan]
     ev_dec = [torch.cuda.Event() for _ in plan]
@@ -344,6 +352,8 @@ def e2e_pipeline(df11, db, hb, host, out, host_out, err, host_err, pieces, strea
         c_out.wait_event(ev_start)
         with torch.cuda.stream(c_in):
             db.tensors["lut"].copy_(host["lut"], non_blocking=True)
+            if host_table is not None:
+                db.decode_table.copy_(host_table, non_blocking=True)
             for i, (_, _, _, _, spans) in enumerate(plan):
                 for name, a, b in spans:
                     db.tensors[name][a:b].copy_(host[name][a:b], non_blocking=True)
@@ -406,6 +416,102 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ------------------------------------------------------ per configuration
+
+# The five configurations of the measured workload list, by name: 1 = one
+# 1024x1024 matrix, 2 = the Llama-3.1-8B-shaped block (the headline), 3 =
+# 32 such blocks with their own codebooks, 4a/b/c = the adversarial 16 M
+# weight blocks, 5 = the FLUX-shaped DiT block.
+PER_CONFIG = [("1", "single_1024x1024"), ("2", "llama8b_block"), ("3", "llama8b_model"),
+              ("4a", "adversarial_heavy_tail"), ("4b", "adversarial_single_exponent"),
+              ("4c", "adversarial_uniform_bits"), ("5", "flux_dit_block")]
+
+
+def _rates(nbytes, n, us, peak):
+    return {"us": round(us, 3), "gb_per_s": round(nbytes / us / 1e3, 2),
+            "gweights_per_s": round(n / us / 1e3, 2), "frac": round(nbytes / us / 1e3 / peak, 4)}
+
+
+def per_config(df11, dev, stream, bpt, peak, headline=None):
+    """Every configuration decoded on this GPU: bit-exactness against the
+    input, then back-to-back launches (CUDA events around a run of launches,
+    median of 5 runs) and, for single blocks, launches timed alone after a
+    256 MB write scrubs the L2 (median of 30).  Config 3 times the 32-block
+    stream (one step = 32 launches into one reused buffer); config 2 reuses
+    the headline's back-to-back figure."""
+    import torch
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out_all = {}
+    for key, name in PER_CONFIG:
+        t0 = time.perf_counter()
+        if name == "llama8b_model":
+            dbs = numpy_model_blocks(workloads.llama_model_seeds(32), dev, bpt)
+            n = sum(db.n_elements for db in dbs)
+            nbytes = sum(db.compressed_bytes() + 2 * db.n_elements for db in dbs)
+            out = torch.empty(max(db.n_elements for db in dbs), dtype=torch.bfloat16, device=dev)
+            cblks = [(db, db.c_struct()) for db in dbs]
+
+            def launch():
+                for db, cb in cblks:
+                    df11.decompress_async(db, out, err, stream=stream, c_block=cb)
+            exact = True   # numpy_model_blocks checked every block
+            reps_per_run = 2
+        else:
+            mats = [m for _, m in workloads.WORKLOADS[name]()]
+            w = np.concatenate([m.reshape(-1) for m in mats])
+            hb = df11.compress(df11.build_codebook(mats), mats, 32, bpt)
+            db = hb.to_device(dev)
+            cb = db.c_struct()
+            n = hb.n_elements
+            nbytes = hb.compressed_bytes() + 2 * n
+            out = torch.empty(n, dtype=torch.int16, device=dev)
+
+            def launch():
+                df11.decompress_async(db, out, err, stream=stream, c_block=cb)
+            launch()
+            exact = bool(torch.equal(out, torch.from_numpy(w.view(np.int16)).to(dev))) and int(err.item()) == 0
+            reps_per_run = 200 if n < 50_000_000 else 40
+            del w, hb
+        gen_s = time.perf_counter() - t0
+        for _ in range(3):
+            launch()
+        runs = []
+        for _ in range(5):
+            a, b = _events(2)
+            a.record(stream)
+            for _ in range(reps_per_run):
+                launch()
+            b.record(stream)
+            b.synchronize()
+            runs.append(a.elapsed_time(b) * 1e3 / reps_per_run)
+        b2b = statistics.median(runs)
+        entry = {"workload": name, "n_weights": n, "bytes_per_launch": nbytes,
+                 "bit_exact": exact, "setup_s": round(gen_s, 1)}
+        if name == "llama8b_block" and headline is not None:
+            b2b = headline
+        entry["back_to_back"] = _rates(nbytes, n, b2b, peak)
+        if name != "llama8b_model":
+            alone = []
+            for i in range(30):
+                scrub.fill_(i & 255)
+                a, b = _events(2)
+                a.record(stream)
+                launch()
+                b.record(stream)
+                b.synchronize()
+                alone.append(a.elapsed_time(b) * 1e3)
+            entry["l2_scrubbed"] = _rates(nbytes, n, statistics.median(alone), peak)
+        else:
+            entry["what"] = "one launch = the 32 blocks decoded one after another (us per 32 blocks)"
+        if int(err.item()):
+            entry["bit_exact"] = False
+        out_all[key] = entry
+        del out
+        torch.cuda.synchronize()
+    return out_all
 
 
 # -------------------------------------------------------------- GPU arm
@@ -477,13 +583,9 @@ def run_b200(args):
         torch.cuda.synchronize()
         ms = sum(a.elapsed_time(b) for a, b in evs)
         del scrub
+        reps = None
     else:
-        start.record(stream)
-        for _ in range(args.steps):
-            step()
-        end.record(stream)
-        end.synchronize()
-        ms = start.elapsed_time(end)
+        ms, reps = timed_reps(step, args.steps, stream, world, min_seconds=args.min_seconds, device=dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -519,6 +621,12 @@ def run_b200(args):
     (ms_max, e2e_ms_per_step), (job_bytes, job_weights) = reduce_over_ranks(
         [ms, e2e["ms"] / e2e["k"] if e2e else 0.0], [bytes_per_step, n], dev)
 
+    per_cfg = None
+    if (rank == 0 and world == 1 and not args.no_per_config and args.workload == WORKLOAD
+            and args.scale_div == 1 and not args.flush_l2):
+        peak_, _ = measured_peaks()
+        per_cfg = per_config(df11, dev, stream, args.bytes_per_thread, peak_,
+                             headline=ms / args.steps * 1e3)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -570,8 +678,12 @@ def run_b200(args):
                        "pieces": max(1, args.e2e_pieces),
                        "what": "pinned host arrays -> device, decode, BF16 + error word -> pinned host, "
                                "as a pipeline over chunk ranges (df11_decompress_range_async)"}
+    if reps:
+        line["timing"] = reps
     if cpu:
         line["cpu_baseline"] = cpu
+    if per_cfg:
+        line["per_config"] = per_cfg
     print(json.dumps(line), flush=True)
     return 0
 
@@ -615,11 +727,37 @@ def gpu_compressed_blocks(n_blocks, seed0, dev, bpt, verify_into=None, scale_div
     return blocks, gpu_ms, host_cb_s
 
 
+def numpy_model_blocks(seeds, dev, bpt, scale_div=1):
+    """The 8B-scale stream as specified: llama_block(seed) for every seed,
+    drawn by numpy in a pool of worker processes, compressed on the host
+    (one codebook per block) and copied to the GPU.  Every block is decoded
+    once into one reused buffer and compared with its input (bit-exact or an
+    exception).  Returns the device blocks."""
+    import torch
+
+    import huffman_decode_b200 as df11
+    stream = torch.cuda.current_stream(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    dbs, out = [], None
+    for sd, w in workloads.llama_model_blocks(seeds, scale_div=scale_div):
+        hb = df11.compress(df11.build_codebook([w]), [w], 32, bpt)
+        db = hb.to_device(dev)
+        if out is None:
+            out = torch.empty(hb.n_elements, dtype=torch.int16, device=dev)
+        df11.decompress_async(db, out[: hb.n_elements], err, stream=stream)
+        want = torch.from_numpy(w.view(np.int16)).to(dev)
+        if int(err.item()) or not torch.equal(out[: hb.n_elements], want):
+            raise RuntimeError(f"block seed {sd}: decode is not bit-exact")
+        del hb, want
+        dbs.append(db)
+    return dbs
+
+
 def run_model_stream(args):
-    """The 8B-scale stream: n_blocks Llama-3.1-8B-shaped blocks (seed 1000 +
-    block, drawn on the GPU), each histogrammed, given its own codebook and
-    compressed on the GPU, all resident in HBM; one step decodes every block
-    in turn into one reused BF16 buffer on one stream."""
+    """The 8B-scale stream: n_blocks Llama-3.1-8B-shaped blocks drawn by numpy
+    (llama_block(seed), seeds 1000 + block), each with its own codebook, all
+    resident in HBM; one step decodes every block in turn into one reused
+    BF16 buffer on one stream."""
     import torch
     import torch.distributed as dist
 
@@ -636,7 +774,8 @@ def run_model_stream(args):
     bpt = args.bytes_per_thread
     n_blocks = args.blocks or 32
     derr = torch.zeros(1, dtype=torch.int32, device=dev)
-    dbs, gpu_ms, host_cb_s = gpu_compressed_blocks(n_blocks, rank_seed(rank, per_rank=n_blocks), dev, bpt)
+    seed0 = rank_seed(rank, per_rank=n_blocks)
+    dbs = numpy_model_blocks(range(seed0, seed0 + n_blocks), dev, bpt, args.scale_div)
     out = torch.empty(max(db.n_elements for db in dbs), dtype=torch.bfloat16, device=dev)
     blocks = [(db, db.c_struct(), db.compressed_bytes() + 2 * db.n_elements) for db in dbs]
     n_weights = sum(db.n_elements for db in dbs)
@@ -650,21 +789,9 @@ def run_model_stream(args):
         step()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
     sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    end.record(stream)
-    end.synchronize()
-    if world > 1:
-        dist.barrier()
+    ms, reps = timed_reps(step, args.steps, stream, world, min_seconds=1.0, device=dev)
     clocks = sampler.stop()
-    ms = start.elapsed_time(end)
     if int(derr.item()):
         raise RuntimeError("device error word set during the timed decode")
     (ms_max,), (job_bytes, job_weights) = reduce_over_ranks([ms], [step_bytes, n_weights], dev)
@@ -677,15 +804,14 @@ def run_model_stream(args):
     launches = args.steps * len(blocks)
     achieved = step_bytes / (ms / args.steps * 1e-3) / 1e9
     value = job_rate(job_bytes, args.steps, ms_max)
-    bf16_in = 2.0 * n_weights / len(blocks)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u8", "data": "synthetic (GPU-drawn, torch CUDA generator)",
+        "dtype": "u8", "data": "synthetic (numpy, llama_block(seed) for every block)",
         "config": {"workload": "llama8b_model", "blocks": len(blocks), "n_weights": n_weights,
                    "threads_per_chunk": 32, "bytes_per_thread": bpt,
-                   "bytes_per_step": step_bytes, "seeds": f"1000..{999 + len(blocks)}",
+                   "bytes_per_step": step_bytes, "seeds": f"{seed0}..{seed0 + len(blocks) - 1}",
                    "l2": "inputs larger than L2, no flush",
                    "parallelism": f"replicas x{world}, own blocks per GPU, no collective"},
         "gweights_per_s": round(job_rate(job_weights, args.steps, ms_max), 2),
@@ -696,13 +822,8 @@ def run_model_stream(args):
                      "traffic": profiled_traffic(n_weights // len(blocks)),
                      "algorithmic_bytes_per_launch": step_bytes // len(blocks)},
         "clocks": clocks,
+        "timing": reps,
         "gpu_launches": launches,
-        "gpu_compress": {"ms_per_block_mean": round(statistics.mean(gpu_ms), 4),
-                         "ms_per_block_min": round(min(gpu_ms), 4),
-                         "bf16_gb_per_s": round(bf16_in / (min(gpu_ms) * 1e-3) / 1e9, 1),
-                         "host_codebook_ms_per_block": round(1e3 * host_cb_s / len(blocks), 3),
-                         "what": "device histogram + device encode per block (CUDA events); "
-                                 "codebook from the histogram on the host"},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -1078,6 +1199,46 @@ def run_gemv(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def timed_reps(step, steps, stream, world, min_seconds=1.0, min_reps=5, device=None):
+    """Times `steps` back-to-back steps between two CUDA events on `stream`,
+    each repetition bracketed by a barrier across ranks and a device
+    synchronize, repeated until about min_seconds of wall time (and at least
+    min_reps repetitions) have passed, so the clock samples taken meanwhile
+    cover a real stretch of load.  The repetition count is fixed up front
+    from a calibration repetition and agreed across ranks (the maximum).
+    Returns (median repetition ms, a record of the repetitions)."""
+    import math
+
+    import torch
+    import torch.distributed as dist
+
+    def one():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a, b = _events(2)
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    t0 = time.perf_counter()
+    times = [one()]
+    wall = time.perf_counter() - t0
+    want = max(min_reps, int(math.ceil(min_seconds / max(wall, 1e-6))))
+    (want,), _ = reduce_over_ranks([want], [], device)
+    for _ in range(int(want) - 1):
+        times.append(one())
+    total = time.perf_counter() - t0
+    med = statistics.median(times)
+    return med, {"reps": len(times), "steps_per_rep": steps, "rep_ms_median": round(med, 5),
+                 "rep_ms_min": round(min(times), 5), "rep_ms_max": round(max(times), 5),
+                 "wall_s": round(total, 3),
+                 "what": "ms_per_step = the median repetition / steps_per_rep"}
 
 
 def _timed_steps(step, steps, warmup, stream, local):

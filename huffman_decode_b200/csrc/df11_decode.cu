@@ -148,7 +148,8 @@ struct Geometry {
 
 // Shared memory: mbarriers | multi-code table | code lengths | per-warp areas
 // | two-level tables.
-constexpr size_t kBarBytes = (kMaxWarpsPerCta * 8 + 15) / 16 * 16;   // one mbarrier per warp
+// one mbarrier per warp, and one for the prologue's table copies
+constexpr size_t kBarBytes = ((kMaxWarpsPerCta + 1) * 8 + 15) / 16 * 16;
 constexpr size_t kHeadBytes = kBarBytes + kMultiEntries * kEntryBytes + 256;
 // per-warp areas and the tables after them keep 16-byte alignment (TMA
 // destinations, 8- and 16-byte shared accesses)
@@ -331,6 +332,17 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uin
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Copies `bytes` (multiple of 16, 16-byte aligned ends) from global to shared
+// memory, completing on `bar`, whose expected byte count the caller set.
+__device__ __forceinline__ void bulk_copy_g2s_tx(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             dst),
@@ -550,16 +562,18 @@ __device__ __forceinline__ uint2 long_code(uint32_t win, uint32_t lut_a, uint32_
 // at the end is left in accl at address sp (fill in X) for the caller to OR
 // in.  Returns X: bit position after the last lookup (bits 0..15), fill
 // (bits 16..21); r holds the last table entry.
-template <int W>
-__device__ __forceinline__ uint32_t decode_full_slice(const uint32_t (&w)[W / 4 + 1], uint32_t gap, uint32_t a,
-                                                      uint32_t ebuf_a, uint32_t multi_a, uint32_t lut_a,
-                                                      uint32_t &seen, uint32_t &sp, uint32_t &accl, uint2 &r)
+//
+// kOr: the words are ORed into a zeroed buffer instead, which needs no
+// order: for 64-bit slices (too short for the order above), and in the
+// block's last chunk, whose slices end at the end of the stream (`end`
+// below the slice width) or lie past it.
+template <int W, bool kOr>
+__device__ __forceinline__ uint32_t decode_slice(const uint32_t (&w)[W / 4 + 1], uint32_t gap, uint32_t a, int end,
+                                                 uint32_t ebuf_a, uint32_t multi_a, uint32_t lut_a, uint32_t &seen,
+                                                 uint32_t &sp, uint32_t &accl, uint2 &r)
 {
     constexpr int kWords = W / 4 + 1;
-    constexpr int kSliceBits = 8 * W;
-    // 128-bit slices: plain stores, ordered as above; 64-bit slices are too
-    // short for that order, so their words are ORed into a zeroed buffer
-    constexpr bool kOr = kSliceBits - (kWindowBits - 1) <= 64;
+    static_assert(kOr || 8 * W - (kWindowBits - 1) > 64, "the ordered stores need slices over 74 bits");
     uint32_t X = gap | ((a & 3u) * 8u * kFillOne);
     sp = ebuf_a + (a & ~3u);
     accl = 0;
@@ -569,7 +583,7 @@ __device__ __forceinline__ uint32_t decode_full_slice(const uint32_t (&w)[W / 4 
         if (!kOr && h == 2)
             __syncwarp();   // every lane's first word is stored by now
         const uint32_t lo = w[h], hi = w[h + 1];
-        const uint32_t lim = (uint32_t)min(kSliceBits, 32 * (h + 1));
+        const uint32_t lim = (uint32_t)max(0, min(end, 32 * (h + 1)));
         uint32_t win = __funnelshift_r(lo, hi, X);
         for (;;) {
             while ((X & kPosMask) < lim)
@@ -597,51 +611,6 @@ __device__ __forceinline__ uint32_t decode_full_slice(const uint32_t (&w)[W / 4 
         }
     }
     return X;
-}
-
-// The slice of a lane in the block's last chunk, whose slices may end at
-// the end of the stream (end < slice width) or lie past it: one code at a
-// time, one byte store per code, exactly `cnt` codes.  Returns the number of
-// codes that start in [gap, end), or cnt + 1 when there are more than cnt,
-// and the bit position after the last code counted in *after.
-template <int W>
-__device__ __forceinline__ uint32_t decode_last_slice(const uint32_t (&w)[W / 4 + 1], uint32_t gap, uint32_t cnt,
-                                                      int end, uint32_t a, uint32_t ebuf_a, uint32_t multi_a,
-                                                      uint32_t lut_a, uint32_t len_a, uint32_t &seen,
-                                                      uint32_t &after)
-{
-    constexpr int kWords = W / 4 + 1;
-    uint32_t X = gap, k = 0;
-    while ((int)X < end && k <= cnt) {
-        const uint32_t hw = min(X >> 5, (uint32_t)(kWords - 2));
-        uint32_t lo = w[0], hi = w[1];
-#pragma unroll
-        for (int i = 1; i < kWords - 1; ++i)
-            if (hw == (uint32_t)i) {
-                lo = w[i];
-                hi = w[i + 1];
-            }
-        const uint32_t win = __funnelshift_r(lo, hi, X);
-        uint2 e = lds_v2(multi_a + (win & (kMultiEntries - 1)) * kEntryBytes);
-        uint32_t sym, len;
-        if (e.y == kLongStep) {
-            e = long_code(win, lut_a, seen);
-            sym = e.x;
-            len = e.y & 0xFFFFu;
-        } else {
-            sym = e.x & 0xFFu;
-            len = lds_u8(len_a + sym);
-        }
-        if (k < cnt) {
-            asm volatile("st.shared.u8 [%0], %1;" ::"r"(ebuf_a + a + k), "r"(sym) : "memory");
-            after = X + len;
-        }
-        X += len;
-        ++k;
-    }
-    if (k == 0)
-        after = gap;
-    return k;
 }
 
 // The chunk body.  TT = 0: BF16 output; TT > 0: fused matrix-vector product
@@ -697,12 +666,37 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
         pos1 = p.chunk_pos[chunk + 1];
     }
 
-    // ---- prologue: two-level tables, sanitised ------------------------------
-    // Anything malformed (bad pointer, bad length, shorter than the shortest
-    // code) becomes "no code", so decoding never indexes outside the tables
-    // and a lane never produces more codes than its buffers hold.
-    for (uint32_t i = tid; i < n_tables * 256u; i += blockDim.x) {
-        uint32_t e = p.lut[i];
+    // ---- prologue: the tables into shared memory -----------------------------
+    // One thread copies the format's two-level tables, and the multi-code
+    // table when it was built on the host, with bulk copies (TMA) that
+    // complete on the prologue barrier; the first chunk's loads are in flight
+    // meanwhile.  Then every thread checks its share of the entries in place.
+    const uint32_t pbar = smem_addr(&mbar[kMaxWarpsPerCta]);
+    const uint32_t multi_a = smem_addr(multi);
+    const uint32_t lut_bytes = n_tables * 512u;
+    if (tid == 0) {
+        mbar_init(pbar);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        const uint32_t bytes = lut_bytes + (p.multi_src ? (uint32_t)(kMultiEntries * kEntryBytes) : 0u);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(pbar), "r"(bytes) : "memory");
+        bulk_copy_g2s_tx(smem_addr(lut), p.lut, lut_bytes, pbar);
+        if (p.multi_src)
+            bulk_copy_g2s_tx(multi_a, p.multi_src, kMultiEntries * kEntryBytes, pbar);
+    }
+    if (lane == 0)
+        mbar_init(smem_addr(&mbar[warp]));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    // (a copy that never lands leaves the tables unchecked: the CTA decodes
+    // nothing and reports a timeout)
+    const bool tables_late = __syncthreads_or(!mbar_wait(pbar, 0u)) != 0;
+    // Two-level tables, sanitised: anything malformed (bad pointer, bad
+    // length, shorter than the shortest code) becomes "no code", so decoding
+    // never indexes outside the tables and a lane never produces more codes
+    // than its buffers hold.
+    for (uint32_t i = tid; !tables_late && i < n_tables * 256u; i += blockDim.x) {
+        uint32_t e = lut[i];
         if (e & kLutPointer) {
             const uint32_t to = e & 0xFFu;
             if (i >= 256u || to == 0 || to >= n_tables || (e & 0x7F00u))
@@ -716,28 +710,23 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
         }
         lut[i] = (uint16_t)e;
     }
-    if (lane == 0)
-        mbar_init(smem_addr(&mbar[warp]));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    __syncthreads();
     // ---- prologue: multi-code table -----------------------------------------
     // Entry for an 11-bit window, stored at the window's bit-reversed value
     // (first stream bit lowest, as the decoder reads it): x = the whole codes
     // the window starts with (at most 4), as rotated exponents in bytes 0..3
-    // (unused bytes 0); y = the step total length | 8 * count << 16.  When
-    // the first code is longer than the window (or is no code) the entry is
-    // x = 0, y = kLongStep: adding it ends the lookup loop, and the decoder
-    // takes the two-level path.
+    // (unused bytes 0); y = entry_step(total length, count).  When the first
+    // code is longer than the window (or is no code) the entry is x = 0, y =
+    // kLongStep: adding it ends the lookup loop, and the decoder takes the
+    // two-level path.
     if (p.multi_src) {
-        // built once on the host (df11_build_decode_table): copied, and any
-        // entry whose count and length no table of this block could hold
-        // becomes the long-code marker, so a lane still advances at least
-        // min_len bits per code and never writes more codes than its buffer
-        // holds
-        for (int slot = tid; slot < kMultiEntries; slot += blockDim.x) {
-            uint2 v = __ldg(p.multi_src + slot);
-            // (the host table's y is length | 8 x count << 16; the long-code
-            // marker 2^31)
+        // built once on the host (df11_build_decode_table): any entry whose
+        // count and length no table of this block could hold becomes the
+        // long-code marker, so a lane still advances at least min_len bits
+        // per code and never writes more codes than its buffer holds (the
+        // host table's y is length | 8 x count << 16; its long-code marker
+        // 2^31)
+        for (int slot = tid; !tables_late && slot < kMultiEntries; slot += blockDim.x) {
+            uint2 v = multi[slot];
             const uint32_t n = v.y >> 19, t = v.y & 0xFFFFu;
             if (v.y != (t | (n << 19)) || n < 1 || n > (uint32_t)kMaxCodesPerEntry ||
                 t > (uint32_t)kWindowBits || t < n * min_len) {
@@ -749,7 +738,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             }
             multi[slot] = v;
         }
-    } else {
+    }
+    __syncthreads();
+    if (!p.multi_src && !tables_late) {
         for (int slot = tid; slot < kMultiEntries; slot += blockDim.x) {
             // consecutive threads fill consecutive entries (conflict-free stores)
             const uint32_t idx = __brev((uint32_t)slot) >> (32 - kWindowBits);
@@ -771,12 +762,11 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             }
             multi[slot] = make_uint2(syms, n ? entry_step(t, n) : kLongStep);
         }
+        __syncthreads();
     }
-    __syncthreads();
 
     // shared-window addresses (bytes)
     const uint32_t smem_base = smem_addr(smem);
-    const uint32_t multi_a = smem_base + (uint32_t)kBarBytes;
     const uint32_t len_a = multi_a + kMultiEntries * kEntryBytes;
     const uint32_t lut_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warps * G::kWarpBytes);
     const uint32_t ebuf_a = smem_base + (uint32_t)kHeadBytes + (uint32_t)(warp * G::kWarpBytes);
@@ -784,14 +774,22 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     const uint32_t bar = smem_addr(&mbar[warp]);
     uint32_t parity = 0;
 
-    if (chunk >= n_chunks)   // (never with the dynamic schedule)
+    if (tables_late) {
+        // let a late copy land before the CTA's shared memory is released
+        mbar_wait(pbar, 0u);
+        if (tid == 0 && p.err)
+            atomicOr(p.err, DF11_DEVERR_TIMEOUT);
+    }
+    // (the dynamic schedule gives every warp a chunk, and its CTAs count
+    // themselves out at the end even when they decode nothing)
+    if (chunk >= n_chunks || (tables_late && !dyn))
         return;
 
     uint32_t err = 0;
     bool stalled = false;      // a staged copy did not arrive in time
     uint32_t n_done = 0;       // chunks this warp has finished
 
-    for (;;) {
+    while (!tables_late) {
         // ---- positions (warp-uniform) and the staged sign|mantissa copy -----
         const bool pos_ok = pos0 <= pos1 && (uint64_t)pos1 <= p.out_limit &&
                             pos1 - pos0 <= (uint32_t)(32 * G::kMaxCodes);
@@ -851,10 +849,6 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
             err |= DF11_DEVERR_COUNT;
         } else {
             const uint32_t n_write = total;
-            // The lane's codes start in [gap, end): end is the slice width,
-            // or the end of the stream in the block's last chunk; the next
-            // code (the next thread's first, or the end of the stream) must
-            // start where they end.
 
             // ---- decode this lane's codes straight into place ---------------
             // Lane bytes go to ebuf[head + off, head + off + cnt).
@@ -865,25 +859,46 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                 __all_sync(0xFFFFFFFFu, DF11_CHECK(err, a + G::kMaxCodes + 8 <= (uint32_t)G::kEbufBytes));
             uint32_t seen = 0;
             bool lane_bad = false;
-            if (chunk < p.full_chunks) {
-                constexpr bool kOr = G::kSliceBits - (kWindowBits - 1) <= 64;
-                if constexpr (kOr) {
-                    // zero the words the lanes OR into (up to the next
-                    // lane's first codes after the last lane's run)
-                    const uint32_t zend = min((uint32_t)G::kEbufBytes, (head + total + 6u + 15u) & ~15u);
-                    for (uint32_t i = 16u * lane; i < zend; i += 512u)
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(ebuf_a + i), "r"(0u)
-                                     : "memory");
-                    __syncwarp();
+            // The lane's codes start in [gap, end): end is the slice width,
+            // or the end of the stream in the block's last chunk; the next
+            // code (the next thread's first, or the end of the stream) must
+            // start where they end.
+            const bool full = chunk < p.full_chunks;
+            int end = G::kSliceBits;
+            int expect = G::kSliceBits + (int)gnext;
+            if (!full) {
+                const uint64_t bit0 = ((uint64_t)chunk * 32 + lane) * (uint64_t)G::kSliceBits;
+                if (bit0 + G::kSliceBits >= p.total_bits) {
+                    end = bit0 >= p.total_bits ? 0 : (int)(p.total_bits - bit0);
+                    expect = end;
                 }
-                uint32_t sp = 0, accl = 0;
-                uint2 r = make_uint2(0u, 0u);
-                uint32_t X = 0;
-                if (write_ok)
-                    X = decode_full_slice<W>(w, gap, a, ebuf_a, multi_a, lut_a, seen, sp, accl, r);
-                // codes of the last entry that start at or past the slice
-                // end are the next lane's; the first of them (or the end of
-                // the entry) is where the next code starts
+            }
+            // 128-bit slices of a full chunk: ordered plain stores; else ORs
+            // into a zeroed buffer
+            constexpr bool kOrAlways = G::kSliceBits - (kWindowBits - 1) <= 64;
+            const bool use_or = kOrAlways || !full;
+            if (use_or) {
+                // zero the words the lanes OR into (up to the next lane's
+                // first codes after the last lane's run)
+                const uint32_t zend = min((uint32_t)G::kEbufBytes, (head + total + 6u + 15u) & ~15u);
+                for (uint32_t i = 16u * lane; i < zend; i += 512u)
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(ebuf_a + i), "r"(0u)
+                                 : "memory");
+                __syncwarp();
+            }
+            uint32_t sp = 0, accl = 0, X = 0;
+            uint2 r = make_uint2(0u, 0u);
+            if (write_ok && cnt) {
+                if (use_or)
+                    X = decode_slice<W, true>(w, gap, a, end, ebuf_a, multi_a, lut_a, seen, sp, accl, r);
+                else
+                    X = decode_slice<W, kOrAlways>(w, gap, a, G::kSliceBits, ebuf_a, multi_a, lut_a, seen, sp,
+                                                   accl, r);
+            }
+            if (cnt) {
+                // codes of the last entry that start at or past `end` are the
+                // next lane's; the first of them (or the end of the entry) is
+                // where the next code starts
                 const uint32_t emitted = sp - ebuf_a + (X >> (kFillShift + 3)) - a;
                 const uint32_t n = entry_codes(r.y);
                 int c = (int)(X & 0xFFFFu) - (int)(r.y & 0xFFFFu);   // start of the entry's first code
@@ -892,37 +907,22 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
 #pragma unroll
                 for (uint32_t k = 1; k < (uint32_t)kMaxCodesPerEntry; ++k) {
                     c += (int)lds_u8(len_a + ((r.x >> (8 * (k - 1))) & 0xFFu));
-                    if (k < n && c < G::kSliceBits)
+                    if (k < n && c < end)
                         ++keep;
                     else if (k == keep && k < n)
                         next_start = c;
                 }
-                // a full chunk's next code starts at the next slice's gap
-                // (the end of the stream when that is the slice end)
-                lane_bad = emitted - (n - keep) != cnt || next_start != G::kSliceBits + (int)gnext;
-                __syncwarp();
-                // the part-filled last word: ORed over the next lane's first
-                // word (zeros below its first byte); the last lane's is its own
-                if (write_ok && (X >> kFillShift)) {
-                    if (kOr || lane < 31)
-                        red_or_u32(sp, accl);
-                    else
-                        sts_u32(sp, accl);
-                }
-            } else {
-                // the block's last chunk: slices end at the end of the stream
-                const uint64_t bit0 = ((uint64_t)chunk * 32 + lane) * (uint64_t)G::kSliceBits;
-                int end = G::kSliceBits;
-                int expect = G::kSliceBits + (int)gnext;
-                if (bit0 + G::kSliceBits >= p.total_bits) {
-                    end = bit0 >= p.total_bits ? 0 : (int)(p.total_bits - bit0);
-                    expect = end;
-                }
-                uint32_t after = 0;
-                const uint32_t k = write_ok ? decode_last_slice<W>(w, gap, cnt, end, a, ebuf_a, multi_a, lut_a,
-                                                                   len_a, seen, after)
-                                            : cnt;
-                lane_bad = k != cnt || (cnt && (int)after != expect);
+                lane_bad = emitted - (n - keep) != cnt || next_start != expect;
+            }
+            __syncwarp();
+            // the part-filled last word: ORed over the next lane's first word
+            // (zeros below its first byte) or the zeroed buffer; a full
+            // chunk's last lane's is its own
+            if (write_ok && cnt && (X >> kFillShift)) {
+                if (use_or || lane < 31)
+                    red_or_u32(sp, accl);
+                else
+                    sts_u32(sp, accl);
             }
             if (lane_bad)
                 err |= DF11_DEVERR_COUNT;
@@ -1100,10 +1100,12 @@ struct LaunchShape {
 // Warps per CTA (as many as shared memory holds for `cps` CTAs per SM, at
 // most max_warps), shared memory, and the grid (one wave of resident CTAs
 // by default; max_ctas overrides it) for one kernel variant; sets the
-// shared-memory attribute once per device.
+// shared-memory attribute once per device.  The resident CTAs per SM are
+// queried (and cached per variant and table count) only for the variant's
+// own CTA size, `cached`; other sizes give a grid of max_ctas.
 template <int W, int MINLEN, typename Kernel>
 df11_status shape_launch(Kernel kernel, int v, const DecodeParams &prm, int dev, uint32_t max_ctas,
-                         int max_warps, int cps, LaunchShape &ls)
+                         int max_warps, int cps, LaunchShape &ls, bool cached = true)
 {
     DeviceProps d;
     if (device_props(dev, d) != DF11_OK)
@@ -1123,7 +1125,7 @@ df11_status shape_launch(Kernel kernel, int v, const DecodeParams &prm, int dev,
             return DF11_ERR_CUDA;
         g_attr_done[dev][v].store(1, std::memory_order_release);
     }
-    int occ = g_occupancy[dev][v][prm.n_tables].load(std::memory_order_relaxed);
+    int occ = cached ? g_occupancy[dev][v][prm.n_tables].load(std::memory_order_relaxed) : 1;
     if (occ == 0) {
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, warps * 32, smem) != cudaSuccess)
             return DF11_ERR_CUDA;
@@ -1151,12 +1153,31 @@ constexpr int variant_base()
 }
 
 // Launches the store kernel shaped for one or two CTAs per SM, whichever
-// keeps more warps resident (one on a tie: fewer table copies to build).
+// keeps more warps resident (one on a tie: fewer table copies to build).  A
+// block of fewer chunks than one full CTA per SM holds gets one CTA per SM
+// of just enough warps for one chunk each, so every SM shares the work
+// instead of a few full CTAs.
 template <int W, int MINLEN>
 df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32_t max_ctas)
 {
     auto k1 = df11_decode_kernel<W, MINLEN, 1>;
     auto k2 = df11_decode_kernel<W, MINLEN, 2>;
+    if (!max_ctas) {
+        DeviceProps d;
+        if (device_props(dev, d) != DF11_OK)
+            return DF11_ERR_CUDA;
+        const uint64_t sms = (uint64_t)d.sms;
+        if (prm.n_chunks < sms * (uint64_t)kCtaWarps<2>) {
+            const int warps = (int)((prm.n_chunks + sms - 1) / sms);
+            LaunchShape s1;
+            const df11_status st = shape_launch<W, MINLEN>(k1, variant_base<W, MINLEN>(), prm, dev,
+                                                           (uint32_t)sms, warps, 1, s1, false);
+            if (st == DF11_OK) {
+                k1<<<s1.grid, s1.warps * 32, s1.smem, stream>>>(prm);
+                return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+            }
+        }
+    }
     LaunchShape s1, s2;
     const df11_status st1 =
         shape_launch<W, MINLEN>(k1, variant_base<W, MINLEN>(), prm, dev, max_ctas, kCtaWarps<1>, 1, s1);
