@@ -434,15 +434,61 @@ def _rates(nbytes, n, us, peak):
             "gweights_per_s": round(n / us / 1e3, 2), "frac": round(nbytes / us / 1e3 / peak, 4)}
 
 
+def graph_us(launch, k, scrub=None, reps=5):
+    """Device time of one `launch` (microseconds), from CUDA-graph replays of
+    k back-to-back launches (median of `reps` replays) -- so a launch that
+    takes less time than the host needs to issue one is still timed by the
+    GPU's clock.  With `scrub` (a tensor larger than the L2), each launch
+    follows a write of the whole tensor: the time of a graph of k (scrub,
+    launch) pairs minus that of k scrubs alone, i.e. a launch that starts
+    from an L2 holding none of its data."""
+    import torch
+    side = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            fn()
+        return g
+
+    def run(g):
+        out = []
+        with torch.cuda.stream(side):
+            g.replay()
+            torch.cuda.synchronize()
+            for _ in range(reps):
+                a, b = _events(2)
+                a.record(side)
+                g.replay()
+                b.record(side)
+                b.synchronize()
+                out.append(a.elapsed_time(b) * 1e3 / k)
+        return statistics.median(out)
+
+    if scrub is None:
+        return run(capture(lambda: [launch(side) for _ in range(k)]))
+
+    def pairs():
+        for i in range(k):
+            scrub.fill_(i & 255)
+            launch(side)
+    t_pairs = run(capture(pairs))
+    t_scrub = run(capture(lambda: [scrub.fill_(i & 255) for i in range(k)]))
+    return t_pairs - t_scrub
+
+
 def per_config(df11, dev, stream, bpt, peak, headline=None):
     """Every configuration decoded on this GPU: bit-exactness against the
-    input, then back-to-back launches (CUDA events around a run of launches,
-    median of 5 runs) and, for single blocks, launches timed alone after a
-    256 MB write scrubs the L2 (median of 30).  Config 3 times the 32-block
-    stream (one step = 32 launches into one reused buffer); config 2 reuses
-    the headline's back-to-back figure."""
+    input, then its device time per launch from CUDA-graph replays
+    (graph_us): back to back, and for single blocks from an L2 scrubbed by a
+    256 MB write before each launch.  Config 3 times the 32-block stream
+    (one launch = the 32 blocks decoded one after another into one reused
+    buffer).  Config 2 also carries the headline's figure (direct launches,
+    median repetition under sustained load)."""
     import torch
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.zeros(df11.SCHED_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
     scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     out_all = {}
     for key, name in PER_CONFIG:
@@ -454,11 +500,11 @@ def per_config(df11, dev, stream, bpt, peak, headline=None):
             out = torch.empty(max(db.n_elements for db in dbs), dtype=torch.bfloat16, device=dev)
             cblks = [(db, db.c_struct()) for db in dbs]
 
-            def launch():
+            def launch(st):
                 for db, cb in cblks:
-                    df11.decompress_async(db, out, err, stream=stream, c_block=cb)
+                    df11.decompress_async(db, out, err, stream=st, c_block=cb, workspace=ws)
             exact = True   # numpy_model_blocks checked every block
-            reps_per_run = 2
+            k = 2
         else:
             mats = [m for _, m in workloads.WORKLOADS[name]()]
             w = np.concatenate([m.reshape(-1) for m in mats])
@@ -469,43 +515,23 @@ def per_config(df11, dev, stream, bpt, peak, headline=None):
             nbytes = hb.compressed_bytes() + 2 * n
             out = torch.empty(n, dtype=torch.int16, device=dev)
 
-            def launch():
-                df11.decompress_async(db, out, err, stream=stream, c_block=cb)
-            launch()
+            def launch(st):
+                df11.decompress_async(db, out, err, stream=st, c_block=cb, workspace=ws)
+            launch(stream)
+            torch.cuda.synchronize()
             exact = bool(torch.equal(out, torch.from_numpy(w.view(np.int16)).to(dev))) and int(err.item()) == 0
-            reps_per_run = 200 if n < 50_000_000 else 40
+            k = 100 if n < 50_000_000 else 20
             del w, hb
-        gen_s = time.perf_counter() - t0
-        for _ in range(3):
-            launch()
-        runs = []
-        for _ in range(5):
-            a, b = _events(2)
-            a.record(stream)
-            for _ in range(reps_per_run):
-                launch()
-            b.record(stream)
-            b.synchronize()
-            runs.append(a.elapsed_time(b) * 1e3 / reps_per_run)
-        b2b = statistics.median(runs)
-        entry = {"workload": name, "n_weights": n, "bytes_per_launch": nbytes,
-                 "bit_exact": exact, "setup_s": round(gen_s, 1)}
-        if name == "llama8b_block" and headline is not None:
-            b2b = headline
-        entry["back_to_back"] = _rates(nbytes, n, b2b, peak)
+        setup_s = time.perf_counter() - t0
+        entry = {"workload": name, "n_weights": n, "bytes_per_launch": nbytes, "bit_exact": exact,
+                 "setup_s": round(setup_s, 1)}
+        entry["back_to_back"] = _rates(nbytes, n, graph_us(launch, k), peak)
         if name != "llama8b_model":
-            alone = []
-            for i in range(30):
-                scrub.fill_(i & 255)
-                a, b = _events(2)
-                a.record(stream)
-                launch()
-                b.record(stream)
-                b.synchronize()
-                alone.append(a.elapsed_time(b) * 1e3)
-            entry["l2_scrubbed"] = _rates(nbytes, n, statistics.median(alone), peak)
+            entry["l2_scrubbed"] = _rates(nbytes, n, graph_us(launch, max(k // 4, 5), scrub=scrub), peak)
         else:
             entry["what"] = "one launch = the 32 blocks decoded one after another (us per 32 blocks)"
+        if name == "llama8b_block" and headline is not None:
+            entry["headline_direct_launches"] = _rates(nbytes, n, headline, peak)
         if int(err.item()):
             entry["bit_exact"] = False
         out_all[key] = entry
