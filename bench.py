@@ -478,6 +478,48 @@ def graph_us(launch, k, scrub=None, reps=5):
     return t_pairs - t_scrub
 
 
+def integrity_figures(df11, dev, stream, hb, db, cb, out, w_dev, ws, scrub, launch, k, peak):
+    """The integrity checks on one block, graph-timed like the decode: the
+    decode that checks every chunk's sum as it decodes (one launch), the
+    CRC-32C list check alone, and the CRC check followed by the plain
+    decode (two launches, the block read twice)."""
+    import torch
+    nbytes = hb.compressed_bytes() + 2 * hb.n_elements
+    n = hb.n_elements
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    first = torch.full((1,), -1, dtype=torch.int64, device=dev)
+    sums = torch.from_numpy(df11.chunk_sums(hb).view(np.int32)).to(dev)
+    crcs = torch.from_numpy(df11.checksum(hb).view(np.int32)).to(dev)
+
+    def verified(st):
+        df11.decompress_verified_async(db, out, sums, err, first, stream=st, c_block=cb, workspace=ws)
+
+    def crc_only(st):
+        df11.verify_device(db, crcs, err, first, stream=st)
+
+    def crc_then_decode(st):
+        crc_only(st)
+        launch(st)
+    out.zero_()
+    verified(stream)
+    crc_only(stream)
+    torch.cuda.synchronize()
+    clean = int(err.item()) == 0 and int(first.item()) == -1
+    res = {"bit_exact": bool(torch.equal(out, w_dev)), "clean_block_passes": clean,
+           "chunk_sums_bytes": 4 * int(hb.header.n_chunks)}
+    res["verified_decode"] = {"back_to_back": _rates(nbytes, n, graph_us(verified, k), peak),
+                              "l2_scrubbed": _rates(nbytes, n, graph_us(verified, max(k // 4, 5), scrub=scrub),
+                                                    peak)}
+    crc_bytes = hb.compressed_bytes()
+    us = graph_us(crc_only, k)
+    res["crc_check_alone"] = {"us": round(us, 2), "gb_per_s": round(crc_bytes / us / 1e3, 1),
+                              "frac_of_peak": round(crc_bytes / us / 1e3 / peak, 4)}
+    res["crc_check_then_decode"] = {"back_to_back": _rates(nbytes, n, graph_us(crc_then_decode, k), peak)}
+    if int(err.item()) or int(first.item()) != -1:
+        res["clean_block_passes"] = False
+    return res
+
+
 def per_config(df11, dev, stream, bpt, peak, headline=None):
     """Every configuration decoded on this GPU: bit-exactness against the
     input, then its device time per launch from CUDA-graph replays
@@ -519,9 +561,12 @@ def per_config(df11, dev, stream, bpt, peak, headline=None):
                 df11.decompress_async(db, out, err, stream=st, c_block=cb, workspace=ws)
             launch(stream)
             torch.cuda.synchronize()
-            exact = bool(torch.equal(out, torch.from_numpy(w.view(np.int16)).to(dev))) and int(err.item()) == 0
+            w_dev = torch.from_numpy(w.view(np.int16)).to(dev)
+            exact = bool(torch.equal(out, w_dev)) and int(err.item()) == 0
             k = 100 if n < 50_000_000 else 20
-            del w, hb
+            if name == "llama8b_block":
+                integrity = integrity_figures(df11, dev, stream, hb, db, cb, out, w_dev, ws, scrub, launch, k, peak)
+            del w, hb, w_dev
         setup_s = time.perf_counter() - t0
         entry = {"workload": name, "n_weights": n, "bytes_per_launch": nbytes, "bit_exact": exact,
                  "setup_s": round(setup_s, 1)}
@@ -532,6 +577,9 @@ def per_config(df11, dev, stream, bpt, peak, headline=None):
             entry["what"] = "one launch = the 32 blocks decoded one after another (us per 32 blocks)"
         if name == "llama8b_block" and headline is not None:
             entry["headline_direct_launches"] = _rates(nbytes, n, headline, peak)
+        if name == "llama8b_block":
+            entry["integrity"] = integrity
+            integrity = None
         if int(err.item()):
             entry["bit_exact"] = False
         out_all[key] = entry

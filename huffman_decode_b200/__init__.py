@@ -11,7 +11,7 @@ from .df11 import (  # noqa: F401
     DeviceBlock, EXPORTED_SYMBOLS, LAYOUTS, HostBlock, PinnedHostBlock, Pipeline, build_codebook,
     decode_gemv_async, SCHED_WORKSPACE_BYTES, sched_workspace, decompress_range_async,
     selftest_bounded_wait,
-    build_codebook_from_histogram, build_decode_table, compress, compress_device, compress_device_noalloc,
+    build_codebook_from_histogram, build_decode_table, chunk_sums, decompress_verified_async, compress, compress_device, compress_device_noalloc,
     compress_device_scratch_bytes,
     compress_sizes, decompress_async, histogram_device, library_path, load_library, validate,
 )

@@ -347,3 +347,77 @@ extern "C" df11_status df11_verify_device_async(const df11_device_block *blk, co
         return DF11_ERR_INVALID_ARGUMENT;
     return launch_crc(blk, nullptr, d_expected, n_crc, d_error, d_first_bad, stream);
 }
+
+// ---- per-chunk sums (host) ---------------------------------------------------
+// The same sums the decode kernel's verifying path computes (include/df11.h):
+// the chunk's stream words (bit-reversed big-endian words), the threads'
+// gap and count, the two positions, the sign|mantissa bytes (whole 8-element
+// groups as two words, the rest byte by byte), and in chunk 0 the tables.
+
+namespace {
+
+inline uint32_t chunk_mix(uint32_t v, uint32_t tag)
+{
+    const uint32_t y = (v ^ (tag * 0x9E3779B1u)) * 0x85EBCA6Bu;
+    return y ^ (y >> 16);
+}
+
+inline uint32_t brev32(uint32_t x)
+{
+    x = ((x >> 1) & 0x55555555u) | ((x & 0x55555555u) << 1);
+    x = ((x >> 2) & 0x33333333u) | ((x & 0x33333333u) << 2);
+    x = ((x >> 4) & 0x0F0F0F0Fu) | ((x & 0x0F0F0F0Fu) << 4);
+    return __builtin_bswap32(x);   // bytes reversed too: the whole word bit-reversed
+}
+
+inline uint32_t le32(const uint8_t *p)
+{
+    uint32_t v;
+    std::memcpy(&v, p, 4);
+    return v;
+}
+
+}  // namespace
+
+extern "C" df11_status df11_chunk_sums(const df11_host_block *blk, uint32_t *sums, uint64_t n)
+{
+    if (!blk || !sums || !blk->exp_stream || !blk->gaps || !blk->counts || !blk->chunk_pos ||
+        !blk->signmant || !blk->lut || n != blk->hdr.n_chunks || blk->hdr.threads_per_chunk != 32 ||
+        (blk->hdr.bytes_per_thread != 8 && blk->hdr.bytes_per_thread != 16))
+        return DF11_ERR_INVALID_ARGUMENT;
+    const uint64_t W = blk->hdr.bytes_per_thread;
+    if (blk->exp_stream_bytes < 32 * W * n || blk->gaps_bytes < 16 * n || blk->counts_bytes < 32 * n ||
+        blk->chunk_pos_count < n + 1 || blk->lut_entries < 256ull * blk->hdr.n_tables)
+        return DF11_ERR_INVALID_ARGUMENT;
+    for (uint64_t c = 0; c < n; ++c) {
+        uint32_t sum = 0;
+        const uint8_t *st = blk->exp_stream + 32 * W * c;
+        for (uint32_t k = 0; k < 8 * W; ++k)   // stream bit 32k + i at bit i: bit-reversed big-endian word
+            sum += chunk_mix(brev32(__builtin_bswap32(le32(st + 4 * k))), k);
+        for (uint32_t t = 0; t < 32; ++t) {
+            const uint64_t g = 32 * c + t;
+            const uint32_t gap = (blk->gaps[g >> 1] >> ((g & 1) * 4)) & 0xFu;
+            sum += chunk_mix(gap | ((uint32_t)blk->counts[g] << 8), 0x10000u + t);
+        }
+        const uint64_t p0 = blk->chunk_pos[c], p1 = blk->chunk_pos[c + 1];
+        if (p1 < p0 || p1 > blk->signmant_bytes)
+            return DF11_ERR_INVALID_ARGUMENT;
+        sum += chunk_mix((uint32_t)p0, 0x20000u) + chunk_mix((uint32_t)p1, 0x20001u);
+        const uint64_t b = p0 & ~7ull;
+        const uint64_t g_first = (p0 + 7) >> 3, g_end = p1 >> 3;   // whole groups [g_first, g_end)
+        for (uint64_t q = g_first; q < g_end; ++q) {
+            const uint32_t r = (uint32_t)(q - (b >> 3));
+            sum += chunk_mix(le32(blk->signmant + 8 * q), 0x100000u + 2 * r) +
+                   chunk_mix(le32(blk->signmant + 8 * q + 4), 0x100000u + 2 * r + 1);
+        }
+        const uint64_t whole_lo = g_first < g_end ? 8 * g_first : p1, whole_hi = g_first < g_end ? 8 * g_end : p1;
+        for (uint64_t e = p0; e < p1; ++e)
+            if (e < whole_lo || e >= whole_hi)
+                sum += chunk_mix(blk->signmant[e], (uint32_t)(0x200000u + (e - b)));
+        if (c == 0)
+            for (uint32_t i = 0; i < 128u * blk->hdr.n_tables; ++i)
+                sum += chunk_mix(blk->lut[2 * i] | ((uint32_t)blk->lut[2 * i + 1] << 16), 0x400000u + i);
+        sums[c] = sum;
+    }
+    return DF11_OK;
+}

@@ -97,6 +97,8 @@ struct DecodeParams {
     uint64_t gaps_limit;  // gap bytes readable from `gaps` (the next thread's gap after the last chunk)
     uint32_t *sched;      // scheduling workspace, zero between launches; or null
     const uint2 *multi_src;   // the multi-code table built on the host, or null
+    const uint32_t *sums;     // verifying decode: the expected per-chunk sums
+    uint64_t *first_bad;      // verifying decode: lowest chunk found bad, or null
 };
 // Scheduling workspace: claim counter q at word q * kSchedStride (pools on
 // separate 256-byte stretches, so on different L2 lines), CTAs done at word
@@ -197,6 +199,15 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
+
+// One item of a chunk's integrity sum (the definition is in df11.h):
+// mix(v, tag) with tag_mul = tag * 0x9E3779B1 precomputed.
+__device__ __forceinline__ uint32_t chunk_mix(uint32_t v, uint32_t tag_mul)
+{
+    const uint32_t y = (v ^ tag_mul) * 0x85EBCA6Bu;
+    return y ^ (y >> 16);
+}
+constexpr uint32_t kTagMul = 0x9E3779B1u;
 
 // ---- 32-bit shared-window accesses -----------------------------------------
 // The hot loops address shared memory with 32-bit shared-window offsets.
@@ -614,10 +625,12 @@ __device__ __forceinline__ uint32_t decode_slice(const uint32_t (&w)[W / 4 + 1],
 }
 
 // The chunk body.  TT = 0: BF16 output; TT > 0: fused matrix-vector product
-// for up to TT tokens (gp != nullptr).
-template <int W, int MINLEN, int TT>
+// for up to TT tokens (gp != nullptr).  VER: also sum every chunk's bytes as
+// they are read and compare with p.sums (BF16 output only).
+template <int W, int MINLEN, int TT, bool VER = false>
 __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvParams *gp)
 {
+    static_assert(!VER || TT == 0, "the verifying decode writes BF16");
     using G = Geometry<W, MINLEN>;
     extern __shared__ __align__(16) uint8_t smem[];
     const int warps = blockDim.x >> 5;
@@ -788,6 +801,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     uint32_t err = 0;
     bool stalled = false;      // a staged copy did not arrive in time
     uint32_t n_done = 0;       // chunks this warp has finished
+    // (verifying) kReported in err: this warp has reported a bad chunk
+    constexpr uint32_t kReported = 0x80000000u;
 
     while (!tables_late) {
         // ---- positions (warp-uniform) and the staged sign|mantissa copy -----
@@ -830,6 +845,21 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
         // thread metadata: gap, count and the next thread's gap
         const uint32_t gap = meta & 0xFu;
         const uint32_t cnt = meta >> 8;
+        // (verifying) the lane's items of the chunk sum: its stream words,
+        // its gap and count, and on lane 0 the two positions
+        // The lanes' sums add up to zero for an intact chunk: lane 0 starts
+        // from minus the expected sum.
+        uint32_t vsum = 0;
+        if constexpr (VER) {
+#pragma unroll
+            for (int j = 0; j < W / 4; ++j)
+                vsum += chunk_mix(w[j], (uint32_t)((W / 4) * lane + j) * kTagMul);
+            vsum += chunk_mix(gap | (cnt << 8), (0x10000u + (uint32_t)lane) * kTagMul);
+            if (lane == 0)
+                vsum += chunk_mix(pos0, 0x20000u * kTagMul) + chunk_mix(pos1, 0x20001u * kTagMul) -
+                        p.sums[chunk];
+
+        }
         const uint32_t gap_up = __shfl_down_sync(0xFFFFFFFFu, gap, 1);
         const uint32_t gnext = lane == 31 ? (meta >> 4) & 0xFu : gap_up;
         // ---- warp scan of the stored counts: each lane's output offset -----
@@ -959,6 +989,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                     const uint2 x = join4(e8.x, s8.x);
                     const uint2 y = join4(e8.y, s8.y);
                     out16[i] = make_uint4(x.x, x.y, y.x, y.y);
+                    if constexpr (VER) {
+                        const uint32_t t = (0x100000u + 2u * i) * kTagMul;
+                        vsum += chunk_mix(s8.x, t) + chunk_mix(s8.y, t + kTagMul);
+                    }
                 }
                 const uint32_t fs = gfirst * 8;                    // first whole-group element
                 const uint32_t hend = min(fs, span);               // head part: [head, hend)
@@ -971,14 +1005,39 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                     if (tbeg + (lane - 8) < span)
                         l = tbeg + (lane - 8);
                 }
-                if (l != 0xFFFFFFFFu)
-                    p.out[base + l] = join1(lds_u8_m(ebuf_a + l), lds_u8_m(sgrp_a + l));
+                if (l != 0xFFFFFFFFu) {
+                    const uint32_t sm = lds_u8_m(sgrp_a + l);
+                    p.out[base + l] = join1(lds_u8_m(ebuf_a + l), sm);
+                    if constexpr (VER)
+                        vsum += chunk_mix(sm, (0x200000u + l) * kTagMul);
+                }
+            }
+            if constexpr (VER) {
+                if (chunk == 0) {
+                    // chunk 0 also covers the tables, read as they are stored
+                    const uint32_t *lw = reinterpret_cast<const uint32_t *>(p.lut);
+                    for (uint32_t i = (uint32_t)lane; i < 128u * n_tables; i += 32u)
+                        vsum += chunk_mix(lw[i], (0x400000u + i) * kTagMul);
+                }
+                // (all lanes: a merge that did not run leaves the sum short)
+                if (__reduce_add_sync(0xFFFFFFFFu, vsum) != 0u)
+                    err |= DF11_DEVERR_CHECKSUM;
             }
             if constexpr (TT > 0) {
                 if (!stalled && merge_ok)
                     gemv_chunk<TT>(gp, head, n_write, base, lane, ebuf_a, sbuf_a + (pos0 & 8u));
             }
             __syncwarp();
+        }
+        if constexpr (VER) {
+            // a chunk is bad when its sum differs or its decode failed (the
+            // warp's flags only grow and its chunks come in increasing order,
+            // so reporting its first bad chunk gives the minimum)
+            if (!(err & kReported) && __any_sync(0xFFFFFFFFu, err != 0)) {
+                err |= kReported;
+                if (lane == 0 && p.first_bad)
+                    atomicMin(reinterpret_cast<unsigned long long *>(p.first_bad), (unsigned long long)chunk);
+            }
         }
 
         ++n_done;
@@ -994,6 +1053,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
     }
     if (stalled)   // let the late copy land before this CTA's shared memory is released
         mbar_wait(bar, parity ^ 1u);
+    if constexpr (VER)
+        err &= ~kReported;
     if (err && p.err)
         atomicOr(p.err, err);
     if (dyn) {
@@ -1035,13 +1096,15 @@ __global__ void bounded_wait_kernel(uint32_t polls, uint32_t *status)
 // (11.5 warps per SM sub-partition), and two 23-warp CTAs fill the SM's
 // shared memory with 46 warps instead of 32.  Each CTA holds its own copy
 // of the tables.
-template <int CPS>
-constexpr int kCtaWarps = CPS == 1 ? kMaxWarpsPerCta : 23;
+// (The verifying decode keeps two more values per lane: 20 warps, 48
+// registers.)
+template <int CPS, bool VER = false>
+constexpr int kCtaWarps = CPS == 1 ? kMaxWarpsPerCta : VER ? 23 : 23;
 
-template <int W, int MINLEN, int CPS>
-__global__ void __launch_bounds__(kCtaWarps<CPS> * 32, CPS) df11_decode_kernel(DecodeParams p)
+template <int W, int MINLEN, int CPS, bool VER = false>
+__global__ void __launch_bounds__(kCtaWarps<CPS, VER> * 32, CPS) df11_decode_kernel(DecodeParams p)
 {
-    decode_body<W, MINLEN, 0>(p, nullptr);
+    decode_body<W, MINLEN, 0, VER>(p, nullptr);
 }
 
 template <int W, int MINLEN, int TT>
@@ -1055,8 +1118,9 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_gemv_kernel(DecodeP
 
 constexpr int kMaxDevices = 64;
 // kernel variants: (slice width, shortest code) x (store with one CTA per
-// SM, products for 1, 2, 4, 8 tokens, store with two CTAs per SM)
-constexpr int kVariantsPerLayout = 6;
+// SM, products for 1, 2, 4, 8 tokens, store with two CTAs per SM, the
+// verifying store with one and with two CTAs per SM)
+constexpr int kVariantsPerLayout = 8;
 constexpr int kVariants = 4 * kVariantsPerLayout;
 // resident CTAs per SM, by device, kernel variant and table count
 std::atomic<int> g_occupancy[kMaxDevices][kVariants][257];
@@ -1157,21 +1221,22 @@ constexpr int variant_base()
 // block of fewer chunks than one full CTA per SM holds gets one CTA per SM
 // of just enough warps for one chunk each, so every SM shares the work
 // instead of a few full CTAs.
-template <int W, int MINLEN>
+template <int W, int MINLEN, bool VER = false>
 df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32_t max_ctas)
 {
-    auto k1 = df11_decode_kernel<W, MINLEN, 1>;
-    auto k2 = df11_decode_kernel<W, MINLEN, 2>;
+    auto k1 = df11_decode_kernel<W, MINLEN, 1, VER>;
+    auto k2 = df11_decode_kernel<W, MINLEN, 2, VER>;
+    const int v1 = variant_base<W, MINLEN>() + (VER ? 6 : 0), v2 = variant_base<W, MINLEN>() + (VER ? 7 : 5);
     if (!max_ctas) {
         DeviceProps d;
         if (device_props(dev, d) != DF11_OK)
             return DF11_ERR_CUDA;
         const uint64_t sms = (uint64_t)d.sms;
-        if (prm.n_chunks < sms * (uint64_t)kCtaWarps<2>) {
+        if (prm.n_chunks < sms * (uint64_t)kCtaWarps<2, VER>) {
             const int warps = (int)((prm.n_chunks + sms - 1) / sms);
             LaunchShape s1;
-            const df11_status st = shape_launch<W, MINLEN>(k1, variant_base<W, MINLEN>(), prm, dev,
-                                                           (uint32_t)sms, warps, 1, s1, false);
+            const df11_status st =
+                shape_launch<W, MINLEN>(k1, v1, prm, dev, (uint32_t)sms, warps, 1, s1, false);
             if (st == DF11_OK) {
                 k1<<<s1.grid, s1.warps * 32, s1.smem, stream>>>(prm);
                 return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
@@ -1179,10 +1244,8 @@ df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32
         }
     }
     LaunchShape s1, s2;
-    const df11_status st1 =
-        shape_launch<W, MINLEN>(k1, variant_base<W, MINLEN>(), prm, dev, max_ctas, kCtaWarps<1>, 1, s1);
-    const df11_status st2 =
-        shape_launch<W, MINLEN>(k2, variant_base<W, MINLEN>() + 5, prm, dev, max_ctas, kCtaWarps<2>, 2, s2);
+    const df11_status st1 = shape_launch<W, MINLEN>(k1, v1, prm, dev, max_ctas, kCtaWarps<1, VER>, 1, s1);
+    const df11_status st2 = shape_launch<W, MINLEN>(k2, v2, prm, dev, max_ctas, kCtaWarps<2, VER>, 2, s2);
     if (st1 != DF11_OK && st2 != DF11_OK)
         return st1;
     if (st2 == DF11_OK && (st1 != DF11_OK || s2.resident_warps > s1.resident_warps))
@@ -1280,6 +1343,8 @@ df11_status block_params(const df11_device_block *blk, uint16_t *out_bf16, uint6
     prm.full_chunks = (uint32_t)(h.total_bits / chunk_bits);
     prm.sched = nullptr;
     prm.multi_src = reinterpret_cast<const uint2 *>(blk->decode_table);
+    prm.sums = nullptr;
+    prm.first_bad = nullptr;
     return DF11_OK;
 }
 
@@ -1394,4 +1459,26 @@ extern "C" df11_status df11_decode_gemv_async(const df11_device_block *blk, cons
     if (blk->hdr.bytes_per_thread == 8)
         return prm.min_len >= 2 ? launch_gemv_tokens<8, 2>(prm, gp, dev, s) : launch_gemv_tokens<8, 1>(prm, gp, dev, s);
     return prm.min_len >= 2 ? launch_gemv_tokens<16, 2>(prm, gp, dev, s) : launch_gemv_tokens<16, 1>(prm, gp, dev, s);
+}
+
+extern "C" df11_status df11_decompress_verified_async(const df11_device_block *blk, uint16_t *out_bf16,
+                                                      uint64_t out_capacity, uint32_t *d_error,
+                                                      const uint32_t *d_sums, uint64_t *d_first_bad,
+                                                      void *workspace, void *stream)
+{
+    if (!out_bf16 || !d_error || !d_sums || !aligned(d_sums, 4) || !aligned(d_first_bad, 8) ||
+        !aligned(workspace, 16))
+        return DF11_ERR_INVALID_ARGUMENT;
+    DecodeParams prm;
+    int dev = 0;
+    const df11_status st = block_params(blk, out_bf16, out_capacity, d_error, prm, dev);
+    if (st != DF11_OK)
+        return st;
+    prm.sched = static_cast<uint32_t *>(workspace);
+    prm.sums = d_sums;
+    prm.first_bad = d_first_bad;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (blk->hdr.bytes_per_thread == 8)
+        return prm.min_len >= 2 ? launch<8, 2, true>(prm, dev, s, 0) : launch<8, 1, true>(prm, dev, s, 0);
+    return prm.min_len >= 2 ? launch<16, 2, true>(prm, dev, s, 0) : launch<16, 1, true>(prm, dev, s, 0);
 }

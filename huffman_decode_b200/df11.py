@@ -54,7 +54,7 @@ EXPORTED_SYMBOLS = (
     "df11_checksum_device_async", "df11_verify_device_async", "df11_pipeline_verify",
     "df11_decode_gemv_async", "df11_decompress_async_ws", "df11_decompress_range_async",
     "df11_selftest_bounded_wait", "df11_serialized_bytes", "df11_serialize", "df11_deserialize",
-    "df11_build_decode_table",
+    "df11_build_decode_table", "df11_chunk_sums", "df11_decompress_verified_async",
 )
 SCHED_WORKSPACE_BYTES = 2048
 CRC_SEGMENT_BYTES = 4096
@@ -189,6 +189,8 @@ def load_library(path: str | None = None):
         ("df11_serialize", S, [P, P, U64]),
         ("df11_deserialize", S, [P, U64, P, P]),
         ("df11_build_decode_table", S, [P, U32, U32, P]),
+        ("df11_chunk_sums", S, [P, P, U64]),
+        ("df11_decompress_verified_async", S, [P, P, U64, P, P, P, P, P]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -801,6 +803,38 @@ def verify_device(db: "DeviceBlock", expected, error, first_bad=None, stream=Non
                                                    expected.numel(), error.data_ptr(), fb,
                                                    _raw_stream(stream, error.device)),
            "df11_verify_device_async")
+
+
+def chunk_sums(hb: HostBlock) -> np.ndarray:
+    """df11_chunk_sums: the block's per-chunk integrity sums (uint32, one per
+    chunk), computed on the host."""
+    n = int(hb.header.n_chunks)
+    out = np.empty(n, np.uint32)
+    b = hb.c_struct()
+    _check(load_library().df11_chunk_sums(ctypes.byref(b), out.ctypes.data, n), "df11_chunk_sums")
+    return out
+
+
+def decompress_verified_async(db: "DeviceBlock", out, sums, error, first_bad=None, stream=None,
+                              c_block=None, workspace=True) -> None:
+    """df11_decompress_verified_async: decodes the whole block into `out` as
+    decompress_async does and checks every chunk's sum against `sums` (int32
+    CUDA tensor of the chunk_sums values' bit patterns); a mismatch ORs
+    DEVERR_CHECKSUM into `error` (int32 CUDA tensor), and `first_bad` (int64
+    CUDA tensor preset to -1, i.e. UINT64_MAX) receives the lowest chunk whose
+    sum differs or whose decode failed."""
+    if out.element_size() != 2 or not out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CUDA tensor of 16-bit elements")
+    if sums.element_size() != 4 or not sums.is_cuda or sums.numel() < db.header.n_chunks:
+        raise ValueError("sums must be a CUDA tensor of n_chunks 32-bit values")
+    handle = _raw_stream(stream, out.device)
+    blk = c_block if c_block is not None else db.c_struct()
+    fb = first_bad.data_ptr() if first_bad is not None else None
+    _check(load_library().df11_decompress_verified_async(ctypes.byref(blk), out.data_ptr(), out.numel(),
+                                                         error.data_ptr(), sums.data_ptr(), fb,
+                                                         _workspace_ptr(workspace, out.device, handle),
+                                                         handle),
+           "df11_decompress_verified_async")
 
 
 # ------------------------------------------------ decode fused with products

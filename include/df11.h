@@ -96,7 +96,9 @@ typedef enum {
 #define DF11_DEVERR_MISMATCH 0x10u /* GPU compressor: an exponent without a code,
                                      or a bit total other than the codebook's  */
 #define DF11_DEVERR_CHECKSUM 0x20u /* df11_verify_device_async: a segment's
-                                     CRC-32C differs from the expected value   */
+                                     CRC-32C differs from the expected value;
+                                     df11_decompress_verified_async: a chunk's
+                                     sum differs                              */
 #define DF11_DEVERR_BOUNDS 0x40u   /* checked build (libdf11_checked.so) only: an
                                      invariant that keeps an access in bounds
                                      failed; the access was skipped            */
@@ -480,6 +482,49 @@ df11_status df11_checksum_device_async(const df11_device_block *blk, uint32_t *d
 df11_status df11_verify_device_async(const df11_device_block *blk, const uint32_t *d_expected,
                                      uint64_t n_crc, uint32_t *d_error, uint64_t *d_first_bad,
                                      void *stream);
+
+/* ---- Integrity inside the decode: per-chunk sums -------------------------
+ * A checksum the decode kernel can check as it decodes, from the bytes it
+ * reads anyway (this library's addition; the pages ask only to checksum
+ * artifacts, "How to run it in production").  One 32-bit sum per chunk c
+ * (threads 32c .. 32c + 31, B = 8 * bytes_per_thread bits per slice): the
+ * sum mod 2^32 of mix(v, tag) over
+ *   - the chunk's 32 B stream bits as B words: bit i of word k is chunk
+ *     stream bit 32k + i (MSB-first within bytes); tag k;
+ *   - each thread t = 0..31: v = gap | count << 8; tag 0x10000 + t;
+ *   - v = chunk_pos[c] (tag 0x20000) and chunk_pos[c + 1] (tag 0x20001);
+ *   - the sign|mantissa bytes of elements [p0, p1) = [chunk_pos[c],
+ *     chunk_pos[c + 1]), b = p0 rounded down to a multiple of 8: each group
+ *     [8q, 8q + 8) inside [p0, p1) as two little-endian words, tags 0x100000
+ *     + 2r and 0x100000 + 2r + 1 (r = q - b / 8); every other element e as its
+ *     byte, tag 0x200000 + e - b;
+ *   - chunk 0 only: the tables as little-endian words (entries 2i, 2i + 1),
+ *     tag 0x400000 + i;
+ * mix(v, tag) = y ^ (y >> 16) with y = (v ^ tag * 0x9E3779B1) * 0x85EBCA6B,
+ * all mod 2^32 -- for a fixed tag a bijection of v, so a change in any one
+ * item changes the sum.  Unlike the CRC-32C list it can be checked by the
+ * decode itself at a small cost (about five instructions per 4 bytes), and
+ * it points at the damaged chunk.  The decoder's multi-code table is not
+ * covered (it is derived from the tables). */
+
+/* Host.  Writes the n_chunks per-chunk sums of blk into sums[0 .. n).
+ * INVALID_ARGUMENT for null pointers or n != blk->hdr.n_chunks. */
+df11_status df11_chunk_sums(const df11_host_block *blk, uint32_t *sums, uint64_t n);
+
+/* GPU.  df11_decompress_range_async over the whole block (chunk_begin = 0,
+ * chunk_end = n_chunks) that also computes every chunk's sum as it decodes
+ * and compares it with d_sums[c] (device, n_chunks values of
+ * df11_chunk_sums): a mismatch ORs DF11_DEVERR_CHECKSUM into *d_error.  A
+ * chunk is bad when its sum differs or its decode reports an error (its
+ * flag); when d_first_bad (device uint64, 8-byte aligned, set to UINT64_MAX
+ * by the caller) is given, it is lowered to the lowest bad chunk.  Chunks of
+ * a CTA whose tables never arrived are neither decoded nor summed (that
+ * sets DF11_DEVERR_TIMEOUT).  The output is written as by
+ * df11_decompress_async.  Errors: those of df11_decompress_async_ws, and
+ * INVALID_ARGUMENT for null or misaligned d_sums, d_error or d_first_bad. */
+df11_status df11_decompress_verified_async(const df11_device_block *blk, uint16_t *out_bf16,
+                                           uint64_t out_capacity, uint32_t *d_error, const uint32_t *d_sums,
+                                           uint64_t *d_first_bad, void *workspace, void *stream);
 
 /* ---- Streamed decoding: upload -> decode -> consume ----------------------
  * The pages decode each transformer block right before its matrix products

@@ -66,6 +66,7 @@ def _load():
         "orc_decode": (I, [P, U64, U64, U64, P, P, P]),
         "orc_first_code_table": (I, [P, P, P]),
         "orc_metadata": (I, [P, U64, P, U32, U32, U64, P, P, P]),
+        "orc_chunk_sums": (I, [P, P, P, P, P, U64, P, U32, U32, U64, P]),
         "orc_crc32c": (U32, [P, U64]),
         "orc_segment_crcs": (U64, [P, U64, U64, P]),
     }
@@ -292,3 +293,23 @@ def block_checksums(exp_stream, gaps, counts, chunk_pos, signmant, lut, seg: int
     order exp_stream, gaps, counts, chunk_pos, signmant, lut (raw
     little-endian bytes of each array as given)."""
     return np.concatenate([segment_crcs(a, seg) for a in (exp_stream, gaps, counts, chunk_pos, signmant, lut)])
+
+
+# ----------------------------------------------------------- chunk sums
+
+def chunk_sums(stream, gaps, counts, chunk_pos, signmant, lut, n_tables: int, bytes_per_thread: int,
+               n_chunks: int) -> np.ndarray:
+    """The per-chunk sums of a block (see orc_chunk_sums in df11_oracle.h):
+    gaps packed two per byte, counts one byte per thread, chunk_pos uint32."""
+    stream, gaps, counts, signmant = _u8(stream), _u8(gaps), _u8(counts), _u8(signmant)
+    pos = np.ascontiguousarray(chunk_pos, dtype=np.uint32)
+    lut = np.ascontiguousarray(lut, dtype=np.uint16)
+    out = np.zeros(max(int(n_chunks), 1), np.uint32)
+    if pos.size < int(n_chunks) + 1 or stream.size < 32 * int(bytes_per_thread) * int(n_chunks) or \
+            gaps.size < 16 * int(n_chunks) or counts.size < 32 * int(n_chunks) or lut.size < 256 * int(n_tables):
+        raise ValueError("chunk_sums: arrays shorter than the block")
+    rc = _load().orc_chunk_sums(_ptr(stream), _ptr(gaps), _ptr(counts), _ptr(pos), _ptr(signmant), signmant.size,
+                                _ptr(lut), int(n_tables), int(bytes_per_thread), int(n_chunks), _ptr(out))
+    if rc != 0:
+        raise ValueError("chunk_sums failed")
+    return out[: int(n_chunks)]

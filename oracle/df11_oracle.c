@@ -500,3 +500,71 @@ uint64_t orc_segment_crcs(const uint8_t *data, uint64_t n, uint64_t seg, uint32_
         out[k] = orc_crc32c(data + off, n - off < seg ? n - off : seg);
     return k;
 }
+
+/* ----------------------------------------------------------- chunk sums */
+
+static uint32_t orc_mix(uint32_t v, uint32_t tag)
+{
+    uint32_t x = v ^ (uint32_t)(tag * 0x9E3779B1u);
+    uint32_t y = x * 0x85EBCA6Bu;
+    return y ^ (y >> 16);
+}
+
+int orc_chunk_sums(const uint8_t *stream, const uint8_t *gaps, const uint8_t *counts, const uint32_t *pos,
+                   const uint8_t *signmant, uint64_t signmant_bytes, const uint16_t *lut, uint32_t n_tables,
+                   uint32_t bytes_per_thread, uint64_t n_chunks, uint32_t *out)
+{
+    if (bytes_per_thread == 0 || n_tables == 0)
+        return -1;
+    for (uint64_t c = 0; c < n_chunks; ++c)
+        if (pos[c] > pos[c + 1] || pos[c + 1] > signmant_bytes)
+            return -1;
+    const uint64_t slice_bits = 8ull * bytes_per_thread;
+    const uint64_t chunk_bytes = 32ull * bytes_per_thread;
+    for (uint64_t c = 0; c < n_chunks; ++c) {
+        uint32_t sum = 0;
+        /* stream words, bit by bit */
+        for (uint64_t k = 0; k < slice_bits; ++k) {
+            uint32_t v = 0;
+            for (uint32_t i = 0; i < 32; ++i) {
+                uint64_t j = 32 * k + i;
+                uint8_t byte = stream[chunk_bytes * c + j / 8];
+                uint32_t bit = (byte >> (7 - j % 8)) & 1u;
+                v |= bit << i;
+            }
+            sum += orc_mix(v, (uint32_t)k);
+        }
+        /* thread words */
+        for (uint32_t t = 0; t < 32; ++t) {
+            uint64_t g = 32 * c + t;
+            uint32_t gap = (gaps[g / 2] >> (4 * (g % 2))) & 15u;
+            sum += orc_mix(gap | ((uint32_t)counts[g] << 8), 0x10000u + t);
+        }
+        /* positions */
+        uint64_t p0 = pos[c], p1 = pos[c + 1];
+        sum += orc_mix((uint32_t)p0, 0x20000u);
+        sum += orc_mix((uint32_t)p1, 0x20001u);
+        /* sign|mantissa bytes */
+        uint64_t b = p0 - p0 % 8;
+        for (uint64_t e = p0; e < p1; ++e) {
+            uint64_t q = e / 8;
+            int whole = 8 * q >= p0 && 8 * q + 8 <= p1;
+            if (!whole)
+                sum += orc_mix(signmant[e], (uint32_t)(0x200000u + (e - b)));
+        }
+        for (uint64_t q = (p0 + 7) / 8; 8 * q + 8 <= p1; ++q) {
+            const uint8_t *g8 = signmant + 8 * q;
+            uint32_t v0 = g8[0] | ((uint32_t)g8[1] << 8) | ((uint32_t)g8[2] << 16) | ((uint32_t)g8[3] << 24);
+            uint32_t v1 = g8[4] | ((uint32_t)g8[5] << 8) | ((uint32_t)g8[6] << 16) | ((uint32_t)g8[7] << 24);
+            uint64_t r = q - b / 8;
+            sum += orc_mix(v0, (uint32_t)(0x100000u + 2 * r));
+            sum += orc_mix(v1, (uint32_t)(0x100000u + 2 * r + 1));
+        }
+        /* the tables, in chunk 0 */
+        if (c == 0)
+            for (uint64_t i = 0; i < 128ull * n_tables; ++i)
+                sum += orc_mix(lut[2 * i] | ((uint32_t)lut[2 * i + 1] << 16), (uint32_t)(0x400000u + i));
+        out[c] = sum;
+    }
+    return 0;
+}

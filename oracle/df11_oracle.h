@@ -121,6 +121,33 @@ uint32_t orc_crc32c(const uint8_t *data, uint64_t n);
  * number of values written to out (ceil(n / seg)). */
 uint64_t orc_segment_crcs(const uint8_t *data, uint64_t n, uint64_t seg, uint32_t *out);
 
+/* Per-chunk sum: the integrity check the library's decoder can run as it
+ * decodes (the pages ask only to checksum artifacts, "How to run it in
+ * production"; this is the library's own check, computed by the decode
+ * kernel from the bytes it already holds).  For chunk c (threads 32c..32c+31,
+ * B = 8 * bytes_per_thread bits per slice), the sum mod 2^32 of mix(v, tag)
+ * over these items:
+ *   - stream words k = 0 .. B - 1 (the chunk's 32 B stream bits, words of 32):
+ *     bit i of v is chunk stream bit 32k + i (MSB-first within bytes); tag k;
+ *   - threads t = 0..31: v = gap | count << 8 of thread 32c + t;
+ *     tag 0x10000 + t;
+ *   - v = chunk_pos[c], tag 0x20000; v = chunk_pos[c + 1], tag 0x20001;
+ *   - sign|mantissa bytes of elements [p0, p1) = [chunk_pos[c],
+ *     chunk_pos[c + 1]), with b = p0 rounded down to a multiple of 8: each
+ *     8-element group [8q, 8q + 8) inside [p0, p1) gives two little-endian
+ *     words of its bytes, tags 0x100000 + 2r and 0x100000 + 2r + 1 (r = q -
+ *     b / 8); every other element e gives its byte alone, tag 0x200000 + e - b;
+ *   - chunk 0 only: the tables as little-endian words (entries 2i and 2i + 1,
+ *     i < 128 n_tables), tag 0x400000 + i.
+ * mix(v, tag) = y ^ (y >> 16), y = (v ^ tag * 0x9E3779B1) * 0x85EBCA6B (mod
+ * 2^32): for each tag a bijection of v, so any change of one item changes
+ * the sum.  gaps are packed (two per byte), counts one byte per thread.
+ * Returns 0, or -1 for bad arguments (positions that decrease or pass
+ * signmant_bytes among them). */
+int orc_chunk_sums(const uint8_t *stream, const uint8_t *gaps, const uint8_t *counts, const uint32_t *pos,
+                   const uint8_t *signmant, uint64_t signmant_bytes, const uint16_t *lut, uint32_t n_tables,
+                   uint32_t bytes_per_thread, uint64_t n_chunks, uint32_t *out);
+
 #ifdef __cplusplus
 }
 #endif

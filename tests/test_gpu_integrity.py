@@ -151,3 +151,165 @@ def test_pipeline_verify_stage():
         assert [int(e.item()) for e in errs] == want
         if want[1]:
             assert int(firsts[1].item()) == lists[1].numel() - 1
+
+
+# ------------------------------------------------ decode with chunk sums
+# df11_decompress_verified_async: the decode kernel sums every chunk's bytes
+# as it reads them and compares with the sums of df11_chunk_sums; the
+# expected sums here are the oracle's.
+
+def _oracle_chunk_sums(hb):
+    h = hb.header
+    return oracle.chunk_sums(hb.exp_stream, hb.gaps, hb.counts, hb.chunk_pos, hb.signmant, hb.lut,
+                             h.n_tables, h.bytes_per_thread, h.n_chunks)
+
+
+def _block_input(name):
+    mats = {
+        "llama_div256": lambda: workloads.llama_block(1003, scale_div=256),
+        "heavy_tail_512": lambda: workloads.heavy_tail(4001, (512, 512)),
+        "single_exponent_64": lambda: workloads.single_exponent(4002, (64, 64)),
+        "uniform_bits_256": lambda: workloads.uniform_bits(4003, (256, 256)),
+        "tiny_3x8": lambda: workloads.single_matrix(5, shape=(3, 8)),
+    }[name]()
+    return np.concatenate([m.reshape(-1) for _, m in mats])
+
+
+def _verified(db, sums, n):
+    out = torch.empty(n, dtype=torch.int16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    first = torch.full((1,), -1, dtype=torch.int64, device="cuda")
+    df11.decompress_verified_async(db, out, sums, err, first)
+    torch.cuda.synchronize()
+    return out, int(err.item()), int(first.item())
+
+
+@pytest.mark.parametrize("name", NAMES)
+@pytest.mark.parametrize("bpt", [8, 16])
+def test_verified_decode_of_clean_blocks(name, bpt):
+    w = _block_input(name)
+    cb = df11.build_codebook([w])
+    hb = df11.compress(cb, [w], 32, bpt)
+    sums = _oracle_chunk_sums(hb)
+    assert np.array_equal(df11.chunk_sums(hb), sums)
+    db = hb.to_device("cuda")
+    out, err, first = _verified(db, torch.from_numpy(sums.view(np.int32)).cuda(), w.size)
+    assert err == 0 and first == -1
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), w)
+    # a wrong expected sum is reported at its chunk, and the output is still written
+    for c in sorted({0, hb.header.n_chunks - 1, hb.header.n_chunks // 2}):
+        bad = sums.copy()
+        bad[c] ^= np.uint32(1 << (c % 32))
+        out, err, first = _verified(db, torch.from_numpy(bad.view(np.int32)).cuda(), w.size)
+        assert err == df11.DEVERR_CHECKSUM and first == c
+        assert np.array_equal(out.cpu().numpy().view(np.uint16), w)
+
+
+def _allowed_first_bad(hb, array, byte, bit):
+    """Chunks a flipped bit may be reported at: the lowest chunk whose sum
+    covers it, or the chunk before, which also reads the next chunk's first
+    stream word (codes that cross into it) and its first thread's gap (where
+    its last code must end); None for bytes no chunk covers."""
+    h = hb.header
+    cb = 32 * h.bytes_per_thread
+    n = h.n_chunks
+    pos = hb.chunk_pos
+    if array == "exp_stream":
+        if byte >= n * cb:
+            return None
+        c = byte // cb
+        return {c, c - 1} - {-1} if byte % cb < 4 else {c}
+    if array == "gaps":
+        if 2 * byte >= 32 * n:
+            return None
+        c = (2 * byte) // 32
+        return {c, c - 1} - {-1} if byte % 16 == 0 and bit < 4 else {c}
+    if array == "counts":
+        return {byte // 32} if byte < 32 * n else None
+    if array == "chunk_pos":
+        k = byte // 4
+        return {max(k - 1, 0)} if k <= n else None
+    if array == "signmant":
+        owners = [c for c in range(n) if pos[c] <= byte < pos[c + 1]]
+        return {owners[0]} if owners else None
+    if array == "lut":
+        return {0}
+    raise KeyError(array)
+
+
+@pytest.mark.parametrize("name", ["llama_div256", "heavy_tail_512", "single_exponent_64"])
+@pytest.mark.parametrize("bpt", [8, 16])
+def test_verified_decode_reports_a_flipped_bit_at_its_chunk(name, bpt):
+    """One bit flipped in each array at several places (ends, chunk edges,
+    random): the launch reports an error and the lowest bad chunk the flip
+    can spoil; a bit outside every chunk changes nothing."""
+    w = _block_input(name)
+    cb = df11.build_codebook([w])
+    hb = df11.compress(cb, [w], 32, bpt)
+    sums = torch.from_numpy(_oracle_chunk_sums(hb).view(np.int32)).cuda()
+    db = hb.to_device("cuda")
+    rng = np.random.default_rng(17)
+    n = hb.header.n_chunks
+    cbytes = 32 * hb.header.bytes_per_thread
+    for a in ARRAYS:
+        t = db.tensors[a]
+        nbytes = getattr(hb, a).nbytes
+        places = {0, nbytes - 1, int(rng.integers(0, nbytes)), int(rng.integers(0, nbytes))}
+        if a == "exp_stream":
+            places |= {cbytes * min(1, n - 1), cbytes * min(1, n - 1) + 5, n * cbytes}
+        if a == "gaps":
+            places |= {16 * min(1, n - 1)}
+        if a == "chunk_pos":
+            places |= {4 * n, 4 * min(1, n), 4 * n + 3}
+        if a == "signmant":
+            places |= {int(hb.chunk_pos[min(1, n)]), hb.n_elements - 1}
+        for byte in sorted(p for p in places if p < nbytes):
+            for bit in sorted({int(rng.integers(0, 8)), 0, 7}):
+                allowed = _allowed_first_bad(hb, a, byte, bit)
+                t[byte] ^= (1 << bit)
+                out, err, first = _verified(db, sums, w.size)
+                t[byte] ^= (1 << bit)
+                if allowed is None:
+                    assert err == 0 and first == -1, (a, byte, bit)
+                    assert np.array_equal(out.cpu().numpy().view(np.uint16), w), (a, byte, bit)
+                else:
+                    assert err != 0 and first in allowed, (a, byte, bit, err, first, allowed)
+    out, err, first = _verified(db, sums, w.size)
+    assert err == 0 and first == -1
+
+
+@pytest.mark.slow
+def test_verified_decode_full_block():
+    """Llama-3.1-8B-shaped block compressed on the GPU: the oracle's chunk
+    sums equal the library's; the verified decode of the clean block is
+    exact and silent; one flipped bit in each array is reported at its
+    chunk."""
+    d_in = workloads.llama_block_device(1000, "cuda")
+    hist = df11.histogram_device(d_in)
+    cb = df11.build_codebook_from_histogram(hist.cpu().numpy().astype(np.uint64))
+    db = df11.compress_device(cb, d_in)
+    host = {a: db.tensors[a][: db.sizes[a]].cpu().numpy() for a in ARRAYS}
+    hb = df11.HostBlock(header=db.header, exp_stream=host["exp_stream"], gaps=host["gaps"],
+                        counts=host["counts"], chunk_pos=host["chunk_pos"].view(np.uint32),
+                        signmant=host["signmant"], lut=host["lut"].view(np.uint16))
+    ref = _oracle_chunk_sums(hb)
+    assert np.array_equal(df11.chunk_sums(hb), ref)
+    sums = torch.from_numpy(ref.view(np.int32)).cuda()
+    n = d_in.numel()
+    out, err, first = _verified(db, sums, n)
+    assert err == 0 and first == -1
+    assert torch.equal(out, d_in)
+    rng = np.random.default_rng(23)
+    for a in ARRAYS:
+        t = db.tensors[a]
+        nbytes = db.sizes[a]
+        byte = int(rng.integers(0, nbytes))
+        bit = int(rng.integers(0, 8))
+        allowed = _allowed_first_bad(hb, a, byte, bit)
+        t[byte] ^= (1 << bit)
+        out, err, first = _verified(db, sums, n)
+        t[byte] ^= (1 << bit)
+        if allowed is None:
+            assert err == 0 and first == -1, (a, byte)
+        else:
+            assert err != 0 and first in allowed, (a, byte, err, first, allowed)

@@ -439,6 +439,61 @@ def test_checksum_list_equals_oracle(name):
     assert np.array_equal(got, ref)
 
 
+def _oracle_chunk_sums(hb):
+    h = hb.header
+    return oracle.chunk_sums(hb.exp_stream, hb.gaps, hb.counts, hb.chunk_pos, hb.signmant, hb.lut,
+                             h.n_tables, h.bytes_per_thread, h.n_chunks)
+
+
+@pytest.mark.parametrize("name", ["single_1024x1024", "heavy_tail_512", "single_exponent_512", "tiny"])
+@pytest.mark.parametrize("bpt", [8, 16])
+def test_chunk_sums_equal_oracle(name, bpt):
+    """df11_chunk_sums (the library's word-level code) against the oracle's
+    bit-by-bit definition, every chunk, both slice widths."""
+    mats = ([workloads.single_matrix(3, shape=(3, 5))[0][1]] if name == "tiny"
+            else [m for _, m in SMALL_WORKLOADS[name]()])
+    cb = df11.build_codebook(mats)
+    hb = df11.compress(cb, mats, 32, bpt)
+    got = df11.chunk_sums(hb)
+    assert got.size == hb.header.n_chunks
+    assert np.array_equal(got, _oracle_chunk_sums(hb))
+
+
+def test_chunk_sums_reject_bad_arguments():
+    hb = _fresh_block()
+    lib = df11.load_library()
+    b = hb.c_struct()
+    n = int(hb.header.n_chunks)
+    out = np.empty(n + 1, np.uint32)
+    assert lib.df11_chunk_sums(ctypes.byref(b), out.ctypes.data, n) == 0
+    assert lib.df11_chunk_sums(ctypes.byref(b), out.ctypes.data, n + 1) == 1
+    assert lib.df11_chunk_sums(ctypes.byref(b), None, n) == 1
+    assert lib.df11_chunk_sums(None, out.ctypes.data, n) == 1
+    pos = hb.chunk_pos.copy()
+    pos[1], pos[2] = pos[2], pos[1] - 1        # decreasing positions
+    bad = df11.HostBlock(header=hb.header, exp_stream=hb.exp_stream, gaps=hb.gaps, counts=hb.counts,
+                         chunk_pos=pos, signmant=hb.signmant, lut=hb.lut)
+    bb = bad.c_struct()
+    assert lib.df11_chunk_sums(ctypes.byref(bb), out.ctypes.data, n) == 1
+    # the verified decode's host-side checks, before any CUDA call
+    fake = 1 << 20
+    d = binding._Block()
+    d.hdr = hb.header
+    for name in ("exp_stream", "gaps", "counts", "chunk_pos", "signmant", "lut"):
+        setattr(d, name, fake)
+    d.exp_stream_bytes, d.gaps_bytes, d.counts_bytes = hb.exp_stream.nbytes, hb.gaps.nbytes, hb.counts.nbytes
+    d.chunk_pos_count, d.signmant_bytes, d.lut_entries = hb.chunk_pos.size, hb.signmant.nbytes, hb.lut.size
+    m = hb.n_elements
+    v = lib.df11_decompress_verified_async
+    assert v(ctypes.byref(d), fake, m, fake, None, None, None, None) == 1          # no sums
+    assert v(ctypes.byref(d), fake, m, None, fake, None, None, None) == 1          # no error word
+    assert v(ctypes.byref(d), fake, m, fake, fake + 2, None, None, None) == 1      # misaligned sums
+    assert v(ctypes.byref(d), fake, m, fake, fake, fake + 4, None, None) == 1      # misaligned first_bad
+    assert v(ctypes.byref(d), None, m, fake, fake, None, None, None) == 1
+    assert v(None, fake, m, fake, fake, None, None, None) == 1
+    assert v(ctypes.byref(d), fake, m - 1, fake, fake, None, None, None) == 1      # too little room
+
+
 def test_crc32c_equals_oracle_any_length_and_offset():
     rng = np.random.default_rng(11)
     buf = rng.integers(0, 256, 20000, dtype=np.uint8)

@@ -466,3 +466,109 @@ def test_segment_crcs_split_and_ragged_tail():
         assert s[k] == _crc32c_by_division(a[4096 * k: 4096 * (k + 1)].tobytes())
     assert oracle.segment_crcs(np.zeros(0, np.uint8)).size == 0
     assert oracle.segment_crcs(np.zeros(4096, np.uint8)).size == 1
+
+
+# ------------------------------------------------------------ chunk sums
+# The per-chunk sum is this library's own check (the page asks only that
+# artifacts be checksummed, "How to run it in production"), so no page
+# prints a value of it.  It is pinned to what it is for: every one-bit
+# change of any array it covers changes exactly the sums of the chunks that
+# read that bit, bytes outside every chunk change nothing, and the sum
+# depends on where each item sits, not only on the multiset of items.
+
+def _tiny_artifact(seed, W):
+    """A small oracle artifact with 32 threads per chunk: (stream, packed
+    gaps, counts, pos, signmant, lut, n_tables, n_chunks)."""
+    rng = np.random.default_rng(seed)
+    mats = [workloads.to_bf16((rng.standard_normal(5000 + 97 * seed) * 0.02).astype(np.float32))]
+    ob = oracle.compress_block(mats, threads_per_chunk=32, bytes_per_thread=W)
+    gap = np.zeros(ob.gap.size + (ob.gap.size & 1), np.uint8)
+    gap[: ob.gap.size] = ob.gap
+    packed = (gap[0::2] | (gap[1::2] << 4)).astype(np.uint8)
+    sm = np.concatenate([ob.signmant, rng.integers(0, 256, 5, dtype=np.uint8)])   # bytes past the end
+    n_tables = 2
+    lut = rng.integers(0, 65536, 256 * n_tables, dtype=np.uint16)
+    return [ob.stream.copy(), packed, ob.thread_count.copy(), ob.pos.copy(), sm, lut, n_tables, ob.n_chunks]
+
+
+def _sums(a, W):
+    stream, gaps, counts, pos, sm, lut, n_tables, n_chunks = a
+    return oracle.chunk_sums(stream, gaps, counts, pos, sm, lut, n_tables, W, n_chunks)
+
+
+@pytest.mark.parametrize("W", [8, 16])
+def test_chunk_sums_every_bit_flip_changes_exactly_its_chunks(W):
+    a = _tiny_artifact(1, W)
+    stream, gaps, counts, pos, sm, lut, n_tables, n_chunks = a
+    assert n_chunks >= 3
+    base = _sums(a, W)
+    chunk_bytes = 32 * W
+
+    def owners(name, i):
+        if name == "stream":
+            return {i // chunk_bytes} if i < n_chunks * chunk_bytes else set()
+        if name == "gaps":
+            return {(2 * i) // 32} if 2 * i < 32 * n_chunks else set()
+        if name == "counts":
+            return {i // 32} if i < 32 * n_chunks else set()
+        if name == "signmant":
+            return {c for c in range(n_chunks) if pos[c] <= i < pos[c + 1]}
+        if name == "lut":
+            return {0}
+        raise AssertionError(name)
+
+    for idx, name in ((0, "stream"), (1, "gaps"), (2, "counts"), (4, "signmant"), (5, "lut")):
+        arr = a[idx].view(np.uint8)
+        for i in range(arr.size):
+            want = owners(name, i // a[idx].itemsize if name == "lut" else i)
+            for bit in range(8):
+                arr[i] ^= 1 << bit
+                changed = set(np.nonzero(_sums(a, W) != base)[0].tolist())
+                arr[i] ^= 1 << bit
+                assert changed == want, (name, i, bit)
+    # positions: a flip that keeps them ordered and in range changes the two
+    # chunks that share the position; any other is rejected
+    for c in range(n_chunks + 1):
+        for bit in range(32):
+            pos[c] ^= np.uint32(1 << bit)
+            ok = all(pos[k] <= pos[k + 1] for k in range(n_chunks)) and pos[n_chunks] <= sm.size
+            if ok:
+                changed = set(np.nonzero(_sums(a, W) != base)[0].tolist())
+                assert changed == {k for k in (c - 1, c) if 0 <= k < n_chunks}, (c, bit)
+            else:
+                with pytest.raises(ValueError):
+                    _sums(a, W)
+            pos[c] ^= np.uint32(1 << bit)
+    assert np.array_equal(_sums(a, W), base)
+
+
+def test_chunk_sums_depend_on_item_places():
+    """Swapping two unequal items of one chunk (stream words, threads'
+    metadata, 8-byte groups, single bytes) changes its sum: every item
+    carries its place."""
+    W = 16
+    a = _tiny_artifact(2, W)
+    stream, gaps, counts, pos, sm, lut, n_tables, n_chunks = a
+    base = _sums(a, W)
+    s32 = stream[: 32 * W * n_chunks].view(np.uint32)
+    k = next(k for k in range(1, 32) if s32[k] != s32[0])
+    s32[[0, k]] = s32[[k, 0]]
+    assert _sums(a, W)[0] != base[0]
+    s32[[0, k]] = s32[[k, 0]]
+    t = next(t for t in range(1, 32) if counts[t] != counts[0])
+    counts[[0, t]] = counts[[t, 0]]
+    assert _sums(a, W)[0] != base[0]
+    counts[[0, t]] = counts[[t, 0]]
+    c = 1
+    p0, p1 = int(pos[c]), int(pos[c + 1])
+    q0 = (p0 + 7) // 8
+    assert 8 * q0 + 16 <= p1
+    g = sm[8 * q0: 8 * q0 + 16].copy()
+    sm[8 * q0: 8 * q0 + 16] = np.concatenate([g[8:], g[:8]])
+    assert _sums(a, W)[c] != base[c] or np.array_equal(g[8:], g[:8])
+    sm[8 * q0: 8 * q0 + 16] = g
+    e = next(e for e in range(p0 + 1, p1) if sm[e] != sm[p0])
+    sm[[p0, e]] = sm[[e, p0]]
+    assert _sums(a, W)[c] != base[c]
+    sm[[p0, e]] = sm[[e, p0]]
+    assert np.array_equal(_sums(a, W), base)
