@@ -9,15 +9,16 @@
 //   2. (host) df11_build_codebook_from_histogram -- code lengths, canonical
 //                                 codes and tables from that histogram;
 //   3. df11_compress_device    -- bit count per segment of 8192 elements
-//      (one warp per segment), a scan of the segment counts, then one
-//      encode pass in which every thread knows its first bit: it appends its
-//      codes MSB-first into the segment's stream words staged in shared
-//      memory (words shared with a neighbouring thread are ORed), records
-//      the gap of every slice whose first code it owns (staged too) and the
-//      output position of every chunk that starts in such a slice, adds the
-//      number of its codes that start in each slice to a staged per-slice
-//      count, and writes its sign|mantissa bytes; the staged words then go
-//      to global memory with plain stores, ORing only the two words a
+//      (one warp per segment; also summed per run of 256 segments), then one
+//      encode pass, a CTA per segment, in which every thread knows its first
+//      bit (the run totals and segment counts before its segment, and a CTA
+//      scan): it appends its codes MSB-first to a bit accumulator and stores
+//      each stream word it completes into the segment's staging in shared
+//      memory, ORs its part-filled last word into the next thread's, records
+//      the gap of every slice whose first code it owns and the output
+//      position of every chunk that starts in such a slice, counts its codes
+//      per slice, and writes its sign|mantissa bytes; the staged words then
+//      go to global memory with plain stores, ORing only the two words a
 //      segment may share with its neighbours, and the staged counts are
 //      added into the (zeroed) counts array, four per word.
 // The result is byte-identical to df11_compress (host) for the same
@@ -39,7 +40,7 @@ namespace {
 constexpr int kEncThreads = 256;
 constexpr int kElemsPerThread = 32;
 constexpr int kSegElems = kEncThreads * kElemsPerThread;   // 8192 elements per segment
-constexpr int kScanThreads = 1024;
+constexpr int kRunSegs = 256;   // segments per run: an encode CTA sums <= kRunSegs - 1 counts and the run totals
 
 // Code table passed by value: entry s = code | (length << 24); length 0 = absent.
 struct CodeTable {
@@ -54,7 +55,8 @@ struct EncodeParams {
     uint32_t *chunk_pos;
     uint8_t *signmant;
     uint32_t *seg_bits;     // scratch: bits per segment
-    uint64_t *seg_start;    // scratch: first bit per segment (exclusive scan)
+    uint64_t *run_bits;     // scratch: bits per run of kRunSegs segments
+    uint32_t *code_table;   // scratch: the code table (code | length << 24), as in CodeTable
     uint16_t *grp_bits;     // scratch: bits per 32 elements of full segments, or null
     uint32_t *err;          // optional device error word
     uint64_t n;
@@ -96,18 +98,10 @@ __global__ void __launch_bounds__(256) histogram_kernel(const uint16_t *in, uint
 
 // ---- encode: per-thread code lengths -----------------------------------------
 
-// Loads this thread's up to 32 elements (zero past n) and returns their
-// bits: counted in the bit-count pass for a full segment when the scratch
-// holds the group counts, else here (*bad is then set when an element's
-// exponent has no code).
-__device__ __forceinline__ uint32_t load_elems(const EncodeParams &p, const uint32_t *len_tab,
-                                               uint64_t e0, uint32_t (&w)[16], bool &bad)
+// Loads this thread's up to 32 elements, two to a word, element 2i in the
+// low half of w[i] (zero past n).
+__device__ __forceinline__ void load_words(const EncodeParams &p, uint64_t e0, uint32_t (&w)[16])
 {
-    const uint64_t seg = e0 / kSegElems;
-    const bool counted = p.grp_bits != nullptr && (seg + 1) * kSegElems <= p.n;
-    uint32_t counted_bits = 0;
-    if (counted)
-        counted_bits = p.grp_bits[e0 / kElemsPerThread];
     if (e0 + kElemsPerThread <= p.n) {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.in + e0);
 #pragma unroll
@@ -127,14 +121,20 @@ __device__ __forceinline__ uint32_t load_elems(const EncodeParams &p, const uint
             w[k] = a | (b << 16);
         }
     }
-    if (counted)
-        return counted_bits;
+}
+
+// Bits of this thread's elements, counted here (when the bit-count pass kept
+// no group counts, or in the last segment); *bad is set when an element's
+// exponent has no code.
+__device__ __forceinline__ uint32_t count_bits(const EncodeParams &p, const uint2 *code_tab, uint64_t e0,
+                                               const uint32_t (&w)[16], bool &bad)
+{
     uint32_t bits = 0;
 #pragma unroll
     for (int k = 0; k < kElemsPerThread; ++k) {
         if (e0 + k < p.n) {
             const uint32_t x = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
-            const uint32_t l = len_tab[(x >> 7) & 0xFFu];
+            const uint32_t l = code_tab[(x >> 7) & 0xFFu].y;
             bad |= l == 0;
             bits += l;
         }
@@ -177,11 +177,12 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
 
 // Bits of every segment: one warp per segment, whose lanes read it 512
 // contiguous bytes at a time (lane l takes bytes [16 l, 16 l + 16) of each),
-// then a warp sum.
-__global__ void __launch_bounds__(256) segment_bits_kernel(EncodeParams p, CodeTable ct)
+// then a warp sum, also added to the total of the segment's run of
+// kRunSegs segments.
+__global__ void __launch_bounds__(256) segment_bits_kernel(EncodeParams p)
 {
     __shared__ uint32_t len_tab[256];
-    len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
+    len_tab[threadIdx.x] = p.code_table[threadIdx.x] >> 24;
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x >> 5);
@@ -223,68 +224,31 @@ __global__ void __launch_bounds__(256) segment_bits_kernel(EncodeParams p, CodeT
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             bits += __shfl_xor_sync(0xFFFFFFFFu, bits, o);
-        if (lane == 0)
+        if (lane == 0) {
             p.seg_bits[seg] = bits;
+            atomicAdd(reinterpret_cast<unsigned long long *>(p.run_bits + seg / kRunSegs),
+                      (unsigned long long)bits);
+        }
     }
     if (bad && p.err)
         atomicOr(p.err, DF11_DEVERR_MISMATCH);
 }
 
-// Exclusive scan of the segment bit counts (one CTA): thread t sums a run of
-// consecutive segments, the CTA scans the run totals, then every thread
-// writes its run's starts.  Checks the grand total against the codebook.
-__global__ void __launch_bounds__(kScanThreads) segment_scan_kernel(EncodeParams p)
-{
-    __shared__ unsigned long long warp_tot[kScanThreads / 32 + 1];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint64_t per = (p.n_seg + kScanThreads - 1) / kScanThreads;
-    const uint64_t lo = (uint64_t)threadIdx.x * per;
-    const uint64_t hi = lo + per < p.n_seg ? lo + per : p.n_seg;
-    unsigned long long run = 0;
-    for (uint64_t i = lo; i < hi; ++i)
-        run += p.seg_bits[i];
-    unsigned long long incl = run;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d)
-            incl += y;
-    }
-    if (lane == 31)
-        warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const unsigned long long t = warp_tot[lane];
-        unsigned long long ti = t;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, ti, d);
-            if (lane >= d)
-                ti += y;
-        }
-        warp_tot[lane] = ti - t;
-        if (lane == 31)
-            warp_tot[kScanThreads / 32] = ti;
-    }
-    __syncthreads();
-    unsigned long long start = warp_tot[warp] + incl - run;
-    for (uint64_t i = lo; i < hi; ++i) {
-        p.seg_start[i] = start;
-        start += p.seg_bits[i];
-    }
-    if (threadIdx.x == 0 && warp_tot[kScanThreads / 32] != p.total_bits && p.err)
-        atomicOr(p.err, DF11_DEVERR_MISMATCH);
-}
-
-// Zeroes the stream, gaps, counts and sign|mantissa tail; fills chunk
-// positions with n.
-__global__ void prepare_kernel(EncodeParams p, uint64_t stream_words, uint64_t gap_words,
+// Zeroes the stream, gaps, counts, run totals and sign|mantissa tail; fills
+// chunk positions with n; copies the code table into global memory (read
+// there with per-thread indices, which a kernel parameter would serialise).
+__global__ void prepare_kernel(EncodeParams p, CodeTable ct, uint64_t stream_words, uint64_t gap_words,
                                uint64_t n_chunks, uint64_t sm_bytes)
 {
     const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (tid < 256)
+        p.code_table[tid] = ct.e[tid];
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    uint4 *s128 = reinterpret_cast<uint4 *>(p.stream);
+    for (uint64_t i = tid; i < stream_words / 4; i += stride)
+        s128[i] = make_uint4(0u, 0u, 0u, 0u);
     uint32_t *s32 = reinterpret_cast<uint32_t *>(p.stream);
-    for (uint64_t i = tid; i < stream_words; i += stride)
+    for (uint64_t i = stream_words / 4 * 4 + tid; i < stream_words; i += stride)
         s32[i] = 0;
     uint32_t *g32 = reinterpret_cast<uint32_t *>(p.gaps);
     for (uint64_t i = tid; i < gap_words; i += stride)
@@ -296,55 +260,141 @@ __global__ void prepare_kernel(EncodeParams p, uint64_t stream_words, uint64_t g
         p.chunk_pos[i] = (uint32_t)p.n;
     for (uint64_t i = p.n + tid; i < sm_bytes; i += stride)
         p.signmant[i] = 0;
-}
-
-__device__ __forceinline__ void red_or_shared_if(bool p, uint32_t a, uint32_t v)
-{
-    asm volatile("{ .reg .pred q; setp.ne.u32 q, %0, 0; @q red.shared.or.b32 [%1], %2; }" ::"r"((uint32_t)p), "r"(a),
-                 "r"(v)
-                 : "memory");
+    for (uint64_t i = tid; i < (p.n_seg + kRunSegs - 1) / kRunSegs; i += stride)
+        p.run_bits[i] = 0;
 }
 
 // Shared staging of one segment's output: stream words in bit order (bit 31
-// = first bit), and gap words (8 nibbles each, as in the gaps array).
-constexpr int kStageWords = kSegElems * 16 / 32 + 2;          // 16-bit codes at most
-constexpr int kGapStageWords = kSegElems * 16 / 64 / 8 + 2;   // 64-bit slices at the finest
+// = first bit), and one word per slice that a code of the segment opens:
+// the opening element's index in the segment | gap << 16 | kOpened.
+constexpr int kStageWords = kSegElems * 16 / 32 + 4;            // 16-bit codes at most
+constexpr int kSliceStage = (kSegElems * 16 / 64 / 8 + 2) * 8;  // 64-bit slices at the finest
+constexpr uint32_t kOpened = 0x80000000u;
 
-__global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, CodeTable ct)
+// Bits of one segment's encode, per thread: the codes of its elements are
+// appended to a right-aligned bit accumulator (hi:lo, nb bits) that starts
+// with the thread's offset into its first stream word as zero bits, so each
+// 32 bits it completes are one whole stream word.
+struct BitSink {
+    uint32_t lo, hi, nb;
+    uint32_t sp;   // shared address of the next stream word
+    __device__ __forceinline__ void put(uint32_t c, uint32_t l)   // l <= 32, nb < 32
+    {
+        asm volatile(
+            "{\n\t"
+            ".reg .pred p;\n\t"
+            ".reg .b32 t, s;\n\t"
+            "shf.l.clamp.b32 %1, %0, %1, %4;\n\t"   // hi:lo <<= l
+            "shl.b32 t, %0, %4;\n\t"
+            "or.b32 %0, t, %5;\n\t"
+            "add.u32 %2, %2, %4;\n\t"
+            "setp.ge.u32 p, %2, 32;\n\t"
+            "sub.u32 s, %2, 32;\n\t"
+            "shf.r.clamp.b32 t, %0, %1, s;\n\t"     // the completed word: bits [nb - 32, nb)
+            "@p st.shared.u32 [%3], t;\n\t"
+            "@p add.u32 %3, %3, 4;\n\t"
+            "@p mov.u32 %2, s;\n\t"
+            "}"
+            : "+r"(lo), "+r"(hi), "+r"(nb), "+r"(sp)
+            : "r"(l), "r"(c)
+            : "memory");
+    }
+};
+
+// One segment of 8192 elements per CTA, 32 per thread.  Every thread knows
+// its first bit (the segment's start, from the run totals and the segment
+// counts before it, plus a CTA scan of the kept group counts) and encodes its
+// codes MSB-first.  A completed stream word is stored by the thread that
+// completes it (its first bits may be the previous thread's: zeros here);
+// after a barrier each thread ORs its part-filled last word into the word
+// the next thread completed.  A slice that one of the thread's codes opens
+// gets its gap, and a chunk that starts there its output position (rare: a
+// branch, tested once per four codes); the codes of each slice are counted
+// into its staged byte.  Then the staged words go to global memory.
+__global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(EncodeParams p)
 {
-    __shared__ uint32_t code_tab[256];   // code | length << 24
-    __shared__ uint32_t len_tab[256];
+    __shared__ uint2 code_tab[256];   // code (right-aligned), length; length 0 = absent
     __shared__ uint32_t warp_tot[kEncThreads / 32 + 1];
-    __shared__ uint32_t sw[kStageWords];
-    __shared__ uint32_t sg[kGapStageWords * 2];   // one byte per slice's gap (plain byte stores)
-    __shared__ uint32_t sc[kGapStageWords * 8];   // one count per slice (shared atomic adds)
-    code_tab[threadIdx.x] = ct.e[threadIdx.x];
-    len_tab[threadIdx.x] = ct.e[threadIdx.x] >> 24;
-    for (int i = threadIdx.x; i < kStageWords; i += kEncThreads)
-        sw[i] = 0;
-    for (int i = threadIdx.x; i < kGapStageWords * 2; i += kEncThreads)
-        sg[i] = 0;
-    for (int i = threadIdx.x; i < kGapStageWords * 8; i += kEncThreads)
-        sc[i] = 0;
-    uint8_t *const sgb = reinterpret_cast<uint8_t *>(sg);
-    __syncthreads();
-
+    __shared__ unsigned long long seg_first;
+    __shared__ uint32_t last_elem[kEncThreads / 32];   // each warp's last element
+    __shared__ __align__(16) uint32_t sw[kStageWords];
+    __shared__ __align__(16) uint32_t so[kSliceStage];
+    const uint32_t tid = threadIdx.x;
     const uint64_t seg = blockIdx.x;
-    const uint64_t e0 = seg * kSegElems + (uint64_t)threadIdx.x * kElemsPerThread;
+    const bool tail = (seg + 1) * kSegElems > p.n;
+    // Global loads first, all independent: this thread's elements (and its
+    // group's kept bit count), and in warp 0 the run totals and segment
+    // counts before this segment in its run, spread over the 32 lanes.
+    const uint64_t e0 = seg * kSegElems + (uint64_t)tid * kElemsPerThread;
     uint32_t w[16];
+    const bool counted = p.grp_bits != nullptr && !tail;
+    const uint32_t counted_bits = counted ? p.grp_bits[e0 / kElemsPerThread] : 0u;
+    load_words(p, e0, w);
+    unsigned long long acc = 0;
+    if (tid < 32) {
+        const uint64_t run = seg / kRunSegs;
+        const uint64_t first = run * kRunSegs;
+        uint32_t sb[kRunSegs / 32];
+#pragma unroll
+        for (int i = 0; i < kRunSegs / 32; ++i) {
+            const uint64_t j = first + (uint64_t)(32 * i) + tid;
+            sb[i] = j < seg ? p.seg_bits[j] : 0u;
+        }
+        for (uint64_t r = tid; r < run; r += 32)
+            acc += p.run_bits[r];
+#pragma unroll
+        for (int i = 0; i < kRunSegs / 32; ++i)
+            acc += sb[i];
+    }
+    // the element before this thread's first: the previous thread's last
+    // (thread 0: loaded)
+    uint32_t prev = __shfl_up_sync(0xFFFFFFFFu, w[15] >> 16, 1);
+    if ((tid & 31) == 0)
+        prev = tid == 0 ? (e0 > 0 ? (uint32_t)p.in[e0 - 1] : 0u) : 0xFFFFFFFFu;
+    {
+        const uint32_t e = p.code_table[tid];
+        code_tab[tid] = make_uint2(e & 0xFFFFFFu, e >> 24);
+    }
+    static_assert(kSliceStage % 4 == 0 && kStageWords % 4 == 0, "vector zeroing");
+    for (uint32_t i = tid; i < kSliceStage / 4; i += kEncThreads)
+        reinterpret_cast<uint4 *>(so)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (tail)   // words nobody completes in the last segment
+        for (uint32_t i = tid; i < kStageWords / 4; i += kEncThreads)
+            reinterpret_cast<uint4 *>(sw)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if ((tid & 31) == 31)
+        last_elem[tid >> 5] = w[15] >> 16;
+    if (tid < 32) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+        if (tid == 0)
+            seg_first = acc;
+    }
+    __syncthreads();
+    if (prev == 0xFFFFFFFFu)
+        prev = last_elem[(tid >> 5) - 1];
+
     bool bad = false;
-    const uint32_t bits = load_elems(p, len_tab, e0, w, bad);
+    uint32_t bits = counted_bits;
+    if (!counted)
+        bits = count_bits(p, code_tab, e0, w, bad);
     uint32_t seg_total;
     const uint32_t off = block_exclusive_scan(bits, warp_tot, seg_total);
-    const uint64_t S = p.seg_start[seg];                  // first bit of the segment
+    const uint64_t S = seg_first;                         // first bit of the segment
     const uint64_t wbase = S >> 5;                        // stream word of sw[0]
     const uint32_t sh = p.slice_shift;
     const uint64_t gS = S >> sh;                          // slice of the segment's first bit
     const uint64_t gbase = gS >> 3;                       // gap word of staged slice 0
     // Positions below are local: lb = bit - (gS << sh), so the slice of a
-    // local bit is gS + (lb >> sh) and its staged gap byte (lb >> sh) + (gS & 7).
+    // local bit is gS + (lb >> sh) and its staged byte (lb >> sh) + (gS & 7).
     const uint32_t lb0 = (uint32_t)(S - (gS << sh));
+    const uint32_t sw_a = (uint32_t)__cvta_generic_to_shared(sw);
 
+    BitSink out;
+    out.lo = out.hi = 0;
+    out.nb = (uint32_t)((S + off) & 31);
+    out.sp = sw_a + 4u * (uint32_t)(((S + off) >> 5) - wbase);
+    uint32_t cnt = 0;
     if (e0 < p.n) {
         uint32_t lb = lb0 + off;                          // local bit of the next code
         // First local bit of the slice after the one holding the previous
@@ -352,86 +402,61 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
         // segment's first slice): a code starting at or past it opens a slice.
         uint32_t next_open = 0;
         if (e0 > 0) {
-            const uint32_t lp = len_tab[(p.in[e0 - 1] >> 7) & 0xFFu];
+            const uint32_t lp = code_tab[(prev >> 7) & 0xFFu].y;
             if (lb >= lp)
                 next_open = (((lb - lp) >> sh) + 1) << sh;
         }
         const uint32_t goff = (uint32_t)(gS & 7u);
-        const uint32_t slice_mask = (1u << sh) - 1;
-        uint32_t j = (uint32_t)(((S + off) >> 5) - wbase);   // staging word being filled
-        uint32_t fill = (uint32_t)((S + off) & 31);          // its bits already placed
-        uint32_t cur = 0;
-        const uint32_t cnt = (uint32_t)min((uint64_t)kElemsPerThread, p.n - e0);
-        const uint32_t sw_a = (uint32_t)__cvta_generic_to_shared(sw);
-        // this thread's codes from element run_k on start in staged slice
-        // cur_gi (its first code's slice to begin with)
-        uint32_t cur_gi = (lb >> sh) + goff;
-        uint32_t run_k = 0;
-        // Two elements k, k + 1 (the second may be absent past the end):
-        // their codes joined into one of at most 32 bits, appended MSB-first
-        // at bit `fill` of staged word j (a full word is ORed into the
-        // staging: its first bits may be the previous thread's).  A slice one
-        // of the codes opens gets its gap nibble, and a chunk that starts
-        // there its output position (rare: a branch).  At most one of the
-        // two opens a slice: an opening code starts within 15 bits of its
-        // slice's start, so the next one starts within 31, short of the
-        // next slice (at least 64 bits on).
-        auto pair = [&](uint32_t k, bool second) {
-            const uint32_t x = w[k >> 1];                  // element k low, k + 1 high
-            const uint32_t ce1 = code_tab[(x >> 7) & 0xFFu];
-            const uint32_t ce2 = second ? code_tab[(x >> 23) & 0xFFu] : 0u;
-            const uint32_t l1 = ce1 >> 24, l2 = ce2 >> 24;
-            const uint32_t lb2 = lb + l1;                  // start of the second code
-            if ((second ? lb2 : lb) >= next_open) {
-                const bool by_first = lb >= next_open;
-                const uint32_t ob = by_first ? lb : lb2;
-                const uint32_t gl = ob >> sh;
-                const uint32_t gi = gl + goff;             // slice index relative to gbase * 8
-                sgb[gi] = (uint8_t)(ob & slice_mask & 0xFu);
-                const uint32_t k_open = k + (by_first ? 0u : 1u);
-                if (((gS + gl) & (DF11_THREADS_PER_CHUNK - 1)) == 0)
-                    p.chunk_pos[(gS + gl) / DF11_THREADS_PER_CHUNK] = (uint32_t)(e0 + k_open);
-                if (k_open > run_k)
-                    atomicAdd(&sc[cur_gi], k_open - run_k);
-                cur_gi = gi;
-                run_k = k_open;
-                next_open = (gl + 1) << sh;
-            }
-            const uint32_t l = l1 + l2;
-            lb += l;
-            const uint32_t code = ((ce1 & 0xFFFFu) << l2) | (ce2 & 0xFFFFu);
-            const uint32_t t = fill + l;                   // <= 63: one word fills at most
-            const uint64_t add = (uint64_t)code << (64u - t);
-            cur |= (uint32_t)(add >> 32);
-            const bool full = t >= 32;
-            red_or_shared_if(full, sw_a + 4u * j, cur);
-            cur = full ? (uint32_t)add : cur;
-            j += full ? 1u : 0u;
-            fill = full ? t - 32 : t;
+        const uint32_t so_a = (uint32_t)__cvta_generic_to_shared(so) + 4u * goff;
+        const uint32_t k0 = tid * kElemsPerThread;         // first element, in the segment
+        cnt = (uint32_t)min((uint64_t)kElemsPerThread, p.n - e0);
+        // The code of element k, starting at local bit s, opens a slice (its
+        // gap s - slice start is below 16, so s & 15).
+        auto open = [&](uint32_t k, uint32_t s) {
+            const uint32_t gl = s >> sh;
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(so_a + 4u * gl), "r"((k0 + k) | (s & 15u) << 16 | kOpened)
+                         : "memory");
+            next_open = (gl + 1) << sh;
         };
         if (cnt == kElemsPerThread) {
+            // Four codes at a time.  At most one of them opens a slice: an
+            // opening code starts within 15 bits of its slice's start, and
+            // the next three start within 48 bits after it, short of the
+            // next slice (at least 64 bits on).
 #pragma unroll
-            for (uint32_t k = 0; k < kElemsPerThread; k += 2)
-                pair(k, true);
+            for (uint32_t q = 0; q < kElemsPerThread / 4; ++q) {
+                const uint32_t x0 = w[2 * q], x1 = w[2 * q + 1];
+                const uint2 c0 = code_tab[(x0 >> 7) & 0xFFu];
+                const uint2 c1 = code_tab[(x0 >> 23) & 0xFFu];
+                const uint2 c2 = code_tab[(x1 >> 7) & 0xFFu];
+                const uint2 c3 = code_tab[(x1 >> 23) & 0xFFu];
+                const uint32_t l01 = c0.y + c1.y;
+                const uint32_t l012 = l01 + c2.y;
+                if (lb + l012 >= next_open) {
+                    const uint32_t k = lb >= next_open ? 0u : lb + c0.y >= next_open ? 1u
+                                                          : lb + l01 >= next_open ? 2u : 3u;
+                    const uint32_t s = lb + (k == 0 ? 0u : k == 1 ? c0.y : k == 2 ? l01 : l012);
+                    open(4 * q + k, s);
+                }
+                lb += l012 + c3.y;
+                out.put((c0.x << c1.y) | c1.x, l01);
+                out.put((c2.x << c3.y) | c3.x, c2.y + c3.y);
+            }
         } else {
 #pragma unroll
-            for (uint32_t k = 0; k < kElemsPerThread; k += 2) {
+            for (uint32_t k = 0; k < kElemsPerThread; ++k) {
                 if (k >= cnt)
                     break;
-                pair(k, k + 1 < cnt);
+                const uint2 c = code_tab[(w[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu];
+                if (lb >= next_open)
+                    open(k, lb);
+                lb += c.y;
+                out.put(c.x, c.y);
             }
         }
-        if (fill)
-            atomicOr(&sw[j], cur);                                // shared with the next thread
-        atomicAdd(&sc[cur_gi], cnt - run_k);
         // the end of the stream counts as a code start for the gap of its slice
-        if (e0 + cnt == p.n) {
-            const uint32_t gl = lb >> sh;
-            if (gS + (uint64_t)gl < p.n_threads && lb >= next_open) {
-                const uint32_t gi = gl + goff;
-                sgb[gi] = (uint8_t)(lb & slice_mask & 0xFu);
-            }
-        }
+        if (e0 + cnt == p.n && gS + (uint64_t)(lb >> sh) < p.n_threads && lb >= next_open)
+            open(cnt, lb);
         // sign|mantissa bytes
         if (cnt == kElemsPerThread) {
             uint32_t sm[8];
@@ -458,15 +483,27 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
     }
     if (bad && p.err)
         atomicOr(p.err, DF11_DEVERR_MISMATCH);
+    // The part-filled last word: the next thread of a full segment completes
+    // it, so ORed after the barrier; the last thread's is the segment's own
+    // last word, stored.  (The last segment's words start zeroed: its last
+    // threads may complete none.)
+    const uint32_t part = out.nb ? out.lo << (32u - out.nb) : 0u;
+    if (out.nb && !tail && tid == kEncThreads - 1)
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(out.sp), "r"(part) : "memory");
+    __syncthreads();
+    if (out.nb && (tail || tid != kEncThreads - 1))
+        asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(out.sp), "r"(part) : "memory");
     __syncthreads();
 
     // ---- staged words -> global: words that may be shared with the
     // neighbouring segments (the first and the last) are ORed in
     const uint64_t end_bit = S + seg_total;
+    if (seg == p.n_seg - 1 && tid == 0 && end_bit != p.total_bits && p.err)
+        atomicOr(p.err, DF11_DEVERR_MISMATCH);
     if (seg_total) {
         const uint32_t nw = (uint32_t)(((end_bit + 31) >> 5) - wbase);
         uint32_t *g32 = reinterpret_cast<uint32_t *>(p.stream) + wbase;
-        for (uint32_t i = threadIdx.x; i < nw; i += kEncThreads) {
+        for (uint32_t i = tid; i < nw; i += kEncThreads) {
             const uint32_t v = bswap32(sw[i]);
             if (i == 0 || i == nw - 1)
                 atomicOr(g32 + i, v);
@@ -474,34 +511,67 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncodeParams p, Cod
                 g32[i] = v;
         }
     }
+    // ---- slices: gaps, counts, chunk positions.  Staged slice gi is slice
+    // gbase * 8 + gi.  This segment's bits lie in staged slices [goff,
+    // gend), and its end bit in slice glend (gend - 1, or gend when the end
+    // bit starts a slice).  Its codes starting in slice gi are a(gi + 1) -
+    // a(gi), a(gi) = the element that opens slice gi if one of this
+    // segment's does, else 0 for the first slice (opened before the segment)
+    // and ne for slices past the segment's last code start (a(gend) = ne).
+    // The previous segment's end bit lies in slice goff and the next one's
+    // first bit in slice glend: words holding those two slices are ORed
+    // (gaps) or added (counts) into the zeroed arrays, the others stored.
     {
-        const uint64_t glast = (end_bit >> p.slice_shift) >> 3;   // the end may open a slice
-        const uint32_t ng = (uint32_t)(glast - gbase + 1);
+        const uint32_t goff = (uint32_t)(gS & 7u);
+        const uint32_t ne = (uint32_t)min((uint64_t)kSegElems, p.n - seg * kSegElems);
+        const uint32_t glend = (uint32_t)((end_bit >> sh) - gS) + goff;
+        const uint32_t gend = seg_total ? (uint32_t)(((end_bit - 1) >> sh) - gS) + 1 + goff : goff;
+        auto a_of = [&](uint32_t gi) -> uint32_t {
+            const uint32_t v = so[gi];
+            return (v & kOpened) ? (v & 0xFFFFu) : gi == goff ? 0u : ne;
+        };
         const uint64_t gwords = p.n_threads / 8;                  // gaps array length in words
         uint32_t *gg = reinterpret_cast<uint32_t *>(p.gaps) + gbase;
-        for (uint32_t i = threadIdx.x; i < ng && gbase + i < gwords; i += kEncThreads) {
-            // eight gap bytes (each < 16) -> eight nibbles, slice 8i + k at bits 4k
+        for (uint32_t i = tid; i <= glend / 8 && gbase + i < gwords; i += kEncThreads) {
+            // eight gap nibbles, slice 8i + k at bits 4k
             uint32_t v = 0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t x = sg[2 * i + h];
-                const uint32_t y = x | (x >> 4);                 // bytes 0, 2: two nibbles each
-                v |= ((y & 0xFFu) | ((y >> 8) & 0xFF00u)) << (16 * h);
-            }
-            if (i == 0 || i == ng - 1)
+            for (int k = 0; k < 8; ++k)
+                v |= ((so[8 * i + k] >> 16) & 0xFu) << (4 * k);
+            if (i == 0 || i == glend / 8)
                 atomicOr(gg + i, v);
             else
                 gg[i] = v;
         }
-        // counts: staged slice 4i + k at byte k of word i; slices this
-        // segment shares with its neighbours get all their contributions
-        // added (a count is at most 128, so bytes never carry)
+        // counts: slice 4i + k at byte k of word i (a count is at most 128,
+        // so bytes never carry)
         uint32_t *cc = reinterpret_cast<uint32_t *>(p.counts) + 2 * gbase;
         const uint64_t cwords = p.n_threads / 4;
-        for (uint32_t i = threadIdx.x; i < 2 * ng && 2 * gbase + i < cwords; i += kEncThreads) {
-            const uint32_t v = sc[4 * i] | (sc[4 * i + 1] << 8) | (sc[4 * i + 2] << 16) | (sc[4 * i + 3] << 24);
-            if (v)
-                atomicAdd(cc + i, v);
+        for (uint32_t i = goff / 4 + tid; gend > goff && i <= (gend - 1) / 4 && 2 * gbase + i < cwords;
+             i += kEncThreads) {
+            uint32_t v = 0;
+#pragma unroll
+            for (uint32_t k = 0; k < 4; ++k) {
+                const uint32_t gi = 4 * i + k;
+                if (gi >= goff && gi < gend) {
+                    const uint32_t a_next = gi + 1 < gend ? a_of(gi + 1) : ne;
+                    v |= (a_next - a_of(gi)) << (8 * k);
+                }
+            }
+            if (i == goff / 4 || i == glend / 4) {
+                if (v)
+                    atomicAdd(cc + i, v);
+            } else {
+                cc[i] = v;
+            }
+        }
+        // output position of every chunk whose first slice a code of this
+        // segment (or the end of the stream) opens
+        const uint32_t c0 = (uint32_t)((gbase * 8 + 31) / 32 * 32 - gbase * 8);   // first staged chunk start
+        for (uint32_t gi = c0 + 32 * tid; gi <= glend; gi += 32 * kEncThreads) {
+            const uint32_t v = so[gi];
+            if (v & kOpened)
+                p.chunk_pos[(gbase * 8 + gi) / DF11_THREADS_PER_CHUNK] = (uint32_t)(seg * kSegElems + (v & 0xFFFFu));
         }
     }
 }
@@ -510,13 +580,17 @@ bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>
 
 uint64_t n_segments(uint64_t n) { return (n + kSegElems - 1) / kSegElems; }
 
-// Scratch: segment starts (8 bytes per segment) | segment bits (4 bytes per
-// segment, rounded to 16) | group bits (2 bytes per 32 elements of every
-// segment).  The allocation-free path goes without the group bits.
+// Scratch: code table (1 KB) | segment bits (4 bytes per segment, rounded to 16) | run totals
+// (8 bytes per run of kRunSegs segments, rounded to 16) | group bits (2 bytes
+// per 32 elements of every segment).  The allocation-free path goes without
+// the group bits.
+constexpr uint64_t kTableBytes = 256 * 4;
+uint64_t run_bits_offset(uint64_t n) { return kTableBytes + ((n_segments(n) * 4 + 15) & ~15ull); }
+
 uint64_t segment_scratch_bytes(uint64_t n)
 {
-    const uint64_t ns = n_segments(n);
-    return ns * 8 + ((ns * 4 + 15) & ~15ull);
+    const uint64_t runs = (n_segments(n) + kRunSegs - 1) / kRunSegs;
+    return run_bits_offset(n) + ((runs * 8 + 15) & ~15ull);
 }
 
 df11_status compress_device_impl(const df11_codebook *cb, const df11_layout *layout, const uint16_t *d_in,
@@ -596,8 +670,9 @@ df11_status compress_device_impl(const df11_codebook *cb, const df11_layout *lay
     p.chunk_pos = const_cast<uint32_t *>(out->chunk_pos);
     p.signmant = const_cast<uint8_t *>(out->signmant);
     p.n_seg = n_segments(n);
-    p.seg_start = reinterpret_cast<uint64_t *>(d_scratch);
-    p.seg_bits = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(d_scratch) + p.n_seg * 8);
+    p.code_table = reinterpret_cast<uint32_t *>(d_scratch);
+    p.seg_bits = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(d_scratch) + kTableBytes);
+    p.run_bits = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(d_scratch) + run_bits_offset(n));
     p.grp_bits = group_bits ? reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(d_scratch) +
                                                            segment_scratch_bytes(n))
                             : nullptr;
@@ -616,12 +691,11 @@ df11_status compress_device_impl(const df11_codebook *cb, const df11_layout *lay
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return DF11_ERR_CUDA;
-    prepare_kernel<<<sms * 4, 256, 0, s>>>(p, z.exp_stream_bytes / 4, (z.gaps_bytes + 3) / 4,
-                                            z.n_chunks, z.signmant_bytes);
+    prepare_kernel<<<sms * 4, 256, 0, s>>>(p, ct, z.exp_stream_bytes / 4, (z.gaps_bytes + 3) / 4,
+                                                z.n_chunks, z.signmant_bytes);
     segment_bits_kernel<<<(unsigned)((p.n_seg + 7) / 8 < (uint64_t)sms * 8 ? (p.n_seg + 7) / 8 : (uint64_t)sms * 8),
-                          256, 0, s>>>(p, ct);
-    segment_scan_kernel<<<1, kScanThreads, 0, s>>>(p);
-    encode_kernel<<<(unsigned)p.n_seg, kEncThreads, 0, s>>>(p, ct);
+                          256, 0, s>>>(p);
+    encode_kernel<<<(unsigned)p.n_seg, kEncThreads, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess)
         return DF11_ERR_CUDA;
     out->hdr.max_code_len = cb->max_code_len;
