@@ -72,9 +72,11 @@ def parse_args():
     ap.add_argument("--tokens", default=None,
                     help="comma-separated token counts of the activations (llama8b_overlap: "
                          "default 1,256,2048,8192; llama8b_gemv: default 1,4,8)")
-    ap.add_argument("--max-ctas", default="0,1184",
+    ap.add_argument("--runs", type=int, default=10,
+                    help="llama8b_overlap: repetitions of every measurement (median and range reported)")
+    ap.add_argument("--max-ctas", default="0,148,74",
                     help="llama8b_overlap: comma-separated decode CTA counts (0 = one resident "
-                         "wave; large = one short-lived CTA per 16 chunks)")
+                         "wave on every SM; 148 or 74 leave part of the SMs to the products)")
     ap.add_argument("--consumer-priority", type=int, default=-1,
                     help="llama8b_overlap: CUDA priority of the consumer stream (lower = higher)")
     ap.add_argument("--scale-div", type=int, default=1,
@@ -521,7 +523,8 @@ def integrity_figures(df11, dev, stream, hb, db, cb, out, w_dev, ws, scrub, laun
 
 
 def per_config(df11, dev, stream, bpt, peak, headline=None):
-    """Every configuration decoded on this GPU: bit-exactness against the
+    """Every configuration decoded on this GPU, each single block in the slice
+    layout the library prefers for it: bit-exactness against the
     input, then its device time per launch from CUDA-graph replays
     (graph_us): back to back, and for single blocks from an L2 scrubbed by a
     256 MB write before each launch.  Config 3 times the 32-block stream
@@ -532,6 +535,7 @@ def per_config(df11, dev, stream, bpt, peak, headline=None):
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     ws = torch.zeros(df11.SCHED_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
     scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     out_all = {}
     for key, name in PER_CONFIG:
         t0 = time.perf_counter()
@@ -550,7 +554,11 @@ def per_config(df11, dev, stream, bpt, peak, headline=None):
         else:
             mats = [m for _, m in workloads.WORKLOADS[name]()]
             w = np.concatenate([m.reshape(-1) for m in mats])
-            hb = df11.compress(df11.build_codebook(mats), mats, 32, bpt)
+            cbk = df11.build_codebook(mats)
+            # each block in the slice layout the library prefers for it
+            # (16 bytes for the large blocks, 8 for small or 1-bit-code ones)
+            bpt_c = df11.preferred_bytes_per_thread(cbk, sms)
+            hb = df11.compress(cbk, mats, 32, bpt_c)
             db = hb.to_device(dev)
             cb = db.c_struct()
             n = hb.n_elements
@@ -569,7 +577,7 @@ def per_config(df11, dev, stream, bpt, peak, headline=None):
             del w, hb, w_dev
         setup_s = time.perf_counter() - t0
         entry = {"workload": name, "n_weights": n, "bytes_per_launch": nbytes, "bit_exact": exact,
-                 "setup_s": round(setup_s, 1)}
+                 "bytes_per_thread": bpt if name == "llama8b_model" else bpt_c, "setup_s": round(setup_s, 1)}
         entry["back_to_back"] = _rates(nbytes, n, graph_us(launch, k), peak)
         if name != "llama8b_model":
             entry["l2_scrubbed"] = _rates(nbytes, n, graph_us(launch, max(k // 4, 5), scrub=scrub), peak)
@@ -919,7 +927,9 @@ def run_overlap(args):
                 order: decode just before the block runs);
       overlap - the pipeline: block i+1 decodes on its own stream while the
                 products of block i run, two output slots.
-    hidden = (serial - overlap) / decode: the share of decode time hidden."""
+    hidden = (serial - overlap) / decode: the share of decode time hidden.
+    Each measurement is repeated --runs times, interleaved (every variant
+    once per run), and reported as the median with its range."""
     import torch
 
     import huffman_decode_b200 as df11
@@ -1003,20 +1013,29 @@ def run_overlap(args):
             return fn
 
         reps = max(1, args.steps)
-        t_dec = timed(run_decode, reps)
-        t_gemm = timed(run_gemm, reps)
-        t_ser = timed(run_serial, reps)
-        ref = [t.clone() for t in y]
-        row = {"tokens": T, "decode_ms": round(t_dec, 4), "gemm_ms": round(t_gemm, 4),
+        variants = [(c, w) for c in cap_list for w in (True, False)]
+        samples = {"decode": [], "gemm": [], "serial": [], **{v: [] for v in variants}}
+        same = True
+        for run in range(max(1, args.runs)):
+            samples["decode"].append(timed(run_decode, reps))
+            samples["gemm"].append(timed(run_gemm, reps))
+            samples["serial"].append(timed(run_serial, reps))
+            ref = [t.clone() for t in y]
+            for v in variants:
+                samples[v].append(timed(run_overlap_cap(*v), reps))
+                same = same and all(torch.equal(a, b) for a, b in zip(ref, y))
+        med = {k: float(np.median(v)) for k, v in samples.items()}
+        t_dec, t_gemm, t_ser = med["decode"], med["gemm"], med["serial"]
+        row = {"tokens": T, "runs": max(1, args.runs), "decode_ms": round(t_dec, 4), "gemm_ms": round(t_gemm, 4),
                "serial_ms": round(t_ser, 4), "overlap": []}
-        for cap, claimed in [(c, w) for c in cap_list for w in (True, False)]:
-            t_ov = timed(run_overlap_cap(cap, claimed), reps)
-            same = all(torch.equal(a, b) for a, b in zip(ref, y))
+        for cap, claimed in variants:
+            hid = [(s_ - o) / d for s_, o, d in zip(samples["serial"], samples[(cap, claimed)], samples["decode"])]
             row["overlap"].append({
                 "max_ctas": cap, "schedule": "claimed tail" if claimed else "static",
-                "overlap_ms": round(t_ov, 4),
-                "hidden_frac": round((t_ser - t_ov) / t_dec, 4),
-                "overhead_vs_bf16": round(t_ov / t_gemm, 4),
+                "overlap_ms": round(med[(cap, claimed)], 4),
+                "hidden_frac": round(float(np.median(hid)), 4),
+                "hidden_frac_range": [round(min(hid), 4), round(max(hid), 4)],
+                "overhead_vs_bf16": round(med[(cap, claimed)] / t_gemm, 4),
                 "outputs_equal_serial": bool(same)})
         flops = 2.0 * T * offs[-1] * n_blocks
         row["gemm_tflops"] = round(flops / (t_gemm * 1e-3) / 1e12, 1)

@@ -13,5 +13,6 @@ from .df11 import (  # noqa: F401
     selftest_bounded_wait,
     build_codebook_from_histogram, build_decode_table, chunk_sums, decompress_verified_async, compress, compress_device, compress_device_noalloc,
     compress_device_scratch_bytes,
-    compress_sizes, decompress_async, histogram_device, library_path, load_library, validate,
+    compress_sizes, decompress_async, histogram_device, library_path, load_library, preferred_bytes_per_thread,
+    validate,
 )

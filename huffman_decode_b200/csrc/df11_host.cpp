@@ -351,6 +351,21 @@ df11_status df11_build_codebook_from_histogram(const uint64_t hist[256], uint32_
     return DF11_OK;
 }
 
+extern "C" uint32_t df11_preferred_bytes_per_thread(const df11_codebook *cb, uint32_t sm_count)
+{
+    if (!cb || cb->total_bits == 0 || sm_count == 0)
+        return 0;
+    uint32_t shortest = DF11_MAX_CODE_LEN;
+    for (int s = 0; s < 256; ++s)
+        if (cb->code_len[s] && cb->code_len[s] < shortest)
+            shortest = cb->code_len[s];
+    if (shortest == 1)
+        return 8;
+    const uint64_t chunk_bits = (uint64_t)DF11_THREADS_PER_CHUNK * 8 * 16;
+    const uint64_t chunks = (cb->total_bits + chunk_bits - 1) / chunk_bits;
+    return chunks < (uint64_t)sm_count * DF11_DECODE_WARPS_PER_SM ? 8u : 16u;
+}
+
 df11_status df11_compress_sizes(const df11_codebook *cb, const df11_layout *layout,
                                 df11_sizes *out)
 {

@@ -55,6 +55,7 @@ EXPORTED_SYMBOLS = (
     "df11_decode_gemv_async", "df11_decompress_async_ws", "df11_decompress_range_async",
     "df11_selftest_bounded_wait", "df11_serialized_bytes", "df11_serialize", "df11_deserialize",
     "df11_build_decode_table", "df11_chunk_sums", "df11_decompress_verified_async",
+    "df11_preferred_bytes_per_thread",
 )
 SCHED_WORKSPACE_BYTES = 2048
 CRC_SEGMENT_BYTES = 4096
@@ -191,6 +192,7 @@ def load_library(path: str | None = None):
         ("df11_build_decode_table", S, [P, U32, U32, P]),
         ("df11_chunk_sums", S, [P, P, U64]),
         ("df11_decompress_verified_async", S, [P, P, U64, P, P, P, P, P]),
+        ("df11_preferred_bytes_per_thread", U32, [P, U32]),
     ):
         fn = getattr(lib, name)
         fn.restype = res
@@ -227,6 +229,19 @@ def build_codebook(mats, max_code_len: int = MAX_CODE_LEN) -> Codebook:
     _check(load_library().df11_build_codebook(ptrs, numel, len(arrs), max_code_len,
                                                ctypes.byref(cb)), "df11_build_codebook")
     return cb
+
+
+def preferred_bytes_per_thread(cb: Codebook, sm_count: int | None = None) -> int:
+    """df11_preferred_bytes_per_thread: the slice width (8 or 16 bytes per
+    thread) this library decodes the block fastest with on a GPU of sm_count
+    SMs (default: the current CUDA device's)."""
+    if sm_count is None:
+        import torch
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    v = int(load_library().df11_preferred_bytes_per_thread(ctypes.byref(cb), int(sm_count)))
+    if v == 0:
+        raise ValueError("empty codebook or sm_count == 0")
+    return v
 
 
 def compress_sizes(cb: Codebook, threads_per_chunk: int = THREADS_PER_CHUNK,

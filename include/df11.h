@@ -211,6 +211,17 @@ df11_status df11_build_codebook_from_histogram(const uint64_t histogram[256], ui
 df11_status df11_compress_sizes(const df11_codebook *cb, const df11_layout *layout,
                                 df11_sizes *out);
 
+/* Host.  The slice width this library decodes a block fastest with: 8 bytes
+ * per thread (the pages' layout, "Architecture") when the block's shortest
+ * code is 1 bit -- 16-byte slices of 1-bit codes need twice the decoder's
+ * per-warp buffers, so half the warps fit -- or when the block has fewer
+ * 16-byte-slice chunks than the decoder keeps warps resident on sm_count
+ * SMs (DF11_DECODE_WARPS_PER_SM each): shorter chunks then finish sooner and
+ * spread over more warps; otherwise 16.  Returns 0 for a null or empty
+ * codebook or sm_count == 0. */
+#define DF11_DECODE_WARPS_PER_SM 46u
+uint32_t df11_preferred_bytes_per_thread(const df11_codebook *cb, uint32_t sm_count);
+
 /* Host.  Encodes one block ("Architecture": Gaps, BlockOutputPos; "How it
  * works": encode).  `out` carries caller buffers of at least the sizes
  * df11_compress_sizes reports; the call fills them and out->hdr.  The

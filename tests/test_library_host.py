@@ -637,3 +637,24 @@ def test_decode_table_reads_malformed_tables_as_no_code():
         df11.build_decode_table(hb.lut, nt, 0)
     with pytest.raises(df11.DF11Error):
         df11.build_decode_table(hb.lut, nt, 17)
+
+
+def test_preferred_bytes_per_thread_rule():
+    """8-byte slices for a 1-bit shortest code or a block with fewer 16-byte
+    chunks than the decoder's resident warps; 16 otherwise (the rule
+    include/df11.h states)."""
+    one_bit = [m for _, m in workloads.single_exponent(4002, (256, 256))]
+    assert df11.preferred_bytes_per_thread(df11.build_codebook(one_bit), 148) == 8
+    small = [m for _, m in workloads.single_matrix(0)]
+    cb = df11.build_codebook(small)
+    assert min(l for l in cb.lengths() if l) >= 2
+    chunks16 = -(-int(cb.total_bits) // (32 * 128))
+    assert chunks16 < 148 * 46
+    assert df11.preferred_bytes_per_thread(cb, 148) == 8
+    # the same codebook on a GPU with few SMs: enough chunks for every warp
+    sm_few = chunks16 // 46
+    assert df11.preferred_bytes_per_thread(cb, sm_few) == 16
+    assert df11.preferred_bytes_per_thread(cb, sm_few + 1) == 8
+    lib = df11.load_library()
+    assert lib.df11_preferred_bytes_per_thread(None, 148) == 0
+    assert lib.df11_preferred_bytes_per_thread(ctypes.byref(cb), 0) == 0
