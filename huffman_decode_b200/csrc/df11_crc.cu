@@ -208,25 +208,47 @@ __global__ void __launch_bounds__(kCrcThreads) crc_kernel(ArrayView av, uint32_t
         const uint32_t n = (uint32_t)(rem < kSeg ? rem : kSeg);
         uint32_t c = 0;
         if (n == (uint32_t)kSeg) {
-            // a full segment: lane l folds bytes [128 l, 128 l + 128), all
-            // eight loads in flight first; then a five-level tree in which
-            // lanes 2^(j+1) i join the CRC of the 128 * 2^j bytes after
-            // their own (lane 0 ends with the segment's)
-            uint4 v[kLaneBytes / 16];
+            // a full segment: lane l folds the four 32-byte runs l, l + 32,
+            // l + 64 and l + 96 (bytes 32 l + 1024 k), so each load
+            // instruction reads 1 KB of contiguous bytes, as four independent
+            // chains; joins them (advancing over the 1 KB between runs);
+            // then a five-level tree in which lanes 2^(j+1) i join the value
+            // of the lane 2^j on, advanced over 32 * 2^j bytes (lane 0 ends
+            // with the segment's)
+            uint32_t v[kLaneBytes / 4];
+            const uint8_t *src = base + 32 * lane;
+            if ((reinterpret_cast<uintptr_t>(aptr) & 31u) == 0) {
 #pragma unroll
-            for (int i = 0; i < kLaneBytes / 16; ++i)
-                v[i] = __ldg(reinterpret_cast<const uint4 *>(base + kLaneBytes * lane) + i);
+                for (int k = 0; k < 4; ++k)
+                    asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                                 : "=r"(v[8 * k]), "=r"(v[8 * k + 1]), "=r"(v[8 * k + 2]), "=r"(v[8 * k + 3]),
+                                   "=r"(v[8 * k + 4]), "=r"(v[8 * k + 5]), "=r"(v[8 * k + 6]), "=r"(v[8 * k + 7])
+                                 : "l"(src + 1024 * k));
+            } else {
 #pragma unroll
-            for (int i = 0; i < kLaneBytes / 16; ++i) {
-                c = fold_word(lane_priv, c, v[i].x);
-                c = fold_word(lane_priv, c, v[i].y);
-                c = fold_word(lane_priv, c, v[i].z);
-                c = fold_word(lane_priv, c, v[i].w);
+                for (int k = 0; k < 8; ++k) {
+                    const uint4 q = __ldg(reinterpret_cast<const uint4 *>(src + 1024 * (k >> 1)) + (k & 1));
+                    v[4 * k] = q.x;
+                    v[4 * k + 1] = q.y;
+                    v[4 * k + 2] = q.z;
+                    v[4 * k + 3] = q.w;
+                }
             }
+            uint32_t r[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    r[k] = fold_word(lane_priv, r[k], v[8 * k + w]);
+            }
+            c = r[0];
+#pragma unroll
+            for (int k = 1; k < 4; ++k)
+                c = advance(ops + 10 * 1024, c) ^ r[k];         // S_10: over 1024 zero bytes
 #pragma unroll
             for (int j = 0; j < 5; ++j) {
                 const uint32_t right = __shfl_down_sync(0xFFFFFFFFu, c, 1 << j);
-                c = advance(ops + (7 + j) * 1024, c) ^ right;   // S_{7+j}: over 128 * 2^j zero bytes
+                c = advance(ops + (5 + j) * 1024, c) ^ right;   // S_{5+j}: over 32 * 2^j zero bytes
             }
         } else {
             // the short last segment of an array: lanes fold what they have,

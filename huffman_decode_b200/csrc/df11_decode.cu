@@ -9,45 +9,53 @@
 //
 // B200 design (differs from the page's kernel):
 //   * one warp = one chunk: output positions are stored per 32 threads, so
-//     every warp counts, scans (shuffles), decodes and stores on its own,
-//     with no block-wide barrier after the prologue (the claimed schedule
-//     below adds one at the very end, to count the CTA out);
-//   * two passes over the lane's slice, as on the page (count, then decode
-//     and write), both with a multi-code table: an 11-bit window indexes a
-//     2048-entry table (built in shared memory from the format's two-level
-//     16-bit tables) that yields up to four whole codes per lookup; longer
-//     codes fall back to the two-level tables;
-//   * the second pass writes each lane's exponents straight to their place
-//     in a contiguous, 8-element-aligned per-warp exponent buffer: four per
-//     word, ORed into the zeroed buffer, since a lane's first and last words
-//     are shared with its neighbours.  A lane's last lookup may also decode
-//     the next lane's first codes; they come from the same bit position, so
-//     ORing them again changes nothing.  No staging columns, no compaction:
-//     a warp needs 4.1 KB of shared memory instead of 6.3 KB;
+//     every warp scans, decodes and stores on its own, with no block-wide
+//     barrier after the prologue (the claimed schedule below adds one at
+//     the very end, to count the CTA out);
+//   * one decode pass instead of the page's two: the format stores each
+//     thread's code count, so a warp scan of the stored counts (shuffles)
+//     gives each lane its output offset before it decodes, and the lane
+//     decodes its slice once, writing its exponents four per 32-bit word
+//     straight into place in a contiguous, 8-element-aligned per-warp
+//     exponent buffer.  Full chunks of 128-bit slices store plain words
+//     (every lane's first word lands before any lane's third segment, and
+//     each lane's part-filled last word is ORed over its neighbour's first
+//     at the end); 64-bit slices and the block's last chunk OR into a zeroed
+//     buffer.  A tail check confirms that each lane decoded exactly its
+//     stored count and ended where the next code starts;
+//   * up to four codes per lookup: an 11-bit window indexes a 2048-entry
+//     table (built once on the host, or in shared memory from the format's
+//     two-level 16-bit tables); longer codes fall back to the two-level
+//     tables.  The lane state packs the bit position and the fill of the
+//     word being built, so one add steps both;
 //   * exponents travel rotated right by one bit (bit 0 on top), which is
 //     where the BF16 halves want them: the merge is two bit-selects and two
-//     byte permutes per four weights, with no shifts;
+//     byte permutes per four weights, with no shifts, and one 16-byte store
+//     per lane and group;
 //   * the chunk's sign|mantissa bytes are staged into shared memory by one
-//     TMA bulk copy (cp.async.bulk + mbarrier) issued before decoding; the
-//     next chunk's stream words are loaded into registers a chunk ahead;
+//     TMA bulk copy (cp.async.bulk + mbarrier) issued before decoding, and
+//     the tables by bulk copies in the prologue; the next chunk's stream
+//     words, counts and positions are loaded into registers a chunk ahead;
 //   * per-warp buffers are sized by the codebook's shortest code (the kernel
 //     rejects table entries shorter than it), so blocks whose codes are at
 //     least 2 bits long fit twice as many warps per SM;
-//   * the merge builds four BF16 values with two bit-selects and two byte
-//     permutes and writes one 16-byte vector per lane and group;
-//   * persistent CTAs, grid = resident CTAs per SM x SM count: one CTA of up
-//     to 32 warps per SM, or two of up to 23 (a 40-register build), whichever
-//     keeps more warps resident -- two 23-warp CTAs for typical blocks;
+//   * persistent CTAs, grid = resident CTAs per SM x SM count: two CTAs of
+//     23 warps per SM (a 40-register build, 46 warps) or one of up to 32,
+//     whichever keeps more warps resident; a block smaller than one full CTA
+//     per SM gets one CTA per SM of just enough warps;
 //   * with a scheduling workspace, the last few rounds of chunks are not
 //     dealt out but claimed one at a time from four global counters (each
 //     warp claims a chunk ahead, so the atomic's latency hides behind a
 //     decode): warps and SMs that ran slower take fewer of them and all
 //     finish within about one chunk of each other.  Claiming only the tail
 //     keeps the atomics off the memory system for most of the launch.  The
-//     last CTA out resets the counters.
+//     last CTA out resets the counters;
+//   * optionally (the verifying build) every chunk's bytes are summed as
+//     they are read and checked against a per-chunk list.
 // Also here: decoding a chunk range alone (df11_decompress_range_async), the
-// fused matrix-vector products (df11_decode_gemv_async), the bounded-wait
-// self-test, and the run-time bound checks of the checked build.
+// verifying decode (df11_decompress_verified_async), the fused matrix-vector
+// products (df11_decode_gemv_async), the bounded-wait self-test, and the
+// run-time bound checks of the checked build.
 // No tensor cores: this is integer decode, bounded by HBM traffic and issue.
 #include "df11.h"
 
@@ -1169,7 +1177,8 @@ struct LaunchShape {
 // own CTA size, `cached`; other sizes give a grid of max_ctas.
 template <int W, int MINLEN, typename Kernel>
 df11_status shape_launch(Kernel kernel, int v, const DecodeParams &prm, int dev, uint32_t max_ctas,
-                         int max_warps, int cps, LaunchShape &ls, bool cached = true)
+                         int max_warps, int cps, LaunchShape &ls, bool cached = true,
+                         int carveout = (int)cudaSharedmemCarveoutMaxShared)
 {
     DeviceProps d;
     if (device_props(dev, d) != DF11_OK)
@@ -1184,8 +1193,8 @@ df11_status shape_launch(Kernel kernel, int v, const DecodeParams &prm, int dev,
     if (!g_attr_done[dev][v].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+            cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carveout) !=
+                cudaSuccess)
             return DF11_ERR_CUDA;
         g_attr_done[dev][v].store(1, std::memory_order_release);
     }
@@ -1255,13 +1264,20 @@ df11_status launch(const DecodeParams &prm, int dev, cudaStream_t stream, uint32
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
+// The fused products' one CTA per SM needs about two thirds of the shared
+// memory; asking for no more leaves the rest to L1, which then holds the
+// activation rows the warps read over and over (2-4% faster than the
+// largest shared-memory split).
+constexpr int kGemvCarveout = 70;   // percent of the SM's shared memory
+
 template <int W, int MINLEN, int TT>
 df11_status launch_gemv(const DecodeParams &prm, const GemvParams &gp, int dev, cudaStream_t stream)
 {
     auto kernel = df11_gemv_kernel<W, MINLEN, TT>;
     constexpr int v = variant_base<W, MINLEN>() + (TT == 1 ? 1 : TT == 2 ? 2 : TT == 4 ? 3 : 4);
     LaunchShape ls;
-    const df11_status st = shape_launch<W, MINLEN>(kernel, v, prm, dev, 0, kMaxWarpsPerCta, 1, ls);
+    const df11_status st =
+        shape_launch<W, MINLEN>(kernel, v, prm, dev, 0, kMaxWarpsPerCta, 1, ls, true, kGemvCarveout);
     if (st != DF11_OK)
         return st;
     kernel<<<ls.grid, ls.warps * 32, ls.smem, stream>>>(prm, gp);

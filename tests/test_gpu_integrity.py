@@ -313,3 +313,31 @@ def test_verified_decode_full_block():
             assert err == 0 and first == -1, (a, byte)
         else:
             assert err != 0 and first in allowed, (a, byte, err, first, allowed)
+
+
+def test_checksum_of_arrays_only_16_byte_aligned():
+    """The GPU checksum list of a block whose every array starts 16 bytes
+    past a 32-byte boundary (the kernel's 16-byte load path) equals the
+    oracle's, and verification and decode work on it."""
+    hb = _block("llama_div256")
+    aligned = hb.to_device("cuda")
+    t = {}
+    for a in ARRAYS:
+        raw = aligned.tensors[a]
+        buf = torch.zeros(raw.numel() + 64, dtype=torch.uint8, device="cuda")
+        off = (16 - buf.data_ptr() % 32) % 32
+        view = buf[off: off + raw.numel()]
+        assert view.data_ptr() % 32 == 16
+        view.copy_(raw)
+        t[a] = view
+    db = df11.DeviceBlock(header=aligned.header, tensors=t, sizes=aligned.sizes,
+                          matrix_numel=aligned.matrix_numel)
+    got = df11.checksum_device(db)
+    torch.cuda.synchronize()
+    ref = _oracle_list(hb)
+    assert np.array_equal(got.cpu().numpy().view(np.uint32), ref)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    first = torch.full((1,), -1, dtype=torch.int64, device="cuda")
+    df11.verify_device(db, torch.from_numpy(ref.view(np.int32)).cuda(), err, first)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and int(first.item()) == -1
