@@ -519,7 +519,9 @@ df11_status df11_verify_device_async(const df11_device_block *blk, const uint32_
  * covered (it is derived from the tables). */
 
 /* Host.  Writes the n_chunks per-chunk sums of blk into sums[0 .. n).
- * INVALID_ARGUMENT for null pointers or n != blk->hdr.n_chunks. */
+ * INVALID_ARGUMENT for null pointers, n != blk->hdr.n_chunks, a layout the
+ * library does not decode, arrays shorter than the header implies, or
+ * positions that decrease or pass the sign|mantissa bytes. */
 df11_status df11_chunk_sums(const df11_host_block *blk, uint32_t *sums, uint64_t n);
 
 /* GPU.  df11_decompress_range_async over the whole block (chunk_begin = 0,
@@ -528,7 +530,10 @@ df11_status df11_chunk_sums(const df11_host_block *blk, uint32_t *sums, uint64_t
  * df11_chunk_sums): a mismatch ORs DF11_DEVERR_CHECKSUM into *d_error.  A
  * chunk is bad when its sum differs or its decode reports an error (its
  * flag); when d_first_bad (device uint64, 8-byte aligned, set to UINT64_MAX
- * by the caller) is given, it is lowered to the lowest bad chunk.  Chunks of
+ * by the caller) is given, it is lowered to the lowest bad chunk.  A damaged
+ * byte is reported at its own chunk or at the chunk before it, which also
+ * reads the next chunk's first stream word (codes that cross into it) and
+ * its first thread's gap.  workspace: as for df11_decompress_async_ws.  Chunks of
  * a CTA whose tables never arrived are neither decoded nor summed (that
  * sets DF11_DEVERR_TIMEOUT).  The output is written as by
  * df11_decompress_async.  Errors: those of df11_decompress_async_ws, and
