@@ -430,8 +430,30 @@ __device__ __forceinline__ int gemv_matrix_of(const GemvParams *gp, uint32_t e)
     return lo;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+// acc + w * x for BF16 w and x (each the low or high half of a 32-bit
+// word) in one FP32 fused multiply-add.  A product of two BF16 values is
+// exact in FP32, so this equals fmaf(float(w), float(x), acc), bit for bit;
+// the halves are read in place, with no conversion instructions.
+__device__ __forceinline__ float fma_bf16_lo(uint32_t w, uint32_t x, float acc)
+{
+    asm("{ .reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %1;\n\t"
+        "mov.b32 {xl, xh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
+        "}"
+        : "+f"(acc) : "r"(w), "r"(x));
+    return acc;
+}
+__device__ __forceinline__ float fma_bf16_hi(uint32_t w, uint32_t x, float acc)
+{
+    asm("{ .reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %1;\n\t"
+        "mov.b32 {xl, xh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, wh, xh, %0;\n\t"
+        "}"
+        : "+f"(acc) : "r"(w), "r"(x));
+    return acc;
+}
 
 // Adds the chunk's products to y.  The groups of 8 elements that touch
 // the chunk's range [head, head + n_write) (relative to base, 8-aligned)
@@ -441,8 +463,11 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 // partial sum per token, and a warp sum adds each token's total to y with
 // one atomic add.  Matrix and row are located once per chunk and then
 // stepped.  In the first and last groups only the chunk's own elements
-// count.  ebuf holds the chunk's rotated exponents, sgrp its
-// sign|mantissa bytes (group 0 of the chunk at offset 0 of both).
+// count: their other bytes are zeroed first, in both buffers, which makes
+// those weights +0 (exactly what masking them would give), so the product
+// loop has no end cases.  ebuf holds the chunk's rotated exponents, sgrp
+// its sign|mantissa bytes (group 0 of the chunk at offset 0 of both); the
+// staged copy has landed, and both are this warp's own.
 template <int TT>
 __device__ __forceinline__ void gemv_chunk(const GemvParams *gp, uint32_t head, uint32_t n_write, uint64_t base,
                                            int lane, uint32_t ebuf_a, uint32_t sgrp_a)
@@ -452,6 +477,22 @@ __device__ __forceinline__ void gemv_chunk(const GemvParams *gp, uint32_t head, 
     const uint32_t ngroups = (span + 7) >> 3;
     if (ngroups == 0)
         return;
+    {
+        // lanes 0..7: bytes [0, head) of group 0; lanes 8..15: bytes
+        // [span, 8 ngroups) of the last group
+        const uint32_t j = lane < 8 ? (uint32_t)lane : span + (uint32_t)lane - 8u;
+        const uint32_t lim = lane < 8 ? head : 8u * ngroups;
+        if (lane < 16 && j < lim) {
+            asm volatile("st.shared.u8 [%0], %1;" ::"r"(ebuf_a + j), "r"(0u) : "memory");
+            asm volatile("st.shared.u8 [%0], %1;" ::"r"(sgrp_a + j), "r"(0u) : "memory");
+        }
+        __syncwarp();
+        // the product loop's shared loads are plain (schedulable) asm: route
+        // their base addresses through ordered asm so no load can be placed
+        // above these stores
+        asm volatile("mov.b32 %0, %0;" : "+r"(ebuf_a)::"memory");
+        asm volatile("mov.b32 %0, %0;" : "+r"(sgrp_a)::"memory");
+    }
     // matrix, row and column of group 0
     int m = gemv_matrix_of(gp, (uint32_t)base);
     uint32_t cols = gp->m[m].cols, rows = gp->m[m].rows;
@@ -471,7 +512,7 @@ __device__ __forceinline__ void gemv_chunk(const GemvParams *gp, uint32_t head, 
 #pragma unroll
         for (int t = 0; t < TT; ++t)
             acc[t] = 0.f;
-        // The buffers were filled before the warp's last __syncwarp, which
+        // The buffers were written before the warp's last __syncwarp, which
         // orders these plain shared loads; the activation loads go first so
         // their latency overlaps the weight assembly.
 #pragma unroll(TT <= 2 ? 2 : 1)
@@ -485,20 +526,8 @@ __device__ __forceinline__ void gemv_chunk(const GemvParams *gp, uint32_t head, 
                                     : make_uint4(0u, 0u, 0u, 0u);
             const uint2 e8 = lds_v2(ebuf_a + 8u * i);
             const uint2 s8 = lds_v2(sgrp_a + 8u * i);
-            uint2 wa = join4(e8.x, s8.x);
-            uint2 wb = join4(e8.y, s8.y);
-            if (i == 0 || i + 1 == ngroups) {
-                // a group at an end of the chunk: zero the weights outside it
-                const uint32_t lo = i == 0 ? head : 0u;
-                const uint32_t hi = min(8u, span - 8u * i);
-                const uint32_t keep = (0xFFu >> (8 - hi)) & (0xFFu << lo);   // element mask
-                wa.x &= ((keep & 1u) ? 0x0000FFFFu : 0u) | ((keep & 2u) ? 0xFFFF0000u : 0u);
-                wa.y &= ((keep & 4u) ? 0x0000FFFFu : 0u) | ((keep & 8u) ? 0xFFFF0000u : 0u);
-                wb.x &= ((keep & 16u) ? 0x0000FFFFu : 0u) | ((keep & 32u) ? 0xFFFF0000u : 0u);
-                wb.y &= ((keep & 64u) ? 0x0000FFFFu : 0u) | ((keep & 128u) ? 0xFFFF0000u : 0u);
-            }
-            const float w0 = bf16_lo(wa.x), w1 = bf16_hi(wa.x), w2 = bf16_lo(wa.y), w3 = bf16_hi(wa.y);
-            const float w4 = bf16_lo(wb.x), w5 = bf16_hi(wb.x), w6 = bf16_lo(wb.y), w7 = bf16_hi(wb.y);
+            const uint2 wa = join4(e8.x, s8.x);   // weights 0, 1 | 2, 3 of the group
+            const uint2 wb = join4(e8.y, s8.y);   // weights 4, 5 | 6, 7
 #pragma unroll
             for (int t0 = 0; t0 < TT; t0 += TP) {
 #pragma unroll
@@ -513,14 +542,14 @@ __device__ __forceinline__ void gemv_chunk(const GemvParams *gp, uint32_t head, 
                     if (t < (int)nt) {
                         const uint4 xv_t = xv[u];
                         float a = acc[t];
-                        a = fmaf(w0, bf16_lo(xv_t.x), a);
-                        a = fmaf(w1, bf16_hi(xv_t.x), a);
-                        a = fmaf(w2, bf16_lo(xv_t.y), a);
-                        a = fmaf(w3, bf16_hi(xv_t.y), a);
-                        a = fmaf(w4, bf16_lo(xv_t.z), a);
-                        a = fmaf(w5, bf16_hi(xv_t.z), a);
-                        a = fmaf(w6, bf16_lo(xv_t.w), a);
-                        a = fmaf(w7, bf16_hi(xv_t.w), a);
+                        a = fma_bf16_lo(wa.x, xv_t.x, a);
+                        a = fma_bf16_hi(wa.x, xv_t.x, a);
+                        a = fma_bf16_lo(wa.y, xv_t.y, a);
+                        a = fma_bf16_hi(wa.y, xv_t.y, a);
+                        a = fma_bf16_lo(wb.x, xv_t.z, a);
+                        a = fma_bf16_hi(wb.x, xv_t.z, a);
+                        a = fma_bf16_lo(wb.y, xv_t.w, a);
+                        a = fma_bf16_hi(wb.y, xv_t.w, a);
                         acc[t] = a;
                     }
                 }
@@ -934,23 +963,23 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                                                    accl, r);
             }
             if (cnt) {
-                // codes of the last entry that start at or past `end` are the
+                // Codes of the last entry that start at or past `end` are the
                 // next lane's; the first of them (or the end of the entry) is
-                // where the next code starts
+                // where the next code starts.  The entry's code starts c0 <=
+                // c1 <= c2 <= c3 never fall (lengths are unsigned), so the
+                // codes that pass `end` are a suffix and the next start is the
+                // lowest start at or past it.
                 const uint32_t emitted = sp - ebuf_a + (X >> (kFillShift + 3)) - a;
                 const uint32_t n = entry_codes(r.y);
-                int c = (int)(X & 0xFFFFu) - (int)(r.y & 0xFFFFu);   // start of the entry's first code
-                uint32_t keep = n ? 1u : 0u;
-                int next_start = (int)(X & 0xFFFFu);
-#pragma unroll
-                for (uint32_t k = 1; k < (uint32_t)kMaxCodesPerEntry; ++k) {
-                    c += (int)lds_u8(len_a + ((r.x >> (8 * (k - 1))) & 0xFFu));
-                    if (k < n && c < end)
-                        ++keep;
-                    else if (k == keep && k < n)
-                        next_start = c;
-                }
-                lane_bad = emitted - (n - keep) != cnt || next_start != expect;
+                const int pos = (int)(X & 0xFFFFu);
+                const int c0 = pos - (int)(r.y & 0xFFFFu);   // start of the entry's first code
+                const int c1 = c0 + (int)lds_u8(len_a + (r.x & 0xFFu));
+                const int c2 = c1 + (int)lds_u8(len_a + ((r.x >> 8) & 0xFFu));
+                const int c3 = c2 + (int)lds_u8(len_a + ((r.x >> 16) & 0xFFu));
+                const bool p1 = n > 1u && c1 >= end, p2 = n > 2u && c2 >= end, p3 = n > 3u && c3 >= end;
+                const uint32_t passed = (uint32_t)p1 + (uint32_t)p2 + (uint32_t)p3;
+                const int next_start = p1 ? c1 : p2 ? c2 : p3 ? c3 : pos;
+                lane_bad = emitted - passed != cnt || next_start != expect;
             }
             __syncwarp();
             // the part-filled last word: ORed over the next lane's first word
@@ -990,10 +1019,17 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                 const uint32_t mend = span >> 3;                   // whole groups end
                 const uint32_t sgrp_a = sbuf_a + (pos0 & 8u);     // group 0 of the chunk
                 uint4 *const out16 = reinterpret_cast<uint4 *>(p.out + base);
+                // The group loads are plain asm, so the two groups of an
+                // unrolled pair load together; their bases pass through
+                // ordered asm after the staged copy's wait, which keeps every
+                // load below it.
+                uint32_t eb = ebuf_a, sg = sgrp_a;
+                asm volatile("mov.b32 %0, %0;" : "+r"(eb)::"memory");
+                asm volatile("mov.b32 %0, %0;" : "+r"(sg)::"memory");
 #pragma unroll 2
                 for (uint32_t i = gfirst + lane; i < mend; i += 32) {
-                    const uint2 e8 = lds_v2_m(ebuf_a + 8u * i);
-                    const uint2 s8 = lds_v2_m(sgrp_a + 8u * i);
+                    const uint2 e8 = lds_v2(eb + 8u * i);
+                    const uint2 s8 = lds_v2(sg + 8u * i);
                     const uint2 x = join4(e8.x, s8.x);
                     const uint2 y = join4(e8.y, s8.y);
                     out16[i] = make_uint4(x.x, x.y, y.x, y.y);
@@ -1005,15 +1041,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const GemvPar
                 const uint32_t fs = gfirst * 8;                    // first whole-group element
                 const uint32_t hend = min(fs, span);               // head part: [head, hend)
                 const uint32_t tbeg = max(mend * 8, fs);           // tail part: [tbeg, span)
-                uint32_t l = 0xFFFFFFFFu;
-                if (lane < 8) {
-                    if (head + lane < hend)
-                        l = head + lane;
-                } else if (lane < 16) {
-                    if (tbeg + (lane - 8) < span)
-                        l = tbeg + (lane - 8);
-                }
-                if (l != 0xFFFFFFFFu) {
+                // lanes 0..7 take the head part's elements, lanes 8..15 the tail's
+                const uint32_t l = lane < 8 ? head + (uint32_t)lane : tbeg + (uint32_t)lane - 8u;
+                const uint32_t lim = lane < 8 ? hend : span;
+                if (lane < 16 && l < lim) {
                     const uint32_t sm = lds_u8_m(sgrp_a + l);
                     p.out[base + l] = join1(lds_u8_m(ebuf_a + l), sm);
                     if constexpr (VER)
