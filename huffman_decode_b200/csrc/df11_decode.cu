@@ -246,12 +246,6 @@ __device__ __forceinline__ uint32_t lds_u8_m(uint32_t a)
     asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
     return v;
 }
-__device__ __forceinline__ uint2 lds_v2_m(uint32_t a)
-{
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
-    return v;
-}
 __device__ __forceinline__ void red_or_u32(uint32_t a, uint32_t v)
 {
     asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
@@ -1146,9 +1140,13 @@ __global__ void __launch_bounds__(kCtaWarps<CPS, VER> * 32, CPS) df11_decode_ker
     decode_body<W, MINLEN, 0, VER>(p, nullptr);
 }
 
-template <int W, int MINLEN, int TT>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_gemv_kernel(DecodeParams p,
-                                                                         const __grid_constant__ GemvParams gp)
+// The fused products at one token also come as two CTAs of up to 20 warps
+// per SM (48 registers, no spills; 40 warps per SM against 32).
+constexpr int kGemv2Warps = 20;
+
+template <int W, int MINLEN, int TT, int CPS>
+__global__ void __launch_bounds__(CPS == 1 ? kMaxWarpsPerCta * 32 : kGemv2Warps * 32, CPS)
+    df11_gemv_kernel(DecodeParams p, const __grid_constant__ GemvParams gp)
 {
     decode_body<W, MINLEN, TT>(p, &gp);
 }
@@ -1158,8 +1156,9 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32) df11_gemv_kernel(DecodeP
 constexpr int kMaxDevices = 64;
 // kernel variants: (slice width, shortest code) x (store with one CTA per
 // SM, products for 1, 2, 4, 8 tokens, store with two CTAs per SM, the
-// verifying store with one and with two CTAs per SM)
-constexpr int kVariantsPerLayout = 8;
+// verifying store with one and with two CTAs per SM, products for 1 token
+// with two CTAs per SM)
+constexpr int kVariantsPerLayout = 9;
 constexpr int kVariants = 4 * kVariantsPerLayout;
 // resident CTAs per SM, by device, kernel variant and table count
 std::atomic<int> g_occupancy[kMaxDevices][kVariants][257];
@@ -1304,11 +1303,21 @@ constexpr int kGemvCarveout = 70;   // percent of the SM's shared memory
 template <int W, int MINLEN, int TT>
 df11_status launch_gemv(const DecodeParams &prm, const GemvParams &gp, int dev, cudaStream_t stream)
 {
-    auto kernel = df11_gemv_kernel<W, MINLEN, TT>;
+    auto kernel = df11_gemv_kernel<W, MINLEN, TT, 1>;
     constexpr int v = variant_base<W, MINLEN>() + (TT == 1 ? 1 : TT == 2 ? 2 : TT == 4 ? 3 : 4);
     LaunchShape ls;
     const df11_status st =
         shape_launch<W, MINLEN>(kernel, v, prm, dev, 0, kMaxWarpsPerCta, 1, ls, true, kGemvCarveout);
+    if constexpr (TT == 1) {
+        // the two-CTA shape when it keeps more warps resident
+        auto k2 = df11_gemv_kernel<W, MINLEN, TT, 2>;
+        LaunchShape l2;
+        if (shape_launch<W, MINLEN>(k2, variant_base<W, MINLEN>() + 8, prm, dev, 0, kGemv2Warps, 2, l2) == DF11_OK &&
+            (st != DF11_OK || l2.resident_warps > ls.resident_warps)) {
+            k2<<<l2.grid, l2.warps * 32, l2.smem, stream>>>(prm, gp);
+            return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+        }
+    }
     if (st != DF11_OK)
         return st;
     kernel<<<ls.grid, ls.warps * 32, ls.smem, stream>>>(prm, gp);
