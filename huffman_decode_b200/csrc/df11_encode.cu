@@ -178,8 +178,10 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
 // Bits of every segment: one warp per segment, whose lanes read it 512
 // contiguous bytes at a time (lane l takes bytes [16 l, 16 l + 16) of each),
 // then a warp sum, also added to the total of the segment's run of
-// kRunSegs segments.
-__global__ void __launch_bounds__(256) segment_bits_kernel(EncodeParams p)
+// kRunSegs segments.  Built for 8 resident CTAs per SM (32 registers, no
+// spills), so the launch's 8 CTAs per SM all start at once: at 40 registers
+// only 6 fit and the last quarter of the CTAs ran as a second wave.
+__global__ void __launch_bounds__(256, 8) segment_bits_kernel(EncodeParams p)
 {
     __shared__ uint32_t len_tab[256];
     len_tab[threadIdx.x] = p.code_table[threadIdx.x] >> 24;
@@ -691,7 +693,7 @@ df11_status compress_device_impl(const df11_codebook *cb, const df11_layout *lay
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return DF11_ERR_CUDA;
-    prepare_kernel<<<sms * 4, 256, 0, s>>>(p, ct, z.exp_stream_bytes / 4, (z.gaps_bytes + 3) / 4,
+    prepare_kernel<<<sms * 8, 256, 0, s>>>(p, ct, z.exp_stream_bytes / 4, (z.gaps_bytes + 3) / 4,
                                                 z.n_chunks, z.signmant_bytes);
     segment_bits_kernel<<<(unsigned)((p.n_seg + 7) / 8 < (uint64_t)sms * 8 ? (p.n_seg + 7) / 8 : (uint64_t)sms * 8),
                           256, 0, s>>>(p);
